@@ -1,0 +1,214 @@
+"""Plain fp64 CPU oracle for the rotated low-bit linear -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` /
+``--impl reference`` legs of ``bench.py`` may import this package.  The
+product library never loads it and shares no code with it: the arithmetic
+lives in ``hq_oracle.c`` (scalar loops, double precision) and this module
+only marshals numpy arrays into it.
+
+The formulas and the readings of the pages they rest on are in
+``hq_oracle.h``: the random-sign Hadamard rotation x' = H.diag(s).x/sqrt(K)
+("group-128 GPTQ in a Hadamard-rotated basis" with "rotation signs":
+LLaDA2.2-mini Orin-Nano model card, Properties table and file list), the
+group-128 dequantisation w = scale.(q - z), the fp64 contraction, and the
+SwiGLU MoE expert composition.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "hq_oracle.c")
+_HDR = os.path.join(_HERE, "hq_oracle.h")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+
+_lib = None
+_lock = threading.Lock()
+
+
+def build(force: bool = False) -> str:
+    """Compile hq_oracle.c into oracle/liboracle.so with gcc (-O2, no fast-math)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+class Expert(ctypes.Structure):
+    _fields_ = [
+        ("bits", ctypes.c_int), ("zero", ctypes.c_int),
+        ("q_gate", ctypes.c_void_p), ("q_up", ctypes.c_void_p), ("q_down", ctypes.c_void_p),
+        ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
+    ]
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            L = ctypes.CDLL(_LIB_PATH)
+            vp, i, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+            L.hqo_f16_to_f64.argtypes = [ctypes.c_uint16]
+            L.hqo_f16_to_f64.restype = ctypes.c_double
+            L.hqo_unpack.argtypes = [vp, i, sz, vp]
+            L.hqo_pack.argtypes = [vp, i, sz, vp]
+            L.hqo_fwht.argtypes = [vp, i]
+            L.hqo_rotate.argtypes = [vp, vp, i, vp]
+            L.hqo_rotate_f16.argtypes = [vp, vp, i, vp]
+            L.hqo_dequant_dot.argtypes = [i, i, i, i, vp, vp, vp, i, i, i, vp, vp]
+            L.hqo_linear.argtypes = [i, i, i, i, vp, vp, vp, vp, i, i, i, vp, vp]
+            L.hqo_moe.argtypes = [vp, i, i, i, vp, i, vp, vp, i, vp, vp, i, i, vp, vp, vp]
+            for f in ("hqo_unpack", "hqo_pack", "hqo_fwht", "hqo_rotate", "hqo_rotate_f16",
+                      "hqo_dequant_dot", "hqo_linear", "hqo_moe"):
+                getattr(L, f).restype = None
+            _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return None if a is None else np.ascontiguousarray(a, dtype=dtype)
+
+
+def f16_to_f64(bits_u16: int) -> float:
+    return lib().hqo_f16_to_f64(int(bits_u16))
+
+
+def unpack(words, bits: int, n_codes: int) -> np.ndarray:
+    words = _c(words, np.uint32)
+    assert words.size * 32 >= bits * n_codes
+    out = np.empty(n_codes, np.uint8)
+    lib().hqo_unpack(_p(words), bits, n_codes, _p(out))
+    return out
+
+
+def pack(codes, bits: int) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    n = codes.size
+    out = np.empty((bits * n + 31) // 32, np.uint32)
+    lib().hqo_pack(_p(codes), bits, n, _p(out))
+    return out
+
+
+def fwht(v) -> np.ndarray:
+    v = np.array(v, dtype=np.float64, copy=True)
+    lib().hqo_fwht(_p(v), v.size)
+    return v
+
+
+def rotate(x, signs=None) -> np.ndarray:
+    """x: [..., K] float64 (or fp16 array) -> H.diag(s).x/sqrt(K) per row, float64."""
+    x = np.asarray(x)
+    K = x.shape[-1]
+    rows = x.reshape(-1, K)
+    s = _c(signs, np.int8)
+    out = np.empty(rows.shape, np.float64)
+    if rows.dtype == np.float16:
+        r16 = np.ascontiguousarray(rows).view(np.uint16)
+        for r in range(rows.shape[0]):
+            lib().hqo_rotate_f16(_p(r16[r]), _p(s), K, _p(out[r]))
+    else:
+        rd = np.ascontiguousarray(rows, dtype=np.float64)
+        for r in range(rows.shape[0]):
+            lib().hqo_rotate(_p(rd[r]), _p(s), K, _p(out[r]))
+    return out.reshape(x.shape)
+
+
+def dequant_dot(bits, M, K, zero, q, scales, xr, m_begin=0, m_end=None, with_bound=True):
+    """y[n][m] = sum_k scale.(q - zero).xr[n][k] for already-rotated xr [N][K]."""
+    q = _c(q, np.uint32)
+    sc = np.ascontiguousarray(scales).view(np.uint16) if np.asarray(scales).dtype == np.float16 \
+        else _c(scales, np.uint16)
+    xr = _c(xr, np.float64).reshape(-1, K)
+    N = xr.shape[0]
+    m_end = M if m_end is None else m_end
+    y = np.zeros((N, M), np.float64)
+    b = np.zeros((N, M), np.float64) if with_bound else None
+    lib().hqo_dequant_dot(bits, M, K, zero, _p(q), _p(sc), _p(xr), N, m_begin, m_end, _p(y), _p(b))
+    return (y, b) if with_bound else y
+
+
+def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads=1):
+    """Full rotated linear in fp64.  x: fp16 [N][K].  Returns (y, bound) float64 [N][M].
+
+    threads > 1 splits the output rows across Python threads (the C call
+    releases the GIL), each running the unchanged scalar code on its rows.
+    """
+    q = _c(q, np.uint32)
+    sc = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+    s = _c(signs, np.int8)
+    x16 = np.ascontiguousarray(x, dtype=np.float16).reshape(-1, K).view(np.uint16)
+    N = x16.shape[0]
+    m_end = M if m_end is None else m_end
+    y = np.zeros((N, M), np.float64)
+    b = np.zeros((N, M), np.float64)
+
+    def run(lo, hi):
+        lib().hqo_linear(bits, M, K, zero, _p(q), _p(sc), _p(s), _p(x16), N, lo, hi, _p(y), _p(b))
+
+    if threads <= 1:
+        run(m_begin, m_end)
+    else:
+        edges = np.linspace(m_begin, m_end, threads + 1).astype(int)
+        ts = [threading.Thread(target=run, args=(int(edges[t]), int(edges[t + 1])))
+              for t in range(threads)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+    return y, b
+
+
+def moe(experts, hidden, inter, x, topk_ids, topk_w, s_in, s_mid, t_begin=0, t_end=None,
+        want_h=False, threads=1):
+    """MoE expert layer in fp64.  experts: list of dicts with keys bits, zero,
+    q_gate, q_up, q_down (uint32 arrays) and s_gate, s_up, s_down (fp16 arrays).
+    Returns (y [T][hidden], bound [T][hidden], h [T*k][inter] or None)."""
+    keep = []
+    arr = (Expert * len(experts))()
+    for i, e in enumerate(experts):
+        qs = [_c(e[n], np.uint32) for n in ("q_gate", "q_up", "q_down")]
+        ss = [np.ascontiguousarray(e[n], dtype=np.float16).view(np.uint16)
+              for n in ("s_gate", "s_up", "s_down")]
+        keep += qs + ss
+        arr[i] = Expert(int(e["bits"]), int(e["zero"]), *[a.ctypes.data for a in qs + ss])
+    x16 = np.ascontiguousarray(x, dtype=np.float16).reshape(-1, hidden).view(np.uint16)
+    T = x16.shape[0]
+    ids = _c(topk_ids, np.int32).reshape(T, -1)
+    k = ids.shape[1]
+    w = _c(topk_w, np.float32).reshape(T, k)
+    si, sm = _c(s_in, np.int8), _c(s_mid, np.int8)
+    t_end = T if t_end is None else t_end
+    y = np.zeros((T, hidden), np.float64)
+    b = np.zeros((T, hidden), np.float64)
+    h = np.zeros((T * k, inter), np.float64) if want_h else None
+
+    def run(lo, hi):
+        lib().hqo_moe(ctypes.cast(arr, ctypes.c_void_p), len(experts), hidden, inter, _p(x16), T,
+                      _p(ids), _p(w), k, _p(si), _p(sm), lo, hi, _p(y), _p(b), _p(h))
+
+    if threads <= 1:
+        run(t_begin, t_end)
+    else:
+        edges = np.linspace(t_begin, t_end, threads + 1).astype(int)
+        ts = [threading.Thread(target=run, args=(int(edges[t]), int(edges[t + 1])))
+              for t in range(threads)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+    del keep
+    return y, b, h

@@ -1,0 +1,187 @@
+/*
+ * hq_oracle.c -- plain fp64 CPU oracle (TEST INFRASTRUCTURE ONLY).
+ *
+ * Only tests/, the smoke check and the benchmark's CPU-baseline leg may load
+ * this code.  It includes nothing from the CUDA library and the library
+ * includes nothing from here.  Every function follows its definition with
+ * scalar loops in the definition's own order; see hq_oracle.h for the
+ * formulas and the readings of the pages they rest on.
+ */
+#include "hq_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 mantissa bits. */
+double hqo_f16_to_f64(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 0x1f;
+  int m = h & 0x3ff;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -24); /* subnormal or zero: m * 2^-14 * 2^-10 */
+  } else if (e == 31) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = ldexp((double)(1024 + m), e - 25); /* (1.m) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+/* Bit i of the little-endian stream formed by the words. */
+static int stream_bit(const uint32_t* words, size_t i) {
+  return (int)((words[i / 32] >> (i % 32)) & 1u);
+}
+
+void hqo_unpack(const uint32_t* words, int bits, size_t n_codes,
+                uint8_t* codes) {
+  for (size_t j = 0; j < n_codes; ++j) {
+    int c = 0;
+    for (int t = 0; t < bits; ++t) {
+      c |= stream_bit(words, (size_t)bits * j + (size_t)t) << t;
+    }
+    codes[j] = (uint8_t)c;
+  }
+}
+
+void hqo_pack(const uint8_t* codes, int bits, size_t n_codes,
+              uint32_t* words) {
+  size_t n_words = ((size_t)bits * n_codes + 31) / 32;
+  memset(words, 0, n_words * sizeof(uint32_t));
+  for (size_t j = 0; j < n_codes; ++j) {
+    for (int t = 0; t < bits; ++t) {
+      size_t i = (size_t)bits * j + (size_t)t;
+      uint32_t b = (uint32_t)((codes[j] >> t) & 1);
+      words[i / 32] |= b << (i % 32);
+    }
+  }
+}
+
+/* Sylvester-order butterflies: at stride h, (a, b) -> (a + b, a - b). */
+void hqo_fwht(double* v, int n) {
+  for (int h = 1; h < n; h *= 2) {
+    for (int i = 0; i < n; i += 2 * h) {
+      for (int j = i; j < i + h; ++j) {
+        double a = v[j];
+        double b = v[j + h];
+        v[j] = a + b;
+        v[j + h] = a - b;
+      }
+    }
+  }
+}
+
+static double sign_of(const int8_t* signs, int i) {
+  if (signs == NULL) return 1.0;
+  return signs[i] < 0 ? -1.0 : 1.0;
+}
+
+void hqo_rotate(const double* x, const int8_t* signs, int K, double* out) {
+  for (int i = 0; i < K; ++i) out[i] = sign_of(signs, i) * x[i];
+  hqo_fwht(out, K);
+  double inv = 1.0 / sqrt((double)K);
+  for (int i = 0; i < K; ++i) out[i] *= inv;
+}
+
+void hqo_rotate_f16(const uint16_t* x, const int8_t* signs, int K,
+                    double* out) {
+  double* xd = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int i = 0; i < K; ++i) xd[i] = hqo_f16_to_f64(x[i]);
+  hqo_rotate(xd, signs, K, out);
+  free(xd);
+}
+
+void hqo_dequant_dot(int bits, int M, int K, int zero, const uint32_t* q,
+                     const uint16_t* scales, const double* xr, int N,
+                     int m_begin, int m_end, double* y, double* bound) {
+  const int G = K / 128;
+  const size_t words_per_row = (size_t)K * (size_t)bits / 32;
+  uint8_t* codes = (uint8_t*)malloc((size_t)K);
+  double* w = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int m = m_begin; m < m_end; ++m) {
+    hqo_unpack(q + (size_t)m * words_per_row, bits, (size_t)K, codes);
+    for (int k = 0; k < K; ++k) {
+      double s = hqo_f16_to_f64(scales[(size_t)m * G + k / 128]);
+      w[k] = s * (double)((int)codes[k] - zero);
+    }
+    for (int n = 0; n < N; ++n) {
+      const double* xn = xr + (size_t)n * K;
+      double acc = 0.0, abs_acc = 0.0;
+      for (int k = 0; k < K; ++k) {
+        double p = w[k] * xn[k];
+        acc += p;
+        abs_acc += fabs(p);
+      }
+      y[(size_t)n * M + m] = acc;
+      if (bound) bound[(size_t)n * M + m] = abs_acc;
+    }
+  }
+  free(w);
+  free(codes);
+}
+
+void hqo_linear(int bits, int M, int K, int zero, const uint32_t* q,
+                const uint16_t* scales, const int8_t* signs, const uint16_t* x,
+                int N, int m_begin, int m_end, double* y, double* bound) {
+  double* xr = (double*)malloc(sizeof(double) * (size_t)N * (size_t)K);
+  for (int n = 0; n < N; ++n) {
+    hqo_rotate_f16(x + (size_t)n * K, signs, K, xr + (size_t)n * K);
+  }
+  hqo_dequant_dot(bits, M, K, zero, q, scales, xr, N, m_begin, m_end, y,
+                  bound);
+  free(xr);
+}
+
+void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
+             const uint16_t* x, int T, const int32_t* topk_ids,
+             const float* topk_w, int k, const int8_t* s_in,
+             const int8_t* s_mid, int t_begin, int t_end, double* y,
+             double* bound, double* h_out) {
+  (void)n_experts;
+  double* xr = (double*)malloc(sizeof(double) * (size_t)hidden);
+  double* g = (double*)malloc(sizeof(double) * (size_t)inter);
+  double* u = (double*)malloc(sizeof(double) * (size_t)inter);
+  double* h = (double*)malloc(sizeof(double) * (size_t)inter);
+  double* hr = (double*)malloc(sizeof(double) * (size_t)inter);
+  double* d = (double*)malloc(sizeof(double) * (size_t)hidden);
+  double* db = (double*)malloc(sizeof(double) * (size_t)hidden);
+  for (int t = t_begin; t < t_end; ++t) {
+    hqo_rotate_f16(x + (size_t)t * hidden, s_in, hidden, xr);
+    double* yt = y + (size_t)t * hidden;
+    double* bt = bound ? bound + (size_t)t * hidden : NULL;
+    for (int i = 0; i < hidden; ++i) {
+      yt[i] = 0.0;
+      if (bt) bt[i] = 0.0;
+    }
+    for (int j = 0; j < k; ++j) {
+      const hqo_expert* e = &experts[topk_ids[(size_t)t * k + j]];
+      hqo_dequant_dot(e->bits, inter, hidden, e->zero, e->q_gate, e->s_gate,
+                      xr, 1, 0, inter, g, NULL);
+      hqo_dequant_dot(e->bits, inter, hidden, e->zero, e->q_up, e->s_up, xr,
+                      1, 0, inter, u, NULL);
+      for (int i = 0; i < inter; ++i) {
+        h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
+      }
+      if (h_out) {
+        memcpy(h_out + ((size_t)t * k + j) * inter, h,
+               sizeof(double) * (size_t)inter);
+      }
+      hqo_rotate(h, s_mid, inter, hr);
+      hqo_dequant_dot(e->bits, hidden, inter, e->zero, e->q_down, e->s_down,
+                      hr, 1, 0, hidden, d, db);
+      double wj = (double)topk_w[(size_t)t * k + j];
+      for (int i = 0; i < hidden; ++i) {
+        yt[i] += wj * d[i];
+        if (bt) bt[i] += fabs(wj) * db[i];
+      }
+    }
+  }
+  free(db);
+  free(d);
+  free(hr);
+  free(h);
+  free(u);
+  free(g);
+  free(xr);
+}

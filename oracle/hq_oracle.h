@@ -1,0 +1,112 @@
+/*
+ * hq_oracle.h -- plain fp64 CPU oracle for the rotated low-bit linear.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product library links, includes
+ * or calls this code; only the tests, the smoke check and the benchmark's
+ * CPU-baseline leg do.  It shares no header, helper or constant with the CUDA
+ * path.
+ *
+ * What it computes (all in double precision, scalar loops, no blocking):
+ *   - the random-sign Hadamard rotation  x' = H_K . diag(s) . x / sqrt(K)
+ *     ("group-128 GPTQ in a Hadamard-rotated basis", rotation signs kept in
+ *     small.bin: LLaDA2.2-mini Orin-Nano model card, Properties table and the
+ *     file-list paragraph; "behind a random Hadamard rotation": Qwen3.8-27B
+ *     Pingala-8 2-bit card, "What this is"),
+ *   - the group-128 dequantisation  w[m][k] = scale[m][k/128] * (q[m][k] - z),
+ *   - the contraction  y[n][m] = sum_k w[m][k] * x'[n][k],
+ *   - the MoE expert composition (gate/up, SwiGLU, down, weighted combine).
+ *
+ * Readings where the pages are silent (each is listed in the design doc):
+ *   - H_K is the Sylvester Hadamard matrix in natural order,
+ *     H[i][j] = (-1)^popcount(i & j); the 1/sqrt(K) factor is applied once.
+ *   - sign s_i = -1 where signs[i] < 0, else +1; a NULL sign vector means s = 1.
+ *   - packed codes: code j of a row occupies bits [b*j, b*j+b) of the row's
+ *     little-endian bit stream (word w holds stream bits [32w, 32w+32)).
+ *     For b = 3 this makes three words carry 32 codes, codes 10 and 21
+ *     straddling a word boundary.
+ *   - zero point z is one integer per tensor (2^(b-1) in every workload).
+ *
+ * Parity pins (tests/test_oracle_pins.py): dense brute-force Hadamard,
+ * H.H^T = K.I, norm preservation, involution, closed forms, numpy bit
+ * unpacking, an explicit dense W_eff = dequant(Q).H.diag(s)/sqrt(K) product,
+ * and MoE reductions to single-expert chains.
+ */
+#ifndef HQ_ORACLE_H
+#define HQ_ORACLE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* IEEE binary16 bit pattern -> double (normals, subnormals, zeros, inf, nan). */
+double hqo_f16_to_f64(uint16_t h);
+
+/* Decode n_codes codes of width bits (1..8) from the packed little-endian bit
+ * stream in words.  codes[j] = stream bits [bits*j, bits*j+bits). */
+void hqo_unpack(const uint32_t* words, int bits, size_t n_codes, uint8_t* codes);
+
+/* Inverse of hqo_unpack.  Words must have room for ceil(bits*n_codes/32)
+ * entries; they are fully overwritten (unused high bits are zero). */
+void hqo_pack(const uint8_t* codes, int bits, size_t n_codes, uint32_t* words);
+
+/* In-place unnormalised fast Walsh-Hadamard transform, v <- H_n v, n a power
+ * of two, Sylvester natural order. */
+void hqo_fwht(double* v, int n);
+
+/* out = H_K diag(s) x / sqrt(K) for one row.  x in double. */
+void hqo_rotate(const double* x, const int8_t* signs, int K, double* out);
+
+/* Same, input row given as fp16 bit patterns. */
+void hqo_rotate_f16(const uint16_t* x, const int8_t* signs, int K, double* out);
+
+/* Dequantise-and-dot for output rows [m_begin, m_end):
+ *   y[n][m]     = sum_k scale[m][k/128] * (q[m][k] - zero) * xr[n][k]
+ *   bound[n][m] = sum_k |scale[m][k/128] * (q[m][k] - zero) * xr[n][k]|
+ * q: row-major packed codes, K*bits/32 words per row.
+ * scales: fp16 bit patterns [M][K/128].  xr: already-rotated inputs [N][K].
+ * y, bound: [N][M] (only columns m_begin..m_end-1 are written; bound may be
+ * NULL). */
+void hqo_dequant_dot(int bits, int M, int K, int zero, const uint32_t* q,
+                     const uint16_t* scales, const double* xr, int N,
+                     int m_begin, int m_end, double* y, double* bound);
+
+/* The whole rotated linear for rows [m_begin, m_end): rotate each of the N
+ * fp16 input rows with signs, then hqo_dequant_dot. */
+void hqo_linear(int bits, int M, int K, int zero, const uint32_t* q,
+                const uint16_t* scales, const int8_t* signs, const uint16_t* x,
+                int N, int m_begin, int m_end, double* y, double* bound);
+
+/* One routed expert: three packed linears with a shared bit width. */
+typedef struct {
+  int bits;
+  int zero;
+  const uint32_t* q_gate; /* [inter][hidden*bits/32] */
+  const uint32_t* q_up;   /* [inter][hidden*bits/32] */
+  const uint32_t* q_down; /* [hidden][inter*bits/32] */
+  const uint16_t* s_gate; /* [inter][hidden/128] */
+  const uint16_t* s_up;   /* [inter][hidden/128] */
+  const uint16_t* s_down; /* [hidden][inter/128] */
+} hqo_expert;
+
+/* MoE expert layer for tokens [t_begin, t_end):
+ *   x'_t   = rot(x_t, s_in)                        (hidden)
+ *   g, u   = W_gate^e x'_t, W_up^e x'_t            (inter)
+ *   h      = g / (1 + exp(-g)) * u                 (SwiGLU)
+ *   h'     = rot(h, s_mid)                         (inter)
+ *   d      = W_down^e h'                           (hidden)
+ *   y_t    = sum_{j=0..k-1} topk_w[t][j] * d_{t,j}  (j ascending)
+ *   bound_t = sum_j |topk_w[t][j]| * sum_k |w_down * h'|
+ * h_out (optional, [T*k][inter]) receives h for pair (t, j) at row t*k+j. */
+void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
+             const uint16_t* x, int T, const int32_t* topk_ids,
+             const float* topk_w, int k, const int8_t* s_in,
+             const int8_t* s_mid, int t_begin, int t_end, double* y,
+             double* bound, double* h_out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HQ_ORACLE_H */

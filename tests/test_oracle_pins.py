@@ -1,0 +1,326 @@
+"""Pins for the fp64 CPU oracle against facts that do not come from the oracle itself.
+
+Each test checks one oracle function against something fixed independently of
+its code: a brute-force dense Hadamard matrix built from its definition
+H[i][j] = (-1)^popcount(i & j), scipy's Sylvester construction, exact algebraic
+identities (H.H^T = K.I, orthogonality, involution), hand-derived fixtures in
+tests/golden/, numpy's own bit unpacking, numpy's fp16 decoding, closed forms,
+and an explicit dense W_eff = dequant(Q).H.diag(s)/sqrt(K) product built with
+numpy/scipy.  A dropped term, a wrong sign or index, or a transposed operand
+anywhere in the oracle fails at least one of them.
+"""
+import os
+
+import numpy as np
+import pytest
+import scipy.linalg
+
+import oracle
+from bit_hadamard_rotated_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ---------------------------------------------------------------- helpers (independent of the oracle)
+def dense_hadamard(K):
+    i = np.arange(K)
+    pc = np.vectorize(lambda v: bin(v).count("1"))(i[:, None] & i[None, :])
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+def np_unpack(words, bits, n):
+    """Codes from the little-endian bit stream via numpy.unpackbits."""
+    stream = np.unpackbits(np.ascontiguousarray(words, dtype="<u4").view(np.uint8), bitorder="little")
+    stream = stream[: bits * n].reshape(n, bits).astype(np.int64)
+    return (stream << np.arange(bits)).sum(axis=1)
+
+
+def sign_vec(signs, K):
+    return np.ones(K) if signs is None else np.where(np.asarray(signs) < 0, -1.0, 1.0)
+
+
+def dense_weff(q, scales, bits, zero, M, K, signs):
+    """Explicit effective weight W_eff = dequant(Q) . H_K . diag(s) / sqrt(K)."""
+    codes = np.stack([np_unpack(q[m], bits, K) for m in range(M)])
+    sc = np.repeat(np.asarray(scales, dtype=np.float16).astype(np.float64), 128, axis=1)
+    Wq = sc * (codes - zero)
+    H = scipy.linalg.hadamard(K).astype(np.float64)
+    return Wq, Wq @ H @ np.diag(sign_vec(signs, K)) / np.sqrt(K)
+
+
+# ---------------------------------------------------------------- fp16 decode
+def test_f16_decode_every_pattern():
+    pats = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ref = pats.view(np.float16).astype(np.float64)
+    got = np.array([oracle.f16_to_f64(int(p)) for p in pats])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    assert np.array_equal(got[~nan], ref[~nan])
+    # signed zeros too
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+# ---------------------------------------------------------------- FWHT
+@pytest.mark.parametrize("K", [2, 4, 8, 16, 32, 64, 128, 256])
+def test_fwht_equals_bruteforce_dense(K):
+    rng = np.random.default_rng(K)
+    v = rng.integers(-1000, 1000, size=K).astype(np.float64)
+    assert np.array_equal(oracle.fwht(v), dense_hadamard(K) @ v)
+
+
+@pytest.mark.parametrize("K", [512, 2048, 4096])
+def test_fwht_equals_scipy_sylvester(K):
+    rng = np.random.default_rng(K)
+    v = rng.integers(-1000, 1000, size=K).astype(np.float64)
+    assert np.array_equal(oracle.fwht(v), scipy.linalg.hadamard(K) @ v)
+
+
+def test_hadamard_hht_is_k_identity():
+    K = 64
+    H = np.stack([oracle.fwht(np.eye(K)[i]) for i in range(K)], axis=1)
+    assert np.array_equal(H @ H.T, K * np.eye(K))
+    assert np.array_equal(H, H.T)
+
+
+@pytest.mark.parametrize("K", [128, 512, 2048, 8192])
+def test_rotation_preserves_norm_and_inverts(K):
+    rng = np.random.default_rng(7 + K)
+    x = rng.standard_normal(K)
+    s = synth.signs(rng, K)
+    xr = oracle.rotate(x, s)
+    assert abs(np.linalg.norm(xr) - np.linalg.norm(x)) <= 1e-13 * np.linalg.norm(x)
+    # inverse: diag(s) H x' / sqrt(K) == x
+    back = sign_vec(s, K) * oracle.fwht(xr) / np.sqrt(K)
+    assert np.max(np.abs(back - x)) <= 1e-12
+
+
+@pytest.mark.parametrize("K", [128, 4096])
+def test_rotation_closed_forms(K):
+    e0 = np.zeros(K)
+    e0[0] = 1.0
+    assert np.allclose(oracle.rotate(e0), np.full(K, 1 / np.sqrt(K)), rtol=0, atol=1e-15)
+    one = np.ones(K)
+    want = np.zeros(K)
+    want[0] = np.sqrt(K)
+    assert np.allclose(oracle.rotate(one), want, rtol=0, atol=1e-12)
+
+
+def test_rotation_hand_fixtures():
+    for line in open(os.path.join(GOLDEN, "hadamard_small.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        K, s, x, want = [f.split() for f in line.split("|")]
+        K = int(K[0])
+        s = np.array([int(v) for v in s], np.int8)
+        x = np.array([float(v) for v in x])
+        got = oracle.rotate(x, s) * np.sqrt(K)
+        assert np.allclose(got, [float(v) for v in want], rtol=0, atol=1e-12), line
+
+
+def test_rotation_sign_convention_and_null_signs():
+    K = 256
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal(K)
+    s_pos = np.ones(K, np.int8)
+    s_mixed = np.array(rng.integers(-3, 4, size=K), np.int8)  # 0 counts as +1, any negative as -1
+    assert np.array_equal(oracle.rotate(x, None), oracle.rotate(x, s_pos))
+    H = scipy.linalg.hadamard(K)
+    want = H @ (np.where(s_mixed < 0, -1.0, 1.0) * x) / np.sqrt(K)
+    assert np.allclose(oracle.rotate(x, s_mixed), want, rtol=0, atol=1e-12)
+
+
+def test_rotation_of_fp16_input_reads_fp16_bits():
+    K = 512
+    rng = np.random.default_rng(11)
+    x16 = rng.standard_normal((3, K)).astype(np.float16)
+    s = synth.signs(rng, K)
+    got = oracle.rotate(x16, s)
+    H = scipy.linalg.hadamard(K)
+    want = (H @ (sign_vec(s, K)[:, None] * x16.astype(np.float64).T)).T / np.sqrt(K)
+    assert np.allclose(got, want, rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------------- packing
+def test_unpack_hand_fixtures():
+    n = 0
+    for line in open(os.path.join(GOLDEN, "unpack_patterns.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        bits, words, codes = [f.split() for f in line.split("|")]
+        bits = int(bits[0])
+        words = np.array([int(w, 16) for w in words], np.uint32)
+        codes = np.array([int(c) for c in codes])
+        assert np.array_equal(oracle.unpack(words, bits, codes.size), codes), line
+        assert np.array_equal(oracle.pack(codes, bits), words), line
+        n += 1
+    assert n >= 8
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_unpack_matches_numpy_unpackbits(bits):
+    rng = np.random.default_rng(100 + bits)
+    n = 32 * 97
+    words = rng.integers(0, 2**32, size=n * bits // 32, dtype=np.uint64).astype(np.uint32)
+    assert np.array_equal(oracle.unpack(words, bits, n), np_unpack(words, bits, n))
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_pack_unpack_round_trip(bits):
+    rng = np.random.default_rng(200 + bits)
+    codes = rng.integers(0, 1 << bits, size=4096).astype(np.uint8)
+    words = oracle.pack(codes, bits)
+    assert words.size == 4096 * bits // 32
+    assert np.array_equal(oracle.unpack(words, bits, codes.size), codes)
+    assert np.array_equal(np_unpack(words, bits, codes.size), codes)
+
+
+def test_three_bit_straddling_codes_single_bits():
+    """A single set stream bit p in a 3-bit triplet lands in code p//3 as 1 << (p%3)."""
+    for p in range(96):
+        words = np.zeros(3, np.uint32)
+        words[p // 32] = np.uint32(1 << (p % 32))
+        codes = oracle.unpack(words, 3, 32)
+        want = np.zeros(32, np.int64)
+        want[p // 3] = 1 << (p % 3)
+        assert np.array_equal(codes, want), p
+
+
+# ---------------------------------------------------------------- dequant + dot
+def _mk(bits, M, K, N, seed, signs=True):
+    d = synth.linear(M, K, bits, N, seed=seed)
+    if not signs:
+        d["signs"] = None
+    return d
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_zero_codes_give_exact_zero(bits):
+    M, K, N = 8, 256, 2
+    d = _mk(bits, M, K, N, 1)
+    z = 1 << (bits - 1)
+    q = np.stack([oracle.pack(np.full(K, z, np.uint8), bits) for _ in range(M)])
+    y, b = oracle.linear(bits, M, K, z, q, d["scales"], d["signs"], d["x"])
+    assert np.array_equal(y, np.zeros((N, M)))
+    assert np.array_equal(b, np.zeros((N, M)))
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_constant_codes_closed_form(bits):
+    """q = z+1 everywhere and one constant scale c: y_m = c . sum_k x'_k."""
+    M, K, N = 4, 512, 3
+    d = _mk(bits, M, K, N, 2)
+    z = 1 << (bits - 1)
+    c = np.float16(0.0117)
+    q = np.stack([oracle.pack(np.full(K, z + 1, np.uint8), bits) for _ in range(M)])
+    sc = np.full((M, K // 128), c, np.float16)
+    y, _ = oracle.linear(bits, M, K, z, q, sc, d["signs"], d["x"])
+    H = scipy.linalg.hadamard(K)
+    xr = (H @ (sign_vec(d["signs"], K)[:, None] * d["x"].astype(np.float64).T)).T / np.sqrt(K)
+    want = float(c) * xr.sum(axis=1)
+    assert np.allclose(y, np.repeat(want[:, None], M, axis=1), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_unit_input_gives_row_sums(bits):
+    """s = 1 and x = e0: x' = 1/sqrt(K) everywhere, so y_m = sum_k w_mk / sqrt(K)."""
+    M, K = 16, 256
+    d = _mk(bits, M, K, 1, 3)
+    x = np.zeros((1, K), np.float16)
+    x[0, 0] = 1.0
+    y, _ = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], None, x)
+    Wq, _ = dense_weff(d["q"], d["scales"], bits, d["zero"], M, K, None)
+    assert np.allclose(y[0], Wq.sum(axis=1) / np.sqrt(K), rtol=1e-13, atol=1e-15)
+
+
+@pytest.mark.parametrize("bits,M,K,N", [(2, 64, 512, 3), (3, 40, 256, 2), (4, 33, 512, 4),
+                                         (8, 17, 128, 5), (3, 8, 512, 1)])
+def test_linear_equals_explicit_dense_weff(bits, M, K, N):
+    d = _mk(bits, M, K, N, 10 + bits)
+    y, b = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    Wq, Weff = dense_weff(d["q"], d["scales"], bits, d["zero"], M, K, d["signs"])
+    xd = d["x"].astype(np.float64)
+    want = xd @ Weff.T
+    assert np.allclose(y, want, rtol=1e-12, atol=1e-12)
+    # the tolerance base: sum_k |w_k x'_k| with x' rotated explicitly
+    H = scipy.linalg.hadamard(K)
+    xr = (H @ (sign_vec(d["signs"], K)[:, None] * xd.T)).T / np.sqrt(K)
+    want_b = np.abs(Wq[None, :, :] * xr[:, None, :]).sum(axis=2)
+    assert np.allclose(b, want_b, rtol=1e-12, atol=1e-12)
+    assert np.all(np.abs(y) <= b * (1 + 1e-12))
+
+
+def test_linear_row_ranges_compose():
+    d = _mk(4, 50, 256, 2, 21)
+    y_all, b_all = oracle.linear(4, 50, 256, 8, d["q"], d["scales"], d["signs"], d["x"])
+    y_t, b_t = oracle.linear(4, 50, 256, 8, d["q"], d["scales"], d["signs"], d["x"], threads=3)
+    assert np.array_equal(y_all, y_t) and np.array_equal(b_all, b_t)
+
+
+# ---------------------------------------------------------------- MoE composition
+def _small_moe(seed, E=6, hidden=256, inter=128, T=5, k=2, probs=(0.4, 0.3, 0.3)):
+    return synth.moe(seed=seed, E=E, hidden=hidden, inter=inter, T=T, k=k, probs=probs)
+
+
+def _dense_expert_chain(e, x_row, s_in, s_mid, hidden, inter):
+    _, Wg = dense_weff(e["q_gate"], e["s_gate"], e["bits"], e["zero"], inter, hidden, s_in)
+    _, Wu = dense_weff(e["q_up"], e["s_up"], e["bits"], e["zero"], inter, hidden, s_in)
+    _, Wd = dense_weff(e["q_down"], e["s_down"], e["bits"], e["zero"], hidden, inter, s_mid)
+    g = Wg @ x_row
+    u = Wu @ x_row
+    h = g * u / (1.0 + np.exp(-g))
+    return Wd @ h, h
+
+
+def test_moe_top1_equals_dense_chain():
+    m = _small_moe(31, k=1)
+    T = m["T"]
+    ids = m["topk_ids"]
+    w1 = np.ones((T, 1), np.float32)
+    y, b, h = oracle.moe(m["experts"], m["hidden"], m["inter"], m["x"], ids, w1, m["s_in"],
+                         m["s_mid"], want_h=True)
+    for t in range(T):
+        e = m["experts"][int(ids[t, 0])]
+        want, hw = _dense_expert_chain(e, m["x"][t].astype(np.float64), m["s_in"], m["s_mid"],
+                                       m["hidden"], m["inter"])
+        assert np.allclose(y[t], want, rtol=1e-11, atol=1e-12)
+        assert np.allclose(h[t], hw, rtol=1e-11, atol=1e-12)
+        assert np.all(np.abs(y[t]) <= b[t] * (1 + 1e-12))
+
+
+def test_moe_weighted_combine_order_and_weights():
+    m = _small_moe(32, k=3)
+    y, _, _ = oracle.moe(m["experts"], m["hidden"], m["inter"], m["x"], m["topk_ids"], m["topk_w"],
+                         m["s_in"], m["s_mid"])
+    for t in range(m["T"]):
+        want = np.zeros(m["hidden"])
+        for j in range(m["k"]):
+            e = m["experts"][int(m["topk_ids"][t, j])]
+            d, _ = _dense_expert_chain(e, m["x"][t].astype(np.float64), m["s_in"], m["s_mid"],
+                                       m["hidden"], m["inter"])
+            want += float(m["topk_w"][t, j]) * d
+        assert np.allclose(y[t], want, rtol=1e-11, atol=1e-12)
+
+
+def test_moe_identical_experts_reduce_to_one():
+    m = _small_moe(33, k=4, E=5)
+    same = [m["experts"][0]] * m["E"]
+    y, _, _ = oracle.moe(same, m["hidden"], m["inter"], m["x"], m["topk_ids"], m["topk_w"],
+                         m["s_in"], m["s_mid"])
+    for t in range(m["T"]):
+        want, _ = _dense_expert_chain(same[0], m["x"][t].astype(np.float64), m["s_in"], m["s_mid"],
+                                      m["hidden"], m["inter"])
+        assert np.allclose(y[t], want, rtol=1e-6, atol=1e-9)  # weights sum to 1 in fp32
+
+
+# ---------------------------------------------------------------- routing inputs
+def test_routing_weights_and_ties():
+    rng = np.random.default_rng(5)
+    _, ids, w = synth.routing(rng, 32, 256, 8)
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+    assert np.all(np.diff(w, axis=1) <= 0)          # descending logits -> descending weights
+    for t in range(32):
+        assert len(set(ids[t].tolist())) == 8
+    # ties: equal logits keep the lower index first
+    logits = np.zeros((1, 16), np.float32)
+    order = np.argsort(-logits, axis=1, kind="stable")[:, :4]
+    assert order.tolist() == [[0, 1, 2, 3]]
