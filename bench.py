@@ -1,0 +1,436 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated low-bit linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one pass of the hot path over one batch: the rotated linears of the
+bit-width-coverage workload (out 12288, in 4096, group-128 codes at 2, 3 and 8
+bits, zero point 2^(b-1), fp16 activations N(0,1), batch 1), each one call of
+the C ABI's hq_linear (rotation, unpack, dequantisation and contraction).
+Metric: effective weight GB/s = (packed-code + scale bytes) / time, whole job.
+
+Weights are cycled over enough distinct copies that every step reads HBM, not
+L2 (inputs larger than L2 between uses of a copy).  Steps are replayed from
+CUDA graphs and timed with CUDA events on the launching stream, bracketed by a
+barrier and a device synchronisation; the job time is the max over ranks.
+
+Under torchrun every rank runs the same workload on its own GPU with its own
+weights (weak scaling); there is no collective on the data path.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_hadamard_rotated_b200 import dist, synth  # noqa: E402
+
+METRIC = "rotated 2/3/4-bit linear: weight GB/s (% HBM peak) at B=1; TFLOP/s at B=64"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+WORKLOAD = "rotated linear M=12288 K=4096, bits 2/3/8, batch 1"
+LAYERS = [(12288, 4096, 2), (12288, 4096, 3), (12288, 4096, 8)]
+B64 = (28672, 8192, 2, 64)
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS,
+                bf16_sustained=1400.0, source="fallback")
+
+
+# ---------------------------------------------------------------- clocks during the timed region
+class Clocks:
+    Q = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        self.proc = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.uuid = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.splitlines():
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 10:
+                continue
+            if self.uuid and self.uuid.replace("GPU-", "") not in f[1]:
+                continue
+            rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i] == "Active"})
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(rows),
+                "power_w_max": max(float(r[4]) for r in rows
+                                   if r[4].replace(".", "").isdigit())}
+
+
+# ---------------------------------------------------------------- workload
+def build_layers(device, copies, seed):
+    """copies x layers of packed weights; copy 0 from the seeded host generator,
+    the others drawn on the device from a seeded torch generator (same laws)."""
+    from bit_hadamard_rotated_b200 import RotatedLinear
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    base = [synth.linear(M, K, b, 1, seed=seed) for (M, K, b) in LAYERS]
+    xs = [torch.from_numpy(d["x"]).to(device) for d in base]
+    layers = []
+    for c in range(copies):
+        row = []
+        for d in base:
+            M, K, b = d["M"], d["K"], d["bits"]
+            if c == 0:
+                q = torch.from_numpy(d["q"].view(np.int32)).to(device)
+                sc = torch.from_numpy(d["scales"]).to(device)
+            else:
+                q = torch.randint(-2**31, 2**31 - 1, (M, K * b // 32), dtype=torch.int32,
+                                  device=device, generator=gen)
+                sc = (torch.rand((M, K // 128), device=device, generator=gen) * 0.015 + 0.005
+                      ).to(torch.float16)
+            s = torch.from_numpy(d["signs"]).to(device)
+            row.append(RotatedLinear(q, sc, s, b, d["zero"], max_batch=1))
+        layers.append(row)
+    return layers, xs
+
+
+def weight_bytes(M, K, b):
+    return M * K * b // 8 + M * (K // 128) * 2
+
+
+def algorithmic_bytes(M, K, b, N):
+    """Bytes the linear must move at least once: codes, scales, signs, x, y."""
+    return weight_bytes(M, K, b) + K + N * K * 2 + N * M * 4
+
+
+def run_ours(a):
+    rank, local_rank, world = dist.env_world()
+    device = torch.device("cuda", local_rank)
+    torch.cuda.set_device(device)
+    dist.init("nccl")
+    import bit_hadamard_rotated_b200 as hq
+    from bit_hadamard_rotated_b200 import _lib
+    _lib.lib()  # fail loudly if the CUDA library is missing
+
+    props = torch.cuda.get_device_properties(device)
+    l2 = getattr(props, "L2_cache_size", 126 * 2**20)
+    step_w = sum(weight_bytes(M, K, b) for (M, K, b) in LAYERS)
+    copies = max(2, math.ceil(4 * l2 / step_w))
+    layers, xs = build_layers(device, copies, seed=1234 + rank)
+    ys = [torch.empty((1, M), dtype=torch.float32, device=device) for (M, K, b) in LAYERS]
+    stream = torch.cuda.Stream(device)
+
+    def step(c):
+        for li in range(len(LAYERS)):
+            layers[c][li](xs[li], out=ys[li])
+
+    with torch.cuda.stream(stream):
+        for i in range(max(a.warmup, 3)):
+            step(i % copies)
+    torch.cuda.synchronize(device)
+    for row in layers:
+        for lin in row:
+            lin.check_status(stream)
+
+    # One graph per weight copy (one step each) and one block graph of `rep` rounds.
+    rep = 8
+    g1 = []
+    n0 = hq.hq_launch_count()
+    with torch.cuda.stream(stream):
+        for c in range(copies):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                step(c)
+            g1.append(g)
+        launches_per_step = (hq.hq_launch_count() - n0) // copies
+        gb = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gb, stream=stream):
+            for _ in range(rep):
+                for c in range(copies):
+                    step(c)
+    block = rep * copies
+    for i in range(a.warmup):
+        with torch.cuda.stream(stream):
+            g1[i % copies].replay()
+    torch.cuda.synchronize(device)
+
+    clocks = Clocks(device)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    time.sleep(0.3)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        done = 0
+        while a.steps - done >= block:
+            gb.replay()
+            done += block
+        while done < a.steps:
+            g1[done % copies].replay()
+            done += 1
+        ev1.record(stream)
+    torch.cuda.synchronize(device)
+    ck = clocks.stop()
+    dist.barrier(device)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = dist.max_over_ranks(ms, device)
+    for row in layers:
+        for lin in row:
+            lin.check_status(stream)
+
+    total_w = step_w * a.steps * world
+    value = total_w / (ms_max / 1e3) / 1e9
+    pk = peaks()
+    alg = sum(algorithmic_bytes(M, K, b, 1) for (M, K, b) in LAYERS)
+    achieved = alg / ((ms / a.steps) / 1e3) / 1e9
+
+    # per-bit-width breakdown (each layer's own graph, same protocol)
+    per_bits = {}
+    for li, (M, K, b) in enumerate(LAYERS):
+        gs = []
+        with torch.cuda.stream(stream):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for _ in range(rep):
+                    for c in range(copies):
+                        layers[c][li](xs[li], out=ys[li])
+            gs.append(g)
+            reps = max(1, 2000 // block)
+            g.replay()
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) * 1e3 / (reps * block)
+        per_bits[str(b)] = {"us_per_linear": round(us, 3),
+                            "weight_gbs": round(weight_bytes(M, K, b) / (us * 1e-6) / 1e9, 1),
+                            "frac_hbm": round(weight_bytes(M, K, b) / (us * 1e-6) / 1e9
+                                              / pk["hbm"], 4)}
+
+    b64 = measure_b64(device, stream, pk) if a.b64 else None
+    e2e = measure_e2e(device, layers, xs, a)
+    e2e_ms = dist.max_over_ranks(e2e.pop("ms"), device)
+    e2e["value"] = round(step_w * e2e["steps"] * world / (e2e_ms * 1e-3) / 1e9, 3)
+
+    cpu = None
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        cpu = cpu_baseline(a.cpu_seconds)
+
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_max / a.steps, 6),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+        "data": "synthetic (seeded; uniform codes, fp16 scales U[0.005,0.02], x ~ N(0,1))",
+        "config": {"workload": WORKLOAD, "layers": [f"{M}x{K} b{b}" for (M, K, b) in LAYERS],
+                   "batch": 1, "group": 128, "weight_bytes_per_step": step_w,
+                   "weight_copies": copies, "l2_bytes": l2,
+                   "l2_policy": f"{copies} weight copies cycled; {copies * step_w / 2**20:.0f} MiB "
+                                f"> L2 between reuses of a copy",
+                   "parallelism": f"replicas x{world} (weak scaling, no data-path collective)"},
+        "frac_hbm": round(value / world / pk["hbm"], 4),
+        "roofline": {"bound": "hbm", "kernel": "prep_gemv + gemv_kernel (aggregate of the step)",
+                     "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
+                     "frac": round(achieved / pk["hbm"], 4), "traffic": None,
+                     "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
+        "per_bits": per_bits,
+        "b64": b64,
+        "e2e": e2e,
+        "gpu_launches": int(launches_per_step * a.steps),
+        "launches_per_step": int(launches_per_step),
+        "clocks": ck,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del g1, gb
+    dist.finish()
+
+
+def measure_b64(device, stream, pk):
+    """TFLOP/s of the large dense MLP linear (28672x8192, 2-bit) at batch 64."""
+    from bit_hadamard_rotated_b200 import RotatedLinear
+    M, K, b, N = B64
+    d = synth.linear(M, K, b, N, seed=77, scale_dist="loguniform", outlier_frac=0.01)
+    lin = RotatedLinear(torch.from_numpy(d["q"].view(np.int32)).to(device),
+                        torch.from_numpy(d["scales"]).to(device),
+                        torch.from_numpy(d["signs"]).to(device), b, d["zero"], max_batch=N)
+    x = torch.from_numpy(d["x"]).to(device)
+    y = torch.empty((N, M), dtype=torch.float32, device=device)
+    flush = torch.empty(2 * 126 * 2**20 // 4, dtype=torch.float32, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            lin(x, out=y)
+        torch.cuda.synchronize(device)
+        times = []
+        for _ in range(20):
+            flush.zero_()  # L2 flush between timed calls (outside the timed interval)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            lin(x, out=y)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    tflops = 2.0 * M * K * N / (ms * 1e-3) / 1e12
+    return {"workload": f"rotated linear M={M} K={K} b{b} batch {N}", "ms": round(ms, 4),
+            "tflops": round(tflops, 2), "frac_bf16_peak": round(tflops / pk["bf16"], 4),
+            "weight_gbs": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9, 1),
+            "launches": lin.launches(N), "timing": "median of 20, L2 flushed before each"}
+
+
+def measure_e2e(device, layers, xs, a):
+    """Same metric through the public Python API with host buffers: every step
+    copies each layer's activations from pinned host memory and reads the
+    outputs back to pinned host memory, inside the timed region."""
+    copies = len(layers)
+    xh = [x.cpu().pin_memory() for x in xs]
+    xd = [torch.empty_like(x) for x in xs]
+    yh = [torch.empty((1, M), dtype=torch.float32).pin_memory() for (M, K, b) in LAYERS]
+    yd = [torch.empty((1, M), dtype=torch.float32, device=device) for (M, K, b) in LAYERS]
+    steps = min(a.steps, 2000)
+    stream = torch.cuda.current_stream(device)
+
+    def one(c):
+        for li in range(len(LAYERS)):
+            xd[li].copy_(xh[li], non_blocking=True)
+            layers[c][li](xd[li], out=yd[li])
+            yh[li].copy_(yd[li], non_blocking=True)
+
+    for i in range(3):
+        one(i % copies)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        one(i % copies)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1)
+    step_w = sum(weight_bytes(M, K, b) for (M, K, b) in LAYERS)
+    return {"ms": ms, "value": None, "unit": "GB/s", "steps": steps,
+            "h2d_bytes_per_step": sum(int(x.numel() * 2) for x in xs),
+            "d2h_bytes_per_step": sum(M * 4 for (M, K, b) in LAYERS),
+            "api": "RotatedLinear.__call__ -> hq_linear (C ABI), eager launches"}
+
+
+# ---------------------------------------------------------------- CPU oracle baseline
+def cpu_baseline(seconds: float):
+    """The fp64 oracle as it stands, on this host's cores, over a bounded sample
+    of the workload (the first R rows of each layer, batch 1), scaled to GB/s."""
+    import oracle
+    cores = os.cpu_count() or 1
+    ds = [synth.linear(M, K, b, 1, seed=99) for (M, K, b) in LAYERS]
+    probe = 64
+    t0 = time.perf_counter()
+    for d in ds:
+        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                      d["x"], 0, probe, threads=1)
+    per_row = (time.perf_counter() - t0) / (probe * len(ds))
+    rows = int(min(min(M for (M, K, b) in LAYERS), max(probe, seconds * cores / per_row / 3)))
+    t0 = time.perf_counter()
+    for d in ds:
+        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                      d["x"], 0, rows, threads=cores)
+    dt = time.perf_counter() - t0
+    wb = sum(rows * (K * b // 8 + (K // 128) * 2) for (M, K, b) in LAYERS)
+    return {"value": round(wb / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {rows} of 12288 rows of each layer (b2, b3, b8), batch 1, "
+                      f"{dt:.1f} s wall on {cores} threads"}
+
+
+def run_reference(a):
+    rank, _, world = dist.env_world()
+    if rank != 0:
+        return
+    import oracle
+    cores = os.cpu_count() or 1
+    ds = [synth.linear(M, K, b, 1, seed=99) for (M, K, b) in LAYERS]
+    rows = a.ref_rows
+    for _ in range(max(a.warmup, 0)):
+        for d in ds:
+            oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                          d["x"], 0, rows, threads=cores)
+    t0 = time.perf_counter()
+    for _ in range(a.steps):
+        for d in ds:
+            oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                          d["x"], 0, rows, threads=cores)
+    dt = time.perf_counter() - t0
+    wb = a.steps * sum(rows * (K * b // 8 + (K // 128) * 2) for (M, K, b) in LAYERS)
+    v = wb / dt / 1e9
+    sample = f"each step: first {rows} of 12288 rows of each layer (b2, b3, b8), batch 1"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s",
+        "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
+        "ms_per_step": round(dt * 1e3 / a.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": round(v, 5), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 5), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-b64", dest="b64", action="store_false")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-rows", type=int, default=256)
+    a = ap.parse_args()
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_ours(a)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+// hq_api.cu -- the C ABI of libhq: argument validation, workspace layout and
+// kernel dispatch.  Every check happens on the host before any launch; no
+// entry point allocates or frees memory.
+#include <atomic>
+#include <cstdint>
+
+#include "hq_internal.h"
+
+namespace hq {
+
+static std::atomic<uint64_t> g_launches{0};
+static std::atomic<int> g_tc_min_batch{9};
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static bool aligned(const void* p, uintptr_t a) {
+  return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+}
+static bool is_pow2(long v) { return v > 0 && (v & (v - 1)) == 0; }
+static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+constexpr size_t kStatusBytes = 256;
+constexpr int kMaxColBlock = 8;
+
+static hq_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return HQ_OK;
+  (void)cudaGetLastError();  // clear a non-sticky launch error
+  return HQ_ERR_CUDA;
+}
+
+static hq_status check_weight(const hq_weight* w) {
+  if (w == nullptr) return HQ_ERR_INVALID_ARG;
+  if (w->M <= 0 || w->K <= 0 || w->M > (1 << 28)) return HQ_ERR_INVALID_ARG;
+  if (!(w->bits == 2 || w->bits == 3 || w->bits == 4 || w->bits == 8)) {
+    return (w->bits >= 1 && w->bits <= 8) ? HQ_ERR_UNSUPPORTED : HQ_ERR_INVALID_ARG;
+  }
+  if (!is_pow2(w->K) || w->K < 128 || w->K > 16384) return HQ_ERR_UNSUPPORTED;
+  if (w->zero < 0 || w->zero >= (1 << w->bits)) return HQ_ERR_INVALID_ARG;
+  if (w->qweight == nullptr || w->scales == nullptr) return HQ_ERR_INVALID_ARG;
+  if (!aligned(w->qweight, 16) || !aligned(w->scales, 16)) return HQ_ERR_INVALID_ARG;
+  if (w->signs != nullptr && !aligned(w->signs, 16)) return HQ_ERR_INVALID_ARG;
+  return HQ_OK;
+}
+
+// Largest GEMV column block whose tile fits in one CTA's shared memory.
+static int gemv_col_block(int bits, int K) {
+  for (int nb = kMaxColBlock; nb >= 1; nb >>= 1) {
+    if (gemv_smem_bytes(bits, K, nb) != 0) return nb;
+  }
+  return 0;
+}
+
+struct LinearWs {
+  uint32_t* status;
+  uint16_t* xs;
+  float* corr;
+  size_t bytes;
+};
+
+static LinearWs linear_ws(void* base, int K) {
+  LinearWs l{};
+  const size_t xs_bytes = align256(static_cast<size_t>(kMaxColBlock) * K * 2);
+  const size_t corr_bytes = align256(static_cast<size_t>(K / 128) * kMaxColBlock * 4);
+  uint8_t* b = static_cast<uint8_t*>(base);
+  l.status = reinterpret_cast<uint32_t*>(b);
+  l.xs = reinterpret_cast<uint16_t*>(b + kStatusBytes);
+  l.corr = reinterpret_cast<float*>(b + kStatusBytes + xs_bytes);
+  l.bytes = kStatusBytes + xs_bytes + corr_bytes;
+  return l;
+}
+
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" {
+
+const char* hq_status_string(hq_status s) {
+  switch (s) {
+    case HQ_OK: return "HQ_OK";
+    case HQ_ERR_INVALID_ARG: return "HQ_ERR_INVALID_ARG: bad pointer, size, alignment or value";
+    case HQ_ERR_UNSUPPORTED: return "HQ_ERR_UNSUPPORTED: valid but not implemented";
+    case HQ_ERR_WORKSPACE: return "HQ_ERR_WORKSPACE: workspace missing, misaligned or too small";
+    case HQ_ERR_CUDA: return "HQ_ERR_CUDA: a CUDA launch or runtime call failed";
+    case HQ_ERR_DATA: return "HQ_ERR_DATA: device data out of range";
+    case HQ_ERR_TIMEOUT: return "HQ_ERR_TIMEOUT: a bounded device-side wait ran out";
+  }
+  return "HQ_ERR_UNKNOWN";
+}
+
+uint64_t hq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int hq_set_tc_min_batch(int n) {
+  if (n < 1) return g_tc_min_batch.load();
+  return g_tc_min_batch.exchange(n);
+}
+
+hq_status hq_rotate(const void* x, hq_dtype x_dtype, void* x_rot, hq_dtype out_dtype, int n_rows,
+                    int K, const int8_t* signs, hq_stream_t stream) {
+  if (n_rows < 0) return HQ_ERR_INVALID_ARG;
+  if (x_dtype < HQ_F16 || x_dtype > HQ_F32 || out_dtype < HQ_F16 || out_dtype > HQ_F32) {
+    return HQ_ERR_INVALID_ARG;
+  }
+  if (K <= 0) return HQ_ERR_INVALID_ARG;
+  if (!is_pow2(K) || K < 32 || K > 32768) return HQ_ERR_UNSUPPORTED;
+  if (n_rows == 0) return HQ_OK;
+  if (x == nullptr || x_rot == nullptr) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_rot, 16)) return HQ_ERR_INVALID_ARG;
+  if (signs != nullptr && !aligned(signs, 16)) return HQ_ERR_INVALID_ARG;
+  if (n_rows > 0x7fffffff / 2) return HQ_ERR_INVALID_ARG;
+  return from_cuda(launch_rotate(x_dtype, out_dtype, x, x_rot, n_rows, K, signs,
+                                 reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t hq_linear_workspace_size(const hq_weight* w, int batch) {
+  if (check_weight(w) != HQ_OK || batch < 0) return 0;
+  return linear_ws(nullptr, w->K).bytes;
+}
+
+int hq_linear_launches(const hq_weight* w, int batch) {
+  if (check_weight(w) != HQ_OK || batch <= 0) return 0;
+  const int nb = gemv_col_block(w->bits, w->K);
+  if (nb == 0) return 0;
+  return 2 * ((batch + nb - 1) / nb);
+}
+
+hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, void* workspace,
+                    size_t ws_bytes, hq_stream_t stream) {
+  const hq_status ws_ok = check_weight(w);
+  if (ws_ok != HQ_OK) return ws_ok;
+  if (batch < 0 || batch > 65535) return HQ_ERR_INVALID_ARG;
+  if (batch == 0) return HQ_OK;
+  if (x == nullptr || y == nullptr) return HQ_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
+  const LinearWs l = linear_ws(workspace, w->K);
+  if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < l.bytes) {
+    return HQ_ERR_WORKSPACE;
+  }
+  const int nb = gemv_col_block(w->bits, w->K);
+  if (nb == 0) return HQ_ERR_UNSUPPORTED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const __half* xh = reinterpret_cast<const __half*>(x);
+  for (int n0 = 0; n0 < batch; n0 += nb) {
+    const int nbk = batch - n0 < nb ? batch - n0 : nb;
+    cudaError_t e = launch_prep_gemv(w->bits, w->K, xh + static_cast<size_t>(n0) * w->K,
+                                     w->signs, l.xs, l.corr, nbk, w->zero, st);
+    if (e != cudaSuccess) return from_cuda(e);
+    GemvArgs a;
+    a.bits = w->bits;
+    a.M = w->M;
+    a.K = w->K;
+    a.N = nbk;
+    a.zero = w->zero;
+    a.q = w->qweight;
+    a.scales = w->scales;
+    a.xs = l.xs;
+    a.corr = l.corr;
+    a.y = y + static_cast<size_t>(n0) * w->M;
+    a.ldy = w->M;
+    a.status = l.status;
+    e = launch_gemv(a, st);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  return HQ_OK;
+}
+
+hq_status hq_check_status(void* workspace, hq_stream_t stream) {
+  if (workspace == nullptr || !aligned(workspace, 256)) return HQ_ERR_WORKSPACE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) {
+    return from_cuda(cudaErrorUnknown);
+  }
+  if (v == 0) return HQ_OK;
+  if (cudaMemset(workspace, 0, sizeof(v)) != cudaSuccess) return from_cuda(cudaErrorUnknown);
+  if (v & HQ_DEV_TIMEOUT) return HQ_ERR_TIMEOUT;
+  return HQ_ERR_DATA;
+}
+
+hq_status hq_unpack_codes(const uint32_t* packed, int bits, size_t n_codes, uint8_t* codes_out,
+                          hq_stream_t stream) {
+  if (bits < 1 || bits > 8) return HQ_ERR_INVALID_ARG;
+  if (n_codes == 0) return HQ_OK;
+  if (packed == nullptr || codes_out == nullptr || !aligned(packed, 4)) return HQ_ERR_INVALID_ARG;
+  return from_cuda(
+      launch_unpack(packed, bits, n_codes, codes_out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
+
+// The MoE entry points are defined in moe.cu.

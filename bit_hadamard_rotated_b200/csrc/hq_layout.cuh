@@ -1,0 +1,204 @@
+// hq_layout.cuh -- register-level decode of packed codes into fp16 MMA operands.
+//
+// A lane of the GEMV owns a "bundle" of 32 consecutive codes of one weight row
+// inside a 128-code group: BITS words (2-bit: 2 words, 3-bit: one 96-bit
+// triplet, 4-bit: 4 words, 8-bit: 8 words).  decode16<BITS> turns the bundle
+// into 16 half2 registers P[p], each holding two codes (lo, hi) as the fp16
+// values 1024 + (code << a): the code's bits are masked straight into the
+// mantissa of 1024.0 (exponent 0x19), with no shift when the field already
+// sits in a mantissa slot, so one LOP3 (or PRMT for bytes) yields two codes.
+//
+// kPairs<BITS>[p] names, for each half, the code index inside the bundle and
+// its shift a.  The activation side compensates exactly: the tensor-core B
+// operand holds x'_k * 2^-a_k, so the MMA computes
+//     sum_k (1024 + 2^a_k q_k) x'_k 2^-a_k = 1024 sum_k B_k + sum_k q_k x'_k
+// and the per-(group, column) constant  sum_k (1024 + zero 2^a_k) B_k  is
+// subtracted once (it is the accumulator's initial value, negated).  This is
+// how the dequantisation w = scale (q - zero) is applied inside the matmul
+// without per-weight subtract or multiply instructions; the group scale
+// multiplies the fp32 group sum.
+//
+// Step s (0..7) of a 128-code group feeds the m16n8k16 MMA with P[2s] as the
+// A-fragment columns (2t, 2t+1) and P[2s+1] as columns (2t+8, 2t+9), t = lane
+// & 3; the B fragment of lane (n, t) at that step holds the matching four
+// activations, in that order.
+#pragma once
+
+#include <stdint.h>
+
+#include "hq_common.cuh"
+
+namespace hq {
+
+struct PairDesc {
+  uint8_t c_lo, a_lo, c_hi, a_hi;
+};
+
+template <int BITS>
+struct Pairs;
+
+template <>
+struct Pairs<2> {
+  // word u (codes 16u..16u+15), pair i = codes (i, i+8): fields at 2i for
+  // i < 5, then at 2(i-5) after >> 10.
+  static __host__ __device__ constexpr PairDesc get(int p) {
+    return PairDesc{static_cast<uint8_t>(16 * (p >> 3) + (p & 7)),
+                    static_cast<uint8_t>((p & 7) < 5 ? 2 * (p & 7) : 2 * ((p & 7) - 5)),
+                    static_cast<uint8_t>(16 * (p >> 3) + (p & 7) + 8),
+                    static_cast<uint8_t>((p & 7) < 5 ? 2 * (p & 7) : 2 * ((p & 7) - 5))};
+  }
+};
+
+template <>
+struct Pairs<4> {
+  // word u (codes 8u..8u+7), pair i = codes (i, i+4): fields at 0, 4, then
+  // 0, 4 after >> 8.
+  static __host__ __device__ constexpr PairDesc get(int p) {
+    return PairDesc{static_cast<uint8_t>(8 * (p >> 2) + (p & 3)),
+                    static_cast<uint8_t>(4 * (p & 1)),
+                    static_cast<uint8_t>(8 * (p >> 2) + (p & 3) + 4),
+                    static_cast<uint8_t>(4 * (p & 1))};
+  }
+};
+
+template <>
+struct Pairs<8> {
+  // word u (codes 4u..4u+3), pair i = bytes (i, i+2) placed by PRMT.
+  static __host__ __device__ constexpr PairDesc get(int p) {
+    return PairDesc{static_cast<uint8_t>(4 * (p >> 1) + (p & 1)), 0,
+                    static_cast<uint8_t>(4 * (p >> 1) + (p & 1) + 2), 0};
+  }
+};
+
+template <>
+struct Pairs<3> {
+  // 96-bit triplet, code c at stream bits [3c, 3c+3).  Seven shifted views
+  // of the triplet each expose two or three (lo, hi) pairs whose fields lie
+  // in mantissa slots: lo within bits 0..9, hi within bits 16..25.
+  static __host__ __device__ constexpr PairDesc get(int p) {
+    constexpr uint8_t t[16][4] = {{0, 1, 5, 0},   {1, 4, 6, 3},   {2, 7, 7, 6},   {3, 1, 8, 0},
+                                  {4, 4, 9, 3},   {10, 0, 16, 2}, {11, 3, 17, 5}, {12, 0, 18, 2},
+                                  {13, 3, 19, 5}, {14, 0, 20, 2}, {15, 3, 21, 5}, {22, 1, 27, 0},
+                                  {23, 4, 28, 3}, {24, 7, 29, 6}, {25, 1, 30, 0}, {26, 4, 31, 3}};
+    return PairDesc{t[p][0], t[p][1], t[p][2], t[p][3]};
+  }
+};
+
+constexpr uint32_t kMagic = 0x64006400u;  // half2(1024, 1024)
+
+template <int BITS>
+__device__ __forceinline__ void decode16(const uint32_t (&w)[BITS], uint32_t (&P)[16]);
+
+template <>
+__device__ __forceinline__ void decode16<2>(const uint32_t (&w)[2], uint32_t (&P)[16]) {
+#pragma unroll
+  for (int u = 0; u < 2; ++u) {
+    const uint32_t x = w[u];
+    const uint32_t x2 = x >> 10;
+#pragma unroll
+    for (int i = 0; i < 5; ++i) P[8 * u + i] = and_or(x, 0x00030003u << (2 * i), kMagic);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) P[8 * u + 5 + i] = and_or(x2, 0x00030003u << (2 * i), kMagic);
+  }
+}
+
+template <>
+__device__ __forceinline__ void decode16<4>(const uint32_t (&w)[4], uint32_t (&P)[16]) {
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const uint32_t x = w[u];
+    const uint32_t x2 = x >> 8;
+    P[4 * u + 0] = and_or(x, 0x000F000Fu, kMagic);
+    P[4 * u + 1] = and_or(x, 0x00F000F0u, kMagic);
+    P[4 * u + 2] = and_or(x2, 0x000F000Fu, kMagic);
+    P[4 * u + 3] = and_or(x2, 0x00F000F0u, kMagic);
+  }
+}
+
+template <>
+__device__ __forceinline__ void decode16<8>(const uint32_t (&w)[8], uint32_t (&P)[16]) {
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    P[2 * u + 0] = prmt(w[u], 0x64646464u, 0x4240u);
+    P[2 * u + 1] = prmt(w[u], 0x64646464u, 0x4341u);
+  }
+}
+
+__device__ __forceinline__ constexpr uint32_t m3(int a_lo, int a_hi) {
+  return (7u << a_lo) | (7u << (16 + a_hi));
+}
+
+template <>
+__device__ __forceinline__ void decode16<3>(const uint32_t (&w)[3], uint32_t (&P)[16]) {
+  const uint32_t v1 = w[0] << 1;
+  const uint32_t v2 = w[0] >> 8;
+  const uint32_t v3 = funnel_r(w[0], w[1], 30);
+  const uint32_t v4 = w[1] >> 4;
+  const uint32_t v5 = funnel_r(w[1], w[2], 10);
+  const uint32_t v6 = w[2] >> 1;
+  const uint32_t v7 = w[2] >> 10;
+  P[0] = and_or(v1, m3(1, 0), kMagic);
+  P[1] = and_or(v1, m3(4, 3), kMagic);
+  P[2] = and_or(v1, m3(7, 6), kMagic);
+  P[3] = and_or(v2, m3(1, 0), kMagic);
+  P[4] = and_or(v2, m3(4, 3), kMagic);
+  P[5] = and_or(v3, m3(0, 2), kMagic);
+  P[6] = and_or(v3, m3(3, 5), kMagic);
+  P[7] = and_or(v4, m3(0, 2), kMagic);
+  P[8] = and_or(v4, m3(3, 5), kMagic);
+  P[9] = and_or(v5, m3(0, 2), kMagic);
+  P[10] = and_or(v5, m3(3, 5), kMagic);
+  P[11] = and_or(v6, m3(1, 0), kMagic);
+  P[12] = and_or(v6, m3(4, 3), kMagic);
+  P[13] = and_or(v6, m3(7, 6), kMagic);
+  P[14] = and_or(v7, m3(1, 0), kMagic);
+  P[15] = and_or(v7, m3(4, 3), kMagic);
+}
+
+// Load a lane's BITS-word bundle from shared memory (16-byte aligned for
+// BITS 4 and 8, 8-byte for BITS 2, 4-byte for BITS 3).
+template <int BITS>
+__device__ __forceinline__ void load_bundle(const uint8_t* p, uint32_t (&w)[BITS]);
+
+template <>
+__device__ __forceinline__ void load_bundle<2>(const uint8_t* p, uint32_t (&w)[2]) {
+  const uint2 v = *reinterpret_cast<const uint2*>(p);
+  w[0] = v.x;
+  w[1] = v.y;
+}
+template <>
+__device__ __forceinline__ void load_bundle<3>(const uint8_t* p, uint32_t (&w)[3]) {
+  const uint32_t* q = reinterpret_cast<const uint32_t*>(p);
+  w[0] = q[0];
+  w[1] = q[1];
+  w[2] = q[2];
+}
+template <>
+__device__ __forceinline__ void load_bundle<4>(const uint8_t* p, uint32_t (&w)[4]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  w[0] = v.x;
+  w[1] = v.y;
+  w[2] = v.z;
+  w[3] = v.w;
+}
+template <>
+__device__ __forceinline__ void load_bundle<8>(const uint8_t* p, uint32_t (&w)[8]) {
+  const uint4 v = *reinterpret_cast<const uint4*>(p);
+  const uint4 u = *reinterpret_cast<const uint4*>(p + 16);
+  w[0] = v.x;
+  w[1] = v.y;
+  w[2] = v.z;
+  w[3] = v.w;
+  w[4] = u.x;
+  w[5] = u.y;
+  w[6] = u.z;
+  w[7] = u.w;
+}
+
+// Shared-memory row stride (in 32-bit words, mod 32) that keeps the lanes'
+// bundle loads free of bank conflicts (8 rows x 4 lanes per warp).
+__host__ __device__ constexpr int bank_target_words(int bits) {
+  return bits == 2 ? 8 : bits == 3 ? 4 : bits == 4 ? 16 : 4;
+}
+
+}  // namespace hq

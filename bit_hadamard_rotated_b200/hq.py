@@ -1,0 +1,171 @@
+"""Python entry points with the C ABI's names (include/hq.h).
+
+Each function checks tensor devices/dtypes/shapes, marshals pointers and the
+current CUDA stream, and calls libhq.  Nothing is computed here.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from ._lib import (HQ_BF16, HQ_F16, HQ_F32, HqError, HqExpert, HqWeight, check, lib)
+
+_DT = {torch.float16: HQ_F16, torch.bfloat16: HQ_BF16, torch.float32: HQ_F32}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("libhq takes CUDA tensors only (no CPU fallback)")
+
+
+def hq_rotate(x: torch.Tensor, signs: torch.Tensor | None = None, out_dtype=torch.float32,
+              out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """x' = H_K diag(s) x / sqrt(K) for every row of x ([..., K])."""
+    _need_cuda(x, signs)
+    K = x.shape[-1]
+    x = x.contiguous()
+    if out is None:
+        out = torch.empty(x.shape, dtype=out_dtype, device=x.device)
+    n_rows = x.numel() // K if K else 0
+    st = lib().hq_rotate(_ptr(x), _DT[x.dtype], _ptr(out), _DT[out.dtype], n_rows, K,
+                         _ptr(signs), _stream(stream))
+    check(st, "hq_rotate")
+    return out
+
+
+def make_weight(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
+                bits: int, zero: int | None = None) -> HqWeight:
+    M = qweight.shape[0]
+    K = qweight.shape[1] * 32 // bits
+    z = (1 << (bits - 1)) if zero is None else int(zero)
+    return HqWeight(bits, M, K, z, qweight.data_ptr(), scales.data_ptr(),
+                    None if signs is None else signs.data_ptr())
+
+
+def hq_linear_workspace_size(w: HqWeight, batch: int) -> int:
+    return int(lib().hq_linear_workspace_size(ctypes.byref(w), batch))
+
+
+def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
+              x: torch.Tensor, bits: int, zero: int | None = None,
+              out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """y[n][m] = sum_k scale (q - zero) x'[n][k]; x fp16 [N][K] -> y fp32 [N][M]."""
+    _need_cuda(qweight, scales, signs, x)
+    w = make_weight(qweight, scales, signs, bits, zero)
+    N = x.shape[0]
+    if out is None:
+        out = torch.empty((N, w.M), dtype=torch.float32, device=x.device)
+    need = hq_linear_workspace_size(w, N)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
+    st = lib().hq_linear(ctypes.byref(w), _ptr(x), N, _ptr(out), _ptr(workspace),
+                         workspace.numel(), _stream(stream))
+    check(st, "hq_linear")
+    return out
+
+
+class RotatedLinear:
+    """A packed, rotated linear layer bound to its device tensors and workspace."""
+
+    def __init__(self, qweight, scales, signs, bits, zero=None, max_batch=64):
+        _need_cuda(qweight, scales, signs)
+        self.qweight, self.scales, self.signs, self.bits = qweight, scales, signs, bits
+        self.w = make_weight(qweight, scales, signs, bits, zero)
+        self.workspace = torch.zeros(max(hq_linear_workspace_size(self.w, max_batch), 256),
+                                     dtype=torch.uint8, device=qweight.device)
+
+    @property
+    def M(self):
+        return self.w.M
+
+    @property
+    def K(self):
+        return self.w.K
+
+    def launches(self, batch: int) -> int:
+        return int(lib().hq_linear_launches(ctypes.byref(self.w), batch))
+
+    def __call__(self, x, out=None, stream=None):
+        N = x.shape[0]
+        if out is None:
+            out = torch.empty((N, self.w.M), dtype=torch.float32, device=x.device)
+        st = lib().hq_linear(ctypes.byref(self.w), _ptr(x), N, _ptr(out), _ptr(self.workspace),
+                             self.workspace.numel(), _stream(stream))
+        check(st, "hq_linear")
+        return out
+
+    def check_status(self, stream=None):
+        check(lib().hq_check_status(_ptr(self.workspace), _stream(stream)), "device status")
+
+
+def hq_moe_workspace_size(n_experts, hidden, inter, T, k) -> int:
+    return int(lib().hq_moe_workspace_size(n_experts, hidden, inter, T, k))
+
+
+def expert_table(experts: list[dict], device) -> torch.Tensor:
+    """Device array of hq_expert descriptors (bytes) for a list of expert dicts
+    holding CUDA tensors q_gate, q_up, q_down, s_gate, s_up, s_down."""
+    arr = (HqExpert * len(experts))()
+    for i, e in enumerate(experts):
+        arr[i] = HqExpert(int(e["bits"]), int(e["zero"]), *[e[n].data_ptr() for n in
+                          ("q_gate", "q_up", "q_down", "s_gate", "s_up", "s_down")])
+    raw = bytes(memoryview(arr).cast("B"))
+    return torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(device)
+
+
+def hq_moe_experts(table: torch.Tensor, n_experts: int, hidden: int, inter: int,
+                   x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor,
+                   signs_in: torch.Tensor | None, signs_mid: torch.Tensor | None,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    _need_cuda(table, x, topk_ids, topk_w, signs_in, signs_mid)
+    T, k = topk_ids.shape
+    if out is None:
+        out = torch.empty((T, hidden), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.zeros(max(hq_moe_workspace_size(n_experts, hidden, inter, T, k), 256),
+                                dtype=torch.uint8, device=x.device)
+    st = lib().hq_moe_experts(_ptr(table), n_experts, hidden, inter, _ptr(x), T, _ptr(topk_ids),
+                              _ptr(topk_w), k, _ptr(signs_in), _ptr(signs_mid), _ptr(out),
+                              _ptr(workspace), workspace.numel(), _stream(stream))
+    check(st, "hq_moe_experts")
+    return out
+
+
+def hq_check_status(workspace: torch.Tensor, stream=None) -> None:
+    check(lib().hq_check_status(_ptr(workspace), _stream(stream)), "device status")
+
+
+def hq_unpack_codes(packed: torch.Tensor, bits: int, n_codes: int,
+                    out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    _need_cuda(packed)
+    if out is None:
+        out = torch.empty(n_codes, dtype=torch.uint8, device=packed.device)
+    check(lib().hq_unpack_codes(_ptr(packed), bits, n_codes, _ptr(out), _stream(stream)),
+          "hq_unpack_codes")
+    return out
+
+
+def hq_launch_count() -> int:
+    return int(lib().hq_launch_count())
+
+
+def hq_set_tc_min_batch(n: int) -> int:
+    return int(lib().hq_set_tc_min_batch(n))
+
+
+__all__ = ["hq_rotate", "hq_linear", "hq_linear_workspace_size", "RotatedLinear",
+           "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
+           "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

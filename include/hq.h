@@ -1,0 +1,187 @@
+/*
+ * hq.h -- C ABI of libhq: matmuls over packed low-bit, Hadamard-rotated
+ * weights on NVIDIA B200 (sm_100a).
+ *
+ * The method (LLaDA2.2-mini Orin-Nano model card, Properties table and the
+ * file-list paragraph): routed-expert weights are "group-128 GPTQ in a
+ * Hadamard-rotated basis", 2/3/4 bits per expert, non-expert layers 8-bit,
+ * with the rotation signs stored beside them.  The weights stay packed for
+ * the whole run and are dequantised inside the matmul (Qwen3-8B BPDQ 2-bit
+ * card, introduction: "kept that way for the whole run"; decode time follows
+ * the weight bytes: Laguna-S-2.1 gridbook card, "Reading it honestly").
+ *
+ * Definitions used by every entry point (this library's reading of the pages,
+ * which give no formulas):
+ *   rotation     x' = H_K . diag(s) . x / sqrt(K)
+ *                H_K: Sylvester Hadamard matrix, natural order,
+ *                H[i][j] = (-1)^popcount(i & j); s_i = -1 if signs[i] < 0,
+ *                else +1; signs == NULL means s = 1.
+ *   codes        row m of a packed matrix is K*bits/32 uint32 words; code k of
+ *                the row occupies bits [bits*k, bits*k + bits) of the row's
+ *                little-endian bit stream (word w holds stream bits
+ *                [32w, 32w+32)).  For bits = 3, three words carry 32 codes and
+ *                codes 10 and 21 of each triplet straddle a word boundary.
+ *   dequant      w[m][k] = scale[m][k/128] * (q[m][k] - zero), group size 128
+ *                along K, scale an IEEE fp16 bit pattern, zero an integer.
+ *   linear       y[n][m] = sum_k w[m][k] * x'[n][k], fp32 output.
+ *
+ * Conventions:
+ *   - Every pointer argument is a DEVICE pointer owned by the caller unless
+ *     stated otherwise.  The library allocates and frees nothing.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream) and returns before the work finishes, except
+ *     hq_check_status, which synchronises the stream.
+ *   - Argument errors are detected on the host before anything is launched;
+ *     the call then returns the status and writes nothing.  A launch failure
+ *     returns HQ_ERR_CUDA.  Errors found by device code (a bounded wait that
+ *     ran out, an expert id or bit width out of range in device data) are
+ *     OR-ed into the status word at the start of the caller's workspace and
+ *     read back by hq_check_status; device code never traps.
+ *   - A workspace must be at least the queried size, 256-byte aligned, and its
+ *     first 256 bytes must be zero before its first use (the status word).
+ *   - Outputs are overwritten, never accumulated into.  Inputs and outputs
+ *     must not alias.
+ *   - Alignment: packed weights, scales, activations and outputs must be
+ *     16-byte aligned; the library checks this and returns
+ *     HQ_ERR_INVALID_ARG otherwise.
+ */
+#ifndef HQ_H
+#define HQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+/* The same handle as cudaStream_t. */
+typedef struct CUstream_st* hq_stream_t;
+
+typedef enum {
+  HQ_OK = 0,
+  HQ_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or value */
+  HQ_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. K not a power of two) */
+  HQ_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or smaller than queried */
+  HQ_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+  HQ_ERR_DATA = 5,        /* device data out of range (expert id, bits, zero) */
+  HQ_ERR_TIMEOUT = 6      /* a bounded device-side wait ran out */
+} hq_status;
+
+typedef enum { HQ_F16 = 0, HQ_BF16 = 1, HQ_F32 = 2 } hq_dtype;
+
+/* One packed, rotated weight matrix W [M][K]. */
+typedef struct {
+  int bits;                /* 2, 3, 4 or 8 */
+  int M;                   /* output features, >= 1 */
+  int K;                   /* input features: power of two, 128 <= K <= 16384 */
+  int zero;                /* integer zero point, 0 <= zero < 2^bits (2^(bits-1) usual) */
+  const uint32_t* qweight; /* [M][K*bits/32] packed codes, 16-byte aligned */
+  const uint16_t* scales;  /* [M][K/128] fp16 bit patterns, 16-byte aligned */
+  const int8_t* signs;     /* [K] rotation signs, or NULL for s = 1 */
+} hq_weight;
+
+/*
+ * hq_rotate -- the random-sign Hadamard rotation alone, row by row.
+ *   x_rot[r][:] = H_K diag(s) x[r][:] / sqrt(K),   r < n_rows.
+ * x: [n_rows][K] of x_dtype (HQ_F16, HQ_BF16 or HQ_F32), row-major.
+ * x_rot: [n_rows][K] of out_dtype (HQ_F16, HQ_BF16 or HQ_F32).
+ * K: power of two, 32 <= K <= 32768.  n_rows >= 0 (0 launches nothing).
+ * Computed in fp32 (butterflies), rounded once to out_dtype.
+ * Cites: "Hadamard-rotated basis" and "rotation signs" (LLaDA2.2-mini
+ * Orin-Nano model card, Properties table, file list); "behind a random
+ * Hadamard rotation" (Qwen3.8-27B Pingala-8 2-bit card, "What this is").
+ */
+hq_status hq_rotate(const void* x, hq_dtype x_dtype, void* x_rot, hq_dtype out_dtype,
+                    int n_rows, int K, const int8_t* signs, hq_stream_t stream);
+
+/* Bytes of workspace hq_linear needs for this weight and batch (0 on a bad
+ * argument).  Constant for a given (bits, M, K, batch). */
+size_t hq_linear_workspace_size(const hq_weight* w, int batch);
+
+/*
+ * hq_linear -- y = dequant(Q) . x' with x' the rotated activations:
+ *   y[n][m] = sum_k scale[m][k/128] (q[m][k] - zero) (H_K diag(s) x[n] / sqrt(K))[k]
+ * w: host pointer to the weight descriptor (device pointers inside).
+ * x: [batch][K] fp16 activations.  batch >= 0 (0 launches nothing).
+ * y: [batch][M] fp32 output.
+ * workspace: >= hq_linear_workspace_size(w, batch) bytes.
+ * Small batches run a fused unpack-dequant kernel that streams the packed
+ * codes; larger batches run a tensor-core GEMM.  Both accumulate in fp32.
+ * Cites: group-128 codes, 2/3/4-bit experts and 8-bit non-expert layers
+ * (LLaDA2.2-mini Orin-Nano model card, Properties table).
+ */
+hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y,
+                    void* workspace, size_t ws_bytes, hq_stream_t stream);
+
+/* One routed expert: SwiGLU FFN with packed gate/up [inter][hidden] and
+ * down [hidden][inter], all at one bit width.  Device-side table entry. */
+typedef struct {
+  int bits;               /* 2, 3 or 4 (8 also accepted) */
+  int zero;               /* 0 <= zero < 2^bits */
+  const uint32_t* q_gate; /* [inter][hidden*bits/32] */
+  const uint32_t* q_up;   /* [inter][hidden*bits/32] */
+  const uint32_t* q_down; /* [hidden][inter*bits/32] */
+  const uint16_t* s_gate; /* [inter][hidden/128] fp16 */
+  const uint16_t* s_up;   /* [inter][hidden/128] fp16 */
+  const uint16_t* s_down; /* [hidden][inter/128] fp16 */
+} hq_expert;
+
+size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k);
+
+/*
+ * hq_moe_experts -- the routed-expert part of an MoE layer, all experts and
+ * bit widths in one pass per phase, no host synchronisation:
+ *   x'_t  = H_hidden diag(s_in) x_t / sqrt(hidden)
+ *   g, u  = W_gate^e x'_t,  W_up^e x'_t           for e = topk_ids[t][j]
+ *   h     = g / (1 + exp(-g)) * u                  (SwiGLU)
+ *   h'    = H_inter diag(s_mid) h / sqrt(inter)
+ *   d     = W_down^e h'
+ *   y_t   = sum_{j=0..k-1} topk_w[t][j] * d_{t,j}  (j ascending, fixed order)
+ * experts: DEVICE array [n_experts] of hq_expert.  x: [T][hidden] fp16.
+ * topk_ids: [T][k] int32, topk_w: [T][k] fp32.  signs_in [hidden], signs_mid
+ * [inter] (NULL = no sign flip).  y: [T][hidden] fp32.
+ * hidden, inter: powers of two in [128, 16384].  1 <= k <= 32.
+ * An expert id outside [0, n_experts), or an expert whose bits or zero is out
+ * of range, is skipped (its contribution is zero) and sets HQ_ERR_DATA in the
+ * workspace status word.
+ * Cites: mixed 2/3/4-bit routed experts with per-expert widths in a manifest
+ * and the 32-token denoising block (LLaDA2.2-mini Orin-Nano model card,
+ * Properties table and "Measured Throughput").
+ */
+hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, int inter,
+                         const uint16_t* x, int T, const int32_t* topk_ids,
+                         const float* topk_w, int k, const int8_t* signs_in,
+                         const int8_t* signs_mid, float* y, void* workspace,
+                         size_t ws_bytes, hq_stream_t stream);
+
+/* Synchronises `stream`, reads the status word of a workspace used by
+ * hq_linear or hq_moe_experts, clears it, and returns HQ_OK or the first
+ * recorded device error (HQ_ERR_TIMEOUT before HQ_ERR_DATA). */
+hq_status hq_check_status(void* workspace, hq_stream_t stream);
+
+/*
+ * hq_unpack_codes -- decode n_codes codes of width bits (1..8) from a packed
+ * little-endian bit stream into one byte each.  Bit-exact; test-facing.
+ */
+hq_status hq_unpack_codes(const uint32_t* packed, int bits, size_t n_codes,
+                          uint8_t* codes_out, hq_stream_t stream);
+
+/* Static string for a status code. */
+const char* hq_status_string(hq_status s);
+
+/* Total number of kernels this process has enqueued through libhq. */
+uint64_t hq_launch_count(void);
+
+/* Kernels one hq_linear call enqueues for this weight and batch. */
+int hq_linear_launches(const hq_weight* w, int batch);
+
+/* Batch size from which hq_linear uses the tensor-core GEMM (default 9).
+ * Returns the previous value; values < 1 are ignored. */
+int hq_set_tc_min_batch(int n);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HQ_H */

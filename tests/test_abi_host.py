@@ -1,0 +1,111 @@
+"""Host-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments on the host before launching
+anything (these calls never reach the GPU, so they run on a CPU-only box)."""
+import ctypes
+
+import pytest
+
+from bit_hadamard_rotated_b200 import _lib
+from bit_hadamard_rotated_b200._lib import (HQ_ERR_INVALID_ARG, HQ_ERR_UNSUPPORTED,
+                                            HQ_ERR_WORKSPACE, HQ_OK, HqWeight)
+
+FAKE = 0x100000  # aligned, never dereferenced: every call below fails validation first
+
+
+@pytest.fixture(scope="module")
+def L():
+    from bit_hadamard_rotated_b200 import build
+    build.build()
+    return _lib.lib()
+
+
+def test_exports_every_declared_function(L):
+    names = _lib.header_functions()
+    assert {"hq_rotate", "hq_linear", "hq_moe_experts", "hq_unpack_codes",
+            "hq_check_status", "hq_linear_workspace_size", "hq_moe_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for s in range(7):
+        assert _lib.status_string(s).startswith("HQ_")
+
+
+def W(**kw):
+    d = dict(bits=4, M=64, K=4096, zero=8, qweight=FAKE, scales=FAKE, signs=None)
+    d.update(kw)
+    return HqWeight(d["bits"], d["M"], d["K"], d["zero"], d["qweight"], d["scales"], d["signs"])
+
+
+def lin(L, w, batch=1, x=FAKE, y=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    return L.hq_linear(None if w is None else ctypes.byref(w), x, batch, y, ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("kw,want", [
+    (dict(bits=5), HQ_ERR_UNSUPPORTED), (dict(bits=0), HQ_ERR_INVALID_ARG),
+    (dict(bits=9), HQ_ERR_INVALID_ARG), (dict(K=4096 + 128), HQ_ERR_UNSUPPORTED),
+    (dict(K=64), HQ_ERR_UNSUPPORTED), (dict(K=32768), HQ_ERR_UNSUPPORTED),
+    (dict(K=0), HQ_ERR_INVALID_ARG), (dict(M=0), HQ_ERR_INVALID_ARG),
+    (dict(zero=16), HQ_ERR_INVALID_ARG), (dict(zero=-1), HQ_ERR_INVALID_ARG),
+    (dict(qweight=FAKE + 8), HQ_ERR_INVALID_ARG), (dict(scales=FAKE + 2), HQ_ERR_INVALID_ARG),
+    (dict(signs=FAKE + 1), HQ_ERR_INVALID_ARG), (dict(qweight=None), HQ_ERR_INVALID_ARG),
+])
+def test_linear_rejects_bad_weight(L, kw, want):
+    before = L.hq_launch_count()
+    assert lin(L, W(**kw)) == want
+    assert L.hq_launch_count() == before
+
+
+def test_linear_rejects_bad_call_args(L):
+    before = L.hq_launch_count()
+    w = W()
+    assert lin(L, None) == HQ_ERR_INVALID_ARG
+    assert lin(L, w, batch=-1) == HQ_ERR_INVALID_ARG
+    assert lin(L, w, batch=0) == HQ_OK                     # nothing to do, nothing launched
+    assert lin(L, w, x=None) == HQ_ERR_INVALID_ARG
+    assert lin(L, w, x=FAKE + 2) == HQ_ERR_INVALID_ARG
+    assert lin(L, w, y=FAKE + 4) == HQ_ERR_INVALID_ARG
+    assert lin(L, w, ws=None) == HQ_ERR_WORKSPACE
+    assert lin(L, w, ws=FAKE + 16) == HQ_ERR_WORKSPACE     # needs 256-byte alignment
+    need = L.hq_linear_workspace_size(ctypes.byref(w), 1)
+    assert need > 0
+    assert lin(L, w, ws_bytes=need - 1) == HQ_ERR_WORKSPACE
+    assert L.hq_launch_count() == before
+
+
+def test_workspace_size_queries(L):
+    assert L.hq_linear_workspace_size(ctypes.byref(W(bits=7)), 1) == 0
+    assert L.hq_linear_workspace_size(ctypes.byref(W()), -1) == 0
+    a = L.hq_linear_workspace_size(ctypes.byref(W(K=4096)), 1)
+    b = L.hq_linear_workspace_size(ctypes.byref(W(K=8192)), 1)
+    assert 0 < a < b and a % 256 == 0
+
+
+def test_rotate_rejects_bad_args(L):
+    before = L.hq_launch_count()
+    r = lambda **kw: L.hq_rotate(kw.get("x", FAKE), kw.get("xd", 0), kw.get("o", FAKE),
+                                 kw.get("od", 2), kw.get("n", 1), kw.get("K", 1024),
+                                 kw.get("s", None), None)
+    assert r(K=100) == HQ_ERR_UNSUPPORTED
+    assert r(K=16) == HQ_ERR_UNSUPPORTED
+    assert r(K=65536) == HQ_ERR_UNSUPPORTED
+    assert r(K=0) == HQ_ERR_INVALID_ARG
+    assert r(n=-1) == HQ_ERR_INVALID_ARG
+    assert r(n=0) == HQ_OK
+    assert r(xd=7) == HQ_ERR_INVALID_ARG
+    assert r(od=-1) == HQ_ERR_INVALID_ARG
+    assert r(x=None) == HQ_ERR_INVALID_ARG
+    assert r(x=FAKE + 2) == HQ_ERR_INVALID_ARG
+    assert r(s=FAKE + 3) == HQ_ERR_INVALID_ARG
+    assert L.hq_launch_count() == before
+
+
+def test_unpack_rejects_bad_args(L):
+    before = L.hq_launch_count()
+    assert L.hq_unpack_codes(FAKE, 0, 10, FAKE, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_unpack_codes(FAKE, 9, 10, FAKE, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_unpack_codes(FAKE, 3, 0, FAKE, None) == HQ_OK
+    assert L.hq_unpack_codes(FAKE + 2, 3, 10, FAKE, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_unpack_codes(None, 3, 10, FAKE, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_launch_count() == before

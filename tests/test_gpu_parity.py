@@ -1,0 +1,214 @@
+"""GPU parity: libhq (through the C ABI) against the fp64 CPU oracle.
+
+Tolerances:
+  * unpack: bit-exact.
+  * rotation, fp32 output: |d_i| <= (log2 K + 2) 2^-24 sum_j|x_j| / sqrt(K) + 1e-12
+    (one fp32 rounding per butterfly stage of values bounded by sum|x|/sqrt(K)
+    after scaling, plus the final scale); fp16/bf16 output adds one rounding
+    of x' (2^-11 / 2^-8 relative, 2^-25 absolute for fp16 subnormals).
+  * linear / MoE: |y - y_oracle| <= 2e-3 sum_k |w_k x'_k| + 1e-5 per element,
+    with the sum taken by the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_hadamard_rotated_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2e-3, 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_hadamard_rotated_b200 import build
+    build.build()
+    import bit_hadamard_rotated_b200._lib as L
+    L.lib()
+    return torch.device("cuda:0")
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def assert_within(y, want, bound, rel=REL, abs_=ABS, what=""):
+    err = np.abs(y.astype(np.float64) - want)
+    lim = rel * bound + abs_
+    bad = err > lim
+    if bad.any():
+        i = np.unravel_index(np.argmax(err / lim), err.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {err.size} outside tolerance; worst at {i}: "
+                             f"got {y[i]!r} want {want[i]!r} err {err[i]:.3e} lim {lim[i]:.3e}")
+
+
+# ---------------------------------------------------------------- unpack (bit-exact)
+@pytest.mark.parametrize("bits", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_unpack_codes_bit_exact(bits):
+    from bit_hadamard_rotated_b200 import hq_unpack_codes
+    rng = np.random.default_rng(bits)
+    n = 32 * 40000 + (0 if bits in (1, 2, 4, 8) else 0)
+    words = rng.integers(0, 2**32, size=n * bits // 32, dtype=np.uint64).astype(np.uint32)
+    # pattern words at the front: all ones, alternating bits, single bits
+    words[:3] = [0xFFFFFFFF, 0xAAAAAAAA, 0x55555555]
+    got = hq_unpack_codes(dev(words.view(np.int32)), bits, n).cpu().numpy()
+    assert np.array_equal(got, oracle.unpack(words, bits, n))
+
+
+def test_unpack_ragged_tail_does_not_read_past_end():
+    from bit_hadamard_rotated_b200 import hq_unpack_codes
+    words = np.array([0x88FAC688, 0xC688FAC6], np.uint32)  # 64 bits -> 21 whole 3-bit codes
+    got = hq_unpack_codes(dev(words.view(np.int32)), 3, 21).cpu().numpy()
+    assert np.array_equal(got, oracle.unpack(words, 3, 21))
+
+
+# ---------------------------------------------------------------- rotation
+@pytest.mark.parametrize("K", [32, 64, 128, 512, 2048, 4096, 8192, 32768])
+@pytest.mark.parametrize("in_dt,out_dt", [(torch.float16, torch.float32),
+                                          (torch.float32, torch.float32),
+                                          (torch.float16, torch.float16),
+                                          (torch.bfloat16, torch.bfloat16)])
+def test_rotate_parity(K, in_dt, out_dt):
+    from bit_hadamard_rotated_b200 import hq_rotate
+    rng = np.random.default_rng(K)
+    rows = 5
+    x = rng.standard_normal((rows, K)) * np.where(rng.random(K) < 0.01, 20.0, 1.0)
+    s = synth.signs(rng, K)
+    xt = torch.from_numpy(x).to(in_dt)
+    x_used = xt.float().double().numpy()  # the exact input values the kernel sees
+    got = hq_rotate(xt.cuda(), dev(s), out_dtype=out_dt).float().cpu().numpy()
+    want = oracle.rotate(x_used, s)
+    L = math.log2(K)
+    bound = (L + 2) * 2.0**-24 * np.abs(x_used).sum(axis=1, keepdims=True) / math.sqrt(K)
+    bound = bound + 1e-12
+    if out_dt == torch.float16:
+        bound = bound + 2.0**-11 * np.abs(want) + 2.0**-25
+    if out_dt == torch.bfloat16:
+        bound = bound + 2.0**-8 * np.abs(want) + 1e-38
+    assert np.all(np.abs(got - want) <= bound), np.max(np.abs(got - want) / bound)
+
+
+def test_rotate_null_signs_and_zero_rows():
+    from bit_hadamard_rotated_b200 import hq_rotate
+    K = 1024
+    x = torch.zeros((3, K), dtype=torch.float16)
+    x[0, 0] = 1.0
+    x[1] = 1.0
+    got = hq_rotate(x.cuda(), None).cpu().numpy()
+    assert np.allclose(got[0], 1 / math.sqrt(K), atol=1e-7)
+    assert abs(got[1, 0] - math.sqrt(K)) < 1e-4 and np.allclose(got[1, 1:], 0, atol=1e-5)
+    assert np.array_equal(got[2], np.zeros(K, np.float32))
+    empty = hq_rotate(torch.zeros((0, K), dtype=torch.float16).cuda())
+    assert empty.shape == (0, K)
+
+
+# ---------------------------------------------------------------- linear, small shapes (full check)
+def run_linear(d, out=None):
+    from bit_hadamard_rotated_b200 import hq_linear
+    return hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]),
+                     dev(d["x"]), d["bits"], d["zero"], out=out)
+
+
+SMALL = [(16, 128, 1), (17, 256, 3), (33, 512, 8), (100, 1024, 5), (64, 4096, 2),
+         (257, 2048, 7), (5, 128, 9), (40, 8192, 4), (16, 16384, 1), (48, 1024, 17),
+         (1, 128, 1), (31, 256, 16)]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("M,K,N", SMALL)
+def test_linear_parity_small(bits, M, K, N):
+    d = synth.linear(M, K, bits, N, seed=7 * M + K + N)
+    y = run_linear(d).cpu().numpy()
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y, want, bound, what=f"b{bits} M{M} K{K} N{N}")
+
+
+@pytest.mark.parametrize("bits", [2, 4])
+def test_linear_outliers_and_loguniform_scales(bits):
+    d = synth.linear(96, 8192, bits, 3, seed=3, scale_dist="loguniform", outlier_frac=0.01)
+    y = run_linear(d).cpu().numpy()
+    want, bound = oracle.linear(bits, 96, 8192, d["zero"], d["q"], d["scales"], d["signs"],
+                                d["x"])
+    assert_within(y, want, bound, what="outliers")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_linear_nondefault_zero_and_null_signs(bits):
+    d = synth.linear(40, 512, bits, 2, seed=11)
+    d["zero"] = (1 << bits) - 1
+    d["signs"] = None
+    from bit_hadamard_rotated_b200 import hq_linear
+    y = hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), None, dev(d["x"]), bits,
+                  d["zero"]).cpu().numpy()
+    want, bound = oracle.linear(bits, 40, 512, d["zero"], d["q"], d["scales"], None, d["x"])
+    assert_within(y, want, bound, what="zero/null signs")
+
+
+def test_linear_special_codes():
+    """All codes at the zero point give exactly 0; all at zero+1 give scale * sum x'."""
+    bits, M, K, N = 4, 32, 1024, 3
+    d = synth.linear(M, K, bits, N, seed=5)
+    q0 = np.stack([oracle.pack(np.full(K, 8, np.uint8), bits)] * M)
+    d0 = dict(d, q=q0)
+    y0 = run_linear(d0).cpu().numpy()
+    assert np.array_equal(y0, np.zeros((N, M), np.float32))
+    q1 = np.stack([oracle.pack(np.full(K, 9, np.uint8), bits)] * M)
+    d1 = dict(d, q=q1)
+    y1 = run_linear(d1).cpu().numpy()
+    want, bound = oracle.linear(bits, M, K, 8, q1, d["scales"], d["signs"], d["x"])
+    assert_within(y1, want, bound, what="constant codes")
+
+
+def test_linear_batch_zero_and_determinism():
+    from bit_hadamard_rotated_b200 import hq_linear
+    d = synth.linear(256, 4096, 2, 4, seed=9)
+    a = run_linear(d)
+    b = run_linear(d)
+    assert torch.equal(a, b)
+    empty = hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]),
+                      dev(d["x"][:0]), 2)
+    assert empty.shape == (0, 256)
+
+
+def test_linear_output_overwritten_not_accumulated():
+    d = synth.linear(64, 1024, 3, 2, seed=12)
+    out = torch.full((2, 64), 123.0, device="cuda")
+    y = run_linear(d, out=out).cpu().numpy()
+    want, bound = oracle.linear(3, 64, 1024, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y, want, bound, what="overwrite")
+
+
+# ---------------------------------------------------------------- linear, full workload sizes (sampled rows)
+def sample_rows(M, rng, n=24):
+    rows = set(range(0, 8)) | set(range(M - 8, M)) | set(rng.choice(M, n, replace=False).tolist())
+    return sorted(rows)
+
+
+FULL = [
+    # (M, K, bits, N, scale_dist, outlier_frac)
+    (4096, 4096, 4, 1, "uniform", 0.0),
+    (12288, 4096, 2, 1, "uniform", 0.0), (12288, 4096, 2, 8, "uniform", 0.0),
+    (12288, 4096, 3, 1, "uniform", 0.0), (12288, 4096, 3, 4, "uniform", 0.0),
+    (12288, 4096, 8, 1, "uniform", 0.0), (12288, 4096, 8, 2, "uniform", 0.0),
+    (28672, 8192, 2, 1, "loguniform", 0.01), (28672, 8192, 2, 16, "loguniform", 0.01),
+    (28672, 8192, 2, 64, "loguniform", 0.01),
+    (8192, 8192, 3, 32, "uniform", 0.0), (8192, 8192, 8, 128, "uniform", 0.0),
+]
+
+
+@pytest.mark.parametrize("M,K,bits,N,sd,of", FULL)
+def test_linear_parity_full_size_sampled(M, K, bits, N, sd, of):
+    d = synth.linear(M, K, bits, N, seed=1, scale_dist=sd, outlier_frac=of)
+    y = run_linear(d).cpu().numpy()
+    rng = np.random.default_rng(M + N)
+    for m in sample_rows(M, rng):
+        want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"],
+                                    d["x"], m_begin=m, m_end=m + 1)
+        assert_within(y[:, m], want[:, m], bound[:, m], what=f"row {m}")
+    assert np.all(np.isfinite(y))
