@@ -356,27 +356,26 @@ def measure_e2e(device, layers, xs, a):
 
 # ---------------------------------------------------------------- CPU oracle baseline
 def cpu_baseline(seconds: float):
-    """The fp64 oracle as it stands, on this host's cores, over a bounded sample
-    of the workload (the first R rows of each layer, batch 1), scaled to GB/s."""
+    """The fp64 oracle as it stands, on this host's cores (rows split across
+    threads), over a bounded sample: whole passes over the workload's three
+    layers at batch 1, repeated until about `seconds` of wall time."""
     import oracle
     cores = os.cpu_count() or 1
     ds = [synth.linear(M, K, b, 1, seed=99) for (M, K, b) in LAYERS]
-    probe = 64
+    passes = 0
     t0 = time.perf_counter()
-    for d in ds:
-        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
-                      d["x"], 0, probe, threads=1)
-    per_row = (time.perf_counter() - t0) / (probe * len(ds))
-    rows = int(min(min(M for (M, K, b) in LAYERS), max(probe, seconds * cores / per_row / 3)))
-    t0 = time.perf_counter()
-    for d in ds:
-        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
-                      d["x"], 0, rows, threads=cores)
-    dt = time.perf_counter() - t0
-    wb = sum(rows * (K * b // 8 + (K // 128) * 2) for (M, K, b) in LAYERS)
+    while True:
+        for d in ds:
+            oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                          d["x"], threads=cores)
+        passes += 1
+        dt = time.perf_counter() - t0
+        if dt >= seconds:
+            break
+    wb = passes * sum(weight_bytes(M, K, b) for (M, K, b) in LAYERS)
     return {"value": round(wb / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"first {rows} of 12288 rows of each layer (b2, b3, b8), batch 1, "
-                      f"{dt:.1f} s wall on {cores} threads"}
+            "sample": f"{passes} full passes over the 3 layers (12288x4096 at b2, b3, b8), "
+                      f"batch 1, {dt:.1f} s wall on {cores} threads"}
 
 
 def run_reference(a):

@@ -2,25 +2,28 @@
 //
 // H_K in Sylvester natural order factors over the bits of the index: with
 // K = 32 * E * W and i = w*(32E) + l*E + e (warp w, lane l, register e),
-// H_K = H_W (x) H_32 (x) H_E.  So a block of 32*W threads transforms one row:
+// H_K = H_W (x) H_32 (x) H_E.  So 32*W threads transform one row:
 //   1. butterflies over e inside each thread's E registers,
 //   2. butterflies over l with warp shuffles (xor 1..16),
 //   3. butterflies over w after one transpose through shared memory, where each
 //      thread gathers the W values of E/W (l, e) columns.
-// No global synchronisation, log2(K) butterfly stages in total, two
-// __syncthreads.  The butterfly (a, b) -> (a + b, a - b) is the definition
-// of the Sylvester matrix applied one index bit at a time.
+// log2(K) butterfly stages in total, two __syncthreads.  The butterfly
+// (a, b) -> (a + b, a - b) is the Sylvester matrix applied one index bit at a
+// time.  W is capped at 2^LOGW_MAX so that the transform fits the CTA that
+// calls it; threads beyond 32*W skip the arithmetic but still reach every
+// barrier.
 #pragma once
 
 #include <stdint.h>
 
 namespace hq {
 
-template <int LOGK>
+template <int LOGK, int LOGW_MAX = 5>
 struct FwhtShape {
   static constexpr int K = 1 << LOGK;
-  static constexpr int LOGE = (LOGK - 5 + 1) / 2;
-  static constexpr int LOGW = (LOGK - 5) / 2;
+  static constexpr int LOGW_NAT = (LOGK - 5) / 2;
+  static constexpr int LOGW = LOGW_NAT < LOGW_MAX ? LOGW_NAT : LOGW_MAX;
+  static constexpr int LOGE = LOGK - 5 - LOGW;
   static constexpr int E = 1 << LOGE;
   static constexpr int W = 1 << LOGW;
   static constexpr int THREADS = 32 * W;
@@ -32,61 +35,66 @@ struct FwhtShape {
 
 __device__ __forceinline__ int fwht_pad(int i) { return i + (i >> 5); }
 
-// On entry thread tid = 32*w + l holds v[e] = u[tid*E + e].  On exit the
-// transformed (unnormalised) row is in buf[fwht_pad(i)], i in [0, K), and the
-// block has synchronised.  buf holds FwhtShape<LOGK>::SMEM_FLOATS floats.
-template <int LOGK>
-__device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK>::E], float* buf) {
-  using S = FwhtShape<LOGK>;
+// On entry thread tid = 32*w + l < THREADS holds v[e] = u[tid*E + e].  On exit
+// the transformed (unnormalised) row is in buf[fwht_pad(i)], i in [0, K), and
+// the block has synchronised.  Every thread of the block must call this.
+template <int LOGK, int LOGW_MAX>
+__device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>::E], float* buf) {
+  using S = FwhtShape<LOGK, LOGW_MAX>;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
+  const bool active = tid < S::THREADS;
+  if (active) {
 #pragma unroll
-  for (int h = 1; h < S::E; h <<= 1) {
+    for (int h = 1; h < S::E; h <<= 1) {
 #pragma unroll
-    for (int e = 0; e < S::E; ++e) {
-      if ((e & h) == 0) {
-        const float a = v[e], b = v[e + h];
-        v[e] = a + b;
-        v[e + h] = a - b;
-      }
-    }
-  }
-#pragma unroll
-  for (int m = 1; m < 32; m <<= 1) {
-    const bool upper = (lane & m) != 0;
-#pragma unroll
-    for (int e = 0; e < S::E; ++e) {
-      const float p = __shfl_xor_sync(0xffffffffu, v[e], m);
-      v[e] = upper ? (p - v[e]) : (v[e] + p);
-    }
-  }
-#pragma unroll
-  for (int e = 0; e < S::E; ++e) buf[fwht_pad(tid * S::E + e)] = v[e];
-  __syncthreads();
-  if constexpr (S::W > 1) {
-    float r[S::C][S::W];
-#pragma unroll
-    for (int j = 0; j < S::C; ++j)
-#pragma unroll
-      for (int w = 0; w < S::W; ++w) r[j][w] = buf[fwht_pad(w * 32 * S::E + tid * S::C + j)];
-#pragma unroll
-    for (int j = 0; j < S::C; ++j) {
-#pragma unroll
-      for (int h = 1; h < S::W; h <<= 1) {
-#pragma unroll
-        for (int w = 0; w < S::W; ++w) {
-          if ((w & h) == 0) {
-            const float a = r[j][w], b = r[j][w + h];
-            r[j][w] = a + b;
-            r[j][w + h] = a - b;
-          }
+      for (int e = 0; e < S::E; ++e) {
+        if ((e & h) == 0) {
+          const float a = v[e], b = v[e + h];
+          v[e] = a + b;
+          v[e + h] = a - b;
         }
       }
     }
 #pragma unroll
-    for (int j = 0; j < S::C; ++j)
+    for (int m = 1; m < 32; m <<= 1) {
+      const bool upper = (lane & m) != 0;
 #pragma unroll
-      for (int w = 0; w < S::W; ++w) buf[fwht_pad(w * 32 * S::E + tid * S::C + j)] = r[j][w];
+      for (int e = 0; e < S::E; ++e) {
+        const float p = __shfl_xor_sync(0xffffffffu, v[e], m);
+        v[e] = upper ? (p - v[e]) : (v[e] + p);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < S::E; ++e) buf[fwht_pad(tid * S::E + e)] = v[e];
+  }
+  __syncthreads();
+  if constexpr (S::W > 1) {
+    if (active) {
+      float r[S::C][S::W];
+#pragma unroll
+      for (int j = 0; j < S::C; ++j)
+#pragma unroll
+        for (int w = 0; w < S::W; ++w) r[j][w] = buf[fwht_pad(w * 32 * S::E + tid * S::C + j)];
+#pragma unroll
+      for (int j = 0; j < S::C; ++j) {
+#pragma unroll
+        for (int h = 1; h < S::W; h <<= 1) {
+#pragma unroll
+          for (int w = 0; w < S::W; ++w) {
+            if ((w & h) == 0) {
+              const float a = r[j][w], b = r[j][w + h];
+              r[j][w] = a + b;
+              r[j][w + h] = a - b;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < S::C; ++j)
+#pragma unroll
+        for (int w = 0; w < S::W; ++w) buf[fwht_pad(w * 32 * S::E + tid * S::C + j)] = r[j][w];
+    }
     __syncthreads();
   }
 }

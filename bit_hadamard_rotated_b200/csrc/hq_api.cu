@@ -42,7 +42,7 @@ static hq_status check_weight(const hq_weight* w) {
   return HQ_OK;
 }
 
-// Largest GEMV column block whose tile fits in one CTA's shared memory.
+// Largest GEMV batch block whose ring plan fits in one CTA.
 static int gemv_col_block(int bits, int K) {
   for (int nb = kMaxColBlock; nb >= 1; nb >>= 1) {
     if (gemv_smem_bytes(bits, K, nb) != 0) return nb;
@@ -50,22 +50,23 @@ static int gemv_col_block(int bits, int K) {
   return 0;
 }
 
+// hq_linear workspace: [status 256 B][GEMV partial tiles][tile counters].
 struct LinearWs {
   uint32_t* status;
-  uint16_t* xs;
-  float* corr;
+  void* part;
+  uint32_t* cnt;
   size_t bytes;
 };
 
-static LinearWs linear_ws(void* base, int K) {
+static LinearWs linear_ws(void* base, int M) {
   LinearWs l{};
-  const size_t xs_bytes = align256(static_cast<size_t>(kMaxColBlock) * K * 2);
-  const size_t corr_bytes = align256(static_cast<size_t>(K / 128) * kMaxColBlock * 4);
+  const size_t part_bytes = align256(static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16);
+  const size_t cnt_bytes = align256(static_cast<size_t>((M + 15) / 16) * 4);
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
-  l.xs = reinterpret_cast<uint16_t*>(b + kStatusBytes);
-  l.corr = reinterpret_cast<float*>(b + kStatusBytes + xs_bytes);
-  l.bytes = kStatusBytes + xs_bytes + corr_bytes;
+  l.part = b + kStatusBytes;
+  l.cnt = reinterpret_cast<uint32_t*>(b + kStatusBytes + part_bytes);
+  l.bytes = kStatusBytes + part_bytes + cnt_bytes;
   return l;
 }
 
@@ -114,14 +115,14 @@ hq_status hq_rotate(const void* x, hq_dtype x_dtype, void* x_rot, hq_dtype out_d
 
 size_t hq_linear_workspace_size(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch < 0) return 0;
-  return linear_ws(nullptr, w->K).bytes;
+  return linear_ws(nullptr, w->M).bytes;
 }
 
 int hq_linear_launches(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch <= 0) return 0;
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return 0;
-  return 2 * ((batch + nb - 1) / nb);
+  return (batch + nb - 1) / nb;
 }
 
 hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, void* workspace,
@@ -132,33 +133,30 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
   if (batch == 0) return HQ_OK;
   if (x == nullptr || y == nullptr) return HQ_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
-  const LinearWs l = linear_ws(workspace, w->K);
+  const LinearWs l = linear_ws(workspace, w->M);
   if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < l.bytes) {
     return HQ_ERR_WORKSPACE;
   }
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return HQ_ERR_UNSUPPORTED;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const __half* xh = reinterpret_cast<const __half*>(x);
   for (int n0 = 0; n0 < batch; n0 += nb) {
-    const int nbk = batch - n0 < nb ? batch - n0 : nb;
-    cudaError_t e = launch_prep_gemv(w->bits, w->K, xh + static_cast<size_t>(n0) * w->K,
-                                     w->signs, l.xs, l.corr, nbk, w->zero, st);
-    if (e != cudaSuccess) return from_cuda(e);
     GemvArgs a;
     a.bits = w->bits;
     a.M = w->M;
     a.K = w->K;
-    a.N = nbk;
+    a.N = batch - n0 < nb ? batch - n0 : nb;
     a.zero = w->zero;
     a.q = w->qweight;
     a.scales = w->scales;
-    a.xs = l.xs;
-    a.corr = l.corr;
+    a.x = x + static_cast<size_t>(n0) * w->K;
+    a.signs = w->signs;
     a.y = y + static_cast<size_t>(n0) * w->M;
     a.ldy = w->M;
     a.status = l.status;
-    e = launch_gemv(a, st);
+    a.part = l.part;
+    a.cnt = l.cnt;
+    const cudaError_t e = launch_gemv(a, st);
     if (e != cudaSuccess) return from_cuda(e);
   }
   return HQ_OK;

@@ -23,23 +23,24 @@ void note_launch();
 cudaError_t launch_rotate(hq_dtype id, hq_dtype od, const void* x, void* out, int n_rows, int K,
                           const int8_t* signs, cudaStream_t st);
 
-cudaError_t launch_prep_gemv(int bits, int K, const __half* x, const int8_t* signs, uint16_t* xs,
-                             float* corr, int N, int zero, cudaStream_t st);
-
 struct GemvArgs {
   int bits, M, K, N, zero;
   const uint32_t* q;
   const uint16_t* scales;
-  const uint16_t* xs;
-  const float* corr;
-  float* y;  // [N][M] block of outputs, row stride ldy
+  const uint16_t* x;    // [N][K] fp16 activations (not rotated)
+  const int8_t* signs;  // [K] or NULL
+  float* y;             // [N][M] block of outputs, row stride ldy
   int ldy;
   uint32_t* status;
+  void* part;     // gemv_max_warps() * 1 KiB of partial tiles
+  uint32_t* cnt;  // ceil(M/16) counters, zero between launches
 };
 
-// Shared memory the GEMV needs for a column block of nb <= 8 rows (0 if the
-// tile does not fit in one CTA).
+// Shared memory the GEMV needs for a batch block of nb <= 8 rows (0 if no
+// ring configuration fits in one CTA).
 size_t gemv_smem_bytes(int bits, int K, int nb);
+// Upper bound on the GEMV's warps (8 per SM of the current device).
+int gemv_max_warps();
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 
 cudaError_t launch_unpack(const uint32_t* packed, int bits, size_t n, uint8_t* out,

@@ -5,23 +5,19 @@
 // triplet, 4-bit: 4 words, 8-bit: 8 words).  decode16<BITS> turns the bundle
 // into 16 half2 registers P[p], each holding two codes (lo, hi) as the fp16
 // values 1024 + (code << a): the code's bits are masked straight into the
-// mantissa of 1024.0 (exponent 0x19), with no shift when the field already
+// mantissa of 1024.0 (whose ulp is 1), with no shift when the field already
 // sits in a mantissa slot, so one LOP3 (or PRMT for bytes) yields two codes.
-//
-// kPairs<BITS>[p] names, for each half, the code index inside the bundle and
-// its shift a.  The activation side compensates exactly: the tensor-core B
-// operand holds x'_k * 2^-a_k, so the MMA computes
-//     sum_k (1024 + 2^a_k q_k) x'_k 2^-a_k = 1024 sum_k B_k + sum_k q_k x'_k
-// and the per-(group, column) constant  sum_k (1024 + zero 2^a_k) B_k  is
-// subtracted once (it is the accumulator's initial value, negated).  This is
-// how the dequantisation w = scale (q - zero) is applied inside the matmul
-// without per-weight subtract or multiply instructions; the group scale
+// One fused multiply-add per pair, (1024 + 2^a q) * 2^-a - (1024 * 2^-a +
+// zero), then gives q - zero exactly (every intermediate is an integer or a
+// power-of-two multiple below 2048), so the dequantisation w = scale (q -
+// zero) enters the tensor core as an exact small integer and the group scale
 // multiplies the fp32 group sum.
 //
-// Step s (0..7) of a 128-code group feeds the m16n8k16 MMA with P[2s] as the
-// A-fragment columns (2t, 2t+1) and P[2s+1] as columns (2t+8, 2t+9), t = lane
-// & 3; the B fragment of lane (n, t) at that step holds the matching four
-// activations, in that order.
+// Pairs<BITS>::get(p) names, for each half of pair p, the code index inside
+// the bundle and its shift a.  Step s (0..7) of a 128-code group feeds the
+// m16n8k16 MMA with P[2s] as A-fragment columns (2t, 2t+1) and P[2s+1] as
+// columns (2t+8, 2t+9), t = lane & 3; the B fragment of lane (n, t) at that
+// step holds the four activations with those code indices, in that order.
 #pragma once
 
 #include <stdint.h>
@@ -153,6 +149,47 @@ __device__ __forceinline__ void decode16<3>(const uint32_t (&w)[3], uint32_t (&P
   P[13] = and_or(v6, m3(7, 6), kMagic);
   P[14] = and_or(v7, m3(1, 0), kMagic);
   P[15] = and_or(v7, m3(4, 3), kMagic);
+}
+
+// fp16 bit pattern of 2^-a (a <= 14).
+__host__ __device__ constexpr uint32_t half_pow2_neg(int a) {
+  return static_cast<uint32_t>(15 - a) << 10;
+}
+
+// half2 multiplier (2^-a_lo, 2^-a_hi) of pair p.
+template <int BITS>
+__host__ __device__ constexpr uint32_t pair_mult(int p) {
+  return half_pow2_neg(Pairs<BITS>::get(p).a_lo) | (half_pow2_neg(Pairs<BITS>::get(p).a_hi) << 16);
+}
+
+// fp16 bit pattern of -v for an integer 1 <= v < 2048 (exact).
+__host__ __device__ constexpr uint32_t half_neg_int(int v) {
+  int e = 0;
+  while ((v >> (e + 1)) != 0) ++e;
+  return 0x8000u | (static_cast<uint32_t>(e + 15) << 10) |
+         ((static_cast<uint32_t>(v) << (10 - e)) & 0x3FFu);
+}
+
+// half2 addend -(1024 2^-a + zero) of pair p (host side, per launch).
+template <int BITS>
+inline uint32_t pair_addend(int p, int zero) {
+  const PairDesc d = Pairs<BITS>::get(p);
+  return half_neg_int((1024 >> d.a_lo) + zero) | (half_neg_int((1024 >> d.a_hi) + zero) << 16);
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Decode a bundle straight to exact (q - zero) fp16 pairs.
+template <int BITS>
+__device__ __forceinline__ void decode16_exact(const uint32_t (&w)[BITS], const uint32_t* add,
+                                               uint32_t (&P)[16]) {
+  decode16<BITS>(w, P);
+#pragma unroll
+  for (int p = 0; p < 16; ++p) P[p] = hfma2(P[p], pair_mult<BITS>(p), add[p]);
 }
 
 // Load a lane's BITS-word bundle from shared memory (16-byte aligned for

@@ -37,8 +37,11 @@
  *     ran out, an expert id or bit width out of range in device data) are
  *     OR-ed into the status word at the start of the caller's workspace and
  *     read back by hq_check_status; device code never traps.
- *   - A workspace must be at least the queried size, 256-byte aligned, and its
- *     first 256 bytes must be zero before its first use (the status word).
+ *   - A workspace must be at least the queried size, 256-byte aligned, and
+ *     zero-filled before its first use.  Calls leave it ready for the next
+ *     call (counters back at zero) unless a device error was recorded; after
+ *     HQ_ERR_TIMEOUT, zero it again.  One workspace serves one stream at a
+ *     time: calls that overlap on the GPU must not share it.
  *   - Outputs are overwritten, never accumulated into.  Inputs and outputs
  *     must not alias.
  *   - Alignment: packed weights, scales, activations and outputs must be

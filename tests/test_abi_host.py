@@ -77,9 +77,9 @@ def test_linear_rejects_bad_call_args(L):
 def test_workspace_size_queries(L):
     assert L.hq_linear_workspace_size(ctypes.byref(W(bits=7)), 1) == 0
     assert L.hq_linear_workspace_size(ctypes.byref(W()), -1) == 0
-    a = L.hq_linear_workspace_size(ctypes.byref(W(K=4096)), 1)
-    b = L.hq_linear_workspace_size(ctypes.byref(W(K=8192)), 1)
-    assert 0 < a < b and a % 256 == 0
+    a = L.hq_linear_workspace_size(ctypes.byref(W(M=64)), 1)
+    b = L.hq_linear_workspace_size(ctypes.byref(W(M=65536)), 1)
+    assert 0 < a < b and a % 256 == 0          # one tile counter per 16 output rows
 
 
 def test_rotate_rejects_bad_args(L):
