@@ -58,11 +58,12 @@ __device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>:
     }
 #pragma unroll
     for (int m = 1; m < 32; m <<= 1) {
-      const bool upper = (lane & m) != 0;
+      // lower lane: a + b; upper lane: a - b = partner - own
+      const float sgn = (lane & m) ? -1.f : 1.f;
 #pragma unroll
       for (int e = 0; e < S::E; ++e) {
         const float p = __shfl_xor_sync(0xffffffffu, v[e], m);
-        v[e] = upper ? (p - v[e]) : (v[e] + p);
+        v[e] = fmaf(sgn, v[e], p);
       }
     }
 #pragma unroll

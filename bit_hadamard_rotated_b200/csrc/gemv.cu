@@ -8,23 +8,28 @@
 // gridbook card, "Reading it honestly"), so the kernel is shaped to stream the
 // packed codes at HBM rate with the rotation and all dequantisation on chip:
 //
-//   * Persistent grid, one CTA of 8 warps per SM.  The work is the list of
+//   * Persistent grid, one CTA of 16 warps per SM.  The work is the list of
 //     (16-row tile, 128-code group) units; every warp owns one contiguous
-//     range of ~U/(8 * #SMs) units, so the load is balanced to one group.
+//     range of ~U/(16 * #SMs) units, so the load is balanced to one group.
 //   * Each warp streams its range through a private ring of NS shared-memory
-//     slots.  A slot holds up to CH groups of 16 rows (one bulk/TMA copy per
-//     row, rows at a bank-conflict-free padded stride) and the matching fp16
-//     scales (one more bulk copy per row), all completing on one mbarrier.
+//     slots.  A slot holds up to CH groups of 16 rows (rows at a bank-conflict-
+//     free padded stride) and the matching fp16 scales, moved by 16-byte
+//     cp.async copies spread across the lanes, completing on one mbarrier
+//     (many small bulk copies, one per row, were bound by the copy engine's
+//     per-request cost).
 //     The first NS copies are issued before griddepcontrol.wait: weights do not
 //     depend on earlier kernels, so they overlap the previous kernel's tail.
 //   * Meanwhile the CTA rotates its N activation rows in fp32 (fwht.cuh) and
-//     stores x' as fp16 in the order of the MMA B fragments (hq_layout.cuh).
-//   * Per group: each lane decodes 2 x 32 codes into exact fp16 (q - zero)
-//     pairs (one LOP3/PRMT + one HFMA2 per pair), 8 mma.sync m16n8k16 with
-//     fp32 accumulation in two independent chains, then acc += scale * sum.
+//     stores x' as fp16 in the order of the MMA B fragments, each scaled by the
+//     2^-a of its code field (hq_layout.cuh), plus zero * sum_k x'_k per group.
+//   * Per group: each lane masks 2 x 32 codes into exact subnormal fp16 pairs
+//     (one LOP3/PRMT per pair), runs 8 mma.sync m16n8k16 with fp32
+//     accumulation in two chains (one starting at -zero * sum x' * 2^-24), then
+//     acc += (scale * 2^24) * sum.
 //   * A tile split between warps is finished by whichever contributor arrives
 //     last at the tile's counter: it adds all contributors' partial sums in
-//     warp order (deterministic, no waiting) and resets the counter.
+//     warp order (deterministic, no waiting) and resets the counter.  A warp
+//     defers these exchanges to the end of its range.
 #include <algorithm>
 
 #include "fwht.cuh"
@@ -38,6 +43,11 @@ namespace hq {
 
 constexpr int kWarps = 8;
 constexpr int kRows = 16;
+// halves per (group, column, k-quad) block of B fragments: 8 steps x 4, padded
+// to 80 bytes so the 16-byte loads of 8 lanes hit distinct banks
+constexpr int kXq = 40;
+// 2^24: undoes, at the stores, the 2^-24 unit of the subnormal fp16 codes
+constexpr float kUnit = 16777216.f;
 
 struct GemvParams {
   const uint32_t* q;
@@ -51,9 +61,9 @@ struct GemvParams {
   int M, N, ldy;
   uint32_t U;  // units = n_tiles * G
   uint32_t GW;  // active warps
-  int CH, NS, stride, slot_bytes, buf_off, ring_off, bar_off;
+  int zero;
+  int CH, NS, stride, slot_bytes, zc_off, buf_off, ring_off, bar_off;
   float inv_sqrt_k;
-  uint32_t add[16];
 };
 
 __device__ __forceinline__ uint32_t unit_begin(uint32_t gw, uint32_t U, uint32_t GW) {
@@ -65,7 +75,7 @@ __device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t U, uint32_t 
 }
 
 template <int BITS, int LOGK>
-__global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_constant__ GemvParams p) {
   using FS = FwhtShape<LOGK, 3>;
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
@@ -80,18 +90,22 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   const int row_words = K * BITS / 32;
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
+  float* zc = reinterpret_cast<float*>(smem + p.zc_off);
   float* buf = reinterpret_cast<float*>(smem + p.buf_off);
   uint8_t* ring = smem + p.ring_off + warp * p.NS * p.slot_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off) + warp * p.NS;
 
   if (lane == 0) {
-    for (int i = 0; i < p.NS; ++i) mbar_init(&bars[i], 1);
+    for (int i = 0; i < p.NS; ++i) mbar_init(&bars[i], 32);
     fence_mbar_init();
   }
   __syncthreads();
   pdl_launch_dependents();
 
-  // ---- producer side of the warp's ring: one chunk = up to CH groups of a tile
+  // ---- producer side of the warp's ring: one chunk = up to CH groups of a
+  // tile, codes and scales, as 16-byte cp.async copies spread over the lanes
+  // (consecutive lanes read consecutive bytes of a row); every lane then
+  // arrives on the slot's barrier when its copies have landed.
   uint32_t ui = u0;
   int issued = 0;
   auto issue = [&](int slot) {
@@ -101,42 +115,36 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     const int rv = min(kRows, p.M - m0);
     uint8_t* base = ring + slot * p.slot_bytes;
     uint8_t* sdst = base + kRows * p.stride;
-    const uint32_t cbytes = len * GB;
-    uint32_t total = rv * cbytes;
-    uint32_t sg0 = 0, sbytes = 0;
-    bool tile_bulk = false;
-    if constexpr (G >= 8) {
-      sg0 = g0 & ~7u;
-      sbytes = (((g0 + len + 7u) & ~7u) - sg0) * 2u;
-      total += rv * sbytes;
-    } else {
-      tile_bulk = ((rv * G * 2) % 16) == 0;
-      if (tile_bulk) total += rv * G * 2;
-    }
-    if (lane == 0) mbar_arrive_expect_tx(&bars[slot], total);
-    __syncwarp();
-    if (lane < rv) {
-      const uint8_t* src = reinterpret_cast<const uint8_t*>(
-                               p.q + static_cast<size_t>(m0 + lane) * row_words) +
-                           static_cast<size_t>(g0) * GB;
-      bulk_g2s(base + lane * p.stride, src, cbytes, &bars[slot]);
-    }
-    if constexpr (G >= 8) {
-      const int r = lane - 16;
-      if (r >= 0 && r < rv) {
-        bulk_g2s(sdst + r * 32, p.scales + static_cast<size_t>(m0 + r) * G + sg0, sbytes,
-                 &bars[slot]);
-      }
-    } else {
-      if (tile_bulk) {
-        if (lane == 16) {
-          bulk_g2s(sdst, p.scales + static_cast<size_t>(m0) * G, rv * G * 2, &bars[slot]);
-        }
-      } else {
-        uint16_t* sd = reinterpret_cast<uint16_t*>(sdst);
-        for (int i = lane; i < rv * G; i += 32) sd[i] = p.scales[static_cast<size_t>(m0) * G + i];
+    const int pr = static_cast<int>(len) * BITS;  // 16-byte pieces per row
+    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<size_t>(m0) * row_words) +
+                          static_cast<size_t>(g0) * GB;
+    // lanes in groups of 2^lg (>= pieces per row, <= 32); one row per group per pass
+    const int lg = pr <= 8 ? 3 : pr <= 16 ? 4 : 5;
+    const int rpp = 32 >> lg;  // rows per pass
+    const int c = lane & ((1 << lg) - 1);
+    for (int r = lane >> lg; r < rv; r += rpp) {
+      for (int cc = c; cc < pr; cc += (1 << lg)) {
+        cp_async16(base + r * p.stride + cc * 16,
+                   qsrc + static_cast<size_t>(r) * row_words * 4 + cc * 16, 16);
       }
     }
+    if constexpr (G >= 8) {
+      const uint32_t sg0 = g0 & ~7u;
+      const int nblk = static_cast<int>((((g0 + len + 7u) & ~7u) - sg0) / 8u);
+      const int r = lane & 15, blk = lane >> 4;
+      if (r < rv && blk < nblk) {
+        cp_async16(sdst + r * 32 + blk * 16, p.scales + static_cast<size_t>(m0 + r) * G + sg0 + 8 * blk,
+                   16);
+      }
+    } else {
+      const int bytes = rv * G * 2;
+      const int lo = lane * 16;
+      if (lane < 2 * G && lo < bytes) {
+        cp_async16(sdst + lo, reinterpret_cast<const uint8_t*>(p.scales + static_cast<size_t>(m0) * G) + lo,
+                   static_cast<uint32_t>(min(16, bytes - lo)));
+      }
+    }
+    cp_async_mbar_arrive(&bars[slot]);
     ui += len;
     ++issued;
   };
@@ -144,75 +152,154 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
   // ---- rotate the activations (depends on the previous kernel)
   pdl_wait();
-  for (int n = 0; n < p.N; ++n) {
-    float v[FS::E];
-    if (tid < FS::THREADS) {
-      load_chunk<__half, FS::E>(p.x + static_cast<size_t>(n) * K + tid * FS::E, v);
-      apply_signs<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr, v);
-    }
-    fwht_block<LOGK, 3>(v, buf);
-    for (int qd = tid; qd < K / 4; qd += kWarps * 32) {
-      const int S = qd >> 2, tt = qd & 3;
-      uint16_t hv[4];
+  {
+    // lane (s, t) writes the B-fragment quad of step s for k-quad t
+    const int s = lane >> 2;
+    int kc[4], ka[4];
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const PairDesc pd = Pairs<BITS>::get(2 * (S & 7) + (r >> 1));
-        const int k = kGroup * (S >> 3) + 32 * tt + ((r & 1) ? pd.c_hi : pd.c_lo);
-        hv[r] = __half_as_ushort(__float2half_rn(buf[fwht_pad(k)] * p.inv_sqrt_k));
-      }
-      uint2 pk;
-      pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
-      pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
-      *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(S) * p.N + n) * 4 + tt) * 4) = pk;
+    for (int r = 0; r < 4; ++r) {
+      const PairDesc pd = Pairs<BITS>::get(2 * s + (r >> 1));
+      kc[r] = 32 * t + ((r & 1) ? pd.c_hi : pd.c_lo);
+      ka[r] = (r & 1) ? pd.a_hi : pd.a_lo;
     }
+    // zero-point terms of absent batch columns and the B block of lanes
+    // without a column stay zero
+    for (int i = tid; i < G * 8; i += kWarps * 32) zc[i] = 0.f;
+    if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;
     __syncthreads();
+    for (int n = 0; n < p.N; ++n) {
+      float v[FS::E];
+      if (tid < FS::THREADS) {
+        load_chunk<__half, FS::E>(p.x + static_cast<size_t>(n) * K + tid * FS::E, v);
+        apply_signs<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr, v);
+      }
+      fwht_block<LOGK, 3>(v, buf);
+      for (int gg = warp; gg < G; gg += kWarps) {
+        uint16_t hv[4];
+        float part = 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + kc[r])] *
+                                                        p.inv_sqrt_k));
+          const __half b = __float2half_rn(xv * __int_as_float((127 - ka[r]) << 23));
+          hv[r] = __half_as_ushort(b);
+          part += __half2float(b) * __int_as_float((127 + ka[r]) << 23);
+        }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+        uint2 pk;
+        pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
+        pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
+        *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * p.N + n) * 4 + t) * kXq + s * 4) =
+            pk;
+        if (lane == 0) zc[gg * 8 + n] = -static_cast<float>(p.zero) * part * 5.9604644775390625e-8f;
+      }
+      __syncthreads();
+    }
   }
 
   // ---- consumer: decode + MMA over the warp's units
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float head[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums of a first tile shared with other warps
+  int head_tile = -1;
   int tile_start = -1;
   int consumed = 0;
   bool ok = true;
-  const bool has_b = g < p.N;
-  const int xs_step = p.N * 16;
+  const int N = p.N, M = p.M, ldy = p.ldy, CH = p.CH, NS = p.NS, stride = p.stride;
+  const int slot_bytes = p.slot_bytes;
+  const bool n0 = 2 * t < N, n1 = 2 * t + 1 < N;
+  // lane's B-fragment stream: its column's blocks, or a zero block (stride 0)
+  const bool has_b = g < N;
+  const uint4* xs_lane = has_b ? reinterpret_cast<const uint4*>(xs + (static_cast<size_t>(g) * 4 + t) * kXq)
+                               : reinterpret_cast<const uint4*>(zc + G * 8);
+  const int xs_gstride = has_b ? N * 4 * kXq / 8 : 0;  // uint4 per group
+  const uint32_t first_tile = u0 / G;
   uint32_t uc = u0;
+
+  // Partial sums of tiles shared with other warps: each contributor publishes
+  // its partial, one fence orders them before the arrival counters, and the
+  // last arrival at a tile adds all contributors' partials in warp order and
+  // stores y.  A warp has at most two shared tiles (the first and the last
+  // of its range); both are exchanged together at the end of the range.
+  auto publish = [&](uint32_t tile, const float (&v)[4]) {
+    const int which = (tile == first_tile) ? 0 : 1;
+    p.part[(static_cast<size_t>(gw) * 2 + which) * 32 + lane] =
+        make_float4(v[0] * kUnit, v[1] * kUnit, v[2] * kUnit, v[3] * kUnit);
+  };
+  auto complete = [&](uint32_t tile) {
+    uint32_t old = 0;
+    if (lane == 0) old = atomicAdd(&p.cnt[tile], 1u);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    const uint32_t gwf = unit_owner(tile * G, p.U, p.GW);
+    const uint32_t gwl = unit_owner(tile * G + G - 1, p.U, p.GW);
+    if (old != gwl - gwf) return;
+    __threadfence();
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (uint32_t c = gwf; c <= gwl; ++c) {
+      const int wc = (tile == unit_begin(c, p.U, p.GW) / G) ? 0 : 1;
+      const float4 q4 = __ldcg(&p.part[(static_cast<size_t>(c) * 2 + wc) * 32 + lane]);
+      o.x += q4.x;
+      o.y += q4.y;
+      o.z += q4.z;
+      o.w += q4.w;
+    }
+    if (lane == 0) p.cnt[tile] = 0u;
+    const int m0 = tile * kRows;
+    const int rv = min(kRows, M - m0);
+    if (g < rv) {
+      if (n0) p.y[static_cast<size_t>(2 * t) * ldy + m0 + g] = o.x;
+      if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g] = o.y;
+    }
+    if (g + 8 < rv) {
+      if (n0) p.y[static_cast<size_t>(2 * t) * ldy + m0 + g + 8] = o.z;
+      if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g + 8] = o.w;
+    }
+  };
+  int tail_tile = -1;
+
   while (uc < u1) {
     const uint32_t tile = uc / G, g0 = uc % G;
-    const uint32_t len = min(static_cast<uint32_t>(p.CH), min(G - g0, u1 - uc));
-    const int slot = consumed % p.NS;
-    if (!mbar_wait(&bars[slot], (consumed / p.NS) & 1)) {
+    const uint32_t len = min(static_cast<uint32_t>(CH), min(G - g0, u1 - uc));
+    const int slot = consumed % NS;
+    if (!mbar_wait(&bars[slot], (consumed / NS) & 1)) {
       ok = false;
       break;
     }
     __syncwarp();
     if (tile_start < 0) tile_start = static_cast<int>(g0);
-    const uint8_t* base = ring + slot * p.slot_bytes;
-    const __half* sc = reinterpret_cast<const __half*>(base + kRows * p.stride);
-    const uint8_t* rowa = base + g * p.stride + t * 4 * BITS;
-    const uint8_t* rowb = base + (g + 8) * p.stride + t * 4 * BITS;
-    const uint32_t sg0 = (G >= 8) ? (g0 & ~7u) : 0u;
+    const uint8_t* base = ring + slot * slot_bytes;
+    const uint8_t* ra = base + g * stride + t * 4 * BITS;
+    const uint8_t* rb = ra + 8 * stride;
     const int sstride = (G >= 8) ? 16 : G;
+    const __half* sca = reinterpret_cast<const __half*>(base + kRows * stride) + g * sstride +
+                        (G >= 8 ? (g0 & 7u) : g0);
+    const __half* scb = sca + 8 * sstride;
+    const float2* zp = reinterpret_cast<const float2*>(zc + g0 * 8 + 2 * t);
+    const uint4* xb = xs_lane + static_cast<size_t>(g0) * xs_gstride;
 #pragma unroll 1
     for (uint32_t j = 0; j < len; ++j) {
-      const uint32_t gi = g0 + j;
       uint32_t wa[BITS], wb[BITS];
-      load_bundle<BITS>(rowa + j * GB, wa);
-      load_bundle<BITS>(rowb + j * GB, wb);
-      const float sa = __half2float(sc[g * sstride + (gi - sg0)]);
-      const float sb = __half2float(sc[(g + 8) * sstride + (gi - sg0)]);
+      load_bundle<BITS>(ra, wa);
+      load_bundle<BITS>(rb, wb);
+      ra += GB;
+      rb += GB;
+      // group scales (the 2^24 subnormal unit is applied once, at the store)
+      const float sa = __half2float(*sca++);
+      const float sb = __half2float(*scb++);
+      const float2 z = *zp;
+      zp += 4;
+      uint4 bq[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bq[i] = xb[i];
+      xb += xs_gstride;
       uint32_t Pa[16], Pb[16];
-      decode16_exact<BITS>(wa, p.add, Pa);
-      decode16_exact<BITS>(wb, p.add, Pb);
-      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-      const uint16_t* xb = xs + (static_cast<size_t>(8 * gi) * p.N + g) * 16 + t * 4;
+      decode16<BITS>(wa, Pa);
+      decode16<BITS>(wb, Pb);
+      float c0[4] = {z.x, z.y, z.x, z.y}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        uint32_t b0 = 0u, b1 = 0u;
-        if (has_b) {
-          const uint2 bb = *reinterpret_cast<const uint2*>(xb + s * xs_step);
-          b0 = bb.x;
-          b1 = bb.y;
-        }
+        const uint32_t b0 = (s & 1) ? bq[s >> 1].z : bq[s >> 1].x;
+        const uint32_t b1 = (s & 1) ? bq[s >> 1].w : bq[s >> 1].y;
         const uint32_t a[4] = {Pa[2 * s], Pb[2 * s], Pa[2 * s + 1], Pb[2 * s + 1]};
         if (s & 1) {
           mma_16816(c1, a, b0, b1, c1);
@@ -226,57 +313,45 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       acc[3] = fmaf(sb, c0[3] + c1[3], acc[3]);
     }
     __syncwarp();
-    fence_proxy_async_smem();
     if (ui < u1) issue(slot);
     uc += len;
     ++consumed;
 
     if (g0 + len == G || uc >= u1) {
-      // ---- finish this warp's part of the tile
-      const int m0 = tile * kRows;
-      const int rv = min(kRows, p.M - m0);
+      // ---- this warp's part of the tile is done
       const bool full = tile_start == 0 && g0 + len == G;
-      float4 out = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      bool store = full;
-      if (!full) {
-        const int which = (tile == u0 / G) ? 0 : 1;
-        p.part[(static_cast<size_t>(gw) * 2 + which) * 32 + lane] = out;
-        __threadfence();
-        __syncwarp();
-        uint32_t old = 0;
-        if (lane == 0) old = atomicAdd(&p.cnt[tile], 1u);
-        old = __shfl_sync(0xffffffffu, old, 0);
-        const uint32_t gwf = unit_owner(tile * G, p.U, p.GW);
-        const uint32_t gwl = unit_owner(tile * G + G - 1, p.U, p.GW);
-        if (old == gwl - gwf) {
-          __threadfence();
-          out = make_float4(0.f, 0.f, 0.f, 0.f);
-          for (uint32_t c = gwf; c <= gwl; ++c) {
-            const int wc = (tile == unit_begin(c, p.U, p.GW) / G) ? 0 : 1;
-            const float4 v = __ldcg(&p.part[(static_cast<size_t>(c) * 2 + wc) * 32 + lane]);
-            out.x += v.x;
-            out.y += v.y;
-            out.z += v.z;
-            out.w += v.w;
-          }
-          if (lane == 0) p.cnt[tile] = 0u;
-          store = true;
-        }
-      }
-      if (store) {
-        const int c0 = 2 * t, c1 = 2 * t + 1;
+      if (full) {
+        const int m0 = tile * kRows;
+        const int rv = min(kRows, M - m0);
         if (g < rv) {
-          if (c0 < p.N) p.y[static_cast<size_t>(c0) * p.ldy + m0 + g] = out.x;
-          if (c1 < p.N) p.y[static_cast<size_t>(c1) * p.ldy + m0 + g] = out.y;
+          if (n0) p.y[static_cast<size_t>(2 * t) * ldy + m0 + g] = acc[0] * kUnit;
+          if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g] = acc[1] * kUnit;
         }
         if (g + 8 < rv) {
-          if (c0 < p.N) p.y[static_cast<size_t>(c0) * p.ldy + m0 + g + 8] = out.z;
-          if (c1 < p.N) p.y[static_cast<size_t>(c1) * p.ldy + m0 + g + 8] = out.w;
+          if (n0) p.y[static_cast<size_t>(2 * t) * ldy + m0 + g + 8] = acc[2] * kUnit;
+          if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g + 8] = acc[3] * kUnit;
         }
+      } else if (tile == first_tile && uc < u1) {
+        head[0] = acc[0];  // shared first tile: exchange at the end of the range
+        head[1] = acc[1];
+        head[2] = acc[2];
+        head[3] = acc[3];
+        head_tile = static_cast<int>(tile);
+      } else {
+        publish(tile, acc);  // shared last tile (the range ends here)
+        tail_tile = static_cast<int>(tile);
       }
       acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
       tile_start = -1;
     }
+  }
+  if (ok && (head_tile >= 0 || tail_tile >= 0)) {
+    if (head_tile >= 0) publish(static_cast<uint32_t>(head_tile), head);
+    __syncwarp();
+    if (lane == 0) __threadfence();
+    __syncwarp();
+    if (head_tile >= 0) complete(static_cast<uint32_t>(head_tile));
+    if (tail_tile >= 0) complete(static_cast<uint32_t>(tail_tile));
   }
   if (!ok) {
     if (lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
@@ -287,17 +362,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host planning
 struct GemvPlan {
-  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, buf_off = 0, ring_off = 0, bar_off = 0;
+  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, buf_off = 0, ring_off = 0, bar_off = 0;
   size_t smem = 0;
 };
 
 constexpr size_t kMaxSmem = 227 * 1024;
+// Budget that lets two CTAs (of consecutive launches) share an SM, so that a
+// launch's weight stream overlaps its predecessor's compute and tail.
+constexpr size_t kPairSmem = 110 * 1024;
 
-static GemvPlan gemv_plan(int bits, int K, int nb) {
+static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
   GemvPlan best;
   const int G = K / kGroup;
-  const size_t xs = static_cast<size_t>(nb) * K * 2;
-  const size_t buf_off = (xs + 127) & ~static_cast<size_t>(127);
+  const size_t xs = static_cast<size_t>(nb) * G * 4 * kXq * 2;
+  const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
+  const size_t buf_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
   const size_t buf = static_cast<size_t>(K + K / 32) * 4;
   const size_t ring_off = (buf_off + buf + 127) & ~static_cast<size_t>(127);
   for (int CH : {8, 4, 2, 1}) {
@@ -310,12 +389,13 @@ static GemvPlan gemv_plan(int bits, int K, int nb) {
     for (int NS : {4, 3, 2}) {
       const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * NS * slot;
       const size_t smem = bar_off + static_cast<size_t>(kWarps) * NS * 8;
-      if (smem > kMaxSmem) continue;
+      if (smem > budget) continue;
       if (static_cast<long>(ch) * NS > static_cast<long>(best.CH) * best.NS) {
         best.CH = ch;
         best.NS = NS;
         best.stride = stride;
         best.slot_bytes = slot;
+        best.zc_off = static_cast<int>(zc_off);
         best.buf_off = static_cast<int>(buf_off);
         best.ring_off = static_cast<int>(ring_off);
         best.bar_off = static_cast<int>(bar_off);
@@ -325,6 +405,12 @@ static GemvPlan gemv_plan(int bits, int K, int nb) {
     }
   }
   return best;
+}
+
+static GemvPlan gemv_plan(int bits, int K, int nb) {
+  GemvPlan pl = gemv_plan_budget(bits, K, nb, kPairSmem);
+  if (pl.smem == 0) pl = gemv_plan_budget(bits, K, nb, kMaxSmem);
+  return pl;
 }
 
 size_t gemv_smem_bytes(int bits, int K, int nb) { return gemv_plan(bits, K, nb).smem; }
@@ -342,11 +428,6 @@ int gemv_max_warps() {
     }
   }
   return sms * kWarps;
-}
-
-template <int BITS>
-static void fill_addends(GemvParams& p, int zero) {
-  for (int i = 0; i < 16; ++i) p.add[i] = pair_addend<BITS>(i, zero);
 }
 
 template <int BITS>
@@ -392,15 +473,17 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.NS = pl.NS;
   p.stride = pl.stride;
   p.slot_bytes = pl.slot_bytes;
+  p.zc_off = pl.zc_off;
   p.buf_off = pl.buf_off;
+  p.zero = a.zero;
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;
   p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   switch (a.bits) {
-    case 2: fill_addends<2>(p, a.zero); return gemv_launch_b<2>(a.K, p, pl.smem, grid, st);
-    case 3: fill_addends<3>(p, a.zero); return gemv_launch_b<3>(a.K, p, pl.smem, grid, st);
-    case 4: fill_addends<4>(p, a.zero); return gemv_launch_b<4>(a.K, p, pl.smem, grid, st);
-    case 8: fill_addends<8>(p, a.zero); return gemv_launch_b<8>(a.K, p, pl.smem, grid, st);
+    case 2: return gemv_launch_b<2>(a.K, p, pl.smem, grid, st);
+    case 3: return gemv_launch_b<3>(a.K, p, pl.smem, grid, st);
+    case 4: return gemv_launch_b<4>(a.K, p, pl.smem, grid, st);
+    case 8: return gemv_launch_b<8>(a.K, p, pl.smem, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }

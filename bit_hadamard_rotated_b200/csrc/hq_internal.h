@@ -5,7 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/hq.h"
+#include "hq.h"
 
 namespace hq {
 

@@ -3,15 +3,16 @@
 // A lane of the GEMV owns a "bundle" of 32 consecutive codes of one weight row
 // inside a 128-code group: BITS words (2-bit: 2 words, 3-bit: one 96-bit
 // triplet, 4-bit: 4 words, 8-bit: 8 words).  decode16<BITS> turns the bundle
-// into 16 half2 registers P[p], each holding two codes (lo, hi) as the fp16
-// values 1024 + (code << a): the code's bits are masked straight into the
-// mantissa of 1024.0 (whose ulp is 1), with no shift when the field already
-// sits in a mantissa slot, so one LOP3 (or PRMT for bytes) yields two codes.
-// One fused multiply-add per pair, (1024 + 2^a q) * 2^-a - (1024 * 2^-a +
-// zero), then gives q - zero exactly (every intermediate is an integer or a
-// power-of-two multiple below 2048), so the dequantisation w = scale (q -
-// zero) enters the tensor core as an exact small integer and the group scale
-// multiplies the fp32 group sum.
+// into 16 half2 registers P[p], each holding two codes (lo, hi).  A code's
+// bits are masked straight into the mantissa field of an fp16 whose exponent
+// field is zero, i.e. the subnormal value code * 2^(a - 24), where a is the
+// field's bit offset inside its 16-bit half: one LOP3 (or PRMT for bytes)
+// yields two codes, with no shift when the field already lies in the low 10
+// bits of its half, and the value is exact.  The activation operand carries
+// the compensating 2^-a (so every product is q x' 2^-24 exactly), the group
+// scale carries 2^24, and the zero point enters as zero * sum_k x'_k per group,
+// folded into the accumulator's initial value: w = scale (q - zero) is applied
+// inside the matmul without a per-weight instruction.
 //
 // Pairs<BITS>::get(p) names, for each half of pair p, the code index inside
 // the bundle and its shift a.  Step s (0..7) of a 128-code group feeds the
@@ -80,7 +81,11 @@ struct Pairs<3> {
   }
 };
 
-constexpr uint32_t kMagic = 0x64006400u;  // half2(1024, 1024)
+constexpr uint32_t kMagic = 0u;  // exponent field 0: the masked code is a subnormal
+
+__device__ __forceinline__ uint32_t mask_field(uint32_t x, uint32_t m, uint32_t /*exponent*/) {
+  return x & m;
+}
 
 template <int BITS>
 __device__ __forceinline__ void decode16(const uint32_t (&w)[BITS], uint32_t (&P)[16]);
@@ -92,9 +97,9 @@ __device__ __forceinline__ void decode16<2>(const uint32_t (&w)[2], uint32_t (&P
     const uint32_t x = w[u];
     const uint32_t x2 = x >> 10;
 #pragma unroll
-    for (int i = 0; i < 5; ++i) P[8 * u + i] = and_or(x, 0x00030003u << (2 * i), kMagic);
+    for (int i = 0; i < 5; ++i) P[8 * u + i] = mask_field(x, 0x00030003u << (2 * i), kMagic);
 #pragma unroll
-    for (int i = 0; i < 3; ++i) P[8 * u + 5 + i] = and_or(x2, 0x00030003u << (2 * i), kMagic);
+    for (int i = 0; i < 3; ++i) P[8 * u + 5 + i] = mask_field(x2, 0x00030003u << (2 * i), kMagic);
   }
 }
 
@@ -104,10 +109,10 @@ __device__ __forceinline__ void decode16<4>(const uint32_t (&w)[4], uint32_t (&P
   for (int u = 0; u < 4; ++u) {
     const uint32_t x = w[u];
     const uint32_t x2 = x >> 8;
-    P[4 * u + 0] = and_or(x, 0x000F000Fu, kMagic);
-    P[4 * u + 1] = and_or(x, 0x00F000F0u, kMagic);
-    P[4 * u + 2] = and_or(x2, 0x000F000Fu, kMagic);
-    P[4 * u + 3] = and_or(x2, 0x00F000F0u, kMagic);
+    P[4 * u + 0] = mask_field(x, 0x000F000Fu, kMagic);
+    P[4 * u + 1] = mask_field(x, 0x00F000F0u, kMagic);
+    P[4 * u + 2] = mask_field(x2, 0x000F000Fu, kMagic);
+    P[4 * u + 3] = mask_field(x2, 0x00F000F0u, kMagic);
   }
 }
 
@@ -115,8 +120,8 @@ template <>
 __device__ __forceinline__ void decode16<8>(const uint32_t (&w)[8], uint32_t (&P)[16]) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    P[2 * u + 0] = prmt(w[u], 0x64646464u, 0x4240u);
-    P[2 * u + 1] = prmt(w[u], 0x64646464u, 0x4341u);
+    P[2 * u + 0] = prmt(w[u], 0u, 0x4240u);
+    P[2 * u + 1] = prmt(w[u], 0u, 0x4341u);
   }
 }
 
@@ -133,63 +138,22 @@ __device__ __forceinline__ void decode16<3>(const uint32_t (&w)[3], uint32_t (&P
   const uint32_t v5 = funnel_r(w[1], w[2], 10);
   const uint32_t v6 = w[2] >> 1;
   const uint32_t v7 = w[2] >> 10;
-  P[0] = and_or(v1, m3(1, 0), kMagic);
-  P[1] = and_or(v1, m3(4, 3), kMagic);
-  P[2] = and_or(v1, m3(7, 6), kMagic);
-  P[3] = and_or(v2, m3(1, 0), kMagic);
-  P[4] = and_or(v2, m3(4, 3), kMagic);
-  P[5] = and_or(v3, m3(0, 2), kMagic);
-  P[6] = and_or(v3, m3(3, 5), kMagic);
-  P[7] = and_or(v4, m3(0, 2), kMagic);
-  P[8] = and_or(v4, m3(3, 5), kMagic);
-  P[9] = and_or(v5, m3(0, 2), kMagic);
-  P[10] = and_or(v5, m3(3, 5), kMagic);
-  P[11] = and_or(v6, m3(1, 0), kMagic);
-  P[12] = and_or(v6, m3(4, 3), kMagic);
-  P[13] = and_or(v6, m3(7, 6), kMagic);
-  P[14] = and_or(v7, m3(1, 0), kMagic);
-  P[15] = and_or(v7, m3(4, 3), kMagic);
-}
-
-// fp16 bit pattern of 2^-a (a <= 14).
-__host__ __device__ constexpr uint32_t half_pow2_neg(int a) {
-  return static_cast<uint32_t>(15 - a) << 10;
-}
-
-// half2 multiplier (2^-a_lo, 2^-a_hi) of pair p.
-template <int BITS>
-__host__ __device__ constexpr uint32_t pair_mult(int p) {
-  return half_pow2_neg(Pairs<BITS>::get(p).a_lo) | (half_pow2_neg(Pairs<BITS>::get(p).a_hi) << 16);
-}
-
-// fp16 bit pattern of -v for an integer 1 <= v < 2048 (exact).
-__host__ __device__ constexpr uint32_t half_neg_int(int v) {
-  int e = 0;
-  while ((v >> (e + 1)) != 0) ++e;
-  return 0x8000u | (static_cast<uint32_t>(e + 15) << 10) |
-         ((static_cast<uint32_t>(v) << (10 - e)) & 0x3FFu);
-}
-
-// half2 addend -(1024 2^-a + zero) of pair p (host side, per launch).
-template <int BITS>
-inline uint32_t pair_addend(int p, int zero) {
-  const PairDesc d = Pairs<BITS>::get(p);
-  return half_neg_int((1024 >> d.a_lo) + zero) | (half_neg_int((1024 >> d.a_hi) + zero) << 16);
-}
-
-__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
-  uint32_t d;
-  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
-  return d;
-}
-
-// Decode a bundle straight to exact (q - zero) fp16 pairs.
-template <int BITS>
-__device__ __forceinline__ void decode16_exact(const uint32_t (&w)[BITS], const uint32_t* add,
-                                               uint32_t (&P)[16]) {
-  decode16<BITS>(w, P);
-#pragma unroll
-  for (int p = 0; p < 16; ++p) P[p] = hfma2(P[p], pair_mult<BITS>(p), add[p]);
+  P[0] = mask_field(v1, m3(1, 0), kMagic);
+  P[1] = mask_field(v1, m3(4, 3), kMagic);
+  P[2] = mask_field(v1, m3(7, 6), kMagic);
+  P[3] = mask_field(v2, m3(1, 0), kMagic);
+  P[4] = mask_field(v2, m3(4, 3), kMagic);
+  P[5] = mask_field(v3, m3(0, 2), kMagic);
+  P[6] = mask_field(v3, m3(3, 5), kMagic);
+  P[7] = mask_field(v4, m3(0, 2), kMagic);
+  P[8] = mask_field(v4, m3(3, 5), kMagic);
+  P[9] = mask_field(v5, m3(0, 2), kMagic);
+  P[10] = mask_field(v5, m3(3, 5), kMagic);
+  P[11] = mask_field(v6, m3(1, 0), kMagic);
+  P[12] = mask_field(v6, m3(4, 3), kMagic);
+  P[13] = mask_field(v6, m3(7, 6), kMagic);
+  P[14] = mask_field(v7, m3(1, 0), kMagic);
+  P[15] = mask_field(v7, m3(4, 3), kMagic);
 }
 
 // Load a lane's BITS-word bundle from shared memory (16-byte aligned for

