@@ -187,4 +187,3 @@ hq_status hq_unpack_codes(const uint32_t* packed, int bits, size_t n_codes, uint
 
 }  // extern "C"
 
-// The MoE entry points are defined in moe.cu.

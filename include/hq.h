@@ -180,6 +180,10 @@ uint64_t hq_launch_count(void);
 /* Kernels one hq_linear call enqueues for this weight and batch. */
 int hq_linear_launches(const hq_weight* w, int batch);
 
+/* Kernels one hq_moe_experts call enqueues (route, rotate x, gate/up,
+ * rotate h, down, combine). */
+int hq_moe_launches(void);
+
 /* Batch size from which hq_linear uses the tensor-core GEMM (default 9).
  * Returns the previous value; values < 1 are ignored. */
 int hq_set_tc_min_batch(int n);

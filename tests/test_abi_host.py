@@ -109,3 +109,33 @@ def test_unpack_rejects_bad_args(L):
     assert L.hq_unpack_codes(FAKE + 2, 3, 10, FAKE, None) == HQ_ERR_INVALID_ARG
     assert L.hq_unpack_codes(None, 3, 10, FAKE, None) == HQ_ERR_INVALID_ARG
     assert L.hq_launch_count() == before
+
+
+def moe_call(L, **kw):
+    a = dict(ex=FAKE, E=8, hidden=256, inter=128, x=FAKE, T=4, ids=FAKE, w=FAKE, k=2,
+             si=None, sm=None, y=FAKE, ws=FAKE, ws_bytes=1 << 30)
+    a.update(kw)
+    return L.hq_moe_experts(a["ex"], a["E"], a["hidden"], a["inter"], a["x"], a["T"], a["ids"],
+                            a["w"], a["k"], a["si"], a["sm"], a["y"], a["ws"], a["ws_bytes"], None)
+
+
+def test_moe_rejects_bad_args(L):
+    before = L.hq_launch_count()
+    assert moe_call(L, E=0) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, k=0) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, k=33) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, T=-1) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, hidden=384) == HQ_ERR_UNSUPPORTED
+    assert moe_call(L, inter=64) == HQ_ERR_UNSUPPORTED
+    assert moe_call(L, T=0) == HQ_OK
+    assert moe_call(L, x=None) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, x=FAKE + 8) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, ex=FAKE + 4) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, si=FAKE + 1) == HQ_ERR_INVALID_ARG
+    assert moe_call(L, ws=None) == HQ_ERR_WORKSPACE
+    need = L.hq_moe_workspace_size(8, 256, 128, 4, 2)
+    assert need > 0 and need % 256 == 0
+    assert moe_call(L, ws_bytes=need - 1) == HQ_ERR_WORKSPACE
+    assert L.hq_moe_workspace_size(0, 256, 128, 4, 2) == 0
+    assert L.hq_moe_launches() == 6
+    assert L.hq_launch_count() == before
