@@ -1,0 +1,127 @@
+// noalloc.cu -- hq_linear_noalloc: the rotated low-bit linear with its scratch
+// memory in a fixed, file-scope device array instead of a caller workspace.
+//
+// Who needs it: callers that cannot allocate device memory for a workspace.
+// A plug-in running inside another program's process may find the device heap
+// owned by that program's pool allocator, with no way to add buffers of its
+// own; a latency-critical loop cannot afford cudaMalloc, which may
+// synchronise the device and takes unbounded time; and a thin foreign-language
+// binding may have device pointers to its tensors but no allocator to manage a
+// scratch buffer's lifetime.  This entry point needs nothing beyond the
+// weight, input and output buffers.
+//
+// Costs of that convenience:
+//   * every GPU that loads the library keeps kScratchBytes (2 MiB) of device
+//     memory until the process exits;
+//   * every call shares the one array, so calls that overlap on the GPU (two
+//     streams, or two host threads) race on it and must be serialised by the
+//     caller;
+//   * device-side wait timeouts are recorded in the array's status word, which
+//     the next call clears; there is no way to read it back.
+#include <mutex>
+
+#include "hq_internal.h"
+
+namespace hq {
+namespace {
+
+constexpr size_t kScratchBytes = size_t{2} << 20;  // 2 MiB in total
+constexpr size_t kStatus = 256;                    // status word, kept zero
+constexpr size_t kPartBytes = size_t{1280} << 10;  // partial tiles: up to 1280 GEMV warps
+constexpr size_t kCntBytes = kScratchBytes - kStatus - kPartBytes;  // tile counters
+// Largest output-row count: one 4-byte counter per 16 rows.
+constexpr long kMaxRows = static_cast<long>(kCntBytes / 4) * 16;
+
+// The scratch: [status][tile counters][split-tile partials].  Static storage
+// starts zeroed; each call clears the status word and the counters it uses.
+__device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mu;
+uint8_t* g_scratch_addr[kMaxDevices] = {};
+
+// Device address of the array on the current device (looked up once per
+// device: the host-side name of a __device__ variable is not a device address).
+cudaError_t scratch_on_current_device(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_scratch_addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+}  // namespace hq
+
+using namespace hq;
+
+extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, int batch, float* y,
+                                       hq_stream_t stream) {
+  auto aligned = [](const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
+  };
+  auto pow2 = [](int v) { return v > 0 && (v & (v - 1)) == 0; };
+  if (w == nullptr || w->M <= 0 || w->K <= 0 || w->M > (1 << 28)) return HQ_ERR_INVALID_ARG;
+  if (!(w->bits == 2 || w->bits == 3 || w->bits == 4 || w->bits == 8)) {
+    return (w->bits >= 1 && w->bits <= 8) ? HQ_ERR_UNSUPPORTED : HQ_ERR_INVALID_ARG;
+  }
+  if (!pow2(w->K) || w->K < 128 || w->K > 16384) return HQ_ERR_UNSUPPORTED;
+  if (w->zero < 0 || w->zero >= (1 << w->bits)) return HQ_ERR_INVALID_ARG;
+  if (!w->qweight || !w->scales || !aligned(w->qweight, 16) || !aligned(w->scales, 16) ||
+      (w->signs && !aligned(w->signs, 16))) {
+    return HQ_ERR_INVALID_ARG;
+  }
+  if (batch < 0 || batch > 65535) return HQ_ERR_INVALID_ARG;
+  if (batch == 0) return HQ_OK;
+  if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
+  // sizes beyond what the fixed scratch holds
+  if (w->M > kMaxRows) return HQ_ERR_WORKSPACE;
+  if (static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16 > kPartBytes) return HQ_ERR_WORKSPACE;
+  int nb = 0;
+  for (int b = 8; b >= 1 && nb == 0; b >>= 1) {
+    if (gemv_smem_bytes(w->bits, w->K, b) != 0) nb = b;
+  }
+  if (nb == 0) return HQ_ERR_UNSUPPORTED;
+
+  uint8_t* scratch = nullptr;
+  if (scratch_on_current_device(&scratch) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return HQ_ERR_CUDA;
+  }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const size_t n_tiles = static_cast<size_t>((w->M + 15) / 16);
+  if (cudaMemsetAsync(scratch, 0, kStatus + n_tiles * 4, st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return HQ_ERR_CUDA;
+  }
+  for (int n0 = 0; n0 < batch; n0 += nb) {
+    GemvArgs a;
+    a.bits = w->bits;
+    a.M = w->M;
+    a.K = w->K;
+    a.N = batch - n0 < nb ? batch - n0 : nb;
+    a.zero = w->zero;
+    a.q = w->qweight;
+    a.scales = w->scales;
+    a.x = x + static_cast<size_t>(n0) * w->K;
+    a.signs = w->signs;
+    a.y = y + static_cast<size_t>(n0) * w->M;
+    a.ldy = w->M;
+    a.status = reinterpret_cast<uint32_t*>(scratch);
+    a.cnt = reinterpret_cast<uint32_t*>(scratch + kStatus);
+    a.part = scratch + kStatus + kCntBytes;
+    if (launch_gemv(a, st) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return HQ_ERR_CUDA;
+    }
+  }
+  return HQ_OK;
+}

@@ -76,6 +76,21 @@ def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor |
     return out
 
 
+def hq_linear_noalloc(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
+                      x: torch.Tensor, bits: int, zero: int | None = None,
+                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """hq_linear without a workspace (the library's fixed device scratch is
+    used instead; calls must not overlap on the GPU)."""
+    _need_cuda(qweight, scales, signs, x)
+    w = make_weight(qweight, scales, signs, bits, zero)
+    N = x.shape[0]
+    if out is None:
+        out = torch.empty((N, w.M), dtype=torch.float32, device=x.device)
+    check(lib().hq_linear_noalloc(ctypes.byref(w), _ptr(x), N, _ptr(out), _stream(stream)),
+          "hq_linear_noalloc")
+    return out
+
+
 class RotatedLinear:
     """A packed, rotated linear layer bound to its device tensors and workspace."""
 
@@ -166,6 +181,6 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
-__all__ = ["hq_rotate", "hq_linear", "hq_linear_workspace_size", "RotatedLinear",
+__all__ = ["hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
            "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

@@ -159,6 +159,25 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
                          const int8_t* signs_mid, float* y, void* workspace,
                          size_t ws_bytes, hq_stream_t stream);
 
+/*
+ * hq_linear_noalloc -- hq_linear without a workspace, for callers that cannot
+ * allocate device memory (a plug-in whose host program owns the device heap, a
+ * latency-critical loop that must not call cudaMalloc, a binding with device
+ * pointers but no allocator).  The pages have no counterpart: this is a
+ * packaging variant of hq_linear, same arguments minus the workspace, same
+ * results (same kernels and work split).
+ * Its scratch is a 2 MiB array in the library's device memory, held on every
+ * GPU that loads the library until the process exits.  Limits: M <= 3,144,704
+ * output rows (HQ_ERR_WORKSPACE beyond), other limits as hq_linear.
+ * The first call on a device looks up the array's device address (a CUDA
+ * runtime query, no allocation); make that first call before any stream
+ * capture.  All calls share the array: calls that overlap on the GPU race and
+ * must be serialised by the caller.  Each call clears the part of the array
+ * that must start at zero; device-side wait timeouts cannot be read back.
+ */
+hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, int batch, float* y,
+                            hq_stream_t stream);
+
 /* Synchronises `stream`, reads the status word of a workspace used by
  * hq_linear or hq_moe_experts, clears it, and returns HQ_OK or the first
  * recorded device error (HQ_ERR_TIMEOUT before HQ_ERR_DATA). */
