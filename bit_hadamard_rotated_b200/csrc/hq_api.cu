@@ -50,23 +50,35 @@ static int gemv_col_block(int bits, int K) {
   return 0;
 }
 
-// hq_linear workspace: [status 256 B][GEMV partial tiles][tile counters].
+// Batches of at least the tensor-core threshold run on the tcgen05 GEMM
+// (when a tile plan fits this width and K); smaller ones on the GEMV.
+static bool use_tc(const hq_weight* w, int batch) {
+  return batch >= g_tc_min_batch.load(std::memory_order_relaxed) &&
+         tc_col_block(w->bits, w->K) > 0;
+}
+
+// hq_linear workspace: [status 256 B][GEMV partial tiles][tile counters]
+// [tensor-core path only: rotated activations, batch x K fp16].
 struct LinearWs {
   uint32_t* status;
   void* part;
   uint32_t* cnt;
+  void* xp;
   size_t bytes;
 };
 
-static LinearWs linear_ws(void* base, int M) {
+static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
   const size_t part_bytes = align256(static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16);
-  const size_t cnt_bytes = align256(static_cast<size_t>((M + 15) / 16) * 4);
+  const size_t cnt_bytes = align256(static_cast<size_t>((w->M + 15) / 16) * 4);
+  const size_t xp_bytes =
+      use_tc(w, batch) ? align256(static_cast<size_t>(batch) * w->K * 2) : 0;
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
   l.part = b + kStatusBytes;
   l.cnt = reinterpret_cast<uint32_t*>(b + kStatusBytes + part_bytes);
-  l.bytes = kStatusBytes + part_bytes + cnt_bytes;
+  l.xp = b + kStatusBytes + part_bytes + cnt_bytes;
+  l.bytes = kStatusBytes + part_bytes + cnt_bytes + xp_bytes;
   return l;
 }
 
@@ -115,11 +127,15 @@ hq_status hq_rotate(const void* x, hq_dtype x_dtype, void* x_rot, hq_dtype out_d
 
 size_t hq_linear_workspace_size(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch < 0) return 0;
-  return linear_ws(nullptr, w->M).bytes;
+  return linear_ws(nullptr, w, batch).bytes;
 }
 
 int hq_linear_launches(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch <= 0) return 0;
+  if (use_tc(w, batch)) {
+    const int nb = tc_col_block(w->bits, w->K);
+    return 1 + (batch + nb - 1) / nb;  // prep + one GEMM per batch block
+  }
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return 0;
   return (batch + nb - 1) / nb;
@@ -133,13 +149,30 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
   if (batch == 0) return HQ_OK;
   if (x == nullptr || y == nullptr) return HQ_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
-  const LinearWs l = linear_ws(workspace, w->M);
+  const LinearWs l = linear_ws(workspace, w, batch);
   if (workspace == nullptr || !aligned(workspace, 256) || ws_bytes < l.bytes) {
     return HQ_ERR_WORKSPACE;
   }
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (use_tc(w, batch)) {
+    TcArgs a;
+    a.bits = w->bits;
+    a.M = w->M;
+    a.K = w->K;
+    a.N = batch;
+    a.zero = w->zero;
+    a.q = w->qweight;
+    a.scales = w->scales;
+    a.x = x;
+    a.signs = w->signs;
+    a.y = y;
+    a.ldy = w->M;
+    a.status = l.status;
+    a.xp = l.xp;
+    return from_cuda(launch_linear_tc(a, st));
+  }
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return HQ_ERR_UNSUPPORTED;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   for (int n0 = 0; n0 < batch; n0 += nb) {
     GemvArgs a;
     a.bits = w->bits;

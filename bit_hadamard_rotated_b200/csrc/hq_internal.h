@@ -43,6 +43,22 @@ size_t gemv_smem_bytes(int bits, int K, int nb);
 int gemv_max_warps();
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 
+// Tensor-core path (tcgen05) for larger batches.
+struct TcArgs {
+  int bits, M, K, N, zero;
+  const uint32_t* q;
+  const uint16_t* scales;
+  const uint16_t* x;
+  const int8_t* signs;
+  float* y;
+  int ldy;
+  uint32_t* status;
+  void* xp;  // workspace: [N][K] fp16 rotated, pair-permuted activations
+};
+// Largest batch block per GEMM launch for this width and K (0: path unavailable).
+int tc_col_block(int bits, int K);
+cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st);
+
 cudaError_t launch_unpack(const uint32_t* packed, int bits, size_t n, uint8_t* out,
                           cudaStream_t st);
 

@@ -83,45 +83,49 @@ struct Pairs<3> {
 
 constexpr uint32_t kMagic = 0u;  // exponent field 0: the masked code is a subnormal
 
-__device__ __forceinline__ uint32_t mask_field(uint32_t x, uint32_t m, uint32_t /*exponent*/) {
-  return x & m;
+// (x & m) | e: the code field(s) of x with exponent bits e (0: subnormal).
+__device__ __forceinline__ uint32_t mask_field(uint32_t x, uint32_t m, uint32_t e) {
+  return e ? and_or(x, m, e) : (x & m);
 }
 
-template <int BITS>
+template <int B>
+struct int_tag {};
+
+template <int BITS, uint32_t MAGIC = kMagic>
 __device__ __forceinline__ void decode16(const uint32_t (&w)[BITS], uint32_t (&P)[16]);
 
-template <>
-__device__ __forceinline__ void decode16<2>(const uint32_t (&w)[2], uint32_t (&P)[16]) {
+template <int BITS, uint32_t MAGIC>
+__device__ __forceinline__ void decode16_impl(const uint32_t (&w)[2], uint32_t (&P)[16], int_tag<2>) {
 #pragma unroll
   for (int u = 0; u < 2; ++u) {
     const uint32_t x = w[u];
     const uint32_t x2 = x >> 10;
 #pragma unroll
-    for (int i = 0; i < 5; ++i) P[8 * u + i] = mask_field(x, 0x00030003u << (2 * i), kMagic);
+    for (int i = 0; i < 5; ++i) P[8 * u + i] = mask_field(x, 0x00030003u << (2 * i), MAGIC);
 #pragma unroll
-    for (int i = 0; i < 3; ++i) P[8 * u + 5 + i] = mask_field(x2, 0x00030003u << (2 * i), kMagic);
+    for (int i = 0; i < 3; ++i) P[8 * u + 5 + i] = mask_field(x2, 0x00030003u << (2 * i), MAGIC);
   }
 }
 
-template <>
-__device__ __forceinline__ void decode16<4>(const uint32_t (&w)[4], uint32_t (&P)[16]) {
+template <int BITS, uint32_t MAGIC>
+__device__ __forceinline__ void decode16_impl(const uint32_t (&w)[4], uint32_t (&P)[16], int_tag<4>) {
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
     const uint32_t x = w[u];
     const uint32_t x2 = x >> 8;
-    P[4 * u + 0] = mask_field(x, 0x000F000Fu, kMagic);
-    P[4 * u + 1] = mask_field(x, 0x00F000F0u, kMagic);
-    P[4 * u + 2] = mask_field(x2, 0x000F000Fu, kMagic);
-    P[4 * u + 3] = mask_field(x2, 0x00F000F0u, kMagic);
+    P[4 * u + 0] = mask_field(x, 0x000F000Fu, MAGIC);
+    P[4 * u + 1] = mask_field(x, 0x00F000F0u, MAGIC);
+    P[4 * u + 2] = mask_field(x2, 0x000F000Fu, MAGIC);
+    P[4 * u + 3] = mask_field(x2, 0x00F000F0u, MAGIC);
   }
 }
 
-template <>
-__device__ __forceinline__ void decode16<8>(const uint32_t (&w)[8], uint32_t (&P)[16]) {
+template <int BITS, uint32_t MAGIC>
+__device__ __forceinline__ void decode16_impl(const uint32_t (&w)[8], uint32_t (&P)[16], int_tag<8>) {
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    P[2 * u + 0] = prmt(w[u], 0u, 0x4240u);
-    P[2 * u + 1] = prmt(w[u], 0u, 0x4341u);
+    P[2 * u + 0] = prmt(w[u], MAGIC ? 0x64646464u : 0u, 0x4240u);
+    P[2 * u + 1] = prmt(w[u], MAGIC ? 0x64646464u : 0u, 0x4341u);
   }
 }
 
@@ -129,8 +133,8 @@ __device__ __forceinline__ constexpr uint32_t m3(int a_lo, int a_hi) {
   return (7u << a_lo) | (7u << (16 + a_hi));
 }
 
-template <>
-__device__ __forceinline__ void decode16<3>(const uint32_t (&w)[3], uint32_t (&P)[16]) {
+template <int BITS, uint32_t MAGIC>
+__device__ __forceinline__ void decode16_impl(const uint32_t (&w)[3], uint32_t (&P)[16], int_tag<3>) {
   const uint32_t v1 = w[0] << 1;
   const uint32_t v2 = w[0] >> 8;
   const uint32_t v3 = funnel_r(w[0], w[1], 30);
@@ -138,22 +142,67 @@ __device__ __forceinline__ void decode16<3>(const uint32_t (&w)[3], uint32_t (&P
   const uint32_t v5 = funnel_r(w[1], w[2], 10);
   const uint32_t v6 = w[2] >> 1;
   const uint32_t v7 = w[2] >> 10;
-  P[0] = mask_field(v1, m3(1, 0), kMagic);
-  P[1] = mask_field(v1, m3(4, 3), kMagic);
-  P[2] = mask_field(v1, m3(7, 6), kMagic);
-  P[3] = mask_field(v2, m3(1, 0), kMagic);
-  P[4] = mask_field(v2, m3(4, 3), kMagic);
-  P[5] = mask_field(v3, m3(0, 2), kMagic);
-  P[6] = mask_field(v3, m3(3, 5), kMagic);
-  P[7] = mask_field(v4, m3(0, 2), kMagic);
-  P[8] = mask_field(v4, m3(3, 5), kMagic);
-  P[9] = mask_field(v5, m3(0, 2), kMagic);
-  P[10] = mask_field(v5, m3(3, 5), kMagic);
-  P[11] = mask_field(v6, m3(1, 0), kMagic);
-  P[12] = mask_field(v6, m3(4, 3), kMagic);
-  P[13] = mask_field(v6, m3(7, 6), kMagic);
-  P[14] = mask_field(v7, m3(1, 0), kMagic);
-  P[15] = mask_field(v7, m3(4, 3), kMagic);
+  P[0] = mask_field(v1, m3(1, 0), MAGIC);
+  P[1] = mask_field(v1, m3(4, 3), MAGIC);
+  P[2] = mask_field(v1, m3(7, 6), MAGIC);
+  P[3] = mask_field(v2, m3(1, 0), MAGIC);
+  P[4] = mask_field(v2, m3(4, 3), MAGIC);
+  P[5] = mask_field(v3, m3(0, 2), MAGIC);
+  P[6] = mask_field(v3, m3(3, 5), MAGIC);
+  P[7] = mask_field(v4, m3(0, 2), MAGIC);
+  P[8] = mask_field(v4, m3(3, 5), MAGIC);
+  P[9] = mask_field(v5, m3(0, 2), MAGIC);
+  P[10] = mask_field(v5, m3(3, 5), MAGIC);
+  P[11] = mask_field(v6, m3(1, 0), MAGIC);
+  P[12] = mask_field(v6, m3(4, 3), MAGIC);
+  P[13] = mask_field(v6, m3(7, 6), MAGIC);
+  P[14] = mask_field(v7, m3(1, 0), MAGIC);
+  P[15] = mask_field(v7, m3(4, 3), MAGIC);
+}
+
+template <int BITS, uint32_t MAGIC>
+__device__ __forceinline__ void decode16(const uint32_t (&w)[BITS], uint32_t (&P)[16]) {
+  decode16_impl<BITS, MAGIC>(w, P, int_tag<BITS>{});
+}
+
+// ---- normal-range variant (tensor-core GEMM): with exponent field 0x6400
+// the pair holds 1024 + (code << a); one exact fp16 FMA per pair turns it
+// into q - zero: (1024 + 2^a q) * 2^-a - (1024 * 2^-a + zero).
+constexpr uint32_t kMagic1024 = 0x64006400u;
+
+__host__ __device__ constexpr uint32_t half_pow2_neg(int a) {
+  return static_cast<uint32_t>(15 - a) << 10;
+}
+
+template <int BITS>
+__host__ __device__ constexpr uint32_t pair_mult(int p) {
+  return half_pow2_neg(Pairs<BITS>::get(p).a_lo) | (half_pow2_neg(Pairs<BITS>::get(p).a_hi) << 16);
+}
+
+// fp16 bit pattern of -v for an integer 1 <= v < 2048 (exact).
+__host__ __device__ constexpr uint32_t half_neg_int(int v) {
+  int e = 0;
+  while ((v >> (e + 1)) != 0) ++e;
+  return 0x8000u | (static_cast<uint32_t>(e + 15) << 10) |
+         ((static_cast<uint32_t>(v) << (10 - e)) & 0x3FFu);
+}
+
+template <int BITS>
+__host__ __device__ inline uint32_t pair_addend(int p, int zero) {
+  return half_neg_int((1024 >> Pairs<BITS>::get(p).a_lo) + zero) |
+         (half_neg_int((1024 >> Pairs<BITS>::get(p).a_hi) + zero) << 16);
+}
+
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 // Load a lane's BITS-word bundle from shared memory (16-byte aligned for

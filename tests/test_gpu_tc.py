@@ -1,0 +1,159 @@
+"""GPU parity of the tensor-core (tcgen05) path of hq_linear against the oracle.
+
+hq_linear sends batches of at least the tensor-core threshold (9 by default)
+with K >= 1024 to the tcgen05 GEMM.  These cases check it element by element
+against the fp64 oracle with the same tolerance as the GEMV path,
+|y - y_oracle| <= 2e-3 sum_k |w_k x'_k| + 1e-5, over ragged row counts (partial
+128-row tiles), ragged batches (column blocks padded to 32), several column
+blocks per call, several tiles per CTA, every code width, null signs and
+non-default zero points.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_hadamard_rotated_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+REL, ABS = 2e-3, 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_hadamard_rotated_b200 import build
+    build.build()
+    import bit_hadamard_rotated_b200._lib as L
+    L.lib()
+    return torch.device("cuda:0")
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def assert_within(y, want, bound, what=""):
+    err = np.abs(y.astype(np.float64) - want)
+    lim = REL * bound + ABS
+    bad = err > lim
+    if bad.any():
+        i = np.unravel_index(np.argmax(err / lim), err.shape)
+        raise AssertionError(f"{what}: {bad.sum()} of {err.size} outside tolerance; worst at {i}: "
+                             f"got {y[i]!r} want {want[i]!r} err {err[i]:.3e} lim {lim[i]:.3e}")
+
+
+def weight(d):
+    from bit_hadamard_rotated_b200 import make_weight
+    q, s, g = dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"])
+    return q, s, g, make_weight(q, s, g, d["bits"], d["zero"])
+
+
+def run(d, signs=True):
+    from bit_hadamard_rotated_b200 import hq_launch_count, hq_linear
+    from bit_hadamard_rotated_b200._lib import lib
+    import ctypes
+    q, s, g, w = weight(d)
+    if not signs:
+        g = None
+        w.signs = None
+    expect = int(lib().hq_linear_launches(ctypes.byref(w), d["N"]))
+    x = dev(d["x"])
+    torch.cuda.synchronize()
+    n0 = hq_launch_count()
+    y = hq_linear(q, s, g, x, d["bits"], d["zero"])
+    torch.cuda.synchronize()
+    return y.cpu().numpy(), hq_launch_count() - n0, expect
+
+
+def tc_blocks(bits, K, N):
+    """Expected tensor-core launches: the prep kernel plus one GEMM per batch block."""
+    per = {2: 128, 3: 128, 4: 128, 8: 128}[bits]
+    # mirror of the shared-memory plan: blocks shrink where 4 ring slots do not fit
+    G = K // 128
+    cstride = 16 * bits + (0 if bits & 1 else 16)
+    b_off = (128 * cstride + 127) & ~127
+    sstride = (G * 2 + 15) & ~15
+    if (sstride >> 4) % 2 == 0:
+        sstride += 16
+    while per >= 32:
+        smem = ((4 * (b_off + 256 * per) + 2 * 128 * sstride + 15) & ~15) + 15 * 8 + 16
+        if smem <= 226 * 1024:
+            break
+        per -= 32
+    return 1 + (N + per - 1) // per
+
+
+CASES = [
+    # (M, K, N): ragged tiles, ragged batches, several blocks and tiles per CTA
+    (128, 1024, 9), (1, 1024, 16), (129, 1024, 31), (300, 2048, 33), (77, 4096, 64),
+    (256, 8192, 100), (200, 16384, 128), (130, 1024, 129), (64, 2048, 200),
+    (20000, 1024, 24),
+]
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("M,K,N", CASES)
+def test_tc_linear_parity(bits, M, K, N):
+    d = synth.linear(M, K, bits, N, seed=11 * M + K + 3 * N + bits)
+    y, launches, expect = run(d)
+    assert launches == expect == tc_blocks(bits, K, N), (launches, expect)
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y, want, bound, what=f"tc b{bits} M{M} K{K} N{N}")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_tc_nondefault_zero_null_signs_loguniform(bits):
+    M, K, N = 200, 2048, 40
+    d = synth.linear(M, K, bits, N, seed=99 + bits, scale_dist="loguniform", outlier_frac=0.01)
+    d["zero"] = (1 << bits) - 1 if bits < 8 else 3
+    y, _, _ = run(d, signs=False)
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], None, d["x"])
+    assert_within(y, want, bound, what=f"tc zero/null-signs b{bits}")
+
+
+def test_tc_matches_gemv_and_is_deterministic():
+    from bit_hadamard_rotated_b200 import hq_linear, hq_set_tc_min_batch
+    M, K, N, bits = 1000, 4096, 48, 3
+    d = synth.linear(M, K, bits, N, seed=5)
+    q, s, g, _ = weight(d)
+    x = dev(d["x"])
+    y1 = hq_linear(q, s, g, x, bits, d["zero"])
+    y2 = hq_linear(q, s, g, x, bits, d["zero"])
+    assert torch.equal(y1, y2)
+    old = hq_set_tc_min_batch(1 << 20)
+    try:
+        yg = hq_linear(q, s, g, x, bits, d["zero"])
+    finally:
+        hq_set_tc_min_batch(old)
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y1.cpu().numpy(), want, bound, what="tc")
+    assert_within(yg.cpu().numpy(), want, bound, what="gemv")
+
+
+def test_tc_output_overwritten_and_status_clean():
+    from bit_hadamard_rotated_b200 import RotatedLinear
+    M, K, N, bits = 300, 1024, 20, 2
+    d = synth.linear(M, K, bits, N, seed=8)
+    q, s, g, _ = weight(d)
+    lin = RotatedLinear(q, s, g, bits, d["zero"], max_batch=N)
+    out = torch.full((N, M), float("nan"), device="cuda")
+    lin(dev(d["x"]), out=out)
+    lin.check_status()
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(out.cpu().numpy(), want, bound, what="overwrite")
+
+
+def test_tc_workspace_too_small_is_rejected():
+    from bit_hadamard_rotated_b200 import HqError, hq_linear, hq_linear_workspace_size
+    M, K, N, bits = 256, 2048, 64, 4
+    d = synth.linear(M, K, bits, N, seed=3)
+    q, s, g, w = weight(d)
+    small = hq_linear_workspace_size(w, 8)
+    big = hq_linear_workspace_size(w, N)
+    assert big >= small + N * K * 2
+    ws = torch.zeros(small, dtype=torch.uint8, device="cuda")
+    with pytest.raises(HqError):
+        hq_linear(q, s, g, dev(d["x"]), bits, d["zero"], workspace=ws)
