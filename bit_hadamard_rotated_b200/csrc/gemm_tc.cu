@@ -3,22 +3,31 @@
 // At batch 16..256 the contraction is a dense one, so it runs on the
 // 5th-generation tensor cores with the fp32 accumulator in tensor memory:
 //   * a prep kernel rotates x (fp32 butterflies) and writes x' as fp16 in the
-//     k order of the decoded code pairs (hq_layout.cuh), so that A and B agree;
-//   * per CTA, one 128-row tile at a time: a producer warp streams each 128-code
-//     group (codes, scales, and the matching N x 128 block of x') through a
-//     4-slot cp.async ring, the B block landing in the canonical no-swizzle
-//     K-major core-matrix layout the MMA reads from shared memory;
+//     k order of the decoded code pairs (hq_layout.cuh), so that A and B agree,
+//     already in the shared-memory image the MMA reads (no-swizzle K-major
+//     core matrices), one contiguous block per 128-code group;
+//   * per CTA, one 128-row tile at a time: one producer thread streams each
+//     128-code group through a 4-slot ring -- the tile's 128 code rows in one
+//     2D TMA load (swizzled so the decoders' 16-byte row reads are free of
+//     bank conflicts), the group's x' image in one bulk copy, and at the
+//     tile's first group its scales in one bulk copy -- all completing on the
+//     slot's mbarrier (expected byte count);
 //   * two warpgroups alternate groups: each thread owns one weight row,
 //     decodes its 128 codes into exact fp16 (q - zero) (one LOP3 and one fp16
 //     FMA per pair), multiplies by the group scale (one fp16 multiply per pair:
 //     the weight's only rounding) and stores the row into tensor memory as the
 //     MMA's A operand (tcgen05.st), one TMEM lane per row;
-//   * the same producer warp issues 8 tcgen05.mma (M=128, N, K=16, A from TMEM,
-//     B from shared memory) per group and commits their completion to the
-//     slot's mbarrier; the tile's last commit releases the epilogue, which reads
-//     the fp32 accumulator with tcgen05.ld and writes y.
+//   * an MMA warp issues 8 tcgen05.mma (M=128, N, K=16, A from TMEM, B from
+//     shared memory) per group and commits their completion to the slot's
+//     mbarrier, which frees the slot for the producer; the tile's last commit
+//     releases the epilogue, which reads the fp32 accumulator with tcgen05.ld
+//     and writes y.
 // Waits are bounded (status word on timeout); tensor memory is freed on exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "fwht.cuh"
 #include "hq_common.cuh"
@@ -33,7 +42,9 @@ namespace tc {
 constexpr int kTileM = 128;
 constexpr int kNS = 4;            // ring slots (and A stages in tensor memory)
 constexpr int kDeqWarps = 8;      // two warpgroups
-constexpr int kThreads = (kDeqWarps + 1) * 32;
+constexpr int kProducerWarp = kDeqWarps;
+constexpr int kMmaWarp = kDeqWarps + 1;
+constexpr int kThreads = (kDeqWarps + 2) * 32;
 constexpr int kTmemCols = 512;
 constexpr int kAColBase = 256;    // A stages at columns 256 + 64 s; D at 0
 
@@ -102,6 +113,27 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "memory");
 }
 
+// 2D TMA tile load (no multicast) global -> shared, completing on bar.
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+      "{%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// 16-byte unit holding unit i of code row r in a slot: the TMA swizzle for
+// the row width (32 B rows: 32-byte swizzle, 64 B: 64-byte, 128 B: 128-byte;
+// 48 B rows are conflict-free unswizzled).
+template <int BITS>
+__device__ __forceinline__ int code_unit(int i, int r) {
+  if constexpr (BITS == 2) return i ^ ((r >> 2) & 1);
+  else if constexpr (BITS == 4) return i ^ ((r >> 1) & 3);
+  else if constexpr (BITS == 8) return i ^ (r & 7);
+  else return i;
+}
+
 // Shared-memory matrix descriptor, no swizzle, K-major: core matrices of
 // 8 rows x 16 bytes; lbo = byte distance between the two core matrices along
 // K, sbo = byte distance between consecutive 8-row groups.
@@ -116,47 +148,74 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// ---------------------------------------------------------------- prep: rotate + permute
-// One CTA per batch row: x'[n] (fp16) in the k order of the decoded pairs:
-// position 128 g + 32 t + 2 p + h holds x'[128 g + 32 t + code(p, h)].
+
+// ---------------------------------------------------------------- prep: rotate, permute, lay out
+// Byte offset of row n, k-position i (pair order) inside a batch block's
+// image: per 128-code group g a block of 256 Npad bytes holding the 8 K=16
+// slices (32 Npad bytes each) of an Npad x 128 K-major no-swizzle operand:
+// [slice ks][8-element half kc][row group n/8][row n%8][8 fp16].
+__host__ __device__ constexpr size_t img_offset(int g, int i, int n, int npad) {
+  return static_cast<size_t>(g) * 256 * npad + ((i >> 4) & 7) * 32 * npad + ((i >> 3) & 1) * 16 * npad +
+         (n >> 3) * 128 + (n & 7) * 16;
+}
+
+// Grid (nb, n_blocks): CTA (j, b) builds image row j of batch block b (rows
+// b*nb .. b*nb + nb - 1 of x); rows past the batch but inside the block's
+// 32-row padding are written as zeros, the rest of the CTAs exit at once.
+// Image of block b at byte b * K * 2 * nb of xp.  Position i of group g holds
+// x'[128 g + 32 t + code(p, h)] with i = 32 t + 2 p + h.
 template <int BITS, int LOGK>
 __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
     tc_prep_kernel(const __half* __restrict__ x, const int8_t* __restrict__ signs,
-                   __half* __restrict__ xp, float inv) {
+                   uint8_t* __restrict__ xp, int N, int nb, float inv) {
   using S = FwhtShape<LOGK>;
   extern __shared__ float buf[];
   pdl_launch_dependents();
+  const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int rows = min(nb, N - b * nb);
+  const int npad = (rows + 31) & ~31;
+  if (j >= npad) return;  // whole CTA: no barrier is reached
   pdl_wait();
-  const int tid = threadIdx.x, n = blockIdx.x;
-  float v[S::E];
-  load_chunk<__half, S::E>(x + static_cast<size_t>(n) * S::K + tid * S::E, v);
-  apply_signs<S::E>(signs ? signs + tid * S::E : nullptr, v);
-  fwht_block<LOGK, 5>(v, buf);
-  __half* out = xp + static_cast<size_t>(n) * S::K;
-  for (int i = tid; i < S::K; i += S::THREADS) {
-    const int g = i >> 7, t = (i >> 5) & 3, p = (i >> 1) & 15, h = i & 1;
-    const PairDesc pd = Pairs<BITS>::get(p);
-    const int k = kGroup * g + 32 * t + (h ? pd.c_hi : pd.c_lo);
-    out[i] = __float2half_rn(buf[fwht_pad(k)] * inv);
+  uint8_t* img = xp + static_cast<size_t>(b) * S::K * 2 * nb;
+  const int n = b * nb + j;
+  if (j < rows) {
+    float v[S::E];
+    load_chunk<__half, S::E>(x + static_cast<size_t>(n) * S::K + tid * S::E, v);
+    apply_signs<S::E>(signs ? signs + tid * S::E : nullptr, v);
+    fwht_block<LOGK, 5>(v, buf);
+  }
+  for (int seg = tid; seg < S::K / 8; seg += S::THREADS) {
+    const int g = seg >> 4, i0 = (seg * 8) & 127;
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (j < rows) {
+      const int t = i0 >> 5;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const PairDesc pd = Pairs<BITS>::get(((i0 >> 1) & 15) + q);
+        const int k0 = kGroup * g + 32 * t;
+        const __half lo = __float2half_rn(buf[fwht_pad(k0 + pd.c_lo)] * inv);
+        const __half hi = __float2half_rn(buf[fwht_pad(k0 + pd.c_hi)] * inv);
+        w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) |
+               (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
+      }
+    }
+    *reinterpret_cast<uint4*>(img + img_offset(g, i0, j, npad)) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
-
 // ---------------------------------------------------------------- the GEMM
 struct TcParams {
-  const uint32_t* q;
-  const __half* scales;
-  const __half* xp;  // [N][K] rotated, pair-permuted activations
-  float* y;
+  CUtensorMap qmap;       // packed codes [M][K bits / 8] as bytes; box 16 bits x 128 rows
+  const uint8_t* scales;  // fp16 [M][K/128]
+  const uint8_t* img;     // this batch block's x' image (G blocks of 256 Npad bytes)
+  float* y;               // this batch block's first output row
   uint32_t* status;
   int M, K, N, Npad, ldy;
   int n_tiles;
-  int cstride;     // bytes between code rows in a slot
   int slot_bytes;  // codes + B block
   int b_off;       // B block offset inside a slot
   int sbuf_off;    // per-tile scale buffers (two)
   int sbuf_bytes;
-  int sstride;     // bytes between scale rows in a scale buffer
   int bar_off;
   uint32_t idesc;
   uint32_t add[16];
@@ -164,7 +223,10 @@ struct TcParams {
 
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
-  extern __shared__ __align__(1024) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // swizzled TMA tiles need 1 KiB-aligned slots: round the base up (the
+  // launch asks for 1 KiB more than the plan)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.K / kGroup;
   const int CB = 16 * BITS;  // code bytes of one row in one 128-code group
@@ -175,18 +237,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   uint64_t* dfree = dready + 1;
   uint64_t* drain = dfree + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
-  __shared__ int abort_flag;
 
   if (tid == 0) {
     for (int i = 0; i < kNS; ++i) {
-      mbar_init(&full[i], 32);
+      mbar_init(&full[i], 1);
       mbar_init(&freeb[i], 1);
       mbar_init(&aready[i], 128);
     }
     mbar_init(dready, 1);
     mbar_init(dfree, 2 * 128);
     mbar_init(drain, 1);
-    abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
@@ -199,48 +259,50 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 
   const int n_my = (p.n_tiles - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
   const int total = n_my * G;
+  auto tile_m0 = [&](int ti) {
+    return (static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x)) * kTileM;
+  };
 
-  if (warp == kDeqWarps) {
-    // ---------------- producer + MMA issue
-    const uint8_t* qb = reinterpret_cast<const uint8_t*>(p.q);
-    const size_t row_bytes = static_cast<size_t>(p.K) * BITS / 8;
-    auto load = [&](int c) {
-      const int sl = c % kNS, ti = c / G, g = c % G;
-      const int m0 = (static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x)) * kTileM;
-      uint8_t* base = smem + sl * p.slot_bytes;
-      if (g == 0) {  // the tile's scales: rows m0..m0+127, all groups, padded rows
-        uint8_t* sb = smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes;
-        const int row_b = G * 2, pieces = (row_b + 15) >> 4;
-        for (int i = lane; i < kTileM * pieces; i += 32) {
-          const int r = i / pieces, pc = i - r * pieces;
-          const int nb = (m0 + r < p.M) ? min(16, row_b - pc * 16) : 0;
-          const uint8_t* src = reinterpret_cast<const uint8_t*>(p.scales) +
-                               (nb ? (static_cast<size_t>(m0 + r) * G * 2 + pc * 16) : 0);
-          cp_async16(sb + r * p.sstride + pc * 16, src, nb);
+  if (warp == kProducerWarp) {
+    // ---------------- producer (one thread): TMA + bulk copies into the ring
+    if (lane == 0) {
+      const uint32_t b_bytes = 256u * p.Npad;
+      const uint32_t code_bytes = kTileM * CB;
+      bool ok = true;
+      int issued = 0;
+      for (int c = 0; c < total; ++c) {
+        const int sl = c % kNS, ti = c / G, g = c - ti * G;
+        if (c >= kNS && !mbar_wait(&freeb[sl], ((c / kNS) - 1) & 1)) {
+          ok = false;
+          break;
         }
+        const int m0 = tile_m0(ti);
+        const int rows = min(kTileM, p.M - m0);
+        uint8_t* base = smem + sl * p.slot_bytes;
+        // a TMA tile always delivers the whole box (rows past M read as zero)
+        const uint32_t s_bytes = g == 0 ? static_cast<uint32_t>(rows) * G * 2 : 0u;
+        mbar_arrive_expect_tx(&full[sl], code_bytes + b_bytes + s_bytes);
+        tma_load_2d(base, &p.qmap, g * CB, m0, &full[sl]);
+        bulk_g2s(base + p.b_off, p.img + static_cast<size_t>(g) * b_bytes, b_bytes, &full[sl]);
+        if (g == 0) {
+          bulk_g2s(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes,
+                   p.scales + static_cast<size_t>(m0) * G * 2, s_bytes, &full[sl]);
+        }
+        issued = c + 1;
       }
-      for (int i = lane; i < kTileM * BITS; i += 32) {
-        const int r = i / BITS, c16 = i - r * BITS;
-        const bool ok = m0 + r < p.M;
-        const uint8_t* src = ok ? qb + static_cast<size_t>(m0 + r) * row_bytes +
-                                      static_cast<size_t>(g) * CB + c16 * 16
-                                : qb;
-        cp_async16(base + r * p.cstride + c16 * 16, src, ok ? 16 : 0);
+      // Drain: the copies of the last slots must have landed before exit (they
+      // have on the normal path, where the dequant warps consumed them).
+      for (int c = max(0, issued - kNS); c < issued; ++c) {
+        if (!mbar_wait(&full[c % kNS], (c / kNS) & 1)) ok = false;
       }
-      uint8_t* bdst = base + p.b_off;
-      for (int i = lane; i < 16 * p.Npad; i += 32) {
-        const int n = i >> 4, ks = (i >> 1) & 7, kc = i & 1;
-        const bool ok = n < p.N;
-        const __half* src = ok ? p.xp + static_cast<size_t>(n) * p.K + g * kGroup + ks * 16 + kc * 8 : p.xp;
-        cp_async16(bdst + ks * 32 * p.Npad + kc * 16 * p.Npad + (n >> 3) * 128 + (n & 7) * 16, src,
-                   ok ? 16 : 0);
-      }
-      cp_async_mbar_arrive(&full[sl]);
-    };
-    for (int c = 0; c < kNS && c < total; ++c) load(c);
+      if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMA issue
     bool ok = true;
     for (int c = 0; c < total && ok; ++c) {
-      const int sl = c % kNS, ti = c / G, g = c % G;
+      const int sl = c % kNS, ti = c / G, g = c - ti * G;
       if (g == 0 && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
       ok = ok && mbar_wait(&aready[sl], (c / kNS) & 1);
       if (!ok) break;
@@ -257,23 +319,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (g == G - 1) tc_commit(dready);
       }
       __syncwarp();
-      if (c >= 1 && c - 1 + kNS < total) {
-        ok = mbar_wait(&freeb[(c - 1) % kNS], ((c - 1) / kNS) & 1);
-        if (ok) load(c - 1 + kNS);
-      }
     }
-    if (!ok) {
-      if (lane == 0) {
-        record_error(p.status, HQ_DEV_TIMEOUT);
-        atomicExch(&abort_flag, 1);
-      }
-    }
-    // Drain: no copy or MMA of this CTA may be in flight when tensor memory
-    // is freed (matters only after a timeout; a no-op on the normal path).
-    asm volatile("cp.async.wait_all;" ::: "memory");
+    // Drain: no MMA may be in flight when tensor memory is freed.
     if (lane == 0) tc_commit(drain);
     __syncwarp();
-    if (!mbar_wait(drain, 0) && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
+    if (!mbar_wait(drain, 0)) ok = false;
+    if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
   } else {
     // ---------------- dequant (two warpgroups, alternate groups) + epilogue
     const int wg = warp >> 2;
@@ -292,7 +343,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         return;
       }
       tc_fence_after();
-      const int m = (static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x)) * kTileM + r;
+      const int m = tile_m0(ti) + r;
       const int half = p.Npad / 2;
       for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 16) {
         uint32_t v[16];
@@ -310,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       mbar_arrive(dfree);
     };
     for (int c = wg; c < total && ok; c += 2) {
-      const int sl = c % kNS, ti = c / G, g = c % G;
+      const int sl = c % kNS, ti = c / G, g = c - ti * G;
       if (ti != prev_ti) {
         if (prev_ti >= 0) epilogue(prev_ti);
         prev_ti = ti;
@@ -320,10 +371,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         ok = false;
         break;
       }
-      const uint8_t* rowp = smem + sl * p.slot_bytes + r * p.cstride;
+      const uint4* rowp = reinterpret_cast<const uint4*>(smem + sl * p.slot_bytes + r * CB);
       if ((g & 7) < 2) {  // first group of this warpgroup in a block of 8
         scache = *reinterpret_cast<const uint4*>(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes +
-                                                 r * p.sstride + (g >> 3) * 16);
+                                                 r * G * 2 + (g >> 3) * 16);
       }
       const int j = (g >> 1) & 3;
       const uint32_t sw = j == 0 ? scache.x : j == 1 ? scache.y : j == 2 ? scache.z : scache.w;
@@ -332,7 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       uint32_t rw[4 * BITS];  // the row's 128 codes, 16-byte loads
 #pragma unroll
       for (int i = 0; i < BITS; ++i) {
-        const uint4 u = reinterpret_cast<const uint4*>(rowp)[i];
+        const uint4 u = rowp[code_unit<BITS>(i, r)];
         rw[4 * i] = u.x;
         rw[4 * i + 1] = u.y;
         rw[4 * i + 2] = u.z;
@@ -351,16 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       }
       tc_wait_st();
       tc_fence_before();
-      // the slot's B block arrived through cp.async (generic proxy); the MMA
-      // reads it through the async proxy
-      fence_proxy_async_smem();
       mbar_arrive(&aready[sl]);
     }
     if (ok && prev_ti >= 0) epilogue(prev_ti);
-    if (!ok) {
-      if (lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
-      atomicExch(&abort_flag, 1);
-    }
+    if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
   }
   tc_fence_before();
   __syncthreads();
@@ -371,66 +416,110 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   }
 }
 
-
 // ---------------------------------------------------------------- host side
 struct TcPlan {
-  int cstride = 0, slot = 0, b_off = 0, sbuf_off = 0, sbuf_bytes = 0, sstride = 0, bar_off = 0;
+  int slot = 0, b_off = 0, sbuf_off = 0, sbuf_bytes = 0, bar_off = 0;
   size_t smem = 0;
 };
 
-constexpr size_t kMaxSmemTc = 226 * 1024;  // dynamic; leaves room for the static words
-constexpr size_t kMinSmemTc = 116 * 1024;  // > half an SM's shared memory
+constexpr size_t kMaxSmemTc = 227 * 1024 - 1024;  // dynamic; the base is rounded up to 1 KiB
+constexpr size_t kMinSmemTc = 116 * 1024;         // > half an SM's shared memory
 
 static TcPlan tc_plan(int bits, int K, int npad) {
   TcPlan pl;
   const int G = K / kGroup;
-  // code rows: 16*bits bytes, padded to an odd number of 16-byte units so that
-  // the 16-byte row loads of 8 consecutive threads hit distinct banks
-  pl.cstride = 16 * bits + ((bits & 1) ? 0 : 16);
-  pl.b_off = (kTileM * pl.cstride + 127) & ~127;
+  // slot: [128 code rows, 16*bits bytes each, dense and swizzled][x' image];
+  // both sizes are multiples of 1 KiB, so every slot keeps the swizzle atom
+  pl.b_off = kTileM * 16 * bits;
   pl.slot = pl.b_off + 256 * npad;
   pl.sbuf_off = kNS * pl.slot;
-  // scale rows padded to an odd number of 16-byte units (conflict-free uint4 reads)
-  pl.sstride = ((G * 2 + 15) & ~15);
-  if (((pl.sstride >> 4) & 1) == 0) pl.sstride += 16;
-  pl.sbuf_bytes = kTileM * pl.sstride;
-  pl.bar_off = (pl.sbuf_off + 2 * pl.sbuf_bytes + 15) & ~15;
-  pl.smem = static_cast<size_t>(pl.bar_off) + (3 * kNS + 3) * 8 + 16;
+  pl.sbuf_bytes = kTileM * G * 2;
+  pl.bar_off = pl.sbuf_off + 2 * pl.sbuf_bytes;
+  pl.smem = static_cast<size_t>(pl.bar_off) + (3 * kNS + 3) * 8 + 16 + 1024;
   // one CTA per SM: each holds all 512 tensor-memory columns
   pl.smem = std::max(pl.smem, kMinSmemTc);
   return pl;
 }
 
+using EncodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
+
+static EncodeTiled encode_tiled() {
+  static std::once_flag once;
+  static EncodeTiled fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiled>(f);
+    }
+  });
+  return fn;
+}
+
+// Codes of W as a 2D byte tensor [M][K bits / 8]; box = one group's 16*bits
+// bytes x 128 rows.
+static cudaError_t code_map(CUtensorMap* map, const void* q, int bits, int M, int K) {
+  EncodeTiled fn = encode_tiled();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(K) * bits / 8;
+  const cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * bits), static_cast<cuuint32_t>(kTileM)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = bits == 2   ? CU_TENSOR_MAP_SWIZZLE_32B
+                                 : bits == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                 : bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                             : CU_TENSOR_MAP_SWIZZLE_NONE;
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(q), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace tc
 
 int tc_col_block(int bits, int K) {
-  // K >= 1024: whole 16-byte scale pieces per row, and >= 8 groups per tile
-  // (a tile's scale buffer is reloaded only after the previous tile's MMAs)
-  if (K < 1024) return 0;
+  // K >= 1024: whole 16-byte scale rows, and >= 8 groups per tile (a tile's
+  // scale buffer is refilled only after the MMAs two tiles back are done)
+  if (K < 1024 || K > 16384) return 0;
   for (int nb = 128; nb >= 32; nb -= 32) {
     if (tc::tc_plan(bits, K, nb).smem <= tc::kMaxSmemTc) return nb;
   }
   return 0;
 }
 
+size_t tc_xp_bytes(int bits, int K, int batch) {
+  const int nb = tc_col_block(bits, K);
+  if (nb == 0) return 0;
+  return static_cast<size_t>((batch + nb - 1) / nb) * nb * K * 2;
+}
+
+int tc_launches(int bits, int K, int batch) {
+  const int nb = tc_col_block(bits, K);
+  return nb == 0 ? 0 : 1 + (batch + nb - 1) / nb;
+}
+
 template <int BITS, int LOGK>
-static cudaError_t tc_prep_t(const __half* x, const int8_t* s, __half* xp, int N, cudaStream_t st) {
+static cudaError_t tc_prep_t(const __half* x, const int8_t* s, uint8_t* xp, int N, int nb,
+                             cudaStream_t st) {
   using S = FwhtShape<LOGK>;
   const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(S::K)));
-  return launch_pdl(tc::tc_prep_kernel<BITS, LOGK>, dim3(N), dim3(S::THREADS),
-                    S::SMEM_FLOATS * sizeof(float), st, true, x, s, xp, inv);
+  const dim3 grid(nb, (N + nb - 1) / nb);
+  return launch_pdl(tc::tc_prep_kernel<BITS, LOGK>, grid, dim3(S::THREADS),
+                    S::SMEM_FLOATS * sizeof(float), st, true, x, s, xp, N, nb, inv);
 }
 
 template <int BITS>
-static cudaError_t tc_prep_b(int K, const __half* x, const int8_t* s, __half* xp, int N,
+static cudaError_t tc_prep_b(int K, const __half* x, const int8_t* s, uint8_t* xp, int N, int nb,
                              cudaStream_t st) {
   switch (K) {
-    case 512: return tc_prep_t<BITS, 9>(x, s, xp, N, st);
-    case 1024: return tc_prep_t<BITS, 10>(x, s, xp, N, st);
-    case 2048: return tc_prep_t<BITS, 11>(x, s, xp, N, st);
-    case 4096: return tc_prep_t<BITS, 12>(x, s, xp, N, st);
-    case 8192: return tc_prep_t<BITS, 13>(x, s, xp, N, st);
-    case 16384: return tc_prep_t<BITS, 14>(x, s, xp, N, st);
+    case 1024: return tc_prep_t<BITS, 10>(x, s, xp, N, nb, st);
+    case 2048: return tc_prep_t<BITS, 11>(x, s, xp, N, nb, st);
+    case 4096: return tc_prep_t<BITS, 12>(x, s, xp, N, nb, st);
+    case 8192: return tc_prep_t<BITS, 13>(x, s, xp, N, nb, st);
+    case 16384: return tc_prep_t<BITS, 14>(x, s, xp, N, nb, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -443,27 +532,30 @@ static void tc_addends(uint32_t (&add)[16], int zero) {
 cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
   const int nb = tc_col_block(a.bits, a.K);
   if (nb == 0) return cudaErrorInvalidValue;
-  __half* xp = static_cast<__half*>(a.xp);
+  uint8_t* xp = static_cast<uint8_t*>(a.xp);
   const __half* xh = reinterpret_cast<const __half*>(a.x);
   cudaError_t e;
   switch (a.bits) {
-    case 2: e = tc_prep_b<2>(a.K, xh, a.signs, xp, a.N, st); break;
-    case 3: e = tc_prep_b<3>(a.K, xh, a.signs, xp, a.N, st); break;
-    case 4: e = tc_prep_b<4>(a.K, xh, a.signs, xp, a.N, st); break;
-    case 8: e = tc_prep_b<8>(a.K, xh, a.signs, xp, a.N, st); break;
+    case 2: e = tc_prep_b<2>(a.K, xh, a.signs, xp, a.N, nb, st); break;
+    case 3: e = tc_prep_b<3>(a.K, xh, a.signs, xp, a.N, nb, st); break;
+    case 4: e = tc_prep_b<4>(a.K, xh, a.signs, xp, a.N, nb, st); break;
+    case 8: e = tc_prep_b<8>(a.K, xh, a.signs, xp, a.N, nb, st); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
+  CUtensorMap qmap;
+  e = tc::code_map(&qmap, a.q, a.bits, a.M, a.K);
+  if (e != cudaSuccess) return e;
   const int n_tiles = (a.M + tc::kTileM - 1) / tc::kTileM;
   const unsigned grid = static_cast<unsigned>(std::min(n_tiles, gemv_max_warps() / 8));
-  for (int n0 = 0; n0 < a.N; n0 += nb) {
+  for (int b = 0, n0 = 0; n0 < a.N; ++b, n0 += nb) {
     const int nk = std::min(nb, a.N - n0);
     const int npad = (nk + 31) & ~31;
     const tc::TcPlan pl = tc::tc_plan(a.bits, a.K, npad);
     tc::TcParams p{};
-    p.q = a.q;
-    p.scales = reinterpret_cast<const __half*>(a.scales);
-    p.xp = xp + static_cast<size_t>(n0) * a.K;
+    p.qmap = qmap;
+    p.scales = reinterpret_cast<const uint8_t*>(a.scales);
+    p.img = xp + static_cast<size_t>(b) * a.K * 2 * nb;
     p.y = a.y + static_cast<size_t>(n0) * a.ldy;
     p.status = a.status;
     p.M = a.M;
@@ -472,20 +564,18 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.Npad = npad;
     p.ldy = a.ldy;
     p.n_tiles = n_tiles;
-    p.cstride = pl.cstride;
     p.slot_bytes = pl.slot;
     p.b_off = pl.b_off;
     p.sbuf_off = pl.sbuf_off;
     p.sbuf_bytes = pl.sbuf_bytes;
-    p.sstride = pl.sstride;
     p.bar_off = pl.bar_off;
     p.idesc = tc::idesc_f16(tc::kTileM, npad);
-    const dim3 g(grid), b(tc::kThreads);
+    const dim3 g(grid), blk(tc::kThreads);
     switch (a.bits) {
-      case 2: tc_addends<2>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<2>, g, b, pl.smem, st, true, p); break;
-      case 3: tc_addends<3>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<3>, g, b, pl.smem, st, true, p); break;
-      case 4: tc_addends<4>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<4>, g, b, pl.smem, st, true, p); break;
-      default: tc_addends<8>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<8>, g, b, pl.smem, st, true, p); break;
+      case 2: tc_addends<2>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<2>, g, blk, pl.smem, st, true, p); break;
+      case 3: tc_addends<3>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<3>, g, blk, pl.smem, st, true, p); break;
+      case 4: tc_addends<4>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<4>, g, blk, pl.smem, st, true, p); break;
+      default: tc_addends<8>(p.add, a.zero); e = launch_pdl(tc::tc_gemm_kernel<8>, g, blk, pl.smem, st, true, p); break;
     }
     if (e != cudaSuccess) return e;
   }

@@ -58,7 +58,8 @@ static bool use_tc(const hq_weight* w, int batch) {
 }
 
 // hq_linear workspace: [status 256 B][GEMV partial tiles][tile counters]
-// [tensor-core path only: rotated activations, batch x K fp16].
+// [tensor-core path only: rotated activation images, batch rounded up to whole
+// batch blocks, x K fp16].
 struct LinearWs {
   uint32_t* status;
   void* part;
@@ -71,8 +72,7 @@ static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
   const size_t part_bytes = align256(static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16);
   const size_t cnt_bytes = align256(static_cast<size_t>((w->M + 15) / 16) * 4);
-  const size_t xp_bytes =
-      use_tc(w, batch) ? align256(static_cast<size_t>(batch) * w->K * 2) : 0;
+  const size_t xp_bytes = use_tc(w, batch) ? align256(tc_xp_bytes(w->bits, w->K, batch)) : 0;
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
   l.part = b + kStatusBytes;
@@ -132,10 +132,7 @@ size_t hq_linear_workspace_size(const hq_weight* w, int batch) {
 
 int hq_linear_launches(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch <= 0) return 0;
-  if (use_tc(w, batch)) {
-    const int nb = tc_col_block(w->bits, w->K);
-    return 1 + (batch + nb - 1) / nb;  // prep + one GEMM per batch block
-  }
+  if (use_tc(w, batch)) return tc_launches(w->bits, w->K, batch);
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return 0;
   return (batch + nb - 1) / nb;

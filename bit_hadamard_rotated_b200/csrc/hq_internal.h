@@ -53,10 +53,14 @@ struct TcArgs {
   float* y;
   int ldy;
   uint32_t* status;
-  void* xp;  // workspace: [N][K] fp16 rotated, pair-permuted activations
+  void* xp;  // workspace: tc_xp_bytes(bits, K, N) bytes, 256-byte aligned
 };
 // Largest batch block per GEMM launch for this width and K (0: path unavailable).
 int tc_col_block(int bits, int K);
+// Workspace bytes for the rotated activation images of a batch.
+size_t tc_xp_bytes(int bits, int K, int batch);
+// Kernel launches of one tensor-core hq_linear call (prep + one GEMM per block).
+int tc_launches(int bits, int K, int batch);
 cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st);
 
 cudaError_t launch_unpack(const uint32_t* packed, int bits, size_t n, uint8_t* out,

@@ -70,17 +70,14 @@ def run(d, signs=True):
 
 def tc_blocks(bits, K, N):
     """Expected tensor-core launches: the prep kernel plus one GEMM per batch block."""
-    per = {2: 128, 3: 128, 4: 128, 8: 128}[bits]
-    # mirror of the shared-memory plan: blocks shrink where 4 ring slots do not fit
+    # mirror of the shared-memory plan: 4 ring slots of [128 code rows][x' image],
+    # two tile scale buffers, barriers, 1 KiB alignment pad; blocks shrink from
+    # 128 columns in steps of 32 until the plan fits
     G = K // 128
-    cstride = 16 * bits + (0 if bits & 1 else 16)
-    b_off = (128 * cstride + 127) & ~127
-    sstride = (G * 2 + 15) & ~15
-    if (sstride >> 4) % 2 == 0:
-        sstride += 16
+    per = 128
     while per >= 32:
-        smem = ((4 * (b_off + 256 * per) + 2 * 128 * sstride + 15) & ~15) + 15 * 8 + 16
-        if smem <= 226 * 1024:
+        smem = 4 * (128 * 16 * bits + 256 * per) + 2 * 128 * G * 2 + 15 * 8 + 16 + 1024
+        if smem <= 227 * 1024 - 1024:
             break
         per -= 32
     return 1 + (N + per - 1) // per
