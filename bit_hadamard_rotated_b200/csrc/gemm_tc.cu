@@ -17,11 +17,15 @@
 //     FMA per pair), multiplies by the group scale (one fp16 multiply per pair:
 //     the weight's only rounding) and stores the row into tensor memory as the
 //     MMA's A operand (tcgen05.st), one TMEM lane per row;
-//   * an MMA warp issues 8 tcgen05.mma (M=128, N, K=16, A from TMEM, B from
-//     shared memory) per group and commits their completion to the slot's
-//     mbarrier, which frees the slot for the producer; the tile's last commit
-//     releases the epilogue, which reads the fp32 accumulator with tcgen05.ld
-//     and writes y.
+//   * n_mma MMA warps (4 when the batch block pads to <= 64 columns, else 2)
+//     take the groups round robin; each issues 8 tcgen05.mma (M=128, N, K=16,
+//     A from TMEM, B from shared memory) per group into its own fp32
+//     accumulator in tensor memory and commits their completion to the slot's
+//     mbarrier, which frees the slot for the producer.  A single issuing
+//     thread sustains only one MMA per ~60-80 cycles whatever N is, so at
+//     batch <= 128 several issuers are what keeps the tensor pipe busy;
+//   * the tile's last commits release the epilogue, which sums the
+//     accumulators (tcgen05.ld) and writes y.
 // Waits are bounded (status word on timeout); tensor memory is freed on exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -43,10 +47,11 @@ constexpr int kTileM = 128;
 constexpr int kNS = 4;            // ring slots (and A stages in tensor memory)
 constexpr int kDeqWarps = 8;      // two warpgroups
 constexpr int kProducerWarp = kDeqWarps;
-constexpr int kMmaWarp = kDeqWarps + 1;
-constexpr int kThreads = (kDeqWarps + 2) * 32;
+constexpr int kMmaWarp0 = kDeqWarps + 1;
+constexpr int kMmaWarps = 4;      // issuing threads: one thread issues an MMA per ~60-80 cycles
+constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps) * 32;
 constexpr int kTmemCols = 512;
-constexpr int kAColBase = 256;    // A stages at columns 256 + 64 s; D at 0
+constexpr int kAColBase = 256;    // A stages at columns 256 + 64 s; accumulators below 256
 
 // ---------------------------------------------------------------- tcgen05 wrappers
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -217,6 +222,8 @@ struct TcParams {
   int sbuf_off;    // per-tile scale buffers (two)
   int sbuf_bytes;
   int bar_off;
+  int n_mma;    // MMA warps (accumulators) in use: 2 or 4
+  int dstride;  // tensor-memory columns between accumulators (256 / n_mma >= Npad)
   uint32_t idesc;
   uint32_t add[16];
 };
@@ -244,9 +251,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       mbar_init(&freeb[i], 1);
       mbar_init(&aready[i], 128);
     }
-    mbar_init(dready, 1);
+    mbar_init(dready, p.n_mma);
     mbar_init(dfree, 2 * 128);
-    mbar_init(drain, 1);
+    mbar_init(drain, p.n_mma);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
@@ -270,25 +277,41 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const uint32_t code_bytes = kTileM * CB;
       bool ok = true;
       int issued = 0;
+      // ring position kept incrementally (no divisions on the issue path)
+      int sl = 0, g = 0;
+      uint32_t rph = 0;  // parity of the ring round of chunk c
+      int m0 = tile_m0(0), ti = 0;
+      int rows = min(kTileM, p.M - m0);
+      const uint8_t* bsrc = p.img;
       for (int c = 0; c < total; ++c) {
-        const int sl = c % kNS, ti = c / G, g = c - ti * G;
-        if (c >= kNS && !mbar_wait(&freeb[sl], ((c / kNS) - 1) & 1)) {
+        // slot reuse: the MMAs of chunk c - kNS (previous round) are done
+        if (c >= kNS && !mbar_wait(&freeb[sl], rph ^ 1u)) {
           ok = false;
           break;
         }
-        const int m0 = tile_m0(ti);
-        const int rows = min(kTileM, p.M - m0);
         uint8_t* base = smem + sl * p.slot_bytes;
         // a TMA tile always delivers the whole box (rows past M read as zero)
         const uint32_t s_bytes = g == 0 ? static_cast<uint32_t>(rows) * G * 2 : 0u;
         mbar_arrive_expect_tx(&full[sl], code_bytes + b_bytes + s_bytes);
         tma_load_2d(base, &p.qmap, g * CB, m0, &full[sl]);
-        bulk_g2s(base + p.b_off, p.img + static_cast<size_t>(g) * b_bytes, b_bytes, &full[sl]);
+        bulk_g2s(base + p.b_off, bsrc, b_bytes, &full[sl]);
         if (g == 0) {
           bulk_g2s(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes,
                    p.scales + static_cast<size_t>(m0) * G * 2, s_bytes, &full[sl]);
         }
         issued = c + 1;
+        bsrc += b_bytes;
+        if (++sl == kNS) {
+          sl = 0;
+          rph ^= 1u;
+        }
+        if (++g == G) {
+          g = 0;
+          ++ti;
+          m0 += static_cast<int>(gridDim.x) * kTileM;
+          rows = min(kTileM, p.M - m0);
+          bsrc = p.img;
+        }
       }
       // Drain: the copies of the last slots must have landed before exit (they
       // have on the normal path, where the dequant warps consumed them).
@@ -298,33 +321,53 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ---------------- MMA issue
-    bool ok = true;
-    for (int c = 0; c < total && ok; ++c) {
-      const int sl = c % kNS, ti = c / G, g = c - ti * G;
-      if (g == 0 && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
-      ok = ok && mbar_wait(&aready[sl], (c / kNS) & 1);
-      if (!ok) break;
-      tc_fence_after();
-      if (lane == 0) {
-        const uint32_t a0 = tmem + kAColBase + sl * 64;
-        const uint32_t b0 = smem_u32(smem + sl * p.slot_bytes + p.b_off);
+  } else if (warp >= kMmaWarp0) {
+    // ---------------- MMA issue: warp j takes chunks j, j + n_mma, ...
+    const int j = warp - kMmaWarp0;
+    if (j < p.n_mma) {
+      bool ok = true;
+      // B descriptors: the slot-0, slice-0 descriptor plus start-address steps
+      // (in 16-byte units; every address stays below 2^18, so the 14-bit
+      // field never carries)
+      const uint64_t bdesc0 = smem_desc(smem_u32(smem + p.b_off), 16 * p.Npad, 128);
+      const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
+      const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
+      const uint32_t dacc = tmem + j * p.dstride;
+      const int step = p.n_mma;  // divides kNS and G
+      int sl = j, g = j, ti = 0;
+      uint32_t rph = 0;
+      for (int c = j; c < total && ok; c += step) {
+        if (g == j && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
+        ok = ok && mbar_wait(&aready[sl], rph);
+        if (!ok) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = tmem + kAColBase + sl * 64;
+          const uint64_t d0 = bdesc0 + sl * slot16;
+          tc_mma_ts(dacc, a0, d0, p.idesc, g >= step ? 1u : 0u);
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint64_t bd = smem_desc(b0 + ks * 32 * p.Npad, 16 * p.Npad, 128);
-          tc_mma_ts(tmem, a0 + ks * 8, bd, p.idesc, (g > 0 || ks > 0) ? 1u : 0u);
+          for (int ks = 1; ks < 8; ++ks) tc_mma_ts(dacc, a0 + ks * 8, d0 + ks * ks16, p.idesc, 1u);
+          tc_commit(&freeb[sl]);
+          if (g + step >= G) tc_commit(dready);
         }
-        tc_commit(&freeb[sl]);
-        if (g == G - 1) tc_commit(dready);
+        __syncwarp();
+        sl += step;
+        if (sl >= kNS) {
+          sl -= kNS;
+          rph ^= 1u;
+        }
+        g += step;
+        if (g >= G) {
+          g -= G;
+          ++ti;
+        }
       }
+      // Drain: no MMA may be in flight when tensor memory is freed.
+      if (lane == 0) tc_commit(drain);
       __syncwarp();
+      if (!mbar_wait(drain, 0)) ok = false;
+      if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
     }
-    // Drain: no MMA may be in flight when tensor memory is freed.
-    if (lane == 0) tc_commit(drain);
-    __syncwarp();
-    if (!mbar_wait(drain, 0)) ok = false;
-    if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
   } else {
     // ---------------- dequant (two warpgroups, alternate groups) + epilogue
     const int wg = warp >> 2;
@@ -346,28 +389,43 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const int m = tile_m0(ti) + r;
       const int half = p.Npad / 2;
       for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 16) {
-        uint32_t v[16];
-        tc_ld16(tmem + lane_base + c0, v);
-        tc_wait_ld();
+        float acc[16];
+        {
+          uint32_t v[16];
+          tc_ld16(tmem + lane_base + c0, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
+        }
+        for (int a = 1; a < p.n_mma; ++a) {
+          uint32_t v[16];
+          tc_ld16(tmem + lane_base + a * p.dstride + c0, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
+        }
         if (m < p.M) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = c0 + j;
-            if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = __uint_as_float(v[j]);
+          for (int i = 0; i < 16; ++i) {
+            const int n = c0 + i;
+            if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i];
           }
         }
       }
       tc_fence_before();
       mbar_arrive(dfree);
     };
+    // this warpgroup's chunks c = wg, wg + 2, ...: slot, round parity, group
+    // and tile advance incrementally (G and kNS are even)
+    int sl = wg, g = wg, ti = 0;
+    uint32_t rph = 0;
     for (int c = wg; c < total && ok; c += 2) {
-      const int sl = c % kNS, ti = c / G, g = c - ti * G;
       if (ti != prev_ti) {
         if (prev_ti >= 0) epilogue(prev_ti);
         prev_ti = ti;
         if (!ok) break;
       }
-      if (!mbar_wait(&full[sl], (c / kNS) & 1)) {
+      if (!mbar_wait(&full[sl], rph)) {
         ok = false;
         break;
       }
@@ -403,6 +461,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       tc_wait_st();
       tc_fence_before();
       mbar_arrive(&aready[sl]);
+      sl += 2;
+      if (sl >= kNS) {
+        sl -= kNS;
+        rph ^= 1u;
+      }
+      g += 2;
+      if (g >= G) {
+        g -= G;
+        ++ti;
+      }
     }
     if (ok && prev_ti >= 0) epilogue(prev_ti);
     if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
@@ -569,6 +637,8 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.sbuf_off = pl.sbuf_off;
     p.sbuf_bytes = pl.sbuf_bytes;
     p.bar_off = pl.bar_off;
+    p.n_mma = npad <= 64 ? 4 : 2;
+    p.dstride = 256 / p.n_mma;
     p.idesc = tc::idesc_f16(tc::kTileM, npad);
     const dim3 g(grid), blk(tc::kThreads);
     switch (a.bits) {
