@@ -7,25 +7,29 @@
 //     already in the shared-memory image the MMA reads (no-swizzle K-major
 //     core matrices), one contiguous block per 128-code group;
 //   * per CTA, one 128-row tile at a time: one producer thread streams each
-//     128-code group through a 4-slot ring -- the tile's 128 code rows in one
-//     2D TMA load (swizzled so the decoders' 16-byte row reads are free of
-//     bank conflicts), the group's x' image in one bulk copy, and at the
-//     tile's first group its scales in one bulk copy -- all completing on the
-//     slot's mbarrier (expected byte count);
-//   * two warpgroups alternate groups: each thread owns one weight row,
-//     decodes its 128 codes into exact fp16 (q - zero) (one LOP3 and one fp16
-//     FMA per pair), multiplies by the group scale (one fp16 multiply per pair:
-//     the weight's only rounding) and stores the row into tensor memory as the
-//     MMA's A operand (tcgen05.st), one TMEM lane per row;
-//   * n_mma MMA warps (4 when the batch block pads to <= 64 columns, else 2)
-//     take the groups round robin; each issues 8 tcgen05.mma (M=128, N, K=16,
-//     A from TMEM, B from shared memory) per group into its own fp32
-//     accumulator in tensor memory and commits their completion to the slot's
-//     mbarrier, which frees the slot for the producer.  A single issuing
+//     128-code group through a ring of 4, 6 or 8 shared-memory slots (as many
+//     as fit) -- the tile's 128 code rows in one 2D TMA load (swizzled so the
+//     decoders' 16-byte row reads are free of bank conflicts), the group's x'
+//     image in one bulk copy, and at the tile's first group its scales in one
+//     bulk copy -- all completing on the slot's mbarrier (expected bytes);
+//   * two warpgroups take the groups in turn (group c to warpgroup c mod 2):
+//     each thread owns one weight row, decodes its 128 codes into exact fp16
+//     (q - zero) (one LOP3 and one fp16 FMA per pair), multiplies by the group
+//     scale (one fp16 multiply per pair: the weight's only rounding) and
+//     stores the row into tensor memory as the MMA's A operand (tcgen05.st),
+//     one TMEM lane per row, in A stage c mod as (as = 4 or 6 stages, so each
+//     warpgroup rotates through 2 or 3 and decodes ahead while the MMAs of its
+//     previous groups run);
+//   * two MMA warps take the groups in the same turn (warp c mod 2); each
+//     issues 8 tcgen05.mma (M=128, N, K=16, A from TMEM, B from shared memory)
+//     per group into its own fp32 accumulator in tensor memory and commits
+//     their completion to the slot's and the A stage's mbarriers.  One issuing
 //     thread sustains only one MMA per ~60-80 cycles whatever N is, so at
-//     batch <= 128 several issuers are what keeps the tensor pipe busy;
-//   * the tile's last commits release the epilogue, which sums the
+//     batch <= 128 a second issuer doubles the tensor-pipe rate;
+//   * the tile's last commits release the epilogue, which sums the two
 //     accumulators (tcgen05.ld) and writes y.
+// Every barrier's consecutive phases are waited for by one agent, in order
+// (ring depths are multiples of two), so phase-parity waits are unambiguous.
 // Waits are bounded (status word on timeout); tensor memory is freed on exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -44,14 +48,27 @@ namespace hq {
 namespace tc {
 
 constexpr int kTileM = 128;
-constexpr int kNS = 4;            // ring slots (and A stages in tensor memory)
-constexpr int kDeqWarps = 8;      // two warpgroups
+constexpr int kNSMax = 8;         // shared-memory ring slots: 4 or 8, as many as fit
+constexpr int kNSMin = 4;
+constexpr int kASMax = 6;         // A stages in tensor memory (64 columns each): 4 or 6
+constexpr int kDeqWG = 2;         // dequant warpgroups (groups round robin)
+constexpr int kDeqWarps = 4 * kDeqWG;
 constexpr int kProducerWarp = kDeqWarps;
 constexpr int kMmaWarp0 = kDeqWarps + 1;
-constexpr int kMmaWarps = 4;      // issuing threads: one thread issues an MMA per ~60-80 cycles
+constexpr int kMmaWarps = 2;      // issuing threads: one thread issues an MMA per ~60-80 cycles
 constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps) * 32;
+// Phase-parity waits are unambiguous only if a barrier's consecutive phases
+// are waited for by the same agent (it cannot wait for round r + 1 before
+// round r completed): every ring depth is a multiple of the dequant
+// warpgroup count, and the A-stage count a multiple of it and of the MMA
+// warp count.
+static_assert(kNSMin % kDeqWG == 0 && kNSMax % kDeqWG == 0 && kASMax % kDeqWG == 0 &&
+                  kMmaWarps == kDeqWG,
+              "ring depths must be multiples of the agent counts");
 constexpr int kTmemCols = 512;
-constexpr int kAColBase = 256;    // A stages at columns 256 + 64 s; accumulators below 256
+// Tensor memory: accumulator j at columns [j Npad, (j + 1) Npad); A stage s at
+// a_base + 64 s, a_base = 2 Npad rounded up to 64; as many stages as fit,
+// rounded down to even (6 for Npad <= 64, 4 for Npad <= 128).
 
 // ---------------------------------------------------------------- tcgen05 wrappers
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -222,8 +239,9 @@ struct TcParams {
   int sbuf_off;    // per-tile scale buffers (two)
   int sbuf_bytes;
   int bar_off;
-  int n_mma;    // MMA warps (accumulators) in use: 2 or 4
-  int dstride;  // tensor-memory columns between accumulators (256 / n_mma >= Npad)
+  int ns;       // shared-memory ring slots (kNSMin..kNSMax)
+  int as;       // A stages in tensor memory (4 or 6)
+  int a_base;   // tensor-memory column of A stage 0
   uint32_t idesc;
   uint32_t add[16];
 };
@@ -238,22 +256,26 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   const int G = p.K / kGroup;
   const int CB = 16 * BITS;  // code bytes of one row in one 128-code group
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
-  uint64_t* freeb = full + kNS;
-  uint64_t* aready = freeb + kNS;
-  uint64_t* dready = aready + kNS;
+  uint64_t* freeb = full + kNSMax;    // slot's MMAs done (producer may refill)
+  uint64_t* aready = freeb + kNSMax;  // A stage written (MMA may read)
+  uint64_t* afree = aready + kASMax;  // A stage's MMAs done (dequant may rewrite)
+  uint64_t* dready = afree + kASMax;
   uint64_t* dfree = dready + 1;
   uint64_t* drain = dfree + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
 
   if (tid == 0) {
-    for (int i = 0; i < kNS; ++i) {
+    for (int i = 0; i < p.ns; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&freeb[i], 1);
-      mbar_init(&aready[i], 128);
     }
-    mbar_init(dready, p.n_mma);
-    mbar_init(dfree, 2 * 128);
-    mbar_init(drain, p.n_mma);
+    for (int i = 0; i < p.as; ++i) {
+      mbar_init(&aready[i], 128);
+      mbar_init(&afree[i], 1);
+    }
+    mbar_init(dready, kMmaWarps);
+    mbar_init(dfree, kDeqWG * 128);
+    mbar_init(drain, kMmaWarps);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
@@ -284,8 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       int rows = min(kTileM, p.M - m0);
       const uint8_t* bsrc = p.img;
       for (int c = 0; c < total; ++c) {
-        // slot reuse: the MMAs of chunk c - kNS (previous round) are done
-        if (c >= kNS && !mbar_wait(&freeb[sl], rph ^ 1u)) {
+        // slot reuse: the MMAs of chunk c - ns (previous round) are done
+        if (c >= p.ns && !mbar_wait(&freeb[sl], rph ^ 1u)) {
           ok = false;
           break;
         }
@@ -301,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
         issued = c + 1;
         bsrc += b_bytes;
-        if (++sl == kNS) {
+        if (++sl == p.ns) {
           sl = 0;
           rph ^= 1u;
         }
@@ -315,16 +337,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       }
       // Drain: the copies of the last slots must have landed before exit (they
       // have on the normal path, where the dequant warps consumed them).
-      for (int c = max(0, issued - kNS); c < issued; ++c) {
-        if (!mbar_wait(&full[c % kNS], (c / kNS) & 1)) ok = false;
+      for (int c = max(0, issued - p.ns); c < issued; ++c) {
+        if (!mbar_wait(&full[c % p.ns], (c / p.ns) & 1)) ok = false;
       }
       if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
     }
     __syncwarp();
   } else if (warp >= kMmaWarp0) {
-    // ---------------- MMA issue: warp j takes chunks j, j + n_mma, ...
+    // ---------------- MMA issue: warp j takes chunks j, j + kMmaWarps, ...
     const int j = warp - kMmaWarp0;
-    if (j < p.n_mma) {
+    {
       bool ok = true;
       // B descriptors: the slot-0, slice-0 descriptor plus start-address steps
       // (in 16-byte units; every address stays below 2^18, so the 14-bit
@@ -332,29 +354,32 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const uint64_t bdesc0 = smem_desc(smem_u32(smem + p.b_off), 16 * p.Npad, 128);
       const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
       const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
-      const uint32_t dacc = tmem + j * p.dstride;
-      const int step = p.n_mma;  // divides kNS and G
-      int sl = j, g = j, ti = 0;
-      uint32_t rph = 0;
+      const uint32_t dacc = tmem + j * p.Npad;
+      const int step = kMmaWarps;  // divides as and G; <= ns
+      int sl = j, st = j, g = j, ti = 0;  // slot (mod ns), A stage (mod as)
+      uint32_t aph = 0;                   // A-stage round parity
       for (int c = j; c < total && ok; c += step) {
         if (g == j && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
-        ok = ok && mbar_wait(&aready[sl], rph);
+        ok = ok && mbar_wait(&aready[st], aph);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t a0 = tmem + kAColBase + sl * 64;
+          const uint32_t a0 = tmem + p.a_base + st * 64;
           const uint64_t d0 = bdesc0 + sl * slot16;
           tc_mma_ts(dacc, a0, d0, p.idesc, g >= step ? 1u : 0u);
 #pragma unroll
           for (int ks = 1; ks < 8; ++ks) tc_mma_ts(dacc, a0 + ks * 8, d0 + ks * ks16, p.idesc, 1u);
           tc_commit(&freeb[sl]);
+          tc_commit(&afree[st]);
           if (g + step >= G) tc_commit(dready);
         }
         __syncwarp();
         sl += step;
-        if (sl >= kNS) {
-          sl -= kNS;
-          rph ^= 1u;
+        if (sl >= p.ns) sl -= p.ns;
+        st += step;
+        if (st >= p.as) {
+          st -= p.as;
+          aph ^= 1u;
         }
         g += step;
         if (g >= G) {
@@ -369,7 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
     }
   } else {
-    // ---------------- dequant (two warpgroups, alternate groups) + epilogue
+    // ---------------- dequant (kDeqWG warpgroups, groups round robin) + epilogue
     const int wg = warp >> 2;
     const int sub = warp & 3;
     const int r = 32 * sub + lane;  // tile row = TMEM lane
@@ -380,6 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     int prev_ti = -1;
     bool ok = true;
     uint4 scache = make_uint4(0, 0, 0, 0);  // this row's scales for 8 groups
+    int sblock = -1;                         // which block of 8 groups scache holds
     auto epilogue = [&](int ti) {
       if (!mbar_wait(dready, ti & 1)) {
         ok = false;
@@ -387,8 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       }
       tc_fence_after();
       const int m = tile_m0(ti) + r;
-      const int half = p.Npad / 2;
-      for (int c0 = wg * half; c0 < (wg + 1) * half; c0 += 16) {
+      // the warpgroups take the 16-column blocks round robin
+      for (int c0 = wg * 16; c0 < p.Npad; c0 += 16 * kDeqWG) {
         float acc[16];
         {
           uint32_t v[16];
@@ -397,9 +423,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
           for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
         }
-        for (int a = 1; a < p.n_mma; ++a) {
+        for (int a = 1; a < kMmaWarps; ++a) {
           uint32_t v[16];
-          tc_ld16(tmem + lane_base + a * p.dstride + c0, v);
+          tc_ld16(tmem + lane_base + a * p.Npad + c0, v);
           tc_wait_ld();
 #pragma unroll
           for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
@@ -415,29 +441,35 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(dfree);
     };
-    // this warpgroup's chunks c = wg, wg + 2, ...: slot, round parity, group
-    // and tile advance incrementally (G and kNS are even)
-    int sl = wg, g = wg, ti = 0;
-    uint32_t rph = 0;
-    for (int c = wg; c < total && ok; c += 2) {
+    // this warpgroup's chunks c = wg, wg + kDeqWG, ...: slot (mod ns), A
+    // stage (mod as), their round parities, group and tile advance
+    // incrementally (kDeqWG divides as and ns; kDeqWG < G).  Every round of
+    // this warpgroup's slots and stages is waited for by this warpgroup alone,
+    // in order, so a parity wait never meets a phase two rounds old.
+    int sl = wg, st = wg, g = wg, ti = 0;
+    uint32_t sph = 0, aph = 0;
+    for (int c = wg; c < total && ok; c += kDeqWG) {
       if (ti != prev_ti) {
         if (prev_ti >= 0) epilogue(prev_ti);
         prev_ti = ti;
+        sblock = -1;  // the new tile's scales are in the other buffer
         if (!ok) break;
       }
-      if (!mbar_wait(&full[sl], rph)) {
+      // the slot's copies have landed, and the A stage's previous MMAs are done
+      if (!mbar_wait(&full[sl], sph) || (c >= p.as && !mbar_wait(&afree[st], aph ^ 1u))) {
         ok = false;
         break;
       }
       const uint4* rowp = reinterpret_cast<const uint4*>(smem + sl * p.slot_bytes + r * CB);
-      if ((g & 7) < 2) {  // first group of this warpgroup in a block of 8
+      if ((g >> 3) != sblock) {  // first group of this warpgroup in a block of 8
+        sblock = g >> 3;
         scache = *reinterpret_cast<const uint4*>(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes +
                                                  r * G * 2 + (g >> 3) * 16);
       }
       const int j = (g >> 1) & 3;
       const uint32_t sw = j == 0 ? scache.x : j == 1 ? scache.y : j == 2 ? scache.z : scache.w;
       const uint32_t s2 = ((g & 1) ? (sw >> 16) : (sw & 0xFFFFu)) * 0x10001u;
-      const uint32_t a0 = tmem + lane_base + kAColBase + sl * 64;
+      const uint32_t a0 = tmem + lane_base + p.a_base + st * 64;
       uint32_t rw[4 * BITS];  // the row's 128 codes, 16-byte loads
 #pragma unroll
       for (int i = 0; i < BITS; ++i) {
@@ -460,13 +492,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       }
       tc_wait_st();
       tc_fence_before();
-      mbar_arrive(&aready[sl]);
-      sl += 2;
-      if (sl >= kNS) {
-        sl -= kNS;
-        rph ^= 1u;
+      mbar_arrive(&aready[st]);
+      sl += kDeqWG;
+      if (sl >= p.ns) {
+        sl -= p.ns;
+        sph ^= 1u;
       }
-      g += 2;
+      st += kDeqWG;
+      if (st >= p.as) {
+        st -= p.as;
+        aph ^= 1u;
+      }
+      g += kDeqWG;
       if (g >= G) {
         g -= G;
         ++ti;
@@ -486,27 +523,42 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host side
 struct TcPlan {
-  int slot = 0, b_off = 0, sbuf_off = 0, sbuf_bytes = 0, bar_off = 0;
+  int ns = 0, slot = 0, b_off = 0, sbuf_off = 0, sbuf_bytes = 0, bar_off = 0;
   size_t smem = 0;
 };
 
 constexpr size_t kMaxSmemTc = 227 * 1024 - 1024;  // dynamic; the base is rounded up to 1 KiB
 constexpr size_t kMinSmemTc = 116 * 1024;         // > half an SM's shared memory
+constexpr size_t kBarBytes = 256;                  // mbarriers and the TMEM address word
 
-static TcPlan tc_plan(int bits, int K, int npad) {
+// Plan with ns ring slots (0 smem when it does not fit).
+static TcPlan tc_plan_ns(int bits, int K, int npad, int ns) {
   TcPlan pl;
   const int G = K / kGroup;
   // slot: [128 code rows, 16*bits bytes each, dense and swizzled][x' image];
   // both sizes are multiples of 1 KiB, so every slot keeps the swizzle atom
+  pl.ns = ns;
   pl.b_off = kTileM * 16 * bits;
   pl.slot = pl.b_off + 256 * npad;
-  pl.sbuf_off = kNS * pl.slot;
+  pl.sbuf_off = ns * pl.slot;
   pl.sbuf_bytes = kTileM * G * 2;
   pl.bar_off = pl.sbuf_off + 2 * pl.sbuf_bytes;
-  pl.smem = static_cast<size_t>(pl.bar_off) + (3 * kNS + 3) * 8 + 16 + 1024;
-  // one CTA per SM: each holds all 512 tensor-memory columns
-  pl.smem = std::max(pl.smem, kMinSmemTc);
+  pl.smem = static_cast<size_t>(pl.bar_off) + kBarBytes + 1024;
+  if (pl.smem > kMaxSmemTc) pl.smem = 0;
   return pl;
+}
+
+// The deepest ring that fits (at least kNSMin slots; smem 0 if none fits).
+static TcPlan tc_plan(int bits, int K, int npad) {
+  TcPlan best = tc_plan_ns(bits, K, npad, kNSMin);
+  for (int ns = kNSMin + kDeqWG; ns <= kNSMax && best.smem != 0; ns += kDeqWG) {
+    const TcPlan pl = tc_plan_ns(bits, K, npad, ns);
+    if (pl.smem == 0) break;
+    best = pl;
+  }
+  // one CTA per SM: each holds all 512 tensor-memory columns
+  if (best.smem != 0) best.smem = std::max(best.smem, kMinSmemTc);
+  return best;
 }
 
 using EncodeTiled = PFN_cuTensorMapEncodeTiled_v12000;
@@ -553,7 +605,7 @@ int tc_col_block(int bits, int K) {
   // scale buffer is refilled only after the MMAs two tiles back are done)
   if (K < 1024 || K > 16384) return 0;
   for (int nb = 128; nb >= 32; nb -= 32) {
-    if (tc::tc_plan(bits, K, nb).smem <= tc::kMaxSmemTc) return nb;
+    if (tc::tc_plan(bits, K, nb).smem != 0) return nb;
   }
   return 0;
 }
@@ -637,8 +689,10 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.sbuf_off = pl.sbuf_off;
     p.sbuf_bytes = pl.sbuf_bytes;
     p.bar_off = pl.bar_off;
-    p.n_mma = npad <= 64 ? 4 : 2;
-    p.dstride = 256 / p.n_mma;
+    p.ns = pl.ns;
+    p.a_base = (tc::kMmaWarps * npad + 63) & ~63;
+    p.as = ((tc::kTmemCols - p.a_base) / 64) & ~1;
+    if (p.as > tc::kASMax) p.as = tc::kASMax;
     p.idesc = tc::idesc_f16(tc::kTileM, npad);
     const dim3 g(grid), blk(tc::kThreads);
     switch (a.bits) {

@@ -70,13 +70,13 @@ def run(d, signs=True):
 
 def tc_blocks(bits, K, N):
     """Expected tensor-core launches: the prep kernel plus one GEMM per batch block."""
-    # mirror of the shared-memory plan: 4 ring slots of [128 code rows][x' image],
-    # two tile scale buffers, barriers, 1 KiB alignment pad; blocks shrink from
-    # 128 columns in steps of 32 until the plan fits
+    # mirror of the shared-memory plan: at least 4 ring slots of [128 code rows]
+    # [x' image], two tile scale buffers, 256 B of barriers, 1 KiB alignment
+    # pad; blocks shrink from 128 columns in steps of 32 until the plan fits
     G = K // 128
     per = 128
     while per >= 32:
-        smem = 4 * (128 * 16 * bits + 256 * per) + 2 * 128 * G * 2 + 15 * 8 + 16 + 1024
+        smem = 4 * (128 * 16 * bits + 256 * per) + 2 * 128 * G * 2 + 256 + 1024
         if smem <= 227 * 1024 - 1024:
             break
         per -= 32
