@@ -262,7 +262,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   uint64_t* dready = afree + kASMax;
   uint64_t* dfree = dready + 1;
   uint64_t* drain = dfree + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sready = drain + 1;  // [2]: a tile's scales landed in buffer ti & 1
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sready + 2);
 
   if (tid == 0) {
     for (int i = 0; i < p.ns; ++i) {
@@ -276,6 +277,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     mbar_init(dready, kMmaWarps);
     mbar_init(dfree, kDeqWG * 128);
     mbar_init(drain, kMmaWarps);
+    mbar_init(&sready[0], 1);
+    mbar_init(&sready[1], 1);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
@@ -312,15 +315,18 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           break;
         }
         uint8_t* base = smem + sl * p.slot_bytes;
+        // the tile's scales, once per tile, on the buffer's own barrier (a
+        // bulk copy's completion shows only on the barrier it signals)
+        if (g == 0) {
+          const uint32_t s_bytes = static_cast<uint32_t>(rows) * G * 2;
+          mbar_arrive_expect_tx(&sready[ti & 1], s_bytes);
+          bulk_g2s(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes,
+                   p.scales + static_cast<size_t>(m0) * G * 2, s_bytes, &sready[ti & 1]);
+        }
         // a TMA tile always delivers the whole box (rows past M read as zero)
-        const uint32_t s_bytes = g == 0 ? static_cast<uint32_t>(rows) * G * 2 : 0u;
-        mbar_arrive_expect_tx(&full[sl], code_bytes + b_bytes + s_bytes);
+        mbar_arrive_expect_tx(&full[sl], code_bytes + b_bytes);
         tma_load_2d(base, &p.qmap, g * CB, m0, &full[sl]);
         bulk_g2s(base + p.b_off, bsrc, b_bytes, &full[sl]);
-        if (g == 0) {
-          bulk_g2s(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes,
-                   p.scales + static_cast<size_t>(m0) * G * 2, s_bytes, &full[sl]);
-        }
         issued = c + 1;
         bsrc += b_bytes;
         if (++sl == p.ns) {
@@ -340,6 +346,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       for (int c = max(0, issued - p.ns); c < issued; ++c) {
         if (!mbar_wait(&full[c % p.ns], (c / p.ns) & 1)) ok = false;
       }
+      if (issued > 0) {
+        const int lt = (issued - 1) / G;  // the last tile whose scales were requested
+        if (!mbar_wait(&sready[lt & 1], (lt >> 1) & 1)) ok = false;
+      }
       if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
     }
     __syncwarp();
@@ -355,12 +365,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
       const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
       const uint32_t dacc = tmem + j * p.Npad;
-      const int step = kMmaWarps;  // divides as and G; <= ns
+      const int step = kMmaWarps;  // divides as, ns and G
       int sl = j, st = j, g = j, ti = 0;  // slot (mod ns), A stage (mod as)
-      uint32_t aph = 0;                   // A-stage round parity
+      uint32_t aph = 0, sph = 0;          // A-stage and slot round parities
       for (int c = j; c < total && ok; c += step) {
         if (g == j && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
         ok = ok && mbar_wait(&aready[st], aph);
+        // B arrived by TMA: observe its barrier here too (already complete)
+        ok = ok && mbar_wait(&full[sl], sph);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -375,7 +387,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         }
         __syncwarp();
         sl += step;
-        if (sl >= p.ns) sl -= p.ns;
+        if (sl >= p.ns) {
+          sl -= p.ns;
+          sph ^= 1u;
+        }
         st += step;
         if (st >= p.as) {
           st -= p.as;
@@ -453,7 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (prev_ti >= 0) epilogue(prev_ti);
         prev_ti = ti;
         sblock = -1;  // the new tile's scales are in the other buffer
-        if (!ok) break;
+        if (!ok || !mbar_wait(&sready[ti & 1], (ti >> 1) & 1)) {
+          ok = false;
+          break;
+        }
       }
       // the slot's copies have landed, and the A stage's previous MMAs are done
       if (!mbar_wait(&full[sl], sph) || (c >= p.as && !mbar_wait(&afree[st], aph ^ 1u))) {
@@ -529,7 +547,7 @@ struct TcPlan {
 
 constexpr size_t kMaxSmemTc = 227 * 1024 - 1024;  // dynamic; the base is rounded up to 1 KiB
 constexpr size_t kMinSmemTc = 116 * 1024;         // > half an SM's shared memory
-constexpr size_t kBarBytes = 256;                  // mbarriers and the TMEM address word
+constexpr size_t kBarBytes = 320;  // 33 mbarriers and the TMEM address word
 
 // Plan with ns ring slots (0 smem when it does not fit).
 static TcPlan tc_plan_ns(int bits, int K, int npad, int ns) {

@@ -62,9 +62,75 @@ struct GemvParams {
   uint32_t U;  // units = n_tiles * G
   uint32_t GW;  // active warps
   int zero;
-  int CH, NS, stride, slot_bytes, zc_off, buf_off, ring_off, bar_off;
-  float inv_sqrt_k;
+  const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, then zc [G][8] fp32
+  int CH, NS, stride, slot_bytes, zc_off, ring_off, bar_off;
 };
+
+// Bytes of the prep output for a batch block of nb columns (16-byte multiple).
+__host__ __device__ constexpr size_t gemv_xs_bytes(int G, int nb) {
+  return static_cast<size_t>(G) * nb * 4 * kXq * 2;
+}
+__host__ __device__ constexpr size_t gemv_xg_bytes(int G, int nb) {
+  return gemv_xs_bytes(G, nb) + static_cast<size_t>(G) * 8 * 4;
+}
+
+// ---------------------------------------------------------------- prep: rotate once per call
+// CTA n rotates activation row n in fp32, rounds x' to fp16, and writes it in
+// the order of the MMA B fragments, each value scaled by the 2^-a of its code
+// field, plus the zero-point term -zero * sum_k x'_k * 2^-24 of each group;
+// CTA 0 also zeroes the zero-point terms of the absent columns (N..7).
+template <int BITS, int LOGK>
+__global__ void __launch_bounds__(kWarps * 32) gemv_prep_kernel(const __half* __restrict__ x,
+                                                                 const int8_t* __restrict__ signs,
+                                                                 uint8_t* __restrict__ xg, int N,
+                                                                 int zero, float inv_sqrt_k) {
+  using FS = FwhtShape<LOGK, 3>;
+  constexpr int K = 1 << LOGK;
+  constexpr int G = K / kGroup;
+  extern __shared__ __align__(128) float buf[];
+  pdl_launch_dependents();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int n = blockIdx.x;
+  const int s = lane >> 2, t = lane & 3;
+  uint16_t* xs = reinterpret_cast<uint16_t*>(xg);
+  float* zc = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
+  // lane (s, t) writes the B-fragment quad of step s for k-quad t
+  int kc[4], ka[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const PairDesc pd = Pairs<BITS>::get(2 * s + (r >> 1));
+    kc[r] = 32 * t + ((r & 1) ? pd.c_hi : pd.c_lo);
+    ka[r] = (r & 1) ? pd.a_hi : pd.a_lo;
+  }
+  pdl_wait();  // x is the previous kernel's output; xg may still be read by it
+  if (n == 0) {
+    for (int i = tid; i < G * (8 - N); i += kWarps * 32) zc[(i / (8 - N)) * 8 + N + i % (8 - N)] = 0.f;
+  }
+  float v[FS::E];
+  if (tid < FS::THREADS) {
+    load_chunk<__half, FS::E>(x + static_cast<size_t>(n) * K + tid * FS::E, v);
+    apply_signs<FS::E>(signs ? signs + tid * FS::E : nullptr, v);
+  }
+  fwht_block<LOGK, 3>(v, buf);
+  for (int gg = warp; gg < G; gg += kWarps) {
+    uint16_t hv[4];
+    float part = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + kc[r])] * inv_sqrt_k));
+      const __half b = __float2half_rn(xv * __int_as_float((127 - ka[r]) << 23));
+      hv[r] = __half_as_ushort(b);
+      part += __half2float(b) * __int_as_float((127 + ka[r]) << 23);
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+    uint2 pk;
+    pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
+    pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
+    *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * N + n) * 4 + t) * kXq + s * 4) = pk;
+    if (lane == 0) zc[gg * 8 + n] = -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
+  }
+}
 
 __device__ __forceinline__ uint32_t unit_begin(uint32_t gw, uint32_t U, uint32_t GW) {
   return static_cast<uint32_t>((static_cast<uint64_t>(gw) * U) / GW);
@@ -76,7 +142,6 @@ __device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t U, uint32_t 
 
 template <int BITS, int LOGK>
 __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_constant__ GemvParams p) {
-  using FS = FwhtShape<LOGK, 3>;
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
   constexpr int GB = 16 * BITS;  // bytes of one group of one row
@@ -91,7 +156,6 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   float* zc = reinterpret_cast<float*>(smem + p.zc_off);
-  float* buf = reinterpret_cast<float*>(smem + p.buf_off);
   uint8_t* ring = smem + p.ring_off + warp * p.NS * p.slot_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off) + warp * p.NS;
 
@@ -150,52 +214,19 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
   };
   for (int s = 0; s < p.NS && ui < u1; ++s) issue(s);
 
-  // ---- rotate the activations (depends on the previous kernel)
+  // ---- the rotated activations and zero-point terms (from the prep kernel)
   pdl_wait();
   {
-    // lane (s, t) writes the B-fragment quad of step s for k-quad t
-    const int s = lane >> 2;
-    int kc[4], ka[4];
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const PairDesc pd = Pairs<BITS>::get(2 * s + (r >> 1));
-      kc[r] = 32 * t + ((r & 1) ? pd.c_hi : pd.c_lo);
-      ka[r] = (r & 1) ? pd.a_hi : pd.a_lo;
+    const int xs_bytes = static_cast<int>(gemv_xs_bytes(G, p.N));
+    for (int i = tid * 16; i < xs_bytes; i += kWarps * 32 * 16) {
+      cp_async16(smem + i, p.xg + i, 16);
     }
-    // zero-point terms of absent batch columns and the B block of lanes
-    // without a column stay zero
-    for (int i = tid; i < G * 8; i += kWarps * 32) zc[i] = 0.f;
-    if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;
+    for (int i = tid * 16; i < G * 8 * 4; i += kWarps * 32 * 16) {
+      cp_async16(smem + p.zc_off + i, p.xg + xs_bytes + i, 16);
+    }
+    if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;  // zero B block
+    asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
-    for (int n = 0; n < p.N; ++n) {
-      float v[FS::E];
-      if (tid < FS::THREADS) {
-        load_chunk<__half, FS::E>(p.x + static_cast<size_t>(n) * K + tid * FS::E, v);
-        apply_signs<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr, v);
-      }
-      fwht_block<LOGK, 3>(v, buf);
-      for (int gg = warp; gg < G; gg += kWarps) {
-        uint16_t hv[4];
-        float part = 0.f;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + kc[r])] *
-                                                        p.inv_sqrt_k));
-          const __half b = __float2half_rn(xv * __int_as_float((127 - ka[r]) << 23));
-          hv[r] = __half_as_ushort(b);
-          part += __half2float(b) * __int_as_float((127 + ka[r]) << 23);
-        }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-        uint2 pk;
-        pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
-        pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
-        *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * p.N + n) * 4 + t) * kXq + s * 4) =
-            pk;
-        if (lane == 0) zc[gg * 8 + n] = -static_cast<float>(p.zero) * part * 5.9604644775390625e-8f;
-      }
-      __syncthreads();
-    }
   }
 
   // ---- consumer: decode + MMA over the warp's units
@@ -362,7 +393,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host planning
 struct GemvPlan {
-  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, buf_off = 0, ring_off = 0, bar_off = 0;
+  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, ring_off = 0, bar_off = 0;
   size_t smem = 0;
 };
 
@@ -370,23 +401,24 @@ constexpr size_t kMaxSmem = 227 * 1024;
 // Budget that lets two CTAs (of consecutive launches) share an SM, so that a
 // launch's weight stream overlaps its predecessor's compute and tail.
 constexpr size_t kPairSmem = 110 * 1024;
+constexpr int kMaxNS = 8;
 
+// The ring with the most groups in flight per warp (CH x NS) that fits the
+// budget; among equal products, more and smaller slots (finer refills).
 static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
   GemvPlan best;
   const int G = K / kGroup;
-  const size_t xs = static_cast<size_t>(nb) * G * 4 * kXq * 2;
+  const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
-  const size_t buf_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
-  const size_t buf = static_cast<size_t>(K + K / 32) * 4;
-  const size_t ring_off = (buf_off + buf + 127) & ~static_cast<size_t>(127);
-  for (int CH : {8, 4, 2, 1}) {
+  const size_t ring_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
+  for (int CH : {1, 2, 4, 8}) {
     const int ch = std::min(CH, G);
     const int row = ch * 16 * bits;
     const int pad_w = ((bank_target_words(bits) - row / 4) % 32 + 32) % 32;
     const int stride = row + 4 * pad_w;
     const int sbytes = G >= 8 ? kRows * 32 : ((kRows * G * 2 + 15) & ~15);
     const int slot = kRows * stride + sbytes;
-    for (int NS : {4, 3, 2}) {
+    for (int NS = kMaxNS; NS >= 2; --NS) {
       const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * NS * slot;
       const size_t smem = bar_off + static_cast<size_t>(kWarps) * NS * 8;
       if (smem > budget) continue;
@@ -396,7 +428,6 @@ static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
         best.stride = stride;
         best.slot_bytes = slot;
         best.zc_off = static_cast<int>(zc_off);
-        best.buf_off = static_cast<int>(buf_off);
         best.ring_off = static_cast<int>(ring_off);
         best.bar_off = static_cast<int>(bar_off);
         best.smem = smem;
@@ -447,9 +478,43 @@ static cudaError_t gemv_launch_b(int K, GemvParams& p, size_t smem, unsigned gri
   }
 }
 
+size_t gemv_scratch_bytes(int K, int nb) { return gemv_xg_bytes(K / kGroup, nb); }
+
+template <int BITS>
+static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
+  const dim3 g(a.N), b(kWarps * 32);
+  const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(K)));
+  const __half* x = reinterpret_cast<const __half*>(a.x);
+  uint8_t* xg = static_cast<uint8_t*>(a.xg);
+#define HQ_PREP(LK)                                                                            \
+  launch_pdl(gemv_prep_kernel<BITS, LK>, g, b, FwhtShape<LK, 3>::SMEM_FLOATS * sizeof(float), st, \
+             true, x, a.signs, xg, a.N, a.zero, inv)
+  switch (K) {
+    case 128: return HQ_PREP(7);
+    case 256: return HQ_PREP(8);
+    case 512: return HQ_PREP(9);
+    case 1024: return HQ_PREP(10);
+    case 2048: return HQ_PREP(11);
+    case 4096: return HQ_PREP(12);
+    case 8192: return HQ_PREP(13);
+    case 16384: return HQ_PREP(14);
+    default: return cudaErrorInvalidValue;
+  }
+#undef HQ_PREP
+}
+
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   const GemvPlan pl = gemv_plan(a.bits, a.K, a.N);
   if (pl.smem == 0) return cudaErrorInvalidValue;
+  cudaError_t e;
+  switch (a.bits) {
+    case 2: e = gemv_prep_b<2>(a.K, a, st); break;
+    case 3: e = gemv_prep_b<3>(a.K, a, st); break;
+    case 4: e = gemv_prep_b<4>(a.K, a, st); break;
+    case 8: e = gemv_prep_b<8>(a.K, a, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
   const int G = a.K / kGroup;
   const uint32_t n_tiles = static_cast<uint32_t>((a.M + kRows - 1) / kRows);
   const uint32_t U = n_tiles * static_cast<uint32_t>(G);
@@ -474,11 +539,10 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.stride = pl.stride;
   p.slot_bytes = pl.slot_bytes;
   p.zc_off = pl.zc_off;
-  p.buf_off = pl.buf_off;
+  p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = a.zero;
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;
-  p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   switch (a.bits) {
     case 2: return gemv_launch_b<2>(a.K, p, pl.smem, grid, st);
     case 3: return gemv_launch_b<3>(a.K, p, pl.smem, grid, st);

@@ -1,6 +1,7 @@
 // hq_api.cu -- the C ABI of libhq: argument validation, workspace layout and
 // kernel dispatch.  Every check happens on the host before any launch; no
 // entry point allocates or frees memory.
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 
@@ -58,8 +59,9 @@ static bool use_tc(const hq_weight* w, int batch) {
 }
 
 // hq_linear workspace: [status 256 B][GEMV partial tiles][tile counters]
-// [tensor-core path only: rotated activation images, batch rounded up to whole
-// batch blocks, x K fp16].
+// [activations: on the tensor-core path the rotated activation images (batch
+// rounded up to whole batch blocks, x K fp16); on the GEMV path the rotated
+// activations of one batch block in fragment order (blocks run in turn)].
 struct LinearWs {
   uint32_t* status;
   void* part;
@@ -72,7 +74,10 @@ static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
   const size_t part_bytes = align256(static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16);
   const size_t cnt_bytes = align256(static_cast<size_t>((w->M + 15) / 16) * 4);
-  const size_t xp_bytes = use_tc(w, batch) ? align256(tc_xp_bytes(w->bits, w->K, batch)) : 0;
+  const int nb = gemv_col_block(w->bits, w->K);
+  const size_t xp_bytes = use_tc(w, batch)
+                              ? align256(tc_xp_bytes(w->bits, w->K, batch))
+                              : align256(gemv_scratch_bytes(w->K, nb > 0 ? std::min(nb, std::max(batch, 1)) : 1));
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
   l.part = b + kStatusBytes;
@@ -135,7 +140,7 @@ int hq_linear_launches(const hq_weight* w, int batch) {
   if (use_tc(w, batch)) return tc_launches(w->bits, w->K, batch);
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return 0;
-  return (batch + nb - 1) / nb;
+  return 2 * ((batch + nb - 1) / nb);  // prep + GEMV per batch block
 }
 
 hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, void* workspace,
@@ -186,6 +191,7 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     a.status = l.status;
     a.part = l.part;
     a.cnt = l.cnt;
+    a.xg = l.xp;
     const cudaError_t e = launch_gemv(a, st);
     if (e != cudaSuccess) return from_cuda(e);
   }

@@ -34,13 +34,17 @@ struct GemvArgs {
   uint32_t* status;
   void* part;     // gemv_max_warps() * 1 KiB of partial tiles
   uint32_t* cnt;  // ceil(M/16) counters, zero between launches
+  void* xg;       // gemv_scratch_bytes(K, N) bytes, 16-byte aligned: prep output
 };
 
 // Shared memory the GEMV needs for a batch block of nb <= 8 rows (0 if no
 // ring configuration fits in one CTA).
 size_t gemv_smem_bytes(int bits, int K, int nb);
+// Scratch for the rotated activations of one GEMV launch of nb <= 8 columns.
+size_t gemv_scratch_bytes(int K, int nb);
 // Upper bound on the GEMV's warps (8 per SM of the current device).
 int gemv_max_warps();
+// Two launches: the rotation (prep) and the GEMV.
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 
 // Tensor-core path (tcgen05) for larger batches.

@@ -27,13 +27,15 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t{2} << 20;  // 2 MiB in total
 constexpr size_t kStatus = 256;                    // status word, kept zero
+constexpr size_t kXgBytes = size_t{340} << 10;     // rotated activations of one batch block
 constexpr size_t kPartBytes = size_t{1280} << 10;  // partial tiles: up to 1280 GEMV warps
-constexpr size_t kCntBytes = kScratchBytes - kStatus - kPartBytes;  // tile counters
+constexpr size_t kCntBytes = kScratchBytes - kStatus - kXgBytes - kPartBytes;  // tile counters
 // Largest output-row count: one 4-byte counter per 16 rows.
 constexpr long kMaxRows = static_cast<long>(kCntBytes / 4) * 16;
 
-// The scratch: [status][tile counters][split-tile partials].  Static storage
-// starts zeroed; each call clears the status word and the counters it uses.
+// The scratch: [status][tile counters][rotated activations][split-tile
+// partials].  Static storage starts zeroed; each call clears the status word
+// and the counters it uses.
 __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -90,6 +92,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     if (gemv_smem_bytes(w->bits, w->K, b) != 0) nb = b;
   }
   if (nb == 0) return HQ_ERR_UNSUPPORTED;
+  if (gemv_scratch_bytes(w->K, nb) > kXgBytes) return HQ_ERR_WORKSPACE;
 
   uint8_t* scratch = nullptr;
   if (scratch_on_current_device(&scratch) != cudaSuccess) {
@@ -117,7 +120,8 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     a.ldy = w->M;
     a.status = reinterpret_cast<uint32_t*>(scratch);
     a.cnt = reinterpret_cast<uint32_t*>(scratch + kStatus);
-    a.part = scratch + kStatus + kCntBytes;
+    a.xg = scratch + kStatus + kCntBytes;
+    a.part = scratch + kStatus + kCntBytes + kXgBytes;
     if (launch_gemv(a, st) != cudaSuccess) {
       (void)cudaGetLastError();
       return HQ_ERR_CUDA;

@@ -71,12 +71,12 @@ def run(d, signs=True):
 def tc_blocks(bits, K, N):
     """Expected tensor-core launches: the prep kernel plus one GEMM per batch block."""
     # mirror of the shared-memory plan: at least 4 ring slots of [128 code rows]
-    # [x' image], two tile scale buffers, 256 B of barriers, 1 KiB alignment
+    # [x' image], two tile scale buffers, 320 B of barriers, 1 KiB alignment
     # pad; blocks shrink from 128 columns in steps of 32 until the plan fits
     G = K // 128
     per = 128
     while per >= 32:
-        smem = 4 * (128 * 16 * bits + 256 * per) + 2 * 128 * G * 2 + 256 + 1024
+        smem = 4 * (128 * 16 * bits + 256 * per) + 2 * 128 * G * 2 + 320 + 1024
         if smem <= 227 * 1024 - 1024:
             break
         per -= 32
@@ -154,3 +154,27 @@ def test_tc_workspace_too_small_is_rejected():
     ws = torch.zeros(small, dtype=torch.uint8, device="cuda")
     with pytest.raises(HqError):
         hq_linear(q, s, g, dev(d["x"]), bits, d["zero"], workspace=ws)
+
+
+@pytest.mark.parametrize("bits,M,K,N", [(3, 8192, 2048, 32), (2, 8192, 8192, 32), (8, 4096, 4096, 64),
+                                        (4, 8192, 1024, 128)])
+def test_tc_every_output_finite_over_repeated_calls(bits, M, K, N):
+    """Many tiles, every call on a fresh zeroed workspace: each tile's scales must
+    have landed before any warpgroup reads them (a stale scale shows as a
+    non-finite or wrong row), on every call."""
+    from bit_hadamard_rotated_b200 import hq_linear, hq_linear_workspace_size
+    d = synth.linear(M, K, bits, N, seed=17 + bits)
+    q, s, g, w = weight(d)
+    x = dev(d["x"])
+    rng = np.random.default_rng(M + K)
+    rows = sorted(set(rng.choice(M, 12, replace=False).tolist()) | {0, M - 1})
+    want = {}
+    for m in rows:
+        want[m] = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"],
+                                m_begin=m, m_end=m + 1)
+    for _ in range(4):
+        ws = torch.zeros(hq_linear_workspace_size(w, N), dtype=torch.uint8, device="cuda")
+        y = hq_linear(q, s, g, x, bits, d["zero"], workspace=ws).cpu().numpy()
+        assert np.all(np.isfinite(y))
+        for m in rows:
+            assert_within(y[:, m], want[m][0][:, m], want[m][1][:, m], what=f"row {m}")
