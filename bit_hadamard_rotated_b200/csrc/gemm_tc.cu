@@ -685,7 +685,7 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
   e = tc::code_map(&qmap, a.q, a.bits, a.M, a.K);
   if (e != cudaSuccess) return e;
   const int n_tiles = (a.M + tc::kTileM - 1) / tc::kTileM;
-  const unsigned grid = static_cast<unsigned>(std::min(n_tiles, gemv_max_warps() / 8));
+  const unsigned grid = static_cast<unsigned>(std::min(n_tiles, sm_count()));
   for (int b = 0, n0 = 0; n0 < a.N; ++b, n0 += nb) {
     const int nk = std::min(nb, a.N - n0);
     const int npad = (nk + 31) & ~31;

@@ -41,7 +41,7 @@
 
 namespace hq {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 constexpr int kRows = 16;
 // halves per (group, column, k-quad) block of B fragments: 8 steps x 4, padded
 // to 80 bytes so the 16-byte loads of 8 lanes hit distinct banks
@@ -56,14 +56,13 @@ struct GemvParams {
   const int8_t* signs;
   float* y;
   uint32_t* status;
-  float4* part;   // [GWmax][2][32] partial tiles
+  float4* part;   // [#CTAs][2][32] partial tiles of tiles shared between CTAs
   uint32_t* cnt;  // [n_tiles] arrival counters, zero between launches
   int M, N, ldy;
   uint32_t U;  // units = n_tiles * G
-  uint32_t GW;  // active warps
   int zero;
   const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, then zc [G][8] fp32
-  int CH, NS, stride, slot_bytes, zc_off, ring_off, bar_off;
+  int CH, NS, stride, slot_bytes, zc_off, sp_off, ring_off, bar_off;
 };
 
 // Bytes of the prep output for a batch block of nb columns (16-byte multiple).
@@ -132,26 +131,30 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_prep_kernel(const __half* __
   }
 }
 
-__device__ __forceinline__ uint32_t unit_begin(uint32_t gw, uint32_t U, uint32_t GW) {
-  return static_cast<uint32_t>((static_cast<uint64_t>(gw) * U) / GW);
+// Splitting U units into n contiguous ranges: range i is [unit_begin(i), unit_begin(i + 1)).
+__device__ __forceinline__ uint32_t unit_begin(uint32_t i, uint32_t U, uint32_t n) {
+  return static_cast<uint32_t>((static_cast<uint64_t>(i) * U) / n);
 }
-// Warp whose range contains unit u.
-__device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t U, uint32_t GW) {
-  return static_cast<uint32_t>((static_cast<uint64_t>(u) * GW + GW - 1) / U);
+// The range that contains unit u (the last of several starting at the same
+// unit: the earlier ones are empty).
+__device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t U, uint32_t n) {
+  return static_cast<uint32_t>((static_cast<uint64_t>(u) * n + n - 1) / U);
 }
 
 template <int BITS, int LOGK>
-__global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_constant__ GemvParams p) {
+__global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
   constexpr int GB = 16 * BITS;  // bytes of one group of one row
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  const uint32_t gw = blockIdx.x * kWarps + warp;
-  const bool active = gw < p.GW;
-  const uint32_t u0 = active ? unit_begin(gw, p.U, p.GW) : 0u;
-  const uint32_t u1 = active ? unit_begin(gw + 1, p.U, p.GW) : 0u;
+  // the CTA owns units [cb, ce); its warps split them into contiguous ranges
+  const uint32_t GC = gridDim.x;
+  const uint32_t cb = unit_begin(blockIdx.x, p.U, GC), ce = unit_begin(blockIdx.x + 1, p.U, GC);
+  const uint32_t cl = ce - cb;
+  const uint32_t u0 = cb + unit_begin(warp, cl, kWarps);
+  const uint32_t u1 = cb + unit_begin(warp + 1, cl, kWarps);
   const int row_words = K * BITS / 32;
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
@@ -231,8 +234,10 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
 
   // ---- consumer: decode + MMA over the warp's units
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float head[4] = {0.f, 0.f, 0.f, 0.f};  // partial sums of a first tile shared with other warps
-  int head_tile = -1;
+  // Tiles this warp covers only in part: its first (0) and last (1); their
+  // partial sums go to shared-memory slot sp[warp][which] (scaled by 2^24).
+  int ptile0 = -1, ptile1 = -1;
+  float4* sp = reinterpret_cast<float4*>(smem + p.sp_off);
   int tile_start = -1;
   int consumed = 0;
   bool ok = true;
@@ -247,34 +252,8 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
   const uint32_t first_tile = u0 / G;
   uint32_t uc = u0;
 
-  // Partial sums of tiles shared with other warps: each contributor publishes
-  // its partial, one fence orders them before the arrival counters, and the
-  // last arrival at a tile adds all contributors' partials in warp order and
-  // stores y.  A warp has at most two shared tiles (the first and the last
-  // of its range); both are exchanged together at the end of the range.
-  auto publish = [&](uint32_t tile, const float (&v)[4]) {
-    const int which = (tile == first_tile) ? 0 : 1;
-    p.part[(static_cast<size_t>(gw) * 2 + which) * 32 + lane] =
-        make_float4(v[0] * kUnit, v[1] * kUnit, v[2] * kUnit, v[3] * kUnit);
-  };
-  auto complete = [&](uint32_t tile) {
-    uint32_t old = 0;
-    if (lane == 0) old = atomicAdd(&p.cnt[tile], 1u);
-    old = __shfl_sync(0xffffffffu, old, 0);
-    const uint32_t gwf = unit_owner(tile * G, p.U, p.GW);
-    const uint32_t gwl = unit_owner(tile * G + G - 1, p.U, p.GW);
-    if (old != gwl - gwf) return;
-    __threadfence();
-    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (uint32_t c = gwf; c <= gwl; ++c) {
-      const int wc = (tile == unit_begin(c, p.U, p.GW) / G) ? 0 : 1;
-      const float4 q4 = __ldcg(&p.part[(static_cast<size_t>(c) * 2 + wc) * 32 + lane]);
-      o.x += q4.x;
-      o.y += q4.y;
-      o.z += q4.z;
-      o.w += q4.w;
-    }
-    if (lane == 0) p.cnt[tile] = 0u;
+  const uint32_t cta_first_tile = cb / G;
+  auto store_tile = [&](uint32_t tile, const float4& o) {
     const int m0 = tile * kRows;
     const int rv = min(kRows, M - m0);
     if (g < rv) {
@@ -286,7 +265,35 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
       if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g + 8] = o.w;
     }
   };
-  int tail_tile = -1;
+  // A tile shared with other CTAs: this CTA's sum is published, one fence
+  // orders it before the tile's arrival counter, and the last CTA to arrive
+  // adds every CTA's sum in CTA order (deterministic, no waiting) and stores.
+  auto exchange = [&](uint32_t tile, const float4& o) {
+    const int which = (tile == cta_first_tile) ? 0 : 1;
+    p.part[(static_cast<size_t>(blockIdx.x) * 2 + which) * 32 + lane] = o;
+    __syncwarp();
+    uint32_t old = 0;
+    if (lane == 0) {
+      __threadfence();
+      old = atomicAdd(&p.cnt[tile], 1u);
+    }
+    old = __shfl_sync(0xffffffffu, old, 0);
+    const uint32_t cf = unit_owner(tile * G, p.U, GC);
+    const uint32_t cz = unit_owner(tile * G + G - 1, p.U, GC);
+    if (old != cz - cf) return;
+    __threadfence();
+    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (uint32_t c = cf; c <= cz; ++c) {
+      const int wc = (tile == unit_begin(c, p.U, GC) / G) ? 0 : 1;
+      const float4 q4 = __ldcg(&p.part[(static_cast<size_t>(c) * 2 + wc) * 32 + lane]);
+      s4.x += q4.x;
+      s4.y += q4.y;
+      s4.z += q4.z;
+      s4.w += q4.w;
+    }
+    if (lane == 0) p.cnt[tile] = 0u;
+    store_tile(tile, s4);
+  };
 
   while (uc < u1) {
     const uint32_t tile = uc / G, g0 = uc % G;
@@ -351,38 +358,52 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
     if (g0 + len == G || uc >= u1) {
       // ---- this warp's part of the tile is done
       const bool full = tile_start == 0 && g0 + len == G;
+      const float4 o = make_float4(acc[0] * kUnit, acc[1] * kUnit, acc[2] * kUnit, acc[3] * kUnit);
       if (full) {
-        const int m0 = tile * kRows;
-        const int rv = min(kRows, M - m0);
-        if (g < rv) {
-          if (n0) p.y[static_cast<size_t>(2 * t) * ldy + m0 + g] = acc[0] * kUnit;
-          if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g] = acc[1] * kUnit;
-        }
-        if (g + 8 < rv) {
-          if (n0) p.y[static_cast<size_t>(2 * t) * ldy + m0 + g + 8] = acc[2] * kUnit;
-          if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g + 8] = acc[3] * kUnit;
-        }
-      } else if (tile == first_tile && uc < u1) {
-        head[0] = acc[0];  // shared first tile: exchange at the end of the range
-        head[1] = acc[1];
-        head[2] = acc[2];
-        head[3] = acc[3];
-        head_tile = static_cast<int>(tile);
+        store_tile(tile, o);
       } else {
-        publish(tile, acc);  // shared last tile (the range ends here)
-        tail_tile = static_cast<int>(tile);
+        const int which = (tile == first_tile) ? 0 : 1;
+        sp[(warp * 2 + which) * 32 + lane] = o;
+        if (which == 0) {
+          ptile0 = static_cast<int>(tile);
+        } else {
+          ptile1 = static_cast<int>(tile);
+        }
       }
       acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
       tile_start = -1;
     }
   }
-  if (ok && (head_tile >= 0 || tail_tile >= 0)) {
-    if (head_tile >= 0) publish(static_cast<uint32_t>(head_tile), head);
-    __syncwarp();
-    if (lane == 0) __threadfence();
-    __syncwarp();
-    if (head_tile >= 0) complete(static_cast<uint32_t>(head_tile));
-    if (tail_tile >= 0) complete(static_cast<uint32_t>(tail_tile));
+  // ---- tiles split between warps: the first contributing warp of the CTA
+  // adds the CTA's partials in warp order (shared memory), then stores the
+  // tile, or exchanges it with the other CTAs that share it
+  __syncthreads();
+  if (ok) {
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const int tl = which == 0 ? ptile0 : ptile1;
+      if (tl < 0 || (which == 1 && tl == ptile0)) continue;
+      const uint32_t tile = static_cast<uint32_t>(tl);
+      const uint32_t tf = max(tile * G, cb), tz = min(tile * G + G, ce) - 1;
+      if (unit_owner(tf - cb, cl, kWarps) != static_cast<uint32_t>(warp)) continue;
+      const uint32_t wz = unit_owner(tz - cb, cl, kWarps);
+      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (uint32_t w = warp; w <= wz; ++w) {
+        const uint32_t wb = cb + unit_begin(w, cl, kWarps);
+        if (wb == cb + unit_begin(w + 1, cl, kWarps)) continue;  // empty range
+        const int ww = (tile == wb / G) ? 0 : 1;
+        const float4 q4 = sp[(w * 2 + ww) * 32 + lane];
+        o.x += q4.x;
+        o.y += q4.y;
+        o.z += q4.z;
+        o.w += q4.w;
+      }
+      if (tile * G >= cb && tile * G + G <= ce) {
+        store_tile(tile, o);
+      } else {
+        exchange(tile, o);
+      }
+    }
   }
   if (!ok) {
     if (lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
@@ -393,15 +414,15 @@ __global__ void __launch_bounds__(kWarps * 32, 2) gemv_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host planning
 struct GemvPlan {
-  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, ring_off = 0, bar_off = 0;
+  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, sp_off = 0, ring_off = 0, bar_off = 0;
   size_t smem = 0;
 };
 
+// One 16-warp CTA per SM (its registers fill the SM) with all of the
+// shared memory: the deeper each warp's ring, the more weight bytes in flight.
 constexpr size_t kMaxSmem = 227 * 1024;
-// Budget that lets two CTAs (of consecutive launches) share an SM, so that a
-// launch's weight stream overlaps its predecessor's compute and tail.
-constexpr size_t kPairSmem = 110 * 1024;
 constexpr int kMaxNS = 8;
+constexpr size_t kSpBytes = static_cast<size_t>(kWarps) * 2 * 32 * 16;  // partial-tile slots
 
 // The ring with the most groups in flight per warp (CH x NS) that fits the
 // budget; among equal products, more and smaller slots (finer refills).
@@ -410,7 +431,8 @@ static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
-  const size_t ring_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
+  const size_t sp_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
+  const size_t ring_off = sp_off + kSpBytes;
   for (int CH : {1, 2, 4, 8}) {
     const int ch = std::min(CH, G);
     const int row = ch * 16 * bits;
@@ -428,6 +450,7 @@ static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
         best.stride = stride;
         best.slot_bytes = slot;
         best.zc_off = static_cast<int>(zc_off);
+        best.sp_off = static_cast<int>(sp_off);
         best.ring_off = static_cast<int>(ring_off);
         best.bar_off = static_cast<int>(bar_off);
         best.smem = smem;
@@ -438,15 +461,11 @@ static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
   return best;
 }
 
-static GemvPlan gemv_plan(int bits, int K, int nb) {
-  GemvPlan pl = gemv_plan_budget(bits, K, nb, kPairSmem);
-  if (pl.smem == 0) pl = gemv_plan_budget(bits, K, nb, kMaxSmem);
-  return pl;
-}
+static GemvPlan gemv_plan(int bits, int K, int nb) { return gemv_plan_budget(bits, K, nb, kMaxSmem); }
 
 size_t gemv_smem_bytes(int bits, int K, int nb) { return gemv_plan(bits, K, nb).smem; }
 
-int gemv_max_warps() {
+int sm_count() {
   static int sms = 0;
   if (sms == 0) {
     int dev = 0, v = 0;
@@ -455,11 +474,13 @@ int gemv_max_warps() {
       sms = v;
     } else {
       (void)cudaGetLastError();
-      return 148 * kWarps;
+      return 148;
     }
   }
-  return sms * kWarps;
+  return sms;
 }
+
+size_t gemv_part_bytes() { return static_cast<size_t>(sm_count()) * 2 * 32 * 16; }
 
 template <int BITS>
 static cudaError_t gemv_launch_b(int K, GemvParams& p, size_t smem, unsigned grid,
@@ -518,8 +539,8 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   const int G = a.K / kGroup;
   const uint32_t n_tiles = static_cast<uint32_t>((a.M + kRows - 1) / kRows);
   const uint32_t U = n_tiles * static_cast<uint32_t>(G);
-  const int max_warps = gemv_max_warps();
-  const uint32_t grid = std::min<uint32_t>(max_warps / kWarps, (U + kWarps - 1) / kWarps);
+  // one CTA per SM, at most one per kWarps units (so every CTA has units)
+  const uint32_t grid = std::min<uint32_t>(static_cast<uint32_t>(sm_count()), (U + kWarps - 1) / kWarps);
   GemvParams p{};
   p.q = a.q;
   p.scales = a.scales;
@@ -533,12 +554,12 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.N = a.N;
   p.ldy = a.ldy;
   p.U = U;
-  p.GW = std::min<uint32_t>(grid * kWarps, U);
   p.CH = pl.CH;
   p.NS = pl.NS;
   p.stride = pl.stride;
   p.slot_bytes = pl.slot_bytes;
   p.zc_off = pl.zc_off;
+  p.sp_off = pl.sp_off;
   p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = a.zero;
   p.ring_off = pl.ring_off;

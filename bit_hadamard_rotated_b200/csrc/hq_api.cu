@@ -72,7 +72,7 @@ struct LinearWs {
 
 static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
-  const size_t part_bytes = align256(static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16);
+  const size_t part_bytes = align256(gemv_part_bytes());
   const size_t cnt_bytes = align256(static_cast<size_t>((w->M + 15) / 16) * 4);
   const int nb = gemv_col_block(w->bits, w->K);
   const size_t xp_bytes = use_tc(w, batch)

@@ -32,7 +32,7 @@ struct GemvArgs {
   float* y;             // [N][M] block of outputs, row stride ldy
   int ldy;
   uint32_t* status;
-  void* part;     // gemv_max_warps() * 1 KiB of partial tiles
+  void* part;     // gemv_part_bytes(): partial tiles shared between CTAs
   uint32_t* cnt;  // ceil(M/16) counters, zero between launches
   void* xg;       // gemv_scratch_bytes(K, N) bytes, 16-byte aligned: prep output
 };
@@ -42,8 +42,10 @@ struct GemvArgs {
 size_t gemv_smem_bytes(int bits, int K, int nb);
 // Scratch for the rotated activations of one GEMV launch of nb <= 8 columns.
 size_t gemv_scratch_bytes(int K, int nb);
-// Upper bound on the GEMV's warps (8 per SM of the current device).
-int gemv_max_warps();
+// Streaming multiprocessors of the current device (148 if the query fails).
+int sm_count();
+// Bytes of the GEMV's cross-CTA partial-tile buffer.
+size_t gemv_part_bytes();
 // Two launches: the rotation (prep) and the GEMV.
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 

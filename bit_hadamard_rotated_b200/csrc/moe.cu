@@ -600,7 +600,7 @@ static cudaError_t moe_launch_rot_h(int inter, const hq_expert* ex, const int32_
 #undef HQ_ROTH
 }
 
-static int moe_grid() { return gemv_max_warps() / 8; }  // one CTA per SM
+static int moe_grid() { return sm_count(); }  // one CTA per SM
 
 }  // namespace hq
 

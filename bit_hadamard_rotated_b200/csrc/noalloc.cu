@@ -28,7 +28,7 @@ namespace {
 constexpr size_t kScratchBytes = size_t{2} << 20;  // 2 MiB in total
 constexpr size_t kStatus = 256;                    // status word, kept zero
 constexpr size_t kXgBytes = size_t{340} << 10;     // rotated activations of one batch block
-constexpr size_t kPartBytes = size_t{1280} << 10;  // partial tiles: up to 1280 GEMV warps
+constexpr size_t kPartBytes = size_t{256} << 10;   // partial tiles shared between CTAs: up to 256 SMs
 constexpr size_t kCntBytes = kScratchBytes - kStatus - kXgBytes - kPartBytes;  // tile counters
 // Largest output-row count: one 4-byte counter per 16 rows.
 constexpr long kMaxRows = static_cast<long>(kCntBytes / 4) * 16;
@@ -86,7 +86,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
   // sizes beyond what the fixed scratch holds
   if (w->M > kMaxRows) return HQ_ERR_WORKSPACE;
-  if (static_cast<size_t>(gemv_max_warps()) * 2 * 32 * 16 > kPartBytes) return HQ_ERR_WORKSPACE;
+  if (gemv_part_bytes() > kPartBytes) return HQ_ERR_WORKSPACE;
   int nb = 0;
   for (int b = 8; b >= 1 && nb == 0; b >>= 1) {
     if (gemv_smem_bytes(w->bits, w->K, b) != 0) nb = b;

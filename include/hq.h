@@ -167,7 +167,7 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
  * packaging variant of hq_linear, same arguments minus the workspace, same
  * results (same kernels and work split).
  * Its scratch is a 2 MiB array in the library's device memory, held on every
- * GPU that loads the library until the process exits.  Limits: M <= 1,752,064
+ * GPU that loads the library until the process exits.  Limits: M <= 5,946,368
  * output rows (HQ_ERR_WORKSPACE beyond), other limits as hq_linear.
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, no allocation); make that first call before any stream

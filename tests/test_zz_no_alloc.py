@@ -54,6 +54,6 @@ def test_noalloc_matches_hq_linear_twice(M, K, bits, N):
 def test_noalloc_rejects_rows_beyond_its_scratch():
     from bit_hadamard_rotated_b200 import _lib
     from bit_hadamard_rotated_b200._lib import HQ_ERR_WORKSPACE, HqWeight
-    big = HqWeight(4, 3_144_704 + 16, 128, 8, 0x100000, 0x100000, None)
+    big = HqWeight(4, 5_946_368 + 16, 128, 8, 0x100000, 0x100000, None)
     st = _lib.lib().hq_linear_noalloc(ctypes.byref(big), 0x100000, 1, 0x100000, None)
     assert st == HQ_ERR_WORKSPACE
