@@ -42,6 +42,7 @@
 namespace hq {
 
 constexpr int kWarps = 16;
+constexpr int kPrepWarps = 8;  // the FWHT uses at most 8 warps for K <= 8192
 constexpr int kRows = 16;
 // halves per (group, column, k-quad) block of B fragments: 8 steps x 4, padded
 // to 80 bytes so the 16-byte loads of 8 lanes hit distinct banks
@@ -62,7 +63,7 @@ struct GemvParams {
   uint32_t U;  // units = n_tiles * G
   int zero;
   const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, then zc [G][8] fp32
-  int CH, NS, stride, slot_bytes, zc_off, sp_off, ring_off, bar_off;
+  int CH, NS, stride, slot_bytes, zc_off, ring_off, bar_off;
 };
 
 // Bytes of the prep output for a batch block of nb columns (16-byte multiple).
@@ -79,7 +80,7 @@ __host__ __device__ constexpr size_t gemv_xg_bytes(int G, int nb) {
 // field, plus the zero-point term -zero * sum_k x'_k * 2^-24 of each group;
 // CTA 0 also zeroes the zero-point terms of the absent columns (N..7).
 template <int BITS, int LOGK>
-__global__ void __launch_bounds__(kWarps * 32) gemv_prep_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half* __restrict__ x,
                                                                  const int8_t* __restrict__ signs,
                                                                  uint8_t* __restrict__ xg, int N,
                                                                  int zero, float inv_sqrt_k) {
@@ -103,7 +104,7 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_prep_kernel(const __half* __
   }
   pdl_wait();  // x is the previous kernel's output; xg may still be read by it
   if (n == 0) {
-    for (int i = tid; i < G * (8 - N); i += kWarps * 32) zc[(i / (8 - N)) * 8 + N + i % (8 - N)] = 0.f;
+    for (int i = tid; i < G * (8 - N); i += kPrepWarps * 32) zc[(i / (8 - N)) * 8 + N + i % (8 - N)] = 0.f;
   }
   float v[FS::E];
   if (tid < FS::THREADS) {
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(kWarps * 32) gemv_prep_kernel(const __half* __
     apply_signs<FS::E>(signs ? signs + tid * FS::E : nullptr, v);
   }
   fwht_block<LOGK, 3>(v, buf);
-  for (int gg = warp; gg < G; gg += kWarps) {
+  for (int gg = warp; gg < G; gg += kPrepWarps) {
     uint16_t hv[4];
     float part = 0.f;
 #pragma unroll
@@ -234,10 +235,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
   // ---- consumer: decode + MMA over the warp's units
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  // Tiles this warp covers only in part: its first (0) and last (1); their
-  // partial sums go to shared-memory slot sp[warp][which] (scaled by 2^24).
+  // Tiles this warp covers only in part: its first (0) and last (1), with
+  // their partial sums (scaled by 2^24), kept in registers until the loop
+  // ends and then left in the warp's own (by then idle) ring memory.
   int ptile0 = -1, ptile1 = -1;
-  float4* sp = reinterpret_cast<float4*>(smem + p.sp_off);
+  float4 psum0 = make_float4(0.f, 0.f, 0.f, 0.f), psum1 = psum0;
   int tile_start = -1;
   int consumed = 0;
   bool ok = true;
@@ -362,12 +364,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (full) {
         store_tile(tile, o);
       } else {
-        const int which = (tile == first_tile) ? 0 : 1;
-        sp[(warp * 2 + which) * 32 + lane] = o;
-        if (which == 0) {
+        if (tile == first_tile) {
           ptile0 = static_cast<int>(tile);
+          psum0 = o;
         } else {
           ptile1 = static_cast<int>(tile);
+          psum1 = o;
         }
       }
       acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
@@ -376,7 +378,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   }
   // ---- tiles split between warps: the first contributing warp of the CTA
   // adds the CTA's partials in warp order (shared memory), then stores the
-  // tile, or exchanges it with the other CTAs that share it
+  // tile, or exchanges it with the other CTAs that share it.  Partial slots:
+  // the first 1 KiB of each warp's ring (its copies have all been consumed).
+  auto sp_slot = [&](uint32_t w, int which) {
+    return reinterpret_cast<float4*>(smem + p.ring_off + w * p.NS * p.slot_bytes) + which * 32 + lane;
+  };
+  if (ok) {
+    *sp_slot(warp, 0) = psum0;
+    *sp_slot(warp, 1) = psum1;
+  }
   __syncthreads();
   if (ok) {
 #pragma unroll
@@ -392,7 +402,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         const uint32_t wb = cb + unit_begin(w, cl, kWarps);
         if (wb == cb + unit_begin(w + 1, cl, kWarps)) continue;  // empty range
         const int ww = (tile == wb / G) ? 0 : 1;
-        const float4 q4 = sp[(w * 2 + ww) * 32 + lane];
+        const float4 q4 = *sp_slot(w, ww);
         o.x += q4.x;
         o.y += q4.y;
         o.z += q4.z;
@@ -414,54 +424,57 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host planning
 struct GemvPlan {
-  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, sp_off = 0, ring_off = 0, bar_off = 0;
+  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, ring_off = 0, bar_off = 0;
   size_t smem = 0;
 };
 
-// One 16-warp CTA per SM (its registers fill the SM) with all of the
-// shared memory: the deeper each warp's ring, the more weight bytes in flight.
+// One 16-warp CTA per SM (its registers fill the SM), up to all of the
+// shared memory.
 constexpr size_t kMaxSmem = 227 * 1024;
-constexpr int kMaxNS = 8;
-constexpr size_t kSpBytes = static_cast<size_t>(kWarps) * 2 * 32 * 16;  // partial-tile slots
+constexpr int kMaxNS = 4;
 
-// The ring with the most groups in flight per warp (CH x NS) that fits the
-// budget; among equal products, more and smaller slots (finer refills).
-static GemvPlan gemv_plan_budget(int bits, int K, int nb, size_t budget) {
-  GemvPlan best;
+// Ring shape, from a sweep of slot shapes on this B200 (batch 1, back-to-back
+// calls): slots of about 4 KiB of codes per warp (16 / bits groups: 8, 4, 4
+// and 2 at 2, 3, 4 and 8 bits) beat many small slots by 1.3-2x, and two to
+// four of them per warp are enough; leaving shared memory for a prep CTA of
+// the next call made no measurable difference.  If no two such slots fit,
+// the slot halves.
+static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t budget) {
+  GemvPlan pl;
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
-  const size_t sp_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
-  const size_t ring_off = sp_off + kSpBytes;
-  for (int CH : {1, 2, 4, 8}) {
-    const int ch = std::min(CH, G);
-    const int row = ch * 16 * bits;
-    const int pad_w = ((bank_target_words(bits) - row / 4) % 32 + 32) % 32;
-    const int stride = row + 4 * pad_w;
-    const int sbytes = G >= 8 ? kRows * 32 : ((kRows * G * 2 + 15) & ~15);
-    const int slot = kRows * stride + sbytes;
-    for (int NS = kMaxNS; NS >= 2; --NS) {
-      const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * NS * slot;
-      const size_t smem = bar_off + static_cast<size_t>(kWarps) * NS * 8;
-      if (smem > budget) continue;
-      if (static_cast<long>(ch) * NS > static_cast<long>(best.CH) * best.NS) {
-        best.CH = ch;
-        best.NS = NS;
-        best.stride = stride;
-        best.slot_bytes = slot;
-        best.zc_off = static_cast<int>(zc_off);
-        best.sp_off = static_cast<int>(sp_off);
-        best.ring_off = static_cast<int>(ring_off);
-        best.bar_off = static_cast<int>(bar_off);
-        best.smem = smem;
-      }
-      break;  // the largest NS that fits for this CH
-    }
-  }
-  return best;
+  const size_t ring_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
+  const int row = ch * 16 * bits;
+  const int pad_w = ((bank_target_words(bits) - row / 4) % 32 + 32) % 32;
+  const int stride = row + 4 * pad_w;
+  const int sbytes = G >= 8 ? kRows * 32 : ((kRows * G * 2 + 15) & ~15);
+  const int slot = kRows * stride + sbytes;
+  const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * ns * slot;
+  const size_t smem = bar_off + static_cast<size_t>(kWarps) * ns * 8;
+  // a warp's partial-tile slots (1 KiB) live in its ring
+  if (smem > budget || static_cast<size_t>(ns) * slot < 1024) return pl;
+  pl.CH = ch;
+  pl.NS = ns;
+  pl.stride = stride;
+  pl.slot_bytes = slot;
+  pl.zc_off = static_cast<int>(zc_off);
+  pl.ring_off = static_cast<int>(ring_off);
+  pl.bar_off = static_cast<int>(bar_off);
+  pl.smem = smem;
+  return pl;
 }
 
-static GemvPlan gemv_plan(int bits, int K, int nb) { return gemv_plan_budget(bits, K, nb, kMaxSmem); }
+static GemvPlan gemv_plan(int bits, int K, int nb) {
+  const int G = K / kGroup;
+  for (int ch = std::min(G, 16 / bits >= 8 ? 8 : 16 / bits >= 4 ? 4 : 2); ch >= 1; ch >>= 1) {
+    for (int ns = kMaxNS; ns >= 2; --ns) {
+      const GemvPlan pl = gemv_plan_shape(bits, K, nb, ch, ns, kMaxSmem);
+      if (pl.smem != 0) return pl;
+    }
+  }
+  return GemvPlan{};
+}
 
 size_t gemv_smem_bytes(int bits, int K, int nb) { return gemv_plan(bits, K, nb).smem; }
 
@@ -503,7 +516,7 @@ size_t gemv_scratch_bytes(int K, int nb) { return gemv_xg_bytes(K / kGroup, nb);
 
 template <int BITS>
 static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
-  const dim3 g(a.N), b(kWarps * 32);
+  const dim3 g(a.N), b(kPrepWarps * 32);
   const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(K)));
   const __half* x = reinterpret_cast<const __half*>(a.x);
   uint8_t* xg = static_cast<uint8_t*>(a.xg);
@@ -559,7 +572,6 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.stride = pl.stride;
   p.slot_bytes = pl.slot_bytes;
   p.zc_off = pl.zc_off;
-  p.sp_off = pl.sp_off;
   p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = a.zero;
   p.ring_off = pl.ring_off;
