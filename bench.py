@@ -269,7 +269,9 @@ def run_ours(a):
                                 f"> L2 between reuses of a copy",
                    "parallelism": f"replicas x{world} (weak scaling, no data-path collective)"},
         "frac_hbm": round(value / world / pk["hbm"], 4),
-        "roofline": {"bound": "hbm", "kernel": "prep_gemv + gemv_kernel (aggregate of the step)",
+        "roofline": {"bound": "hbm",
+                     "kernel": "gemv_kernel, with its gemv_prep_kernel (one pair per linear; "
+                               "aggregate over the step's three linears)",
                      "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
                      "frac": round(achieved / pk["hbm"], 4), "traffic": None,
                      "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
@@ -288,35 +290,44 @@ def run_ours(a):
 
 
 def measure_b64(device, stream, pk):
-    """TFLOP/s of the large dense MLP linear (28672x8192, 2-bit) at batch 64."""
+    """TFLOP/s of the large dense MLP linear (28672x8192, 2-bit) at batch 64 (and 16)."""
     from bit_hadamard_rotated_b200 import RotatedLinear
     M, K, b, N = B64
     d = synth.linear(M, K, b, N, seed=77, scale_dist="loguniform", outlier_frac=0.01)
     lin = RotatedLinear(torch.from_numpy(d["q"].view(np.int32)).to(device),
                         torch.from_numpy(d["scales"]).to(device),
                         torch.from_numpy(d["signs"]).to(device), b, d["zero"], max_batch=N)
-    x = torch.from_numpy(d["x"]).to(device)
-    y = torch.empty((N, M), dtype=torch.float32, device=device)
     flush = torch.empty(2 * 126 * 2**20 // 4, dtype=torch.float32, device=device)
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            lin(x, out=y)
-        torch.cuda.synchronize(device)
-        times = []
-        for _ in range(20):
-            flush.zero_()  # L2 flush between timed calls (outside the timed interval)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            lin(x, out=y)
-            e1.record(stream)
+    out = {}
+    for n in (N, 16):
+        x = torch.from_numpy(np.ascontiguousarray(d["x"][:n])).to(device)
+        y = torch.empty((n, M), dtype=torch.float32, device=device)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                lin(x, out=y)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                lin(x, out=y)
             torch.cuda.synchronize(device)
-            times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
-    tflops = 2.0 * M * K * N / (ms * 1e-3) / 1e12
-    return {"workload": f"rotated linear M={M} K={K} b{b} batch {N}", "ms": round(ms, 4),
-            "tflops": round(tflops, 2), "frac_bf16_peak": round(tflops / pk["bf16"], 4),
-            "weight_gbs": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9, 1),
-            "launches": lin.launches(N), "timing": "median of 20, L2 flushed before each"}
+            times = []
+            for _ in range(20):
+                flush.zero_()  # L2 flush between timed calls (outside the timed interval)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize(device)
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        tflops = 2.0 * M * K * n / (ms * 1e-3) / 1e12
+        out[n] = {"ms": round(ms, 4), "tflops": round(tflops, 2),
+                  "frac_bf16_peak": round(tflops / pk["bf16"], 4),
+                  "weight_gbs": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9, 1),
+                  "launches": lin.launches(n)}
+    r = {"workload": f"rotated linear M={M} K={K} b{b} batch {N}", **out[N],
+         "timing": "CUDA-graph replay of one call, median of 20, L2 flushed before each",
+         "batch16": out[16]}
+    return r
 
 
 def measure_e2e(device, layers, xs, a):

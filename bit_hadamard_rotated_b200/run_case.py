@@ -1,0 +1,101 @@
+"""Run one hq_linear (or one MoE layer) case a few times on seeded synthetic inputs.
+
+A reproducible target for profilers and quick timing:
+
+    python -m bit_hadamard_rotated_b200.run_case --M 12288 --K 4096 --bits 2 --batch 1
+    python -m bit_hadamard_rotated_b200.run_case --moe
+
+Inputs come from bit_hadamard_rotated_b200.synth (seeded); every call goes
+through the C ABI.  Prints the mean device time per call (CUDA events around
+--reps back-to-back calls after --warmup calls) and checks the device status.
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+import torch
+
+from . import synth
+from .hq import RotatedLinear, expert_table, hq_check_status, hq_moe_experts, hq_moe_workspace_size
+
+
+def run_linear(a):
+    d = synth.linear(a.M, a.K, a.bits, a.batch, seed=a.seed, scale_dist=a.scales)
+    dev = torch.device("cuda", 0)
+    lin = RotatedLinear(torch.from_numpy(d["q"].view(np.int32)).to(dev),
+                        torch.from_numpy(d["scales"]).to(dev),
+                        torch.from_numpy(d["signs"]).to(dev), a.bits, d["zero"], max_batch=a.batch)
+    x = torch.from_numpy(d["x"]).to(dev)
+    y = torch.empty((a.batch, a.M), dtype=torch.float32, device=dev)
+    for _ in range(a.warmup):
+        lin(x, out=y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        lin(x, out=y)
+    e1.record()
+    torch.cuda.synchronize()
+    lin.check_status()
+    us = e0.elapsed_time(e1) * 1e3 / max(a.reps, 1)
+    wb = d["q"].nbytes + d["scales"].nbytes
+    print(f"linear M={a.M} K={a.K} b{a.bits} batch {a.batch}: {us:.2f} us/call "
+          f"({wb / (us * 1e-6) / 1e9:.0f} GB/s weights, {lin.launches(a.batch)} launches/call)")
+
+
+def run_moe(a):
+    m = synth.moe(seed=a.seed)
+    dev = torch.device("cuda", 0)
+
+    def put(v):
+        return torch.from_numpy(np.ascontiguousarray(v)).to(dev)
+
+    experts = []
+    for e in m["experts"]:
+        d = dict(bits=e["bits"], zero=e["zero"])
+        for n in ("q_gate", "q_up", "q_down"):
+            d[n] = put(e[n].view(np.int32))
+        for n in ("s_gate", "s_up", "s_down"):
+            d[n] = put(e[n])
+        experts.append(d)
+    table = expert_table(experts, dev)
+    E, H, I, T, k = len(experts), m["hidden"], m["inter"], m["T"], m["k"]
+    x, ids = put(m["x"]), put(m["topk_ids"].astype(np.int32))
+    w = put(m["topk_w"].astype(np.float32))
+    s_in, s_mid = put(m["s_in"]), put(m["s_mid"])
+    ws = torch.zeros(hq_moe_workspace_size(E, H, I, T, k), dtype=torch.uint8, device=dev)
+    out = torch.empty((T, H), dtype=torch.float32, device=dev)
+    for _ in range(a.warmup):
+        hq_moe_experts(table, E, H, I, x, ids, w, s_in, s_mid, out=out, workspace=ws)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        hq_moe_experts(table, E, H, I, x, ids, w, s_in, s_mid, out=out, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    hq_check_status(ws)
+    us = e0.elapsed_time(e1) * 1e3 / max(a.reps, 1)
+    tb = synth.touched_weight_bytes(m)
+    print(f"moe E={E} hidden={H} inter={I} tokens={T} top-{k}: {us:.2f} us/call "
+          f"({tb / (us * 1e-6) / 1e9:.0f} GB/s over {tb / 1e6:.1f} MB of touched expert weights)")
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawTextHelpFormatter)
+    ap.add_argument("--M", type=int, default=12288)
+    ap.add_argument("--K", type=int, default=4096)
+    ap.add_argument("--bits", type=int, default=2)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--scales", default="uniform", choices=["uniform", "loguniform"])
+    ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--moe", action="store_true", help="run the MoE expert layer instead")
+    a = ap.parse_args()
+    if not torch.cuda.is_available():
+        raise SystemExit("run_case needs a CUDA device")
+    run_moe(a) if a.moe else run_linear(a)
+
+
+if __name__ == "__main__":
+    main()
