@@ -1,35 +1,35 @@
-// gemv.cu -- fused rotate + unpack-dequant GEMV over packed low-bit codes,
-// batch <= 8 per launch.
+// gemv.cu -- unpack-dequant GEMV over packed low-bit codes, batch <= 8 per
+// launch, with the rotation of the activations in a small prep kernel.
 //
 //   y[n][m] = sum_k scale[m][k/128] (q[m][k] - zero) x'[n][k],
 //   x'[n]   = H_K diag(s) x[n] / sqrt(K).
 //
-// Decoding is bound by weight bytes ("decode is per-byte neutral": Laguna-S-2.1
-// gridbook card, "Reading it honestly"), so the kernel is shaped to stream the
-// packed codes at HBM rate with the rotation and all dequantisation on chip:
+// At small batch the cost is set by the weight bytes (decode speed follows the
+// bytes streamed: Laguna-S-2.1 gridbook card, "Reading it honestly"), so the
+// GEMV is shaped to stream packed codes at HBM rate with all dequantisation
+// on chip:
 //
-//   * Persistent grid, one CTA of 16 warps per SM.  The work is the list of
-//     (16-row tile, 128-code group) units; every warp owns one contiguous
-//     range of ~U/(16 * #SMs) units, so the load is balanced to one group.
-//   * Each warp streams its range through a private ring of NS shared-memory
-//     slots.  A slot holds up to CH groups of 16 rows (rows at a bank-conflict-
-//     free padded stride) and the matching fp16 scales, moved by 16-byte
-//     cp.async copies spread across the lanes, completing on one mbarrier
-//     (many small bulk copies, one per row, were bound by the copy engine's
-//     per-request cost).
-//     The first NS copies are issued before griddepcontrol.wait: weights do not
-//     depend on earlier kernels, so they overlap the previous kernel's tail.
-//   * Meanwhile the CTA rotates its N activation rows in fp32 (fwht.cuh) and
-//     stores x' as fp16 in the order of the MMA B fragments, each scaled by the
-//     2^-a of its code field (hq_layout.cuh), plus zero * sum_k x'_k per group.
+//   * gemv_prep_kernel (one CTA per batch row) rotates x in fp32 (fwht.cuh)
+//     and writes x' as fp16 in the order of the MMA B fragments, each value
+//     scaled by the 2^-a of its code field (hq_layout.cuh), plus the
+//     zero-point term -zero * sum_k x'_k * 2^-24 of each group.
+//   * gemv_kernel: persistent grid, one 16-warp CTA per SM.  The work is the
+//     list of (16-row tile, 128-code group) units; each CTA owns a contiguous
+//     range of whole tiles and its warps split that range evenly.
+//   * Each warp streams its range through a private ring of shared-memory
+//     slots of about 4 KiB of codes (CH groups of 16 rows at a bank-conflict-
+//     free stride, plus scales), moved by 16-byte cp.async copies that
+//     complete on one mbarrier per slot.  The first slots are requested
+//     before griddepcontrol.wait: weights do not depend on earlier kernels.
+//     After the wait, the CTA copies the prep kernel's fragments into shared
+//     memory.
 //   * Per group: each lane masks 2 x 32 codes into exact subnormal fp16 pairs
 //     (one LOP3/PRMT per pair), runs 8 mma.sync m16n8k16 with fp32
-//     accumulation in two chains (one starting at -zero * sum x' * 2^-24), then
+//     accumulation in two chains (one starting at the zero-point term), then
 //     acc += (scale * 2^24) * sum.
-//   * A tile split between warps is finished by whichever contributor arrives
-//     last at the tile's counter: it adds all contributors' partial sums in
-//     warp order (deterministic, no waiting) and resets the counter.  A warp
-//     defers these exchanges to the end of its range.
+//   * A tile split between warps of the CTA is summed in warp order through
+//     shared memory after one __syncthreads (deterministic); no tile is split
+//     between CTAs, so no global exchange is needed.
 #include <algorithm>
 
 #include "fwht.cuh"
@@ -57,8 +57,6 @@ struct GemvParams {
   const int8_t* signs;
   float* y;
   uint32_t* status;
-  float4* part;   // [#CTAs][2][32] partial tiles of tiles shared between CTAs
-  uint32_t* cnt;  // [n_tiles] arrival counters, zero between launches
   int M, N, ldy;
   uint32_t U;  // units = n_tiles * G
   int zero;
@@ -150,9 +148,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  // the CTA owns units [cb, ce); its warps split them into contiguous ranges
+  // the CTA owns whole tiles, units [cb, ce); its warps split them into
+  // contiguous ranges (a tile is never shared with another CTA)
   const uint32_t GC = gridDim.x;
-  const uint32_t cb = unit_begin(blockIdx.x, p.U, GC), ce = unit_begin(blockIdx.x + 1, p.U, GC);
+  const uint32_t n_tiles = p.U / G;
+  const uint32_t cb = unit_begin(blockIdx.x, n_tiles, GC) * G;
+  const uint32_t ce = unit_begin(blockIdx.x + 1, n_tiles, GC) * G;
   const uint32_t cl = ce - cb;
   const uint32_t u0 = cb + unit_begin(warp, cl, kWarps);
   const uint32_t u1 = cb + unit_begin(warp + 1, cl, kWarps);
@@ -254,7 +255,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   const uint32_t first_tile = u0 / G;
   uint32_t uc = u0;
 
-  const uint32_t cta_first_tile = cb / G;
   auto store_tile = [&](uint32_t tile, const float4& o) {
     const int m0 = tile * kRows;
     const int rv = min(kRows, M - m0);
@@ -267,36 +267,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g + 8] = o.w;
     }
   };
-  // A tile shared with other CTAs: this CTA's sum is published, one fence
-  // orders it before the tile's arrival counter, and the last CTA to arrive
-  // adds every CTA's sum in CTA order (deterministic, no waiting) and stores.
-  auto exchange = [&](uint32_t tile, const float4& o) {
-    const int which = (tile == cta_first_tile) ? 0 : 1;
-    p.part[(static_cast<size_t>(blockIdx.x) * 2 + which) * 32 + lane] = o;
-    __syncwarp();
-    uint32_t old = 0;
-    if (lane == 0) {
-      __threadfence();
-      old = atomicAdd(&p.cnt[tile], 1u);
-    }
-    old = __shfl_sync(0xffffffffu, old, 0);
-    const uint32_t cf = unit_owner(tile * G, p.U, GC);
-    const uint32_t cz = unit_owner(tile * G + G - 1, p.U, GC);
-    if (old != cz - cf) return;
-    __threadfence();
-    float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (uint32_t c = cf; c <= cz; ++c) {
-      const int wc = (tile == unit_begin(c, p.U, GC) / G) ? 0 : 1;
-      const float4 q4 = __ldcg(&p.part[(static_cast<size_t>(c) * 2 + wc) * 32 + lane]);
-      s4.x += q4.x;
-      s4.y += q4.y;
-      s4.z += q4.z;
-      s4.w += q4.w;
-    }
-    if (lane == 0) p.cnt[tile] = 0u;
-    store_tile(tile, s4);
-  };
-
   while (uc < u1) {
     const uint32_t tile = uc / G, g0 = uc % G;
     const uint32_t len = min(static_cast<uint32_t>(CH), min(G - g0, u1 - uc));
@@ -376,10 +346,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       tile_start = -1;
     }
   }
-  // ---- tiles split between warps: the first contributing warp of the CTA
-  // adds the CTA's partials in warp order (shared memory), then stores the
-  // tile, or exchanges it with the other CTAs that share it.  Partial slots:
-  // the first 1 KiB of each warp's ring (its copies have all been consumed).
+  // ---- tiles split between warps: the first contributing warp adds the
+  // CTA's partials in warp order (shared memory) and stores the tile.
+  // Partial slots: the first 1 KiB of each warp's ring (its copies have all
+  // been consumed).
   auto sp_slot = [&](uint32_t w, int which) {
     return reinterpret_cast<float4*>(smem + p.ring_off + w * p.NS * p.slot_bytes) + which * 32 + lane;
   };
@@ -394,7 +364,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       const int tl = which == 0 ? ptile0 : ptile1;
       if (tl < 0 || (which == 1 && tl == ptile0)) continue;
       const uint32_t tile = static_cast<uint32_t>(tl);
-      const uint32_t tf = max(tile * G, cb), tz = min(tile * G + G, ce) - 1;
+      const uint32_t tf = tile * G, tz = tile * G + G - 1;
       if (unit_owner(tf - cb, cl, kWarps) != static_cast<uint32_t>(warp)) continue;
       const uint32_t wz = unit_owner(tz - cb, cl, kWarps);
       float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -408,11 +378,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         o.z += q4.z;
         o.w += q4.w;
       }
-      if (tile * G >= cb && tile * G + G <= ce) {
-        store_tile(tile, o);
-      } else {
-        exchange(tile, o);
-      }
+      store_tile(tile, o);
     }
   }
   if (!ok) {
@@ -493,8 +459,6 @@ int sm_count() {
   return sms;
 }
 
-size_t gemv_part_bytes() { return static_cast<size_t>(sm_count()) * 2 * 32 * 16; }
-
 template <int BITS>
 static cudaError_t gemv_launch_b(int K, GemvParams& p, size_t smem, unsigned grid,
                                  cudaStream_t st) {
@@ -552,8 +516,8 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   const int G = a.K / kGroup;
   const uint32_t n_tiles = static_cast<uint32_t>((a.M + kRows - 1) / kRows);
   const uint32_t U = n_tiles * static_cast<uint32_t>(G);
-  // one CTA per SM, at most one per kWarps units (so every CTA has units)
-  const uint32_t grid = std::min<uint32_t>(static_cast<uint32_t>(sm_count()), (U + kWarps - 1) / kWarps);
+  // one CTA per SM, each owning whole tiles (at least one)
+  const uint32_t grid = std::min<uint32_t>(static_cast<uint32_t>(sm_count()), n_tiles);
   GemvParams p{};
   p.q = a.q;
   p.scales = a.scales;
@@ -561,8 +525,6 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.signs = a.signs;
   p.y = a.y;
   p.status = a.status;
-  p.part = reinterpret_cast<float4*>(a.part);
-  p.cnt = a.cnt;
   p.M = a.M;
   p.N = a.N;
   p.ldy = a.ldy;

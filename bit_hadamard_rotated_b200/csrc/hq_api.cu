@@ -58,32 +58,26 @@ static bool use_tc(const hq_weight* w, int batch) {
          tc_col_block(w->bits, w->K) > 0;
 }
 
-// hq_linear workspace: [status 256 B][GEMV partial tiles][tile counters]
+// hq_linear workspace: [status 256 B]
 // [activations: on the tensor-core path the rotated activation images (batch
 // rounded up to whole batch blocks, x K fp16); on the GEMV path the rotated
 // activations of one batch block in fragment order (blocks run in turn)].
 struct LinearWs {
   uint32_t* status;
-  void* part;
-  uint32_t* cnt;
   void* xp;
   size_t bytes;
 };
 
 static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
-  const size_t part_bytes = align256(gemv_part_bytes());
-  const size_t cnt_bytes = align256(static_cast<size_t>((w->M + 15) / 16) * 4);
   const int nb = gemv_col_block(w->bits, w->K);
   const size_t xp_bytes = use_tc(w, batch)
                               ? align256(tc_xp_bytes(w->bits, w->K, batch))
                               : align256(gemv_scratch_bytes(w->K, nb > 0 ? std::min(nb, std::max(batch, 1)) : 1));
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
-  l.part = b + kStatusBytes;
-  l.cnt = reinterpret_cast<uint32_t*>(b + kStatusBytes + part_bytes);
-  l.xp = b + kStatusBytes + part_bytes + cnt_bytes;
-  l.bytes = kStatusBytes + part_bytes + cnt_bytes + xp_bytes;
+  l.xp = b + kStatusBytes;
+  l.bytes = kStatusBytes + xp_bytes;
   return l;
 }
 
@@ -189,8 +183,6 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     a.y = y + static_cast<size_t>(n0) * w->M;
     a.ldy = w->M;
     a.status = l.status;
-    a.part = l.part;
-    a.cnt = l.cnt;
     a.xg = l.xp;
     const cudaError_t e = launch_gemv(a, st);
     if (e != cudaSuccess) return from_cuda(e);

@@ -32,8 +32,6 @@ struct GemvArgs {
   float* y;             // [N][M] block of outputs, row stride ldy
   int ldy;
   uint32_t* status;
-  void* part;     // gemv_part_bytes(): partial tiles shared between CTAs
-  uint32_t* cnt;  // ceil(M/16) counters, zero between launches
   void* xg;       // gemv_scratch_bytes(K, N) bytes, 16-byte aligned: prep output
 };
 
@@ -44,8 +42,6 @@ size_t gemv_smem_bytes(int bits, int K, int nb);
 size_t gemv_scratch_bytes(int K, int nb);
 // Streaming multiprocessors of the current device (148 if the query fails).
 int sm_count();
-// Bytes of the GEMV's cross-CTA partial-tile buffer.
-size_t gemv_part_bytes();
 // Two launches: the rotation (prep) and the GEMV.
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 

@@ -11,8 +11,10 @@
 // weight, input and output buffers.
 //
 // Costs of that convenience:
-//   * every GPU that loads the library keeps kScratchBytes (2 MiB) of device
+//   * every GPU that loads the library keeps kScratchBytes (512 KiB) of device
 //     memory until the process exits;
+//   * every batch runs the GEMV kernels in blocks of up to 8 columns: the
+//     tensor-core path would need a batch-sized activation buffer;
 //   * every call shares the one array, so calls that overlap on the GPU (two
 //     streams, or two host threads) race on it and must be serialised by the
 //     caller;
@@ -25,17 +27,13 @@
 namespace hq {
 namespace {
 
-constexpr size_t kScratchBytes = size_t{2} << 20;  // 2 MiB in total
-constexpr size_t kStatus = 256;                    // status word, kept zero
-constexpr size_t kXgBytes = size_t{340} << 10;     // rotated activations of one batch block
-constexpr size_t kPartBytes = size_t{256} << 10;   // partial tiles shared between CTAs: up to 256 SMs
-constexpr size_t kCntBytes = kScratchBytes - kStatus - kXgBytes - kPartBytes;  // tile counters
-// Largest output-row count: one 4-byte counter per 16 rows.
-constexpr long kMaxRows = static_cast<long>(kCntBytes / 4) * 16;
+constexpr size_t kScratchBytes = size_t{512} << 10;  // 512 KiB in total
+constexpr size_t kStatus = 256;                      // status word, kept zero
+// Rotated activations of one batch block: at most 332 KiB (K = 16384, 8 columns).
+constexpr size_t kXgBytes = kScratchBytes - kStatus;
 
-// The scratch: [status][tile counters][rotated activations][split-tile
-// partials].  Static storage starts zeroed; each call clears the status word
-// and the counters it uses.
+// The scratch: [status][rotated activations of the current batch block].
+// Static storage starts zeroed; each call clears the status word.
 __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
@@ -84,14 +82,12 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
   if (batch < 0 || batch > 65535) return HQ_ERR_INVALID_ARG;
   if (batch == 0) return HQ_OK;
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
-  // sizes beyond what the fixed scratch holds
-  if (w->M > kMaxRows) return HQ_ERR_WORKSPACE;
-  if (gemv_part_bytes() > kPartBytes) return HQ_ERR_WORKSPACE;
   int nb = 0;
   for (int b = 8; b >= 1 && nb == 0; b >>= 1) {
     if (gemv_smem_bytes(w->bits, w->K, b) != 0) nb = b;
   }
   if (nb == 0) return HQ_ERR_UNSUPPORTED;
+  // beyond what the fixed scratch holds (cannot happen for a supported K)
   if (gemv_scratch_bytes(w->K, nb) > kXgBytes) return HQ_ERR_WORKSPACE;
 
   uint8_t* scratch = nullptr;
@@ -100,8 +96,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     return HQ_ERR_CUDA;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const size_t n_tiles = static_cast<size_t>((w->M + 15) / 16);
-  if (cudaMemsetAsync(scratch, 0, kStatus + n_tiles * 4, st) != cudaSuccess) {
+  if (cudaMemsetAsync(scratch, 0, kStatus, st) != cudaSuccess) {
     (void)cudaGetLastError();
     return HQ_ERR_CUDA;
   }
@@ -119,9 +114,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     a.y = y + static_cast<size_t>(n0) * w->M;
     a.ldy = w->M;
     a.status = reinterpret_cast<uint32_t*>(scratch);
-    a.cnt = reinterpret_cast<uint32_t*>(scratch + kStatus);
-    a.xg = scratch + kStatus + kCntBytes;
-    a.part = scratch + kStatus + kCntBytes + kXgBytes;
+    a.xg = scratch + kStatus;
     if (launch_gemv(a, st) != cudaSuccess) {
       (void)cudaGetLastError();
       return HQ_ERR_CUDA;

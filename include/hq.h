@@ -164,11 +164,15 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
  * allocate device memory (a plug-in whose host program owns the device heap, a
  * latency-critical loop that must not call cudaMalloc, a binding with device
  * pointers but no allocator).  The pages have no counterpart: this is a
- * packaging variant of hq_linear, same arguments minus the workspace, same
- * results (same kernels and work split).
- * Its scratch is a 2 MiB array in the library's device memory, held on every
- * GPU that loads the library until the process exits.  Limits: M <= 5,946,368
- * output rows (HQ_ERR_WORKSPACE beyond), other limits as hq_linear.
+ * packaging variant of hq_linear, same arguments minus the workspace, results
+ * within the same tolerance: every batch runs the GEMV kernels in blocks of up
+ * to 8 columns (the tensor-core path that hq_linear uses from batch 9 needs a
+ * workspace for its activation images).
+ * Its scratch is a 512 KiB array in the library's device memory, held on every
+ * GPU that loads the library until the process exits: the status word and the
+ * rotated activations of one batch block (at most 332 KiB, K = 16384).  Limits:
+ * as hq_linear (HQ_ERR_WORKSPACE if a block's activations did not fit, which
+ * no supported K reaches).
  * The first call on a device looks up the array's device address (a CUDA
  * runtime query, no allocation); make that first call before any stream
  * capture.  All calls share the array: calls that overlap on the GPU race and

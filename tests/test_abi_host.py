@@ -77,9 +77,18 @@ def test_linear_rejects_bad_call_args(L):
 def test_workspace_size_queries(L):
     assert L.hq_linear_workspace_size(ctypes.byref(W(bits=7)), 1) == 0
     assert L.hq_linear_workspace_size(ctypes.byref(W()), -1) == 0
+    # status word + one batch block of rotated activations (GEMV), or the
+    # batch's activation images (tensor-core path): independent of M
     a = L.hq_linear_workspace_size(ctypes.byref(W(M=64)), 1)
     b = L.hq_linear_workspace_size(ctypes.byref(W(M=65536)), 1)
-    assert 0 < a < b and a % 256 == 0          # one tile counter per 16 output rows
+    assert 0 < a == b and a % 256 == 0
+    # G x nb x 320 B of B fragments + G x 8 x 4 B of zero-point terms
+    G = 4096 // 128
+    assert a >= 256 + G * 1 * 320 + G * 32
+    k2 = L.hq_linear_workspace_size(ctypes.byref(W(K=8192)), 1)
+    assert k2 > a
+    big = L.hq_linear_workspace_size(ctypes.byref(W(K=4096)), 64)
+    assert big >= 256 + 64 * 4096 * 2          # tensor-core path: batch x K fp16
 
 
 def test_rotate_rejects_bad_args(L):

@@ -51,9 +51,15 @@ def test_noalloc_matches_hq_linear_twice(M, K, bits, N):
         assert np.all(np.abs(got - want) <= lim), (call, float(np.max(np.abs(got - want) / lim)))
 
 
-def test_noalloc_rejects_rows_beyond_its_scratch():
+def test_noalloc_rejects_what_hq_linear_rejects():
+    """No size limit of its own: unsupported shapes fail with hq_linear's status,
+    before anything is launched."""
     from bit_hadamard_rotated_b200 import _lib
-    from bit_hadamard_rotated_b200._lib import HQ_ERR_WORKSPACE, HqWeight
-    big = HqWeight(4, 5_946_368 + 16, 128, 8, 0x100000, 0x100000, None)
-    st = _lib.lib().hq_linear_noalloc(ctypes.byref(big), 0x100000, 1, 0x100000, None)
-    assert st == HQ_ERR_WORKSPACE
+    from bit_hadamard_rotated_b200._lib import HQ_ERR_UNSUPPORTED, HqWeight
+    L = _lib.lib()
+    before = L.hq_launch_count()
+    for K, want in ((32768, HQ_ERR_UNSUPPORTED), (96, HQ_ERR_UNSUPPORTED)):
+        w = HqWeight(4, 64, K, 8, 0x100000, 0x100000, None)
+        st = L.hq_linear_noalloc(ctypes.byref(w), 0x100000, 1, 0x100000, None)
+        assert st == want
+    assert L.hq_launch_count() == before
