@@ -135,15 +135,6 @@ __device__ __forceinline__ void tc_ld16(uint32_t taddr, uint32_t (&v)[16]) {
       : "memory");
 }
 
-// 2D TMA tile load (no multicast) global -> shared, completing on bar.
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
-      "{%2, %3}], [%4];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
-}
 
 // 16-byte unit holding unit i of code row r in a slot: the TMA swizzle for
 // the row width (32 B rows: 32-byte swizzle, 64 B: 64-byte, 128 B: 128-byte;
@@ -597,26 +588,33 @@ static EncodeTiled encode_tiled() {
 }
 
 // Codes of W as a 2D byte tensor [M][K bits / 8]; box = one group's 16*bits
-// bytes x 128 rows.
+// bytes x 128 rows, swizzled for the decoders' row reads.
 static cudaError_t code_map(CUtensorMap* map, const void* q, int bits, int M, int K) {
-  EncodeTiled fn = encode_tiled();
-  if (fn == nullptr) return cudaErrorNotSupported;
-  const cuuint64_t row_bytes = static_cast<cuuint64_t>(K) * bits / 8;
-  const cuuint64_t dims[2] = {row_bytes, static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(16 * bits), static_cast<cuuint32_t>(kTileM)};
-  const cuuint32_t estr[2] = {1, 1};
   const CUtensorMapSwizzle swz = bits == 2   ? CU_TENSOR_MAP_SWIZZLE_32B
                                  : bits == 4 ? CU_TENSOR_MAP_SWIZZLE_64B
                                  : bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B
                                              : CU_TENSOR_MAP_SWIZZLE_NONE;
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(q), dims, strides, box,
-                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+  const uint64_t row_bytes = static_cast<uint64_t>(K) * bits / 8;
+  return tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, q, row_bytes, static_cast<uint64_t>(M),
+                       row_bytes, static_cast<uint32_t>(16 * bits), kTileM, swz);
 }
 
 }  // namespace tc
+
+cudaError_t tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                          uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                          CUtensorMapSwizzle swizzle) {
+  tc::EncodeTiled fn = tc::encode_tiled();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_stride_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
 
 int tc_col_block(int bits, int K) {
   // K >= 1024: whole 16-byte scale rows, and >= 8 groups per tile (a tile's

@@ -51,6 +51,8 @@ constexpr int kXq = 40;
 constexpr float kUnit = 16777216.f;
 
 struct GemvParams {
+  CUtensorMap qmap;  // codes as bytes [M][K bits / 8]; box 16 bits bytes x 16 rows
+  CUtensorMap smap;  // scales as fp16 [M][K/128]; box 8 x 16 rows (K >= 1024 only)
   const uint32_t* q;
   const uint16_t* scales;
   const __half* x;
@@ -61,7 +63,7 @@ struct GemvParams {
   uint32_t U;  // units = n_tiles * G
   int zero;
   const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, then zc [G][8] fp32
-  int CH, NS, stride, slot_bytes, zc_off, ring_off, bar_off;
+  int CH, NS, slot_bytes, zc_off, ring_off, bar_off;
 };
 
 // Bytes of the prep output for a batch block of nb columns (16-byte multiple).
@@ -145,7 +147,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
   constexpr int GB = 16 * BITS;  // bytes of one group of one row
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // TMA boxes in the 128-byte swizzle need 1 KiB-aligned slots: round the
+  // base up (the launch asks for 1 KiB more than the plan)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   // the CTA owns whole tiles, units [cb, ce); its warps split them into
@@ -157,63 +162,60 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   const uint32_t cl = ce - cb;
   const uint32_t u0 = cb + unit_begin(warp, cl, kWarps);
   const uint32_t u1 = cb + unit_begin(warp + 1, cl, kWarps);
-  const int row_words = K * BITS / 32;
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   float* zc = reinterpret_cast<float*>(smem + p.zc_off);
   uint8_t* ring = smem + p.ring_off + warp * p.NS * p.slot_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off) + warp * p.NS;
+  // slot: [CH groups][16 rows][16 bits bytes] codes (TMA boxes, dense; 8-bit
+  // rows in the 128-byte swizzle), then the scales: K >= 1024: [2 blocks of 8
+  // groups][16 rows][8 halves]; K < 1024: the tile's [16 rows][G halves]
+  const int sc_off = p.CH * kRows * GB;
 
   if (lane == 0) {
-    for (int i = 0; i < p.NS; ++i) mbar_init(&bars[i], 32);
+    for (int i = 0; i < p.NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
   }
   __syncthreads();
   pdl_launch_dependents();
 
-  // ---- producer side of the warp's ring: one chunk = up to CH groups of a
-  // tile, codes and scales, as 16-byte cp.async copies spread over the lanes
-  // (consecutive lanes read consecutive bytes of a row); every lane then
-  // arrives on the slot's barrier when its copies have landed.
+  // ---- producer side of the warp's ring (lane 0): one chunk = up to CH
+  // groups of a tile: one TMA box per group of codes, one or two boxes of
+  // scales, all completing on the slot's barrier (rows past M read as zero)
   uint32_t ui = u0;
   int issued = 0;
   auto issue = [&](int slot) {
     const uint32_t tile = ui / G, g0 = ui % G;
     const uint32_t len = min(static_cast<uint32_t>(p.CH), min(G - g0, u1 - ui));
     const int m0 = tile * kRows;
-    const int rv = min(kRows, p.M - m0);
     uint8_t* base = ring + slot * p.slot_bytes;
-    uint8_t* sdst = base + kRows * p.stride;
-    const int pr = static_cast<int>(len) * BITS;  // 16-byte pieces per row
-    const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(p.q + static_cast<size_t>(m0) * row_words) +
-                          static_cast<size_t>(g0) * GB;
-    // lanes in groups of 2^lg (>= pieces per row, <= 32); one row per group per pass
-    const int lg = pr <= 8 ? 3 : pr <= 16 ? 4 : 5;
-    const int rpp = 32 >> lg;  // rows per pass
-    const int c = lane & ((1 << lg) - 1);
-    for (int r = lane >> lg; r < rv; r += rpp) {
-      for (int cc = c; cc < pr; cc += (1 << lg)) {
-        cp_async16(base + r * p.stride + cc * 16,
-                   qsrc + static_cast<size_t>(r) * row_words * 4 + cc * 16, 16);
+    if (lane == 0) {
+      uint32_t bytes = len * kRows * GB;
+      if constexpr (G >= 8) {
+        const uint32_t nblk = (((g0 + len + 7u) & ~7u) - (g0 & ~7u)) / 8u;
+        bytes += nblk * kRows * 16;
+        mbar_arrive_expect_tx(&bars[slot], bytes);
+        for (uint32_t b = 0; b < nblk; ++b) {
+          tma_load_2d(base + sc_off + b * kRows * 16, &p.smap, static_cast<int>((g0 & ~7u) + 8 * b), m0,
+                      &bars[slot]);
+        }
+      } else {
+        // the tile's scales are one contiguous span; bulk-copy its 16-byte
+        // multiple, plain-copy the rest (only a last, partial tile has one)
+        const int span = min(kRows, p.M - m0) * G * 2;
+        const int bulk = span & ~15;
+        bytes += bulk;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.scales) + static_cast<size_t>(m0) * G * 2;
+        for (int i = bulk; i < span; i += 2) {
+          *reinterpret_cast<uint16_t*>(base + sc_off + i) = *reinterpret_cast<const uint16_t*>(src + i);
+        }
+        mbar_arrive_expect_tx(&bars[slot], bytes);
+        if (bulk > 0) bulk_g2s(base + sc_off, src, bulk, &bars[slot]);
+      }
+      for (uint32_t j = 0; j < len; ++j) {
+        tma_load_2d(base + j * kRows * GB, &p.qmap, static_cast<int>((g0 + j) * GB), m0, &bars[slot]);
       }
     }
-    if constexpr (G >= 8) {
-      const uint32_t sg0 = g0 & ~7u;
-      const int nblk = static_cast<int>((((g0 + len + 7u) & ~7u) - sg0) / 8u);
-      const int r = lane & 15, blk = lane >> 4;
-      if (r < rv && blk < nblk) {
-        cp_async16(sdst + r * 32 + blk * 16, p.scales + static_cast<size_t>(m0 + r) * G + sg0 + 8 * blk,
-                   16);
-      }
-    } else {
-      const int bytes = rv * G * 2;
-      const int lo = lane * 16;
-      if (lane < 2 * G && lo < bytes) {
-        cp_async16(sdst + lo, reinterpret_cast<const uint8_t*>(p.scales + static_cast<size_t>(m0) * G) + lo,
-                   static_cast<uint32_t>(min(16, bytes - lo)));
-      }
-    }
-    cp_async_mbar_arrive(&bars[slot]);
     ui += len;
     ++issued;
   };
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   int tile_start = -1;
   int consumed = 0;
   bool ok = true;
-  const int N = p.N, M = p.M, ldy = p.ldy, CH = p.CH, NS = p.NS, stride = p.stride;
+  const int N = p.N, M = p.M, ldy = p.ldy, CH = p.CH, NS = p.NS;
   const int slot_bytes = p.slot_bytes;
   const bool n0 = 2 * t < N, n1 = 2 * t + 1 < N;
   // lane's B-fragment stream: its column's blocks, or a zero block (stride 0)
@@ -267,35 +269,55 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (n1) p.y[static_cast<size_t>(2 * t + 1) * ldy + m0 + g + 8] = o.w;
     }
   };
+  int slot = 0;
+  uint32_t sph = 0;  // phase parity of the current ring round
   while (uc < u1) {
     const uint32_t tile = uc / G, g0 = uc % G;
     const uint32_t len = min(static_cast<uint32_t>(CH), min(G - g0, u1 - uc));
-    const int slot = consumed % NS;
-    if (!mbar_wait(&bars[slot], (consumed / NS) & 1)) {
+    if (!mbar_wait(&bars[slot], sph)) {
       ok = false;
       break;
     }
     __syncwarp();
     if (tile_start < 0) tile_start = static_cast<int>(g0);
     const uint8_t* base = ring + slot * slot_bytes;
-    const uint8_t* ra = base + g * stride + t * 4 * BITS;
-    const uint8_t* rb = ra + 8 * stride;
-    const int sstride = (G >= 8) ? 16 : G;
-    const __half* sca = reinterpret_cast<const __half*>(base + kRows * stride) + g * sstride +
-                        (G >= 8 ? (g0 & 7u) : g0);
-    const __half* scb = sca + 8 * sstride;
+    // row g of group j at base + j 16 GB + g GB (row g + 8 at + 8 GB); lane t
+    // owns bytes [4 t BITS, 4 (t + 1) BITS) of the row (8-bit: 16-byte chunks
+    // 2t, 2t + 1 in the 128-byte swizzle, XOR row % 8)
+    const uint8_t* ra = base + g * GB + (BITS == 8 ? 0 : t * 4 * BITS);
+    const uint8_t* sc = base + sc_off;
     const float2* zp = reinterpret_cast<const float2*>(zc + g0 * 8 + 2 * t);
     const uint4* xb = xs_lane + static_cast<size_t>(g0) * xs_gstride;
 #pragma unroll 1
     for (uint32_t j = 0; j < len; ++j) {
       uint32_t wa[BITS], wb[BITS];
-      load_bundle<BITS>(ra, wa);
-      load_bundle<BITS>(rb, wb);
-      ra += GB;
-      rb += GB;
+      if constexpr (BITS == 8) {
+        const int sw = g & 7;
+        const uint4 a0 = *reinterpret_cast<const uint4*>(ra + (((2 * t) ^ sw) << 4));
+        const uint4 a1 = *reinterpret_cast<const uint4*>(ra + (((2 * t + 1) ^ sw) << 4));
+        const uint4 b0 = *reinterpret_cast<const uint4*>(ra + 8 * GB + (((2 * t) ^ sw) << 4));
+        const uint4 b1 = *reinterpret_cast<const uint4*>(ra + 8 * GB + (((2 * t + 1) ^ sw) << 4));
+        wa[0] = a0.x; wa[1] = a0.y; wa[2] = a0.z; wa[3] = a0.w;
+        wa[4] = a1.x; wa[5] = a1.y; wa[6] = a1.z; wa[7] = a1.w;
+        wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w;
+        wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
+      } else {
+        load_bundle<BITS>(ra, wa);
+        load_bundle<BITS>(ra + 8 * GB, wb);
+      }
+      ra += kRows * GB;
       // group scales (the 2^24 subnormal unit is applied once, at the store)
-      const float sa = __half2float(*sca++);
-      const float sb = __half2float(*scb++);
+      float sa, sb;
+      if constexpr (G >= 8) {
+        const uint32_t si = (g0 & 7u) + j;
+        const uint8_t* s0 = sc + (si >> 3) * (kRows * 16) + (si & 7u) * 2;
+        sa = __half2float(*reinterpret_cast<const __half*>(s0 + g * 16));
+        sb = __half2float(*reinterpret_cast<const __half*>(s0 + (g + 8) * 16));
+      } else {
+        const uint8_t* s0 = sc + (g0 + j) * 2;
+        sa = __half2float(*reinterpret_cast<const __half*>(s0 + g * G * 2));
+        sb = __half2float(*reinterpret_cast<const __half*>(s0 + (g + 8) * G * 2));
+      }
       const float2 z = *zp;
       zp += 4;
       uint4 bq[4];
@@ -326,6 +348,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     if (ui < u1) issue(slot);
     uc += len;
     ++consumed;
+    if (++slot == NS) {
+      slot = 0;
+      sph ^= 1u;
+    }
 
     if (g0 + len == G || uc >= u1) {
       // ---- this warp's part of the tile is done
@@ -390,7 +416,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host planning
 struct GemvPlan {
-  int CH = 0, NS = 0, stride = 0, slot_bytes = 0, zc_off = 0, ring_off = 0, bar_off = 0;
+  int CH = 0, NS = 0, slot_bytes = 0, zc_off = 0, ring_off = 0, bar_off = 0;
   size_t smem = 0;
 };
 
@@ -410,19 +436,16 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
-  const size_t ring_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 127) & ~static_cast<size_t>(127);
-  const int row = ch * 16 * bits;
-  const int pad_w = ((bank_target_words(bits) - row / 4) % 32 + 32) % 32;
-  const int stride = row + 4 * pad_w;
-  const int sbytes = G >= 8 ? kRows * 32 : ((kRows * G * 2 + 15) & ~15);
-  const int slot = kRows * stride + sbytes;
+  // ring and slots on 1 KiB boundaries (TMA destinations; the 128-byte swizzle atom)
+  const size_t ring_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 1023) & ~static_cast<size_t>(1023);
+  const int sc_bytes = G >= 8 ? 2 * kRows * 16 : ((kRows * G * 2 + 15) & ~15);
+  const int slot = (ch * kRows * 16 * bits + sc_bytes + 1023) & ~1023;
   const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * ns * slot;
-  const size_t smem = bar_off + static_cast<size_t>(kWarps) * ns * 8;
-  // a warp's partial-tile slots (1 KiB) live in its ring
-  if (smem > budget || static_cast<size_t>(ns) * slot < 1024) return pl;
+  // + 1 KiB: the kernel rounds the shared-memory base up to 1 KiB
+  const size_t smem = bar_off + static_cast<size_t>(kWarps) * ns * 8 + 1024;
+  if (smem > budget) return pl;
   pl.CH = ch;
   pl.NS = ns;
-  pl.stride = stride;
   pl.slot_bytes = slot;
   pl.zc_off = static_cast<int>(zc_off);
   pl.ring_off = static_cast<int>(ring_off);
@@ -515,10 +538,23 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int G = a.K / kGroup;
   const uint32_t n_tiles = static_cast<uint32_t>((a.M + kRows - 1) / kRows);
+  GemvParams p{};
+  // codes as a byte matrix [M][K bits / 8], one box = one group x 16 rows
+  // (8-bit rows are 128 bytes: 128-byte swizzle for conflict-free reads)
+  const uint64_t row_bytes = static_cast<uint64_t>(a.K) * a.bits / 8;
+  e = tensor_map_2d(&p.qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q, row_bytes, static_cast<uint64_t>(a.M),
+                    row_bytes, static_cast<uint32_t>(16 * a.bits), kRows,
+                    a.bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (e != cudaSuccess) return e;
+  if (G >= 8) {  // scales [M][G] fp16, one box = 8 groups x 16 rows
+    e = tensor_map_2d(&p.smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.scales, static_cast<uint64_t>(G),
+                      static_cast<uint64_t>(a.M), static_cast<uint64_t>(G) * 2, 8, kRows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+  }
   const uint32_t U = n_tiles * static_cast<uint32_t>(G);
   // one CTA per SM, each owning whole tiles (at least one)
   const uint32_t grid = std::min<uint32_t>(static_cast<uint32_t>(sm_count()), n_tiles);
-  GemvParams p{};
   p.q = a.q;
   p.scales = a.scales;
   p.x = reinterpret_cast<const __half*>(a.x);
@@ -531,7 +567,6 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.U = U;
   p.CH = pl.CH;
   p.NS = pl.NS;
-  p.stride = pl.stride;
   p.slot_bytes = pl.slot_bytes;
   p.zc_off = pl.zc_off;
   p.xg = static_cast<const uint8_t*>(a.xg);

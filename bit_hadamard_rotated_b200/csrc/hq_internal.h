@@ -1,6 +1,7 @@
 // hq_internal.h -- host-side declarations shared by the libhq translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -44,6 +45,14 @@ size_t gemv_scratch_bytes(int K, int nb);
 int sm_count();
 // Two launches: the rotation (prep) and the GEMV.
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
+
+// A 2D tiled TMA tensor map over a row-major [rows][inner] matrix of `dtype`
+// elements (row stride in bytes, a multiple of 16); box = box_inner x box_rows
+// elements; no multicast.  cudaErrorNotSupported if the driver entry point is
+// missing, cudaErrorInvalidValue if the driver rejects the description.
+cudaError_t tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
+                          uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
+                          CUtensorMapSwizzle swizzle);
 
 // Tensor-core path (tcgen05) for larger batches.
 struct TcArgs {
