@@ -55,15 +55,17 @@ constexpr int kDeqWG = 2;         // dequant warpgroups (groups round robin)
 constexpr int kDeqWarps = 4 * kDeqWG;
 constexpr int kProducerWarp = kDeqWarps;
 constexpr int kMmaWarp0 = kDeqWarps + 1;
-constexpr int kMmaWarps = 2;      // issuing threads: one thread issues an MMA per ~60-80 cycles
+constexpr int kMmaWarps = 4;      // issuing threads launched: one issues an MMA per ~60-80 cycles
 constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps) * 32;
 // Phase-parity waits are unambiguous only if a barrier's consecutive phases
 // are waited for by the same agent (it cannot wait for round r + 1 before
 // round r completed): every ring depth is a multiple of the dequant
 // warpgroup count, and the A-stage count a multiple of it and of the MMA
 // warp count.
+// The MMA warps in use (n_mma = 2 or 4) wait for the A stages and ring slots
+// too: the host picks stage counts and ring depths that are multiples of it.
 static_assert(kNSMin % kDeqWG == 0 && kNSMax % kDeqWG == 0 && kASMax % kDeqWG == 0 &&
-                  kMmaWarps == kDeqWG,
+                  kNSMin % kMmaWarps == 0,
               "ring depths must be multiples of the agent counts");
 constexpr int kTmemCols = 512;
 // Tensor memory: accumulator j at columns [j Npad, (j + 1) Npad); A stage s at
@@ -231,8 +233,9 @@ struct TcParams {
   int sbuf_bytes;
   int bar_off;
   int ns;       // shared-memory ring slots (kNSMin..kNSMax)
-  int as;       // A stages in tensor memory (4 or 6)
+  int as;       // A stages in tensor memory (4 or 6; a multiple of n_mma)
   int a_base;   // tensor-memory column of A stage 0
+  int n_mma;    // MMA warps (accumulators) in use: 4 if Npad <= 64, else 2
   uint32_t idesc;
   uint32_t add[16];
 };
@@ -265,9 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       mbar_init(&aready[i], 128);
       mbar_init(&afree[i], 1);
     }
-    mbar_init(dready, kMmaWarps);
+    mbar_init(dready, p.n_mma);
     mbar_init(dfree, kDeqWG * 128);
-    mbar_init(drain, kMmaWarps);
+    mbar_init(drain, p.n_mma);
     mbar_init(&sready[0], 1);
     mbar_init(&sready[1], 1);
     fence_mbar_init();
@@ -345,9 +348,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     }
     __syncwarp();
   } else if (warp >= kMmaWarp0) {
-    // ---------------- MMA issue: warp j takes chunks j, j + kMmaWarps, ...
+    // ---------------- MMA issue: warp j takes chunks j, j + n_mma, ...
     const int j = warp - kMmaWarp0;
-    {
+    if (j < p.n_mma) {
       bool ok = true;
       // B descriptors: the slot-0, slice-0 descriptor plus start-address steps
       // (in 16-byte units; every address stays below 2^18, so the 14-bit
@@ -356,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
       const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
       const uint32_t dacc = tmem + j * p.Npad;
-      const int step = kMmaWarps;  // divides as, ns and G
+      const int step = p.n_mma;  // divides as, ns and G
       int sl = j, st = j, g = j, ti = 0;  // slot (mod ns), A stage (mod as)
       uint32_t aph = 0, sph = 0;          // A-stage and slot round parities
       for (int c = j; c < total && ok; c += step) {
@@ -429,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 #pragma unroll
           for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
         }
-        for (int a = 1; a < kMmaWarps; ++a) {
+        for (int a = 1; a < p.n_mma; ++a) {
           uint32_t v[16];
           tc_ld16(tmem + lane_base + a * p.Npad + c0, v);
           tc_wait_ld();
@@ -705,10 +708,12 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.sbuf_off = pl.sbuf_off;
     p.sbuf_bytes = pl.sbuf_bytes;
     p.bar_off = pl.bar_off;
-    p.ns = pl.ns;
-    p.a_base = (tc::kMmaWarps * npad + 63) & ~63;
-    p.as = ((tc::kTmemCols - p.a_base) / 64) & ~1;
-    if (p.as > tc::kASMax) p.as = tc::kASMax;
+    // accumulators: 4 if they fit in half of tensor memory with 4 A stages
+    p.n_mma = npad <= 64 ? 4 : 2;
+    p.a_base = (p.n_mma * npad + 63) & ~63;
+    p.as = ((tc::kTmemCols - p.a_base) / 64) / p.n_mma * p.n_mma;
+    if (p.as > tc::kASMax) p.as = tc::kASMax / p.n_mma * p.n_mma;
+    p.ns = pl.ns / p.n_mma * p.n_mma;
     p.idesc = tc::idesc_f16(tc::kTileM, npad);
     const dim3 g(grid), blk(tc::kThreads);
     switch (a.bits) {
