@@ -32,7 +32,7 @@ namespace moe {
 constexpr int kRows = 16;
 constexpr int kXq = 40;             // halves per (row, group, k-quad) B block (64 B + pad)
 constexpr float kUnit = 16777216.f;  // 2^24, the subnormal code unit
-constexpr int kWarps = 8;
+constexpr int kWarps = 16;
 
 __host__ __device__ inline int layout_index(int bits) {
   return bits == 2 ? 0 : bits == 3 ? 1 : bits == 4 ? 2 : 3;
@@ -356,7 +356,7 @@ __host__ __device__ inline int chunk_stride(int bits, int len) {
 __host__ __device__ inline int chunk_scale_bytes(int G) {
   return G >= 8 ? kRows * 32 : ((kRows * G * 2 + 15) & ~15);
 }
-constexpr int kChunkBytes = 12 * 1024;
+constexpr int kChunkBytes = 6 * 1024;
 constexpr int kRing = 2;  // slots per warp
 __host__ __device__ inline int chunk_len(int bits, int G, int nmat) {
   for (int len = 8; len > 1; len >>= 1) {
