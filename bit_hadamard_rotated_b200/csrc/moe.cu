@@ -147,6 +147,8 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const hq_expert* __rest
                                                         Dims d, uint32_t* zero_block) {
   pdl_launch_dependents();
   pdl_wait();
+  // first column block of each expert; [E] = total (s_nb0[e+1] - s_nb0[e] = blocks of e)
+  extern __shared__ int s_nb0[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid < 64) zero_block[tid] = 0u;  // B block of lanes without a column
   for (int e = tid; e < d.E; e += blockDim.x) w.counts[e] = 0;
@@ -200,14 +202,9 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const hq_expert* __rest
       }
       if (e < d.E) {
         w.offsets[e] = run + x - cnt;
-        // items of this expert: column blocks x row tiles, block-major
-        const int ia = (run_a + xa - nb) * ta, ib = (run_b + xa - nb) * tb;
-        for (int cb = 0; cb < nb; ++cb) {
-          for (int tl = 0; tl < ta; ++tl)
-            w.items_a[ia + cb * ta + tl] = make_uint2(e, (tl << 16) | cb);
-          for (int tl = 0; tl < tb; ++tl)
-            w.items_b[ib + cb * tb + tl] = make_uint2(e, (tl << 16) | cb);
-        }
+        // first column block of this expert (the items are written below by
+        // all warps: column blocks x row tiles, block-major)
+        s_nb0[e] = run_a + xa - nb;
       }
       run += __shfl_sync(0xffffffffu, x, 31);
       const int tot_nb = __shfl_sync(0xffffffffu, xa, 31);
@@ -218,9 +215,24 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const hq_expert* __rest
       w.offsets[d.E] = run;
       w.n_items[0] = run_a * ta;
       w.n_items[1] = run_b * tb;
+      s_nb0[d.E] = run_a;
     }
   }
   __syncthreads();
+  {
+    // work items, one warp per expert, lanes over the expert's items
+    const int ta = d.inter / kRows, tb = d.hidden / kRows;
+    const int nw = blockDim.x >> 5;
+    for (int e = warp; e < d.E; e += nw) {
+      const int nb0 = s_nb0[e], nb = s_nb0[e + 1] - nb0;
+      for (int i = lane; i < nb * ta; i += 32) {
+        w.items_a[nb0 * ta + i] = make_uint2(e, ((i % ta) << 16) | (i / ta));
+      }
+      for (int i = lane; i < nb * tb; i += 32) {
+        w.items_b[nb0 * tb + i] = make_uint2(e, ((i % tb) << 16) | (i / tb));
+      }
+    }
+  }
   for (int i = tid; i < d.P; i += blockDim.x) {
     const int r = w.pos[i];
     if (r <= -2) {
@@ -606,12 +618,15 @@ static int moe_grid() { return sm_count(); }  // one CTA per SM
 
 using namespace hq;
 
+// The route kernel keeps one int per expert in shared memory.
+constexpr int kMaxExperts = 32768;
+
 extern "C" {
 
 size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k) {
   auto pow2 = [](int v) { return v > 0 && (v & (v - 1)) == 0; };
-  if (n_experts < 1 || T < 0 || k < 1 || k > 32 || !pow2(hidden) || !pow2(inter) ||
-      hidden < 128 || inter < 128 || hidden > 16384 || inter > 16384 ||
+  if (n_experts < 1 || n_experts > kMaxExperts || T < 0 || k < 1 || k > 32 || !pow2(hidden) ||
+      !pow2(inter) || hidden < 128 || inter < 128 || hidden > 16384 || inter > 16384 ||
       static_cast<long>(T) * k > (1L << 24)) {
     return 0;
   }
@@ -630,7 +645,7 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
     return HQ_ERR_INVALID_ARG;
   }
   if (!pow2(hidden) || !pow2(inter) || hidden < 128 || inter < 128 || hidden > 16384 ||
-      inter > 16384) {
+      inter > 16384 || n_experts > kMaxExperts) {
     return HQ_ERR_UNSUPPORTED;
   }
   if (static_cast<long>(T) * k > (1L << 24)) return HQ_ERR_INVALID_ARG;
@@ -648,7 +663,8 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
   uint32_t* zb = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + pl.off[14]);
   const uint4* zb4 = reinterpret_cast<const uint4*>(zb);
   const __half* xh = reinterpret_cast<const __half*>(x);
-  cudaError_t e = launch_pdl(moe::moe_route_kernel, dim3(1), dim3(1024), 0, st, true, experts,
+  cudaError_t e = launch_pdl(moe::moe_route_kernel, dim3(1), dim3(1024),
+                             static_cast<size_t>(n_experts + 1) * sizeof(int), st, true, experts,
                              topk_ids, w, d, zb);
   if (e == cudaSuccess) e = moe_launch_rot_x(hidden, xh, signs_in, w, d, st);
   const size_t psmem = moe::kWarps * moe::kRing * moe::kChunkBytes + moe::kWarps * moe::kRing * 8;

@@ -146,6 +146,7 @@ size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k)
  * topk_ids: [T][k] int32, topk_w: [T][k] fp32.  signs_in [hidden], signs_mid
  * [inter] (NULL = no sign flip).  y: [T][hidden] fp32.
  * hidden, inter: powers of two in [128, 16384].  1 <= k <= 32.
+ * 1 <= n_experts <= 32768 (HQ_ERR_UNSUPPORTED above).
  * An expert id outside [0, n_experts), or an expert whose bits or zero is out
  * of range, is skipped (its contribution is zero) and sets HQ_ERR_DATA in the
  * workspace status word.
