@@ -146,7 +146,7 @@ size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k)
  * topk_ids: [T][k] int32, topk_w: [T][k] fp32.  signs_in [hidden], signs_mid
  * [inter] (NULL = no sign flip).  y: [T][hidden] fp32.
  * hidden, inter: powers of two in [128, 16384].  1 <= k <= 32.
- * 1 <= n_experts <= 32768 (HQ_ERR_UNSUPPORTED above).
+ * 1 <= n_experts <= 16384 (HQ_ERR_UNSUPPORTED above).
  * An expert id outside [0, n_experts), or an expert whose bits or zero is out
  * of range, is skipped (its contribution is zero) and sets HQ_ERR_DATA in the
  * workspace status word.
@@ -204,7 +204,7 @@ uint64_t hq_launch_count(void);
 /* Kernels one hq_linear call enqueues for this weight and batch. */
 int hq_linear_launches(const hq_weight* w, int batch);
 
-/* Kernels one hq_moe_experts call enqueues (route, rotate x, gate/up,
+/* Kernels one hq_moe_experts call enqueues (route + rotate x, gate/up,
  * rotate h, down, combine). */
 int hq_moe_launches(void);
 

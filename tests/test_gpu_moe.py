@@ -94,6 +94,17 @@ def test_moe_with_8bit_experts_and_other_shapes():
     check(y, want, bound, "8-bit mix")
 
 
+@pytest.mark.parametrize("hidden,inter", [(8192, 256), (256, 8192), (4096, 1024), (16384, 128)])
+def test_moe_wide_shapes(hidden, inter):
+    """Widths whose activation fragments do not fit beside the copy rings in
+    shared memory (read from global memory instead), and ones that just fit."""
+    m = synth.moe(seed=11, E=5, hidden=hidden, inter=inter, T=11, k=2, probs=(0.4, 0.3, 0.3),
+                  bits_choices=(2, 3, 4))
+    y, _ = run_moe(m)
+    want, bound, _ = oracle_moe(m)
+    check(y, want, bound, f"hidden {hidden} inter {inter}")
+
+
 def test_moe_expert_with_many_tokens():
     """All 20 tokens choose expert 2 (three column blocks of <= 8 tokens)."""
     m = synth.moe(seed=6, E=4, hidden=256, inter=128, T=20, k=2)
