@@ -270,8 +270,8 @@ def run_ours(a):
                    "parallelism": f"replicas x{world} (weak scaling, no data-path collective)"},
         "frac_hbm": round(value / world / pk["hbm"], 4),
         "roofline": {"bound": "hbm",
-                     "kernel": "gemv_kernel, with its gemv_prep_kernel (one pair per linear; "
-                               "aggregate over the step's three linears)",
+                     "kernel": "gemv_kernel, rotation fused in (one launch per linear at "
+                               "batch 1; aggregate over the step's three linears)",
                      "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
                      "frac": round(achieved / pk["hbm"], 4), "traffic": None,
                      "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},

@@ -619,6 +619,21 @@ cudaError_t tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const voi
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                          const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
+                          const uint32_t (&box)[3], CUtensorMapSwizzle swizzle) {
+  tc::EncodeTiled fn = tc::encode_tiled();
+  if (fn == nullptr) return cudaErrorNotSupported;
+  const cuuint64_t d[3] = {dims[0], dims[1], dims[2]};
+  const cuuint64_t st[2] = {strides_bytes[0], strides_bytes[1]};
+  const cuuint32_t b[3] = {box[0], box[1], box[2]};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, dtype, 3, const_cast<void*>(base), d, st, b, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 int tc_col_block(int bits, int K) {
   // K >= 1024: whole 16-byte scale rows, and >= 8 groups per tile (a tile's
   // scale buffer is refilled only after the MMAs two tiles back are done)

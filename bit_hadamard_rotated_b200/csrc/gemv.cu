@@ -1,5 +1,5 @@
 // gemv.cu -- unpack-dequant GEMV over packed low-bit codes, batch <= 8 per
-// launch, with the rotation of the activations in a small prep kernel.
+// launch, with the rotation of the activations fused in or in a prep kernel.
 //
 //   y[n][m] = sum_k scale[m][k/128] (q[m][k] - zero) x'[n][k],
 //   x'[n]   = H_K diag(s) x[n] / sqrt(K).
@@ -9,20 +9,23 @@
 // GEMV is shaped to stream packed codes at HBM rate with all dequantisation
 // on chip:
 //
-//   * gemv_prep_kernel (one CTA per batch row) rotates x in fp32 (fwht.cuh)
-//     and writes x' as fp16 in the order of the MMA B fragments, each value
+//   * The rotation x' = H diag(s) x / sqrt(K) runs in fp32 (fwht.cuh), and x'
+//     is written as fp16 in the order of the MMA B fragments, each value
 //     scaled by the 2^-a of its code field (hq_layout.cuh), plus the
-//     zero-point term -zero * sum_k x'_k * 2^-24 of each group.
+//     zero-point term -zero * sum_k x'_k * 2^-24 of each group: for one or
+//     two rows of K <= 8192 by every GEMV CTA itself, after its first weight
+//     copies are on their way (one launch per call); otherwise by
+//     gemv_prep_kernel (one CTA per batch row) before the GEMV.
 //   * gemv_kernel: persistent grid, one 16-warp CTA per SM.  The work is the
 //     list of (16-row tile, 128-code group) units; each CTA owns a contiguous
 //     range of whole tiles and its warps split that range evenly.
 //   * Each warp streams its range through a private ring of shared-memory
-//     slots of about 4 KiB of codes (CH groups of 16 rows at a bank-conflict-
-//     free stride, plus scales), moved by 16-byte cp.async copies that
-//     complete on one mbarrier per slot.  The first slots are requested
+//     slots of about 4 KiB of codes (CH groups of 16 rows, plus scales),
+//     moved by TMA copies issued by lane 0 that complete on one mbarrier per
+//     slot (transaction bytes).  The first slots are requested
 //     before griddepcontrol.wait: weights do not depend on earlier kernels.
-//     After the wait, the CTA copies the prep kernel's fragments into shared
-//     memory.
+//     Full slots of codes arrive as one 3-D TMA box ([CH groups][16 rows]
+//     [16 bits bytes]), a slot's scales as one or two 2-D boxes.
 //   * Per group: each lane masks 2 x 32 codes into exact subnormal fp16 pairs
 //     (one LOP3/PRMT per pair), runs 8 mma.sync m16n8k16 with fp32
 //     accumulation in two chains (one starting at the zero-point term), then
@@ -52,6 +55,7 @@ constexpr float kUnit = 16777216.f;
 
 struct GemvParams {
   CUtensorMap qmap;  // codes as bytes [M][K bits / 8]; box 16 bits bytes x 16 rows
+  CUtensorMap qmap3;  // the same as [G][M][16 bits bytes]; box CH groups x 16 rows (a full slot)
   CUtensorMap smap;  // scales as fp16 [M][K/128]; box 8 x 16 rows (K >= 1024 only)
   const uint32_t* q;
   const uint16_t* scales;
@@ -60,11 +64,18 @@ struct GemvParams {
   float* y;
   uint32_t* status;
   int M, N, ldy;
-  uint32_t U;  // units = n_tiles * G
+  uint32_t U;       // units = n_tiles * G
+  uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
   int zero;
   const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, then zc [G][8] fp32
-  int CH, NS, slot_bytes, zc_off, ring_off, bar_off;
+  float inv_sqrt_k;
+  int CH, NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
 };
+
+// Batches whose rotation the GEMV CTAs compute themselves (no prep launch):
+// a row or two of at most 8192 values, a few microseconds of fp32 work that
+// overlaps the first weight copies.
+__host__ __device__ constexpr bool gemv_fused_rotation(int K, int nb) { return nb <= 2 && K <= 8192; }
 
 // Bytes of the prep output for a batch block of nb columns (16-byte multiple).
 __host__ __device__ constexpr size_t gemv_xs_bytes(int G, int nb) {
@@ -74,11 +85,54 @@ __host__ __device__ constexpr size_t gemv_xg_bytes(int G, int nb) {
   return gemv_xs_bytes(G, nb) + static_cast<size_t>(G) * 8 * 4;
 }
 
-// ---------------------------------------------------------------- prep: rotate once per call
-// CTA n rotates activation row n in fp32, rounds x' to fp16, and writes it in
-// the order of the MMA B fragments, each value scaled by the 2^-a of its code
-// field, plus the zero-point term -zero * sum_k x'_k * 2^-24 of each group;
-// CTA 0 also zeroes the zero-point terms of the absent columns (N..7).
+// ---------------------------------------------------------------- rotation -> B fragments
+// Lane (s, t) of a warp writes the B-fragment quad of step s for k-quad t:
+// the code fields (columns kc, exponent offsets ka) of its four values.
+template <int BITS>
+struct FragLane {
+  int kc[4], ka[4];
+  __device__ __forceinline__ explicit FragLane(int lane) {
+    const int s = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const PairDesc pd = Pairs<BITS>::get(2 * s + (r >> 1));
+      kc[r] = 32 * t + ((r & 1) ? pd.c_hi : pd.c_lo);
+      ka[r] = (r & 1) ? pd.a_hi : pd.a_lo;
+    }
+  }
+};
+
+// Group gg of a rotated row (buf: unnormalised fwht_block output): x' rounded
+// to fp16, each value scaled by the 2^-a of its code field, written as column
+// n of the fragment blocks xs [G][nb][4][kXq]; zc[gg * 8 + n] = the zero-point
+// term -zero * sum_k x'_k * 2^-24 of the group.  One warp per group.
+template <int BITS>
+__device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float* buf, int gg, int n,
+                                          int nb, float inv_sqrt_k, int zero, uint16_t* xs,
+                                          float* zc, int lane) {
+  const int s = lane >> 2, t = lane & 3;
+  uint16_t hv[4];
+  float part = 0.f;
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + fl.kc[r])] * inv_sqrt_k));
+    const __half b = __float2half_rn(xv * __int_as_float((127 - fl.ka[r]) << 23));
+    hv[r] = __half_as_ushort(b);
+    part += __half2float(b) * __int_as_float((127 + fl.ka[r]) << 23);
+  }
+#pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
+  uint2 pk;
+  pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
+  pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
+  *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * nb + n) * 4 + t) * kXq + s * 4) = pk;
+  if (lane == 0) zc[gg * 8 + n] = -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
+}
+
+// Prep kernel (batches the GEMV CTAs do not rotate themselves): CTA n rotates
+// activation row n in fp32 and writes its fragments and zero-point terms to
+// global memory; CTA 0 also zeroes the zero-point terms of the absent columns
+// (N..7).
 template <int BITS, int LOGK>
 __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half* __restrict__ x,
                                                                  const int8_t* __restrict__ signs,
@@ -91,17 +145,9 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
   pdl_launch_dependents();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = blockIdx.x;
-  const int s = lane >> 2, t = lane & 3;
   uint16_t* xs = reinterpret_cast<uint16_t*>(xg);
   float* zc = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
-  // lane (s, t) writes the B-fragment quad of step s for k-quad t
-  int kc[4], ka[4];
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const PairDesc pd = Pairs<BITS>::get(2 * s + (r >> 1));
-    kc[r] = 32 * t + ((r & 1) ? pd.c_hi : pd.c_lo);
-    ka[r] = (r & 1) ? pd.a_hi : pd.a_lo;
-  }
+  const FragLane<BITS> fl(lane);
   pdl_wait();  // x is the previous kernel's output; xg may still be read by it
   if (n == 0) {
     for (int i = tid; i < G * (8 - N); i += kPrepWarps * 32) zc[(i / (8 - N)) * 8 + N + i % (8 - N)] = 0.f;
@@ -112,37 +158,15 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
     apply_signs<FS::E>(signs ? signs + tid * FS::E : nullptr, v);
   }
   fwht_block<LOGK, 3>(v, buf);
-  for (int gg = warp; gg < G; gg += kPrepWarps) {
-    uint16_t hv[4];
-    float part = 0.f;
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + kc[r])] * inv_sqrt_k));
-      const __half b = __float2half_rn(xv * __int_as_float((127 - ka[r]) << 23));
-      hv[r] = __half_as_ushort(b);
-      part += __half2float(b) * __int_as_float((127 + ka[r]) << 23);
-    }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) part += __shfl_xor_sync(0xffffffffu, part, m);
-    uint2 pk;
-    pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
-    pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
-    *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * N + n) * 4 + t) * kXq + s * 4) = pk;
-    if (lane == 0) zc[gg * 8 + n] = -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
-  }
+  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, inv_sqrt_k, zero, xs, zc, lane);
 }
 
 // Splitting U units into n contiguous ranges: range i is [unit_begin(i), unit_begin(i + 1)).
 __device__ __forceinline__ uint32_t unit_begin(uint32_t i, uint32_t U, uint32_t n) {
   return static_cast<uint32_t>((static_cast<uint64_t>(i) * U) / n);
 }
-// The range that contains unit u (the last of several starting at the same
-// unit: the earlier ones are empty).
-__device__ __forceinline__ uint32_t unit_owner(uint32_t u, uint32_t U, uint32_t n) {
-  return static_cast<uint32_t>((static_cast<uint64_t>(u) * n + n - 1) / U);
-}
 
-template <int BITS, int LOGK>
+template <int BITS, int LOGK, bool FUSED>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
@@ -153,12 +177,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
-  // the CTA owns whole tiles, units [cb, ce); its warps split them into
-  // contiguous ranges (a tile is never shared with another CTA)
-  const uint32_t GC = gridDim.x;
-  const uint32_t n_tiles = p.U / G;
-  const uint32_t cb = unit_begin(blockIdx.x, n_tiles, GC) * G;
-  const uint32_t ce = unit_begin(blockIdx.x + 1, n_tiles, GC) * G;
+  // the CTA owns whole tiles, units [cb, ce): the first tr CTAs tq + 1
+  // tiles, the others tq; its warps split them into contiguous ranges (a
+  // tile is never shared with another CTA: a cross-CTA sum would put global
+  // memory round trips at the end of every CTA)
+  const uint32_t c = blockIdx.x;
+  const uint32_t cb = (c * p.tq + min(c, p.tr)) * G;
+  const uint32_t ce = cb + (p.tq + (c < p.tr ? 1u : 0u)) * G;
   const uint32_t cl = ce - cb;
   const uint32_t u0 = cb + unit_begin(warp, cl, kWarps);
   const uint32_t u1 = cb + unit_begin(warp + 1, cl, kWarps);
@@ -172,6 +197,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   // groups][16 rows][8 halves]; K < 1024: the tile's [16 rows][G halves]
   const int sc_off = p.CH * kRows * GB;
 
+  if (tid == 0) {
+    prefetch_tensormap(&p.qmap3);
+    prefetch_tensormap(&p.qmap);
+    if constexpr (G >= 8) prefetch_tensormap(&p.smap);
+  }
   if (lane == 0) {
     for (int i = 0; i < p.NS; ++i) mbar_init(&bars[i], 1);
     fence_mbar_init();
@@ -212,8 +242,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         mbar_arrive_expect_tx(&bars[slot], bytes);
         if (bulk > 0) bulk_g2s(base + sc_off, src, bulk, &bars[slot]);
       }
-      for (uint32_t j = 0; j < len; ++j) {
-        tma_load_2d(base + j * kRows * GB, &p.qmap, static_cast<int>((g0 + j) * GB), m0, &bars[slot]);
+      if (len == static_cast<uint32_t>(p.CH)) {
+        tma_load_3d(base, &p.qmap3, 0, m0, static_cast<int>(g0), &bars[slot]);
+      } else {
+        for (uint32_t j = 0; j < len; ++j) {
+          tma_load_2d(base + j * kRows * GB, &p.qmap, static_cast<int>((g0 + j) * GB), m0, &bars[slot]);
+        }
       }
     }
     ui += len;
@@ -221,9 +255,53 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   };
   for (int s = 0; s < p.NS && ui < u1; ++s) issue(s);
 
-  // ---- the rotated activations and zero-point terms (from the prep kernel)
-  pdl_wait();
-  {
+  // ---- the rotated activations and zero-point terms
+  if constexpr (FUSED) {
+    // rotate each row here (the fwht_block shape of the prep kernel, so the
+    // values are the same bit for bit) while the first slots are in flight;
+    // the signs are weights, read before the wait
+    using FS = FwhtShape<LOGK, 3>;
+    static_assert(FS::E <= 32, "one sign bit per register");
+    uint32_t neg = 0;  // bit e: value e of this thread's chunk flips sign
+    if (tid < FS::THREADS && p.signs != nullptr) {
+      const int8_t* sp = p.signs + tid * FS::E;
+      if constexpr (FS::E % 16 == 0) {
+#pragma unroll
+        for (int e = 0; e < FS::E; e += 16) {
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(sp + e));
+          const int8_t* b = reinterpret_cast<const int8_t*>(&u);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) neg |= (b[j] < 0 ? 1u : 0u) << (e + j);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < FS::E; ++e) neg |= (sp[e] < 0 ? 1u : 0u) << e;
+      }
+    }
+    float* buf = reinterpret_cast<float*>(smem + p.buf_off);
+    const FragLane<BITS> fl(lane);
+    for (int i = tid; i < G * 8; i += kWarps * 32) {
+      if ((i & 7) >= p.N) zc[i] = 0.f;  // absent columns
+    }
+    pdl_wait();
+    for (int n = 0; n < p.N; ++n) {
+      float v[FS::E];
+      if (tid < FS::THREADS) {
+        load_chunk<__half, FS::E>(p.x + static_cast<size_t>(n) * K + tid * FS::E, v);
+#pragma unroll
+        for (int e = 0; e < FS::E; ++e) v[e] = (neg >> e & 1u) ? -v[e] : v[e];
+      }
+      fwht_block<LOGK, 3>(v, buf);
+      for (int gg = warp; gg < G; gg += kWarps) {
+        put_group<BITS>(fl, buf, gg, n, p.N, p.inv_sqrt_k, p.zero, xs, zc, lane);
+      }
+      __syncthreads();  // buf is reused by the next row; xs and zc are complete
+    }
+    if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;  // zero B block
+    __syncthreads();
+  } else {
+    // from the prep kernel
+    pdl_wait();
     const int xs_bytes = static_cast<int>(gemv_xs_bytes(G, p.N));
     for (int i = tid * 16; i < xs_bytes; i += kWarps * 32 * 16) {
       cp_async16(smem + i, p.xg + i, 16);
@@ -391,14 +469,16 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (tl < 0 || (which == 1 && tl == ptile0)) continue;
       const uint32_t tile = static_cast<uint32_t>(tl);
       const uint32_t tf = tile * G, tz = tile * G + G - 1;
-      if (unit_owner(tf - cb, cl, kWarps) != static_cast<uint32_t>(warp)) continue;
-      const uint32_t wz = unit_owner(tz - cb, cl, kWarps);
-      float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (uint32_t w = warp; w <= wz; ++w) {
+      // the ranges are contiguous: the warp whose range holds the tile's
+      // first unit adds; the later contributors are the next non-empty
+      // warps whose ranges start inside the tile (the tile is their first)
+      if (tf < u0) continue;
+      float4 o = which == 0 ? psum0 : psum1;
+      for (uint32_t w = warp + 1; w < static_cast<uint32_t>(kWarps); ++w) {
         const uint32_t wb = cb + unit_begin(w, cl, kWarps);
+        if (wb > tz) break;
         if (wb == cb + unit_begin(w + 1, cl, kWarps)) continue;  // empty range
-        const int ww = (tile == wb / G) ? 0 : 1;
-        const float4 q4 = *sp_slot(w, ww);
+        const float4 q4 = *sp_slot(w, 0);
         o.x += q4.x;
         o.y += q4.y;
         o.z += q4.z;
@@ -416,7 +496,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host planning
 struct GemvPlan {
-  int CH = 0, NS = 0, slot_bytes = 0, zc_off = 0, ring_off = 0, bar_off = 0;
+  int CH = 0, NS = 0, slot_bytes = 0, zc_off = 0, buf_off = 0, ring_off = 0, bar_off = 0;
   size_t smem = 0;
 };
 
@@ -436,8 +516,11 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
+  // the FWHT buffer of a fused rotation: K floats + one pad word per 32
+  const size_t buf_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 15) & ~static_cast<size_t>(15);
+  const size_t buf = gemv_fused_rotation(K, nb) ? (static_cast<size_t>(K) + K / 32) * 4 : 0;
   // ring and slots on 1 KiB boundaries (TMA destinations; the 128-byte swizzle atom)
-  const size_t ring_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 1023) & ~static_cast<size_t>(1023);
+  const size_t ring_off = (buf_off + buf + 1023) & ~static_cast<size_t>(1023);
   const int sc_bytes = G >= 8 ? 2 * kRows * 16 : ((kRows * G * 2 + 15) & ~15);
   const int slot = (ch * kRows * 16 * bits + sc_bytes + 1023) & ~1023;
   const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * ns * slot;
@@ -448,6 +531,7 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   pl.NS = ns;
   pl.slot_bytes = slot;
   pl.zc_off = static_cast<int>(zc_off);
+  pl.buf_off = static_cast<int>(buf_off);
   pl.ring_off = static_cast<int>(ring_off);
   pl.bar_off = static_cast<int>(bar_off);
   pl.smem = smem;
@@ -482,22 +566,34 @@ int sm_count() {
   return sms;
 }
 
-template <int BITS>
-static cudaError_t gemv_launch_b(int K, GemvParams& p, size_t smem, unsigned grid,
+template <int BITS, bool FUSED>
+static cudaError_t gemv_launch_f(int K, GemvParams& p, size_t smem, unsigned grid,
                                  cudaStream_t st) {
   const dim3 g(grid), b(kWarps * 32);
   switch (K) {
-    case 128: return launch_pdl(gemv_kernel<BITS, 7>, g, b, smem, st, true, p);
-    case 256: return launch_pdl(gemv_kernel<BITS, 8>, g, b, smem, st, true, p);
-    case 512: return launch_pdl(gemv_kernel<BITS, 9>, g, b, smem, st, true, p);
-    case 1024: return launch_pdl(gemv_kernel<BITS, 10>, g, b, smem, st, true, p);
-    case 2048: return launch_pdl(gemv_kernel<BITS, 11>, g, b, smem, st, true, p);
-    case 4096: return launch_pdl(gemv_kernel<BITS, 12>, g, b, smem, st, true, p);
-    case 8192: return launch_pdl(gemv_kernel<BITS, 13>, g, b, smem, st, true, p);
-    case 16384: return launch_pdl(gemv_kernel<BITS, 14>, g, b, smem, st, true, p);
-    default: return cudaErrorInvalidValue;
+    case 128: return launch_pdl(gemv_kernel<BITS, 7, FUSED>, g, b, smem, st, true, p);
+    case 256: return launch_pdl(gemv_kernel<BITS, 8, FUSED>, g, b, smem, st, true, p);
+    case 512: return launch_pdl(gemv_kernel<BITS, 9, FUSED>, g, b, smem, st, true, p);
+    case 1024: return launch_pdl(gemv_kernel<BITS, 10, FUSED>, g, b, smem, st, true, p);
+    case 2048: return launch_pdl(gemv_kernel<BITS, 11, FUSED>, g, b, smem, st, true, p);
+    case 4096: return launch_pdl(gemv_kernel<BITS, 12, FUSED>, g, b, smem, st, true, p);
+    case 8192: return launch_pdl(gemv_kernel<BITS, 13, FUSED>, g, b, smem, st, true, p);
+    default:
+      if constexpr (!FUSED) {
+        if (K == 16384) return launch_pdl(gemv_kernel<BITS, 14, false>, g, b, smem, st, true, p);
+      }
+      return cudaErrorInvalidValue;
   }
 }
+
+template <int BITS>
+static cudaError_t gemv_launch_b(int K, int nb, GemvParams& p, size_t smem, unsigned grid,
+                                 cudaStream_t st) {
+  return gemv_fused_rotation(K, nb) ? gemv_launch_f<BITS, true>(K, p, smem, grid, st)
+                                    : gemv_launch_f<BITS, false>(K, p, smem, grid, st);
+}
+
+int gemv_launches(int K, int nb) { return gemv_fused_rotation(K, nb) ? 1 : 2; }
 
 size_t gemv_scratch_bytes(int K, int nb) { return gemv_xg_bytes(K / kGroup, nb); }
 
@@ -527,15 +623,18 @@ static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   const GemvPlan pl = gemv_plan(a.bits, a.K, a.N);
   if (pl.smem == 0) return cudaErrorInvalidValue;
-  cudaError_t e;
-  switch (a.bits) {
-    case 2: e = gemv_prep_b<2>(a.K, a, st); break;
-    case 3: e = gemv_prep_b<3>(a.K, a, st); break;
-    case 4: e = gemv_prep_b<4>(a.K, a, st); break;
-    case 8: e = gemv_prep_b<8>(a.K, a, st); break;
-    default: return cudaErrorInvalidValue;
+  const bool fused = gemv_fused_rotation(a.K, a.N);
+  cudaError_t e = cudaSuccess;
+  if (!fused) {
+    switch (a.bits) {
+      case 2: e = gemv_prep_b<2>(a.K, a, st); break;
+      case 3: e = gemv_prep_b<3>(a.K, a, st); break;
+      case 4: e = gemv_prep_b<4>(a.K, a, st); break;
+      case 8: e = gemv_prep_b<8>(a.K, a, st); break;
+      default: return cudaErrorInvalidValue;
+    }
+    if (e != cudaSuccess) return e;
   }
-  if (e != cudaSuccess) return e;
   const int G = a.K / kGroup;
   const uint32_t n_tiles = static_cast<uint32_t>((a.M + kRows - 1) / kRows);
   GemvParams p{};
@@ -546,6 +645,18 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
                     row_bytes, static_cast<uint32_t>(16 * a.bits), kRows,
                     a.bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
   if (e != cudaSuccess) return e;
+  {
+    // the same bytes viewed as [G][M][16 bits] (group stride 16 bits bytes):
+    // one box = a full slot of CH groups x 16 rows, laid out [CH][16][16 bits]
+    const uint64_t gb = 16ull * a.bits;
+    const uint64_t dims[3] = {gb, static_cast<uint64_t>(a.M), static_cast<uint64_t>(G)};
+    const uint64_t strides[2] = {row_bytes, gb};
+    const uint32_t box[3] = {static_cast<uint32_t>(gb), static_cast<uint32_t>(kRows),
+                             static_cast<uint32_t>(pl.CH)};
+    e = tensor_map_3d(&p.qmap3, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q, dims, strides, box,
+                      a.bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+  }
   if (G >= 8) {  // scales [M][G] fp16, one box = 8 groups x 16 rows
     e = tensor_map_2d(&p.smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.scales, static_cast<uint64_t>(G),
                       static_cast<uint64_t>(a.M), static_cast<uint64_t>(G) * 2, 8, kRows,
@@ -565,19 +676,23 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.N = a.N;
   p.ldy = a.ldy;
   p.U = U;
+  p.tq = n_tiles / grid;
+  p.tr = n_tiles % grid;
   p.CH = pl.CH;
   p.NS = pl.NS;
   p.slot_bytes = pl.slot_bytes;
   p.zc_off = pl.zc_off;
+  p.buf_off = pl.buf_off;
+  p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = a.zero;
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;
   switch (a.bits) {
-    case 2: return gemv_launch_b<2>(a.K, p, pl.smem, grid, st);
-    case 3: return gemv_launch_b<3>(a.K, p, pl.smem, grid, st);
-    case 4: return gemv_launch_b<4>(a.K, p, pl.smem, grid, st);
-    case 8: return gemv_launch_b<8>(a.K, p, pl.smem, grid, st);
+    case 2: return gemv_launch_b<2>(a.K, a.N, p, pl.smem, grid, st);
+    case 3: return gemv_launch_b<3>(a.K, a.N, p, pl.smem, grid, st);
+    case 4: return gemv_launch_b<4>(a.K, a.N, p, pl.smem, grid, st);
+    case 8: return gemv_launch_b<8>(a.K, a.N, p, pl.smem, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }

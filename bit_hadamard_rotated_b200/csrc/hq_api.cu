@@ -134,7 +134,9 @@ int hq_linear_launches(const hq_weight* w, int batch) {
   if (use_tc(w, batch)) return tc_launches(w->bits, w->K, batch);
   const int nb = gemv_col_block(w->bits, w->K);
   if (nb == 0) return 0;
-  return 2 * ((batch + nb - 1) / nb);  // prep + GEMV per batch block
+  int n = 0;
+  for (int n0 = 0; n0 < batch; n0 += nb) n += gemv_launches(w->K, std::min(nb, batch - n0));
+  return n;
 }
 
 hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, void* workspace,

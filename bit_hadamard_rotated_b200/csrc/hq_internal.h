@@ -43,8 +43,10 @@ size_t gemv_smem_bytes(int bits, int K, int nb);
 size_t gemv_scratch_bytes(int K, int nb);
 // Streaming multiprocessors of the current device (148 if the query fails).
 int sm_count();
-// Two launches: the rotation (prep) and the GEMV.
+// One GEMV launch, preceded by a rotation (prep) launch unless the GEMV CTAs
+// rotate the batch themselves (gemv_launches tells which: 1 or 2).
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
+int gemv_launches(int K, int nb);
 
 // A 2D tiled TMA tensor map over a row-major [rows][inner] matrix of `dtype`
 // elements (row stride in bytes, a multiple of 16); box = box_inner x box_rows
@@ -53,6 +55,11 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st);
 cudaError_t tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base, uint64_t inner,
                           uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner, uint32_t box_rows,
                           CUtensorMapSwizzle swizzle);
+// The same over a 3-D view: dims and box innermost first, byte strides of
+// dims 1 and 2 (each a multiple of 16; they need not increase).
+cudaError_t tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
+                          const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
+                          const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
 
 // Tensor-core path (tcgen05) for larger batches.
 struct TcArgs {

@@ -72,12 +72,21 @@ struct Pairs<3> {
   // 96-bit triplet, code c at stream bits [3c, 3c+3).  Seven shifted views
   // of the triplet each expose two or three (lo, hi) pairs whose fields lie
   // in mantissa slots: lo within bits 0..9, hi within bits 16..25.
+  // (c_lo, a_lo, c_hi, a_hi) of the 16 pairs:
+  //   (0,1,5,0) (1,4,6,3) (2,7,7,6) (3,1,8,0) (4,4,9,3) (10,0,16,2) (11,3,17,5)
+  //   (12,0,18,2) (13,3,19,5) (14,0,20,2) (15,3,21,5) (22,1,27,0) (23,4,28,3)
+  //   (24,7,29,6) (25,1,30,0) (26,4,31,3)
+  // packed 16 bits each (c_lo | a_lo << 5 | c_hi << 8 | a_hi << 13), four per
+  // word and selected without an array, so that a lookup at a run-time index
+  // stays in registers.
   static __host__ __device__ constexpr PairDesc get(int p) {
-    constexpr uint8_t t[16][4] = {{0, 1, 5, 0},   {1, 4, 6, 3},   {2, 7, 7, 6},   {3, 1, 8, 0},
-                                  {4, 4, 9, 3},   {10, 0, 16, 2}, {11, 3, 17, 5}, {12, 0, 18, 2},
-                                  {13, 3, 19, 5}, {14, 0, 20, 2}, {15, 3, 21, 5}, {22, 1, 27, 0},
-                                  {23, 4, 28, 3}, {24, 7, 29, 6}, {25, 1, 30, 0}, {26, 4, 31, 3}};
-    return PairDesc{t[p][0], t[p][1], t[p][2], t[p][3]};
+    const uint64_t w = (p >> 2) == 0   ? 0x0823c7e266810520ull
+                       : (p >> 2) == 1 ? 0x520cb16b500a6984ull
+                       : (p >> 2) == 2 ? 0x1b36b56f540eb36dull
+                                       : 0x7f9a1e39ddf87c97ull;
+    const uint32_t e = static_cast<uint32_t>(w >> (16 * (p & 3))) & 0xffffu;
+    return PairDesc{static_cast<uint8_t>(e & 31u), static_cast<uint8_t>((e >> 5) & 7u),
+                    static_cast<uint8_t>((e >> 8) & 31u), static_cast<uint8_t>((e >> 13) & 7u)};
   }
 };
 

@@ -187,6 +187,40 @@ def test_linear_output_overwritten_not_accumulated():
     assert_within(y, want, bound, what="overwrite")
 
 
+@pytest.mark.parametrize("bits,M,K,N", [(2, 2400, 1024, 1), (3, 4100, 512, 2), (8, 2376, 2048, 3),
+                                         (4, 4739, 256, 8), (2, 2368, 4096, 1)])
+def test_linear_uneven_tiles_per_cta_all_rows(bits, M, K, N):
+    """Enough 16-row tiles that CTAs own different numbers of them, some tiles
+    split between warps: every row is checked, and a repeat call on the same
+    workspace is bit-identical."""
+    from bit_hadamard_rotated_b200 import hq
+    d = synth.linear(M, K, bits, N, seed=M + K)
+    q, sc, sg, x = dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]), dev(d["x"])
+    need = hq.hq_linear_workspace_size(hq.make_weight(q, sc, sg, bits, d["zero"]), N)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    y1 = hq.hq_linear(q, sc, sg, x, bits, d["zero"], workspace=ws)
+    y2 = hq.hq_linear(q, sc, sg, x, bits, d["zero"], workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y1.cpu().numpy(), want, bound, what=f"b{bits} M{M} K{K} N{N}")
+
+
+def test_linear_workspace_shared_by_paths_and_batches():
+    """One workspace serves GEMV calls of several batches and tensor-core calls
+    in between (results match the oracle each time)."""
+    from bit_hadamard_rotated_b200 import hq
+    d = synth.linear(2400, 2048, 2, 64, seed=21)
+    q, sc, sg = dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"])
+    w = hq.make_weight(q, sc, sg, 2, d["zero"])
+    ws = torch.zeros(max(hq.hq_linear_workspace_size(w, n) for n in (1, 3, 64)), dtype=torch.uint8,
+                     device="cuda")
+    want, bound = oracle.linear(2, 2400, 2048, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    for n in (1, 64, 3, 1, 64, 2):
+        y = hq.hq_linear(q, sc, sg, dev(d["x"][:n]), 2, d["zero"], workspace=ws).cpu().numpy()
+        assert_within(y, want[:n], bound[:n], what=f"batch {n}")
+
+
 # ---------------------------------------------------------------- linear, full workload sizes (sampled rows)
 def sample_rows(M, rng, n=24):
     rows = set(range(0, 8)) | set(range(M - 8, M)) | set(rng.choice(M, n, replace=False).tolist())
