@@ -67,6 +67,10 @@ constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps) * 32;
 static_assert(kNSMin % kDeqWG == 0 && kNSMax % kDeqWG == 0 && kASMax % kDeqWG == 0 &&
                   kNSMin % kMmaWarps == 0,
               "ring depths must be multiples of the agent counts");
+// CTA chunk ranges are whole quanta of kQuant chunks, so every tile portion a
+// CTA computes holds a chunk of every MMA warp and dequant warpgroup.
+constexpr int kQuant = 4;
+static_assert(kQuant % kMmaWarps == 0 && kQuant % kDeqWG == 0, "quantum");
 constexpr int kTmemCols = 512;
 // Tensor memory: accumulator j at columns [j Npad, (j + 1) Npad); A stage s at
 // a_base + 64 s, a_base = 2 Npad rounded up to 64; as many stages as fit,
@@ -227,6 +231,12 @@ struct TcParams {
   uint32_t* status;
   int M, K, N, Npad, ldy;
   int n_tiles;
+  // Chunks (tile-major, 128-code groups inner) in quanta of kQuant: CTA c
+  // owns quanta [c qq + min(c, qr), +qq + (c < qr)); qq kQuant >= G, so a tile
+  // is shared by at most two CTAs.
+  int qq, qr;
+  float* part;      // [grid][2 sides][128 rows][Npad]: shared tiles' partial sums
+  uint32_t* flags;  // [grid]: arrivals at each CTA boundary, zero between calls
   int slot_bytes;  // codes + B block
   int b_off;       // B block offset inside a slot
   int sbuf_off;    // per-tile scale buffers (two)
@@ -258,6 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   uint64_t* drain = dfree + 1;
   uint64_t* sready = drain + 1;  // [2]: a tile's scales landed in buffer ti & 1
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sready + 2);
+  uint32_t* arrival = tmem_holder + 1;  // the epilogue's boundary-counter result
+  // the dequant threads' own barrier (shared-tile epilogues), 8-byte aligned
+  uint64_t* epib = reinterpret_cast<uint64_t*>(tmem_holder + 2);
 
   if (tid == 0) {
     for (int i = 0; i < p.ns; ++i) {
@@ -273,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     mbar_init(drain, p.n_mma);
     mbar_init(&sready[0], 1);
     mbar_init(&sready[1], 1);
+    mbar_init(epib, kDeqWarps * 32);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
@@ -283,11 +297,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   pdl_launch_dependents();
   pdl_wait();
 
-  const int n_my = (p.n_tiles - static_cast<int>(blockIdx.x) + gridDim.x - 1) / gridDim.x;
-  const int total = n_my * G;
-  auto tile_m0 = [&](int ti) {
-    return (static_cast<int>(blockIdx.x) + ti * static_cast<int>(gridDim.x)) * kTileM;
-  };
+  // this CTA's chunks [cb, cb + total); local tile ti is tile tile0 + ti,
+  // the first starting at group g_start (a multiple of kQuant)
+  const int cta = static_cast<int>(blockIdx.x);
+  const int cb = (cta * p.qq + min(cta, p.qr)) * kQuant;
+  const int total = (p.qq + (cta < p.qr ? 1 : 0)) * kQuant;
+  const int tile0 = cb / G, g_start = cb - tile0 * G;
+  const int last_ti = (g_start + total - 1) / G;
+  auto tile_m0 = [&](int ti) { return (tile0 + ti) * kTileM; };
 
   if (warp == kProducerWarp) {
     // ---------------- producer (one thread): TMA + bulk copies into the ring
@@ -297,11 +314,11 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       bool ok = true;
       int issued = 0;
       // ring position kept incrementally (no divisions on the issue path)
-      int sl = 0, g = 0;
+      int sl = 0, g = g_start;
       uint32_t rph = 0;  // parity of the ring round of chunk c
       int m0 = tile_m0(0), ti = 0;
       int rows = min(kTileM, p.M - m0);
-      const uint8_t* bsrc = p.img;
+      const uint8_t* bsrc = p.img + static_cast<size_t>(g_start) * b_bytes;
       for (int c = 0; c < total; ++c) {
         // slot reuse: the MMAs of chunk c - ns (previous round) are done
         if (c >= p.ns && !mbar_wait(&freeb[sl], rph ^ 1u)) {
@@ -311,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         uint8_t* base = smem + sl * p.slot_bytes;
         // the tile's scales, once per tile, on the buffer's own barrier (a
         // bulk copy's completion shows only on the barrier it signals)
-        if (g == 0) {
+        if (g == 0 || c == 0) {
           const uint32_t s_bytes = static_cast<uint32_t>(rows) * G * 2;
           mbar_arrive_expect_tx(&sready[ti & 1], s_bytes);
           bulk_g2s(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes,
@@ -330,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (++g == G) {
           g = 0;
           ++ti;
-          m0 += static_cast<int>(gridDim.x) * kTileM;
+          m0 += kTileM;
           rows = min(kTileM, p.M - m0);
           bsrc = p.img;
         }
@@ -341,7 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (!mbar_wait(&full[c % p.ns], (c / p.ns) & 1)) ok = false;
       }
       if (issued > 0) {
-        const int lt = (issued - 1) / G;  // the last tile whose scales were requested
+        const int lt = (g_start + issued - 1) / G;  // the last tile whose scales were requested
         if (!mbar_wait(&sready[lt & 1], (lt >> 1) & 1)) ok = false;
       }
       if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
@@ -359,11 +376,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
       const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
       const uint32_t dacc = tmem + j * p.Npad;
-      const int step = p.n_mma;  // divides as, ns and G
-      int sl = j, st = j, g = j, ti = 0;  // slot (mod ns), A stage (mod as)
-      uint32_t aph = 0, sph = 0;          // A-stage and slot round parities
+      const int step = p.n_mma;  // divides as, ns, G and kQuant
+      int sl = j, st = j, g = g_start + j, ti = 0;  // slot (mod ns), A stage (mod as)
+      uint32_t aph = 0, sph = 0;                    // A-stage and slot round parities
+      bool first = true;  // the next chunk is this warp's first of its tile portion
       for (int c = j; c < total && ok; c += step) {
-        if (g == j && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
+        // a new tile portion overwrites the accumulators: the previous
+        // portion's epilogue must be done with them
+        if (first && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
         ok = ok && mbar_wait(&aready[st], aph);
         // B arrived by TMA: observe its barrier here too (already complete)
         ok = ok && mbar_wait(&full[sl], sph);
@@ -372,14 +392,16 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (lane == 0) {
           const uint32_t a0 = tmem + p.a_base + st * 64;
           const uint64_t d0 = bdesc0 + sl * slot16;
-          tc_mma_ts(dacc, a0, d0, p.idesc, g >= step ? 1u : 0u);
+          tc_mma_ts(dacc, a0, d0, p.idesc, first ? 0u : 1u);
 #pragma unroll
           for (int ks = 1; ks < 8; ++ks) tc_mma_ts(dacc, a0 + ks * 8, d0 + ks * ks16, p.idesc, 1u);
           tc_commit(&freeb[sl]);
           tc_commit(&afree[st]);
-          if (g + step >= G) tc_commit(dready);
+          // this warp's last chunk of the portion (tile end or range end)
+          if (g + step >= G || c + step >= total) tc_commit(dready);
         }
         __syncwarp();
+        first = false;
         sl += step;
         if (sl >= p.ns) {
           sl -= p.ns;
@@ -394,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         if (g >= G) {
           g -= G;
           ++ti;
+          first = true;
         }
       }
       // Drain: no MMA may be in flight when tensor memory is freed.
@@ -415,36 +438,96 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     bool ok = true;
     uint4 scache = make_uint4(0, 0, 0, 0);  // this row's scales for 8 groups
     int sblock = -1;                         // which block of 8 groups scache holds
-    auto epilogue = [&](int ti) {
-      if (!mbar_wait(dready, ti & 1)) {
-        ok = false;
-        return;
+    // the row's sum of the n_mma accumulators, columns [c0, c0 + 16)
+    auto acc16 = [&](int c0, float (&acc)[16]) {
+      uint32_t v[16];
+      tc_ld16(tmem + lane_base + c0, v);
+      tc_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
+      for (int a = 1; a < p.n_mma; ++a) {
+        tc_ld16(tmem + lane_base + a * p.Npad + c0, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
       }
+    };
+    auto store16 = [&](int m, int c0, const float (&acc)[16]) {
+      if (m < p.M) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int n = c0 + i;
+          if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i];
+        }
+      }
+    };
+    // All dequant threads meet here (bounded: a thread that stopped early
+    // makes the others time out instead of hang).
+    uint32_t eph = 0;
+    auto epi_sync = [&] {
+      mbar_arrive(epib);
+      if (!mbar_wait(epib, eph)) ok = false;
+      eph ^= 1u;
+    };
+    auto epilogue = [&](int ti) {
+      const bool good = mbar_wait(dready, ti & 1);
+      if (!good) ok = false;
       tc_fence_after();
       const int m = tile_m0(ti) + r;
-      // the warpgroups take the 16-column blocks round robin
-      for (int c0 = wg * 16; c0 < p.Npad; c0 += 16 * kDeqWG) {
-        float acc[16];
-        {
-          uint32_t v[16];
-          tc_ld16(tmem + lane_base + c0, v);
-          tc_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
+      // a portion shared with the CTA before (this CTA holds the tile's right
+      // part) or after (left part)
+      const bool right = ti == 0 && g_start != 0;
+      const bool left = ti == last_ti && (g_start + total) % G != 0;
+      if (!right && !left) {
+        // the warpgroups take the 16-column blocks round robin
+        for (int c0 = wg * 16; good && c0 < p.Npad; c0 += 16 * kDeqWG) {
+          float acc[16];
+          acc16(c0, acc);
+          store16(m, c0, acc);
         }
-        for (int a = 1; a < p.n_mma; ++a) {
-          uint32_t v[16];
-          tc_ld16(tmem + lane_base + a * p.Npad + c0, v);
-          tc_wait_ld();
+      } else {
+        // leave this part in the workspace and count the arrival; the second
+        // to arrive adds left + right in that order and stores the tile
+        const int bnd = right ? cta - 1 : cta;
+        float* mine = p.part + ((static_cast<size_t>(bnd) * 2 + (right ? 1 : 0)) * kTileM + r) * p.Npad;
+        const float* other = p.part + ((static_cast<size_t>(bnd) * 2 + (right ? 0 : 1)) * kTileM + r) * p.Npad;
+        for (int c0 = wg * 16; good && c0 < p.Npad; c0 += 16 * kDeqWG) {
+          float acc[16];
+          acc16(c0, acc);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
-        }
-        if (m < p.M) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const int n = c0 + i;
-            if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i];
+          for (int i = 0; i < 16; i += 4) {
+            *reinterpret_cast<float4*>(mine + c0 + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
           }
+        }
+        __threadfence();
+        epi_sync();
+        // after a failed wait the part is not counted (the other side then
+        // finds itself first and leaves; the status word has the error)
+        if (tid == 0) *arrival = ok ? atomicAdd(p.flags + bnd, 1u) : 0u;
+        epi_sync();
+        if (ok && *reinterpret_cast<volatile uint32_t*>(arrival) != 0) {
+          __threadfence();
+          for (int c0 = wg * 16; c0 < p.Npad; c0 += 16 * kDeqWG) {
+            float acc[16];
+            acc16(c0, acc);
+#pragma unroll
+            for (int i = 0; i < 16; i += 4) {
+              const float4 o = __ldcg(reinterpret_cast<const float4*>(other + c0 + i));
+              if (right) {
+                acc[i] = o.x + acc[i];
+                acc[i + 1] = o.y + acc[i + 1];
+                acc[i + 2] = o.z + acc[i + 2];
+                acc[i + 3] = o.w + acc[i + 3];
+              } else {
+                acc[i] = acc[i] + o.x;
+                acc[i + 1] = acc[i + 1] + o.y;
+                acc[i + 2] = acc[i + 2] + o.z;
+                acc[i + 3] = acc[i + 3] + o.w;
+              }
+            }
+            store16(m, c0, acc);
+          }
+          if (tid == 0) p.flags[bnd] = 0;  // ready for the next call
         }
       }
       tc_fence_before();
@@ -455,7 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     // incrementally (kDeqWG divides as and ns; kDeqWG < G).  Every round of
     // this warpgroup's slots and stages is waited for by this warpgroup alone,
     // in order, so a parity wait never meets a phase two rounds old.
-    int sl = wg, st = wg, g = wg, ti = 0;
+    int sl = wg, st = wg, g = g_start + wg, ti = 0;
     uint32_t sph = 0, aph = 0;
     for (int c = wg; c < total && ok; c += kDeqWG) {
       if (ti != prev_ti) {
@@ -541,7 +624,7 @@ struct TcPlan {
 
 constexpr size_t kMaxSmemTc = 227 * 1024 - 1024;  // dynamic; the base is rounded up to 1 KiB
 constexpr size_t kMinSmemTc = 116 * 1024;         // > half an SM's shared memory
-constexpr size_t kBarBytes = 320;  // 33 mbarriers and the TMEM address word
+constexpr size_t kBarBytes = 320;  // 33 mbarriers, the TMEM address and arrival words, 1 mbarrier
 
 // Plan with ns ring slots (0 smem when it does not fit).
 static TcPlan tc_plan_ns(int bits, int K, int npad, int ns) {
@@ -644,10 +727,15 @@ int tc_col_block(int bits, int K) {
   return 0;
 }
 
+// [images of the batch blocks][shared tiles' partial sums: kMaxTcGrid
+// boundaries x 2 sides x 128 rows x nb columns fp32]
+static size_t tc_img_bytes(int nb, int K, int batch) {
+  return (static_cast<size_t>((batch + nb - 1) / nb) * nb * K * 2 + 255) & ~static_cast<size_t>(255);
+}
 size_t tc_xp_bytes(int bits, int K, int batch) {
   const int nb = tc_col_block(bits, K);
   if (nb == 0) return 0;
-  return static_cast<size_t>((batch + nb - 1) / nb) * nb * K * 2;
+  return tc_img_bytes(nb, K, batch) + static_cast<size_t>(kMaxTcGrid) * 2 * tc::kTileM * nb * 4;
 }
 
 int tc_launches(int bits, int K, int batch) {
@@ -701,7 +789,12 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
   e = tc::code_map(&qmap, a.q, a.bits, a.M, a.K);
   if (e != cudaSuccess) return e;
   const int n_tiles = (a.M + tc::kTileM - 1) / tc::kTileM;
-  const unsigned grid = static_cast<unsigned>(std::min(n_tiles, sm_count()));
+  // one CTA per SM; the chunks (tile x group) split evenly in quanta, each CTA
+  // at least a tile's worth (grid <= n_tiles)
+  const int grid_i = std::min(std::min(n_tiles, sm_count()), kMaxTcGrid);
+  const unsigned grid = static_cast<unsigned>(grid_i);
+  const int quanta = n_tiles * (a.K / kGroup) / tc::kQuant;
+  float* part = reinterpret_cast<float*>(xp + tc_img_bytes(nb, a.K, a.N));
   for (int b = 0, n0 = 0; n0 < a.N; ++b, n0 += nb) {
     const int nk = std::min(nb, a.N - n0);
     const int npad = (nk + 31) & ~31;
@@ -718,6 +811,10 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.Npad = npad;
     p.ldy = a.ldy;
     p.n_tiles = n_tiles;
+    p.qq = quanta / grid_i;
+    p.qr = quanta % grid_i;
+    p.part = part;
+    p.flags = a.counters;
     p.slot_bytes = pl.slot;
     p.b_off = pl.b_off;
     p.sbuf_off = pl.sbuf_off;

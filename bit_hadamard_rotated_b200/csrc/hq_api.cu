@@ -58,12 +58,16 @@ static bool use_tc(const hq_weight* w, int batch) {
          tc_col_block(w->bits, w->K) > 0;
 }
 
-// hq_linear workspace: [status 256 B]
-// [activations: on the tensor-core path the rotated activation images (batch
-// rounded up to whole batch blocks, x K fp16); on the GEMV path the rotated
-// activations of one batch block in fragment order (blocks run in turn)].
+// hq_linear workspace: [status 256 B] [tensor-core tile counters 1 KiB, zero
+// between calls] [on the tensor-core path the rotated activation images
+// (batch rounded up to whole batch blocks, x K fp16) and the partial sums of
+// tiles shared by two CTAs; on the GEMV path the rotated activations of one
+// batch block in fragment order (blocks run in turn)].  The counters sit at a
+// fixed offset that neither path writes anything else to, so calls of any
+// width and batch can share the workspace.
 struct LinearWs {
   uint32_t* status;
+  uint32_t* counters;
   void* xp;
   size_t bytes;
 };
@@ -76,8 +80,9 @@ static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
                               : align256(gemv_scratch_bytes(w->K, nb > 0 ? std::min(nb, std::max(batch, 1)) : 1));
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
-  l.xp = b + kStatusBytes;
-  l.bytes = kStatusBytes + xp_bytes;
+  l.counters = reinterpret_cast<uint32_t*>(b + kStatusBytes);
+  l.xp = b + kStatusBytes + kTcCounterBytes;
+  l.bytes = kStatusBytes + kTcCounterBytes + xp_bytes;
   return l;
 }
 
@@ -167,6 +172,7 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     a.ldy = w->M;
     a.status = l.status;
     a.xp = l.xp;
+    a.counters = l.counters;
     return from_cuda(launch_linear_tc(a, st));
   }
   const int nb = gemv_col_block(w->bits, w->K);

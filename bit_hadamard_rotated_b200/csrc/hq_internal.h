@@ -72,10 +72,17 @@ struct TcArgs {
   int ldy;
   uint32_t* status;
   void* xp;  // workspace: tc_xp_bytes(bits, K, N) bytes, 256-byte aligned
+  uint32_t* counters;  // kTcCounterBytes, zero between calls (every call leaves them zero)
 };
+// Arrival counters of the tensor-core GEMM's tiles shared by two CTAs (one
+// per CTA boundary; at most kMaxTcGrid CTAs).
+constexpr int kMaxTcGrid = 160;
+constexpr size_t kTcCounterBytes = 1024;
+static_assert(kMaxTcGrid * 4 <= static_cast<int>(kTcCounterBytes), "counter region");
 // Largest batch block per GEMM launch for this width and K (0: path unavailable).
 int tc_col_block(int bits, int K);
-// Workspace bytes for the rotated activation images of a batch.
+// Workspace bytes for the rotated activation images of a batch and the
+// partial sums of tiles shared by two CTAs.
 size_t tc_xp_bytes(int bits, int K, int batch);
 // Kernel launches of one tensor-core hq_linear call (prep + one GEMM per block).
 int tc_launches(int bits, int K, int batch);

@@ -87,7 +87,7 @@ CASES = [
     # (M, K, N): ragged tiles, ragged batches, several blocks and tiles per CTA
     (128, 1024, 9), (1, 1024, 16), (129, 1024, 31), (300, 2048, 33), (77, 4096, 64),
     (256, 8192, 100), (200, 16384, 128), (130, 1024, 129), (64, 2048, 200),
-    (20000, 1024, 24),
+    (20000, 1024, 24), (19100, 1024, 140),
 ]
 
 
@@ -128,6 +128,28 @@ def test_tc_matches_gemv_and_is_deterministic():
     want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
     assert_within(y1.cpu().numpy(), want, bound, what="tc")
     assert_within(yg.cpu().numpy(), want, bound, what="gemv")
+
+
+def test_tc_tiles_shared_between_ctas_deterministic():
+    """More 128-row tiles than CTAs: CTAs own equal chunk ranges, so tiles are
+    cut between two CTAs and finished by the second to arrive.  Repeat calls on
+    one workspace are bit-identical and leave the tile counters (the 1 KiB after
+    the status word) at zero."""
+    from bit_hadamard_rotated_b200 import hq
+    M, K, N, bits = 24000, 4096, 64, 2
+    d = synth.linear(M, K, bits, N, seed=17)
+    q, s, g, w = weight(d)
+    x = dev(d["x"])
+    ws = torch.zeros(hq.hq_linear_workspace_size(w, N), dtype=torch.uint8, device="cuda")
+    y1 = hq.hq_linear(q, s, g, x, bits, d["zero"], workspace=ws)
+    y2 = hq.hq_linear(q, s, g, x, bits, d["zero"], workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    assert int(ws[256:1280].count_nonzero()) == 0
+    rows = np.r_[0:64, 12000:12300, M - 64:M]
+    want, bound = oracle.linear(bits, len(rows), K, d["zero"], d["q"][rows], d["scales"][rows],
+                                d["signs"], d["x"])
+    assert_within(y1.cpu().numpy()[:, rows], want, bound, what="stream-K rows")
 
 
 def test_tc_output_overwritten_and_status_clean():
