@@ -6,28 +6,33 @@
 //     k order of the decoded code pairs (hq_layout.cuh), so that A and B agree,
 //     already in the shared-memory image the MMA reads (no-swizzle K-major
 //     core matrices), one contiguous block per 128-code group;
-//   * per CTA, one 128-row tile at a time: one producer thread streams each
-//     128-code group through a ring of 4, 6 or 8 shared-memory slots (as many
-//     as fit) -- the tile's 128 code rows in one 2D TMA load (swizzled so the
-//     decoders' 16-byte row reads are free of bank conflicts), the group's x'
-//     image in one bulk copy, and at the tile's first group its scales in one
-//     bulk copy -- all completing on the slot's mbarrier (expected bytes);
-//   * two warpgroups take the groups in turn (group c to warpgroup c mod 2):
+//   * per CTA, an equal contiguous range of (128-row tile, 128-code group)
+//     chunks (stream-K; the first and last tile may be shared with the
+//     neighbouring CTA): one producer thread streams each chunk through a
+//     ring of 4 or 8 shared-memory slots (as many as fit) -- the tile's 128
+//     code rows in one 2D TMA load (swizzled so the decoders' 16-byte row
+//     reads are free of bank conflicts), the group's x' image in one bulk
+//     copy, and at the tile's first chunk its scales in one bulk copy -- all
+//     completing on the slot's mbarrier (expected bytes);
+//   * two warpgroups take the chunks in turn (chunk c to warpgroup c mod 2):
 //     each thread owns one weight row, decodes its 128 codes into exact fp16
 //     (q - zero) (one LOP3 and one fp16 FMA per pair), multiplies by the group
 //     scale (one fp16 multiply per pair: the weight's only rounding) and
 //     stores the row into tensor memory as the MMA's A operand (tcgen05.st),
-//     one TMEM lane per row, in A stage c mod as (as = 4 or 6 stages, so each
-//     warpgroup rotates through 2 or 3 and decodes ahead while the MMAs of its
-//     previous groups run);
-//   * two MMA warps take the groups in the same turn (warp c mod 2); each
-//     issues 8 tcgen05.mma (M=128, N, K=16, A from TMEM, B from shared memory)
-//     per group into its own fp32 accumulator in tensor memory and commits
-//     their completion to the slot's and the A stage's mbarriers.  One issuing
+//     one TMEM lane per row, in A stage c mod as (4 stages, so each
+//     warpgroup decodes ahead while the MMAs of its previous chunks run);
+//   * two or four MMA warps take the chunks in the same turn; each issues 8
+//     tcgen05.mma (M=128, N, K=16, A from TMEM, B from shared memory) per
+//     chunk into its own fp32 accumulator in tensor memory and commits their
+//     completion to the slot's and the A stage's mbarriers.  One issuing
 //     thread sustains only one MMA per ~60-80 cycles whatever N is, so at
-//     batch <= 128 a second issuer doubles the tensor-pipe rate;
-//   * the tile's last commits release the epilogue, which sums the two
-//     accumulators (tcgen05.ld) and writes y.
+//     batch <= 128 more issuers raise the tensor-pipe rate;
+//   * an epilogue warpgroup sums a tile's accumulators (tcgen05.ld) and writes
+//     y, or, for a tile shared with a neighbour, leaves its part in the
+//     workspace and the second CTA to count its arrival adds left + right in
+//     that order (deterministic, no waiting).  With two accumulator sets
+//     (batch <= 32) the next tile's MMAs run while the epilogue reads; the
+//     dequant warps never stop for it.
 // Every barrier's consecutive phases are waited for by one agent, in order
 // (ring depths are multiples of two), so phase-parity waits are unambiguous.
 // Waits are bounded (status word on timeout); tensor memory is freed on exit.
@@ -56,7 +61,9 @@ constexpr int kDeqWarps = 4 * kDeqWG;
 constexpr int kProducerWarp = kDeqWarps;
 constexpr int kMmaWarp0 = kDeqWarps + 1;
 constexpr int kMmaWarps = 4;      // issuing threads launched: one issues an MMA per ~60-80 cycles
-constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps) * 32;
+constexpr int kEpiWarp0 = kMmaWarp0 + kMmaWarps;
+constexpr int kEpiWarps = 4;      // the epilogue warpgroup: one thread per accumulator row
+constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps + kEpiWarps) * 32;
 // Phase-parity waits are unambiguous only if a barrier's consecutive phases
 // are waited for by the same agent (it cannot wait for round r + 1 before
 // round r completed): every ring depth is a multiple of the dequant
@@ -245,10 +252,125 @@ struct TcParams {
   int ns;       // shared-memory ring slots (kNSMin..kNSMax)
   int as;       // A stages in tensor memory (4 or 6; a multiple of n_mma)
   int a_base;   // tensor-memory column of A stage 0
-  int n_mma;    // MMA warps (accumulators) in use: 4 if Npad <= 64, else 2
+  int n_mma;    // MMA warps (accumulators per set) in use: 4 if Npad <= 64, else 2
+  int nacc;     // accumulator sets: 2 (tile ti uses set ti & 1) if they fit beside 4 A stages, else 1
   uint32_t idesc;
   uint32_t add[16];
 };
+
+// The epilogue warpgroup: for each tile portion of the CTA, waits for its
+// accumulator set, sums the n_mma accumulators of its row (TMEM lane) and
+// stores y, or, for a portion shared with a neighbouring CTA, leaves the part
+// in the workspace and lets the second CTA to count its arrival add left +
+// right; then frees the set for the MMAs two portions on (one with a single
+// set).  Runs beside the dequant warps, which never stop for it.
+__device__ __forceinline__ void tc_epilogue(const TcParams& p, uint32_t tmem, uint64_t* dready,
+                                            uint64_t* dfree, uint64_t* epib, uint32_t* arrival,
+                                            int cta, int g_start, int total, int last_ti, int tile0) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int etid = tid - kEpiWarp0 * 32;
+  const int quarter = warp & 3;  // the TMEM lane quarter this warp may access
+  const int r = 32 * quarter + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(32 * quarter) << 16;
+  const int G = p.K / kGroup;
+  const uint32_t acc_set = static_cast<uint32_t>(p.n_mma * p.Npad);
+  bool ok = true;
+  uint32_t eph = 0;
+  // all epilogue threads meet here (bounded: a thread that stopped early
+  // makes the others time out instead of hang)
+  auto epi_sync = [&] {
+    mbar_arrive(epib);
+    if (!mbar_wait(epib, eph)) ok = false;
+    eph ^= 1u;
+  };
+  for (int ti = 0; ti <= last_ti; ++ti) {
+    const int buf = p.nacc == 2 ? (ti & 1) : 0, use = p.nacc == 2 ? (ti >> 1) : ti;
+    const bool good = ok && mbar_wait(&dready[buf], use & 1);
+    if (!good) ok = false;
+    tc_fence_after();
+    const uint32_t acc0 = tmem + lane_base + buf * acc_set;
+    // the row's sum of the n_mma accumulators, columns [c0, c0 + 16)
+    auto acc16 = [&](int c0, float (&acc)[16]) {
+      uint32_t v[16];
+      tc_ld16(acc0 + c0, v);
+      tc_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
+      for (int a = 1; a < p.n_mma; ++a) {
+        tc_ld16(acc0 + a * p.Npad + c0, v);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
+      }
+    };
+    const int m = (tile0 + ti) * kTileM + r;
+    auto store16 = [&](int c0, const float (&acc)[16]) {
+      if (m < p.M) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int n = c0 + i;
+          if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i];
+        }
+      }
+    };
+    // a portion shared with the CTA before (this CTA holds the tile's right
+    // part) or after (left part)
+    const bool right = ti == 0 && g_start != 0;
+    const bool left = ti == last_ti && (g_start + total) % G != 0;
+    if (!right && !left) {
+      for (int c0 = 0; good && c0 < p.Npad; c0 += 16) {
+        float acc[16];
+        acc16(c0, acc);
+        store16(c0, acc);
+      }
+    } else {
+      const int bnd = right ? cta - 1 : cta;
+      float* mine = p.part + ((static_cast<size_t>(bnd) * 2 + (right ? 1 : 0)) * kTileM + r) * p.Npad;
+      const float* other = p.part + ((static_cast<size_t>(bnd) * 2 + (right ? 0 : 1)) * kTileM + r) * p.Npad;
+      for (int c0 = 0; good && c0 < p.Npad; c0 += 16) {
+        float acc[16];
+        acc16(c0, acc);
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          *reinterpret_cast<float4*>(mine + c0 + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
+        }
+      }
+      __threadfence();
+      epi_sync();
+      // after a failed wait the part is not counted (the other side then
+      // finds itself first and leaves; the status word has the error)
+      if (etid == 0) *arrival = ok ? atomicAdd(p.flags + bnd, 1u) : 0u;
+      epi_sync();
+      if (ok && *reinterpret_cast<volatile uint32_t*>(arrival) != 0) {
+        __threadfence();
+        for (int c0 = 0; c0 < p.Npad; c0 += 16) {
+          float acc[16];
+          acc16(c0, acc);
+#pragma unroll
+          for (int i = 0; i < 16; i += 4) {
+            const float4 o = __ldcg(reinterpret_cast<const float4*>(other + c0 + i));
+            if (right) {
+              acc[i] = o.x + acc[i];
+              acc[i + 1] = o.y + acc[i + 1];
+              acc[i + 2] = o.z + acc[i + 2];
+              acc[i + 3] = o.w + acc[i + 3];
+            } else {
+              acc[i] = acc[i] + o.x;
+              acc[i + 1] = acc[i + 1] + o.y;
+              acc[i + 2] = acc[i + 2] + o.z;
+              acc[i + 3] = acc[i + 3] + o.w;
+            }
+          }
+          store16(c0, acc);
+        }
+        if (etid == 0) p.flags[bnd] = 0;  // ready for the next call
+      }
+    }
+    tc_fence_before();
+    mbar_arrive(&dfree[buf]);
+  }
+  if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
+}
 
 template <int BITS>
 __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_constant__ TcParams p) {
@@ -263,13 +385,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   uint64_t* freeb = full + kNSMax;    // slot's MMAs done (producer may refill)
   uint64_t* aready = freeb + kNSMax;  // A stage written (MMA may read)
   uint64_t* afree = aready + kASMax;  // A stage's MMAs done (dequant may rewrite)
-  uint64_t* dready = afree + kASMax;
-  uint64_t* dfree = dready + 1;
-  uint64_t* drain = dfree + 1;
+  uint64_t* dready = afree + kASMax;  // [2]: accumulator set's MMAs done (epilogue may read)
+  uint64_t* dfree = dready + 2;       // [2]: accumulator set read out (MMA may overwrite)
+  uint64_t* drain = dfree + 2;
   uint64_t* sready = drain + 1;  // [2]: a tile's scales landed in buffer ti & 1
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sready + 2);
   uint32_t* arrival = tmem_holder + 1;  // the epilogue's boundary-counter result
-  // the dequant threads' own barrier (shared-tile epilogues), 8-byte aligned
+  // the epilogue threads' own barrier (shared-tile epilogues), 8-byte aligned
   uint64_t* epib = reinterpret_cast<uint64_t*>(tmem_holder + 2);
 
   if (tid == 0) {
@@ -281,12 +403,14 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       mbar_init(&aready[i], 128);
       mbar_init(&afree[i], 1);
     }
-    mbar_init(dready, p.n_mma);
-    mbar_init(dfree, kDeqWG * 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&dready[b], p.n_mma);
+      mbar_init(&dfree[b], kEpiWarps * 32);
+    }
     mbar_init(drain, p.n_mma);
     mbar_init(&sready[0], 1);
     mbar_init(&sready[1], 1);
-    mbar_init(epib, kDeqWarps * 32);
+    mbar_init(epib, kEpiWarps * 32);
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(tmem_holder, kTmemCols);
@@ -364,6 +488,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
     }
     __syncwarp();
+  } else if (warp >= kEpiWarp0) {
+    tc_epilogue(p, tmem, dready, dfree, epib, arrival, cta, g_start, total, last_ti, tile0);
   } else if (warp >= kMmaWarp0) {
     // ---------------- MMA issue: warp j takes chunks j, j + n_mma, ...
     const int j = warp - kMmaWarp0;
@@ -375,21 +501,23 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       const uint64_t bdesc0 = smem_desc(smem_u32(smem + p.b_off), 16 * p.Npad, 128);
       const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
       const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
-      const uint32_t dacc = tmem + j * p.Npad;
+      const uint32_t acc_set = static_cast<uint32_t>(p.n_mma * p.Npad);  // columns per set
       const int step = p.n_mma;  // divides as, ns, G and kQuant
       int sl = j, st = j, g = g_start + j, ti = 0;  // slot (mod ns), A stage (mod as)
       uint32_t aph = 0, sph = 0;                    // A-stage and slot round parities
       bool first = true;  // the next chunk is this warp's first of its tile portion
       for (int c = j; c < total && ok; c += step) {
-        // a new tile portion overwrites the accumulators: the previous
-        // portion's epilogue must be done with them
-        if (first && ti > 0) ok = mbar_wait(dfree, (ti - 1) & 1);
+        // a new tile portion overwrites its accumulator set: the epilogue of
+        // the portion that used the set before must be done with it
+        const int buf = p.nacc == 2 ? (ti & 1) : 0, use = p.nacc == 2 ? (ti >> 1) : ti;
+        if (first && use > 0) ok = mbar_wait(&dfree[buf], (use - 1) & 1);
         ok = ok && mbar_wait(&aready[st], aph);
         // B arrived by TMA: observe its barrier here too (already complete)
         ok = ok && mbar_wait(&full[sl], sph);
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
+          const uint32_t dacc = tmem + buf * acc_set + j * p.Npad;
           const uint32_t a0 = tmem + p.a_base + st * 64;
           const uint64_t d0 = bdesc0 + sl * slot16;
           tc_mma_ts(dacc, a0, d0, p.idesc, first ? 0u : 1u);
@@ -398,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           tc_commit(&freeb[sl]);
           tc_commit(&afree[st]);
           // this warp's last chunk of the portion (tile end or range end)
-          if (g + step >= G || c + step >= total) tc_commit(dready);
+          if (g + step >= G || c + step >= total) tc_commit(&dready[buf]);
         }
         __syncwarp();
         first = false;
@@ -426,7 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
     }
   } else {
-    // ---------------- dequant (kDeqWG warpgroups, groups round robin) + epilogue
+    // ---------------- dequant (kDeqWG warpgroups, groups round robin)
     const int wg = warp >> 2;
     const int sub = warp & 3;
     const int r = 32 * sub + lane;  // tile row = TMEM lane
@@ -438,101 +566,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     bool ok = true;
     uint4 scache = make_uint4(0, 0, 0, 0);  // this row's scales for 8 groups
     int sblock = -1;                         // which block of 8 groups scache holds
-    // the row's sum of the n_mma accumulators, columns [c0, c0 + 16)
-    auto acc16 = [&](int c0, float (&acc)[16]) {
-      uint32_t v[16];
-      tc_ld16(tmem + lane_base + c0, v);
-      tc_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
-      for (int a = 1; a < p.n_mma; ++a) {
-        tc_ld16(tmem + lane_base + a * p.Npad + c0, v);
-        tc_wait_ld();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
-      }
-    };
-    auto store16 = [&](int m, int c0, const float (&acc)[16]) {
-      if (m < p.M) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int n = c0 + i;
-          if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i];
-        }
-      }
-    };
-    // All dequant threads meet here (bounded: a thread that stopped early
-    // makes the others time out instead of hang).
-    uint32_t eph = 0;
-    auto epi_sync = [&] {
-      mbar_arrive(epib);
-      if (!mbar_wait(epib, eph)) ok = false;
-      eph ^= 1u;
-    };
-    auto epilogue = [&](int ti) {
-      const bool good = mbar_wait(dready, ti & 1);
-      if (!good) ok = false;
-      tc_fence_after();
-      const int m = tile_m0(ti) + r;
-      // a portion shared with the CTA before (this CTA holds the tile's right
-      // part) or after (left part)
-      const bool right = ti == 0 && g_start != 0;
-      const bool left = ti == last_ti && (g_start + total) % G != 0;
-      if (!right && !left) {
-        // the warpgroups take the 16-column blocks round robin
-        for (int c0 = wg * 16; good && c0 < p.Npad; c0 += 16 * kDeqWG) {
-          float acc[16];
-          acc16(c0, acc);
-          store16(m, c0, acc);
-        }
-      } else {
-        // leave this part in the workspace and count the arrival; the second
-        // to arrive adds left + right in that order and stores the tile
-        const int bnd = right ? cta - 1 : cta;
-        float* mine = p.part + ((static_cast<size_t>(bnd) * 2 + (right ? 1 : 0)) * kTileM + r) * p.Npad;
-        const float* other = p.part + ((static_cast<size_t>(bnd) * 2 + (right ? 0 : 1)) * kTileM + r) * p.Npad;
-        for (int c0 = wg * 16; good && c0 < p.Npad; c0 += 16 * kDeqWG) {
-          float acc[16];
-          acc16(c0, acc);
-#pragma unroll
-          for (int i = 0; i < 16; i += 4) {
-            *reinterpret_cast<float4*>(mine + c0 + i) = make_float4(acc[i], acc[i + 1], acc[i + 2], acc[i + 3]);
-          }
-        }
-        __threadfence();
-        epi_sync();
-        // after a failed wait the part is not counted (the other side then
-        // finds itself first and leaves; the status word has the error)
-        if (tid == 0) *arrival = ok ? atomicAdd(p.flags + bnd, 1u) : 0u;
-        epi_sync();
-        if (ok && *reinterpret_cast<volatile uint32_t*>(arrival) != 0) {
-          __threadfence();
-          for (int c0 = wg * 16; c0 < p.Npad; c0 += 16 * kDeqWG) {
-            float acc[16];
-            acc16(c0, acc);
-#pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              const float4 o = __ldcg(reinterpret_cast<const float4*>(other + c0 + i));
-              if (right) {
-                acc[i] = o.x + acc[i];
-                acc[i + 1] = o.y + acc[i + 1];
-                acc[i + 2] = o.z + acc[i + 2];
-                acc[i + 3] = o.w + acc[i + 3];
-              } else {
-                acc[i] = acc[i] + o.x;
-                acc[i + 1] = acc[i + 1] + o.y;
-                acc[i + 2] = acc[i + 2] + o.z;
-                acc[i + 3] = acc[i + 3] + o.w;
-              }
-            }
-            store16(m, c0, acc);
-          }
-          if (tid == 0) p.flags[bnd] = 0;  // ready for the next call
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(dfree);
-    };
     // this warpgroup's chunks c = wg, wg + kDeqWG, ...: slot (mod ns), A
     // stage (mod as), their round parities, group and tile advance
     // incrementally (kDeqWG divides as and ns; kDeqWG < G).  Every round of
@@ -542,7 +575,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     uint32_t sph = 0, aph = 0;
     for (int c = wg; c < total && ok; c += kDeqWG) {
       if (ti != prev_ti) {
-        if (prev_ti >= 0) epilogue(prev_ti);
         prev_ti = ti;
         sblock = -1;  // the new tile's scales are in the other buffer
         if (!ok || !mbar_wait(&sready[ti & 1], (ti >> 1) & 1)) {
@@ -604,7 +636,6 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         ++ti;
       }
     }
-    if (ok && prev_ti >= 0) epilogue(prev_ti);
     if (!ok && lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
   }
   tc_fence_before();
@@ -624,7 +655,7 @@ struct TcPlan {
 
 constexpr size_t kMaxSmemTc = 227 * 1024 - 1024;  // dynamic; the base is rounded up to 1 KiB
 constexpr size_t kMinSmemTc = 116 * 1024;         // > half an SM's shared memory
-constexpr size_t kBarBytes = 320;  // 33 mbarriers, the TMEM address and arrival words, 1 mbarrier
+constexpr size_t kBarBytes = 320;  // 35 mbarriers, the TMEM address and arrival words, 1 mbarrier
 
 // Plan with ns ring slots (0 smem when it does not fit).
 static TcPlan tc_plan_ns(int bits, int K, int npad, int ns) {
@@ -820,9 +851,13 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.sbuf_off = pl.sbuf_off;
     p.sbuf_bytes = pl.sbuf_bytes;
     p.bar_off = pl.bar_off;
-    // accumulators: 4 if they fit in half of tensor memory with 4 A stages
+    // accumulators: sets of n_mma, one per MMA warp (at N <= 64 an MMA costs
+    // its issuer about twice its tensor-pipe time, so four issuers), two sets
+    // (so the next tile's MMAs need not wait for the epilogue) while they fit
+    // in half of tensor memory, leaving 4 A stages
     p.n_mma = npad <= 64 ? 4 : 2;
-    p.a_base = (p.n_mma * npad + 63) & ~63;
+    p.nacc = 2 * p.n_mma * npad <= 256 ? 2 : 1;
+    p.a_base = (p.nacc * p.n_mma * npad + 63) & ~63;
     p.as = ((tc::kTmemCols - p.a_base) / 64) / p.n_mma * p.n_mma;
     if (p.as > tc::kASMax) p.as = tc::kASMax / p.n_mma * p.n_mma;
     p.ns = pl.ns / p.n_mma * p.n_mma;
