@@ -65,8 +65,9 @@ struct Dims {
 constexpr int kMaxGrid = 1024;
 
 // Relative cost of one 16-row tile of a width, for splitting the phases'
-// work between CTAs: the code bytes (proportional to the width) plus a fixed
-// part for the per-group instructions that do not depend on it.
+// work between CTAs and warps: the code bytes (proportional to the width)
+// plus a fixed part for the per-group instructions that do not depend on it
+// (a flatter weight, bits + 8, measured 12 % slower on the 256-expert layer).
 __host__ __device__ constexpr int tile_weight(int bits) { return bits + 2; }
 
 }  // namespace moe
@@ -475,11 +476,35 @@ __device__ __forceinline__ void group_mma(const uint8_t* ra, const uint8_t* rb, 
   acc[3] = fmaf(sb, c0[3] + c1[3], acc[3]);
 }
 
-// Shared-memory plan of one phase launch (host and device agree on it).
+// A pass of a phase CTA: up to kMaxSeg consecutive segments (the parts of
+// (expert, column block) blocks in the CTA's item range) with at most 8
+// columns in all, whose activation fragments are staged together.
+constexpr int kMaxSeg = 4;
+
+struct SegInfo {
+  hq_expert ed;
+  int item0, item1;  // items [item0, item1)
+  int tile0;         // row tile of item0 within the expert
+  int unit0;         // first (item, group) unit of the segment within the pass
+  int wt0;           // weight of the pass's units before the segment (tile weight per unit)
+  int off, ncol;     // first sorted pair of the block, its columns (<= 8)
+  int col0;          // column offset of the block in the staged fragments
+  int L;             // activation layout (bit width) of phase A
+};
+
+struct PassMeta {
+  SegInfo seg[kMaxSeg];
+  int nseg, cols, units, wtot;
+};
+static_assert(sizeof(PassMeta) <= 1024, "pass metadata");
+
+// Shared-memory plan of one phase launch (host and device agree on it):
+// [pass metadata 1 KiB][zero-point terms [kMaxSeg][G][8] fp32, zero B block]
+// [staged B fragments [G][8 columns][4 k-quads][64 B] (BSMEM)][rings][barriers]
 struct PhaseSmem {
-  int bsmem;     // 1: the segment's B fragments are staged in shared memory
+  int bsmem;     // 1: the pass's B fragments are staged in shared memory
   int cbytes;    // ring slot bytes
-  int xs_off, ring_off, bar_off, total;
+  int zc_off, xs_off, ring_off, bar_off, total;
 };
 
 __host__ __device__ inline int round128(int v) { return (v + 127) & ~127; }
@@ -489,8 +514,9 @@ __host__ __device__ inline PhaseSmem phase_smem(int G, int nmat) {
   // the largest len-1 chunk of any width must fit a slot
   int need = 0;
   for (int b = 2; b <= 8; b = b == 4 ? 8 : b + 1) need = max(need, chunk_bytes(b, G, nmat, 1));
-  p.xs_off = round128(G * 8 * 4 + 64);  // zero-point terms [G][8], zero B block
-  const int xs_bytes = G * 8 * 4 * 64;  // [G][8 columns][4 k-quads][64 B]
+  p.zc_off = 1024;
+  p.xs_off = round128(p.zc_off + kMaxSeg * G * 8 * 4 + 64);
+  const int xs_bytes = G * 8 * 4 * 64;
   const int ring_off = round128(p.xs_off + xs_bytes);
   const int fit = ((kSmemMax - ring_off - kWarps * kRing * 8) / (kWarps * kRing)) & ~127;
   p.bsmem = fit >= max(need, 4096) ? 1 : 0;  // else the rings would be too shallow
@@ -515,54 +541,105 @@ struct RingState {
   bool ok;  // false once a wait has timed out; the warp then stops
 };
 
-// The part of a segment one warp computes: items [w0, w1) of one block.
-struct SegArgs {
-  int w0, w1, tile0;  // tile of item j is tile0 + j
-  int off, ncol;      // first sorted pair of the block, its columns (<= 8)
-  int G, K, M;
-  size_t brow_g;      // B row of this lane's column g (when g < ncol)
-};
+// B-operand row of column col of a segment (the token's rotated activations
+// in phase A, the pair's rotated h in phase B).
+template <int PHASE>
+__device__ __forceinline__ size_t seg_brow(const Ws& w, const Dims& d, const SegInfo& sg, int col) {
+  const int p = sg.off + col;
+  return PHASE == 0 ? static_cast<size_t>(sg.L) * d.T + w.sorted[p] / d.k : static_cast<size_t>(p);
+}
 
+// Epilogue of one tile: rows g, g+8 of the lane's fragment, columns 2t, 2t+1.
+template <int PHASE>
+__device__ __forceinline__ void seg_store(const Ws& w, const Dims& d, const SegInfo& sg, int m0,
+                                          const float4 (&o)[2], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const int M = PHASE == 0 ? d.inter : d.hidden;
+  const float* og = reinterpret_cast<const float*>(&o[0]);
+  const float* ou = reinterpret_cast<const float*>(&o[PHASE == 0 ? 1 : 0]);
+#pragma unroll
+  for (int q4 = 0; q4 < 4; ++q4) {
+    const int col = 2 * t + (q4 & 1);
+    const int m = m0 + g + 8 * (q4 >> 1);
+    if (col < sg.ncol && m < M) {
+      const size_t prow = static_cast<size_t>(sg.off + col);
+      if (PHASE == 0) {
+        const float gv = og[q4] * kUnit, uv = ou[q4] * kUnit;
+        w.h[prow * d.inter + m] = gv / (1.f + expf(-gv)) * uv;
+      } else {
+        w.d[prow * d.hidden + m] = og[q4] * kUnit;
+      }
+    }
+  }
+}
+
+// Units [ua, ub) (pass-relative (item, group) units, all in segment k) of one
+// warp: codes and scales stream through the warp's ring in chunks of up to
+// len groups of one tile (never crossing an aligned run of 8 groups, whose
+// scales are one 16-byte piece per row); B comes from the staged fragments
+// (BSMEM) or from global memory one group ahead.  A tile the warp covers
+// whole is stored here; a tile it covers in part (only at its range ends u0,
+// u1) is kept in `part` (0: the tile holding u0, 1: the last) for the
+// pass's reduction.
 template <int PHASE, bool BSMEM, int BITS>
-__device__ __forceinline__ void phase_tiles(const hq_expert& ed, Ws& w, const Dims& d,
-                                            const PhaseSmem& ps, const SegArgs& sa, RingState& rs,
-                                            const float* zc, const uint4* xs,
-                                            const uint16_t* bsrc, int lane) {
+__device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, int ub, const Ws& w,
+                                            const Dims& d, const PhaseSmem& ps, RingState& rs,
+                                            const float* zc, const uint4* xs, int cols,
+                                            const uint16_t* bsrc, int u0, float4 (&part)[2][2],
+                                            int (&ptile)[2], int lane) {
   constexpr int NMAT = PHASE == 0 ? 2 : 1;
   constexpr int GB = 16 * BITS;  // code bytes of one row in one group
   const int g = lane >> 2, t = lane & 3;
-  const int G = sa.G;
-  const int len = chunk_len(BITS, G, NMAT, ps.cbytes);  // divides G (both powers of two)
-  const int stride = chunk_stride(BITS, len);
-  const int row_bytes = sa.K * BITS / 8;
+  const int K = PHASE == 0 ? d.hidden : d.inter;
+  const int G = K / kGroup;
+  const int lgG = __ffs(G) - 1;
+  const int len_max = chunk_len(BITS, G, NMAT, ps.cbytes);
+  const int stride = chunk_stride(BITS, len_max);
+  const int row_bytes = K * BITS / 8;
   const int sbytes = chunk_scale_bytes(G);
-  // producer geometry: pr 16-byte pieces per row, 16 rows; lane's first piece
-  // (r0, c0) and the step of 32 pieces (dr rows + dc pieces)
-  const int pr = len * BITS;
-  const int npc = kRows * pr;
-  const int r0 = lane / pr, c0 = lane - r0 * pr;
-  const int dr = 32 / pr, dc = 32 - dr * pr;
   const uint8_t* qbase[NMAT];
   const uint16_t* sbase[NMAT];
   if (PHASE == 0) {
-    qbase[0] = reinterpret_cast<const uint8_t*>(ed.q_gate);
-    qbase[NMAT - 1] = reinterpret_cast<const uint8_t*>(ed.q_up);
-    sbase[0] = ed.s_gate;
-    sbase[NMAT - 1] = ed.s_up;
+    qbase[0] = reinterpret_cast<const uint8_t*>(sg.ed.q_gate);
+    qbase[NMAT - 1] = reinterpret_cast<const uint8_t*>(sg.ed.q_up);
+    sbase[0] = sg.ed.s_gate;
+    sbase[NMAT - 1] = sg.ed.s_up;
   } else {
-    qbase[0] = reinterpret_cast<const uint8_t*>(ed.q_down);
-    sbase[0] = ed.s_down;
+    qbase[0] = reinterpret_cast<const uint8_t*>(sg.ed.q_down);
+    sbase[0] = sg.ed.s_down;
   }
-  int pj = sa.w0, pg = 0;  // next (item, group) to copy
+  auto chunk_of = [&](int u, int& j, int& g0, int& len) {
+    const int r = u - sg.unit0;
+    j = r >> lgG;
+    g0 = r & (G - 1);
+    len = min(min(len_max, G - g0), min(ub - u, 8 - (g0 & 7)));
+  };
+  // producer: the warp's lanes split each chunk's 16-byte pieces; every lane
+  // arrives on the slot's barrier
+  int pu = ua;
+  // the lane's walk over a full-length chunk's 16-byte pieces (pr per row):
+  // first piece (r0, c0), then steps of 32 pieces (dr rows + dc pieces)
+  const int prf = len_max * BITS;
+  const int r0f = lane / prf, c0f = lane - r0f * prf, drf = 32 / prf, dcf = 32 - drf * prf;
   auto issue = [&](int slot) {
-    const int m0 = (sa.tile0 + pj) * kRows;
+    int j, g0, len;
+    chunk_of(pu, j, g0, len);
+    const int m0 = (sg.tile0 + j) * kRows;
     uint8_t* base = rs.ring + slot * ps.cbytes;
+    int pr = prf, r0 = r0f, c0 = c0f, dr = drf, dc = dcf;
+    if (len != len_max) {  // a shorter chunk (tile or range end)
+      pr = len * BITS;
+      r0 = lane / pr;
+      c0 = lane - r0 * pr;
+      dr = 32 / pr;
+      dc = 32 - dr * pr;
+    }
 #pragma unroll
     for (int mi = 0; mi < NMAT; ++mi) {
-      const uint8_t* src = qbase[mi] + static_cast<size_t>(m0) * row_bytes + pg * GB;
+      const uint8_t* src = qbase[mi] + static_cast<size_t>(m0) * row_bytes + g0 * GB;
       uint8_t* cdst = base + mi * kRows * stride;
       int r = r0, c = c0;
-      for (int i = lane; i < npc; i += 32) {
+      for (int i = lane; i < kRows * pr; i += 32) {
         cp_async16(cdst + r * stride + c * 16, src + r * row_bytes + c * 16, 16);
         c += dc;
         r += dr;
@@ -573,102 +650,114 @@ __device__ __forceinline__ void phase_tiles(const hq_expert& ed, Ws& w, const Di
       }
       uint8_t* sdst = base + NMAT * kRows * stride + mi * sbytes;
       if (G >= 8) {
-        if (lane < kRows) cp_async16(sdst + lane * 16, sbase[mi] + static_cast<size_t>(m0 + lane) * G + (pg & ~7), 16);
+        if (lane < kRows) cp_async16(sdst + lane * 16, sbase[mi] + static_cast<size_t>(m0 + lane) * G + (g0 & ~7), 16);
       } else if (lane < 2 * G) {
         cp_async16(sdst + lane * 16, reinterpret_cast<const uint8_t*>(sbase[mi] + static_cast<size_t>(m0) * G) + lane * 16, 16);
       }
     }
     cp_async_mbar_arrive(&rs.bars[slot]);
-    pg += len;
-    if (pg >= G) {
-      pg = 0;
-      ++pj;
-    }
+    pu += len;
     ++rs.issued;
   };
   if (!rs.ok) return;
-  for (int k2 = 0; k2 < kRing && pj < sa.w1; ++k2) issue(rs.issued % kRing);
+  for (int k2 = 0; k2 < kRing && pu < ub; ++k2) issue(rs.issued % kRing);
 
-  // consumer: this lane's B blocks (column g, k-quad t), or the zero block
-  const bool has_b = g < sa.ncol;
-  const uint4* zero_blk = reinterpret_cast<const uint4*>(zc + G * 8);
+  // consumer: this lane's B blocks (column g of the segment, k-quad t), or the zero block
+  const bool has_b = g < sg.ncol;
+  const uint4* zero_blk = reinterpret_cast<const uint4*>(zc + kMaxSeg * G * 8);
+  const float* zck = zc + k * G * 8;
   const uint4* bl;
   int bstep;  // uint4 per group
   int bo[4];  // uint4 offset of piece i within a block
   if constexpr (BSMEM) {
-    bl = has_b ? xs + (g * 4 + t) * 4 : zero_blk;
-    bstep = has_b ? sa.ncol * 16 : 0;
-    const int sw = has_b ? bswz(g, t) : 0;
+    bl = has_b ? xs + ((sg.col0 + g) * 4 + t) * 4 : zero_blk;
+    bstep = has_b ? cols * 16 : 0;
+    const int sw = has_b ? bswz(sg.col0 + g, t) : 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) bo[i] = i ^ sw;
   } else {
-    bl = has_b ? reinterpret_cast<const uint4*>(bsrc + (sa.brow_g * G * 4 + t) * kXq) : zero_blk;
+    bl = has_b ? reinterpret_cast<const uint4*>(bsrc + (seg_brow<PHASE>(w, d, sg, g) * G * 4 + t) * kXq) : zero_blk;
     bstep = has_b ? 4 * kXq / 8 : 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) bo[i] = i;
   }
-  for (int j = sa.w0; j < sa.w1; ++j) {
-    const int m0 = (sa.tile0 + j) * kRows;
-    float acc[NMAT][4] = {};
-    uint4 bq[4];
-    if constexpr (!BSMEM) {
+  float acc[NMAT][4] = {};
+  int tile_g0 = -1;  // first group of the current tile this warp computes
+  uint4 bq[4];
+  for (int u = ua; u < ub;) {
+    int j, g0, len;
+    chunk_of(u, j, g0, len);
+    if (tile_g0 < 0) {
+      tile_g0 = g0;
+      if constexpr (!BSMEM) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) bq[i] = bl[bo[i]];
+        for (int i = 0; i < 4; ++i) bq[i] = bl[g0 * bstep + bo[i]];
+      }
     }
-    for (int g0 = 0; g0 < G; g0 += len) {
-      const int slot = rs.consumed % kRing;
-      if (!mbar_wait(&rs.bars[slot], (rs.consumed / kRing) & 1)) {
-        rs.ok = false;
-        return;
-      }
-      __syncwarp();
-      const uint8_t* base = rs.ring + slot * ps.cbytes;
-      const __half* scb = reinterpret_cast<const __half*>(base + NMAT * kRows * stride);
-      for (int jj = 0; jj < len; ++jj) {
-        const int gi = g0 + jj;
-        uint4 bn[4];
-        if constexpr (BSMEM) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) bq[i] = bl[gi * bstep + bo[i]];
-        } else {
-          // the next group's blocks, one group ahead of their use
-          const int gn = gi + 1 < G ? gi + 1 : gi;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) bn[i] = bl[gn * bstep + bo[i]];
-        }
-        const float2 z = *reinterpret_cast<const float2*>(zc + gi * 8 + 2 * t);
-        const int sa_idx = G >= 8 ? g * 8 + (gi & 7) : g * G + gi;
-        const int sb_idx = G >= 8 ? (g + 8) * 8 + (gi & 7) : (g + 8) * G + gi;
-#pragma unroll
-        for (int mi = 0; mi < NMAT; ++mi) {
-          const uint8_t* ra = base + mi * kRows * stride + g * stride + jj * GB + t * 4 * BITS;
-          const __half* scp = scb + mi * (sbytes / 2);
-          group_mma<BITS>(ra, ra + 8 * stride, bq, z, __half2float(scp[sa_idx]),
-                          __half2float(scp[sb_idx]), acc[mi]);
-        }
-        if constexpr (!BSMEM) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) bq[i] = bn[i];
-        }
-      }
-      __syncwarp();
-      if (pj < sa.w1) issue(slot);
-      ++rs.consumed;
+    const int slot = rs.consumed % kRing;
+    if (!mbar_wait(&rs.bars[slot], (rs.consumed / kRing) & 1)) {
+      rs.ok = false;
+      return;
     }
-    // epilogue: rows g, g+8; columns 2t, 2t+1
+    __syncwarp();
+    const uint8_t* base = rs.ring + slot * ps.cbytes;
+    const __half* scb = reinterpret_cast<const __half*>(base + NMAT * kRows * stride);
+    for (int jj = 0; jj < len; ++jj) {
+      const int gi = g0 + jj;
+      uint4 bn[4];
+      if constexpr (BSMEM) {
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      const int col = 2 * t + (q4 & 1);
-      const int m = m0 + g + 8 * (q4 >> 1);
-      if (col < sa.ncol && m < sa.M) {
-        const size_t prow = static_cast<size_t>(sa.off + col);
-        if (PHASE == 0) {
-          const float gv = acc[0][q4] * kUnit, uv = acc[NMAT - 1][q4] * kUnit;
-          w.h[prow * d.inter + m] = gv / (1.f + expf(-gv)) * uv;
+        for (int i = 0; i < 4; ++i) bq[i] = bl[gi * bstep + bo[i]];
+      } else {
+        // the next group's blocks, one group ahead of their use
+        const int gn = gi + 1 < G ? gi + 1 : gi;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bn[i] = bl[gn * bstep + bo[i]];
+      }
+      const float2 z = *reinterpret_cast<const float2*>(zck + gi * 8 + 2 * t);
+      const int sa_idx = G >= 8 ? g * 8 + (gi & 7) : g * G + gi;
+      const int sb_idx = G >= 8 ? (g + 8) * 8 + (gi & 7) : (g + 8) * G + gi;
+#pragma unroll
+      for (int mi = 0; mi < NMAT; ++mi) {
+        const uint8_t* ra = base + mi * kRows * stride + g * stride + jj * GB + t * 4 * BITS;
+        const __half* scp = scb + mi * (sbytes / 2);
+        group_mma<BITS>(ra, ra + 8 * stride, bq, z, __half2float(scp[sa_idx]),
+                        __half2float(scp[sb_idx]), acc[mi]);
+      }
+      if constexpr (!BSMEM) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) bq[i] = bn[i];
+      }
+    }
+    __syncwarp();
+    if (pu < ub) issue(slot);
+    ++rs.consumed;
+    u += len;
+    if (g0 + len == G || u == ub) {
+      // this warp's part of tile j is done
+      float4 o[2];
+#pragma unroll
+      for (int mi = 0; mi < 2; ++mi) {
+        const int mm = mi < NMAT ? mi : 0;
+        o[mi] = make_float4(acc[mm][0], acc[mm][1], acc[mm][2], acc[mm][3]);
+      }
+      if (tile_g0 == 0 && g0 + len == G) {
+        seg_store<PHASE>(w, d, sg, (sg.tile0 + j) * kRows, o, lane);
+      } else {
+        const int tf = sg.unit0 + (j << lgG);  // the tile's first unit
+        if (tf <= u0 && u0 < tf + G) {  // the tile holding u0 (constant indices: registers)
+          part[0][0] = o[0];
+          part[0][1] = o[1];
+          ptile[0] = sg.item0 + j;
         } else {
-          w.d[prow * d.hidden + m] = acc[0][q4] * kUnit;
+          part[1][0] = o[0];
+          part[1][1] = o[1];
+          ptile[1] = sg.item0 + j;
         }
       }
+#pragma unroll
+      for (int mi = 0; mi < NMAT; ++mi) acc[mi][0] = acc[mi][1] = acc[mi][2] = acc[mi][3] = 0.f;
+      tile_g0 = -1;
     }
   }
 }
@@ -677,33 +766,35 @@ __device__ __forceinline__ void phase_tiles(const hq_expert& ed, Ws& w, const Di
 //
 // Work item i is 16-row tile i % TPB of block i / TPB, a block being one
 // expert's <= 8-token column block (w.blk); CTA c owns items [bounds[c],
-// bounds[c + 1]), split by tile weight, and walks them one segment (the part
-// of one block) at a time.  Per segment the CTA writes the zero-point terms of the
-// block's <= 8 columns to shared memory and, when BSMEM, stages the block's
-// B fragments (the rotated activations, every group) there too; then its
-// warps split the segment's tiles and stream each tile's codes and scales
-// through a private cp.async ring.  Without BSMEM (K too large for the B
-// fragments to fit beside the rings) each lane reads its B blocks from
-// global memory, one group ahead.
+// bounds[c + 1]) (split by tile weight) and walks them in passes.  A pass
+// takes up to kMaxSeg consecutive blocks' parts (segments) with at most 8
+// columns in all; the CTA stages their zero-point terms and, when BSMEM,
+// their B fragments (the rotated activations) in shared memory, then its 16
+// warps split the pass's (item, group) units evenly, each streaming codes and
+// scales through a private cp.async ring.  Tiles split between warps are
+// summed in warp order through shared memory after one barrier.  Without
+// BSMEM (K too large for the fragments beside the rings) lanes read their B
+// blocks from global memory, one group ahead.
 template <int PHASE, bool BSMEM>
 __global__ void __launch_bounds__(kWarps * 32, 1)
     moe_phase_kernel(const hq_expert* __restrict__ ex, Ws w, Dims d, PhaseSmem ps) {
+  constexpr int NMAT = PHASE == 0 ? 2 : 1;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2;
   const int K = PHASE == 0 ? d.hidden : d.inter;
   const int M = PHASE == 0 ? d.inter : d.hidden;
   const int G = K / kGroup;
   const int TPB = M / kRows;  // tiles per block
-  float* zc = reinterpret_cast<float*>(smem);  // [G][8], then a zero B block (64 B)
-  uint4* xs = reinterpret_cast<uint4*>(smem + ps.xs_off);  // [G][ncol][4][4 pieces], swizzled
+  PassMeta& pm = *reinterpret_cast<PassMeta*>(smem);
+  float* zc = reinterpret_cast<float*>(smem + ps.zc_off);  // [kMaxSeg][G][8], then a zero B block
+  uint4* xs = reinterpret_cast<uint4*>(smem + ps.xs_off);  // [G][cols][4][4 pieces], swizzled
   uint8_t* ring = smem + ps.ring_off + warp * kRing * ps.cbytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ps.bar_off) + warp * kRing;
   if (lane == 0) {
     for (int i = 0; i < kRing; ++i) mbar_init(&bars[i], 32);
     fence_mbar_init();
   }
-  if (tid < 16) (zc + G * 8)[tid] = 0.f;
+  if (tid < 16) (zc + kMaxSeg * G * 8)[tid] = 0.f;
   __syncthreads();
   pdl_launch_dependents();
   pdl_wait();  // routing lists and activations come from the previous kernels
@@ -714,64 +805,150 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   RingState rs{ring, bars, 0, 0, true};  // this warp's ring, over the whole kernel
 
   for (int it = ib; it < ie;) {
-    // ---- the segment: items [it, se) of one (expert, column block)
-    const int b = it / TPB;
-    const uint2 bk = w.blk[b];
-    const int e = static_cast<int>(bk.x);
-    const int cb = static_cast<int>(bk.y);
-    const int tile_first = it - b * TPB;
-    const int se = min(ie, (b + 1) * TPB);
-    const hq_expert ed = ex[e];
-    const int bits = ed.bits;
-    const int L = layout_index(bits);
-    const int off = w.offsets[e] + 8 * cb;
-    const int ncol = min(8, w.counts[e] - 8 * cb);
-    // B-operand row of column col of this block
-    auto brow = [&](int col) -> size_t {
-      const int p = off + col;
-      return PHASE == 0 ? static_cast<size_t>(L) * d.T + w.sorted[p] / d.k : static_cast<size_t>(p);
-    };
-    __syncthreads();  // every warp is done with the previous segment's B and zc
-    {
+    __syncthreads();  // the previous pass is done with the metadata, B, zc and rings
+    // ---- plan the pass (warp 0): lane k looks at block b0 + k
+    if (warp == 0) {
+      const int b = it / TPB + lane;
+      const bool valid = lane < kMaxSeg && b * TPB < ie;
+      int e = 0, cb = 0, ncol = 0, off = 0;
+      if (valid) {
+        const uint2 bk = w.blk[b];
+        e = static_cast<int>(bk.x);
+        cb = static_cast<int>(bk.y);
+        off = w.offsets[e] + 8 * cb;
+        ncol = min(8, w.counts[e] - 8 * cb);
+      }
+      const int item0 = max(it, b * TPB), item1 = min(ie, (b + 1) * TPB);
+      const int ni = valid ? item1 - item0 : 0;
+      const hq_expert ede = valid ? ex[e] : hq_expert{};
+      const int wt = valid ? ni * G * tile_weight(ede.bits) : 0;
+      int pc = ncol, pn = ni, pw = wt;  // inclusive prefix sums of columns, items, weights
+#pragma unroll
+      for (int m = 1; m < 32; m <<= 1) {
+        const int yc = __shfl_up_sync(0xffffffffu, pc, m);
+        const int yn = __shfl_up_sync(0xffffffffu, pn, m);
+        const int yw = __shfl_up_sync(0xffffffffu, pw, m);
+        if (lane >= m) {
+          pc += yc;
+          pn += yn;
+          pw += yw;
+        }
+      }
+      const bool take = valid && (lane == 0 || pc <= 8);
+      const int nseg = __popc(__ballot_sync(0xffffffffu, take));
+      if (take) {
+        SegInfo& sg = pm.seg[lane];
+        sg.ed = ede;
+        sg.wt0 = pw - wt;
+        sg.item0 = item0;
+        sg.item1 = item1;
+        sg.tile0 = item0 - b * TPB;
+        sg.unit0 = (pn - ni) * G;
+        sg.off = off;
+        sg.ncol = ncol;
+        sg.col0 = pc - ncol;
+        sg.L = layout_index(sg.ed.bits);
+      }
+      if (lane == nseg - 1) {
+        pm.nseg = nseg;
+        pm.cols = pc;
+        pm.units = pn * G;
+        pm.wtot = pw;
+      }
+    }
+    __syncthreads();
+    const int nseg = pm.nseg, cols = pm.cols, U = pm.units;
+    // ---- stage the pass's zero-point terms and (BSMEM) B fragments
+    for (int k = 0; k < nseg; ++k) {
+      const SegInfo& sg = pm.seg[k];
       if constexpr (BSMEM) {
         // 64 bytes of each 80-byte block (the rest is padding), 16-byte pieces
         const int per_col = G * 16;
-        for (int i = tid; i < ncol * per_col; i += kWarps * 32) {
-          const int col = i / per_col, r = i - col * per_col;
+        for (int i = tid; i < sg.ncol * per_col; i += kWarps * 32) {
+          const int cl = i / per_col, r = i - cl * per_col;
           const int gg = r >> 4, q = (r >> 2) & 3, pc = r & 3;
-          cp_async16(xs + ((gg * ncol + col) * 4 + q) * 4 + (pc ^ bswz(col, q)),
-                     bsrc + ((brow(col) * G + gg) * 4 + q) * kXq + pc * 8, 16);
+          const int col = sg.col0 + cl;
+          cp_async16(xs + ((gg * cols + col) * 4 + q) * 4 + (pc ^ bswz(col, q)),
+                     bsrc + ((seg_brow<PHASE>(w, d, sg, cl) * G + gg) * 4 + q) * kXq + pc * 8, 16);
         }
       }
-      // zero-point terms -zero * sum_k x' * 2^-24 (0 for absent columns)
-      const float zneg = -static_cast<float>(ed.zero) * 5.9604644775390625e-8f;
+      // -zero * sum_k x' * 2^-24 per group and column (0 for absent columns)
+      const float zneg = -static_cast<float>(sg.ed.zero) * 5.9604644775390625e-8f;
       for (int i = tid; i < G * 8; i += kWarps * 32) {
-        const int gg = i >> 3, col = i & 7;
-        zc[i] = col < ncol ? zneg * sums[brow(col) * G + gg] : 0.f;
+        const int gg = i >> 3, cl = i & 7;
+        zc[k * G * 8 + i] = cl < sg.ncol ? zneg * sums[seg_brow<PHASE>(w, d, sg, cl) * G + gg] : 0.f;
       }
-      if constexpr (BSMEM) asm volatile("cp.async.wait_all;" ::: "memory");
     }
+    if constexpr (BSMEM) asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
 
-    // ---- this warp's tiles of the segment: items [w0, w1)
-    const int n = se - it;
-    SegArgs sa;
-    sa.w0 = it + (n * warp) / kWarps;
-    sa.w1 = it + (n * (warp + 1)) / kWarps;
-    sa.tile0 = tile_first - it;  // tile of item j is tile0 + j
-    sa.off = off;
-    sa.ncol = ncol;
-    sa.G = G;
-    sa.K = K;
-    sa.M = M;
-    sa.brow_g = g < ncol ? brow(g) : 0;
-    switch (bits) {
-      case 2: phase_tiles<PHASE, BSMEM, 2>(ed, w, d, ps, sa, rs, zc, xs, bsrc, lane); break;
-      case 3: phase_tiles<PHASE, BSMEM, 3>(ed, w, d, ps, sa, rs, zc, xs, bsrc, lane); break;
-      case 4: phase_tiles<PHASE, BSMEM, 4>(ed, w, d, ps, sa, rs, zc, xs, bsrc, lane); break;
-      default: phase_tiles<PHASE, BSMEM, 8>(ed, w, d, ps, sa, rs, zc, xs, bsrc, lane); break;
+    // ---- this warp's units [u0, u1) of the pass (equal shares of the
+    // weight: unit u of segment k weighs its tile weight), one piece per segment
+    auto unit_at = [&](int wi) {  // first unit whose weight prefix reaches wi / kWarps of the total
+      const int target = static_cast<int>((static_cast<long long>(pm.wtot) * wi) / kWarps);
+      int k = 0;
+      while (k + 1 < nseg && pm.seg[k + 1].wt0 <= target) ++k;
+      const SegInfo& sg = pm.seg[k];
+      const int tw = tile_weight(sg.ed.bits);
+      const int u = sg.unit0 + (target - sg.wt0 + tw - 1) / tw;
+      return min(u, sg.unit0 + (sg.item1 - sg.item0) * G);
+    };
+    const int u0 = warp == 0 ? 0 : unit_at(warp);
+    const int u1 = warp == kWarps - 1 ? U : unit_at(warp + 1);
+    float4 part[2][2];
+    int ptile[2] = {-1, -1};
+    for (int k = 0; k < nseg && rs.ok; ++k) {
+      const SegInfo& sg = pm.seg[k];
+      const int sa = max(u0, sg.unit0), sb = min(u1, sg.unit0 + (sg.item1 - sg.item0) * G);
+      if (sa >= sb) continue;
+      switch (sg.ed.bits) {
+        case 2: phase_piece<PHASE, BSMEM, 2>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        case 3: phase_piece<PHASE, BSMEM, 3>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        case 4: phase_piece<PHASE, BSMEM, 4>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        default: phase_piece<PHASE, BSMEM, 8>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+      }
     }
-    it = se;
+    // ---- tiles split between warps: each warp leaves its partial sums in
+    // its (drained) ring; the warp whose range holds a tile's first unit adds
+    // the later contributors' parts in warp order and runs the epilogue
+    float4* mine = reinterpret_cast<float4*>(ring);  // [2 which][2 mat][32 lanes]
+    if (rs.ok) {
+#pragma unroll
+      for (int wh = 0; wh < 2; ++wh) {
+#pragma unroll
+        for (int mi = 0; mi < NMAT; ++mi) mine[(wh * 2 + mi) * 32 + lane] = part[wh][mi];
+      }
+    }
+    __syncthreads();
+    if (rs.ok) {
+#pragma unroll
+      for (int wh = 0; wh < 2; ++wh) {
+        const int item = ptile[wh];
+        if (item < 0 || (wh == 1 && item == ptile[0])) continue;
+        int k = 0;
+        while (k + 1 < nseg && item >= pm.seg[k].item1) ++k;
+        const SegInfo& sg = pm.seg[k];
+        const int tf = sg.unit0 + (item - sg.item0) * G, tz = tf + G - 1;
+        if (tf < u0) continue;  // an earlier warp holds the tile's first unit
+        float4 o[2] = {part[wh][0], part[wh][1]};
+        for (int w2 = warp + 1; w2 < kWarps; ++w2) {
+          const int wb = unit_at(w2);
+          if (wb > tz) break;
+          if (wb == (w2 == kWarps - 1 ? U : unit_at(w2 + 1))) continue;  // empty range
+          const float4* other = reinterpret_cast<const float4*>(smem + ps.ring_off + w2 * kRing * ps.cbytes);
+#pragma unroll
+          for (int mi = 0; mi < NMAT; ++mi) {
+            const float4 q4 = other[(0 * 2 + mi) * 32 + lane];  // the tile is that warp's first
+            o[mi].x += q4.x;
+            o[mi].y += q4.y;
+            o[mi].z += q4.z;
+            o[mi].w += q4.w;
+          }
+        }
+        seg_store<PHASE>(w, d, sg, (sg.tile0 + item - sg.item0) * kRows, o, lane);
+      }
+    }
+    it += U / G;
   }
   if (!rs.ok) {
     // a ring wait timed out: report it and let the copies still in flight land
