@@ -100,4 +100,80 @@ __device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>:
   }
 }
 
+// The same transform for a 512-thread CTA (16 warps) and 512 <= K <= 8192:
+// K = 16 (warps) x 32 (lanes) x E (registers), E = K / 512.  Stages 1 and 2
+// as above; for the 16 warps (stage 3) thread t takes column p = t / T of the
+// shared-memory image (T = 16 / E threads per column) and the E warps h E ..
+// h E + E - 1 of it (h = t % T): butterflies over those E in registers, then
+// over the T threads of the column with shuffles.  Twice the threads of the
+// 8-warp shape at K = 4096, so half the work per thread on the critical path.
+template <int LOGK>
+struct Fwht512 {
+  static constexpr int K = 1 << LOGK;
+  static constexpr int E = K / 512;
+  static constexpr int T = 16 / E;
+  static constexpr int SMEM_FLOATS = K + K / 32;
+  static_assert(LOGK >= 9 && LOGK <= 13, "K must be in [512, 8192]");
+};
+
+// On entry thread tid (of 512) holds v[e] = u[tid*E + e]; on exit the
+// transformed (unnormalised) row is in buf[fwht_pad(i)] and the block has
+// synchronised.  Every thread of the block must call this.
+template <int LOGK>
+__device__ __forceinline__ void fwht_block512(float (&v)[Fwht512<LOGK>::E], float* buf) {
+  using S = Fwht512<LOGK>;
+  constexpr int E = S::E, T = S::T;
+  const int tid = threadIdx.x, lane = tid & 31;
+#pragma unroll
+  for (int h = 1; h < E; h <<= 1) {
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if ((e & h) == 0) {
+        const float a = v[e], b = v[e + h];
+        v[e] = a + b;
+        v[e + h] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const float sgn = (lane & m) ? -1.f : 1.f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float p = __shfl_xor_sync(0xffffffffu, v[e], m);
+      v[e] = fmaf(sgn, v[e], p);
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < E; ++e) buf[fwht_pad(tid * E + e)] = v[e];
+  __syncthreads();
+  const int col = tid / T, h = tid % T;
+  float r[E];
+#pragma unroll
+  for (int i = 0; i < E; ++i) r[i] = buf[fwht_pad((h * E + i) * 32 * E + col)];
+#pragma unroll
+  for (int hb = 1; hb < E; hb <<= 1) {
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      if ((i & hb) == 0) {
+        const float a = r[i], b = r[i + hb];
+        r[i] = a + b;
+        r[i + hb] = a - b;
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 1; j < T; j <<= 1) {
+    const float sgn = (h & j) ? -1.f : 1.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float q = __shfl_xor_sync(0xffffffffu, r[i], j);
+      r[i] = fmaf(sgn, r[i], q);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < E; ++i) buf[fwht_pad((h * E + i) * 32 * E + col)] = r[i];
+  __syncthreads();
+}
+
 }  // namespace hq

@@ -161,6 +161,21 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
   for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, inv_sqrt_k, zero, xs, zc, lane);
 }
 
+// The FWHT a fused GEMV CTA (16 warps) runs on one row: the 512-thread shape
+// for K >= 512, else the prep kernel's (at most 8 warps).
+template <int LOGK, bool WIDE = (LOGK >= 9)>
+struct FusedFwht;
+template <int LOGK>
+struct FusedFwht<LOGK, true> {
+  static constexpr int E = Fwht512<LOGK>::E, THREADS = 512;
+  static __device__ __forceinline__ void run(float (&v)[E], float* buf) { fwht_block512<LOGK>(v, buf); }
+};
+template <int LOGK>
+struct FusedFwht<LOGK, false> {
+  static constexpr int E = FwhtShape<LOGK, 3>::E, THREADS = FwhtShape<LOGK, 3>::THREADS;
+  static __device__ __forceinline__ void run(float (&v)[E], float* buf) { fwht_block<LOGK, 3>(v, buf); }
+};
+
 // Splitting U units into n contiguous ranges: range i is [unit_begin(i), unit_begin(i + 1)).
 __device__ __forceinline__ uint32_t unit_begin(uint32_t i, uint32_t U, uint32_t n) {
   return static_cast<uint32_t>((static_cast<uint64_t>(i) * U) / n);
@@ -257,10 +272,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
   // ---- the rotated activations and zero-point terms
   if constexpr (FUSED) {
-    // rotate each row here (the fwht_block shape of the prep kernel, so the
-    // values are the same bit for bit) while the first slots are in flight;
-    // the signs are weights, read before the wait
-    using FS = FwhtShape<LOGK, 3>;
+    // rotate each row here while the first slots are in flight (all 16 warps
+    // for K >= 512); the signs are weights, read before the wait
+    using FS = FusedFwht<LOGK>;
     static_assert(FS::E <= 32, "one sign bit per register");
     uint32_t neg = 0;  // bit e: value e of this thread's chunk flips sign
     if (tid < FS::THREADS && p.signs != nullptr) {
@@ -291,7 +305,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 #pragma unroll
         for (int e = 0; e < FS::E; ++e) v[e] = (neg >> e & 1u) ? -v[e] : v[e];
       }
-      fwht_block<LOGK, 3>(v, buf);
+      FS::run(v, buf);
       for (int gg = warp; gg < G; gg += kWarps) {
         put_group<BITS>(fl, buf, gg, n, p.N, p.inv_sqrt_k, p.zero, xs, zc, lane);
       }
