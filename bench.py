@@ -249,6 +249,7 @@ def run_ours(a):
                                               / pk["hbm"], 4)}
 
     b64 = measure_b64(device, stream, pk) if a.b64 else None
+    configs = measure_configs(device, stream, pk, l2) if a.b64 else None
     e2e = measure_e2e(device, layers, xs, a)
     e2e_ms = dist.max_over_ranks(e2e.pop("ms"), device)
     e2e["value"] = round(step_w * e2e["steps"] * world / (e2e_ms * 1e-3) / 1e9, 3)
@@ -277,6 +278,7 @@ def run_ours(a):
                      "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
         "per_bits": per_bits,
         "b64": b64,
+        "configs": configs,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * a.steps),
         "launches_per_step": int(launches_per_step),
@@ -328,6 +330,112 @@ def measure_b64(device, stream, pk):
          "timing": "CUDA-graph replay of one call, median of 20, L2 flushed before each",
          "batch16": out[16]}
     return r
+
+
+def _graph_us(stream, device, calls, reps=5):
+    """Median per-call time (us) of one CUDA graph holding `calls` back to back."""
+    with torch.cuda.stream(stream):
+        for c in calls:
+            c()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for c in calls:
+                c()
+        g.replay()
+        torch.cuda.synchronize(device)
+        times = []
+        for _ in range(reps):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            times.append(e0.elapsed_time(e1) * 1e3 / len(calls))
+    return statistics.median(times)
+
+
+def _device_copies(device, M, K, b, n, gen):
+    """n weight copies drawn on the device (uniform codes, fp16 scales U[0.005, 0.02])."""
+    out = []
+    for _ in range(n):
+        q = torch.randint(-2**31, 2**31 - 1, (M, K * b // 32), dtype=torch.int32, device=device,
+                          generator=gen)
+        sc = (torch.rand((M, K // 128), device=device, generator=gen) * 0.015 + 0.005).half()
+        out.append((q, sc))
+    return out
+
+
+def measure_configs(device, stream, pk, l2):
+    """The other workloads of the metric: the 4096x4096 4-bit linear at batch 1,
+    the 256-expert MoE layer (32 tokens, top-8) and the M=K=8192 sweep over
+    widths and batches (GEMV up to batch 8, tensor cores from 16).  Weights are
+    cycled over enough copies that every call reads HBM; each point is the
+    median over 5 replays of a graph of back-to-back calls."""
+    from bit_hadamard_rotated_b200 import (RotatedLinear, expert_table, hq_moe_experts,
+                                           hq_moe_workspace_size)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(4242)
+    res = {}
+
+    def linear_point(M, K, b, N):
+        wb = weight_bytes(M, K, b)
+        copies = max(2, math.ceil(4 * l2 / wb))
+        signs = torch.from_numpy(synth.linear(16, K, b, 1, seed=5)["signs"]).to(device)
+        lins = [RotatedLinear(q, sc, signs, b, 1 << (b - 1), max_batch=N)
+                for (q, sc) in _device_copies(device, M, K, b, copies, gen)]
+        x = torch.randn((N, K), device=device, generator=gen).half()
+        y = torch.empty((N, M), dtype=torch.float32, device=device)
+        us = _graph_us(stream, device, [lambda l=l: l(x, out=y) for l in lins])
+        gbs = wb / (us * 1e-6) / 1e9
+        tf = 2.0 * M * K * N / (us * 1e-6) / 1e12
+        r = {"us": round(us, 3), "weight_gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 4),
+             "tflops": round(tf, 2), "frac_bf16_peak": round(tf / pk["bf16"], 4),
+             "path": "tensor cores" if lins[0].uses_tensor_cores(N) else "GEMV",
+             "launches": lins[0].launches(N)}
+        del lins
+        return r
+
+    res["cfg_4096x4096_b4_n1"] = linear_point(4096, 4096, 4, 1)
+
+    # MoE layer: two copies of the expert weights, alternated, so calls read HBM
+    m = synth.moe(seed=1)
+    E, H, I, T, k = len(m["experts"]), m["hidden"], m["inter"], m["T"], m["k"]
+
+    def put(v):
+        return torch.from_numpy(np.ascontiguousarray(v)).to(device)
+
+    tables = []
+    for cpy in range(2):
+        ex = []
+        for e in m["experts"]:
+            d = dict(bits=e["bits"], zero=e["zero"])
+            for n in ("q_gate", "q_up", "q_down"):
+                d[n] = put(e[n].view(np.int32)) if cpy == 0 else torch.randint(
+                    -2**31, 2**31 - 1, e[n].shape, dtype=torch.int32, device=device, generator=gen)
+            for n in ("s_gate", "s_up", "s_down"):
+                d[n] = put(e[n])
+            ex.append(d)
+        tables.append((expert_table(ex, device), ex))
+    x, ids, w = put(m["x"]), put(m["topk_ids"].astype(np.int32)), put(m["topk_w"].astype(np.float32))
+    s_in, s_mid = put(m["s_in"]), put(m["s_mid"])
+    ws = torch.zeros(hq_moe_workspace_size(E, H, I, T, k), dtype=torch.uint8, device=device)
+    out = torch.empty((T, H), dtype=torch.float32, device=device)
+    us = _graph_us(stream, device, [lambda t=t: hq_moe_experts(t[0], E, H, I, x, ids, w, s_in, s_mid,
+                                                               out=out, workspace=ws)
+                                    for t in tables] * 4)
+    tb = synth.touched_weight_bytes(m)
+    res["moe_256x2048x512_t32_top8"] = {
+        "us": round(us, 2), "tokens_per_s": round(T / (us * 1e-6), 1),
+        "touched_weight_bytes": tb, "weight_gbs": round(tb / (us * 1e-6) / 1e9, 1),
+        "frac_hbm": round(tb / (us * 1e-6) / 1e9 / pk["hbm"], 4), "launches": 5}
+    del tables
+
+    sweep = {}
+    for b in (2, 3, 4, 8):
+        for N in (1, 2, 4, 8, 16, 32, 64, 128):
+            sweep[f"b{b}_n{N}"] = linear_point(8192, 8192, b, N)
+    res["sweep_8192x8192"] = sweep
+    return res
 
 
 def measure_e2e(device, layers, xs, a):

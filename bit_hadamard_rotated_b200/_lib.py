@@ -70,6 +70,8 @@ def lib() -> ctypes.CDLL:
         L.hq_launch_count.restype = ctypes.c_uint64
         L.hq_linear_launches.argtypes = [ctypes.POINTER(HqWeight), _i]
         L.hq_linear_launches.restype = _i
+        L.hq_linear_uses_tensor_cores.argtypes = [ctypes.POINTER(HqWeight), _i]
+        L.hq_linear_uses_tensor_cores.restype = _i
         L.hq_linear_noalloc.argtypes = [ctypes.POINTER(HqWeight), _vp, _i, _vp, _vp]
         L.hq_linear_noalloc.restype = _i
         L.hq_moe_launches.argtypes = []

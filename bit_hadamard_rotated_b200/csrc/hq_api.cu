@@ -10,7 +10,8 @@
 namespace hq {
 
 static std::atomic<uint64_t> g_launches{0};
-static std::atomic<int> g_tc_min_batch{9};
+// Batch from which hq_linear uses the tensor-core GEMM; 0 = automatic.
+static std::atomic<int> g_tc_min_batch{0};
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -54,7 +55,16 @@ static int gemv_col_block(int bits, int K) {
 // Batches of at least the tensor-core threshold run on the tcgen05 GEMM
 // (when a tile plan fits this width and K); smaller ones on the GEMV.
 static bool use_tc(const hq_weight* w, int batch) {
-  return batch >= g_tc_min_batch.load(std::memory_order_relaxed) &&
+  int min_batch = g_tc_min_batch.load(std::memory_order_relaxed);
+  if (min_batch == 0) {
+    // automatic, from batch sweeps on B200: the GEMV stages its activation
+    // fragments (2.5 K bytes per column) in shared memory; past ~90 KB of
+    // them (5 columns at K = 8192) its copy rings become too shallow for
+    // 3/4/8-bit rows, and the tensor-core GEMM (flat in time up to batch 32)
+    // wins; 2-bit rows and smaller K stay on the GEMV up to batch 8
+    min_batch = (w->bits >= 3 && w->K >= 8192) ? 5 : 9;
+  }
+  return batch >= min_batch &&
          tc_col_block(w->bits, w->K) > 0;
 }
 
@@ -108,7 +118,7 @@ const char* hq_status_string(hq_status s) {
 uint64_t hq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int hq_set_tc_min_batch(int n) {
-  if (n < 1) return g_tc_min_batch.load();
+  if (n < 0) return g_tc_min_batch.load();
   return g_tc_min_batch.exchange(n);
 }
 
@@ -132,6 +142,11 @@ hq_status hq_rotate(const void* x, hq_dtype x_dtype, void* x_rot, hq_dtype out_d
 size_t hq_linear_workspace_size(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch < 0) return 0;
   return linear_ws(nullptr, w, batch).bytes;
+}
+
+int hq_linear_uses_tensor_cores(const hq_weight* w, int batch) {
+  if (check_weight(w) != HQ_OK || batch <= 0) return -1;
+  return use_tc(w, batch) ? 1 : 0;
 }
 
 int hq_linear_launches(const hq_weight* w, int batch) {

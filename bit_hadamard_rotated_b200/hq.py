@@ -112,6 +112,10 @@ class RotatedLinear:
     def launches(self, batch: int) -> int:
         return int(lib().hq_linear_launches(ctypes.byref(self.w), batch))
 
+    def uses_tensor_cores(self, batch: int) -> bool:
+        """Whether a call of this batch runs on the tensor-core GEMM (else the GEMV)."""
+        return int(lib().hq_linear_uses_tensor_cores(ctypes.byref(self.w), batch)) == 1
+
     def __call__(self, x, out=None, stream=None):
         N = x.shape[0]
         if out is None:

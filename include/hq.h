@@ -208,8 +208,14 @@ int hq_linear_launches(const hq_weight* w, int batch);
  * rotate h, down, combine). */
 int hq_moe_launches(void);
 
-/* Batch size from which hq_linear uses the tensor-core GEMM (default 9).
- * Returns the previous value; values < 1 are ignored. */
+/* 1 if hq_linear runs this weight and batch on the tensor-core GEMM, 0 if on
+ * the GEMV, -1 for an invalid weight or batch < 1 (nothing is launched). */
+int hq_linear_uses_tensor_cores(const hq_weight* w, int batch);
+
+/* Batch size from which hq_linear uses the tensor-core GEMM (when K >= 1024).
+ * 0 (the default) selects it automatically: from batch 5 for 3/4/8-bit codes
+ * with K >= 8192, else from batch 9.  A value >= 1 applies to every weight.
+ * Returns the previous value; negative values change nothing. */
 int hq_set_tc_min_batch(int n);
 
 #ifdef __cplusplus

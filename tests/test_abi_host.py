@@ -148,3 +148,30 @@ def test_moe_rejects_bad_args(L):
     assert L.hq_moe_workspace_size(0, 256, 128, 4, 2) == 0
     assert L.hq_moe_launches() == 5
     assert L.hq_launch_count() == before
+
+
+def test_tc_min_batch_override_and_automatic_default():
+    from bit_hadamard_rotated_b200._lib import lib
+    L = lib()
+    old = L.hq_set_tc_min_batch(-1)  # negative: read only
+    assert old == 0                 # automatic by default
+    assert L.hq_set_tc_min_batch(7) == 0
+    assert L.hq_set_tc_min_batch(-5) == 7
+    assert L.hq_set_tc_min_batch(0) == 7
+    assert L.hq_set_tc_min_batch(-1) == 0
+
+
+def test_linear_path_choice():
+    """The automatic GEMV / tensor-core switch (host only: nothing is launched)."""
+    from bit_hadamard_rotated_b200._lib import lib
+    L = lib()
+
+    def path(bits, K, batch):
+        w = HqWeight(bits, 256, K, 1 << (bits - 1), FAKE, FAKE, None)
+        return L.hq_linear_uses_tensor_cores(ctypes.byref(w), batch)
+
+    assert path(3, 8192, 4) == 0 and path(3, 8192, 5) == 1
+    assert path(8, 16384, 5) == 1 and path(4, 4096, 8) == 0 and path(4, 4096, 9) == 1
+    assert path(2, 8192, 8) == 0 and path(2, 8192, 9) == 1
+    assert path(4, 512, 64) == 0      # K < 1024: GEMV at every batch
+    assert path(4, 4096, 0) == -1 and path(5, 4096, 4) == -1

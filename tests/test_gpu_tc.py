@@ -101,6 +101,22 @@ def test_tc_linear_parity(bits, M, K, N):
     assert_within(y, want, bound, what=f"tc b{bits} M{M} K{K} N{N}")
 
 
+@pytest.mark.parametrize("bits,N", [(3, 5), (4, 6), (8, 8), (2, 8), (4, 4)])
+def test_small_batches_at_large_k_either_path(bits, N):
+    """At K = 8192 batches from 5 of 3/4/8-bit codes take the tensor-core GEMM
+    (automatic switch), 2-bit rows and batch 4 the GEMV; both match the oracle."""
+    import ctypes
+    from bit_hadamard_rotated_b200._lib import lib
+    M, K = 300, 8192
+    d = synth.linear(M, K, bits, N, seed=31 + bits + N)
+    _, _, _, w = weight(d)
+    assert lib().hq_linear_uses_tensor_cores(ctypes.byref(w), N) == (1 if bits >= 3 and N >= 5 else 0)
+    y, launches, expect = run(d)
+    assert launches == expect
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y, want, bound, what=f"b{bits} N{N} K{K}")
+
+
 @pytest.mark.parametrize("bits", [2, 3, 4, 8])
 def test_tc_nondefault_zero_null_signs_loguniform(bits):
     M, K, N = 200, 2048, 40
