@@ -440,21 +440,32 @@ def measure_configs(device, stream, pk, l2):
 
 def measure_e2e(device, layers, xs, a):
     """Same metric through the public Python API with host buffers: every step
-    copies each layer's activations from pinned host memory and reads the
-    outputs back to pinned host memory, inside the timed region."""
+    copies the step's activations (the three layers' inputs, one pinned host
+    buffer) to the device in one copy, runs the layers, and reads their outputs
+    back to one pinned host buffer in one copy, inside the timed region."""
     copies = len(layers)
-    xh = [x.cpu().pin_memory() for x in xs]
-    xd = [torch.empty_like(x) for x in xs]
-    yh = [torch.empty((1, M), dtype=torch.float32).pin_memory() for (M, K, b) in LAYERS]
-    yd = [torch.empty((1, M), dtype=torch.float32, device=device) for (M, K, b) in LAYERS]
+    xsz = [x.numel() for x in xs]
+    ysz = [M for (M, K, b) in LAYERS]
+    xh = torch.cat([x.reshape(-1).cpu() for x in xs]).pin_memory()
+    xd = torch.empty_like(xh, device=device)
+    yh = torch.empty(sum(ysz), dtype=torch.float32).pin_memory()
+    yd = torch.empty(sum(ysz), dtype=torch.float32, device=device)
+    xv, yv, o = [], [], 0
+    for li, n in enumerate(xsz):
+        xv.append(xd[o:o + n].view(1, -1))
+        o += n
+    o = 0
+    for n in ysz:
+        yv.append(yd[o:o + n].view(1, -1))
+        o += n
     steps = min(a.steps, 2000)
     stream = torch.cuda.current_stream(device)
 
     def one(c):
+        xd.copy_(xh, non_blocking=True)
         for li in range(len(LAYERS)):
-            xd[li].copy_(xh[li], non_blocking=True)
-            layers[c][li](xd[li], out=yd[li])
-            yh[li].copy_(yd[li], non_blocking=True)
+            layers[c][li](xv[li], out=yv[li])
+        yh.copy_(yd, non_blocking=True)
 
     for i in range(3):
         one(i % copies)
@@ -466,11 +477,10 @@ def measure_e2e(device, layers, xs, a):
     e1.record(stream)
     torch.cuda.synchronize(device)
     ms = e0.elapsed_time(e1)
-    step_w = sum(weight_bytes(M, K, b) for (M, K, b) in LAYERS)
     return {"ms": ms, "value": None, "unit": "GB/s", "steps": steps,
-            "h2d_bytes_per_step": sum(int(x.numel() * 2) for x in xs),
-            "d2h_bytes_per_step": sum(M * 4 for (M, K, b) in LAYERS),
-            "api": "RotatedLinear.__call__ -> hq_linear (C ABI), eager launches"}
+            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 4),
+            "api": "RotatedLinear.__call__ -> hq_linear (C ABI), eager launches; one H2D and "
+                   "one D2H copy per step"}
 
 
 # ---------------------------------------------------------------- CPU oracle baseline

@@ -23,6 +23,15 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
+def _raw_stream(stream, device_index):
+    """The stream handle as an int: the given stream, else the current one of
+    the device (read without building a Stream object)."""
+    if stream is not None:
+        return stream.cuda_stream
+    get = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+    return get(device_index) if get is not None else torch.cuda.current_stream().cuda_stream
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and not t.is_cuda:
@@ -100,6 +109,12 @@ class RotatedLinear:
         self.w = make_weight(qweight, scales, signs, bits, zero)
         self.workspace = torch.zeros(max(hq_linear_workspace_size(self.w, max_batch), 256),
                                      dtype=torch.uint8, device=qweight.device)
+        # per-call marshalling reduced to the two tensor pointers and the stream
+        self._fn = lib().hq_linear
+        self._wref = ctypes.byref(self.w)
+        self._ws = self.workspace.data_ptr()
+        self._ws_bytes = self.workspace.numel()
+        self._dev = qweight.device.index if qweight.device.index is not None else torch.cuda.current_device()
 
     @property
     def M(self):
@@ -120,9 +135,10 @@ class RotatedLinear:
         N = x.shape[0]
         if out is None:
             out = torch.empty((N, self.w.M), dtype=torch.float32, device=x.device)
-        st = lib().hq_linear(ctypes.byref(self.w), _ptr(x), N, _ptr(out), _ptr(self.workspace),
-                             self.workspace.numel(), _stream(stream))
-        check(st, "hq_linear")
+        st = self._fn(self._wref, x.data_ptr(), N, out.data_ptr(), self._ws, self._ws_bytes,
+                      _raw_stream(stream, self._dev))
+        if st:
+            check(st, "hq_linear")
         return out
 
     def check_status(self, stream=None):
