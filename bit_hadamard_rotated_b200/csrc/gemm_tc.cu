@@ -105,6 +105,14 @@ __device__ __forceinline__ void tc_fence_after() {
 }
 __device__ __forceinline__ void tc_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// After tc_wait_ld: makes later uses of registers a tcgen05.ld wrote depend on
+// a point after the wait (nothing else orders the compiler's reads of the
+// load's outputs after the wait).
+__device__ __forceinline__ void tc_tie16(uint32_t (&v)[16]) {
+  asm volatile("" : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+               "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+               "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]));
+}
 
 // Completion of every tcgen05.mma issued so far by this thread arrives once on bar.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -294,11 +302,13 @@ __device__ __forceinline__ void tc_epilogue(const TcParams& p, uint32_t tmem, ui
       uint32_t v[16];
       tc_ld16(acc0 + c0, v);
       tc_wait_ld();
+      tc_tie16(v);
 #pragma unroll
       for (int i = 0; i < 16; ++i) acc[i] = __uint_as_float(v[i]);
       for (int a = 1; a < p.n_mma; ++a) {
         tc_ld16(acc0 + a * p.Npad + c0, v);
         tc_wait_ld();
+        tc_tie16(v);
 #pragma unroll
         for (int i = 0; i < 16; ++i) acc[i] += __uint_as_float(v[i]);
       }
