@@ -64,11 +64,16 @@ struct Dims {
 
 constexpr int kMaxGrid = 1024;
 
-// Relative cost of one 16-row tile of a width, for splitting the phases'
-// work between CTAs and warps: the code bytes (proportional to the width)
-// plus a fixed part for the per-group instructions that do not depend on it
-// (a flatter weight, bits + 8, measured 12 % slower on the 256-expert layer).
-__host__ __device__ constexpr int tile_weight(int bits) { return bits + 2; }
+// Relative cost of one 16-row tile of a width in each phase, for splitting
+// the phases' work between CTAs and warps: a part proportional to the width
+// (code bytes and decode) plus a fixed part (per-tile and per-group overhead).
+// On the 256-expert layer, per-CTA times put a 4-bit gate/up tile (K = 2048)
+// at ~1.7x a 2-bit one (bits + 1: 59.7 -> 57.2 us for the phase); for down
+// (K = 512) bits + 2 measured best (bits + 11, the per-CTA fit, was 12 %
+// slower: the down phase's cost follows its segments, not only its tiles).
+__host__ __device__ constexpr int tile_weight(int phase, int bits) {
+  return phase == 0 ? bits + 1 : bits + 2;
+}
 
 }  // namespace moe
 
@@ -150,12 +155,12 @@ __device__ __forceinline__ bool valid_desc(const hq_expert& e) {
 // increasing i, so the sorted order, and every sum taken over it, is
 // independent of thread timing.  Then the block list and, for each expert
 // phase, the first work item of every CTA, splitting the summed tile weights
-// evenly.  Shared memory: 3 E + 2 ints.
+// evenly.  Shared memory: 3 E + 3 ints.
 __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __restrict__ ids,
                           const Ws& w, const Dims& d, int* sm) {
-  int* s_cnt = sm;              // [E] valid pairs per expert
-  int* s_nb0 = sm + d.E;        // [E + 1] first block of each expert; [E] = blocks in all
-  int* s_sw = s_nb0 + d.E + 1;  // [E + 1] tile weight, then the block-weight prefix
+  int* s_cnt = sm;                  // [E + 1] valid pairs per expert, then phase B's weight prefix
+  int* s_nb0 = sm + d.E + 1;        // [E + 1] first block of each expert; [E] = blocks in all
+  int* s_sw = s_nb0 + d.E + 1;      // [E + 1] width, then phase A's block-weight prefix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
   for (int e = tid; e < d.E; e += nt) {
     s_cnt[e] = 0;
@@ -172,7 +177,7 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
       const hq_expert de = ex[e];
       ok = valid_desc(de);
       if (ok) {
-        s_sw[e] = tile_weight(de.bits);  // same value from every pair of e
+        s_sw[e] = de.bits;  // same value from every pair of e
       } else {
         record_error(w.status, HQ_DEV_BAD_BITS);
       }
@@ -196,23 +201,26 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
       if (e >= 0 && lane == leader) s_cnt[e] = base + __popc(mask);
       __syncwarp();
     }
-    // exclusive scans over experts: pairs, blocks, block weights
-    int run = 0, run_b = 0, run_w = 0;
+    // exclusive scans over experts: pairs, blocks, block weights of each phase
+    int run = 0, run_b = 0, run_w = 0, run_v = 0;
     for (int c = 0; c < d.E; c += 32) {
       const int e = c + lane;
       const int cnt = e < d.E ? s_cnt[e] : 0;
       const int nb = (cnt + 7) / 8;
-      const int wt = nb * (e < d.E ? s_sw[e] : 0);
-      int x = cnt, xb = nb, xw = wt;
+      const int bits = nb > 0 ? s_sw[e] : 0;
+      const int wt = nb * tile_weight(0, bits), wv = nb * tile_weight(1, bits);
+      int x = cnt, xb = nb, xw = wt, xv = wv;
 #pragma unroll
       for (int m = 1; m < 32; m <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, m);
         const int yb = __shfl_up_sync(0xffffffffu, xb, m);
         const int yw = __shfl_up_sync(0xffffffffu, xw, m);
+        const int yv = __shfl_up_sync(0xffffffffu, xv, m);
         if (lane >= m) {
           x += y;
           xb += yb;
           xw += yw;
+          xv += yv;
         }
       }
       if (e < d.E) {
@@ -220,15 +228,18 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
         w.counts[e] = cnt;
         s_nb0[e] = run_b + xb - nb;
         s_sw[e] = run_w + xw - wt;
+        s_cnt[e] = run_v + xv - wv;
       }
       run += __shfl_sync(0xffffffffu, x, 31);
       run_b += __shfl_sync(0xffffffffu, xb, 31);
       run_w += __shfl_sync(0xffffffffu, xw, 31);
+      run_v += __shfl_sync(0xffffffffu, xv, 31);
     }
     if (lane == 0) {
       w.offsets[d.E] = run;
       s_nb0[d.E] = run_b;
       s_sw[d.E] = run_w;
+      s_cnt[d.E] = run_v;
     }
   }
   __syncthreads();
@@ -239,24 +250,27 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
   }
   {
     // CTA bounds.  Work item i of a phase is tile i % TPB of block i / TPB
-    // and weighs its expert's tile weight; CTA c starts at the first item
-    // whose weight prefix reaches c / grid of the total.  Thread c finds the
-    // expert whose block-weight range [s_sw[e], s_sw[e + 1]) holds that point
-    // (s_sw[e] grid <= c tot < s_sw[e + 1] grid) by bisection.
+    // and weighs its expert's tile weight in that phase; CTA c starts at the
+    // first item whose weight prefix reaches c / grid of the total.  Thread
+    // (c, phase) finds the expert whose block-weight range [pre[e],
+    // pre[e + 1]) holds that point (pre[e] grid <= c tot < pre[e + 1] grid)
+    // by bisection.
     const int tpb[2] = {d.inter / kRows, d.hidden / kRows};
-    const long long tot = s_sw[d.E];
     const int gc = d.grid;
-    for (int c = tid; c <= gc; c += nt) {
+    for (int job = tid; job < 2 * (gc + 1); job += nt) {
+      const int ph = job / (gc + 1), c = job - ph * (gc + 1);
+      const int* pre = ph == 0 ? s_sw : s_cnt;
+      const long long tot = pre[d.E];
+      int* out = w.bounds + ph * (kMaxGrid + 1);
       if (tot == 0 || c == gc) {
-        w.bounds[c] = tot == 0 ? 0 : s_nb0[d.E] * tpb[0];
-        w.bounds[kMaxGrid + 1 + c] = tot == 0 ? 0 : s_nb0[d.E] * tpb[1];
+        out[c] = tot == 0 ? 0 : s_nb0[d.E] * tpb[ph];
         continue;
       }
       const long long pt = static_cast<long long>(c) * tot;
-      int lo = 0, hi = d.E - 1;  // largest e with s_sw[e] * gc <= pt
+      int lo = 0, hi = d.E - 1;  // largest e with pre[e] * gc <= pt
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (static_cast<long long>(s_sw[mid]) * gc <= pt) {
+        if (static_cast<long long>(pre[mid]) * gc <= pt) {
           lo = mid;
         } else {
           hi = mid - 1;
@@ -264,15 +278,12 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
       }
       const int e = lo;
       const int nb0 = s_nb0[e], nb = s_nb0[e + 1] - nb0;
-      const long long X = s_sw[e], we = (s_sw[e + 1] - X) / nb;
-#pragma unroll
-      for (int ph = 0; ph < 2; ++ph) {
-        const long long T = tpb[ph];
-        const long long local = (pt * T) / gc - T * X;
-        const long long bo = local / (T * we);
-        const long long tau = (local - bo * T * we + we - 1) / we;
-        w.bounds[ph * (kMaxGrid + 1) + c] = static_cast<int>((nb0 + bo) * T + tau);
-      }
+      const long long X = pre[e], we = (pre[e + 1] - X) / nb;
+      const long long T = tpb[ph];
+      const long long local = (pt * T) / gc - T * X;
+      const long long bo = local / (T * we);
+      const long long tau = (local - bo * T * we + we - 1) / we;
+      out[c] = static_cast<int>((nb0 + bo) * T + tau);
     }
   }
   __syncthreads();
@@ -821,7 +832,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       const int item0 = max(it, b * TPB), item1 = min(ie, (b + 1) * TPB);
       const int ni = valid ? item1 - item0 : 0;
       const hq_expert ede = valid ? ex[e] : hq_expert{};
-      const int wt = valid ? ni * G * tile_weight(ede.bits) : 0;
+      const int wt = valid ? ni * G * tile_weight(PHASE, ede.bits) : 0;
       int pc = ncol, pn = ni, pw = wt;  // inclusive prefix sums of columns, items, weights
 #pragma unroll
       for (int m = 1; m < 32; m <<= 1) {
@@ -889,7 +900,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       int k = 0;
       while (k + 1 < nseg && pm.seg[k + 1].wt0 <= target) ++k;
       const SegInfo& sg = pm.seg[k];
-      const int tw = tile_weight(sg.ed.bits);
+      const int tw = tile_weight(PHASE, sg.ed.bits);
       const int u = sg.unit0 + (target - sg.wt0 + tw - 1) / tw;
       return min(u, sg.unit0 + (sg.item1 - sg.item0) * G);
     };
@@ -966,7 +977,7 @@ static cudaError_t moe_launch_front(int hidden, const hq_expert* ex, const int32
                                     const __half* x, const int8_t* s, const moe::Ws& w,
                                     const moe::Dims& d, cudaStream_t st) {
   const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(hidden)));
-  const size_t route_smem = (3 * static_cast<size_t>(d.E) + 2) * sizeof(int);
+  const size_t route_smem = (3 * static_cast<size_t>(d.E) + 3) * sizeof(int);
 #define HQ_FRONT(LK)                                                                          \
   case (1 << LK):                                                                             \
     return launch_pdl(moe::moe_front_kernel<LK>, dim3(d.T + 1), dim3(FwhtShape<LK>::THREADS),   \
