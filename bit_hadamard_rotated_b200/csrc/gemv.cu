@@ -287,6 +287,18 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 #pragma unroll
           for (int j = 0; j < 16; ++j) neg |= (b[j] < 0 ? 1u : 0u) << (e + j);
         }
+      } else if constexpr (FS::E == 8 || FS::E == 4) {
+        // one 8- or 4-byte load (the signs are 16-byte aligned, E | 16)
+        uint32_t wv[2] = {0u, 0u};
+        if constexpr (FS::E == 8) {
+          const uint2 u = __ldg(reinterpret_cast<const uint2*>(sp));
+          wv[0] = u.x;
+          wv[1] = u.y;
+        } else {
+          wv[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
+        }
+#pragma unroll
+        for (int e = 0; e < FS::E; ++e) neg |= (wv[e >> 2] >> (8 * (e & 3) + 7) & 1u) << e;
       } else {
 #pragma unroll
         for (int e = 0; e < FS::E; ++e) neg |= (sp[e] < 0 ? 1u : 0u) << e;

@@ -167,31 +167,36 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
     s_sw[e] = 0;
   }
   __syncthreads();
-  // validity of every pair (its expert id and that expert's descriptor)
+  // validity of every pair (its expert id and that expert's descriptor):
+  // s_sw[e] = the width of a valid expert that has pairs, else 0
   for (int i = tid; i < d.P; i += nt) {
     const int e = ids[i];
-    int ok = 0;
     if (e < 0 || e >= d.E) {
       record_error(w.status, HQ_DEV_BAD_EXPERT);
+      w.pos[i] = -1;
     } else {
       const hq_expert de = ex[e];
-      ok = valid_desc(de);
-      if (ok) {
+      if (valid_desc(de)) {
         s_sw[e] = de.bits;  // same value from every pair of e
       } else {
         record_error(w.status, HQ_DEV_BAD_BITS);
+        w.pos[i] = -1;
       }
     }
-    w.pos[i] = ok ? e : -1;  // expert id of a valid pair, for the ranking pass
   }
   __syncthreads();
   if (warp == 0) {
-    // ranks in pair order, 32 pairs at a time; the next 32 ids are loaded ahead
-    int e_next = lane < d.P ? w.pos[lane] : -1;
+    // ranks in pair order, 32 pairs at a time; the ids (cached on chip since
+    // the pass above) are loaded one round ahead, validity comes from s_sw
+    auto key = [&](int i) {
+      const int e = i < d.P ? ids[i] : -1;
+      return e >= 0 && e < d.E && s_sw[e] != 0 ? e : -1;
+    };
+    int e_next = key(lane);
     for (int c = 0; c < d.P; c += 32) {
       const int i = c + lane;
       const int e = e_next;
-      e_next = i + 32 < d.P ? w.pos[i + 32] : -1;
+      e_next = key(i + 32);
       const unsigned mask = __match_any_sync(0xffffffffu, e);
       const int before = __popc(mask & ((1u << lane) - 1u));
       const int base = e >= 0 ? s_cnt[e] : 0;
@@ -287,11 +292,14 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
     }
   }
   __syncthreads();
-  // sorted positions (w.offsets is complete after the barrier)
+  // sorted positions (w.offsets is complete after the barrier); the rank and
+  // the expert's offset are loaded together
   for (int i = tid; i < d.P; i += nt) {
+    const int e = ids[i];
+    const int off = w.offsets[e >= 0 && e < d.E ? e : 0];
     const int r = w.pos[i];
     if (r <= -2) {
-      const int p = w.offsets[ids[i]] + (-2 - r);
+      const int p = off + (-2 - r);
       w.pos[i] = p;
       w.sorted[p] = i;
     }
@@ -438,22 +446,22 @@ __global__ void moe_combine_kernel(const float* __restrict__ topk_w, Ws w, Dims 
 // start at multiples of it, so with G >= 8 (G a power of two) a chunk's
 // groups lie in one aligned run of 8 and one 16-byte piece per row holds
 // their scales; with G < 8 the tile's whole [16][G] scale block is copied.
-__host__ __device__ inline int chunk_stride(int bits, int len) {
+__host__ __device__ constexpr int chunk_stride(int bits, int len) {
   const int row = len * 16 * bits;
   const int pad_w = ((bank_target_words(bits) - row / 4) % 32 + 32) % 32;
   return row + 4 * pad_w;
 }
-__host__ __device__ inline int chunk_scale_bytes(int G) {
+__host__ __device__ constexpr int chunk_scale_bytes(int G) {
   return G >= 8 ? kRows * 16 : kRows * G * 2;
 }
 constexpr int kRing = 2;               // slots per warp
 constexpr int kChunkMax = 6 * 1024;    // slot bytes when the B fragments stay in global memory
 constexpr int kSmemMax = 227 * 1024;
-__host__ __device__ inline int chunk_bytes(int bits, int G, int nmat, int len) {
+__host__ __device__ constexpr int chunk_bytes(int bits, int G, int nmat, int len) {
   return nmat * (kRows * chunk_stride(bits, len) + chunk_scale_bytes(G));
 }
 // Longest chunk (8, 4, 2 or 1 groups) that fits `cbytes`; 0 if none does.
-__host__ __device__ inline int chunk_len(int bits, int G, int nmat, int cbytes) {
+__host__ __device__ constexpr int chunk_len(int bits, int G, int nmat, int cbytes) {
   for (int len = 8; len >= 1; len >>= 1) {
     if (len <= G && chunk_bytes(bits, G, nmat, len) <= cbytes) return len;
   }
@@ -518,20 +526,23 @@ struct PhaseSmem {
   int zc_off, xs_off, ring_off, bar_off, total;
 };
 
-__host__ __device__ inline int round128(int v) { return (v + 127) & ~127; }
+__host__ __device__ constexpr int round128(int v) { return (v + 127) & ~127; }
 
-__host__ __device__ inline PhaseSmem phase_smem(int G, int nmat) {
+__host__ __device__ constexpr PhaseSmem phase_smem(int G, int nmat) {
   PhaseSmem p{};
   // the largest len-1 chunk of any width must fit a slot
   int need = 0;
-  for (int b = 2; b <= 8; b = b == 4 ? 8 : b + 1) need = max(need, chunk_bytes(b, G, nmat, 1));
+  for (int b = 2; b <= 8; b = b == 4 ? 8 : b + 1) {
+    const int c = chunk_bytes(b, G, nmat, 1);
+    need = need > c ? need : c;
+  }
   p.zc_off = 1024;
   p.xs_off = round128(p.zc_off + kMaxSeg * G * 8 * 4 + 64);
   const int xs_bytes = G * 8 * 4 * 64;
   const int ring_off = round128(p.xs_off + xs_bytes);
   const int fit = ((kSmemMax - ring_off - kWarps * kRing * 8) / (kWarps * kRing)) & ~127;
-  p.bsmem = fit >= max(need, 4096) ? 1 : 0;  // else the rings would be too shallow
-  p.cbytes = p.bsmem ? min(fit, kChunkMax) : kChunkMax;
+  p.bsmem = fit >= (need > 4096 ? need : 4096) ? 1 : 0;  // else the rings would be too shallow
+  p.cbytes = p.bsmem ? (fit < kChunkMax ? fit : kChunkMax) : kChunkMax;
   p.ring_off = p.bsmem ? ring_off : p.xs_off;
   p.bar_off = p.ring_off + kWarps * kRing * p.cbytes;
   p.total = p.bar_off + kWarps * kRing * 8;
@@ -543,7 +554,7 @@ __host__ __device__ inline PhaseSmem phase_smem(int G, int nmat) {
 // (two columns x four k-quads) read 8 different bank groups.
 __device__ __forceinline__ int bswz(int col, int q) { return ((col & 1) << 1) | (q >> 1); }
 
-// One warp's copy ring: kRing slots of ps.cbytes, one mbarrier each (32
+// One warp's copy ring: kRing slots of the plan's cbytes, one mbarrier each (32
 // arrivals: every lane's cp.async group), counters over the whole kernel.
 struct RingState {
   uint8_t* ring;
@@ -592,22 +603,26 @@ __device__ __forceinline__ void seg_store(const Ws& w, const Dims& d, const SegI
 // whole is stored here; a tile it covers in part (only at its range ends u0,
 // u1) is kept in `part` (0: the tile holding u0, 1: the last) for the
 // pass's reduction.
-template <int PHASE, bool BSMEM, int BITS>
+template <int PHASE, int LOGK, int BITS>
 __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, int ub, const Ws& w,
-                                            const Dims& d, const PhaseSmem& ps, RingState& rs,
+                                            const Dims& d, RingState& rs,
                                             const float* zc, const uint4* xs, int cols,
                                             const uint16_t* bsrc, int u0, float4 (&part)[2][2],
                                             int (&ptile)[2], int lane) {
   constexpr int NMAT = PHASE == 0 ? 2 : 1;
   constexpr int GB = 16 * BITS;  // code bytes of one row in one group
   const int g = lane >> 2, t = lane & 3;
-  const int K = PHASE == 0 ? d.hidden : d.inter;
-  const int G = K / kGroup;
-  const int lgG = __ffs(G) - 1;
-  const int len_max = chunk_len(BITS, G, NMAT, ps.cbytes);
-  const int stride = chunk_stride(BITS, len_max);
-  const int row_bytes = K * BITS / 8;
-  const int sbytes = chunk_scale_bytes(G);
+  // the chunk and slot layout is fixed by K (this phase's input width)
+  constexpr int K = 1 << LOGK;
+  constexpr int G = K / kGroup;
+  constexpr int lgG = LOGK - 7;
+  constexpr PhaseSmem PS = phase_smem(G, NMAT);
+  constexpr bool BSMEM = PS.bsmem != 0;
+  constexpr int len_max = chunk_len(BITS, G, NMAT, PS.cbytes);
+  static_assert(len_max > 0, "a one-group chunk fits a slot");
+  constexpr int stride = chunk_stride(BITS, len_max);
+  constexpr int row_bytes = K * BITS / 8;
+  constexpr int sbytes = chunk_scale_bytes(G);
   const uint8_t* qbase[NMAT];
   const uint16_t* sbase[NMAT];
   if (PHASE == 0) {
@@ -636,7 +651,7 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
     int j, g0, len;
     chunk_of(pu, j, g0, len);
     const int m0 = (sg.tile0 + j) * kRows;
-    uint8_t* base = rs.ring + slot * ps.cbytes;
+    uint8_t* base = rs.ring + slot * PS.cbytes;
     int pr = prf, r0 = r0f, c0 = c0f, dr = drf, dc = dcf;
     if (len != len_max) {  // a shorter chunk (tile or range end)
       pr = len * BITS;
@@ -711,7 +726,7 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
       return;
     }
     __syncwarp();
-    const uint8_t* base = rs.ring + slot * ps.cbytes;
+    const uint8_t* base = rs.ring + slot * PS.cbytes;
     const __half* scb = reinterpret_cast<const __half*>(base + NMAT * kRows * stride);
     for (int jj = 0; jj < len; ++jj) {
       const int gi = g0 + jj;
@@ -786,15 +801,16 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
 // summed in warp order through shared memory after one barrier.  Without
 // BSMEM (K too large for the fragments beside the rings) lanes read their B
 // blocks from global memory, one group ahead.
-template <int PHASE, bool BSMEM>
+template <int PHASE, int LOGK>
 __global__ void __launch_bounds__(kWarps * 32, 1)
-    moe_phase_kernel(const hq_expert* __restrict__ ex, Ws w, Dims d, PhaseSmem ps) {
+    moe_phase_kernel(const hq_expert* __restrict__ ex, Ws w, Dims d) {
   constexpr int NMAT = PHASE == 0 ? 2 : 1;
+  constexpr int G = (1 << LOGK) / kGroup;  // K = hidden (phase A) or inter (phase B)
+  constexpr PhaseSmem ps = phase_smem(G, NMAT);
+  constexpr bool BSMEM = ps.bsmem != 0;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int K = PHASE == 0 ? d.hidden : d.inter;
   const int M = PHASE == 0 ? d.inter : d.hidden;
-  const int G = K / kGroup;
   const int TPB = M / kRows;  // tiles per block
   PassMeta& pm = *reinterpret_cast<PassMeta*>(smem);
   float* zc = reinterpret_cast<float*>(smem + ps.zc_off);  // [kMaxSeg][G][8], then a zero B block
@@ -913,10 +929,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       const int sa = max(u0, sg.unit0), sb = min(u1, sg.unit0 + (sg.item1 - sg.item0) * G);
       if (sa >= sb) continue;
       switch (sg.ed.bits) {
-        case 2: phase_piece<PHASE, BSMEM, 2>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
-        case 3: phase_piece<PHASE, BSMEM, 3>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
-        case 4: phase_piece<PHASE, BSMEM, 4>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
-        default: phase_piece<PHASE, BSMEM, 8>(sg, k, sa, sb, w, d, ps, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        case 2: phase_piece<PHASE, LOGK, 2>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        case 3: phase_piece<PHASE, LOGK, 3>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        case 4: phase_piece<PHASE, LOGK, 4>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        default: phase_piece<PHASE, LOGK, 8>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
       }
     }
     // ---- tiles split between warps: each warp leaves its partial sums in
@@ -1010,18 +1026,23 @@ template <int PHASE>
 static cudaError_t moe_launch_phase(const hq_expert* ex, const moe::Ws& w, const moe::Dims& d,
                                     cudaStream_t st) {
   constexpr int nmat = PHASE == 0 ? 2 : 1;
-  const int G = (PHASE == 0 ? d.hidden : d.inter) / kGroup;
-  const moe::PhaseSmem ps = moe::phase_smem(G, nmat);
+  const int K = PHASE == 0 ? d.hidden : d.inter;
+  const moe::PhaseSmem ps = moe::phase_smem(K / kGroup, nmat);
   for (int b : {2, 3, 4, 8}) {
-    if (moe::chunk_len(b, G, nmat, ps.cbytes) == 0) return cudaErrorInvalidConfiguration;
+    if (moe::chunk_len(b, K / kGroup, nmat, ps.cbytes) == 0) return cudaErrorInvalidConfiguration;
   }
   if (ps.total > moe::kSmemMax) return cudaErrorInvalidConfiguration;
   const dim3 grid(d.grid), block(moe::kWarps * 32);  // one CTA per SM; the routing CTA split
                                                      // the work for exactly d.grid CTAs
-  return ps.bsmem ? launch_pdl(moe::moe_phase_kernel<PHASE, true>, grid, block, ps.total, st, true,
-                               ex, w, d, ps)
-                  : launch_pdl(moe::moe_phase_kernel<PHASE, false>, grid, block, ps.total, st, true,
-                               ex, w, d, ps);
+#define HQ_PHASE(LK) \
+  case (1 << LK): \
+    return launch_pdl(moe::moe_phase_kernel<PHASE, LK>, grid, block, ps.total, st, true, ex, w, d);
+  switch (K) {
+    HQ_PHASE(7) HQ_PHASE(8) HQ_PHASE(9) HQ_PHASE(10) HQ_PHASE(11) HQ_PHASE(12) HQ_PHASE(13)
+    HQ_PHASE(14)
+    default: return cudaErrorInvalidValue;
+  }
+#undef HQ_PHASE
 }
 
 }  // namespace hq
