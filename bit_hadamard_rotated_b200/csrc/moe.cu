@@ -64,7 +64,7 @@ struct Dims {
 
 constexpr int kMaxGrid = 1024;
 
-// Relative cost of one 16-row tile of a width in each phase, for splitting
+// Relative cost of one work item of a width in each phase, for splitting
 // the phases' work between CTAs and warps: a part proportional to the width
 // (code bytes and decode) plus a fixed part (per-tile and per-group overhead).
 // On the 256-expert layer, per-CTA times put a 4-bit gate/up tile (K = 2048)
@@ -74,6 +74,12 @@ constexpr int kMaxGrid = 1024;
 __host__ __device__ constexpr int tile_weight(int phase, int bits) {
   return phase == 0 ? bits + 1 : bits + 2;
 }
+
+// Rows of one work item: a phase-A item is a 16-row tile of gate and of up;
+// a phase-B item is a 32-row tile of down, taken as two 16-row halves.  Either
+// way a group's activation fragments and zero-point terms are loaded once
+// for two 16-row code tiles.
+__host__ __device__ constexpr int item_rows(int phase) { return phase == 0 ? 16 : 32; }
 
 }  // namespace moe
 
@@ -260,7 +266,7 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
     // (c, phase) finds the expert whose block-weight range [pre[e],
     // pre[e + 1]) holds that point (pre[e] grid <= c tot < pre[e + 1] grid)
     // by bisection.
-    const int tpb[2] = {d.inter / kRows, d.hidden / kRows};
+    const int tpb[2] = {d.inter / item_rows(0), d.hidden / item_rows(1)};
     const int gc = d.grid;
     for (int job = tid; job < 2 * (gc + 1); job += nt) {
       const int ph = job / (gc + 1), c = job - ph * (gc + 1);
@@ -441,11 +447,12 @@ __global__ void moe_combine_kernel(const float* __restrict__ topk_w, Ws w, Dims 
 
 // ---------------------------------------------------------------- expert phases
 // Chunk geometry, shared by producer and consumer: a chunk is `len` groups of
-// one item's 16 rows in each of its NMAT matrices, rows at a bank-conflict-
-// free stride, then each matrix's scales.  len is a power of two and chunks
-// start at multiples of it, so with G >= 8 (G a power of two) a chunk's
-// groups lie in one aligned run of 8 and one 16-byte piece per row holds
-// their scales; with G < 8 the tile's whole [16][G] scale block is copied.
+// one item's two 16-row code tiles (gate and up, or the halves of a 32-row
+// down tile), rows at a bank-conflict-free stride, then each tile's scales.
+// len is a power of two and chunks start at multiples of it, so with G >= 8
+// (G a power of two) a chunk's groups lie in one aligned run of 8 and one
+// 16-byte piece per row holds their scales; with G < 8 each tile's whole
+// [16][G] scale block is copied.
 __host__ __device__ constexpr int chunk_stride(int bits, int len) {
   const int row = len * 16 * bits;
   const int pad_w = ((bank_target_words(bits) - row / 4) % 32 + 32) % 32;
@@ -571,14 +578,15 @@ __device__ __forceinline__ size_t seg_brow(const Ws& w, const Dims& d, const Seg
   return PHASE == 0 ? static_cast<size_t>(sg.L) * d.T + w.sorted[p] / d.k : static_cast<size_t>(p);
 }
 
-// Epilogue of one tile: rows g, g+8 of the lane's fragment, columns 2t, 2t+1.
+// Epilogue of one item: rows g, g+8 of the lane's fragments, columns 2t,
+// 2t+1; o[0] and o[1] are gate and up (A) or the item's two 16-row halves (B).
 template <int PHASE>
 __device__ __forceinline__ void seg_store(const Ws& w, const Dims& d, const SegInfo& sg, int m0,
                                           const float4 (&o)[2], int lane) {
   const int g = lane >> 2, t = lane & 3;
   const int M = PHASE == 0 ? d.inter : d.hidden;
   const float* og = reinterpret_cast<const float*>(&o[0]);
-  const float* ou = reinterpret_cast<const float*>(&o[PHASE == 0 ? 1 : 0]);
+  const float* ou = reinterpret_cast<const float*>(&o[1]);
 #pragma unroll
   for (int q4 = 0; q4 < 4; ++q4) {
     const int col = 2 * t + (q4 & 1);
@@ -590,6 +598,7 @@ __device__ __forceinline__ void seg_store(const Ws& w, const Dims& d, const SegI
         w.h[prow * d.inter + m] = gv / (1.f + expf(-gv)) * uv;
       } else {
         w.d[prow * d.hidden + m] = og[q4] * kUnit;
+        w.d[prow * d.hidden + m + kRows] = ou[q4] * kUnit;  // M is a multiple of 32
       }
     }
   }
@@ -609,7 +618,7 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
                                             const float* zc, const uint4* xs, int cols,
                                             const uint16_t* bsrc, int u0, float4 (&part)[2][2],
                                             int (&ptile)[2], int lane) {
-  constexpr int NMAT = PHASE == 0 ? 2 : 1;
+  constexpr int NMAT = 2;  // gate and up, or the two halves of a down tile
   constexpr int GB = 16 * BITS;  // code bytes of one row in one group
   const int g = lane >> 2, t = lane & 3;
   // the chunk and slot layout is fixed by K (this phase's input width)
@@ -632,7 +641,9 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
     sbase[NMAT - 1] = sg.ed.s_up;
   } else {
     qbase[0] = reinterpret_cast<const uint8_t*>(sg.ed.q_down);
+    qbase[1] = qbase[0] + static_cast<size_t>(kRows) * row_bytes;
     sbase[0] = sg.ed.s_down;
+    sbase[1] = sbase[0] + kRows * G;
   }
   auto chunk_of = [&](int u, int& j, int& g0, int& len) {
     const int r = u - sg.unit0;
@@ -650,7 +661,7 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
   auto issue = [&](int slot) {
     int j, g0, len;
     chunk_of(pu, j, g0, len);
-    const int m0 = (sg.tile0 + j) * kRows;
+    const int m0 = (sg.tile0 + j) * item_rows(PHASE);
     uint8_t* base = rs.ring + slot * PS.cbytes;
     int pr = prf, r0 = r0f, c0 = c0f, dr = drf, dc = dcf;
     if (len != len_max) {  // a shorter chunk (tile or range end)
@@ -768,7 +779,7 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
         o[mi] = make_float4(acc[mm][0], acc[mm][1], acc[mm][2], acc[mm][3]);
       }
       if (tile_g0 == 0 && g0 + len == G) {
-        seg_store<PHASE>(w, d, sg, (sg.tile0 + j) * kRows, o, lane);
+        seg_store<PHASE>(w, d, sg, (sg.tile0 + j) * item_rows(PHASE), o, lane);
       } else {
         const int tf = sg.unit0 + (j << lgG);  // the tile's first unit
         if (tf <= u0 && u0 < tf + G) {  // the tile holding u0 (constant indices: registers)
@@ -790,7 +801,7 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
 
 // Phase A (PHASE 0): gate and up, SwiGLU -> h.  Phase B (PHASE 1): down -> d.
 //
-// Work item i is 16-row tile i % TPB of block i / TPB, a block being one
+// Work item i is row tile i % TPB (item_rows) of block i / TPB, a block being one
 // expert's <= 8-token column block (w.blk); CTA c owns items [bounds[c],
 // bounds[c + 1]) (split by tile weight) and walks them in passes.  A pass
 // takes up to kMaxSeg consecutive blocks' parts (segments) with at most 8
@@ -804,14 +815,14 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
 template <int PHASE, int LOGK>
 __global__ void __launch_bounds__(kWarps * 32, 1)
     moe_phase_kernel(const hq_expert* __restrict__ ex, Ws w, Dims d) {
-  constexpr int NMAT = PHASE == 0 ? 2 : 1;
+  constexpr int NMAT = 2;
   constexpr int G = (1 << LOGK) / kGroup;  // K = hidden (phase A) or inter (phase B)
   constexpr PhaseSmem ps = phase_smem(G, NMAT);
   constexpr bool BSMEM = ps.bsmem != 0;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int M = PHASE == 0 ? d.inter : d.hidden;
-  const int TPB = M / kRows;  // tiles per block
+  const int TPB = M / item_rows(PHASE);  // items per block
   PassMeta& pm = *reinterpret_cast<PassMeta*>(smem);
   float* zc = reinterpret_cast<float*>(smem + ps.zc_off);  // [kMaxSeg][G][8], then a zero B block
   uint4* xs = reinterpret_cast<uint4*>(smem + ps.xs_off);  // [G][cols][4][4 pieces], swizzled
@@ -972,7 +983,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
             o[mi].w += q4.w;
           }
         }
-        seg_store<PHASE>(w, d, sg, (sg.tile0 + item - sg.item0) * kRows, o, lane);
+        seg_store<PHASE>(w, d, sg, (sg.tile0 + item - sg.item0) * item_rows(PHASE), o, lane);
       }
     }
     it += U / G;
@@ -1025,7 +1036,7 @@ static cudaError_t moe_launch_rot_h(int inter, const hq_expert* ex, const int32_
 template <int PHASE>
 static cudaError_t moe_launch_phase(const hq_expert* ex, const moe::Ws& w, const moe::Dims& d,
                                     cudaStream_t st) {
-  constexpr int nmat = PHASE == 0 ? 2 : 1;
+  constexpr int nmat = 2;
   const int K = PHASE == 0 ? d.hidden : d.inter;
   const moe::PhaseSmem ps = moe::phase_smem(K / kGroup, nmat);
   for (int b : {2, 3, 4, 8}) {
