@@ -209,13 +209,14 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   const int rows = min(nb, N - b * nb);
   const int npad = (rows + 31) & ~31;
   if (j >= npad) return;  // whole CTA: no barrier is reached
+  const auto neg = sign_bits<S::E>(signs ? signs + tid * S::E : nullptr);
   pdl_wait();
   uint8_t* img = xp + static_cast<size_t>(b) * S::K * 2 * nb;
   const int n = b * nb + j;
   if (j < rows) {
     float v[S::E];
     load_chunk<__half, S::E>(x + static_cast<size_t>(n) * S::K + tid * S::E, v);
-    apply_signs<S::E>(signs ? signs + tid * S::E : nullptr, v);
+    flip_signs<S::E>(neg, v);
     fwht_block<LOGK, 5>(v, buf);
   }
   for (int seg = tid; seg < S::K / 8; seg += S::THREADS) {

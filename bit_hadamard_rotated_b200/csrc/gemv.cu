@@ -148,6 +148,8 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
   uint16_t* xs = reinterpret_cast<uint16_t*>(xg);
   float* zc = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
   const FragLane<BITS> fl(lane);
+  const SignMask<FS::E> neg =
+      tid < FS::THREADS ? sign_bits<FS::E>(signs ? signs + tid * FS::E : nullptr) : 0u;
   pdl_wait();  // x is the previous kernel's output; xg may still be read by it
   if (n == 0) {
     for (int i = tid; i < G * (8 - N); i += kPrepWarps * 32) zc[(i / (8 - N)) * 8 + N + i % (8 - N)] = 0.f;
@@ -155,7 +157,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
   float v[FS::E];
   if (tid < FS::THREADS) {
     load_chunk<__half, FS::E>(x + static_cast<size_t>(n) * K + tid * FS::E, v);
-    apply_signs<FS::E>(signs ? signs + tid * FS::E : nullptr, v);
+    flip_signs<FS::E>(neg, v);
   }
   fwht_block<LOGK, 3>(v, buf);
   for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, inv_sqrt_k, zero, xs, zc, lane);
@@ -276,34 +278,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     // for K >= 512); the signs are weights, read before the wait
     using FS = FusedFwht<LOGK>;
     static_assert(FS::E <= 32, "one sign bit per register");
-    uint32_t neg = 0;  // bit e: value e of this thread's chunk flips sign
-    if (tid < FS::THREADS && p.signs != nullptr) {
-      const int8_t* sp = p.signs + tid * FS::E;
-      if constexpr (FS::E % 16 == 0) {
-#pragma unroll
-        for (int e = 0; e < FS::E; e += 16) {
-          const uint4 u = __ldg(reinterpret_cast<const uint4*>(sp + e));
-          const int8_t* b = reinterpret_cast<const int8_t*>(&u);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) neg |= (b[j] < 0 ? 1u : 0u) << (e + j);
-        }
-      } else if constexpr (FS::E == 8 || FS::E == 4) {
-        // one 8- or 4-byte load (the signs are 16-byte aligned, E | 16)
-        uint32_t wv[2] = {0u, 0u};
-        if constexpr (FS::E == 8) {
-          const uint2 u = __ldg(reinterpret_cast<const uint2*>(sp));
-          wv[0] = u.x;
-          wv[1] = u.y;
-        } else {
-          wv[0] = __ldg(reinterpret_cast<const uint32_t*>(sp));
-        }
-#pragma unroll
-        for (int e = 0; e < FS::E; ++e) neg |= (wv[e >> 2] >> (8 * (e & 3) + 7) & 1u) << e;
-      } else {
-#pragma unroll
-        for (int e = 0; e < FS::E; ++e) neg |= (sp[e] < 0 ? 1u : 0u) << e;
-      }
-    }
+    // bit e: value e of this thread's chunk flips sign
+    const SignMask<FS::E> neg =
+        tid < FS::THREADS ? sign_bits<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr) : 0u;
     float* buf = reinterpret_cast<float*>(smem + p.buf_off);
     const FragLane<BITS> fl(lane);
     for (int i = tid; i < G * 8; i += kWarps * 32) {
@@ -314,8 +291,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       float v[FS::E];
       if (tid < FS::THREADS) {
         load_chunk<__half, FS::E>(p.x + static_cast<size_t>(n) * K + tid * FS::E, v);
-#pragma unroll
-        for (int e = 0; e < FS::E; ++e) v[e] = (neg >> e & 1u) ? -v[e] : v[e];
+        flip_signs<FS::E>(neg, v);
       }
       FS::run(v, buf);
       for (int gg = warp; gg < G; gg += kWarps) {

@@ -2,6 +2,8 @@
 // fp32 registers, 16-byte vectors where the chunk allows, and sign flips.
 #pragma once
 
+#include <type_traits>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <stdint.h>
@@ -58,21 +60,46 @@ __device__ __forceinline__ void load_chunk(const T* p, float (&v)[E]) {
   }
 }
 
+// The signs of a thread's chunk of E consecutive values as a bit mask (bit
+// e set: value e flips), read with the widest aligned loads (the sign vector
+// is 16-byte aligned and the chunk starts at a multiple of E).  The signs are
+// weights, so kernels read them before griddepcontrol.wait.
 template <int E>
-__device__ __forceinline__ void apply_signs(const int8_t* s, float (&v)[E]) {
-  if (s == nullptr) return;
+using SignMask = typename std::conditional<(E <= 32), uint32_t, unsigned long long>::type;
+
+template <int E>
+__device__ __forceinline__ SignMask<E> sign_bits(const int8_t* s) {
+  static_assert(E <= 64, "one bit per value");
+  using Mk = SignMask<E>;
+  if (s == nullptr) return Mk(0);
+  Mk m = 0;
   if constexpr (E % 16 == 0) {
 #pragma unroll
     for (int i = 0; i < E / 16; ++i) {
       const uint4 u = __ldg(reinterpret_cast<const uint4*>(s) + i);
-      const int8_t* b = reinterpret_cast<const int8_t*>(&u);
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int j = 0; j < 16; ++j) v[16 * i + j] = b[j] < 0 ? -v[16 * i + j] : v[16 * i + j];
+      for (int j = 0; j < 16; ++j) m |= static_cast<Mk>(w[j >> 2] >> (8 * (j & 3) + 7) & 1u) << (16 * i + j);
     }
+  } else if constexpr (E == 8) {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(s));
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m |= (((j < 4) ? u.x : u.y) >> (8 * (j & 3) + 7) & 1u) << j;
+  } else if constexpr (E == 4) {
+    const uint32_t u = __ldg(reinterpret_cast<const uint32_t*>(s));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m |= (u >> (8 * j + 7) & 1u) << j;
   } else {
 #pragma unroll
-    for (int e = 0; e < E; ++e) v[e] = s[e] < 0 ? -v[e] : v[e];
+    for (int e = 0; e < E; ++e) m |= (s[e] < 0 ? 1u : 0u) << e;
   }
+  return m;
+}
+
+template <int E>
+__device__ __forceinline__ void flip_signs(SignMask<E> m, float (&v)[E]) {
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = (m >> e & 1u) ? -v[e] : v[e];
 }
 
 }  // namespace hq

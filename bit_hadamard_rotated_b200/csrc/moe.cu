@@ -168,26 +168,24 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
   int* s_nb0 = sm + d.E + 1;        // [E + 1] first block of each expert; [E] = blocks in all
   int* s_sw = s_nb0 + d.E + 1;      // [E + 1] width, then phase A's block-weight prefix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
+  // every expert's width, or -1 for a bad descriptor; the expert table is a
+  // weight (no earlier kernel of the library writes it), read before the wait
   for (int e = tid; e < d.E; e += nt) {
     s_cnt[e] = 0;
-    s_sw[e] = 0;
+    const hq_expert de = ex[e];
+    s_sw[e] = valid_desc(de) ? de.bits : -1;
   }
   __syncthreads();
-  // validity of every pair (its expert id and that expert's descriptor):
-  // s_sw[e] = the width of a valid expert that has pairs, else 0
+  pdl_wait();  // ids may be the previous kernel's output; the workspace is free once it is done
+  // validity of every pair (its expert id and that expert's descriptor)
   for (int i = tid; i < d.P; i += nt) {
     const int e = ids[i];
     if (e < 0 || e >= d.E) {
       record_error(w.status, HQ_DEV_BAD_EXPERT);
       w.pos[i] = -1;
-    } else {
-      const hq_expert de = ex[e];
-      if (valid_desc(de)) {
-        s_sw[e] = de.bits;  // same value from every pair of e
-      } else {
-        record_error(w.status, HQ_DEV_BAD_BITS);
-        w.pos[i] = -1;
-      }
+    } else if (s_sw[e] < 0) {
+      record_error(w.status, HQ_DEV_BAD_BITS);
+      w.pos[i] = -1;
     }
   }
   __syncthreads();
@@ -196,7 +194,7 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
     // the pass above) are loaded one round ahead, validity comes from s_sw
     auto key = [&](int i) {
       const int e = i < d.P ? ids[i] : -1;
-      return e >= 0 && e < d.E && s_sw[e] != 0 ? e : -1;
+      return e >= 0 && e < d.E && s_sw[e] > 0 ? e : -1;
     };
     int e_next = key(lane);
     for (int c = 0; c < d.P; c += 32) {
@@ -371,15 +369,16 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   using S = FwhtShape<LOGK>;
   extern __shared__ float buf[];
   pdl_launch_dependents();
-  pdl_wait();  // the workspace is free once the previous call's kernels are done
   if (blockIdx.x == 0) {
-    route_cta(ex, ids, w, d, reinterpret_cast<int*>(buf));
+    route_cta(ex, ids, w, d, reinterpret_cast<int*>(buf));  // waits inside
     return;
   }
   const int tid = threadIdx.x, t = blockIdx.x - 1;
+  const auto neg = sign_bits<S::E>(signs ? signs + tid * S::E : nullptr);
+  pdl_wait();  // x may be the previous kernel's output
   float v[S::E];
   load_chunk<__half, S::E>(x + static_cast<size_t>(t) * S::K + tid * S::E, v);
-  apply_signs<S::E>(signs ? signs + tid * S::E : nullptr, v);
+  flip_signs<S::E>(neg, v);
   fwht_block<LOGK, 5>(v, buf);
   const int G = S::K / kGroup;
   const int bits_of[4] = {2, 3, 4, 8};
@@ -399,14 +398,15 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   using S = FwhtShape<LOGK>;
   extern __shared__ float buf[];
   pdl_launch_dependents();
-  pdl_wait();
   const int tid = threadIdx.x, p = blockIdx.x;
+  const auto neg = sign_bits<S::E>(signs ? signs + tid * S::E : nullptr);
+  pdl_wait();
   if (p >= w.offsets[d.E]) return;  // block-uniform: no barrier is skipped by part of it
   const int e = ids[w.sorted[p]];
   const int bits = ex[e].bits;
   float v[S::E];
   load_chunk<float, S::E>(w.h + static_cast<size_t>(p) * S::K + tid * S::E, v);
-  apply_signs<S::E>(signs ? signs + tid * S::E : nullptr, v);
+  flip_signs<S::E>(neg, v);
   fwht_block<LOGK, 5>(v, buf);
   const int G = S::K / kGroup;
   write_layout_bits(bits, buf, inv, G, w.hl + static_cast<size_t>(p) * G * 4 * kXq,

@@ -22,12 +22,13 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   using S = FwhtShape<LOGK>;
   extern __shared__ float buf[];
   pdl_launch_dependents();
-  pdl_wait();
   const int tid = threadIdx.x;
   const size_t row = blockIdx.x;
+  const auto neg = sign_bits<S::E>(signs ? signs + tid * S::E : nullptr);
+  pdl_wait();
   float v[S::E];
   load_chunk<InT, S::E>(x + row * S::K + tid * S::E, v);
-  apply_signs<S::E>(signs ? signs + tid * S::E : nullptr, v);
+  flip_signs<S::E>(neg, v);
   fwht_block<LOGK, 5>(v, buf);
   OutT* o = out + row * S::K + tid * S::E;
 #pragma unroll

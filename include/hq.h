@@ -44,6 +44,14 @@
  *     time: calls that overlap on the GPU must not share it.
  *   - Outputs are overwritten, never accumulated into.  Inputs and outputs
  *     must not alias.
+ *   - Kernels are launched with programmatic dependent launch: a call's
+ *     kernels may start while the library kernel before them on the stream is
+ *     finishing, and read the weights (packed codes, scales, signs, the
+ *     expert table) before waiting for it; activations, routing inputs and
+ *     the workspace are read only after it has finished.  Weights must
+ *     therefore not be rewritten by the library call just before on the same
+ *     stream (no library call writes them), and any other kernel or copy that
+ *     writes them must complete, in stream order, before the call.
  *   - Alignment: packed weights, scales, activations and outputs must be
  *     16-byte aligned; the library checks this and returns
  *     HQ_ERR_INVALID_ARG otherwise.
