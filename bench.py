@@ -438,49 +438,140 @@ def measure_configs(device, stream, pk, l2):
     return res
 
 
+class _Rt:
+    """Async copies and event waits on raw stream handles through the CUDA
+    runtime that PyTorch loaded (a few hundred ns of host time each, against
+    several us for the tensor-level calls), or the tensor-level calls when that
+    library cannot be found."""
+
+    def __init__(self):
+        import ctypes
+        import glob
+        self.rt = None
+        here = os.path.dirname(torch.__file__)
+        for c in glob.glob(os.path.join(here, "..", "nvidia", "cuda_runtime", "lib", "libcudart.so*")) + \
+                ["libcudart.so.12", "libcudart.so"]:
+            try:
+                self.rt = ctypes.CDLL(c)
+                break
+            except OSError:
+                continue
+        if self.rt is not None:
+            vp, sz = ctypes.c_void_p, ctypes.c_size_t
+            self.rt.cudaMemcpyAsync.argtypes = [vp, vp, sz, ctypes.c_int, vp]
+            self.rt.cudaEventRecord.argtypes = [vp, vp]
+            self.rt.cudaStreamWaitEvent.argtypes = [vp, vp, ctypes.c_uint]
+        self.ctypes = ctypes
+
+    def event(self):
+        ev = torch.cuda.Event()
+        if self.rt is not None:
+            ev.record()  # creates the event; its handle is then fixed
+            torch.cuda.synchronize()
+        return ev
+
+    def copy(self, dst, src, stream, kind):
+        if self.rt is None:
+            with torch.cuda.stream(stream):
+                dst.copy_(src, non_blocking=True)
+            return
+        n = src.numel() * src.element_size()
+        if self.rt.cudaMemcpyAsync(dst.data_ptr(), src.data_ptr(), n, kind, stream.cuda_stream):
+            raise RuntimeError("cudaMemcpyAsync failed")
+
+    def record(self, ev, stream):
+        if self.rt is None:
+            ev.record(stream)
+        elif self.rt.cudaEventRecord(ev.cuda_event, stream.cuda_stream):
+            raise RuntimeError("cudaEventRecord failed")
+
+    def wait(self, stream, ev):
+        if self.rt is None:
+            stream.wait_event(ev)
+        elif self.rt.cudaStreamWaitEvent(stream.cuda_stream, ev.cuda_event, 0):
+            raise RuntimeError("cudaStreamWaitEvent failed")
+
+
 def measure_e2e(device, layers, xs, a):
     """Same metric through the public Python API with host buffers: every step
     copies the step's activations (the three layers' inputs, one pinned host
-    buffer) to the device in one copy, runs the layers, and reads their outputs
-    back to one pinned host buffer in one copy, inside the timed region."""
+    buffer) to the device in one copy, runs the layers (RotatedLinear launchers
+    prepared once on their buffers, each call one hq_linear call), and reads
+    their outputs back to a pinned host buffer in one copy, all inside the timed
+    region.  The copies run on two copy streams, double-buffered, so step
+    i + 1's upload and step i's download overlap the layers of the neighbouring
+    steps (a serving loop's pipelining); every step moves its own bytes both
+    ways."""
     copies = len(layers)
     xsz = [x.numel() for x in xs]
     ysz = [M for (M, K, b) in LAYERS]
     xh = torch.cat([x.reshape(-1).cpu() for x in xs]).pin_memory()
-    xd = torch.empty_like(xh, device=device)
-    yh = torch.empty(sum(ysz), dtype=torch.float32).pin_memory()
-    yd = torch.empty(sum(ysz), dtype=torch.float32, device=device)
-    xv, yv, o = [], [], 0
-    for li, n in enumerate(xsz):
-        xv.append(xd[o:o + n].view(1, -1))
-        o += n
-    o = 0
-    for n in ysz:
-        yv.append(yd[o:o + n].view(1, -1))
-        o += n
+    NB = 2  # buffer sets in flight
+    xd = [torch.empty_like(xh, device=device) for _ in range(NB)]
+    yd = [torch.empty(sum(ysz), dtype=torch.float32, device=device) for _ in range(NB)]
+    yh = [torch.empty(sum(ysz), dtype=torch.float32).pin_memory() for _ in range(NB)]
+    comp = torch.cuda.current_stream(device)
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    launch = []  # [copy][buffer set] -> the three layers' launchers
+    for c in range(copies):
+        per_b = []
+        for b in range(NB):
+            fns, ox, oy = [], 0, 0
+            for li, (M, K, bits) in enumerate(LAYERS):
+                fns.append(layers[c][li].prepare(xd[b][ox:ox + xsz[li]].view(1, -1),
+                                                 yd[b][oy:oy + M].view(1, -1), stream=comp))
+                ox += xsz[li]
+                oy += M
+            per_b.append(fns)
+        launch.append(per_b)
     steps = min(a.steps, 2000)
-    stream = torch.cuda.current_stream(device)
+    rt = _Rt()
+    x_in, y_out, y_read = ([rt.event() for _ in range(NB)] for _ in range(3))
+    H2D, D2H = 1, 2  # cudaMemcpyKind
 
-    def one(c):
-        xd.copy_(xh, non_blocking=True)
-        for li in range(len(LAYERS)):
-            layers[c][li](xv[li], out=yv[li])
-        yh.copy_(yd, non_blocking=True)
+    def upload(i):
+        b = i % NB
+        if i >= NB:
+            rt.wait(up, y_out[b])  # the layers of step i - NB have read xd[b]
+        rt.copy(xd[b], xh, up, H2D)
+        rt.record(x_in[b], up)
 
-    for i in range(3):
-        one(i % copies)
+    def step(i):
+        b = i % NB
+        rt.wait(comp, x_in[b])
+        if i >= NB:
+            rt.wait(comp, y_read[b])  # step i - NB's download has read yd[b]
+        for fn in launch[i % copies][b]:
+            fn()
+        rt.record(y_out[b], comp)
+        rt.wait(down, y_out[b])
+        rt.copy(yh[b], yd[b], down, D2H)
+        rt.record(y_read[b], down)
+
+    def run(n, start=None):
+        if start is not None:
+            rt.wait(up, start)
+        upload(0)
+        for i in range(n):
+            if i + 1 < n:
+                upload(i + 1)
+            step(i)
+        rt.wait(comp, y_read[(n - 1) % NB])  # the last download is inside the region
+
+    run(3)
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for i in range(steps):
-        one(i % copies)
-    e1.record(stream)
+    e0.record(comp)
+    run(steps, start=e0)
+    e1.record(comp)
     torch.cuda.synchronize(device)
     ms = e0.elapsed_time(e1)
     return {"ms": ms, "value": None, "unit": "GB/s", "steps": steps,
-            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh.numel() * 4),
-            "api": "RotatedLinear.__call__ -> hq_linear (C ABI), eager launches; one H2D and "
-                   "one D2H copy per step"}
+            "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh[0].numel() * 4),
+            "api": "RotatedLinear.prepare launchers -> hq_linear (C ABI), eager, one call per "
+                   "layer per step; one H2D and one D2H copy per step on two copy streams, "
+                   "double-buffered against the layers" +
+                   ("" if rt.rt is not None else " (tensor-level copies)")}
 
 
 # ---------------------------------------------------------------- CPU oracle baseline

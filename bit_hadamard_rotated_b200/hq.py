@@ -141,6 +141,32 @@ class RotatedLinear:
             check(st, "hq_linear")
         return out
 
+    def prepare(self, x, out, stream=None):
+        """A zero-argument launcher of this layer on fixed buffers and a fixed
+        stream (the current one if None), for loops that reuse them, such as a
+        decode step: the buffers are checked once here, and each call is one
+        hq_linear call with its arguments already marshalled."""
+        _need_cuda(x, out)
+        N = x.shape[0]
+        if x.dtype != torch.float16 or x.dim() != 2 or x.shape[1] != self.w.K or not x.is_contiguous():
+            raise ValueError(f"x must be contiguous fp16 [N][{self.w.K}]")
+        if out.dtype != torch.float32 or tuple(out.shape) != (N, self.w.M) or not out.is_contiguous():
+            raise ValueError(f"out must be contiguous fp32 [{N}][{self.w.M}]")
+        if hq_linear_workspace_size(self.w, N) > self._ws_bytes:
+            raise ValueError(f"batch {N} is larger than this layer's workspace allows")
+        fn = self._fn
+        args = (self._wref, ctypes.c_void_p(x.data_ptr()), ctypes.c_int(N),
+                ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(self._ws),
+                ctypes.c_size_t(self._ws_bytes), ctypes.c_void_p(_raw_stream(stream, self._dev)))
+
+        def launch():
+            st = fn(*args)
+            if st:
+                check(st, "hq_linear")
+
+        launch.buffers = (self, x, out)  # keep them alive as long as the launcher
+        return launch
+
     def check_status(self, stream=None):
         check(lib().hq_check_status(_ptr(self.workspace), _stream(stream)), "device status")
 

@@ -221,6 +221,34 @@ def test_linear_workspace_shared_by_paths_and_batches():
         assert_within(y, want[:n], bound[:n], what=f"batch {n}")
 
 
+def test_rotated_linear_prepared_launcher():
+    """RotatedLinear.prepare: a launcher on fixed buffers gives the oracle's
+    result on every call (also after the inputs change in place), and bad
+    buffers are refused when it is made."""
+    from bit_hadamard_rotated_b200 import RotatedLinear
+    d = synth.linear(700, 1024, 3, 2, seed=23)
+    lin = RotatedLinear(dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]), 3, d["zero"],
+                        max_batch=2)
+    x = torch.zeros((2, 1024), dtype=torch.float16, device="cuda")
+    y = torch.full((2, 700), float("nan"), dtype=torch.float32, device="cuda")
+    run = lin.prepare(x, y)
+    want, bound = oracle.linear(3, 700, 1024, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    x.copy_(dev(d["x"]))
+    for _ in range(2):
+        run()
+        assert_within(y.cpu().numpy(), want, bound, what="prepared launcher")
+    x.mul_(-1)  # the launcher reads the buffer's current contents
+    run()
+    assert_within(y.cpu().numpy(), -want, bound, what="prepared launcher, negated input")
+    with pytest.raises(ValueError):
+        lin.prepare(x.float(), y)
+    with pytest.raises(ValueError):
+        lin.prepare(x, y[:, :699])
+    with pytest.raises(ValueError):
+        lin.prepare(torch.zeros((3, 1024), dtype=torch.float16, device="cuda"),
+                    torch.zeros((3, 700), device="cuda"))
+
+
 # ---------------------------------------------------------------- linear, full workload sizes (sampled rows)
 def sample_rows(M, rng, n=24):
     rows = set(range(0, 8)) | set(range(M - 8, M)) | set(rng.choice(M, n, replace=False).tolist())
