@@ -8,12 +8,15 @@
 //     core matrices), one contiguous block per 128-code group;
 //   * per CTA, an equal contiguous range of (128-row tile, 128-code group)
 //     chunks (stream-K; the first and last tile may be shared with the
-//     neighbouring CTA): one producer thread streams each chunk through a
-//     ring of 4 or 8 shared-memory slots (as many as fit) -- the tile's 128
-//     code rows in one 2D TMA load (swizzled so the decoders' 16-byte row
-//     reads are free of bank conflicts), the group's x' image in one bulk
-//     copy, and at the tile's first chunk its scales in one bulk copy -- all
-//     completing on the slot's mbarrier (expected bytes);
+//     neighbouring CTA), streamed through two rings by two producer threads:
+//     the code ring (up to 16 slots, as many as fit: the weights come from
+//     HBM, so it runs far ahead) takes the tile's 128 code rows in one 2D TMA
+//     load per chunk (swizzled so the decoders' 16-byte row reads are free of
+//     bank conflicts), plus each tile's scales in one bulk copy; a slot is
+//     refilled as soon as its warpgroup has the codes in registers.  The x'
+//     ring (4 slots) takes the group's x' image (L2-resident) in one bulk
+//     copy per chunk and is refilled when the chunk's MMAs are done.  Each
+//     copy completes on its slot's mbarrier (expected bytes);
 //   * two warpgroups take the chunks in turn (chunk c to warpgroup c mod 2):
 //     each thread owns one weight row, decodes its 128 codes into exact fp16
 //     (q - zero) (one LOP3 and one fp16 FMA per pair), multiplies by the group
@@ -24,7 +27,7 @@
 //   * two or four MMA warps take the chunks in the same turn; each issues 8
 //     tcgen05.mma (M=128, N, K=16, A from TMEM, B from shared memory) per
 //     chunk into its own fp32 accumulator in tensor memory and commits their
-//     completion to the slot's and the A stage's mbarriers.  One issuing
+//     completion to the x' slot's and the A stage's mbarriers.  One issuing
 //     thread sustains only one MMA per ~60-80 cycles whatever N is, so at
 //     batch <= 128 more issuers raise the tensor-pipe rate;
 //   * an epilogue warpgroup sums a tile's accumulators (tcgen05.ld) and writes
@@ -34,7 +37,8 @@
 //     (batch <= 32) the next tile's MMAs run while the epilogue reads; the
 //     dequant warps never stop for it.
 // Every barrier's consecutive phases are waited for by one agent, in order
-// (ring depths are multiples of two), so phase-parity waits are unambiguous.
+// (ring depths are multiples of the agent counts), so phase-parity waits are
+// unambiguous.
 // Waits are bounded (status word on timeout); tensor memory is freed on exit.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -53,26 +57,29 @@ namespace hq {
 namespace tc {
 
 constexpr int kTileM = 128;
-constexpr int kNSMax = 8;         // shared-memory ring slots: 4 or 8, as many as fit
-constexpr int kNSMin = 4;
+constexpr int kNCMax = 16;        // code ring slots (HBM latency): as many as fit, <= G
+constexpr int kNCMin = 4;
+constexpr int kNB = 4;            // x' image ring slots (L2 latency)
 constexpr int kASMax = 6;         // A stages in tensor memory (64 columns each): 4 or 6
 constexpr int kDeqWG = 2;         // dequant warpgroups (groups round robin)
 constexpr int kDeqWarps = 4 * kDeqWG;
-constexpr int kProducerWarp = kDeqWarps;
-constexpr int kMmaWarp0 = kDeqWarps + 1;
+constexpr int kProducerWarp = kDeqWarps;  // codes and scales
+constexpr int kBWarp = kDeqWarps + 1;     // x' images
+constexpr int kMmaWarp0 = kDeqWarps + 2;
 constexpr int kMmaWarps = 4;      // issuing threads launched: one issues an MMA per ~60-80 cycles
 constexpr int kEpiWarp0 = kMmaWarp0 + kMmaWarps;
 constexpr int kEpiWarps = 4;      // the epilogue warpgroup: one thread per accumulator row
-constexpr int kThreads = (kDeqWarps + 1 + kMmaWarps + kEpiWarps) * 32;
+constexpr int kThreads = (kDeqWarps + 2 + kMmaWarps + kEpiWarps) * 32;
 // Phase-parity waits are unambiguous only if a barrier's consecutive phases
 // are waited for by the same agent (it cannot wait for round r + 1 before
 // round r completed): every ring depth is a multiple of the dequant
 // warpgroup count, and the A-stage count a multiple of it and of the MMA
 // warp count.
-// The MMA warps in use (n_mma = 2 or 4) wait for the A stages and ring slots
-// too: the host picks stage counts and ring depths that are multiples of it.
-static_assert(kNSMin % kDeqWG == 0 && kNSMax % kDeqWG == 0 && kASMax % kDeqWG == 0 &&
-                  kNSMin % kMmaWarps == 0,
+// The code ring is waited for by the dequant warpgroups (its depth is even);
+// the x' ring and the A stages by the MMA warps in use (n_mma = 2 or 4): the
+// host picks stage counts that are multiples of it, and kNB is one.
+static_assert(kNCMin % kDeqWG == 0 && kNCMax % kDeqWG == 0 && kASMax % kDeqWG == 0 &&
+                  kNB % kMmaWarps == 0,
               "ring depths must be multiples of the agent counts");
 // CTA chunk ranges are whole quanta of kQuant chunks, so every tile portion a
 // CTA computes holds a chunk of every MMA warp and dequant warpgroup.
@@ -253,12 +260,11 @@ struct TcParams {
   int qq, qr;
   float* part;      // [grid][2 sides][128 rows][Npad]: shared tiles' partial sums
   uint32_t* flags;  // [grid]: arrivals at each CTA boundary, zero between calls
-  int slot_bytes;  // codes + B block
-  int b_off;       // B block offset inside a slot
+  int b_off;       // x' image ring (kNB slots of 256 Npad bytes), after the code ring
   int sbuf_off;    // per-tile scale buffers (two)
   int sbuf_bytes;
   int bar_off;
-  int ns;       // shared-memory ring slots (kNSMin..kNSMax)
+  int nc;       // code ring slots (kNCMin..kNCMax, even, <= G)
   int as;       // A stages in tensor memory (4 or 6; a multiple of n_mma)
   int a_base;   // tensor-memory column of A stage 0
   int n_mma;    // MMA warps (accumulators per set) in use: 4 if Npad <= 64, else 2
@@ -392,9 +398,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = p.K / kGroup;
   const int CB = 16 * BITS;  // code bytes of one row in one 128-code group
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + p.bar_off);
-  uint64_t* freeb = full + kNSMax;    // slot's MMAs done (producer may refill)
-  uint64_t* aready = freeb + kNSMax;  // A stage written (MMA may read)
+  const uint32_t code_bytes = kTileM * CB;      // one code slot
+  const uint32_t b_bytes = 256u * p.Npad;        // one x' image slot
+  uint64_t* cfull = reinterpret_cast<uint64_t*>(smem + p.bar_off);  // code slot landed
+  uint64_t* cfree = cfull + kNCMax;   // code slot read by its dequant warpgroup (may refill)
+  uint64_t* bfull = cfree + kNCMax;   // x' image slot landed
+  uint64_t* bfree = bfull + kNB;      // x' image slot's MMAs done (may refill)
+  uint64_t* aready = bfree + kNB;     // A stage written (MMA may read)
   uint64_t* afree = aready + kASMax;  // A stage's MMAs done (dequant may rewrite)
   uint64_t* dready = afree + kASMax;  // [2]: accumulator set's MMAs done (epilogue may read)
   uint64_t* dfree = dready + 2;       // [2]: accumulator set read out (MMA may overwrite)
@@ -406,9 +416,13 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   uint64_t* epib = reinterpret_cast<uint64_t*>(tmem_holder + 2);
 
   if (tid == 0) {
-    for (int i = 0; i < p.ns; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&freeb[i], 1);
+    for (int i = 0; i < p.nc; ++i) {
+      mbar_init(&cfull[i], 1);
+      mbar_init(&cfree[i], 128);  // every thread of the warpgroup, after its reads
+    }
+    for (int i = 0; i < kNB; ++i) {
+      mbar_init(&bfull[i], 1);
+      mbar_init(&bfree[i], 1);
     }
     for (int i = 0; i < p.as; ++i) {
       mbar_init(&aready[i], 128);
@@ -442,10 +456,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
   auto tile_m0 = [&](int ti) { return (tile0 + ti) * kTileM; };
 
   if (warp == kProducerWarp) {
-    // ---------------- producer (one thread): TMA + bulk copies into the ring
+    // ---------------- code producer (one thread): TMA loads of the chunks'
+    // code rows into the code ring, as far ahead as the ring allows (the
+    // weights come from HBM), and each tile's scales
     if (lane == 0) {
-      const uint32_t b_bytes = 256u * p.Npad;
-      const uint32_t code_bytes = kTileM * CB;
       bool ok = true;
       int issued = 0;
       // ring position kept incrementally (no divisions on the issue path)
@@ -453,14 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       uint32_t rph = 0;  // parity of the ring round of chunk c
       int m0 = tile_m0(0), ti = 0;
       int rows = min(kTileM, p.M - m0);
-      const uint8_t* bsrc = p.img + static_cast<size_t>(g_start) * b_bytes;
       for (int c = 0; c < total; ++c) {
-        // slot reuse: the MMAs of chunk c - ns (previous round) are done
-        if (c >= p.ns && !mbar_wait(&freeb[sl], rph ^ 1u)) {
+        // slot reuse: chunk c - nc's dequant warpgroup has read the slot.
+        // Waiting for every chunk in order also means that at a tile's first
+        // chunk every chunk two tiles back has read its scales (nc <= G), so
+        // the scale buffer ti & 1 is free again.
+        if (c >= p.nc && !mbar_wait(&cfree[sl], rph ^ 1u)) {
           ok = false;
           break;
         }
-        uint8_t* base = smem + sl * p.slot_bytes;
         // the tile's scales, once per tile, on the buffer's own barrier (a
         // bulk copy's completion shows only on the barrier it signals)
         if (g == 0 || c == 0) {
@@ -470,12 +485,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
                    p.scales + static_cast<size_t>(m0) * G * 2, s_bytes, &sready[ti & 1]);
         }
         // a TMA tile always delivers the whole box (rows past M read as zero)
-        mbar_arrive_expect_tx(&full[sl], code_bytes + b_bytes);
-        tma_load_2d(base, &p.qmap, g * CB, m0, &full[sl]);
-        bulk_g2s(base + p.b_off, bsrc, b_bytes, &full[sl]);
+        mbar_arrive_expect_tx(&cfull[sl], code_bytes);
+        tma_load_2d(smem + sl * code_bytes, &p.qmap, g * CB, m0, &cfull[sl]);
         issued = c + 1;
-        bsrc += b_bytes;
-        if (++sl == p.ns) {
+        if (++sl == p.nc) {
           sl = 0;
           rph ^= 1u;
         }
@@ -484,17 +497,50 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           ++ti;
           m0 += kTileM;
           rows = min(kTileM, p.M - m0);
-          bsrc = p.img;
         }
       }
       // Drain: the copies of the last slots must have landed before exit (they
       // have on the normal path, where the dequant warps consumed them).
-      for (int c = max(0, issued - p.ns); c < issued; ++c) {
-        if (!mbar_wait(&full[c % p.ns], (c / p.ns) & 1)) ok = false;
+      for (int c = max(0, issued - p.nc); c < issued; ++c) {
+        if (!mbar_wait(&cfull[c % p.nc], (c / p.nc) & 1)) ok = false;
       }
       if (issued > 0) {
         const int lt = (g_start + issued - 1) / G;  // the last tile whose scales were requested
         if (!mbar_wait(&sready[lt & 1], (lt >> 1) & 1)) ok = false;
+      }
+      if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
+    }
+    __syncwarp();
+  } else if (warp == kBWarp) {
+    // ---------------- x' producer (one thread): the chunk's group image
+    // (256 Npad bytes, L2-resident) into the x' ring, freed by the MMAs
+    if (lane == 0) {
+      bool ok = true;
+      int issued = 0;
+      int sl = 0, g = g_start;
+      uint32_t rph = 0;
+      const uint8_t* bsrc = p.img + static_cast<size_t>(g_start) * b_bytes;
+      uint8_t* bring = smem + p.b_off;
+      for (int c = 0; c < total; ++c) {
+        if (c >= kNB && !mbar_wait(&bfree[sl], rph ^ 1u)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bfull[sl], b_bytes);
+        bulk_g2s(bring + sl * b_bytes, bsrc, b_bytes, &bfull[sl]);
+        issued = c + 1;
+        bsrc += b_bytes;
+        if (++sl == kNB) {
+          sl = 0;
+          rph ^= 1u;
+        }
+        if (++g == G) {
+          g = 0;
+          bsrc = p.img;
+        }
+      }
+      for (int c = max(0, issued - kNB); c < issued; ++c) {
+        if (!mbar_wait(&bfull[c % kNB], (c / kNB) & 1)) ok = false;
       }
       if (!ok) record_error(p.status, HQ_DEV_TIMEOUT);
     }
@@ -510,12 +556,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       // (in 16-byte units; every address stays below 2^18, so the 14-bit
       // field never carries)
       const uint64_t bdesc0 = smem_desc(smem_u32(smem + p.b_off), 16 * p.Npad, 128);
-      const uint32_t slot16 = static_cast<uint32_t>(p.slot_bytes) >> 4;
+      const uint32_t slot16 = b_bytes >> 4;
       const uint32_t ks16 = 2u * p.Npad;  // 32 Npad bytes
       const uint32_t acc_set = static_cast<uint32_t>(p.n_mma * p.Npad);  // columns per set
-      const int step = p.n_mma;  // divides as, ns, G and kQuant
-      int sl = j, st = j, g = g_start + j, ti = 0;  // slot (mod ns), A stage (mod as)
-      uint32_t aph = 0, sph = 0;                    // A-stage and slot round parities
+      const int step = p.n_mma;  // divides as, kNB, G and kQuant
+      int sl = j, st = j, g = g_start + j, ti = 0;  // x' slot (mod kNB), A stage (mod as)
+      uint32_t aph = 0, sph = 0;                    // A-stage and x' slot round parities
       bool first = true;  // the next chunk is this warp's first of its tile portion
       for (int c = j; c < total && ok; c += step) {
         // a new tile portion overwrites its accumulator set: the epilogue of
@@ -523,8 +569,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         const int buf = p.nacc == 2 ? (ti & 1) : 0, use = p.nacc == 2 ? (ti >> 1) : ti;
         if (first && use > 0) ok = mbar_wait(&dfree[buf], (use - 1) & 1);
         ok = ok && mbar_wait(&aready[st], aph);
-        // B arrived by TMA: observe its barrier here too (already complete)
-        ok = ok && mbar_wait(&full[sl], sph);
+        ok = ok && mbar_wait(&bfull[sl], sph);  // the group's x' image has landed
         if (!ok) break;
         tc_fence_after();
         if (lane == 0) {
@@ -534,7 +579,7 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           tc_mma_ts(dacc, a0, d0, p.idesc, first ? 0u : 1u);
 #pragma unroll
           for (int ks = 1; ks < 8; ++ks) tc_mma_ts(dacc, a0 + ks * 8, d0 + ks * ks16, p.idesc, 1u);
-          tc_commit(&freeb[sl]);
+          tc_commit(&bfree[sl]);
           tc_commit(&afree[st]);
           // this warp's last chunk of the portion (tile end or range end)
           if (g + step >= G || c + step >= total) tc_commit(&dready[buf]);
@@ -542,8 +587,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         __syncwarp();
         first = false;
         sl += step;
-        if (sl >= p.ns) {
-          sl -= p.ns;
+        if (sl >= kNB) {
+          sl -= kNB;
           sph ^= 1u;
         }
         st += step;
@@ -577,9 +622,9 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
     bool ok = true;
     uint4 scache = make_uint4(0, 0, 0, 0);  // this row's scales for 8 groups
     int sblock = -1;                         // which block of 8 groups scache holds
-    // this warpgroup's chunks c = wg, wg + kDeqWG, ...: slot (mod ns), A
+    // this warpgroup's chunks c = wg, wg + kDeqWG, ...: code slot (mod nc), A
     // stage (mod as), their round parities, group and tile advance
-    // incrementally (kDeqWG divides as and ns; kDeqWG < G).  Every round of
+    // incrementally (kDeqWG divides as and nc; kDeqWG < G).  Every round of
     // this warpgroup's slots and stages is waited for by this warpgroup alone,
     // in order, so a parity wait never meets a phase two rounds old.
     int sl = wg, st = wg, g = g_start + wg, ti = 0;
@@ -593,12 +638,12 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
           break;
         }
       }
-      // the slot's copies have landed, and the A stage's previous MMAs are done
-      if (!mbar_wait(&full[sl], sph) || (c >= p.as && !mbar_wait(&afree[st], aph ^ 1u))) {
+      // the slot's codes have landed, and the A stage's previous MMAs are done
+      if (!mbar_wait(&cfull[sl], sph) || (c >= p.as && !mbar_wait(&afree[st], aph ^ 1u))) {
         ok = false;
         break;
       }
-      const uint4* rowp = reinterpret_cast<const uint4*>(smem + sl * p.slot_bytes + r * CB);
+      const uint4* rowp = reinterpret_cast<const uint4*>(smem + sl * code_bytes + r * CB);
       if ((g >> 3) != sblock) {  // first group of this warpgroup in a block of 8
         sblock = g >> 3;
         scache = *reinterpret_cast<const uint4*>(smem + p.sbuf_off + (ti & 1) * p.sbuf_bytes +
@@ -617,6 +662,10 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
         rw[4 * i + 2] = u.z;
         rw[4 * i + 3] = u.w;
       }
+      // the codes (and this block's scales) are in registers: order these
+      // generic-proxy reads before the TMA (async proxy) that refills the slot
+      fence_proxy_async_smem();
+      mbar_arrive(&cfree[sl]);
 #pragma unroll
       for (int t = 0; t < 4; ++t) {
         uint32_t w[BITS];
@@ -632,8 +681,8 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
       tc_fence_before();
       mbar_arrive(&aready[st]);
       sl += kDeqWG;
-      if (sl >= p.ns) {
-        sl -= p.ns;
+      if (sl >= p.nc) {
+        sl -= p.nc;
         sph ^= 1u;
       }
       st += kDeqWG;
@@ -660,24 +709,24 @@ __global__ void __launch_bounds__(kThreads, 1) tc_gemm_kernel(const __grid_const
 
 // ---------------------------------------------------------------- host side
 struct TcPlan {
-  int ns = 0, slot = 0, b_off = 0, sbuf_off = 0, sbuf_bytes = 0, bar_off = 0;
+  int nc = 0, b_off = 0, sbuf_off = 0, sbuf_bytes = 0, bar_off = 0;
   size_t smem = 0;
 };
 
 constexpr size_t kMaxSmemTc = 227 * 1024 - 1024;  // dynamic; the base is rounded up to 1 KiB
 constexpr size_t kMinSmemTc = 116 * 1024;         // > half an SM's shared memory
-constexpr size_t kBarBytes = 320;  // 35 mbarriers, the TMEM address and arrival words, 1 mbarrier
+constexpr size_t kBarBytes = 512;  // 59 mbarriers, the TMEM address and arrival words, 1 mbarrier
 
-// Plan with ns ring slots (0 smem when it does not fit).
-static TcPlan tc_plan_ns(int bits, int K, int npad, int ns) {
+// Plan with nc code slots (0 smem when it does not fit): [nc code slots: 128
+// rows x 16 bits bytes, swizzled, each a multiple of 1 KiB so every slot keeps
+// the swizzle atom][kNB x' image slots of 256 npad bytes][two scale buffers]
+// [barriers].
+static TcPlan tc_plan_nc(int bits, int K, int npad, int nc) {
   TcPlan pl;
   const int G = K / kGroup;
-  // slot: [128 code rows, 16*bits bytes each, dense and swizzled][x' image];
-  // both sizes are multiples of 1 KiB, so every slot keeps the swizzle atom
-  pl.ns = ns;
-  pl.b_off = kTileM * 16 * bits;
-  pl.slot = pl.b_off + 256 * npad;
-  pl.sbuf_off = ns * pl.slot;
+  pl.nc = nc;
+  pl.b_off = nc * kTileM * 16 * bits;
+  pl.sbuf_off = pl.b_off + kNB * 256 * npad;
   pl.sbuf_bytes = kTileM * G * 2;
   pl.bar_off = pl.sbuf_off + 2 * pl.sbuf_bytes;
   pl.smem = static_cast<size_t>(pl.bar_off) + kBarBytes + 1024;
@@ -685,11 +734,14 @@ static TcPlan tc_plan_ns(int bits, int K, int npad, int ns) {
   return pl;
 }
 
-// The deepest ring that fits (at least kNSMin slots; smem 0 if none fits).
+// The deepest code ring that fits: kNCMin..kNCMax slots, even, and at most G
+// (a tile's scale buffer is refilled only once every chunk two tiles back has
+// read it); smem 0 if none fits.
 static TcPlan tc_plan(int bits, int K, int npad) {
-  TcPlan best = tc_plan_ns(bits, K, npad, kNSMin);
-  for (int ns = kNSMin + kDeqWG; ns <= kNSMax && best.smem != 0; ns += kDeqWG) {
-    const TcPlan pl = tc_plan_ns(bits, K, npad, ns);
+  const int G = K / kGroup;
+  TcPlan best = tc_plan_nc(bits, K, npad, kNCMin);
+  for (int nc = kNCMin + kDeqWG; nc <= std::min(kNCMax, G) && best.smem != 0; nc += kDeqWG) {
+    const TcPlan pl = tc_plan_nc(bits, K, npad, nc);
     if (pl.smem == 0) break;
     best = pl;
   }
@@ -857,7 +909,6 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.qr = quanta % grid_i;
     p.part = part;
     p.flags = a.counters;
-    p.slot_bytes = pl.slot;
     p.b_off = pl.b_off;
     p.sbuf_off = pl.sbuf_off;
     p.sbuf_bytes = pl.sbuf_bytes;
@@ -871,7 +922,7 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.a_base = (p.nacc * p.n_mma * npad + 63) & ~63;
     p.as = ((tc::kTmemCols - p.a_base) / 64) / p.n_mma * p.n_mma;
     if (p.as > tc::kASMax) p.as = tc::kASMax / p.n_mma * p.n_mma;
-    p.ns = pl.ns / p.n_mma * p.n_mma;
+    p.nc = pl.nc;
     p.idesc = tc::idesc_f16(tc::kTileM, npad);
     const dim3 g(grid), blk(tc::kThreads);
     switch (a.bits) {
