@@ -16,7 +16,7 @@
  *   - the contraction  y[n][m] = sum_k w[m][k] * x'[n][k],
  *   - the MoE expert composition (gate/up, SwiGLU, down, weighted combine).
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings where the pages are silent (the plainest reading in each case):
  *   - H_K is the Sylvester Hadamard matrix in natural order,
  *     H[i][j] = (-1)^popcount(i & j); the 1/sqrt(K) factor is applied once.
  *   - sign s_i = -1 where signs[i] < 0, else +1; a NULL sign vector means s = 1.
