@@ -168,23 +168,37 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
   int* s_nb0 = sm + d.E + 1;        // [E + 1] first block of each expert; [E] = blocks in all
   int* s_sw = s_nb0 + d.E + 1;      // [E + 1] width, then phase A's block-weight prefix
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nt = blockDim.x;
-  // every expert's width, or -1 for a bad descriptor; the expert table is a
-  // weight (no earlier kernel of the library writes it), read before the wait
+  // s_sw[e]: the width of expert e if its descriptor is valid, else -1 (or 0
+  // while unknown).  With a few descriptors per thread, all of them are
+  // checked before the wait (the expert table is a weight: no earlier kernel
+  // of the library writes it); with more, only those the pairs name, after it.
+  const bool all_desc = d.E <= 4 * nt;
   for (int e = tid; e < d.E; e += nt) {
     s_cnt[e] = 0;
-    const hq_expert de = ex[e];
-    s_sw[e] = valid_desc(de) ? de.bits : -1;
+    int sw = 0;
+    if (all_desc) {
+      const hq_expert de = ex[e];
+      sw = valid_desc(de) ? de.bits : -1;
+    }
+    s_sw[e] = sw;
   }
   __syncthreads();
   pdl_wait();  // ids may be the previous kernel's output; the workspace is free once it is done
   // validity of every pair (its expert id and that expert's descriptor)
   for (int i = tid; i < d.P; i += nt) {
     const int e = ids[i];
-    if (e < 0 || e >= d.E) {
+    bool ok = e >= 0 && e < d.E;
+    if (!ok) {
       record_error(w.status, HQ_DEV_BAD_EXPERT);
-      w.pos[i] = -1;
-    } else if (s_sw[e] < 0) {
-      record_error(w.status, HQ_DEV_BAD_BITS);
+    } else if (all_desc) {
+      ok = s_sw[e] > 0;
+    } else {
+      const hq_expert de = ex[e];
+      ok = valid_desc(de);
+      if (ok) s_sw[e] = de.bits;  // the same value from every pair of e
+    }
+    if (!ok) {
+      if (e >= 0 && e < d.E) record_error(w.status, HQ_DEV_BAD_BITS);
       w.pos[i] = -1;
     }
   }

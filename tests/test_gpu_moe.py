@@ -155,6 +155,33 @@ def test_moe_bad_ids_and_descriptors_are_skipped_and_reported():
     check(y, want, bound, "bad ids")
 
 
+@pytest.mark.parametrize("E", [200, 1500])
+def test_moe_many_experts_untouched_bad_descriptor(E):
+    """Routing over many experts.  With hidden 128 (64-thread routing block)
+    the 200-entry table is checked whole before the dependent-launch wait,
+    the 1500-entry one only where the pairs name it; either way a bad
+    descriptor that no pair names reports nothing and changes nothing.  Expert
+    e's descriptor points at expert e % 5's tensors."""
+    from bit_hadamard_rotated_b200 import expert_table, hq_check_status, hq_moe_experts, \
+        hq_moe_workspace_size
+    T, k = 7, 3
+    m = synth.moe(seed=12, E=5, hidden=128, inter=128, T=T, k=k)
+    base = device_experts(m["experts"])
+    bad_e = E // 2
+    descs = [base[e % 5] for e in range(E)]
+    descs[bad_e] = dict(base[bad_e % 5], bits=5)
+    rng = np.random.default_rng(E)
+    choices = np.array([e for e in range(E) if e != bad_e])
+    ids = np.stack([rng.choice(choices, k, replace=False) for _ in range(T)]).astype(np.int32)
+    w = m["topk_w"].astype(np.float32)
+    ws = torch.zeros(hq_moe_workspace_size(E, 128, 128, T, k), dtype=torch.uint8, device="cuda")
+    y = hq_moe_experts(expert_table(descs, "cuda"), E, 128, 128, dev(m["x"]), dev(ids), dev(w),
+                       dev(m["s_in"]), dev(m["s_mid"]), workspace=ws).cpu().numpy()
+    hq_check_status(ws)  # nothing recorded
+    want, bound, _ = oracle_moe(m, ids=ids % 5, w=w)
+    check(y, want, bound, f"E={E}")
+
+
 def test_moe_zero_tokens():
     from bit_hadamard_rotated_b200 import expert_table, hq_moe_experts
     m = synth.moe(seed=9, E=3, hidden=256, inter=128, T=2, k=1)
