@@ -292,7 +292,8 @@ def run_ours(a):
 
 
 def measure_b64(device, stream, pk):
-    """TFLOP/s of the large dense MLP linear (28672x8192, 2-bit) at batch 64 (and 16)."""
+    """TFLOP/s of the large dense MLP linear (28672x8192, 2-bit) at batch 64 (and 16; batch 1
+    on the GEMV, weight GB/s)."""
     from bit_hadamard_rotated_b200 import RotatedLinear
     M, K, b, N = B64
     d = synth.linear(M, K, b, N, seed=77, scale_dist="loguniform", outlier_frac=0.01)
@@ -301,7 +302,7 @@ def measure_b64(device, stream, pk):
                         torch.from_numpy(d["signs"]).to(device), b, d["zero"], max_batch=N)
     flush = torch.empty(2 * 126 * 2**20 // 4, dtype=torch.float32, device=device)
     out = {}
-    for n in (N, 16):
+    for n in (N, 16, 1):
         x = torch.from_numpy(np.ascontiguousarray(d["x"][:n])).to(device)
         y = torch.empty((n, M), dtype=torch.float32, device=device)
         with torch.cuda.stream(stream):
@@ -325,10 +326,11 @@ def measure_b64(device, stream, pk):
         out[n] = {"ms": round(ms, 4), "tflops": round(tflops, 2),
                   "frac_bf16_peak": round(tflops / pk["bf16"], 4),
                   "weight_gbs": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9, 1),
+                  "frac_hbm": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9 / pk["hbm"], 4),
                   "launches": lin.launches(n)}
     r = {"workload": f"rotated linear M={M} K={K} b{b} batch {N}", **out[N],
          "timing": "CUDA-graph replay of one call, median of 20, L2 flushed before each",
-         "batch16": out[16]}
+         "batch16": out[16], "batch1": out[1]}
     return r
 
 
