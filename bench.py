@@ -519,7 +519,7 @@ def measure_e2e(device, layers, xs, a):
         per_b = []
         for b in range(NB):
             fns, ox, oy = [], 0, 0
-            for li, (M, K, bits) in enumerate(LAYERS):
+            for li, (M, _K, _b) in enumerate(LAYERS):
                 fns.append(layers[c][li].prepare(xd[b][ox:ox + xsz[li]].view(1, -1),
                                                  yd[b][oy:oy + M].view(1, -1), stream=comp))
                 ox += xsz[li]
