@@ -18,6 +18,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "hq.h")
 HQ_OK, HQ_ERR_INVALID_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_WORKSPACE, HQ_ERR_CUDA, HQ_ERR_DATA, \
     HQ_ERR_TIMEOUT = range(7)
 HQ_F16, HQ_BF16, HQ_F32 = 0, 1, 2
+HQ_MOE_POS, HQ_MOE_H, HQ_MOE_D = 0, 1, 2
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -74,6 +75,10 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_uses_tensor_cores.restype = _i
         L.hq_linear_noalloc.argtypes = [ctypes.POINTER(HqWeight), _vp, _i, _vp, _vp]
         L.hq_linear_noalloc.restype = _i
+        L.hq_linear_noalloc_check_status.argtypes = [_vp]
+        L.hq_linear_noalloc_check_status.restype = _i
+        L.hq_moe_workspace_offset.argtypes = [_i, _i, _i, _i, _i, _i]
+        L.hq_moe_workspace_offset.restype = _sz
         L.hq_moe_launches.argtypes = []
         L.hq_moe_launches.restype = _i
         L.hq_set_tc_min_batch.argtypes = [_i]

@@ -1091,6 +1091,18 @@ size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k)
 
 int hq_moe_launches(void) { return 5; }
 
+size_t hq_moe_workspace_offset(int n_experts, int hidden, int inter, int T, int k,
+                               hq_moe_part part) {
+  if (hq_moe_workspace_size(n_experts, hidden, inter, T, k) == 0) return static_cast<size_t>(-1);
+  const MoePlan pl = moe_plan(n_experts, hidden, inter, T, k);
+  switch (part) {
+    case HQ_MOE_POS: return pl.off[3];
+    case HQ_MOE_H: return pl.off[10];
+    case HQ_MOE_D: return pl.off[13];
+  }
+  return static_cast<size_t>(-1);
+}
+
 hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, int inter,
                          const uint16_t* x, int T, const int32_t* topk_ids, const float* topk_w,
                          int k, const int8_t* signs_in, const int8_t* signs_mid, float* y,

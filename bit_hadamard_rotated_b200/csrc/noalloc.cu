@@ -19,9 +19,8 @@
 //     streams, or two host threads) race on it and must be serialised by the
 //     caller;
 //   * device-side wait timeouts are recorded in the array's status word, which
-//     the next call clears; there is no way to read it back.
-#include <mutex>
-
+//     the next call clears: hq_linear_noalloc_check_status reads (and clears)
+//     what the last call recorded.
 #include "hq_internal.h"
 
 namespace hq {
@@ -36,25 +35,19 @@ constexpr size_t kXgBytes = kScratchBytes - kStatus;
 // Static storage starts zeroed; each call clears the status word.
 __device__ __align__(256) uint8_t g_noalloc_scratch[kScratchBytes];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mu;
-uint8_t* g_scratch_addr[kMaxDevices] = {};
-
-// Device address of the array on the current device (looked up once per
-// device: the host-side name of a __device__ variable is not a device address).
-cudaError_t scratch_on_current_device(uint8_t** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+// Device address of the array in the current context.  The host-side name of
+// a __device__ variable is not a device address, and the address belongs to a
+// CUDA context, not to a device ordinal: a host that binds its own
+// (non-primary) context, or a cudaDeviceReset that reloads the module, gives
+// the array a new address.  So it is looked up on every call; the lookup is a
+// runtime query that allocates nothing.  The first lookup in a context loads
+// the library's device code there, which is why the first call belongs before
+// any stream capture.
+cudaError_t scratch_in_current_context(uint8_t** out) {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_setup_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_addr[dev] = static_cast<uint8_t*>(p);
-  }
-  *out = g_scratch_addr[dev];
+  *out = static_cast<uint8_t*>(p);
   return cudaSuccess;
 }
 
@@ -91,7 +84,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
   if (gemv_scratch_bytes(w->K, nb) > kXgBytes) return HQ_ERR_WORKSPACE;
 
   uint8_t* scratch = nullptr;
-  if (scratch_on_current_device(&scratch) != cudaSuccess) {
+  if (scratch_in_current_context(&scratch) != cudaSuccess) {
     (void)cudaGetLastError();
     return HQ_ERR_CUDA;
   }
@@ -121,4 +114,25 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     }
   }
   return HQ_OK;
+}
+
+// The status word is the first word of the scratch: every call clears it
+// before its kernels run, so after a synchronisation it holds what the last
+// call's kernels recorded.
+extern "C" hq_status hq_linear_noalloc_check_status(hq_stream_t stream) {
+  uint8_t* scratch = nullptr;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t v = 0;
+  if (scratch_in_current_context(&scratch) != cudaSuccess ||
+      cudaMemcpyAsync(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return HQ_ERR_CUDA;
+  }
+  if (v == 0) return HQ_OK;
+  if (cudaMemsetAsync(scratch, 0, sizeof(v), st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return HQ_ERR_CUDA;
+  }
+  return (v & HQ_DEV_TIMEOUT) ? HQ_ERR_TIMEOUT : HQ_ERR_DATA;
 }

@@ -66,6 +66,22 @@ def hq_linear_workspace_size(w: HqWeight, batch: int) -> int:
     return int(lib().hq_linear_workspace_size(ctypes.byref(w), batch))
 
 
+def _check_linear_io(w: HqWeight, x: torch.Tensor, out: torch.Tensor | None, dev) -> None:
+    """x must be contiguous fp16 [N][K] and out contiguous fp32 [N][M], both on
+    the weight's device (the kernels read raw pointers: a wrong shape or
+    stride would read out of bounds)."""
+    if x.dtype != torch.float16 or x.dim() != 2 or x.shape[1] != w.K or not x.is_contiguous():
+        raise ValueError(f"x must be contiguous fp16 [N][{w.K}], got {x.dtype} {tuple(x.shape)}")
+    if x.device != dev:
+        raise ValueError(f"x is on {x.device}, the weights on {dev}")
+    if out is not None:
+        N = x.shape[0]
+        if out.dtype != torch.float32 or tuple(out.shape) != (N, w.M) or not out.is_contiguous():
+            raise ValueError(f"out must be contiguous fp32 [{N}][{w.M}]")
+        if out.device != dev:
+            raise ValueError(f"out is on {out.device}, the weights on {dev}")
+
+
 def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
               x: torch.Tensor, bits: int, zero: int | None = None,
               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
@@ -73,14 +89,16 @@ def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor |
     """y[n][m] = sum_k scale (q - zero) x'[n][k]; x fp16 [N][K] -> y fp32 [N][M]."""
     _need_cuda(qweight, scales, signs, x)
     w = make_weight(qweight, scales, signs, bits, zero)
+    _check_linear_io(w, x, out, qweight.device)
     N = x.shape[0]
-    if out is None:
-        out = torch.empty((N, w.M), dtype=torch.float32, device=x.device)
-    need = hq_linear_workspace_size(w, N)
-    if workspace is None:
-        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
-    st = lib().hq_linear(ctypes.byref(w), _ptr(x), N, _ptr(out), _ptr(workspace),
-                         workspace.numel(), _stream(stream))
+    with torch.cuda.device(qweight.device):
+        if out is None:
+            out = torch.empty((N, w.M), dtype=torch.float32, device=x.device)
+        need = hq_linear_workspace_size(w, N)
+        if workspace is None:
+            workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
+        st = lib().hq_linear(ctypes.byref(w), _ptr(x), N, _ptr(out), _ptr(workspace),
+                             workspace.numel(), _stream(stream))
     check(st, "hq_linear")
     return out
 
@@ -92,12 +110,19 @@ def hq_linear_noalloc(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.
     used instead; calls must not overlap on the GPU)."""
     _need_cuda(qweight, scales, signs, x)
     w = make_weight(qweight, scales, signs, bits, zero)
+    _check_linear_io(w, x, out, qweight.device)
     N = x.shape[0]
-    if out is None:
-        out = torch.empty((N, w.M), dtype=torch.float32, device=x.device)
-    check(lib().hq_linear_noalloc(ctypes.byref(w), _ptr(x), N, _ptr(out), _stream(stream)),
-          "hq_linear_noalloc")
+    with torch.cuda.device(qweight.device):
+        if out is None:
+            out = torch.empty((N, w.M), dtype=torch.float32, device=x.device)
+        st = lib().hq_linear_noalloc(ctypes.byref(w), _ptr(x), N, _ptr(out), _stream(stream))
+    check(st, "hq_linear_noalloc")
     return out
+
+
+def hq_linear_noalloc_check_status(stream=None) -> None:
+    """Raise HqError if the last hq_linear_noalloc call recorded a device error."""
+    check(lib().hq_linear_noalloc_check_status(_stream(stream)), "hq_linear_noalloc status")
 
 
 class RotatedLinear:
@@ -227,6 +252,6 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
-__all__ = ["hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_workspace_size", "RotatedLinear",
+__all__ = ["hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
            "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

@@ -182,14 +182,37 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
  * rotated activations of one batch block (at most 332 KiB, K = 16384).  Limits:
  * as hq_linear (HQ_ERR_WORKSPACE if a block's activations did not fit, which
  * no supported K reaches).
- * The first call on a device looks up the array's device address (a CUDA
- * runtime query, no allocation); make that first call before any stream
+ * The array's device address is looked up on every call (a runtime query that
+ * allocates nothing); the first call in a CUDA context also loads the
+ * library's device code there, so make that first call before any stream
  * capture.  All calls share the array: calls that overlap on the GPU race and
- * must be serialised by the caller.  Each call clears the part of the array
- * that must start at zero; device-side wait timeouts cannot be read back.
+ * must be serialised by the caller.  Each call clears the array's status word
+ * before its kernels run; hq_linear_noalloc_check_status reads it back.
  */
 hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, int batch, float* y,
                             hq_stream_t stream);
+
+/* Intermediates an hq_moe_experts call leaves in its workspace, for checking
+ * the layer stage by stage:
+ *   HQ_MOE_POS  int32 [T*k]: row of pair (t, j) (index t*k + j) in the two
+ *               arrays below, or -1 if the pair was skipped (bad id or
+ *               descriptor);
+ *   HQ_MOE_H    fp32 [rows][inter]: h = silu(W_gate x') * (W_up x') of each pair;
+ *   HQ_MOE_D    fp32 [rows][hidden]: d = W_down h' of each pair.
+ * The rows are grouped by expert (the order of the stable sort by expert id). */
+typedef enum { HQ_MOE_POS = 0, HQ_MOE_H = 1, HQ_MOE_D = 2 } hq_moe_part;
+
+/* Byte offset of `part` inside an hq_moe_experts workspace of these sizes,
+ * valid after the call has completed (SIZE_MAX on a bad argument). */
+size_t hq_moe_workspace_offset(int n_experts, int hidden, int inter, int T, int k,
+                               hq_moe_part part);
+
+/* Synchronises `stream`, then reads and clears the status word that the last
+ * hq_linear_noalloc call left in the library's scratch array: HQ_OK, or
+ * HQ_ERR_TIMEOUT if a bounded device-side wait of that call ran out (its
+ * output is then incomplete).  No counterpart on the pages, like
+ * hq_linear_noalloc.  HQ_ERR_CUDA if a CUDA call fails. */
+hq_status hq_linear_noalloc_check_status(hq_stream_t stream);
 
 /* Synchronises `stream`, reads the status word of a workspace used by
  * hq_linear or hq_moe_experts, clears it, and returns HQ_OK or the first

@@ -175,3 +175,17 @@ def test_linear_path_choice():
     assert path(2, 8192, 8) == 0 and path(2, 8192, 9) == 1
     assert path(4, 512, 64) == 0      # K < 1024: GEMV at every batch
     assert path(4, 4096, 0) == -1 and path(5, 4096, 4) == -1
+
+
+def test_moe_workspace_offsets(L):
+    """The stage intermediates lie inside the workspace, 256-byte aligned, in
+    the order pos < h < d; a bad argument or part gives SIZE_MAX."""
+    from bit_hadamard_rotated_b200._lib import HQ_MOE_D, HQ_MOE_H, HQ_MOE_POS
+    E, H, I, T, k = 256, 2048, 512, 32, 8
+    size = L.hq_moe_workspace_size(E, H, I, T, k)
+    pos, h, d = (L.hq_moe_workspace_offset(E, H, I, T, k, p) for p in (HQ_MOE_POS, HQ_MOE_H, HQ_MOE_D))
+    assert pos % 256 == 0 and h % 256 == 0 and d % 256 == 0
+    assert pos + 4 * T * k <= h and h + 4 * T * k * I <= d and d + 4 * T * k * H <= size
+    none = ctypes.c_size_t(-1).value
+    assert L.hq_moe_workspace_offset(E, H + 1, I, T, k, HQ_MOE_H) == none
+    assert L.hq_moe_workspace_offset(E, H, I, T, k, 7) == none

@@ -2,7 +2,9 @@
 
 Tolerance (end to end, two chained contractions): |y - y_oracle| <=
 4e-3 * sum_j |topk_w[t][j]| sum_k |w_down x h'_k| + 1e-5, the oracle's bound;
-each single contraction is held to 2e-3 elsewhere, and the chain doubles it.
+each single contraction is held to 2e-3 (the stage-wise checks below: h
+against the oracle's h, and d against the oracle's down projection of the
+GPU's own h), and the chain doubles it.
 """
 import ctypes
 
@@ -190,3 +192,72 @@ def test_moe_zero_tokens():
     y = hq_moe_experts(table, 3, 256, 128, dev(m["x"][:0]), dev(m["topk_ids"][:0]),
                        dev(m["topk_w"][:0]), dev(m["s_in"]), dev(m["s_mid"]))
     assert y.shape == (0, 256)
+
+
+# ---------------------------------------------------------------- stage by stage
+def _stages(ws, m, E):
+    """pos [T*k], h [rows][inter], d [rows][hidden] as the call left them in its workspace."""
+    from bit_hadamard_rotated_b200 import _lib
+    L = _lib.lib()
+    T, k, H, I = m["T"], m["k"], m["hidden"], m["inter"]
+    raw = ws.cpu().numpy()
+
+    def part(which, count, dtype):
+        off = L.hq_moe_workspace_offset(E, H, I, T, k, which)
+        assert off % 256 == 0
+        return raw[off:off + count * np.dtype(dtype).itemsize].view(dtype)
+
+    rows = T * k
+    return (part(_lib.HQ_MOE_POS, rows, np.int32), part(_lib.HQ_MOE_H, rows * I, np.float32).reshape(rows, I),
+            part(_lib.HQ_MOE_D, rows * H, np.float32).reshape(rows, H))
+
+
+def _check_stages(m, ws):
+    E, T, k, H, I = len(m["experts"]), m["T"], m["k"], m["hidden"], m["inter"]
+    pos, h_gpu, d_gpu = _stages(ws, m, E)
+    _, _, h_want = oracle.moe(m["experts"], H, I, m["x"], m["topk_ids"], m["topk_w"], m["s_in"],
+                              m["s_mid"], want_h=True, threads=8)
+    assert sorted(pos.tolist()) == list(range(T * k))  # every pair valid, rows a permutation
+    xr = oracle.rotate(m["x"], m["s_in"])
+    rel = 2e-3
+    for t in range(T):
+        for j in range(k):
+            e = m["experts"][int(m["topk_ids"][t, j])]
+            r = int(pos[t * k + j])
+            # gate/up + SwiGLU: h = silu(g) u with g, u each within 2e-3 of their own
+            # L1 bases Bg, Bu; to first order |dh| <= max|silu'| |u| dg + |silu(g)| du
+            # (max silu' = 1.0998), plus the product of the two errors
+            g, bg = oracle.dequant_dot(e["bits"], I, H, e["zero"], e["q_gate"], e["s_gate"], xr[t:t + 1])
+            u, bu = oracle.dequant_dot(e["bits"], I, H, e["zero"], e["q_up"], e["s_up"], xr[t:t + 1])
+            g, bg, u, bu = g[0], bg[0], u[0], bu[0]
+            silu = g / (1.0 + np.exp(-g))
+            lim = rel * (1.1 * np.abs(u) * bg + np.abs(silu) * bu) + 1.1 * rel * rel * bg * bu + 1e-5
+            err = np.abs(h_gpu[r].astype(np.float64) - h_want[t * k + j])
+            assert np.all(err <= lim), ("h", t, j, float(np.max(err / lim)))
+            # down, fed the GPU's own h: d = W_down H diag(s_mid) h_gpu / sqrt(inter)
+            hr = oracle.rotate(h_gpu[r].astype(np.float64), m["s_mid"])
+            dw, db = oracle.dequant_dot(e["bits"], H, I, e["zero"], e["q_down"], e["s_down"], hr[None, :])
+            err = np.abs(d_gpu[r].astype(np.float64) - dw[0])
+            lim = rel * db[0] + 1e-5
+            assert np.all(err <= lim), ("d", t, j, float(np.max(err / lim)))
+
+
+@pytest.mark.parametrize("which", ["full", "mixed-small", "mixed-8bit", "wide"])
+def test_moe_stagewise(which):
+    from bit_hadamard_rotated_b200 import hq_moe_workspace_size
+    if which == "full":
+        m = synth.moe(seed=0)
+    elif which == "mixed-small":
+        m = synth.moe(seed=1, E=6, hidden=256, inter=128, T=5, k=2, probs=(0.4, 0.3, 0.3))
+    elif which == "mixed-8bit":
+        m = synth.moe(seed=5, E=7, hidden=512, inter=256, T=9, k=3, probs=(0.25, 0.25, 0.5),
+                      bits_choices=(2, 8, 4))
+    else:
+        m = synth.moe(seed=11, E=5, hidden=8192, inter=256, T=11, k=2, probs=(0.4, 0.3, 0.3))
+    E = len(m["experts"])
+    ws = torch.zeros(hq_moe_workspace_size(E, m["hidden"], m["inter"], m["T"], m["k"]),
+                     dtype=torch.uint8, device="cuda")
+    y, _ = run_moe(m, ws=ws)
+    _check_stages(m, ws)
+    want, bound, _ = oracle_moe(m)
+    check(y, want, bound, which)

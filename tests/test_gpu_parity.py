@@ -267,6 +267,14 @@ FULL = [
 ]
 
 
+# every (bits, batch) point of the bit-width-coverage workload, and the
+# M = K = 8192 roofline sweep at batches 1, 8, 16, 64, 128 for every width
+FULL += [(12288, 4096, b, n, "uniform", 0.0) for b in (2, 3, 8) for n in (1, 2, 4, 8)
+         if (12288, 4096, b, n, "uniform", 0.0) not in FULL]
+FULL += [(8192, 8192, b, n, "uniform", 0.0) for b in (2, 3, 4, 8) for n in (1, 8, 16, 64, 128)
+         if (8192, 8192, b, n, "uniform", 0.0) not in FULL]
+
+
 @pytest.mark.parametrize("M,K,bits,N,sd,of", FULL)
 def test_linear_parity_full_size_sampled(M, K, bits, N, sd, of):
     d = synth.linear(M, K, bits, N, seed=1, scale_dist=sd, outlier_frac=of)
@@ -277,3 +285,43 @@ def test_linear_parity_full_size_sampled(M, K, bits, N, sd, of):
                                     d["x"], m_begin=m, m_end=m + 1)
         assert_within(y[:, m], want[:, m], bound[:, m], what=f"row {m}")
     assert np.all(np.isfinite(y))
+
+
+# ---------------------------------------------------------------- small activation scales
+# The GEMV feeds the tensor cores x' * 2^-a in fp16 (a <= 8: the bit offset of
+# a code's field inside its 16-bit half), so small activations reach fp16's
+# subnormal range there first; the tensor-core path rounds x' itself to fp16.
+# The same tolerance holds at any scale.
+def _scaled(d, f):
+    x = (d["x"].astype(np.float64) * f).astype(np.float16)
+    return dict(d, x=x)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("N", [1, 2, 4, 16])
+@pytest.mark.parametrize("scale", [2.0**-10, 2.0**-14])
+def test_linear_small_activation_scales(bits, N, scale):
+    M, K = 300, 4096
+    d = _scaled(synth.linear(M, K, bits, N, seed=41 + bits + N), scale)
+    assert np.any(np.abs(d["x"].astype(np.float64)) < 2.0**-14) or scale > 2.0**-14
+    y = run_linear(d).cpu().numpy()
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert_within(y, want, bound, what=f"scale {scale} b{bits} N{N}")
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("N", [1, 3, 16])
+@pytest.mark.parametrize("c", [1.0, 2.0**-12])
+def test_linear_single_spike_null_signs(bits, N, c):
+    """x = c e_j (a different j per row) with signs = NULL: x' = c H[:, j] / sqrt(K),
+    every element +-c/sqrt(K), so y[n][m] = c sum_k w[m][k] H[k][j_n] / sqrt(K)."""
+    from bit_hadamard_rotated_b200 import hq_linear
+    M, K = 200, 8192
+    d = synth.linear(M, K, bits, N, seed=51 + bits)
+    x = np.zeros((N, K), np.float16)
+    for n in range(N):
+        x[n, (977 * n + 5) % K] = c
+    y = hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), None, dev(x), bits,
+                  d["zero"]).cpu().numpy()
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], None, x)
+    assert_within(y, want, bound, what=f"spike c={c} b{bits} N{N}")

@@ -312,6 +312,34 @@ def test_moe_identical_experts_reduce_to_one():
         assert np.allclose(y[t], want, rtol=1e-6, atol=1e-9)  # weights sum to 1 in fp32
 
 
+def test_moe_bound_base_for_several_slots():
+    """The MoE tolerance base, bound_t[i] = sum_j |topk_w[t][j]| sum_k |Wq_down[i][k] h'_k|,
+    rebuilt from dense numpy chains at k = 3 and 8 with some negative routing
+    weights (so a dropped |.| or a dropped weight changes it), to 1e-12."""
+    for seed, k in ((34, 3), (35, 8)):
+        m = _small_moe(seed, k=k, E=9)
+        w = m["topk_w"].copy()
+        w[:, 1] *= -1.0
+        y, b, _ = oracle.moe(m["experts"], m["hidden"], m["inter"], m["x"], m["topk_ids"], w,
+                             m["s_in"], m["s_mid"])
+        H = scipy.linalg.hadamard(m["inter"]).astype(np.float64)
+        for t in range(m["T"]):
+            want = np.zeros(m["hidden"])
+            want_y = np.zeros(m["hidden"])
+            for j in range(k):
+                e = m["experts"][int(m["topk_ids"][t, j])]
+                d, h = _dense_expert_chain(e, m["x"][t].astype(np.float64), m["s_in"], m["s_mid"],
+                                           m["hidden"], m["inter"])
+                hr = H @ (sign_vec(m["s_mid"], m["inter"]) * h) / np.sqrt(m["inter"])
+                Wq, _ = dense_weff(e["q_down"], e["s_down"], e["bits"], e["zero"], m["hidden"],
+                                   m["inter"], m["s_mid"])
+                want += abs(float(w[t, j])) * np.abs(Wq * hr[None, :]).sum(axis=1)
+                want_y += float(w[t, j]) * d
+            assert np.allclose(b[t], want, rtol=1e-12, atol=1e-14)
+            assert np.allclose(y[t], want_y, rtol=1e-11, atol=1e-12)
+            assert np.all(np.abs(y[t]) <= b[t] * (1 + 1e-12))
+
+
 # ---------------------------------------------------------------- routing inputs
 def test_routing_weights_and_ties():
     rng = np.random.default_rng(5)

@@ -27,7 +27,13 @@ def gpu():
 
 
 @pytest.mark.parametrize("M,K,bits,N", [(4096, 4096, 4, 1), (1000, 1024, 3, 3), (12288, 4096, 2, 8),
-                                         (257, 8192, 8, 2)])
+                                         (257, 8192, 8, 2),
+                                         # batches past one block of 8 columns: the blocks run
+                                         # in turn through the one scratch region, at offsets
+                                         # n0*K of x and n0*M of y; K = 16384 rotates in a
+                                         # separate kernel for every block
+                                         (257, 4096, 2, 11), (1000, 4096, 3, 17),
+                                         (257, 16384, 4, 20), (333, 2048, 8, 9)])
 def test_noalloc_matches_hq_linear_twice(M, K, bits, N):
     from bit_hadamard_rotated_b200 import _lib, hq_linear, make_weight
     d = synth.linear(M, K, bits, N, seed=M + K + bits)
@@ -49,6 +55,8 @@ def test_noalloc_matches_hq_linear_twice(M, K, bits, N):
         lim = REL * bound + ABS
         assert np.all(np.abs(got - ref) <= lim), (call, float(np.max(np.abs(got - ref) / lim)))
         assert np.all(np.abs(got - want) <= lim), (call, float(np.max(np.abs(got - want) / lim)))
+        st = _lib.lib().hq_linear_noalloc_check_status(stream)
+        assert st == 0, _lib.status_string(st)
 
 
 def test_noalloc_rejects_what_hq_linear_rejects():
