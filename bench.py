@@ -3,16 +3,19 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-One step = one pass of the hot path over one batch: the rotated linears of the
-bit-width-coverage workload (out 12288, in 4096, group-128 codes at 2, 3 and 8
-bits, zero point 2^(b-1), fp16 activations N(0,1), batch 1), each one call of
-the C ABI's hq_linear (rotation, unpack, dequantisation and contraction).
-Metric: effective weight GB/s = (packed-code + scale bytes) / time, whole job.
+One step = one pass of the hot path over one batch: the large dense MLP linear
+(out 28672, in 8192, 2-bit group-128 codes, zero point 2, fp16 scales
+log-uniform in [0.003, 0.03], fp16 activations N(0,1) with 1 % outlier
+channels x20, random signs) at batch 1, one call of the C ABI's hq_linear
+(rotation, unpack, dequantisation and contraction in one kernel).
+Metric: effective weight GB/s = (packed-code + scale bytes) / time, whole job;
+the same weights at batch 16 and 64 are reported in TFLOP/s beside it.
 
-Weights are cycled over enough distinct copies that every step reads HBM, not
-L2 (inputs larger than L2 between uses of a copy).  Steps are replayed from
-CUDA graphs and timed with CUDA events on the launching stream, bracketed by a
-barrier and a device synchronisation; the job time is the max over ranks.
+Weights are cycled over enough distinct copies that every call reads HBM, not
+L2 (inputs larger than L2 between uses of a copy).  The K timed calls are one
+CUDA graph (a few, past 2048 calls), so the time per call does not depend on K;
+CUDA events on the launching stream, a barrier and a device synchronisation
+on both sides; the job time is the max over ranks.
 
 Under torchrun every rank runs the same workload on its own GPU with its own
 weights (weak scaling); there is no collective on the data path.
@@ -39,9 +42,14 @@ from bit_hadamard_rotated_b200 import dist, synth  # noqa: E402
 METRIC = "rotated 2/3/4-bit linear: weight GB/s (% HBM peak) at B=1; TFLOP/s at B=64"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-WORKLOAD = "rotated linear M=12288 K=4096, bits 2/3/8, batch 1"
-LAYERS = [(12288, 4096, 2), (12288, 4096, 3), (12288, 4096, 8)]
-B64 = (28672, 8192, 2, 64)
+HEAD = (28672, 8192, 2)  # M, K, bits of the dense MLP linear
+WORKLOAD = "rotated dense MLP linear M=28672 K=8192, 2-bit group-128, batch 1"
+GRAPH_CALLS = 2048       # calls per captured graph at most
+# Files the GEMV kernel is built from: the ncu traffic figure in the profile
+# summary is reported only while their hash matches the one it was taken at.
+GEMV_SOURCES = ["gemv.cu", "fwht.cuh", "hq_common.cuh", "hq_internal.h", "hq_io.cuh",
+                "hq_launch.cuh", "hq_layout.cuh"]
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemv_kernel_28672x8192_b2_n1.md")
 
 
 def peaks():
@@ -104,33 +112,6 @@ class Clocks:
 
 
 # ---------------------------------------------------------------- workload
-def build_layers(device, copies, seed):
-    """copies x layers of packed weights; copy 0 from the seeded host generator,
-    the others drawn on the device from a seeded torch generator (same laws)."""
-    from bit_hadamard_rotated_b200 import RotatedLinear
-    gen = torch.Generator(device=device)
-    gen.manual_seed(seed)
-    base = [synth.linear(M, K, b, 1, seed=seed) for (M, K, b) in LAYERS]
-    xs = [torch.from_numpy(d["x"]).to(device) for d in base]
-    layers = []
-    for c in range(copies):
-        row = []
-        for d in base:
-            M, K, b = d["M"], d["K"], d["bits"]
-            if c == 0:
-                q = torch.from_numpy(d["q"].view(np.int32)).to(device)
-                sc = torch.from_numpy(d["scales"]).to(device)
-            else:
-                q = torch.randint(-2**31, 2**31 - 1, (M, K * b // 32), dtype=torch.int32,
-                                  device=device, generator=gen)
-                sc = (torch.rand((M, K // 128), device=device, generator=gen) * 0.015 + 0.005
-                      ).to(torch.float16)
-            s = torch.from_numpy(d["signs"]).to(device)
-            row.append(RotatedLinear(q, sc, s, b, d["zero"], max_batch=1))
-        layers.append(row)
-    return layers, xs
-
-
 def weight_bytes(M, K, b):
     return M * K * b // 8 + M * (K // 128) * 2
 
@@ -138,6 +119,100 @@ def weight_bytes(M, K, b):
 def algorithmic_bytes(M, K, b, N):
     """Bytes the linear must move at least once: codes, scales, signs, x, y."""
     return weight_bytes(M, K, b) + K + N * K * 2 + N * M * 4
+
+
+def gemv_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMV_SOURCES:
+        with open(os.path.join(ROOT, "bit_hadamard_rotated_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per launch of the batch-1 GEMV from the committed ncu summary,
+    or None if the summary is missing or the kernel's sources changed since."""
+    try:
+        txt = open(TRAFFIC_PROFILE).read()
+    except OSError:
+        return None, "no profile summary"
+    import re
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", txt)
+    s = re.search(r"source_sha16:\s*([0-9a-f]{16})", txt)
+    if not t or not s:
+        return None, "profile summary without traffic"
+    if s.group(1) != gemv_source_hash():
+        return None, "kernel changed since the profile"
+    return int(t.group(1)), os.path.relpath(TRAFFIC_PROFILE, ROOT)
+
+
+def head_copies(device, copies, seed):
+    """copies of the dense MLP linear's packed weights: copy 0 from the seeded
+    host generator, the others drawn on the device from a seeded torch
+    generator with the same laws (uniform code bits, log-uniform fp16 scales)."""
+    from bit_hadamard_rotated_b200 import RotatedLinear
+    M, K, b = HEAD
+    d = synth.linear(M, K, b, 64, seed=seed, scale_dist="loguniform", outlier_frac=0.01)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    signs = torch.from_numpy(d["signs"]).to(device)
+    lins = []
+    for c in range(copies):
+        if c == 0:
+            q = torch.from_numpy(d["q"].view(np.int32)).to(device)
+            sc = torch.from_numpy(d["scales"]).to(device)
+        else:
+            q = torch.randint(-2**31, 2**31 - 1, (M, K * b // 32), dtype=torch.int32, device=device,
+                              generator=gen)
+            u = torch.rand((M, K // 128), device=device, generator=gen, dtype=torch.float64)
+            sc = torch.exp(math.log(0.003) + u * (math.log(0.03) - math.log(0.003))).half()
+        lins.append(RotatedLinear(q, sc, signs, b, d["zero"], max_batch=64))
+    return lins, torch.from_numpy(d["x"]).to(device)
+
+
+def capture(stream, calls):
+    """One CUDA graph of the given calls back to back."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for c in calls:
+            c()
+    return g
+
+
+def timed_calls(stream, device, lins, x, y, steps, warmup, copies):
+    """Time `steps` calls (call i on weight copy i mod copies) replayed from
+    graphs of up to GRAPH_CALLS calls (a multiple of `copies`, so the cycle
+    continues across replays); returns (ms, graphs) after W warm-up calls."""
+    def calls(n, start=0):
+        return [lambda l=lins[(start + i) % copies]: l(x, out=y) for i in range(n)]
+
+    with torch.cuda.stream(stream):
+        for c in calls(max(warmup, 3)):
+            c()
+        if steps <= GRAPH_CALLS:
+            plan = [(capture(stream, calls(steps)), 1)]
+        else:
+            per = max(copies, GRAPH_CALLS // copies * copies)
+            plan = [(capture(stream, calls(per)), steps // per)]
+            if steps % per:
+                plan.append((capture(stream, calls(steps % per)), 1))
+        # warm-up replays of the captured graphs (uploads them, warms the clocks)
+        for g, _ in plan:
+            g.replay()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier(device)
+    torch.cuda.synchronize(device)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for g, reps in plan:
+            for _ in range(reps):
+                g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize(device)
+    dist.barrier(device)
+    return e0.elapsed_time(e1), plan
 
 
 def run_ours(a):
@@ -149,110 +224,62 @@ def run_ours(a):
     from bit_hadamard_rotated_b200 import _lib
     _lib.lib()  # fail loudly if the CUDA library is missing
 
+    M, K, b = HEAD
     props = torch.cuda.get_device_properties(device)
     l2 = getattr(props, "L2_cache_size", 126 * 2**20)
-    step_w = sum(weight_bytes(M, K, b) for (M, K, b) in LAYERS)
-    copies = max(2, math.ceil(4 * l2 / step_w))
-    layers, xs = build_layers(device, copies, seed=1234 + rank)
-    ys = [torch.empty((1, M), dtype=torch.float32, device=device) for (M, K, b) in LAYERS]
+    wb = weight_bytes(M, K, b)
+    copies = max(2, math.ceil(4 * l2 / wb))
+    lins, x64 = head_copies(device, copies, seed=77 + rank)
+    x1 = x64[:1].contiguous()
+    y1 = torch.empty((1, M), dtype=torch.float32, device=device)
     stream = torch.cuda.Stream(device)
+    pk = peaks()
 
-    def step(c):
-        for li in range(len(LAYERS)):
-            layers[c][li](xs[li], out=ys[li])
-
-    with torch.cuda.stream(stream):
-        for i in range(max(a.warmup, 3)):
-            step(i % copies)
-    torch.cuda.synchronize(device)
-    for row in layers:
-        for lin in row:
-            lin.check_status(stream)
-
-    # One graph per weight copy (one step each) and one block graph of `rep` rounds.
-    rep = 8
-    g1 = []
     n0 = hq.hq_launch_count()
     with torch.cuda.stream(stream):
-        for c in range(copies):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(c)
-            g1.append(g)
-        launches_per_step = (hq.hq_launch_count() - n0) // copies
-        gb = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(gb, stream=stream):
-            for _ in range(rep):
-                for c in range(copies):
-                    step(c)
-    block = rep * copies
-    for i in range(a.warmup):
-        with torch.cuda.stream(stream):
-            g1[i % copies].replay()
+        lins[0](x1, out=y1)
     torch.cuda.synchronize(device)
+    launches_per_step = hq.hq_launch_count() - n0
 
     clocks = Clocks(device)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    dist.barrier(device)
-    torch.cuda.synchronize(device)
     clocks.start()
     time.sleep(0.3)
-    with torch.cuda.stream(stream):
-        ev0.record(stream)
-        done = 0
-        while a.steps - done >= block:
-            gb.replay()
-            done += block
-        while done < a.steps:
-            g1[done % copies].replay()
-            done += 1
-        ev1.record(stream)
-    torch.cuda.synchronize(device)
+    ms, plan = timed_calls(stream, device, lins, x1, y1, a.steps, a.warmup, copies)
     ck = clocks.stop()
-    dist.barrier(device)
-    ms = ev0.elapsed_time(ev1)
+    del plan
     ms_max = dist.max_over_ranks(ms, device)
-    for row in layers:
-        for lin in row:
-            lin.check_status(stream)
+    for lin in lins:
+        lin.check_status(stream)
 
-    total_w = step_w * a.steps * world
-    value = total_w / (ms_max / 1e3) / 1e9
-    pk = peaks()
-    alg = sum(algorithmic_bytes(M, K, b, 1) for (M, K, b) in LAYERS)
+    value = wb * a.steps * world / (ms_max / 1e3) / 1e9
+    alg = algorithmic_bytes(M, K, b, 1)
     achieved = alg / ((ms / a.steps) / 1e3) / 1e9
+    traffic, traffic_src = profiled_traffic()
 
-    # per-bit-width breakdown (each layer's own graph, same protocol)
-    per_bits = {}
-    for li, (M, K, b) in enumerate(LAYERS):
-        gs = []
-        with torch.cuda.stream(stream):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for _ in range(rep):
-                    for c in range(copies):
-                        layers[c][li](xs[li], out=ys[li])
-            gs.append(g)
-            reps = max(1, 2000 // block)
-            g.replay()
-            torch.cuda.synchronize(device)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record(stream)
-            for _ in range(reps):
-                g.replay()
-            e1.record(stream)
-        torch.cuda.synchronize(device)
-        us = e0.elapsed_time(e1) * 1e3 / (reps * block)
-        per_bits[str(b)] = {"us_per_linear": round(us, 3),
-                            "weight_gbs": round(weight_bytes(M, K, b) / (us * 1e-6) / 1e9, 1),
-                            "frac_hbm": round(weight_bytes(M, K, b) / (us * 1e-6) / 1e9
-                                              / pk["hbm"], 4)}
+    # the same weights at batch 16 and 64 (tensor cores), back-to-back calls
+    big = {}
+    for n in (16, 64):
+        xn = x64[:n].contiguous()
+        yn = torch.empty((n, M), dtype=torch.float32, device=device)
+        reps = max(copies, 4 * copies)
+        ms_n, plan = timed_calls(stream, device, lins, xn, yn, reps, 3, copies)
+        del plan
+        ms_n = dist.max_over_ranks(ms_n, device)
+        us = ms_n * 1e3 / reps
+        tf = 2.0 * M * K * n / (us * 1e-6) / 1e12
+        big[f"b{n}"] = {"us_per_call": round(us, 3), "tflops": round(tf, 2),
+                        "frac_bf16_peak": round(tf / pk["bf16"], 4),
+                        "weight_gbs": round(wb / (us * 1e-6) / 1e9, 1),
+                        "frac_hbm": round(wb / (us * 1e-6) / 1e9 / pk["hbm"], 4),
+                        "path": "tensor cores" if lins[0].uses_tensor_cores(n) else "GEMV",
+                        "launches_per_call": lins[0].launches(n),
+                        "timing": f"{reps} back-to-back calls in one graph, {copies} weight "
+                                  f"copies cycled"}
 
-    b64 = measure_b64(device, stream, pk) if a.b64 else None
-    configs = measure_configs(device, stream, pk, l2) if a.b64 else None
-    e2e = measure_e2e(device, layers, xs, a)
+    configs = measure_configs(device, stream, pk, l2) if a.configs else None
+    e2e = measure_e2e(device, lins, x1, a, copies)
     e2e_ms = dist.max_over_ranks(e2e.pop("ms"), device)
-    e2e["value"] = round(step_w * e2e["steps"] * world / (e2e_ms * 1e-3) / 1e9, 3)
+    e2e["value"] = round(wb * e2e["steps"] * world / (e2e_ms * 1e-3) / 1e9, 3)
 
     cpu = None
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -262,22 +289,27 @@ def run_ours(a):
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": a.steps, "warmup": a.warmup, "ms_per_step": round(ms_max / a.steps, 6),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
-        "data": "synthetic (seeded; uniform codes, fp16 scales U[0.005,0.02], x ~ N(0,1))",
-        "config": {"workload": WORKLOAD, "layers": [f"{M}x{K} b{b}" for (M, K, b) in LAYERS],
-                   "batch": 1, "group": 128, "weight_bytes_per_step": step_w,
-                   "weight_copies": copies, "l2_bytes": l2,
-                   "l2_policy": f"{copies} weight copies cycled; {copies * step_w / 2**20:.0f} MiB "
+        "data": "synthetic (seeded; uniform 2-bit codes, fp16 scales log-uniform [0.003,0.03], "
+                "x ~ N(0,1) fp16 with 1% outlier channels x20)",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "bits": b, "batch": 1, "group": 128,
+                   "zero": 2, "weight_bytes_per_step": wb, "weight_copies": copies,
+                   "l2_bytes": l2,
+                   "l2_policy": f"{copies} weight copies cycled; {copies * wb / 2**20:.0f} MiB "
                                 f"> L2 between reuses of a copy",
+                   "timing": "the K calls replayed from one CUDA graph (graphs of up to "
+                             f"{GRAPH_CALLS} calls past that)",
                    "parallelism": f"replicas x{world} (weak scaling, no data-path collective)"},
         "frac_hbm": round(value / world / pk["hbm"], 4),
+        "tflops_b64": big["b64"]["tflops"],
+        "frac_bf16_b64": big["b64"]["frac_bf16_peak"],
+        "b16": big["b16"], "b64": big["b64"],
         "roofline": {"bound": "hbm",
-                     "kernel": "gemv_kernel, rotation fused in (one launch per linear at "
-                               "batch 1; aggregate over the step's three linears)",
+                     "kernel": "gemv_kernel<2, 13, 1> (rotation fused in; the step's only kernel)",
                      "achieved": round(achieved, 1), "peak": pk["hbm"], "unit": "GB/s",
-                     "frac": round(achieved / pk["hbm"], 4), "traffic": None,
-                     "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs)"},
-        "per_bits": per_bits,
-        "b64": b64,
+                     "frac": round(achieved / pk["hbm"], 4), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": alg,
+                     "traffic_source": traffic_src,
+                     "peak_source": pk["source"] + " (MEASURED_PEAKS.json hbm_gbs, copy)"},
         "configs": configs,
         "e2e": e2e,
         "gpu_launches": int(launches_per_step * a.steps),
@@ -287,51 +319,7 @@ def run_ours(a):
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del g1, gb
     dist.finish()
-
-
-def measure_b64(device, stream, pk):
-    """TFLOP/s of the large dense MLP linear (28672x8192, 2-bit) at batch 64 (and 16; batch 1
-    on the GEMV, weight GB/s)."""
-    from bit_hadamard_rotated_b200 import RotatedLinear
-    M, K, b, N = B64
-    d = synth.linear(M, K, b, N, seed=77, scale_dist="loguniform", outlier_frac=0.01)
-    lin = RotatedLinear(torch.from_numpy(d["q"].view(np.int32)).to(device),
-                        torch.from_numpy(d["scales"]).to(device),
-                        torch.from_numpy(d["signs"]).to(device), b, d["zero"], max_batch=N)
-    flush = torch.empty(2 * 126 * 2**20 // 4, dtype=torch.float32, device=device)
-    out = {}
-    for n in (N, 16, 1):
-        x = torch.from_numpy(np.ascontiguousarray(d["x"][:n])).to(device)
-        y = torch.empty((n, M), dtype=torch.float32, device=device)
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                lin(x, out=y)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                lin(x, out=y)
-            torch.cuda.synchronize(device)
-            times = []
-            for _ in range(20):
-                flush.zero_()  # L2 flush between timed calls (outside the timed interval)
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record(stream)
-                g.replay()
-                e1.record(stream)
-                torch.cuda.synchronize(device)
-                times.append(e0.elapsed_time(e1))
-        ms = statistics.median(times)
-        tflops = 2.0 * M * K * n / (ms * 1e-3) / 1e12
-        out[n] = {"ms": round(ms, 4), "tflops": round(tflops, 2),
-                  "frac_bf16_peak": round(tflops / pk["bf16"], 4),
-                  "weight_gbs": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9, 1),
-                  "frac_hbm": round(weight_bytes(M, K, b) / (ms * 1e-3) / 1e9 / pk["hbm"], 4),
-                  "launches": lin.launches(n)}
-    r = {"workload": f"rotated linear M={M} K={K} b{b} batch {N}", **out[N],
-         "timing": "CUDA-graph replay of one call, median of 20, L2 flushed before each",
-         "batch16": out[16], "batch1": out[1]}
-    return r
 
 
 def _graph_us(stream, device, calls, reps=5):
@@ -368,11 +356,11 @@ def _device_copies(device, M, K, b, n, gen):
 
 
 def measure_configs(device, stream, pk, l2):
-    """The other workloads of the metric: the 4096x4096 4-bit linear at batch 1,
-    the 256-expert MoE layer (32 tokens, top-8) and the M=K=8192 sweep over
-    widths and batches (GEMV up to batch 8, tensor cores from 16).  Weights are
-    cycled over enough copies that every call reads HBM; each point is the
-    median over 5 replays of a graph of back-to-back calls."""
+    """The other workloads: the 4096x4096 4-bit linear at batch 1, the bit-width
+    coverage linears (12288x4096 at 2, 3 and 8 bits, batch 1-8), the 256-expert
+    MoE layer (32 tokens, top-8) and the M=K=8192 sweep over widths and batches.
+    Weights are cycled over enough copies that every call reads HBM; each point
+    is the median over 5 replays of a graph of back-to-back calls."""
     from bit_hadamard_rotated_b200 import (RotatedLinear, expert_table, hq_moe_experts,
                                            hq_moe_workspace_size)
     gen = torch.Generator(device=device)
@@ -398,6 +386,8 @@ def measure_configs(device, stream, pk, l2):
         return r
 
     res["cfg_4096x4096_b4_n1"] = linear_point(4096, 4096, 4, 1)
+    res["cfg_12288x4096"] = {f"b{b}_n{n}": linear_point(12288, 4096, b, n)
+                             for b in (2, 3, 8) for n in (1, 2, 4, 8)}
 
     # MoE layer: two copies of the expert weights, alternated, so calls read HBM
     m = synth.moe(seed=1)
@@ -494,38 +484,27 @@ class _Rt:
             raise RuntimeError("cudaStreamWaitEvent failed")
 
 
-def measure_e2e(device, layers, xs, a):
+def measure_e2e(device, lins, x1, a, copies):
     """Same metric through the public Python API with host buffers: every step
-    copies the step's activations (the three layers' inputs, one pinned host
-    buffer) to the device in one copy, runs the layers (RotatedLinear launchers
-    prepared once on their buffers, each call one hq_linear call), and reads
-    their outputs back to a pinned host buffer in one copy, all inside the timed
-    region.  The copies run on two copy streams, double-buffered, so step
-    i + 1's upload and step i's download overlap the layers of the neighbouring
-    steps (a serving loop's pipelining); every step moves its own bytes both
-    ways."""
-    copies = len(layers)
-    xsz = [x.numel() for x in xs]
-    ysz = [M for (M, K, b) in LAYERS]
-    xh = torch.cat([x.reshape(-1).cpu() for x in xs]).pin_memory()
+    copies the step's activations from a pinned host buffer to the device, runs
+    the layer (a RotatedLinear launcher prepared once on its buffers: one
+    hq_linear call), and reads its output back to a pinned host buffer, all
+    inside the timed region.  The copies run on two copy streams,
+    double-buffered, so step i + 1's upload and step i's download overlap the
+    neighbouring steps' layer calls (a serving loop's pipelining); every step
+    moves its own bytes both ways."""
+    M = lins[0].M
+    xh = x1.reshape(-1).cpu().pin_memory()
     NB = 2  # buffer sets in flight
     xd = [torch.empty_like(xh, device=device) for _ in range(NB)]
-    yd = [torch.empty(sum(ysz), dtype=torch.float32, device=device) for _ in range(NB)]
-    yh = [torch.empty(sum(ysz), dtype=torch.float32).pin_memory() for _ in range(NB)]
+    yd = [torch.empty(M, dtype=torch.float32, device=device) for _ in range(NB)]
+    yh = [torch.empty(M, dtype=torch.float32).pin_memory() for _ in range(NB)]
     comp = torch.cuda.current_stream(device)
     up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    launch = []  # [copy][buffer set] -> the three layers' launchers
+    launch = []  # [copy][buffer set] -> the layer's launcher
     for c in range(copies):
-        per_b = []
-        for b in range(NB):
-            fns, ox, oy = [], 0, 0
-            for li, (M, _K, _b) in enumerate(LAYERS):
-                fns.append(layers[c][li].prepare(xd[b][ox:ox + xsz[li]].view(1, -1),
-                                                 yd[b][oy:oy + M].view(1, -1), stream=comp))
-                ox += xsz[li]
-                oy += M
-            per_b.append(fns)
-        launch.append(per_b)
+        launch.append([[lins[c].prepare(xd[b].view(1, -1), yd[b].view(1, -1), stream=comp)]
+                       for b in range(NB)])
     steps = min(a.steps, 2000)
     rt = _Rt()
     x_in, y_out, y_read = ([rt.event() for _ in range(NB)] for _ in range(3))
@@ -570,34 +549,34 @@ def measure_e2e(device, layers, xs, a):
     ms = e0.elapsed_time(e1)
     return {"ms": ms, "value": None, "unit": "GB/s", "steps": steps,
             "h2d_bytes_per_step": int(xh.numel() * 2), "d2h_bytes_per_step": int(yh[0].numel() * 4),
-            "api": "RotatedLinear.prepare launchers -> hq_linear (C ABI), eager, one call per "
-                   "layer per step; one H2D and one D2H copy per step on two copy streams, "
-                   "double-buffered against the layers" +
+            "api": "RotatedLinear.prepare launcher -> hq_linear (C ABI), eager, one call per "
+                   "step; one H2D and one D2H copy per step on two copy streams, "
+                   "double-buffered against the layer calls" +
                    ("" if rt.rt is not None else " (tensor-level copies)")}
 
 
 # ---------------------------------------------------------------- CPU oracle baseline
 def cpu_baseline(seconds: float):
     """The fp64 oracle as it stands, on this host's cores (rows split across
-    threads), over a bounded sample: whole passes over the workload's three
-    layers at batch 1, repeated until about `seconds` of wall time."""
+    threads), over a bounded sample: whole passes over the workload's linear at
+    batch 1, repeated until about `seconds` of wall time."""
     import oracle
     cores = os.cpu_count() or 1
-    ds = [synth.linear(M, K, b, 1, seed=99) for (M, K, b) in LAYERS]
+    M, K, b = HEAD
+    d = synth.linear(M, K, b, 1, seed=99, scale_dist="loguniform", outlier_frac=0.01)
     passes = 0
     t0 = time.perf_counter()
     while True:
-        for d in ds:
-            oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
-                          d["x"], threads=cores)
+        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                      d["x"], threads=cores)
         passes += 1
         dt = time.perf_counter() - t0
         if dt >= seconds:
             break
-    wb = passes * sum(weight_bytes(M, K, b) for (M, K, b) in LAYERS)
+    wb = passes * weight_bytes(M, K, b)
     return {"value": round(wb / dt / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{passes} full passes over the 3 layers (12288x4096 at b2, b3, b8), "
-                      f"batch 1, {dt:.1f} s wall on {cores} threads"}
+            "sample": f"{passes} full passes over the {M}x{K} 2-bit linear, batch 1, "
+                      f"{dt:.1f} s wall on {cores} threads"}
 
 
 def run_reference(a):
@@ -606,21 +585,20 @@ def run_reference(a):
         return
     import oracle
     cores = os.cpu_count() or 1
-    ds = [synth.linear(M, K, b, 1, seed=99) for (M, K, b) in LAYERS]
+    M, K, b = HEAD
+    d = synth.linear(M, K, b, 1, seed=99, scale_dist="loguniform", outlier_frac=0.01)
     rows = a.ref_rows
     for _ in range(max(a.warmup, 0)):
-        for d in ds:
-            oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
-                          d["x"], 0, rows, threads=cores)
+        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                      d["x"], 0, rows, threads=cores)
     t0 = time.perf_counter()
     for _ in range(a.steps):
-        for d in ds:
-            oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
-                          d["x"], 0, rows, threads=cores)
+        oracle.linear(d["bits"], d["M"], d["K"], d["zero"], d["q"], d["scales"], d["signs"],
+                      d["x"], 0, rows, threads=cores)
     dt = time.perf_counter() - t0
-    wb = a.steps * sum(rows * (K * b // 8 + (K // 128) * 2) for (M, K, b) in LAYERS)
+    wb = a.steps * rows * (K * b // 8 + (K // 128) * 2)
     v = wb / dt / 1e9
-    sample = f"each step: first {rows} of 12288 rows of each layer (b2, b3, b8), batch 1"
+    sample = f"each step: the first {rows} of {M} rows of the {M}x{K} 2-bit linear, batch 1"
     print(json.dumps({
         "impl": "reference", "metric": METRIC, "value": round(v, 5), "unit": "GB/s",
         "n_gpus": world, "steps": a.steps, "warmup": a.warmup,
@@ -640,10 +618,11 @@ def main():
     ap.add_argument("--steps", type=int, default=20000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--no-b64", dest="b64", action="store_false")
+    ap.add_argument("--no-configs", dest="configs", action="store_false",
+                    help="skip the side workloads (other shapes, widths, the MoE layer)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--ref-rows", type=int, default=256)
+    ap.add_argument("--ref-rows", type=int, default=512)
     a = ap.parse_args()
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -35,11 +35,22 @@ struct FwhtShape {
 
 __device__ __forceinline__ int fwht_pad(int i) { return i + (i >> 5); }
 
+// Largest |value| held by the lanes of a warp (every lane gets it).
+__device__ __forceinline__ float warp_absmax(float m) {
+#pragma unroll
+  for (int s = 16; s >= 1; s >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, s));
+  return m;
+}
+
 // On entry thread tid = 32*w + l < THREADS holds v[e] = u[tid*E + e].  On exit
 // the transformed (unnormalised) row is in buf[fwht_pad(i)], i in [0, K), and
-// the block has synchronised.  Every thread of the block must call this.
+// the block has synchronised.  With red != nullptr, red[w] (w < W) also holds
+// the largest |value| of the part of the row warp w wrote last, so the row's
+// largest |value| is the max of red[0..W).  Every thread of the block must
+// call this.
 template <int LOGK, int LOGW_MAX>
-__device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>::E], float* buf) {
+__device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>::E], float* buf,
+                                           float* red = nullptr) {
   using S = FwhtShape<LOGK, LOGW_MAX>;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -68,6 +79,15 @@ __device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>:
     }
 #pragma unroll
     for (int e = 0; e < S::E; ++e) buf[fwht_pad(tid * S::E + e)] = v[e];
+    if constexpr (S::W == 1) {
+      if (red != nullptr) {
+        float m = 0.f;
+#pragma unroll
+        for (int e = 0; e < S::E; ++e) m = fmaxf(m, fabsf(v[e]));
+        m = warp_absmax(m);
+        if (lane == 0) red[tid >> 5] = m;
+      }
+    }
   }
   __syncthreads();
   if constexpr (S::W > 1) {
@@ -95,6 +115,15 @@ __device__ __forceinline__ void fwht_block(float (&v)[FwhtShape<LOGK, LOGW_MAX>:
       for (int j = 0; j < S::C; ++j)
 #pragma unroll
         for (int w = 0; w < S::W; ++w) buf[fwht_pad(w * 32 * S::E + tid * S::C + j)] = r[j][w];
+      if (red != nullptr) {
+        float m = 0.f;
+#pragma unroll
+        for (int j = 0; j < S::C; ++j)
+#pragma unroll
+          for (int w = 0; w < S::W; ++w) m = fmaxf(m, fabsf(r[j][w]));
+        m = warp_absmax(m);
+        if (lane == 0) red[tid >> 5] = m;
+      }
     }
     __syncthreads();
   }
@@ -118,9 +147,11 @@ struct Fwht512 {
 
 // On entry thread tid (of 512) holds v[e] = u[tid*E + e]; on exit the
 // transformed (unnormalised) row is in buf[fwht_pad(i)] and the block has
-// synchronised.  Every thread of the block must call this.
+// synchronised; with red != nullptr, red[w] (w < 16) holds the largest
+// |value| written by warp w.  Every thread of the block must call this.
 template <int LOGK>
-__device__ __forceinline__ void fwht_block512(float (&v)[Fwht512<LOGK>::E], float* buf) {
+__device__ __forceinline__ void fwht_block512(float (&v)[Fwht512<LOGK>::E], float* buf,
+                                              float* red = nullptr) {
   using S = Fwht512<LOGK>;
   constexpr int E = S::E, T = S::T;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -173,7 +204,37 @@ __device__ __forceinline__ void fwht_block512(float (&v)[Fwht512<LOGK>::E], floa
   }
 #pragma unroll
   for (int i = 0; i < E; ++i) buf[fwht_pad((h * E + i) * 32 * E + col)] = r[i];
+  if (red != nullptr) {
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < E; ++i) m = fmaxf(m, fabsf(r[i]));
+    m = warp_absmax(m);
+    if (lane == 0) red[tid >> 5] = m;
+  }
   __syncthreads();
 }
+
+// Largest of red[0..n) (the per-warp maxima the transforms above leave).
+__device__ __forceinline__ float red_max(const float* red, int n) {
+  float m = 0.f;
+  for (int i = 0; i < n; ++i) m = fmaxf(m, red[i]);
+  return m;
+}
+
+// Power-of-two exponent e for a row whose largest |x'| is m: x' * 2^e has its
+// largest magnitude in (2^13, 2^14], so when x' is rounded to fp16 (and, in
+// the GEMV, scaled down by up to 2^-8 more) every element within 2^-20 of the
+// largest stays in fp16's normal range, whatever the scale of the input.  The
+// product is undone exactly at the output (times 2^-e).  Rows of zeros (or
+// with an inf or NaN) keep e = 0; e is clamped to [-30, 60].
+__device__ __forceinline__ int row_scale_exp(float m) {
+  if (!(m > 0.f) || !(m < 3.0e38f)) return 0;
+  const int be = (__float_as_int(m) >> 23) & 0xff;  // m < 2^(be - 126)
+  const int e = be == 0 ? 60 : 140 - be;
+  return e < -30 ? -30 : (e > 60 ? 60 : e);
+}
+
+// 2^n as a float, -126 <= n <= 127.
+__device__ __forceinline__ float pow2f(int n) { return __int_as_float((127 + n) << 23); }
 
 }  // namespace hq

@@ -2,10 +2,13 @@
 //   y[n][m] = sum_k scale[m][k/128] (q[m][k] - zero) x'[n][k],  N >= 9.
 // At batch 16..256 the contraction is a dense one, so it runs on the
 // 5th-generation tensor cores with the fp32 accumulator in tensor memory:
-//   * a prep kernel rotates x (fp32 butterflies) and writes x' as fp16 in the
-//     k order of the decoded code pairs (hq_layout.cuh), so that A and B agree,
-//     already in the shared-memory image the MMA reads (no-swizzle K-major
-//     core matrices), one contiguous block per 128-code group;
+//   * a prep kernel rotates x (fp32 butterflies) and writes x' 2^e as fp16 in
+//     the k order of the decoded code pairs (hq_layout.cuh), so that A and B
+//     agree, already in the shared-memory image the MMA reads (no-swizzle
+//     K-major core matrices), one contiguous block per 128-code group; 2^e is
+//     a power of two per batch row that puts the row's largest |x'| just
+//     below 2^14 (small activations stay out of fp16's subnormal range), and
+//     the epilogue multiplies that output column by 2^-e, exactly;
 //   * per CTA, an equal contiguous range of (128-row tile, 128-code group)
 //     chunks (stream-K; the first and last tile may be shared with the
 //     neighbouring CTA), streamed through two rings by two producer threads:
@@ -204,13 +207,15 @@ __host__ __device__ constexpr size_t img_offset(int g, int i, int n, int npad) {
 // b*nb .. b*nb + nb - 1 of x); rows past the batch but inside the block's
 // 32-row padding are written as zeros, the rest of the CTAs exit at once.
 // Image of block b at byte b * K * 2 * nb of xp.  Position i of group g holds
-// x'[128 g + 32 t + code(p, h)] with i = 32 t + 2 p + h.
+// x'[128 g + 32 t + code(p, h)] 2^e with i = 32 t + 2 p + h; fac[b nb + j] =
+// 2^-e, the row's output factor (1 for padding rows).
 template <int BITS, int LOGK>
 __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
     tc_prep_kernel(const __half* __restrict__ x, const int8_t* __restrict__ signs,
-                   uint8_t* __restrict__ xp, int N, int nb, float inv) {
+                   uint8_t* __restrict__ xp, float* __restrict__ fac, int N, int nb, float inv) {
   using S = FwhtShape<LOGK>;
   extern __shared__ float buf[];
+  float* red = buf + S::SMEM_FLOATS;  // per-warp maxima of the transform
   pdl_launch_dependents();
   const int j = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int rows = min(nb, N - b * nb);
@@ -220,11 +225,17 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   pdl_wait();
   uint8_t* img = xp + static_cast<size_t>(b) * S::K * 2 * nb;
   const int n = b * nb + j;
+  float sc = 0.f;
   if (j < rows) {
     float v[S::E];
     load_chunk<__half, S::E>(x + static_cast<size_t>(n) * S::K + tid * S::E, v);
     flip_signs<S::E>(neg, v);
-    fwht_block<LOGK, 5>(v, buf);
+    fwht_block<LOGK, 5>(v, buf, red);
+    const int e = row_scale_exp(red_max(red, S::W) * inv);
+    sc = inv * pow2f(e);
+    if (tid == 0) fac[b * nb + j] = pow2f(-e);
+  } else if (tid == 0) {
+    fac[b * nb + j] = 1.f;
   }
   for (int seg = tid; seg < S::K / 8; seg += S::THREADS) {
     const int g = seg >> 4, i0 = (seg * 8) & 127;
@@ -235,8 +246,8 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
       for (int q = 0; q < 4; ++q) {
         const PairDesc pd = Pairs<BITS>::get(((i0 >> 1) & 15) + q);
         const int k0 = kGroup * g + 32 * t;
-        const __half lo = __float2half_rn(buf[fwht_pad(k0 + pd.c_lo)] * inv);
-        const __half hi = __float2half_rn(buf[fwht_pad(k0 + pd.c_hi)] * inv);
+        const __half lo = __float2half_rn(buf[fwht_pad(k0 + pd.c_lo)] * sc);
+        const __half hi = __float2half_rn(buf[fwht_pad(k0 + pd.c_hi)] * sc);
         w[q] = static_cast<uint32_t>(__half_as_ushort(lo)) |
                (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);
       }
@@ -250,6 +261,7 @@ struct TcParams {
   CUtensorMap qmap;       // packed codes [M][K bits / 8] as bytes; box 16 bits x 128 rows
   const uint8_t* scales;  // fp16 [M][K/128]
   const uint8_t* img;     // this batch block's x' image (G blocks of 256 Npad bytes)
+  const float* fac;       // this batch block's output factors 2^-e per column [Npad]
   float* y;               // this batch block's first output row
   uint32_t* status;
   int M, K, N, Npad, ldy;
@@ -323,10 +335,19 @@ __device__ __forceinline__ void tc_epilogue(const TcParams& p, uint32_t tmem, ui
     const int m = (tile0 + ti) * kTileM + r;
     auto store16 = [&](int c0, const float (&acc)[16]) {
       if (m < p.M) {
+        float f[16];  // the columns' output factors (the same for every thread)
+#pragma unroll
+        for (int i = 0; i < 16; i += 4) {
+          const float4 q = __ldg(reinterpret_cast<const float4*>(p.fac + c0 + i));
+          f[i] = q.x;
+          f[i + 1] = q.y;
+          f[i + 2] = q.z;
+          f[i + 3] = q.w;
+        }
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const int n = c0 + i;
-          if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i];
+          if (n < p.N) p.y[static_cast<size_t>(n) * p.ldy + m] = acc[i] * f[i];
         }
       }
     };
@@ -814,7 +835,7 @@ cudaError_t tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const voi
 int tc_col_block(int bits, int K) {
   // K >= 1024: whole 16-byte scale rows, and >= 8 groups per tile (a tile's
   // scale buffer is refilled only after the MMAs two tiles back are done)
-  if (K < 1024 || K > 16384) return 0;
+  if (K < 1024 || K > 32768) return 0;
   for (int nb = 128; nb >= 32; nb -= 32) {
     if (tc::tc_plan(bits, K, nb).smem != 0) return nb;
   }
@@ -822,14 +843,17 @@ int tc_col_block(int bits, int K) {
 }
 
 // [images of the batch blocks][shared tiles' partial sums: kMaxTcGrid
-// boundaries x 2 sides x 128 rows x nb columns fp32]
+// boundaries x 2 sides x 128 rows x nb columns fp32][output factors: nb per
+// batch block, fp32]
 static size_t tc_img_bytes(int nb, int K, int batch) {
   return (static_cast<size_t>((batch + nb - 1) / nb) * nb * K * 2 + 255) & ~static_cast<size_t>(255);
 }
+static size_t tc_part_bytes(int nb) { return static_cast<size_t>(kMaxTcGrid) * 2 * tc::kTileM * nb * 4; }
 size_t tc_xp_bytes(int bits, int K, int batch) {
   const int nb = tc_col_block(bits, K);
   if (nb == 0) return 0;
-  return tc_img_bytes(nb, K, batch) + static_cast<size_t>(kMaxTcGrid) * 2 * tc::kTileM * nb * 4;
+  return tc_img_bytes(nb, K, batch) + tc_part_bytes(nb) +
+         ((static_cast<size_t>((batch + nb - 1) / nb) * nb * 4 + 255) & ~static_cast<size_t>(255));
 }
 
 int tc_launches(int bits, int K, int batch) {
@@ -838,24 +862,25 @@ int tc_launches(int bits, int K, int batch) {
 }
 
 template <int BITS, int LOGK>
-static cudaError_t tc_prep_t(const __half* x, const int8_t* s, uint8_t* xp, int N, int nb,
-                             cudaStream_t st) {
+static cudaError_t tc_prep_t(const __half* x, const int8_t* s, uint8_t* xp, float* fac, int N,
+                             int nb, cudaStream_t st) {
   using S = FwhtShape<LOGK>;
   const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(S::K)));
   const dim3 grid(nb, (N + nb - 1) / nb);
   return launch_pdl(tc::tc_prep_kernel<BITS, LOGK>, grid, dim3(S::THREADS),
-                    S::SMEM_FLOATS * sizeof(float), st, true, x, s, xp, N, nb, inv);
+                    (S::SMEM_FLOATS + 32) * sizeof(float), st, true, x, s, xp, fac, N, nb, inv);
 }
 
 template <int BITS>
-static cudaError_t tc_prep_b(int K, const __half* x, const int8_t* s, uint8_t* xp, int N, int nb,
-                             cudaStream_t st) {
+static cudaError_t tc_prep_b(int K, const __half* x, const int8_t* s, uint8_t* xp, float* fac, int N,
+                             int nb, cudaStream_t st) {
   switch (K) {
-    case 1024: return tc_prep_t<BITS, 10>(x, s, xp, N, nb, st);
-    case 2048: return tc_prep_t<BITS, 11>(x, s, xp, N, nb, st);
-    case 4096: return tc_prep_t<BITS, 12>(x, s, xp, N, nb, st);
-    case 8192: return tc_prep_t<BITS, 13>(x, s, xp, N, nb, st);
-    case 16384: return tc_prep_t<BITS, 14>(x, s, xp, N, nb, st);
+    case 1024: return tc_prep_t<BITS, 10>(x, s, xp, fac, N, nb, st);
+    case 2048: return tc_prep_t<BITS, 11>(x, s, xp, fac, N, nb, st);
+    case 4096: return tc_prep_t<BITS, 12>(x, s, xp, fac, N, nb, st);
+    case 8192: return tc_prep_t<BITS, 13>(x, s, xp, fac, N, nb, st);
+    case 16384: return tc_prep_t<BITS, 14>(x, s, xp, fac, N, nb, st);
+    case 32768: return tc_prep_t<BITS, 15>(x, s, xp, fac, N, nb, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -870,12 +895,13 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
   if (nb == 0) return cudaErrorInvalidValue;
   uint8_t* xp = static_cast<uint8_t*>(a.xp);
   const __half* xh = reinterpret_cast<const __half*>(a.x);
+  float* fac = reinterpret_cast<float*>(xp + tc_img_bytes(nb, a.K, a.N) + tc_part_bytes(nb));
   cudaError_t e;
   switch (a.bits) {
-    case 2: e = tc_prep_b<2>(a.K, xh, a.signs, xp, a.N, nb, st); break;
-    case 3: e = tc_prep_b<3>(a.K, xh, a.signs, xp, a.N, nb, st); break;
-    case 4: e = tc_prep_b<4>(a.K, xh, a.signs, xp, a.N, nb, st); break;
-    case 8: e = tc_prep_b<8>(a.K, xh, a.signs, xp, a.N, nb, st); break;
+    case 2: e = tc_prep_b<2>(a.K, xh, a.signs, xp, fac, a.N, nb, st); break;
+    case 3: e = tc_prep_b<3>(a.K, xh, a.signs, xp, fac, a.N, nb, st); break;
+    case 4: e = tc_prep_b<4>(a.K, xh, a.signs, xp, fac, a.N, nb, st); break;
+    case 8: e = tc_prep_b<8>(a.K, xh, a.signs, xp, fac, a.N, nb, st); break;
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
@@ -897,6 +923,7 @@ cudaError_t launch_linear_tc(const TcArgs& a, cudaStream_t st) {
     p.qmap = qmap;
     p.scales = reinterpret_cast<const uint8_t*>(a.scales);
     p.img = xp + static_cast<size_t>(b) * a.K * 2 * nb;
+    p.fac = fac + static_cast<size_t>(b) * nb;
     p.y = a.y + static_cast<size_t>(n0) * a.ldy;
     p.status = a.status;
     p.M = a.M;

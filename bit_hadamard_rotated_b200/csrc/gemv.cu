@@ -11,8 +11,11 @@
 //
 //   * The rotation x' = H diag(s) x / sqrt(K) runs in fp32 (fwht.cuh), and x'
 //     is written as fp16 in the order of the MMA B fragments, each value
-//     scaled by the 2^-a of its code field (hq_layout.cuh), plus the
-//     zero-point term -zero * sum_k x'_k * 2^-24 of each group: for one or
+//     scaled by the 2^-a of its code field (hq_layout.cuh) and by a power of
+//     two 2^e of its row that puts the row's largest |x'| just below 2^14
+//     (so small activations do not fall into fp16's subnormal range; the
+//     output is multiplied by 2^(24-e), exactly), plus the zero-point term
+//     -zero * sum_k x'_k * 2^(e-24) of each group: for one or
 //     two rows of K <= 8192 by every GEMV CTA itself, after its first weight
 //     copies are on their way (one launch per call); otherwise by
 //     gemv_prep_kernel (one CTA per batch row) before the GEMV.
@@ -45,13 +48,18 @@
 namespace hq {
 
 constexpr int kWarps = 16;
-constexpr int kPrepWarps = 8;  // the FWHT uses at most 8 warps for K <= 8192
+// Warps of the prep kernel: its FWHT uses at most 8 for K <= 16384 (64 values
+// per thread at K = 16384), and 32 for K = 32768 (32 values per thread).
+__host__ __device__ constexpr int prep_warps(int logk) { return logk >= 15 ? 32 : 8; }
+__host__ __device__ constexpr int prep_logw(int logk) { return logk >= 15 ? 5 : 3; }
 constexpr int kRows = 16;
 // halves per (group, column, k-quad) block of B fragments: 8 steps x 4, padded
 // to 80 bytes so the 16-byte loads of 8 lanes hit distinct banks
 constexpr int kXq = 40;
-// 2^24: undoes, at the stores, the 2^-24 unit of the subnormal fp16 codes
-constexpr float kUnit = 16777216.f;
+// Shared memory after a batch block's zero-point terms: a zero B block (16
+// floats), the per-column output factors 2^(24 - e) (8 floats), the FWHT's
+// per-warp maxima (16 floats).
+constexpr int kZcTail = 64 + 32 + 64;
 
 struct GemvParams {
   CUtensorMap qmap;  // codes as bytes [M][K bits / 8]; box 16 bits bytes x 16 rows
@@ -67,7 +75,7 @@ struct GemvParams {
   uint32_t U;       // units = n_tiles * G
   uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
   int zero;
-  const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, then zc [G][8] fp32
+  const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, zc [G][8] fp32, fac [8] fp32
   float inv_sqrt_k;
   int CH, NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
 };
@@ -77,12 +85,13 @@ struct GemvParams {
 // overlaps the first weight copies.
 __host__ __device__ constexpr bool gemv_fused_rotation(int K, int nb) { return nb <= 2 && K <= 8192; }
 
-// Bytes of the prep output for a batch block of nb columns (16-byte multiple).
+// Bytes of the prep output for a batch block of nb columns (16-byte multiple):
+// the fragments, the zero-point terms [G][8] and the output factors [8].
 __host__ __device__ constexpr size_t gemv_xs_bytes(int G, int nb) {
   return static_cast<size_t>(G) * nb * 4 * kXq * 2;
 }
 __host__ __device__ constexpr size_t gemv_xg_bytes(int G, int nb) {
-  return gemv_xs_bytes(G, nb) + static_cast<size_t>(G) * 8 * 4;
+  return gemv_xs_bytes(G, nb) + static_cast<size_t>(G) * 8 * 4 + 8 * 4;
 }
 
 // ---------------------------------------------------------------- rotation -> B fragments
@@ -102,20 +111,21 @@ struct FragLane {
   }
 };
 
-// Group gg of a rotated row (buf: unnormalised fwht_block output): x' rounded
-// to fp16, each value scaled by the 2^-a of its code field, written as column
-// n of the fragment blocks xs [G][nb][4][kXq]; zc[gg * 8 + n] = the zero-point
-// term -zero * sum_k x'_k * 2^-24 of the group.  One warp per group.
+// Group gg of a rotated row (buf: unnormalised fwht_block output): x' 2^e
+// rounded to fp16 (sc = 2^e / sqrt(K)), each value scaled by the 2^-a of its
+// code field, written as column n of the fragment blocks xs [G][nb][4][kXq];
+// zc[gg * 8 + n] = the zero-point term -zero * sum_k x'_k * 2^(e-24) of the
+// group.  One warp per group.
 template <int BITS>
 __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float* buf, int gg, int n,
-                                          int nb, float inv_sqrt_k, int zero, uint16_t* xs,
+                                          int nb, float sc, int zero, uint16_t* xs,
                                           float* zc, int lane) {
   const int s = lane >> 2, t = lane & 3;
   uint16_t hv[4];
   float part = 0.f;
 #pragma unroll
   for (int r = 0; r < 4; ++r) {
-    const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + fl.kc[r])] * inv_sqrt_k));
+    const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + fl.kc[r])] * sc));
     const __half b = __float2half_rn(xv * __int_as_float((127 - fl.ka[r]) << 23));
     hv[r] = __half_as_ushort(b);
     part += __half2float(b) * __int_as_float((127 + fl.ka[r]) << 23);
@@ -130,15 +140,16 @@ __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float*
 }
 
 // Prep kernel (batches the GEMV CTAs do not rotate themselves): CTA n rotates
-// activation row n in fp32 and writes its fragments and zero-point terms to
-// global memory; CTA 0 also zeroes the zero-point terms of the absent columns
-// (N..7).
+// activation row n in fp32 and writes its fragments, zero-point terms and
+// output factor to global memory; CTA 0 also zeroes the zero-point terms of
+// the absent columns (N..7).
 template <int BITS, int LOGK>
-__global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half* __restrict__ x,
+__global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const __half* __restrict__ x,
                                                                  const int8_t* __restrict__ signs,
                                                                  uint8_t* __restrict__ xg, int N,
                                                                  int zero, float inv_sqrt_k) {
-  using FS = FwhtShape<LOGK, 3>;
+  using FS = FwhtShape<LOGK, prep_logw(LOGK)>;
+  constexpr int kPrepWarps = prep_warps(LOGK);
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
   extern __shared__ __align__(128) float buf[];
@@ -147,6 +158,7 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
   const int n = blockIdx.x;
   uint16_t* xs = reinterpret_cast<uint16_t*>(xg);
   float* zc = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
+  float* red = buf + FS::SMEM_FLOATS;  // per-warp maxima of the transform
   const FragLane<BITS> fl(lane);
   const SignMask<FS::E> neg =
       tid < FS::THREADS ? sign_bits<FS::E>(signs ? signs + tid * FS::E : nullptr) : 0u;
@@ -159,8 +171,11 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(const __half
     load_chunk<__half, FS::E>(x + static_cast<size_t>(n) * K + tid * FS::E, v);
     flip_signs<FS::E>(neg, v);
   }
-  fwht_block<LOGK, 3>(v, buf);
-  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, inv_sqrt_k, zero, xs, zc, lane);
+  fwht_block<LOGK, prep_logw(LOGK)>(v, buf, red);
+  const int e = row_scale_exp(red_max(red, FS::W) * inv_sqrt_k);
+  if (tid == 0) zc[G * 8 + n] = pow2f(24 - e);
+  const float sc = inv_sqrt_k * pow2f(e);
+  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, sc, zero, xs, zc, lane);
 }
 
 // The FWHT a fused GEMV CTA (16 warps) runs on one row: the 512-thread shape
@@ -170,12 +185,16 @@ struct FusedFwht;
 template <int LOGK>
 struct FusedFwht<LOGK, true> {
   static constexpr int E = Fwht512<LOGK>::E, THREADS = 512;
-  static __device__ __forceinline__ void run(float (&v)[E], float* buf) { fwht_block512<LOGK>(v, buf); }
+  static __device__ __forceinline__ void run(float (&v)[E], float* buf, float* red) {
+    fwht_block512<LOGK>(v, buf, red);
+  }
 };
 template <int LOGK>
 struct FusedFwht<LOGK, false> {
   static constexpr int E = FwhtShape<LOGK, 3>::E, THREADS = FwhtShape<LOGK, 3>::THREADS;
-  static __device__ __forceinline__ void run(float (&v)[E], float* buf) { fwht_block<LOGK, 3>(v, buf); }
+  static __device__ __forceinline__ void run(float (&v)[E], float* buf, float* red) {
+    fwht_block<LOGK, prep_logw(LOGK)>(v, buf, red);
+  }
 };
 
 // Splitting U units into n contiguous ranges: range i is [unit_begin(i), unit_begin(i + 1)).
@@ -207,6 +226,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   float* zc = reinterpret_cast<float*>(smem + p.zc_off);
+  float* fac = zc + G * 8 + 16;  // per-column output factors 2^(24 - e)
   uint8_t* ring = smem + p.ring_off + warp * p.NS * p.slot_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off) + warp * p.NS;
   // slot: [CH groups][16 rows][16 bits bytes] codes (TMA boxes, dense; 8-bit
@@ -287,17 +307,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if ((i & 7) >= p.N) zc[i] = 0.f;  // absent columns
     }
     pdl_wait();
+    float* red = fac + 8;
     for (int n = 0; n < p.N; ++n) {
       float v[FS::E];
       if (tid < FS::THREADS) {
         load_chunk<__half, FS::E>(p.x + static_cast<size_t>(n) * K + tid * FS::E, v);
         flip_signs<FS::E>(neg, v);
       }
-      FS::run(v, buf);
+      FS::run(v, buf, red);
+      const int e = row_scale_exp(red_max(red, FS::THREADS / 32) * p.inv_sqrt_k);
+      if (tid == 0) fac[n] = pow2f(24 - e);
+      const float sc = p.inv_sqrt_k * pow2f(e);
       for (int gg = warp; gg < G; gg += kWarps) {
-        put_group<BITS>(fl, buf, gg, n, p.N, p.inv_sqrt_k, p.zero, xs, zc, lane);
+        put_group<BITS>(fl, buf, gg, n, p.N, sc, p.zero, xs, zc, lane);
       }
-      __syncthreads();  // buf is reused by the next row; xs and zc are complete
+      __syncthreads();  // buf and red are reused by the next row; xs, zc, fac are complete
     }
     if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;  // zero B block
     __syncthreads();
@@ -311,6 +335,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     for (int i = tid * 16; i < G * 8 * 4; i += kWarps * 32 * 16) {
       cp_async16(smem + p.zc_off + i, p.xg + xs_bytes + i, 16);
     }
+    if (tid < 2) cp_async16(fac + 4 * tid, p.xg + xs_bytes + G * 8 * 4 + 16 * tid, 16);
     if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;  // zero B block
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
@@ -336,6 +361,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   const int xs_gstride = has_b ? N * 4 * kXq / 8 : 0;  // uint4 per group
   const uint32_t first_tile = u0 / G;
   uint32_t uc = u0;
+  // output factors of the lane's columns 2t, 2t + 1 (unused where absent)
+  const float f0 = fac[2 * t], f1 = fac[2 * t + 1];
 
   auto store_tile = [&](uint32_t tile, const float4& o) {
     const int m0 = tile * kRows;
@@ -436,7 +463,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     if (g0 + len == G || uc >= u1) {
       // ---- this warp's part of the tile is done
       const bool full = tile_start == 0 && g0 + len == G;
-      const float4 o = make_float4(acc[0] * kUnit, acc[1] * kUnit, acc[2] * kUnit, acc[3] * kUnit);
+      const float4 o = make_float4(acc[0] * f0, acc[1] * f1, acc[2] * f0, acc[3] * f1);
       if (full) {
         store_tile(tile, o);
       } else {
@@ -519,7 +546,7 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
   // the FWHT buffer of a fused rotation: K floats + one pad word per 32
-  const size_t buf_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + 64 + 15) & ~static_cast<size_t>(15);
+  const size_t buf_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + kZcTail + 15) & ~static_cast<size_t>(15);
   const size_t buf = gemv_fused_rotation(K, nb) ? (static_cast<size_t>(K) + K / 32) * 4 : 0;
   // ring and slots on 1 KiB boundaries (TMA destinations; the 128-byte swizzle atom)
   const size_t ring_off = (buf_off + buf + 1023) & ~static_cast<size_t>(1023);
@@ -583,6 +610,7 @@ static cudaError_t gemv_launch_f(int K, GemvParams& p, size_t smem, unsigned gri
     default:
       if constexpr (!FUSED) {
         if (K == 16384) return launch_pdl(gemv_kernel<BITS, 14, false>, g, b, smem, st, true, p);
+        if (K == 32768) return launch_pdl(gemv_kernel<BITS, 15, false>, g, b, smem, st, true, p);
       }
       return cudaErrorInvalidValue;
   }
@@ -601,13 +629,14 @@ size_t gemv_scratch_bytes(int K, int nb) { return gemv_xg_bytes(K / kGroup, nb);
 
 template <int BITS>
 static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
-  const dim3 g(a.N), b(kPrepWarps * 32);
+  const dim3 g(a.N);
   const float inv = static_cast<float>(1.0 / sqrt(static_cast<double>(K)));
   const __half* x = reinterpret_cast<const __half*>(a.x);
   uint8_t* xg = static_cast<uint8_t*>(a.xg);
-#define HQ_PREP(LK)                                                                            \
-  launch_pdl(gemv_prep_kernel<BITS, LK>, g, b, FwhtShape<LK, 3>::SMEM_FLOATS * sizeof(float), st, \
-             true, x, a.signs, xg, a.N, a.zero, inv)
+#define HQ_PREP(LK)                                                                          \
+  launch_pdl(gemv_prep_kernel<BITS, LK>, g, dim3(prep_warps(LK) * 32),                         \
+             (FwhtShape<LK, prep_logw(LK)>::SMEM_FLOATS + 32) * sizeof(float), st, true, x, a.signs, \
+             xg, a.N, a.zero, inv)
   switch (K) {
     case 128: return HQ_PREP(7);
     case 256: return HQ_PREP(8);
@@ -617,6 +646,7 @@ static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
     case 4096: return HQ_PREP(12);
     case 8192: return HQ_PREP(13);
     case 16384: return HQ_PREP(14);
+    case 32768: return HQ_PREP(15);
     default: return cudaErrorInvalidValue;
   }
 #undef HQ_PREP

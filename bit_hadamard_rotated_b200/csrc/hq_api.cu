@@ -36,7 +36,7 @@ static hq_status check_weight(const hq_weight* w) {
   if (!(w->bits == 2 || w->bits == 3 || w->bits == 4 || w->bits == 8)) {
     return (w->bits >= 1 && w->bits <= 8) ? HQ_ERR_UNSUPPORTED : HQ_ERR_INVALID_ARG;
   }
-  if (!is_pow2(w->K) || w->K < 128 || w->K > 16384) return HQ_ERR_UNSUPPORTED;
+  if (!is_pow2(w->K) || w->K < 128 || w->K > 32768) return HQ_ERR_UNSUPPORTED;
   if (w->zero < 0 || w->zero >= (1 << w->bits)) return HQ_ERR_INVALID_ARG;
   if (w->qweight == nullptr || w->scales == nullptr) return HQ_ERR_INVALID_ARG;
   if (!aligned(w->qweight, 16) || !aligned(w->scales, 16)) return HQ_ERR_INVALID_ARG;

@@ -8,7 +8,10 @@
 //                         counting sort of the (token, slot) pairs by expert,
 //                         the block list and each phase's per-CTA work split;
 //                         blocks 1..T: x'_t = H diag(s_in) x_t / sqrt(hidden),
-//                         written in the MMA B-fragment layout of every width;
+//                         written in the MMA B-fragment layout of every width
+//                         (scaled by a power of two 2^e per token that puts
+//                         its largest |x'| just below 2^14, undone exactly in
+//                         the phase epilogue, as is the same scale of h');
 //   2. moe_phase_kernel<A>  gate and up of every touched expert in one launch,
 //                         SwiGLU in the epilogue -> h [pairs][inter];
 //   3. moe_rot_h_kernel   h' = H diag(s_mid) h / sqrt(inter) per pair, in the
@@ -32,7 +35,6 @@ namespace moe {
 
 constexpr int kRows = 16;
 constexpr int kXq = 40;             // halves per (row, group, k-quad) B block (64 B + pad)
-constexpr float kUnit = 16777216.f;  // 2^24, the subnormal code unit
 constexpr int kWarps = 16;
 
 __host__ __device__ inline int layout_index(int bits) {
@@ -50,9 +52,11 @@ struct Ws {
   int* bounds;     // [2][kMaxGrid + 1] first work item of each CTA, phase A then B
   uint16_t* xl;    // [4][T][G_h][4][kXq] rotated tokens, per bit-width layout
   float* xsum;     // [4][T][G_h] sum over each group of the effective x'
+  float* xfac;     // [T] output factor 2^(24 - e) of each token's scaled x'
   float* h;        // [P][inter]
   uint16_t* hl;    // [P][G_i][4][kXq] rotated h, in its expert's layout
   float* hsum;     // [P][G_i]
+  float* hfac;     // [P] output factor 2^(24 - e) of each pair's scaled h'
   float* d;        // [P][hidden]
 };
 
@@ -104,7 +108,7 @@ static MoePlan moe_plan(int E, int hidden, int inter, int T, int k) {
   d.nb_max = std::min(E, d.P) + (d.P + 7) / 8;  // bound on sum_e ceil(cnt_e / 8)
   d.grid = std::min(sm_count(), moe::kMaxGrid);
   const size_t Gh = hidden / kGroup, Gi = inter / kGroup;
-  const size_t sizes[14] = {
+  const size_t sizes[15] = {
       256,                                             // status
       sizeof(int) * E,                                 // counts
       sizeof(int) * (E + 1),                           // offsets
@@ -112,16 +116,17 @@ static MoePlan moe_plan(int E, int hidden, int inter, int T, int k) {
       sizeof(int) * d.P,                               // sorted
       sizeof(uint2) * d.nb_max,                        // blk
       sizeof(int) * 2 * (moe::kMaxGrid + 1),           // bounds
-      0,                                               // (unused)
+      4 * static_cast<size_t>(T),                      // xfac
       2 * 4 * static_cast<size_t>(T) * Gh * 4 * moe::kXq,  // xl
       4 * 4 * static_cast<size_t>(T) * Gh,                 // xsum
       4 * static_cast<size_t>(d.P) * inter,                // h
       2 * static_cast<size_t>(d.P) * Gi * 4 * moe::kXq,    // hl
       4 * static_cast<size_t>(d.P) * Gi,                   // hsum
       4 * static_cast<size_t>(d.P) * hidden,               // d
+      4 * static_cast<size_t>(d.P),                        // hfac
   };
   size_t o = 0;
-  for (int i = 0; i < 14; ++i) {
+  for (int i = 0; i < 15; ++i) {
     pl.off[i] = o;
     o += a256(sizes[i]);
   }
@@ -139,12 +144,14 @@ static moe::Ws moe_ws(void* base, const MoePlan& pl) {
   w.sorted = reinterpret_cast<int*>(b + pl.off[4]);
   w.blk = reinterpret_cast<uint2*>(b + pl.off[5]);
   w.bounds = reinterpret_cast<int*>(b + pl.off[6]);
+  w.xfac = reinterpret_cast<float*>(b + pl.off[7]);
   w.xl = reinterpret_cast<uint16_t*>(b + pl.off[8]);
   w.xsum = reinterpret_cast<float*>(b + pl.off[9]);
   w.h = reinterpret_cast<float*>(b + pl.off[10]);
   w.hl = reinterpret_cast<uint16_t*>(b + pl.off[11]);
   w.hsum = reinterpret_cast<float*>(b + pl.off[12]);
   w.d = reinterpret_cast<float*>(b + pl.off[13]);
+  w.hfac = reinterpret_cast<float*>(b + pl.off[14]);
   return w;
 }
 
@@ -325,13 +332,14 @@ __device__ void route_cta(const hq_expert* __restrict__ ex, const int32_t* __res
 }
 
 
-// Write one rotated row (fwht_block output in buf, unnormalised) as fp16 B
-// blocks for the code decode of BITS: block (group gg, k-quad t) holds the
-// 8 steps x 4 activations, each scaled by 2^-a of its code field; sums[gg] =
-// sum over the group of the effective activations (B * 2^a), for the
-// zero-point term.  Warp-per-group; nw warps of the block take part.
+// Write one rotated row (fwht_block output in buf, unnormalised; sc = 2^e /
+// sqrt(K)) as fp16 B blocks for the code decode of BITS: block (group gg,
+// k-quad t) holds the 8 steps x 4 activations x' 2^e, each scaled by 2^-a of
+// its code field; sums[gg] = sum over the group of the effective activations
+// (B * 2^a), for the zero-point term.  Warp-per-group; nw warps of the block
+// take part.
 template <int BITS>
-__device__ __forceinline__ void write_layout(const float* buf, float inv, int G, uint16_t* out,
+__device__ __forceinline__ void write_layout(const float* buf, float sc, int G, uint16_t* out,
                                              float* sums, int warp, int nw, int lane) {
   const int s = lane >> 2, t = lane & 3;
   int kc[4], ka[4];
@@ -346,7 +354,7 @@ __device__ __forceinline__ void write_layout(const float* buf, float inv, int G,
     float part = 0.f;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + kc[r])] * inv));
+      const float xv = __half2float(__float2half_rn(buf[fwht_pad(kGroup * gg + kc[r])] * sc));
       const __half b = __float2half_rn(xv * __int_as_float((127 - ka[r]) << 23));
       hv[r] = __half_as_ushort(b);
       part += __half2float(b) * __int_as_float((127 + ka[r]) << 23);
@@ -361,14 +369,14 @@ __device__ __forceinline__ void write_layout(const float* buf, float inv, int G,
   }
 }
 
-__device__ __forceinline__ void write_layout_bits(int bits, const float* buf, float inv, int G,
+__device__ __forceinline__ void write_layout_bits(int bits, const float* buf, float sc, int G,
                                                   uint16_t* out, float* sums, int warp, int nw,
                                                   int lane) {
   switch (bits) {
-    case 2: write_layout<2>(buf, inv, G, out, sums, warp, nw, lane); break;
-    case 3: write_layout<3>(buf, inv, G, out, sums, warp, nw, lane); break;
-    case 4: write_layout<4>(buf, inv, G, out, sums, warp, nw, lane); break;
-    default: write_layout<8>(buf, inv, G, out, sums, warp, nw, lane); break;
+    case 2: write_layout<2>(buf, sc, G, out, sums, warp, nw, lane); break;
+    case 3: write_layout<3>(buf, sc, G, out, sums, warp, nw, lane); break;
+    case 4: write_layout<4>(buf, sc, G, out, sums, warp, nw, lane); break;
+    default: write_layout<8>(buf, sc, G, out, sums, warp, nw, lane); break;
   }
 }
 
@@ -391,14 +399,18 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   const auto neg = sign_bits<S::E>(signs ? signs + tid * S::E : nullptr);
   pdl_wait();  // x may be the previous kernel's output
   float v[S::E];
+  float* red = buf + S::SMEM_FLOATS;
   load_chunk<__half, S::E>(x + static_cast<size_t>(t) * S::K + tid * S::E, v);
   flip_signs<S::E>(neg, v);
-  fwht_block<LOGK, 5>(v, buf);
+  fwht_block<LOGK, 5>(v, buf, red);
+  const int e = row_scale_exp(red_max(red, S::W) * inv);
+  if (tid == 0) w.xfac[t] = pow2f(24 - e);
+  const float sc = inv * pow2f(e);
   const int G = S::K / kGroup;
   const int bits_of[4] = {2, 3, 4, 8};
   for (int L = 0; L < 4; ++L) {
     const size_t row = static_cast<size_t>(L) * d.T + t;
-    write_layout_bits(bits_of[L], buf, inv, G, w.xl + row * G * 4 * kXq, w.xsum + row * G,
+    write_layout_bits(bits_of[L], buf, sc, G, w.xl + row * G * 4 * kXq, w.xsum + row * G,
                       tid >> 5, S::THREADS / 32, tid & 31);
   }
 }
@@ -419,11 +431,15 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   const int e = ids[w.sorted[p]];
   const int bits = ex[e].bits;
   float v[S::E];
+  float* red = buf + S::SMEM_FLOATS;
   load_chunk<float, S::E>(w.h + static_cast<size_t>(p) * S::K + tid * S::E, v);
   flip_signs<S::E>(neg, v);
-  fwht_block<LOGK, 5>(v, buf);
+  fwht_block<LOGK, 5>(v, buf, red);
+  const int ex_ = row_scale_exp(red_max(red, S::W) * inv);
+  if (tid == 0) w.hfac[p] = pow2f(24 - ex_);
+  const float sc = inv * pow2f(ex_);
   const int G = S::K / kGroup;
-  write_layout_bits(bits, buf, inv, G, w.hl + static_cast<size_t>(p) * G * 4 * kXq,
+  write_layout_bits(bits, buf, sc, G, w.hl + static_cast<size_t>(p) * G * 4 * kXq,
                     w.hsum + static_cast<size_t>(p) * G, tid >> 5, S::THREADS / 32, tid & 31);
 }
 
@@ -530,6 +546,7 @@ struct SegInfo {
   int off, ncol;     // first sorted pair of the block, its columns (<= 8)
   int col0;          // column offset of the block in the staged fragments
   int L;             // activation layout (bit width) of phase A
+  float fac[8];      // output factor 2^(24 - e) of each column (token or pair)
 };
 
 struct PassMeta {
@@ -607,12 +624,13 @@ __device__ __forceinline__ void seg_store(const Ws& w, const Dims& d, const SegI
     const int m = m0 + g + 8 * (q4 >> 1);
     if (col < sg.ncol && m < M) {
       const size_t prow = static_cast<size_t>(sg.off + col);
+      const float f = sg.fac[col];
       if (PHASE == 0) {
-        const float gv = og[q4] * kUnit, uv = ou[q4] * kUnit;
+        const float gv = og[q4] * f, uv = ou[q4] * f;
         w.h[prow * d.inter + m] = gv / (1.f + expf(-gv)) * uv;
       } else {
-        w.d[prow * d.hidden + m] = og[q4] * kUnit;
-        w.d[prow * d.hidden + m + kRows] = ou[q4] * kUnit;  // M is a multiple of 32
+        w.d[prow * d.hidden + m] = og[q4] * f;
+        w.d[prow * d.hidden + m + kRows] = ou[q4] * f;  // M is a multiple of 32
       }
     }
   }
@@ -924,6 +942,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
                      bsrc + ((seg_brow<PHASE>(w, d, sg, cl) * G + gg) * 4 + q) * kXq + pc * 8, 16);
         }
       }
+      // output factors of the segment's columns (written before the barrier
+      // below, read by the epilogue after it)
+      if (tid < sg.ncol) {
+        pm.seg[k].fac[tid] = PHASE == 0 ? w.xfac[w.sorted[sg.off + tid] / d.k] : w.hfac[sg.off + tid];
+      }
       // -zero * sum_k x' * 2^-24 per group and column (0 for absent columns)
       const float zneg = -static_cast<float>(sg.ed.zero) * 5.9604644775390625e-8f;
       for (int i = tid; i < G * 8; i += kWarps * 32) {
@@ -1022,11 +1045,11 @@ static cudaError_t moe_launch_front(int hidden, const hq_expert* ex, const int32
 #define HQ_FRONT(LK)                                                                          \
   case (1 << LK):                                                                             \
     return launch_pdl(moe::moe_front_kernel<LK>, dim3(d.T + 1), dim3(FwhtShape<LK>::THREADS),   \
-                      std::max(FwhtShape<LK>::SMEM_FLOATS * sizeof(float), route_smem), st, true, \
+                      std::max((FwhtShape<LK>::SMEM_FLOATS + 32) * sizeof(float), route_smem), st, true, \
                       ex, ids, x, s, w, d, inv);
   switch (hidden) {
     HQ_FRONT(7) HQ_FRONT(8) HQ_FRONT(9) HQ_FRONT(10) HQ_FRONT(11) HQ_FRONT(12) HQ_FRONT(13)
-    HQ_FRONT(14)
+    HQ_FRONT(14) HQ_FRONT(15)
     default: return cudaErrorInvalidValue;
   }
 #undef HQ_FRONT
@@ -1039,9 +1062,10 @@ static cudaError_t moe_launch_rot_h(int inter, const hq_expert* ex, const int32_
 #define HQ_ROTH(LK)                                                                           \
   case (1 << LK):                                                                             \
     return launch_pdl(moe::moe_rot_h_kernel<LK>, dim3(d.P), dim3(FwhtShape<LK>::THREADS),       \
-                      FwhtShape<LK>::SMEM_FLOATS * sizeof(float), st, true, ex, ids, s, w, d, inv);
+                      (FwhtShape<LK>::SMEM_FLOATS + 32) * sizeof(float), st, true, ex, ids, s, w, d, inv);
   switch (inter) {
     HQ_ROTH(7) HQ_ROTH(8) HQ_ROTH(9) HQ_ROTH(10) HQ_ROTH(11) HQ_ROTH(12) HQ_ROTH(13) HQ_ROTH(14)
+    HQ_ROTH(15)
     default: return cudaErrorInvalidValue;
   }
 #undef HQ_ROTH
@@ -1064,7 +1088,7 @@ static cudaError_t moe_launch_phase(const hq_expert* ex, const moe::Ws& w, const
     return launch_pdl(moe::moe_phase_kernel<PHASE, LK>, grid, block, ps.total, st, true, ex, w, d);
   switch (K) {
     HQ_PHASE(7) HQ_PHASE(8) HQ_PHASE(9) HQ_PHASE(10) HQ_PHASE(11) HQ_PHASE(12) HQ_PHASE(13)
-    HQ_PHASE(14)
+    HQ_PHASE(14) HQ_PHASE(15)
     default: return cudaErrorInvalidValue;
   }
 #undef HQ_PHASE
@@ -1082,7 +1106,7 @@ extern "C" {
 size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k) {
   auto pow2 = [](int v) { return v > 0 && (v & (v - 1)) == 0; };
   if (n_experts < 1 || n_experts > kMaxExperts || T < 0 || k < 1 || k > 32 || !pow2(hidden) ||
-      !pow2(inter) || hidden < 128 || inter < 128 || hidden > 16384 || inter > 16384 ||
+      !pow2(inter) || hidden < 128 || inter < 128 || hidden > 32768 || inter > 32768 ||
       static_cast<long>(T) * k > (1L << 24)) {
     return 0;
   }
@@ -1112,8 +1136,8 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
   if (n_experts < 1 || T < 0 || k < 1 || k > 32 || hidden <= 0 || inter <= 0) {
     return HQ_ERR_INVALID_ARG;
   }
-  if (!pow2(hidden) || !pow2(inter) || hidden < 128 || inter < 128 || hidden > 16384 ||
-      inter > 16384 || n_experts > kMaxExperts) {
+  if (!pow2(hidden) || !pow2(inter) || hidden < 128 || inter < 128 || hidden > 32768 ||
+      inter > 32768 || n_experts > kMaxExperts) {
     return HQ_ERR_UNSUPPORTED;
   }
   if (static_cast<long>(T) * k > (1L << 24)) return HQ_ERR_INVALID_ARG;

@@ -28,7 +28,8 @@ namespace {
 
 constexpr size_t kScratchBytes = size_t{512} << 10;  // 512 KiB in total
 constexpr size_t kStatus = 256;                      // status word, kept zero
-// Rotated activations of one batch block: at most 332 KiB (K = 16384, 8 columns).
+// Rotated activations of one batch block: at most 332 KiB (K = 16384 with 8
+// columns; K = 32768 runs blocks of at most 2).
 constexpr size_t kXgBytes = kScratchBytes - kStatus;
 
 // The scratch: [status][rotated activations of the current batch block].
@@ -66,7 +67,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
   if (!(w->bits == 2 || w->bits == 3 || w->bits == 4 || w->bits == 8)) {
     return (w->bits >= 1 && w->bits <= 8) ? HQ_ERR_UNSUPPORTED : HQ_ERR_INVALID_ARG;
   }
-  if (!pow2(w->K) || w->K < 128 || w->K > 16384) return HQ_ERR_UNSUPPORTED;
+  if (!pow2(w->K) || w->K < 128 || w->K > 32768) return HQ_ERR_UNSUPPORTED;
   if (w->zero < 0 || w->zero >= (1 << w->bits)) return HQ_ERR_INVALID_ARG;
   if (!w->qweight || !w->scales || !aligned(w->qweight, 16) || !aligned(w->scales, 16) ||
       (w->signs && !aligned(w->signs, 16))) {

@@ -86,7 +86,7 @@ typedef enum { HQ_F16 = 0, HQ_BF16 = 1, HQ_F32 = 2 } hq_dtype;
 typedef struct {
   int bits;                /* 2, 3, 4 or 8 */
   int M;                   /* output features, >= 1 */
-  int K;                   /* input features: power of two, 128 <= K <= 16384 */
+  int K;                   /* input features: power of two, 128 <= K <= 32768 */
   int zero;                /* integer zero point, 0 <= zero < 2^bits (2^(bits-1) usual) */
   const uint32_t* qweight; /* [M][K*bits/32] packed codes, 16-byte aligned */
   const uint16_t* scales;  /* [M][K/128] fp16 bit patterns, 16-byte aligned */
@@ -153,7 +153,7 @@ size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k)
  * experts: DEVICE array [n_experts] of hq_expert.  x: [T][hidden] fp16.
  * topk_ids: [T][k] int32, topk_w: [T][k] fp32.  signs_in [hidden], signs_mid
  * [inter] (NULL = no sign flip).  y: [T][hidden] fp32.
- * hidden, inter: powers of two in [128, 16384].  1 <= k <= 32.
+ * hidden, inter: powers of two in [128, 32768].  1 <= k <= 32.
  * 1 <= n_experts <= 16384 (HQ_ERR_UNSUPPORTED above).
  * An expert id outside [0, n_experts), or an expert whose bits or zero is out
  * of range, is skipped (its contribution is zero) and sets HQ_ERR_DATA in the
@@ -179,7 +179,7 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
  * workspace for its activation images).
  * Its scratch is a 512 KiB array in the library's device memory, held on every
  * GPU that loads the library until the process exits: the status word and the
- * rotated activations of one batch block (at most 332 KiB, K = 16384).  Limits:
+ * rotated activations of one batch block (at most 332 KiB).  Limits:
  * as hq_linear (HQ_ERR_WORKSPACE if a block's activations did not fit, which
  * no supported K reaches).
  * The array's device address is looked up on every call (a runtime query that
@@ -221,7 +221,15 @@ hq_status hq_check_status(void* workspace, hq_stream_t stream);
 
 /*
  * hq_unpack_codes -- decode n_codes codes of width bits (1..8) from a packed
- * little-endian bit stream into one byte each.  Bit-exact; test-facing.
+ * little-endian bit stream into one byte each: codes_out[j] = stream bits
+ * [bits*j, bits*j + bits), the layout every packed weight of this library
+ * uses.  Bit-exact; test-facing (it checks the layout on its own, apart from
+ * the matmuls that decode it in registers).
+ * packed: 4-byte aligned, ceil(bits*n_codes/32) words; codes_out: n_codes
+ * bytes.  n_codes = 0 launches nothing.
+ * Cites: the per-expert 2/3/4-bit and 8-bit group-128 integer codes that stay
+ * packed through the run (LLaDA2.2-mini Orin-Nano model card, Properties
+ * table; Qwen3-8B BPDQ 2-bit card, introduction).
  */
 hq_status hq_unpack_codes(const uint32_t* packed, int bits, size_t n_codes,
                           uint8_t* codes_out, hq_stream_t stream);

@@ -45,7 +45,7 @@ def lin(L, w, batch=1, x=FAKE, y=FAKE, ws=FAKE, ws_bytes=1 << 30):
 @pytest.mark.parametrize("kw,want", [
     (dict(bits=5), HQ_ERR_UNSUPPORTED), (dict(bits=0), HQ_ERR_INVALID_ARG),
     (dict(bits=9), HQ_ERR_INVALID_ARG), (dict(K=4096 + 128), HQ_ERR_UNSUPPORTED),
-    (dict(K=64), HQ_ERR_UNSUPPORTED), (dict(K=32768), HQ_ERR_UNSUPPORTED),
+    (dict(K=64), HQ_ERR_UNSUPPORTED), (dict(K=65536), HQ_ERR_UNSUPPORTED),
     (dict(K=0), HQ_ERR_INVALID_ARG), (dict(M=0), HQ_ERR_INVALID_ARG),
     (dict(zero=16), HQ_ERR_INVALID_ARG), (dict(zero=-1), HQ_ERR_INVALID_ARG),
     (dict(qweight=FAKE + 8), HQ_ERR_INVALID_ARG), (dict(scales=FAKE + 2), HQ_ERR_INVALID_ARG),

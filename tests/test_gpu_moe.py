@@ -96,7 +96,8 @@ def test_moe_with_8bit_experts_and_other_shapes():
     check(y, want, bound, "8-bit mix")
 
 
-@pytest.mark.parametrize("hidden,inter", [(8192, 256), (256, 8192), (4096, 1024), (16384, 128)])
+@pytest.mark.parametrize("hidden,inter", [(8192, 256), (256, 8192), (4096, 1024), (16384, 128),
+                                          (32768, 128), (128, 32768)])
 def test_moe_wide_shapes(hidden, inter):
     """Widths whose activation fragments do not fit beside the copy rings in
     shared memory (read from global memory instead), and ones that just fit."""

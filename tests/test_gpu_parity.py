@@ -325,3 +325,17 @@ def test_linear_single_spike_null_signs(bits, N, c):
                   d["zero"]).cpu().numpy()
     want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], None, x)
     assert_within(y, want, bound, what=f"spike c={c} b{bits} N{N}")
+
+
+# ---------------------------------------------------------------- the largest K
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("N", [1, 2, 3, 9, 40])
+def test_linear_k32768(bits, N):
+    """K = 32768, the largest supported width: the GEMV (rotation in a prep
+    kernel of 32 warps, batch blocks of 1 or 2 columns) and, from batch 5 or 9,
+    the tensor-core GEMM with narrower column blocks."""
+    M, K = 300, 32768
+    d = synth.linear(M, K, bits, N, seed=61 + bits + N, scale_dist="loguniform", outlier_frac=0.01)
+    y = run_linear(d).cpu().numpy()
+    want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"], threads=8)
+    assert_within(y, want, bound, what=f"K32768 b{bits} N{N}")

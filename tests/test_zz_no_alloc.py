@@ -33,7 +33,8 @@ def gpu():
                                          # n0*K of x and n0*M of y; K = 16384 rotates in a
                                          # separate kernel for every block
                                          (257, 4096, 2, 11), (1000, 4096, 3, 17),
-                                         (257, 16384, 4, 20), (333, 2048, 8, 9)])
+                                         (257, 16384, 4, 20), (333, 2048, 8, 9),
+                                         (130, 32768, 2, 3), (130, 32768, 8, 2)])
 def test_noalloc_matches_hq_linear_twice(M, K, bits, N):
     from bit_hadamard_rotated_b200 import _lib, hq_linear, make_weight
     d = synth.linear(M, K, bits, N, seed=M + K + bits)
@@ -66,7 +67,7 @@ def test_noalloc_rejects_what_hq_linear_rejects():
     from bit_hadamard_rotated_b200._lib import HQ_ERR_UNSUPPORTED, HqWeight
     L = _lib.lib()
     before = L.hq_launch_count()
-    for K, want in ((32768, HQ_ERR_UNSUPPORTED), (96, HQ_ERR_UNSUPPORTED)):
+    for K, want in ((65536, HQ_ERR_UNSUPPORTED), (96, HQ_ERR_UNSUPPORTED)):
         w = HqWeight(4, 64, K, 8, 0x100000, 0x100000, None)
         st = L.hq_linear_noalloc(ctypes.byref(w), 0x100000, 1, 0x100000, None)
         assert st == want
