@@ -10,8 +10,9 @@ The formulas and the readings of the pages they rest on are in
 ``hq_oracle.h``: the random-sign Hadamard rotation x' = H.diag(s).x/sqrt(K)
 ("group-128 GPTQ in a Hadamard-rotated basis" with "rotation signs":
 LLaDA2.2-mini Orin-Nano model card, Properties table and file list), the
-group-128 dequantisation w = scale.(q - z), the fp64 contraction, and the
-SwiGLU MoE expert composition.
+group-128 dequantisation w = scale.(q - z), the fp64 contraction, the
+SwiGLU MoE expert composition, and the rotated round-to-nearest quantiser
+that produces packed weights.
 """
 from __future__ import annotations
 
@@ -68,8 +69,11 @@ def lib():
             L.hqo_dequant_dot.argtypes = [i, i, i, i, vp, vp, vp, i, i, i, vp, vp]
             L.hqo_linear.argtypes = [i, i, i, i, vp, vp, vp, vp, i, i, i, vp, vp]
             L.hqo_moe.argtypes = [vp, i, i, i, vp, i, vp, vp, i, vp, vp, i, i, vp, vp, vp]
+            L.hqo_f64_to_f16.argtypes = [ctypes.c_double]
+            L.hqo_f64_to_f16.restype = ctypes.c_uint16
+            L.hqo_quantize.argtypes = [vp, i, i, i, vp, i, i, vp, vp, vp]
             for f in ("hqo_unpack", "hqo_pack", "hqo_fwht", "hqo_rotate", "hqo_rotate_f16",
-                      "hqo_dequant_dot", "hqo_linear", "hqo_moe"):
+                      "hqo_dequant_dot", "hqo_linear", "hqo_moe", "hqo_quantize"):
                 getattr(L, f).restype = None
             _lib = L
     return _lib
@@ -85,6 +89,39 @@ def _c(a, dtype):
 
 def f16_to_f64(bits_u16: int) -> float:
     return lib().hqo_f16_to_f64(int(bits_u16))
+
+
+def f64_to_f16(v: float) -> int:
+    """binary16 bit pattern nearest to v (ties to even)."""
+    return int(lib().hqo_f64_to_f16(float(v)))
+
+
+def quantize(W, bits: int, signs=None, m_begin=0, m_end=None, want_rotated=False, threads=1):
+    """Rotated round-to-nearest quantiser (hq_oracle.h).  W: [M][K] (any real
+    dtype, read as float64).  Returns (qweight uint32 [M][K*bits/32], scales
+    fp16 [M][K/128], rotated float64 [M][K] or None)."""
+    Wd = _c(W, np.float64)
+    M, K = Wd.shape
+    s = _c(signs, np.int8)
+    m_end = M if m_end is None else m_end
+    q = np.zeros((M, K * bits // 32), np.uint32)
+    sc = np.zeros((M, K // 128), np.uint16)
+    r = np.zeros((M, K), np.float64) if want_rotated else None
+
+    def run(lo, hi):
+        lib().hqo_quantize(_p(Wd), M, K, bits, _p(s), lo, hi, _p(q), _p(sc), _p(r))
+
+    if threads <= 1:
+        run(m_begin, m_end)
+    else:
+        edges = np.linspace(m_begin, m_end, threads + 1).astype(int)
+        ts = [threading.Thread(target=run, args=(int(edges[t]), int(edges[t + 1])))
+              for t in range(threads)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
+    return q, sc.view(np.float16), r
 
 
 def unpack(words, bits: int, n_codes: int) -> np.ndarray:

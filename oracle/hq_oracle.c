@@ -185,3 +185,67 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
   free(g);
   free(xr);
 }
+
+/* binary16 from the definition: 1 sign bit, 5 exponent bits (bias 15), 10
+ * fraction bits; values below 2^-14 are subnormal multiples of 2^-24. */
+uint16_t hqo_f64_to_f16(double v) {
+  uint16_t sign = signbit(v) ? 0x8000u : 0u;
+  double a = fabs(v);
+  if (isnan(v)) return (uint16_t)(sign | 0x7e00u);
+  /* 65520 is halfway between 65504 (odd fraction) and 65536: ties go to 65536 = inf */
+  if (a >= 65520.0) return (uint16_t)(sign | 0x7c00u);
+  if (a < ldexp(1.0, -14)) {
+    /* subnormal (or zero): a = m 2^-24; m = 1024 is the smallest normal */
+    long m = lrint(ldexp(a, 24));
+    return (uint16_t)(sign | (uint16_t)m);
+  }
+  int e2 = 0;
+  frexp(a, &e2); /* a = f 2^e2, f in [0.5, 1): a in [2^(e2-1), 2^e2) */
+  int E = e2 - 1;
+  long mant = lrint(ldexp(a, 10 - E)); /* in [1024, 2048] */
+  if (mant == 2048) {
+    mant = 1024;
+    E += 1;
+  }
+  if (E > 15) return (uint16_t)(sign | 0x7c00u);
+  return (uint16_t)(sign | (uint16_t)((E + 15) << 10) | (uint16_t)(mant - 1024));
+}
+
+void hqo_quantize(const double* W, int M, int K, int bits, const int8_t* signs,
+                  int m_begin, int m_end, uint32_t* qweight, uint16_t* scales,
+                  double* rotated) {
+  (void)M;
+  const int G = K / 128;
+  const int zero = 1 << (bits - 1);
+  const int qmax = (1 << bits) - 1;
+  const size_t words_per_row = (size_t)K * (size_t)bits / 32;
+  double* r = (double*)malloc(sizeof(double) * (size_t)K);
+  uint8_t* q = (uint8_t*)malloc((size_t)K);
+  for (int m = m_begin; m < m_end; ++m) {
+    hqo_rotate(W + (size_t)m * K, signs, K, r);
+    if (rotated) memcpy(rotated + (size_t)m * K, r, sizeof(double) * (size_t)K);
+    for (int g = 0; g < G; ++g) {
+      double amax = 0.0;
+      for (int k = 128 * g; k < 128 * g + 128; ++k) {
+        if (fabs(r[k]) > amax) amax = fabs(r[k]);
+      }
+      double want = 2.0 * amax / (double)qmax;
+      if (want > 65504.0) want = 65504.0;
+      uint16_t s16 = hqo_f64_to_f16(want);
+      double s = hqo_f16_to_f64(s16);
+      scales[(size_t)m * G + g] = s16;
+      for (int k = 128 * g; k < 128 * g + 128; ++k) {
+        long c = zero;
+        if (s > 0.0) {
+          c = lrint(r[k] / s) + zero;
+          if (c < 0) c = 0;
+          if (c > qmax) c = qmax;
+        }
+        q[k] = (uint8_t)c;
+      }
+    }
+    hqo_pack(q, bits, (size_t)K, qweight + (size_t)m * words_per_row);
+  }
+  free(q);
+  free(r);
+}

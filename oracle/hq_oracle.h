@@ -14,7 +14,8 @@
  *     Pingala-8 2-bit card, "What this is"),
  *   - the group-128 dequantisation  w[m][k] = scale[m][k/128] * (q[m][k] - z),
  *   - the contraction  y[n][m] = sum_k w[m][k] * x'[n][k],
- *   - the MoE expert composition (gate/up, SwiGLU, down, weighted combine).
+ *   - the MoE expert composition (gate/up, SwiGLU, down, weighted combine),
+ *   - the rotated round-to-nearest quantiser that produces packed weights.
  *
  * Readings where the pages are silent (the plainest reading in each case):
  *   - H_K is the Sylvester Hadamard matrix in natural order,
@@ -105,6 +106,28 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
              const float* topk_w, int k, const int8_t* s_in,
              const int8_t* s_mid, int t_begin, int t_end, double* y,
              double* bound, double* h_out);
+
+/* IEEE binary16 bit pattern nearest to v (round to nearest, ties to even;
+ * overflow to infinity, NaN to a quiet NaN). */
+uint16_t hqo_f64_to_f16(double v);
+
+/* Rotated round-to-nearest quantiser, the step that produces the packed
+ * weights ("group-128 GPTQ in a Hadamard-rotated basis": LLaDA2.2-mini
+ * Orin-Nano model card, Properties table; weights "behind a random Hadamard
+ * rotation": Qwen3.8-27B Pingala-8 2-bit card, "What this is"), without
+ * GPTQ's calibration-driven rounding, for rows [m_begin, m_end):
+ *   r        = H_K diag(s) W[m] / sqrt(K)        (fp64; = (W diag(s) H_K)[m] / sqrt(K))
+ *   a_g      = max_{k in group g} |r_k|          (groups of 128 along K)
+ *   scale_g  = fp16(min(2 a_g / (2^b - 1), 65504))   (round to nearest even)
+ *   q_k      = clamp(rint(r_k / scale_g) + 2^(b-1), 0, 2^b - 1), or 2^(b-1)
+ *              where scale_g = 0                  (rint: ties to even)
+ * so that dequant(q) = scale (q - 2^(b-1)) with the library's zero point.
+ * W: [M][K] doubles.  qweight: [M][K*bits/32] words (hqo_pack layout per
+ * row); scales: [M][K/128] fp16 bit patterns; rotated (optional, [M][K]):
+ * r.  Only rows m_begin..m_end-1 are written. */
+void hqo_quantize(const double* W, int M, int K, int bits, const int8_t* signs,
+                  int m_begin, int m_end, uint32_t* qweight, uint16_t* scales,
+                  double* rotated);
 
 #ifdef __cplusplus
 }

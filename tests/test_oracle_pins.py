@@ -352,3 +352,102 @@ def test_routing_weights_and_ties():
     logits = np.zeros((1, 16), np.float32)
     order = np.argsort(-logits, axis=1, kind="stable")[:, :4]
     assert order.tolist() == [[0, 1, 2, 3]]
+
+
+# ---------------------------------------------------------------- rotated round-to-nearest quantiser
+def test_f64_to_f16_matches_numpy():
+    """The oracle's double -> binary16 rounding against numpy's (ties to even),
+    over normals, subnormals, exact ties and the overflow edge."""
+    rng = np.random.default_rng(3)
+    v = np.concatenate([
+        rng.standard_normal(20000) * 10.0 ** rng.uniform(-9, 5, 20000),
+        (np.arange(1, 3000) + 0.5) * 2.0**-24,           # subnormal ties
+        1.0 + (np.arange(0, 2048) + 0.5) * 2.0**-10,     # normal ties at [1, 3)
+        [0.0, -0.0, 65504.0, 65519.99, 2.0**-14, 2.0**-14 - 2.0**-25, 2.0**-25, -2.0**-25],
+    ])
+    with np.errstate(over="ignore"):
+        want = v.astype(np.float16).view(np.uint16)
+    got = np.array([oracle.f64_to_f16(x) for x in v], np.uint16)
+    assert np.array_equal(got, want)
+
+
+def _rand_weights(M, K, seed, outliers=True):
+    rng = np.random.default_rng(seed)
+    W = rng.standard_normal((M, K)) * 0.02
+    if outliers:
+        W[:, rng.choice(K, max(1, K // 100), replace=False)] *= 20.0
+    return W.astype(np.float32).astype(np.float64), synth.signs(rng, K)
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_quantize_rotation_grid_and_packing(bits):
+    """hqo_quantize against what fixes it independently: the rotated row equals
+    W diag(s) H / sqrt(K) built with scipy; every code is a nearest point of
+    its group's grid scale (q - 2^(b-1)), q in [0, 2^b - 1] (brute force over
+    all codes); the group's largest |r| lands on the top code if positive, on
+    code 0 if negative (code 1 only when the fp16 scale rounded up, which
+    moves -2^(b-1) scale past it); the grid spans that largest |r| to within
+    the fp16 rounding of the scale; the words unpack (numpy) to those codes."""
+    M, K = 24, 512
+    W, s = _rand_weights(M, K, 70 + bits)
+    q, sc, r = oracle.quantize(W, bits, s, want_rotated=True)
+    H = scipy.linalg.hadamard(K).astype(np.float64)
+    assert np.allclose(r, W @ np.diag(sign_vec(s, K)) @ H / np.sqrt(K), rtol=1e-12, atol=1e-15)
+    z, qmax = 1 << (bits - 1), (1 << bits) - 1
+    codes = np.stack([np_unpack(q[m], bits, K) for m in range(M)])
+    scale = np.repeat(sc.astype(np.float64), 128, axis=1)
+    err = np.abs(r - scale * (codes - z))
+    grid = scale[..., None] * (np.arange(qmax + 1)[None, None, :] - z)
+    best = np.min(np.abs(r[..., None] - grid), axis=2)
+    assert np.all(err <= best * (1 + 1e-12) + 1e-300)
+    for m in range(M):
+        for g in range(K // 128):
+            seg = r[m, 128 * g:128 * g + 128]
+            i = int(np.argmax(np.abs(seg)))
+            a = abs(seg[i])
+            c = codes[m, 128 * g + i]
+            span = float(sc[m, g]) * qmax / 2
+            assert abs(span - a) <= 2.0**-11 * max(span, a)
+            if seg[i] > 0:
+                assert c == qmax
+            else:
+                assert c == 0 or (c == 1 and span > a)
+    assert np.all(err <= scale / 2 * (1 + 2.0**(bits - 10)))
+
+
+def test_quantize_zero_rows_and_tiny_groups():
+    """A zero row quantises to scale 0 and the zero-point code; a group whose
+    scale underflows fp16 does the same; the rest of the row is unaffected."""
+    K, bits = 256, 4
+    W = np.zeros((2, K))
+    W[1, :] = 1e-3
+    W[1, 0] += 1.0
+    q, sc, r = oracle.quantize(W, bits, None, want_rotated=True)
+    assert np.all(sc[0] == 0) and np.all(np_unpack(q[0], bits, K) == 8)
+    assert np.all(sc[1] > 0)
+    W2 = np.full((1, K), 1e-12)
+    q2, sc2, _ = oracle.quantize(W2, bits, None)
+    assert np.all(sc2 == 0) and np.all(np_unpack(q2[0], bits, K) == 8)
+
+
+@pytest.mark.parametrize("bits", [2, 4, 8])
+def test_quantize_then_linear_approximates_dense_product(bits):
+    """y = dequant(quantize(W)) x' with the oracle's own linear is W x (numpy,
+    dense) up to the quantisation bound sum_g scale_g / 2 (1 + 2^(b-10))
+    sum_{k in g} |x'_k|: the rotation cancels (W x = W_rot x') and every
+    rotated weight is within half a grid step."""
+    M, K, N = 40, 1024, 3
+    W, s = _rand_weights(M, K, 80 + bits)
+    q, sc, _ = oracle.quantize(W, bits, s)
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((N, K)).astype(np.float16)
+    y, _ = oracle.linear(bits, M, K, 1 << (bits - 1), q, sc, s, x)
+    xd = x.astype(np.float64)
+    want = xd @ W.T
+    H = scipy.linalg.hadamard(K).astype(np.float64)
+    xr = (H @ (sign_vec(s, K)[:, None] * xd.T)).T / np.sqrt(K)
+    ax = np.abs(xr).reshape(N, K // 128, 128).sum(axis=2)          # [N][G]
+    bound = (ax @ (sc.astype(np.float64).T / 2)) * (1 + 2.0**(bits - 10))  # [N][M]
+    assert np.all(np.abs(y - want) <= bound * (1 + 1e-9) + 1e-12)
+    # and the bound is not vacuous: the error is a sizeable part of it somewhere
+    assert np.max(np.abs(y - want) / bound) > 0.05
