@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_noalloc.restype = _i
         L.hq_linear_noalloc_check_status.argtypes = [_vp]
         L.hq_linear_noalloc_check_status.restype = _i
+        L.hq_quantize.argtypes = [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]
+        L.hq_quantize.restype = _i
         L.hq_moe_workspace_offset.argtypes = [_i, _i, _i, _i, _i, _i]
         L.hq_moe_workspace_offset.restype = _sz
         L.hq_moe_launches.argtypes = []

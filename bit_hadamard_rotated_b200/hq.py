@@ -53,6 +53,27 @@ def hq_rotate(x: torch.Tensor, signs: torch.Tensor | None = None, out_dtype=torc
     return out
 
 
+def hq_quantize(W: torch.Tensor, bits: int, signs: torch.Tensor | None = None,
+                qweight: torch.Tensor | None = None, scales: torch.Tensor | None = None,
+                stream=None):
+    """Pack real weights W [M][K] (fp16/bf16/fp32) into (qweight int32 [M][K*bits/32],
+    scales fp16 [M][K/128]) with the rotated round-to-nearest quantiser; the zero
+    point of the result is 2^(bits-1)."""
+    _need_cuda(W, signs)
+    if W.dim() != 2 or W.dtype not in _DT or not W.is_contiguous():
+        raise ValueError("W must be a contiguous [M][K] fp16, bf16 or fp32 tensor")
+    M, K = W.shape
+    with torch.cuda.device(W.device):
+        if qweight is None:
+            qweight = torch.empty((M, K * bits // 32), dtype=torch.int32, device=W.device)
+        if scales is None:
+            scales = torch.empty((M, K // 128), dtype=torch.float16, device=W.device)
+        st = lib().hq_quantize(_ptr(W), _DT[W.dtype], M, K, bits, _ptr(signs), _ptr(qweight),
+                               _ptr(scales), _stream(stream))
+    check(st, "hq_quantize")
+    return qweight, scales
+
+
 def make_weight(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
                 bits: int, zero: int | None = None) -> HqWeight:
     M = qweight.shape[0]
@@ -252,6 +273,6 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
-__all__ = ["hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
+__all__ = ["hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
            "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

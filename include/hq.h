@@ -192,6 +192,30 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
 hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, int batch, float* y,
                             hq_stream_t stream);
 
+/*
+ * hq_quantize -- packs real-valued weights W [M][K] into the format above: a
+ * rotated round-to-nearest quantiser (the pages quantise with GPTQ, whose
+ * rounding needs calibration data; this is its data-free counterpart).
+ *   r       = H_K diag(s) W[m] / sqrt(K)                  (computed in fp64)
+ *   scale_g = fp16(min(2 max_{k in g} |r_k| / (2^bits - 1), 65504)),
+ *             g a group of 128 consecutive k (round to nearest even)
+ *   q_k     = clamp(rint(r_k / scale_g) + 2^(bits-1), 0, 2^bits - 1),
+ *             2^(bits-1) where scale_g = 0                 (rint: ties to even)
+ * The result is used as an hq_weight with zero = 2^(bits-1) and the same
+ * signs: then y = dequant(Q) x' approximates W x (the rotation cancels), each
+ * rotated weight within about half a grid step, scale_g / 2.
+ * W: [M][K] of w_dtype (HQ_F16, HQ_BF16 or HQ_F32), row-major, finite values.
+ * qweight: [M][K*bits/32] words, scales: [M][K/128] fp16 bit patterns, both
+ * written whole.  All pointers 16-byte aligned device pointers.  bits 2, 3, 4
+ * or 8; K a power of two in [128, 32768]; M >= 0 (0 launches nothing).
+ * Cites: "group-128 GPTQ in a Hadamard-rotated basis" (LLaDA2.2-mini
+ * Orin-Nano model card, Properties table); weights "behind a random Hadamard
+ * rotation" (Qwen3.8-27B Pingala-8 2-bit card, "What this is").
+ */
+hq_status hq_quantize(const void* W, hq_dtype w_dtype, int M, int K, int bits,
+                      const int8_t* signs, uint32_t* qweight, uint16_t* scales,
+                      hq_stream_t stream);
+
 /* Intermediates an hq_moe_experts call leaves in its workspace, for checking
  * the layer stage by stage:
  *   HQ_MOE_POS  int32 [T*k]: row of pair (t, j) (index t*k + j) in the two
