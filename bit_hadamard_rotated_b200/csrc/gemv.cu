@@ -58,12 +58,14 @@ constexpr int kRows = 16;
 constexpr int kXq = 40;
 // Shared memory after a batch block's zero-point terms: a zero B block (16
 // floats), the per-column output factors 2^(24 - e) (8 floats), the FWHT's
-// per-warp maxima (16 floats).
+// per-warp maxima (16 floats).  The zero-point terms themselves, zq [G][4][4]
+// fp32: for group g and lane quad t, {z(2t), z(2t+1), z(2t), z(2t+1)} with
+// z(n) = -zero sum_k x'_k 2^(e-24) of column n (0 for absent columns), the
+// initial value of the lane's MMA accumulator fragment (rows g and g + 8).
 constexpr int kZcTail = 64 + 32 + 64;
 
 struct GemvParams {
-  CUtensorMap qmap;  // codes as bytes [M][K bits / 8]; box 16 bits bytes x 16 rows
-  CUtensorMap qmap3;  // the same as [G][M][16 bits bytes]; box CH groups x 16 rows (a full slot)
+  CUtensorMap qmap3;  // codes as [G][M][16 bits bytes]; box CH groups x 16 rows (one slot)
   CUtensorMap smap;  // scales as fp16 [M][K/128]; box 8 x 16 rows (K >= 1024 only)
   const uint32_t* q;
   const uint16_t* scales;
@@ -75,9 +77,9 @@ struct GemvParams {
   uint32_t U;       // units = n_tiles * G
   uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
   int zero;
-  const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, zc [G][8] fp32, fac [8] fp32
+  const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, zq [G][16] fp32, fac [8] fp32
   float inv_sqrt_k;
-  int CH, NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
+  int NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
 };
 
 // Batches whose rotation the GEMV CTAs compute themselves (no prep launch):
@@ -86,12 +88,21 @@ struct GemvParams {
 __host__ __device__ constexpr bool gemv_fused_rotation(int K, int nb) { return nb <= 2 && K <= 8192; }
 
 // Bytes of the prep output for a batch block of nb columns (16-byte multiple):
-// the fragments, the zero-point terms [G][8] and the output factors [8].
+// the fragments, the zero-point fragments zq [G][16] and the output factors [8].
 __host__ __device__ constexpr size_t gemv_xs_bytes(int G, int nb) {
   return static_cast<size_t>(G) * nb * 4 * kXq * 2;
 }
+__host__ __device__ constexpr size_t gemv_zq_bytes(int G) { return static_cast<size_t>(G) * 16 * 4; }
 __host__ __device__ constexpr size_t gemv_xg_bytes(int G, int nb) {
-  return gemv_xs_bytes(G, nb) + static_cast<size_t>(G) * 8 * 4 + 8 * 4;
+  return gemv_xs_bytes(G, nb) + gemv_zq_bytes(G) + 8 * 4;
+}
+
+// Groups per ring slot (a "chunk", one 16-row tile): about 4 KiB of codes at
+// 2, 3 and 4 bits (8, 4, 4 groups), 2 groups of 8-bit codes; never more than
+// the G groups of a row.  Slot-shape sweeps on B200 (batch 1) put slots of
+// about 4 KiB at 1.3-2x the rate of many small ones.
+__host__ __device__ constexpr int gemv_ch_max(int bits, int G) {
+  return (bits == 2 ? 8 : bits == 8 ? 2 : 4) < G ? (bits == 2 ? 8 : bits == 8 ? 2 : 4) : G;
 }
 
 // ---------------------------------------------------------------- rotation -> B fragments
@@ -111,15 +122,18 @@ struct FragLane {
   }
 };
 
+// Index in zq of value j (0..3) of lane quad t for group gg.
+__host__ __device__ constexpr int zq_index(int gg, int t, int j) { return (gg * 4 + t) * 4 + j; }
+
 // Group gg of a rotated row (buf: unnormalised fwht_block output): x' 2^e
 // rounded to fp16 (sc = 2^e / sqrt(K)), each value scaled by the 2^-a of its
 // code field, written as column n of the fragment blocks xs [G][nb][4][kXq];
-// zc[gg * 8 + n] = the zero-point term -zero * sum_k x'_k * 2^(e-24) of the
-// group.  One warp per group.
+// the group's zero-point term -zero * sum_k x'_k * 2^(e-24) goes to both
+// places of column n in zq.  One warp per group.
 template <int BITS>
 __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float* buf, int gg, int n,
                                           int nb, float sc, int zero, uint16_t* xs,
-                                          float* zc, int lane) {
+                                          float* zq, int lane) {
   const int s = lane >> 2, t = lane & 3;
   uint16_t hv[4];
   float part = 0.f;
@@ -136,7 +150,18 @@ __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float*
   pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
   pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
   *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * nb + n) * 4 + t) * kXq + s * 4) = pk;
-  if (lane == 0) zc[gg * 8 + n] = -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
+  if (lane < 2) {
+    zq[zq_index(gg, n >> 1, (n & 1) + 2 * lane)] =
+        -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
+  }
+}
+
+// Zero the zero-point terms of the absent columns (N..7) of zq [G][16].
+__device__ __forceinline__ void zq_clear_absent(float* zq, int G, int N, int tid, int nthreads) {
+  for (int i = tid; i < G * 16; i += nthreads) {
+    const int n = 2 * ((i >> 2) & 3) + (i & 1);
+    if (n >= N) zq[i] = 0.f;
+  }
 }
 
 // Prep kernel (batches the GEMV CTAs do not rotate themselves): CTA n rotates
@@ -157,15 +182,14 @@ __global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = blockIdx.x;
   uint16_t* xs = reinterpret_cast<uint16_t*>(xg);
-  float* zc = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
+  float* zq = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
+  float* fac = zq + G * 16;
   float* red = buf + FS::SMEM_FLOATS;  // per-warp maxima of the transform
   const FragLane<BITS> fl(lane);
   const SignMask<FS::E> neg =
       tid < FS::THREADS ? sign_bits<FS::E>(signs ? signs + tid * FS::E : nullptr) : 0u;
   pdl_wait();  // x is the previous kernel's output; xg may still be read by it
-  if (n == 0) {
-    for (int i = tid; i < G * (8 - N); i += kPrepWarps * 32) zc[(i / (8 - N)) * 8 + N + i % (8 - N)] = 0.f;
-  }
+  if (n == 0) zq_clear_absent(zq, G, N, tid, kPrepWarps * 32);
   float v[FS::E];
   if (tid < FS::THREADS) {
     load_chunk<__half, FS::E>(x + static_cast<size_t>(n) * K + tid * FS::E, v);
@@ -173,9 +197,9 @@ __global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const 
   }
   fwht_block<LOGK, prep_logw(LOGK)>(v, buf, red);
   const int e = row_scale_exp(red_max(red, FS::W) * inv_sqrt_k);
-  if (tid == 0) zc[G * 8 + n] = pow2f(24 - e);
+  if (tid == 0) fac[n] = pow2f(24 - e);
   const float sc = inv_sqrt_k * pow2f(e);
-  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, sc, zero, xs, zc, lane);
+  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, sc, zero, xs, zq, lane);
 }
 
 // The FWHT a fused GEMV CTA (16 warps) runs on one row: the 512-thread shape
@@ -193,20 +217,96 @@ template <int LOGK>
 struct FusedFwht<LOGK, false> {
   static constexpr int E = FwhtShape<LOGK, 3>::E, THREADS = FwhtShape<LOGK, 3>::THREADS;
   static __device__ __forceinline__ void run(float (&v)[E], float* buf, float* red) {
-    fwht_block<LOGK, prep_logw(LOGK)>(v, buf, red);
+    fwht_block<LOGK, 3>(v, buf, red);
   }
 };
 
-// Splitting U units into n contiguous ranges: range i is [unit_begin(i), unit_begin(i + 1)).
-__device__ __forceinline__ uint32_t unit_begin(uint32_t i, uint32_t U, uint32_t n) {
-  return static_cast<uint32_t>((static_cast<uint64_t>(i) * U) / n);
+// The CH scales of a lane's row for one chunk, as fp16 bit pairs: CH = 8, 4,
+// 2, 1 -> one 16-, 8-, 4- or 2-byte shared-memory load.
+template <int CH>
+struct ScaleVec {
+  uint32_t h[(CH + 1) / 2];
+  __device__ __forceinline__ void load(const uint8_t* p) {
+    if constexpr (CH == 8) {
+      const uint4 v = *reinterpret_cast<const uint4*>(p);
+      h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
+    } else if constexpr (CH == 4) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      h[0] = v.x; h[1] = v.y;
+    } else if constexpr (CH == 2) {
+      h[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else {
+      h[0] = *reinterpret_cast<const uint16_t*>(p);
+    }
+  }
+  __device__ __forceinline__ float get(int j) const {
+    const uint32_t w = h[j >> 1];
+    return __half2float(__ushort_as_half(static_cast<unsigned short>((j & 1) ? (w >> 16) : (w & 0xFFFFu))));
+  }
+};
+
+// One chunk of a warp: CH groups of one 16-row tile from a full slot.  Per
+// group: the lane's two 32-code bundles (rows g, g + 8) decode into 16 + 16
+// fp16 pairs, 8 MMAs (m16n8k16) run in one chain started at the group's
+// zero-point term, and acc += scale * chain (per row).
+template <int BITS, int CH>
+__device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* sca, const uint8_t* scb,
+                                           const float4* zq4, const uint4* xb, int xs_gstride, int g,
+                                           int t, float (&acc)[4]) {
+  constexpr int GB = 16 * BITS;
+  ScaleVec<CH> sva, svb;
+  sva.load(sca);
+  svb.load(scb);
+  // row g of group j at base + j 16 GB + g GB (row g + 8 at + 8 GB); lane t
+  // owns bytes [4 t BITS, 4 (t + 1) BITS) of the row (8-bit: 16-byte chunks
+  // 2t, 2t + 1 in the 128-byte swizzle, XOR row % 8)
+  const uint8_t* ra = base + g * GB + (BITS == 8 ? 0 : t * 4 * BITS);
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    uint32_t wa[BITS], wb[BITS];
+    if constexpr (BITS == 8) {
+      const int sw = g & 7;
+      const uint4 a0 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + (((2 * t) ^ sw) << 4));
+      const uint4 a1 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + (((2 * t + 1) ^ sw) << 4));
+      const uint4 b0 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + 8 * GB + (((2 * t) ^ sw) << 4));
+      const uint4 b1 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + 8 * GB + (((2 * t + 1) ^ sw) << 4));
+      wa[0] = a0.x; wa[1] = a0.y; wa[2] = a0.z; wa[3] = a0.w;
+      wa[4] = a1.x; wa[5] = a1.y; wa[6] = a1.z; wa[7] = a1.w;
+      wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w;
+      wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
+    } else {
+      load_bundle<BITS>(ra + j * kRows * GB, wa);
+      load_bundle<BITS>(ra + j * kRows * GB + 8 * GB, wb);
+    }
+    const float4 z = zq4[j * 4];
+    uint4 bq[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) bq[i] = xb[j * xs_gstride + i];
+    uint32_t Pa[16], Pb[16];
+    decode16<BITS>(wa, Pa);
+    decode16<BITS>(wb, Pb);
+    float c[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      const uint32_t b0 = (s & 1) ? bq[s >> 1].z : bq[s >> 1].x;
+      const uint32_t b1 = (s & 1) ? bq[s >> 1].w : bq[s >> 1].y;
+      const uint32_t a[4] = {Pa[2 * s], Pb[2 * s], Pa[2 * s + 1], Pb[2 * s + 1]};
+      mma_16816(c, a, b0, b1, c);
+    }
+    const float sa = sva.get(j), sb = svb.get(j);
+    acc[0] = fmaf(sa, c[0], acc[0]);
+    acc[1] = fmaf(sa, c[1], acc[1]);
+    acc[2] = fmaf(sb, c[2], acc[2]);
+    acc[3] = fmaf(sb, c[3], acc[3]);
+  }
 }
 
-template <int BITS, int LOGK, bool FUSED>
+template <int BITS, int LOGK, bool FUSED, int CH>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_constant__ GemvParams p) {
   constexpr int K = 1 << LOGK;
   constexpr int G = K / kGroup;
   constexpr int GB = 16 * BITS;  // bytes of one group of one row
+  static_assert(G % CH == 0 && (G < 8 || 8 % CH == 0), "chunks tile the row and an 8-group scale block");
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   // TMA boxes in the 128-byte swizzle need 1 KiB-aligned slots: round the
   // base up (the launch asks for 1 KiB more than the plan)
@@ -214,29 +314,31 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   // the CTA owns whole tiles, units [cb, ce): the first tr CTAs tq + 1
-  // tiles, the others tq; its warps split them into contiguous ranges (a
-  // tile is never shared with another CTA: a cross-CTA sum would put global
-  // memory round trips at the end of every CTA)
+  // tiles, the others tq; its warps split them into contiguous ranges of
+  // whole chunks (a tile is never shared with another CTA: a cross-CTA sum
+  // would put global memory round trips at the end of every CTA)
   const uint32_t c = blockIdx.x;
   const uint32_t cb = (c * p.tq + min(c, p.tr)) * G;
   const uint32_t ce = cb + (p.tq + (c < p.tr ? 1u : 0u)) * G;
-  const uint32_t cl = ce - cb;
-  const uint32_t u0 = cb + unit_begin(warp, cl, kWarps);
-  const uint32_t u1 = cb + unit_begin(warp + 1, cl, kWarps);
+  const uint32_t nch = (ce - cb) / CH;  // chunks of the CTA
+  auto wbeg = [&](uint32_t w) { return cb + static_cast<uint32_t>((static_cast<uint64_t>(w) * nch) / kWarps) * CH; };
+  const uint32_t u0 = wbeg(warp);
+  const uint32_t u1 = wbeg(warp + 1);
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
-  float* zc = reinterpret_cast<float*>(smem + p.zc_off);
-  float* fac = zc + G * 8 + 16;  // per-column output factors 2^(24 - e)
+  float* zq = reinterpret_cast<float*>(smem + p.zc_off);
+  float* zblk = zq + G * 16;     // a zero B block (16 floats)
+  float* fac = zblk + 16;        // per-column output factors 2^(24 - e)
   uint8_t* ring = smem + p.ring_off + warp * p.NS * p.slot_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off) + warp * p.NS;
-  // slot: [CH groups][16 rows][16 bits bytes] codes (TMA boxes, dense; 8-bit
-  // rows in the 128-byte swizzle), then the scales: K >= 1024: [2 blocks of 8
-  // groups][16 rows][8 halves]; K < 1024: the tile's [16 rows][G halves]
-  const int sc_off = p.CH * kRows * GB;
+  // slot: [CH groups][16 rows][16 bits bytes] codes (one TMA box; 8-bit rows
+  // in the 128-byte swizzle), then the scales: K >= 1024: the tile's [16 rows]
+  // [8 halves] of the aligned block of 8 groups holding the chunk; K < 1024:
+  // the tile's [16 rows][G halves]
+  constexpr int sc_off = CH * kRows * GB;
 
   if (tid == 0) {
     prefetch_tensormap(&p.qmap3);
-    prefetch_tensormap(&p.qmap);
     if constexpr (G >= 8) prefetch_tensormap(&p.smap);
   }
   if (lane == 0) {
@@ -246,26 +348,21 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   __syncthreads();
   pdl_launch_dependents();
 
-  // ---- producer side of the warp's ring (lane 0): one chunk = up to CH
-  // groups of a tile: one TMA box per group of codes, one or two boxes of
-  // scales, all completing on the slot's barrier (rows past M read as zero)
+  // ---- producer side of the warp's ring (lane 0): a chunk is one 3-D TMA
+  // box of codes plus one box (or span) of scales, all completing on the
+  // slot's barrier (rows past M read as zero)
   uint32_t ui = u0;
   int issued = 0;
   auto issue = [&](int slot) {
     const uint32_t tile = ui / G, g0 = ui % G;
-    const uint32_t len = min(static_cast<uint32_t>(p.CH), min(G - g0, u1 - ui));
     const int m0 = tile * kRows;
     uint8_t* base = ring + slot * p.slot_bytes;
     if (lane == 0) {
-      uint32_t bytes = len * kRows * GB;
+      uint32_t bytes = CH * kRows * GB;
       if constexpr (G >= 8) {
-        const uint32_t nblk = (((g0 + len + 7u) & ~7u) - (g0 & ~7u)) / 8u;
-        bytes += nblk * kRows * 16;
+        bytes += kRows * 16;
         mbar_arrive_expect_tx(&bars[slot], bytes);
-        for (uint32_t b = 0; b < nblk; ++b) {
-          tma_load_2d(base + sc_off + b * kRows * 16, &p.smap, static_cast<int>((g0 & ~7u) + 8 * b), m0,
-                      &bars[slot]);
-        }
+        tma_load_2d(base + sc_off, &p.smap, static_cast<int>(g0 & ~7u), m0, &bars[slot]);
       } else {
         // the tile's scales are one contiguous span; bulk-copy its 16-byte
         // multiple, plain-copy the rest (only a last, partial tile has one)
@@ -279,15 +376,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         mbar_arrive_expect_tx(&bars[slot], bytes);
         if (bulk > 0) bulk_g2s(base + sc_off, src, bulk, &bars[slot]);
       }
-      if (len == static_cast<uint32_t>(p.CH)) {
-        tma_load_3d(base, &p.qmap3, 0, m0, static_cast<int>(g0), &bars[slot]);
-      } else {
-        for (uint32_t j = 0; j < len; ++j) {
-          tma_load_2d(base + j * kRows * GB, &p.qmap, static_cast<int>((g0 + j) * GB), m0, &bars[slot]);
-        }
-      }
+      tma_load_3d(base, &p.qmap3, 0, m0, static_cast<int>(g0), &bars[slot]);
     }
-    ui += len;
+    ui += CH;
     ++issued;
   };
   for (int s = 0; s < p.NS && ui < u1; ++s) issue(s);
@@ -303,11 +394,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
         tid < FS::THREADS ? sign_bits<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr) : 0u;
     float* buf = reinterpret_cast<float*>(smem + p.buf_off);
     const FragLane<BITS> fl(lane);
-    for (int i = tid; i < G * 8; i += kWarps * 32) {
-      if ((i & 7) >= p.N) zc[i] = 0.f;  // absent columns
-    }
-    pdl_wait();
+    zq_clear_absent(zq, G, p.N, tid, kWarps * 32);
     float* red = fac + 8;
+    pdl_wait();
     for (int n = 0; n < p.N; ++n) {
       float v[FS::E];
       if (tid < FS::THREADS) {
@@ -319,11 +408,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (tid == 0) fac[n] = pow2f(24 - e);
       const float sc = p.inv_sqrt_k * pow2f(e);
       for (int gg = warp; gg < G; gg += kWarps) {
-        put_group<BITS>(fl, buf, gg, n, p.N, sc, p.zero, xs, zc, lane);
+        put_group<BITS>(fl, buf, gg, n, p.N, sc, p.zero, xs, zq, lane);
       }
-      __syncthreads();  // buf and red are reused by the next row; xs, zc, fac are complete
+      __syncthreads();  // buf and red are reused by the next row; xs, zq, fac are complete
     }
-    if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;  // zero B block
+    if (tid < 16) zblk[tid] = 0.f;
     __syncthreads();
   } else {
     // from the prep kernel
@@ -332,37 +421,38 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     for (int i = tid * 16; i < xs_bytes; i += kWarps * 32 * 16) {
       cp_async16(smem + i, p.xg + i, 16);
     }
-    for (int i = tid * 16; i < G * 8 * 4; i += kWarps * 32 * 16) {
+    for (int i = tid * 16; i < G * 16 * 4; i += kWarps * 32 * 16) {
       cp_async16(smem + p.zc_off + i, p.xg + xs_bytes + i, 16);
     }
-    if (tid < 2) cp_async16(fac + 4 * tid, p.xg + xs_bytes + G * 8 * 4 + 16 * tid, 16);
-    if (tid < 16) reinterpret_cast<float*>(zc + G * 8)[tid] = 0.f;  // zero B block
+    if (tid < 2) cp_async16(fac + 4 * tid, p.xg + xs_bytes + G * 16 * 4 + 16 * tid, 16);
+    if (tid < 16) zblk[tid] = 0.f;
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
   }
 
-  // ---- consumer: decode + MMA over the warp's units
+  // ---- consumer: decode + MMA over the warp's chunks
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   // Tiles this warp covers only in part: its first (0) and last (1), with
-  // their partial sums (scaled by 2^24), kept in registers until the loop
-  // ends and then left in the warp's own (by then idle) ring memory.
+  // their partial sums (scaled to the output), kept in registers until the
+  // loop ends and then left in the warp's own (by then idle) ring memory.
   int ptile0 = -1, ptile1 = -1;
   float4 psum0 = make_float4(0.f, 0.f, 0.f, 0.f), psum1 = psum0;
   int tile_start = -1;
   int consumed = 0;
   bool ok = true;
-  const int N = p.N, M = p.M, ldy = p.ldy, CH = p.CH, NS = p.NS;
+  const int N = p.N, M = p.M, ldy = p.ldy, NS = p.NS;
   const int slot_bytes = p.slot_bytes;
   const bool n0 = 2 * t < N, n1 = 2 * t + 1 < N;
   // lane's B-fragment stream: its column's blocks, or a zero block (stride 0)
   const bool has_b = g < N;
   const uint4* xs_lane = has_b ? reinterpret_cast<const uint4*>(xs + (static_cast<size_t>(g) * 4 + t) * kXq)
-                               : reinterpret_cast<const uint4*>(zc + G * 8);
+                               : reinterpret_cast<const uint4*>(zblk);
   const int xs_gstride = has_b ? N * 4 * kXq / 8 : 0;  // uint4 per group
+  const float4* zq_lane = reinterpret_cast<const float4*>(zq) + t;  // + 4 per group
   const uint32_t first_tile = u0 / G;
-  uint32_t uc = u0;
   // output factors of the lane's columns 2t, 2t + 1 (unused where absent)
   const float f0 = fac[2 * t], f1 = fac[2 * t + 1];
+  uint32_t uc = u0;
 
   auto store_tile = [&](uint32_t tile, const float4& o) {
     const int m0 = tile * kRows;
@@ -380,7 +470,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   uint32_t sph = 0;  // phase parity of the current ring round
   while (uc < u1) {
     const uint32_t tile = uc / G, g0 = uc % G;
-    const uint32_t len = min(static_cast<uint32_t>(CH), min(G - g0, u1 - uc));
     if (!mbar_wait(&bars[slot], sph)) {
       ok = false;
       break;
@@ -388,81 +477,30 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     __syncwarp();
     if (tile_start < 0) tile_start = static_cast<int>(g0);
     const uint8_t* base = ring + slot * slot_bytes;
-    // row g of group j at base + j 16 GB + g GB (row g + 8 at + 8 GB); lane t
-    // owns bytes [4 t BITS, 4 (t + 1) BITS) of the row (8-bit: 16-byte chunks
-    // 2t, 2t + 1 in the 128-byte swizzle, XOR row % 8)
-    const uint8_t* ra = base + g * GB + (BITS == 8 ? 0 : t * 4 * BITS);
     const uint8_t* sc = base + sc_off;
-    const float2* zp = reinterpret_cast<const float2*>(zc + g0 * 8 + 2 * t);
-    const uint4* xb = xs_lane + static_cast<size_t>(g0) * xs_gstride;
-#pragma unroll 1
-    for (uint32_t j = 0; j < len; ++j) {
-      uint32_t wa[BITS], wb[BITS];
-      if constexpr (BITS == 8) {
-        const int sw = g & 7;
-        const uint4 a0 = *reinterpret_cast<const uint4*>(ra + (((2 * t) ^ sw) << 4));
-        const uint4 a1 = *reinterpret_cast<const uint4*>(ra + (((2 * t + 1) ^ sw) << 4));
-        const uint4 b0 = *reinterpret_cast<const uint4*>(ra + 8 * GB + (((2 * t) ^ sw) << 4));
-        const uint4 b1 = *reinterpret_cast<const uint4*>(ra + 8 * GB + (((2 * t + 1) ^ sw) << 4));
-        wa[0] = a0.x; wa[1] = a0.y; wa[2] = a0.z; wa[3] = a0.w;
-        wa[4] = a1.x; wa[5] = a1.y; wa[6] = a1.z; wa[7] = a1.w;
-        wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w;
-        wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
-      } else {
-        load_bundle<BITS>(ra, wa);
-        load_bundle<BITS>(ra + 8 * GB, wb);
-      }
-      ra += kRows * GB;
-      // group scales (the 2^24 subnormal unit is applied once, at the store)
-      float sa, sb;
-      if constexpr (G >= 8) {
-        const uint32_t si = (g0 & 7u) + j;
-        const uint8_t* s0 = sc + (si >> 3) * (kRows * 16) + (si & 7u) * 2;
-        sa = __half2float(*reinterpret_cast<const __half*>(s0 + g * 16));
-        sb = __half2float(*reinterpret_cast<const __half*>(s0 + (g + 8) * 16));
-      } else {
-        const uint8_t* s0 = sc + (g0 + j) * 2;
-        sa = __half2float(*reinterpret_cast<const __half*>(s0 + g * G * 2));
-        sb = __half2float(*reinterpret_cast<const __half*>(s0 + (g + 8) * G * 2));
-      }
-      const float2 z = *zp;
-      zp += 4;
-      uint4 bq[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) bq[i] = xb[i];
-      xb += xs_gstride;
-      uint32_t Pa[16], Pb[16];
-      decode16<BITS>(wa, Pa);
-      decode16<BITS>(wb, Pb);
-      float c0[4] = {z.x, z.y, z.x, z.y}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int s = 0; s < 8; ++s) {
-        const uint32_t b0 = (s & 1) ? bq[s >> 1].z : bq[s >> 1].x;
-        const uint32_t b1 = (s & 1) ? bq[s >> 1].w : bq[s >> 1].y;
-        const uint32_t a[4] = {Pa[2 * s], Pb[2 * s], Pa[2 * s + 1], Pb[2 * s + 1]};
-        if (s & 1) {
-          mma_16816(c1, a, b0, b1, c1);
-        } else {
-          mma_16816(c0, a, b0, b1, c0);
-        }
-      }
-      acc[0] = fmaf(sa, c0[0] + c1[0], acc[0]);
-      acc[1] = fmaf(sa, c0[1] + c1[1], acc[1]);
-      acc[2] = fmaf(sb, c0[2] + c1[2], acc[2]);
-      acc[3] = fmaf(sb, c0[3] + c1[3], acc[3]);
+    const uint8_t* sca;
+    const uint8_t* scb;
+    if constexpr (G >= 8) {
+      sca = sc + g * 16 + (g0 & 7u) * 2;
+      scb = sc + (g + 8) * 16 + (g0 & 7u) * 2;
+    } else {
+      sca = sc + g * G * 2 + g0 * 2;
+      scb = sc + (g + 8) * G * 2 + g0 * 2;
     }
+    gemv_chunk<BITS, CH>(base, sca, scb, zq_lane + g0 * 4, xs_lane + static_cast<size_t>(g0) * xs_gstride,
+                         xs_gstride, g, t, acc);
     __syncwarp();
     if (ui < u1) issue(slot);
-    uc += len;
+    uc += CH;
     ++consumed;
     if (++slot == NS) {
       slot = 0;
       sph ^= 1u;
     }
 
-    if (g0 + len == G || uc >= u1) {
+    if (g0 + CH == G || uc >= u1) {
       // ---- this warp's part of the tile is done
-      const bool full = tile_start == 0 && g0 + len == G;
+      const bool full = tile_start == 0 && g0 + CH == G;
       const float4 o = make_float4(acc[0] * f0, acc[1] * f1, acc[2] * f0, acc[3] * f1);
       if (full) {
         store_tile(tile, o);
@@ -504,9 +542,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (tf < u0) continue;
       float4 o = which == 0 ? psum0 : psum1;
       for (uint32_t w = warp + 1; w < static_cast<uint32_t>(kWarps); ++w) {
-        const uint32_t wb = cb + unit_begin(w, cl, kWarps);
+        const uint32_t wb = wbeg(w);
         if (wb > tz) break;
-        if (wb == cb + unit_begin(w + 1, cl, kWarps)) continue;  // empty range
+        if (wb == wbeg(w + 1)) continue;  // empty range
         const float4 q4 = *sp_slot(w, 0);
         o.x += q4.x;
         o.y += q4.y;
@@ -534,23 +572,17 @@ struct GemvPlan {
 constexpr size_t kMaxSmem = 227 * 1024;
 constexpr int kMaxNS = 4;
 
-// Ring shape, from a sweep of slot shapes on this B200 (batch 1, back-to-back
-// calls): slots of about 4 KiB of codes per warp (16 / bits groups: 8, 4, 4
-// and 2 at 2, 3, 4 and 8 bits) beat many small slots by 1.3-2x, and two to
-// four of them per warp are enough; leaving shared memory for a prep CTA of
-// the next call made no measurable difference.  If no two such slots fit,
-// the slot halves.
 static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t budget) {
   GemvPlan pl;
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
   // the FWHT buffer of a fused rotation: K floats + one pad word per 32
-  const size_t buf_off = (zc_off + static_cast<size_t>(G) * 8 * 4 + kZcTail + 15) & ~static_cast<size_t>(15);
+  const size_t buf_off = (zc_off + gemv_zq_bytes(G) + kZcTail + 15) & ~static_cast<size_t>(15);
   const size_t buf = gemv_fused_rotation(K, nb) ? (static_cast<size_t>(K) + K / 32) * 4 : 0;
   // ring and slots on 1 KiB boundaries (TMA destinations; the 128-byte swizzle atom)
   const size_t ring_off = (buf_off + buf + 1023) & ~static_cast<size_t>(1023);
-  const int sc_bytes = G >= 8 ? 2 * kRows * 16 : ((kRows * G * 2 + 15) & ~15);
+  const int sc_bytes = G >= 8 ? kRows * 16 : ((kRows * G * 2 + 15) & ~15);
   const int slot = (ch * kRows * 16 * bits + sc_bytes + 1023) & ~1023;
   const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * ns * slot;
   // + 1 KiB: the kernel rounds the shared-memory base up to 1 KiB
@@ -567,9 +599,14 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   return pl;
 }
 
+// Chunk lengths the kernels are built for: the full one (gemv_ch_max) and
+// half of it; the deepest ring (2 to 4 slots a warp) of the longer chunk that
+// fits, else of the shorter one.
 static GemvPlan gemv_plan(int bits, int K, int nb) {
   const int G = K / kGroup;
-  for (int ch = std::min(G, 16 / bits >= 8 ? 8 : 16 / bits >= 4 ? 4 : 2); ch >= 1; ch >>= 1) {
+  const int chf = gemv_ch_max(bits, G);
+  for (int ch : {chf, chf > 1 ? chf / 2 : 0}) {
+    if (ch == 0) break;
     for (int ns = kMaxNS; ns >= 2; --ns) {
       const GemvPlan pl = gemv_plan_shape(bits, K, nb, ch, ns, kMaxSmem);
       if (pl.smem != 0) return pl;
@@ -595,32 +632,42 @@ int sm_count() {
   return sms;
 }
 
-template <int BITS, bool FUSED>
-static cudaError_t gemv_launch_f(int K, GemvParams& p, size_t smem, unsigned grid,
-                                 cudaStream_t st) {
+template <int BITS, int LOGK, bool FUSED>
+static cudaError_t gemv_launch_ch(int ch, GemvParams& p, size_t smem, unsigned grid, cudaStream_t st) {
+  constexpr int CHF = gemv_ch_max(BITS, (1 << LOGK) / kGroup);
   const dim3 g(grid), b(kWarps * 32);
+  if (ch == CHF) return launch_pdl(gemv_kernel<BITS, LOGK, FUSED, CHF>, g, b, smem, st, true, p);
+  if constexpr (CHF > 1) {
+    if (ch == CHF / 2) return launch_pdl(gemv_kernel<BITS, LOGK, FUSED, CHF / 2>, g, b, smem, st, true, p);
+  }
+  return cudaErrorInvalidValue;
+}
+
+template <int BITS, bool FUSED>
+static cudaError_t gemv_launch_f(int K, int ch, GemvParams& p, size_t smem, unsigned grid,
+                                 cudaStream_t st) {
   switch (K) {
-    case 128: return launch_pdl(gemv_kernel<BITS, 7, FUSED>, g, b, smem, st, true, p);
-    case 256: return launch_pdl(gemv_kernel<BITS, 8, FUSED>, g, b, smem, st, true, p);
-    case 512: return launch_pdl(gemv_kernel<BITS, 9, FUSED>, g, b, smem, st, true, p);
-    case 1024: return launch_pdl(gemv_kernel<BITS, 10, FUSED>, g, b, smem, st, true, p);
-    case 2048: return launch_pdl(gemv_kernel<BITS, 11, FUSED>, g, b, smem, st, true, p);
-    case 4096: return launch_pdl(gemv_kernel<BITS, 12, FUSED>, g, b, smem, st, true, p);
-    case 8192: return launch_pdl(gemv_kernel<BITS, 13, FUSED>, g, b, smem, st, true, p);
+    case 128: return gemv_launch_ch<BITS, 7, FUSED>(ch, p, smem, grid, st);
+    case 256: return gemv_launch_ch<BITS, 8, FUSED>(ch, p, smem, grid, st);
+    case 512: return gemv_launch_ch<BITS, 9, FUSED>(ch, p, smem, grid, st);
+    case 1024: return gemv_launch_ch<BITS, 10, FUSED>(ch, p, smem, grid, st);
+    case 2048: return gemv_launch_ch<BITS, 11, FUSED>(ch, p, smem, grid, st);
+    case 4096: return gemv_launch_ch<BITS, 12, FUSED>(ch, p, smem, grid, st);
+    case 8192: return gemv_launch_ch<BITS, 13, FUSED>(ch, p, smem, grid, st);
     default:
       if constexpr (!FUSED) {
-        if (K == 16384) return launch_pdl(gemv_kernel<BITS, 14, false>, g, b, smem, st, true, p);
-        if (K == 32768) return launch_pdl(gemv_kernel<BITS, 15, false>, g, b, smem, st, true, p);
+        if (K == 16384) return gemv_launch_ch<BITS, 14, false>(ch, p, smem, grid, st);
+        if (K == 32768) return gemv_launch_ch<BITS, 15, false>(ch, p, smem, grid, st);
       }
       return cudaErrorInvalidValue;
   }
 }
 
 template <int BITS>
-static cudaError_t gemv_launch_b(int K, int nb, GemvParams& p, size_t smem, unsigned grid,
+static cudaError_t gemv_launch_b(int K, int nb, int ch, GemvParams& p, size_t smem, unsigned grid,
                                  cudaStream_t st) {
-  return gemv_fused_rotation(K, nb) ? gemv_launch_f<BITS, true>(K, p, smem, grid, st)
-                                    : gemv_launch_f<BITS, false>(K, p, smem, grid, st);
+  return gemv_fused_rotation(K, nb) ? gemv_launch_f<BITS, true>(K, ch, p, smem, grid, st)
+                                    : gemv_launch_f<BITS, false>(K, ch, p, smem, grid, st);
 }
 
 int gemv_launches(int K, int nb) { return gemv_fused_rotation(K, nb) ? 1 : 2; }
@@ -670,16 +717,11 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   const int G = a.K / kGroup;
   const uint32_t n_tiles = static_cast<uint32_t>((a.M + kRows - 1) / kRows);
   GemvParams p{};
-  // codes as a byte matrix [M][K bits / 8], one box = one group x 16 rows
-  // (8-bit rows are 128 bytes: 128-byte swizzle for conflict-free reads)
   const uint64_t row_bytes = static_cast<uint64_t>(a.K) * a.bits / 8;
-  e = tensor_map_2d(&p.qmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.q, row_bytes, static_cast<uint64_t>(a.M),
-                    row_bytes, static_cast<uint32_t>(16 * a.bits), kRows,
-                    a.bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
-  if (e != cudaSuccess) return e;
   {
-    // the same bytes viewed as [G][M][16 bits] (group stride 16 bits bytes):
+    // the codes viewed as [G][M][16 bits] bytes (group stride 16 bits bytes):
     // one box = a full slot of CH groups x 16 rows, laid out [CH][16][16 bits]
+    // (8-bit rows are 128 bytes: 128-byte swizzle for conflict-free reads)
     const uint64_t gb = 16ull * a.bits;
     const uint64_t dims[3] = {gb, static_cast<uint64_t>(a.M), static_cast<uint64_t>(G)};
     const uint64_t strides[2] = {row_bytes, gb};
@@ -710,7 +752,6 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.U = U;
   p.tq = n_tiles / grid;
   p.tr = n_tiles % grid;
-  p.CH = pl.CH;
   p.NS = pl.NS;
   p.slot_bytes = pl.slot_bytes;
   p.zc_off = pl.zc_off;
@@ -721,10 +762,10 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;
   switch (a.bits) {
-    case 2: return gemv_launch_b<2>(a.K, a.N, p, pl.smem, grid, st);
-    case 3: return gemv_launch_b<3>(a.K, a.N, p, pl.smem, grid, st);
-    case 4: return gemv_launch_b<4>(a.K, a.N, p, pl.smem, grid, st);
-    case 8: return gemv_launch_b<8>(a.K, a.N, p, pl.smem, grid, st);
+    case 2: return gemv_launch_b<2>(a.K, a.N, pl.CH, p, pl.smem, grid, st);
+    case 3: return gemv_launch_b<3>(a.K, a.N, pl.CH, p, pl.smem, grid, st);
+    case 4: return gemv_launch_b<4>(a.K, a.N, pl.CH, p, pl.smem, grid, st);
+    case 8: return gemv_launch_b<8>(a.K, a.N, pl.CH, p, pl.smem, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
