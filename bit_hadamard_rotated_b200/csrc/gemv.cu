@@ -127,12 +127,12 @@ __host__ __device__ constexpr int zq_index(int gg, int t, int j) { return (gg * 
 
 // Group gg of a rotated row (buf: unnormalised fwht_block output): x' 2^e
 // rounded to fp16 (sc = 2^e / sqrt(K)), each value scaled by the 2^-a of its
-// code field, written as column n of the fragment blocks xs [G][nb][4][kXq];
+// code field, written as column n of the fragment blocks xs [nb][G][4][kXq];
 // the group's zero-point term -zero * sum_k x'_k * 2^(e-24) goes to both
 // places of column n in zq.  One warp per group.
 template <int BITS>
 __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float* buf, int gg, int n,
-                                          int nb, float sc, int zero, uint16_t* xs,
+                                          int G, float sc, int zero, uint16_t* xs,
                                           float* zq, int lane) {
   const int s = lane >> 2, t = lane & 3;
   uint16_t hv[4];
@@ -149,7 +149,7 @@ __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float*
   uint2 pk;
   pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
   pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
-  *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(gg) * nb + n) * 4 + t) * kXq + s * 4) = pk;
+  *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(n) * G + gg) * 4 + t) * kXq + s * 4) = pk;
   if (lane < 2) {
     zq[zq_index(gg, n >> 1, (n & 1) + 2 * lane)] =
         -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
@@ -199,7 +199,7 @@ __global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const 
   const int e = row_scale_exp(red_max(red, FS::W) * inv_sqrt_k);
   if (tid == 0) fac[n] = pow2f(24 - e);
   const float sc = inv_sqrt_k * pow2f(e);
-  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, N, sc, zero, xs, zq, lane);
+  for (int gg = warp; gg < G; gg += kPrepWarps) put_group<BITS>(fl, buf, gg, n, G, sc, zero, xs, zq, lane);
 }
 
 // The FWHT a fused GEMV CTA (16 warps) runs on one row: the 512-thread shape
@@ -245,59 +245,88 @@ struct ScaleVec {
   }
 };
 
+// B-fragment blocks (uint4) of one group of one column: 4 k-quads x kXq halves.
+constexpr int kXsGroup = 4 * kXq * 2 / 16;
+
+// The lane's two 32-code bundles (rows g and g + 8) of group j of a slot.
+template <int BITS>
+__device__ __forceinline__ void load_pair_rows(const uint8_t* ra, int j, int g, int t, uint32_t (&wa)[BITS],
+                                               uint32_t (&wb)[BITS]) {
+  constexpr int GB = 16 * BITS;
+  if constexpr (BITS == 8) {
+    const int sw = g & 7;
+    const uint4 a0 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + (((2 * t) ^ sw) << 4));
+    const uint4 a1 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + (((2 * t + 1) ^ sw) << 4));
+    const uint4 b0 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + 8 * GB + (((2 * t) ^ sw) << 4));
+    const uint4 b1 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + 8 * GB + (((2 * t + 1) ^ sw) << 4));
+    wa[0] = a0.x; wa[1] = a0.y; wa[2] = a0.z; wa[3] = a0.w;
+    wa[4] = a1.x; wa[5] = a1.y; wa[6] = a1.z; wa[7] = a1.w;
+    wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w;
+    wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
+  } else {
+    load_bundle<BITS>(ra + j * kRows * GB, wa);
+    load_bundle<BITS>(ra + j * kRows * GB + 8 * GB, wb);
+  }
+}
+
 // One chunk of a warp: CH groups of one 16-row tile from a full slot.  Per
 // group: the lane's two 32-code bundles (rows g, g + 8) decode into 16 + 16
 // fp16 pairs, 8 MMAs (m16n8k16) run in one chain started at the group's
-// zero-point term, and acc += scale * chain (per row).
+// zero-point term, and acc += scale * chain (per row).  Groups are taken two
+// at a time with their chains interleaved, so that each MMA's latency is
+// covered by the other chain's.
 template <int BITS, int CH>
 __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* sca, const uint8_t* scb,
-                                           const float4* zq4, const uint4* xb, int xs_gstride, int g,
-                                           int t, float (&acc)[4]) {
-  constexpr int GB = 16 * BITS;
+                                           const float4* zq4, const uint4* xb, int g, int t,
+                                           float (&acc)[4]) {
+  constexpr int JP = CH >= 2 ? 2 : 1;  // groups in flight
   ScaleVec<CH> sva, svb;
   sva.load(sca);
   svb.load(scb);
   // row g of group j at base + j 16 GB + g GB (row g + 8 at + 8 GB); lane t
   // owns bytes [4 t BITS, 4 (t + 1) BITS) of the row (8-bit: 16-byte chunks
   // 2t, 2t + 1 in the 128-byte swizzle, XOR row % 8)
-  const uint8_t* ra = base + g * GB + (BITS == 8 ? 0 : t * 4 * BITS);
+  const uint8_t* ra = base + g * (16 * BITS) + (BITS == 8 ? 0 : t * 4 * BITS);
 #pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    uint32_t wa[BITS], wb[BITS];
-    if constexpr (BITS == 8) {
-      const int sw = g & 7;
-      const uint4 a0 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + (((2 * t) ^ sw) << 4));
-      const uint4 a1 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + (((2 * t + 1) ^ sw) << 4));
-      const uint4 b0 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + 8 * GB + (((2 * t) ^ sw) << 4));
-      const uint4 b1 = *reinterpret_cast<const uint4*>(ra + j * kRows * GB + 8 * GB + (((2 * t + 1) ^ sw) << 4));
-      wa[0] = a0.x; wa[1] = a0.y; wa[2] = a0.z; wa[3] = a0.w;
-      wa[4] = a1.x; wa[5] = a1.y; wa[6] = a1.z; wa[7] = a1.w;
-      wb[0] = b0.x; wb[1] = b0.y; wb[2] = b0.z; wb[3] = b0.w;
-      wb[4] = b1.x; wb[5] = b1.y; wb[6] = b1.z; wb[7] = b1.w;
-    } else {
-      load_bundle<BITS>(ra + j * kRows * GB, wa);
-      load_bundle<BITS>(ra + j * kRows * GB + 8 * GB, wb);
+  for (int j0 = 0; j0 < CH; j0 += JP) {
+    uint32_t wa[JP][BITS], wb[JP][BITS];
+    uint4 bq[JP][4];
+    float c[JP][4];
+#pragma unroll
+    for (int q = 0; q < JP; ++q) {
+      load_pair_rows<BITS>(ra, j0 + q, g, t, wa[q], wb[q]);
+      const float4 z = zq4[(j0 + q) * 4];
+      c[q][0] = z.x;
+      c[q][1] = z.y;
+      c[q][2] = z.z;
+      c[q][3] = z.w;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) bq[q][i] = xb[(j0 + q) * kXsGroup + i];
     }
-    const float4 z = zq4[j * 4];
-    uint4 bq[4];
+    uint32_t Pa[JP][16], Pb[JP][16];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) bq[i] = xb[j * xs_gstride + i];
-    uint32_t Pa[16], Pb[16];
-    decode16<BITS>(wa, Pa);
-    decode16<BITS>(wb, Pb);
-    float c[4] = {z.x, z.y, z.z, z.w};
+    for (int q = 0; q < JP; ++q) {
+      decode16<BITS>(wa[q], Pa[q]);
+      decode16<BITS>(wb[q], Pb[q]);
+    }
 #pragma unroll
     for (int s = 0; s < 8; ++s) {
-      const uint32_t b0 = (s & 1) ? bq[s >> 1].z : bq[s >> 1].x;
-      const uint32_t b1 = (s & 1) ? bq[s >> 1].w : bq[s >> 1].y;
-      const uint32_t a[4] = {Pa[2 * s], Pb[2 * s], Pa[2 * s + 1], Pb[2 * s + 1]};
-      mma_16816(c, a, b0, b1, c);
+#pragma unroll
+      for (int q = 0; q < JP; ++q) {
+        const uint32_t b0 = (s & 1) ? bq[q][s >> 1].z : bq[q][s >> 1].x;
+        const uint32_t b1 = (s & 1) ? bq[q][s >> 1].w : bq[q][s >> 1].y;
+        const uint32_t a[4] = {Pa[q][2 * s], Pb[q][2 * s], Pa[q][2 * s + 1], Pb[q][2 * s + 1]};
+        mma_16816_acc(c[q], a, b0, b1);
+      }
     }
-    const float sa = sva.get(j), sb = svb.get(j);
-    acc[0] = fmaf(sa, c[0], acc[0]);
-    acc[1] = fmaf(sa, c[1], acc[1]);
-    acc[2] = fmaf(sb, c[2], acc[2]);
-    acc[3] = fmaf(sb, c[3], acc[3]);
+#pragma unroll
+    for (int q = 0; q < JP; ++q) {
+      const float sa = sva.get(j0 + q), sb = svb.get(j0 + q);
+      acc[0] = fmaf(sa, c[q][0], acc[0]);
+      acc[1] = fmaf(sa, c[q][1], acc[1]);
+      acc[2] = fmaf(sb, c[q][2], acc[2]);
+      acc[3] = fmaf(sb, c[q][3], acc[3]);
+    }
   }
 }
 
@@ -327,9 +356,12 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   float* zq = reinterpret_cast<float*>(smem + p.zc_off);
-  float* zblk = zq + G * 16;     // a zero B block (16 floats)
-  float* fac = zblk + 16;        // per-column output factors 2^(24 - e)
-  uint8_t* ring = smem + p.ring_off + warp * p.NS * p.slot_bytes;
+  float* fac = zq + G * 16 + 16;  // per-column output factors 2^(24 - e)
+  // the rings are slot-major: slot s of warp w at (s kWarps + w) slot_bytes,
+  // so the last slot of every warp forms one block (the fused rotation's
+  // FWHT buffer until that slot is first filled)
+  const int ring_stride = kWarps * p.slot_bytes;
+  uint8_t* ring = smem + p.ring_off + warp * p.slot_bytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + p.bar_off) + warp * p.NS;
   // slot: [CH groups][16 rows][16 bits bytes] codes (one TMA box; 8-bit rows
   // in the 128-byte swizzle), then the scales: K >= 1024: the tile's [16 rows]
@@ -356,7 +388,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   auto issue = [&](int slot) {
     const uint32_t tile = ui / G, g0 = ui % G;
     const int m0 = tile * kRows;
-    uint8_t* base = ring + slot * p.slot_bytes;
+    uint8_t* base = ring + slot * ring_stride;
     if (lane == 0) {
       uint32_t bytes = CH * kRows * GB;
       if constexpr (G >= 8) {
@@ -381,7 +413,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     ui += CH;
     ++issued;
   };
-  for (int s = 0; s < p.NS && ui < u1; ++s) issue(s);
+  // all slots now, or (fused rotation) all but the last, whose memory the
+  // rotation uses first
+  for (int s = 0; s < (FUSED ? p.NS - 1 : p.NS) && ui < u1; ++s) issue(s);
 
   // ---- the rotated activations and zero-point terms
   if constexpr (FUSED) {
@@ -392,7 +426,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     // bit e: value e of this thread's chunk flips sign
     const SignMask<FS::E> neg =
         tid < FS::THREADS ? sign_bits<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr) : 0u;
-    float* buf = reinterpret_cast<float*>(smem + p.buf_off);
+    float* buf = reinterpret_cast<float*>(smem + p.ring_off + (p.NS - 1) * ring_stride);
     const FragLane<BITS> fl(lane);
     zq_clear_absent(zq, G, p.N, tid, kWarps * 32);
     float* red = fac + 8;
@@ -408,12 +442,15 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       if (tid == 0) fac[n] = pow2f(24 - e);
       const float sc = p.inv_sqrt_k * pow2f(e);
       for (int gg = warp; gg < G; gg += kWarps) {
-        put_group<BITS>(fl, buf, gg, n, p.N, sc, p.zero, xs, zq, lane);
+        put_group<BITS>(fl, buf, gg, n, G, sc, p.zero, xs, zq, lane);
       }
+      // buf becomes a TMA destination after the loop: order this thread's
+      // accesses to it before that copy (generic -> async proxy)
+      fence_proxy_async_smem();
       __syncthreads();  // buf and red are reused by the next row; xs, zq, fac are complete
     }
-    if (tid < 16) zblk[tid] = 0.f;
-    __syncthreads();
+    if (ui < u1) issue(p.NS - 1);  // the FWHT buffer is free: the warp's last slot
+
   } else {
     // from the prep kernel
     pdl_wait();
@@ -425,7 +462,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       cp_async16(smem + p.zc_off + i, p.xg + xs_bytes + i, 16);
     }
     if (tid < 2) cp_async16(fac + 4 * tid, p.xg + xs_bytes + G * 16 * 4 + 16 * tid, 16);
-    if (tid < 16) zblk[tid] = 0.f;
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
   }
@@ -441,13 +477,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   int consumed = 0;
   bool ok = true;
   const int N = p.N, M = p.M, ldy = p.ldy, NS = p.NS;
-  const int slot_bytes = p.slot_bytes;
   const bool n0 = 2 * t < N, n1 = 2 * t + 1 < N;
-  // lane's B-fragment stream: its column's blocks, or a zero block (stride 0)
-  const bool has_b = g < N;
-  const uint4* xs_lane = has_b ? reinterpret_cast<const uint4*>(xs + (static_cast<size_t>(g) * 4 + t) * kXq)
-                               : reinterpret_cast<const uint4*>(zblk);
-  const int xs_gstride = has_b ? N * 4 * kXq / 8 : 0;  // uint4 per group
+  // lane's B-fragment stream: its column's blocks; lanes of absent columns
+  // read column 0's (their output columns of the MMA are never stored, and a
+  // column of the product depends on that column of B alone)
+  const uint4* xs_lane = reinterpret_cast<const uint4*>(xs + (static_cast<size_t>(g < N ? g : 0) * G * 4 + t) * kXq);
   const float4* zq_lane = reinterpret_cast<const float4*>(zq) + t;  // + 4 per group
   const uint32_t first_tile = u0 / G;
   // output factors of the lane's columns 2t, 2t + 1 (unused where absent)
@@ -476,7 +510,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     }
     __syncwarp();
     if (tile_start < 0) tile_start = static_cast<int>(g0);
-    const uint8_t* base = ring + slot * slot_bytes;
+    const uint8_t* base = ring + slot * ring_stride;
     const uint8_t* sc = base + sc_off;
     const uint8_t* sca;
     const uint8_t* scb;
@@ -487,8 +521,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       sca = sc + g * G * 2 + g0 * 2;
       scb = sc + (g + 8) * G * 2 + g0 * 2;
     }
-    gemv_chunk<BITS, CH>(base, sca, scb, zq_lane + g0 * 4, xs_lane + static_cast<size_t>(g0) * xs_gstride,
-                         xs_gstride, g, t, acc);
+    gemv_chunk<BITS, CH>(base, sca, scb, zq_lane + g0 * 4, xs_lane + g0 * kXsGroup, g, t, acc);
     __syncwarp();
     if (ui < u1) issue(slot);
     uc += CH;
@@ -519,10 +552,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   }
   // ---- tiles split between warps: the first contributing warp adds the
   // CTA's partials in warp order (shared memory) and stores the tile.
-  // Partial slots: the first 1 KiB of each warp's ring (its copies have all
-  // been consumed).
+  // Partial sums: the first 512 bytes of the warp's slots 0 and 1 (a slot is
+  // at least 640 bytes; the warp's copies have all been consumed).
   auto sp_slot = [&](uint32_t w, int which) {
-    return reinterpret_cast<float4*>(smem + p.ring_off + w * p.NS * p.slot_bytes) + which * 32 + lane;
+    return reinterpret_cast<float4*>(smem + p.ring_off + which * ring_stride + w * p.slot_bytes) + lane;
   };
   if (ok) {
     *sp_slot(warp, 0) = psum0;
@@ -577,13 +610,19 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
   const size_t zc_off = (xs + 15) & ~static_cast<size_t>(15);
-  // the FWHT buffer of a fused rotation: K floats + one pad word per 32
-  const size_t buf_off = (zc_off + gemv_zq_bytes(G) + kZcTail + 15) & ~static_cast<size_t>(15);
-  const size_t buf = gemv_fused_rotation(K, nb) ? (static_cast<size_t>(K) + K / 32) * 4 : 0;
-  // ring and slots on 1 KiB boundaries (TMA destinations; the 128-byte swizzle atom)
-  const size_t ring_off = (buf_off + buf + 1023) & ~static_cast<size_t>(1023);
+  // ring on a 1 KiB boundary; slots on 1 KiB (8-bit: the 128-byte swizzle
+  // atom) or 128-byte boundaries (TMA destinations)
+  const size_t ring_off = (zc_off + gemv_zq_bytes(G) + kZcTail + 1023) & ~static_cast<size_t>(1023);
   const int sc_bytes = G >= 8 ? kRows * 16 : ((kRows * G * 2 + 15) & ~15);
-  const int slot = (ch * kRows * 16 * bits + sc_bytes + 1023) & ~1023;
+  const int align = bits == 8 ? 1024 : 128;
+  const int slot = (ch * kRows * 16 * bits + sc_bytes + align - 1) & ~(align - 1);
+  // a fused rotation's FWHT buffer (K floats + one pad word per 32) is the
+  // last slot of every warp, before that slot is first filled
+  if (gemv_fused_rotation(K, nb) &&
+      static_cast<size_t>(kWarps) * slot < (static_cast<size_t>(K) + K / 32) * 4 + 16 * 4) {
+    return pl;
+  }
+  const size_t buf_off = ring_off + static_cast<size_t>(kWarps) * (ns - 1) * slot;
   const size_t bar_off = ring_off + static_cast<size_t>(kWarps) * ns * slot;
   // + 1 KiB: the kernel rounds the shared-memory base up to 1 KiB
   const size_t smem = bar_off + static_cast<size_t>(kWarps) * ns * 8 + 1024;
