@@ -53,16 +53,20 @@ constexpr int kWarps = 16;
 __host__ __device__ constexpr int prep_warps(int logk) { return logk >= 15 ? 32 : 8; }
 __host__ __device__ constexpr int prep_logw(int logk) { return logk >= 15 ? 5 : 3; }
 constexpr int kRows = 16;
-// halves per (group, column, k-quad) block of B fragments: 8 steps x 4, padded
-// to 80 bytes so the 16-byte loads of 8 lanes hit distinct banks
-constexpr int kXq = 40;
-// Shared memory after a batch block's zero-point terms: a zero B block (16
-// floats), the per-column output factors 2^(24 - e) (8 floats), the FWHT's
-// per-warp maxima (16 floats).  The zero-point terms themselves, zq [G][4][4]
+// B fragments of one column: per 128-code group 4 blocks (one per k-quad t)
+// of 64 bytes = 8 MMA steps x 4 fp16 activations; inside block t the four
+// 16-byte pieces are rotated by t (piece i at position (i + t) & 3), and
+// columns are kXsCol bytes apart (an odd multiple of 64 past G * 256), so that
+// the 16-byte loads of a quarter warp (two columns x four k-quads) hit eight
+// different bank groups.
+constexpr int kXsBlock = 64;
+__host__ __device__ constexpr size_t gemv_xs_col(int G) { return static_cast<size_t>(G) * 4 * kXsBlock + 64; }
+// Shared memory after a batch block's zero-point terms: the per-column output
+// factors 2^(24 - e) (8 floats) and the FWHT's per-warp maxima (16 floats).  The zero-point terms themselves, zq [G][4][4]
 // fp32: for group g and lane quad t, {z(2t), z(2t+1), z(2t), z(2t+1)} with
 // z(n) = -zero sum_k x'_k 2^(e-24) of column n (0 for absent columns), the
 // initial value of the lane's MMA accumulator fragment (rows g and g + 8).
-constexpr int kZcTail = 64 + 32 + 64;
+constexpr int kZcTail = 32 + 64;
 
 struct GemvParams {
   CUtensorMap qmap3;  // codes as [G][M][16 bits bytes]; box CH groups x 16 rows (one slot)
@@ -77,7 +81,7 @@ struct GemvParams {
   uint32_t U;       // units = n_tiles * G
   uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
   int zero;
-  const uint8_t* xg;  // prep output: x' fragments [G][N][4][kXq] fp16, zq [G][16] fp32, fac [8] fp32
+  const uint8_t* xg;  // prep output: x' fragments [N][G][4][64 B] fp16, zq [G][16] fp32, fac [8] fp32
   float inv_sqrt_k;
   int NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
 };
@@ -90,7 +94,7 @@ __host__ __device__ constexpr bool gemv_fused_rotation(int K, int nb) { return n
 // Bytes of the prep output for a batch block of nb columns (16-byte multiple):
 // the fragments, the zero-point fragments zq [G][16] and the output factors [8].
 __host__ __device__ constexpr size_t gemv_xs_bytes(int G, int nb) {
-  return static_cast<size_t>(G) * nb * 4 * kXq * 2;
+  return static_cast<size_t>(nb) * gemv_xs_col(G);
 }
 __host__ __device__ constexpr size_t gemv_zq_bytes(int G) { return static_cast<size_t>(G) * 16 * 4; }
 __host__ __device__ constexpr size_t gemv_xg_bytes(int G, int nb) {
@@ -127,7 +131,7 @@ __host__ __device__ constexpr int zq_index(int gg, int t, int j) { return (gg * 
 
 // Group gg of a rotated row (buf: unnormalised fwht_block output): x' 2^e
 // rounded to fp16 (sc = 2^e / sqrt(K)), each value scaled by the 2^-a of its
-// code field, written as column n of the fragment blocks xs [nb][G][4][kXq];
+// code field, written as column n of the fragment blocks (xs, kXsBlock layout);
 // the group's zero-point term -zero * sum_k x'_k * 2^(e-24) goes to both
 // places of column n in zq.  One warp per group.
 template <int BITS>
@@ -149,7 +153,8 @@ __device__ __forceinline__ void put_group(const FragLane<BITS>& fl, const float*
   uint2 pk;
   pk.x = hv[0] | (static_cast<uint32_t>(hv[1]) << 16);
   pk.y = hv[2] | (static_cast<uint32_t>(hv[3]) << 16);
-  *reinterpret_cast<uint2*>(xs + ((static_cast<size_t>(n) * G + gg) * 4 + t) * kXq + s * 4) = pk;
+  *reinterpret_cast<uint2*>(reinterpret_cast<uint8_t*>(xs) + n * gemv_xs_col(G) + (gg * 4 + t) * kXsBlock +
+                            ((((s >> 1) + t) & 3) << 4) + (s & 1) * 8) = pk;
   if (lane < 2) {
     zq[zq_index(gg, n >> 1, (n & 1) + 2 * lane)] =
         -static_cast<float>(zero) * part * 5.9604644775390625e-8f;
@@ -245,8 +250,8 @@ struct ScaleVec {
   }
 };
 
-// B-fragment blocks (uint4) of one group of one column: 4 k-quads x kXq halves.
-constexpr int kXsGroup = 4 * kXq * 2 / 16;
+// Bytes of B fragments of one group of one column.
+constexpr int kXsGroup = 4 * kXsBlock;
 
 // The lane's two 32-code bundles (rows g and g + 8) of group j of a slot.
 template <int BITS>
@@ -277,7 +282,7 @@ __device__ __forceinline__ void load_pair_rows(const uint8_t* ra, int j, int g, 
 // covered by the other chain's.
 template <int BITS, int CH>
 __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* sca, const uint8_t* scb,
-                                           const float4* zq4, const uint4* xb, int g, int t,
+                                           const float4* zq4, const uint8_t* const (&xb)[4], int g, int t,
                                            float (&acc)[4]) {
   constexpr int JP = CH >= 2 ? 2 : 1;  // groups in flight
   ScaleVec<CH> sva, svb;
@@ -301,7 +306,7 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* s
       c[q][2] = z.z;
       c[q][3] = z.w;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) bq[q][i] = xb[(j0 + q) * kXsGroup + i];
+      for (int i = 0; i < 4; ++i) bq[q][i] = *reinterpret_cast<const uint4*>(xb[i] + (j0 + q) * kXsGroup);
     }
     uint32_t Pa[JP][16], Pb[JP][16];
 #pragma unroll
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
 
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem);
   float* zq = reinterpret_cast<float*>(smem + p.zc_off);
-  float* fac = zq + G * 16 + 16;  // per-column output factors 2^(24 - e)
+  float* fac = zq + G * 16;  // per-column output factors 2^(24 - e)
   // the rings are slot-major: slot s of warp w at (s kWarps + w) slot_bytes,
   // so the last slot of every warp forms one block (the fused rotation's
   // FWHT buffer until that slot is first filled)
@@ -481,7 +486,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   // lane's B-fragment stream: its column's blocks; lanes of absent columns
   // read column 0's (their output columns of the MMA are never stored, and a
   // column of the product depends on that column of B alone)
-  const uint4* xs_lane = reinterpret_cast<const uint4*>(xs + (static_cast<size_t>(g < N ? g : 0) * G * 4 + t) * kXq);
+  const uint8_t* xs_lane = reinterpret_cast<const uint8_t*>(xs) + (g < N ? g : 0) * gemv_xs_col(G) + t * kXsBlock;
+  const int rot[4] = {(t & 3) << 4, ((t + 1) & 3) << 4, ((t + 2) & 3) << 4, ((t + 3) & 3) << 4};
   const float4* zq_lane = reinterpret_cast<const float4*>(zq) + t;  // + 4 per group
   const uint32_t first_tile = u0 / G;
   // output factors of the lane's columns 2t, 2t + 1 (unused where absent)
@@ -521,7 +527,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       sca = sc + g * G * 2 + g0 * 2;
       scb = sc + (g + 8) * G * 2 + g0 * 2;
     }
-    gemv_chunk<BITS, CH>(base, sca, scb, zq_lane + g0 * 4, xs_lane + g0 * kXsGroup, g, t, acc);
+    const uint8_t* const xb[4] = {xs_lane + g0 * kXsGroup + rot[0], xs_lane + g0 * kXsGroup + rot[1],
+                                  xs_lane + g0 * kXsGroup + rot[2], xs_lane + g0 * kXsGroup + rot[3]};
+    gemv_chunk<BITS, CH>(base, sca, scb, zq_lane + g0 * 4, xb, g, t, acc);
     __syncwarp();
     if (ui < u1) issue(slot);
     uc += CH;
