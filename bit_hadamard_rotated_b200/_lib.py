@@ -83,6 +83,8 @@ def lib() -> ctypes.CDLL:
         L.hq_moe_workspace_offset.restype = _sz
         L.hq_moe_launches.argtypes = []
         L.hq_moe_launches.restype = _i
+        L.hq_set_test_fault.argtypes = [_i]
+        L.hq_set_test_fault.restype = _i
         L.hq_set_tc_min_batch.argtypes = [_i]
         L.hq_set_tc_min_batch.restype = _i
         _lib = L

@@ -81,6 +81,7 @@ struct GemvParams {
   uint32_t U;       // units = n_tiles * G
   uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
   int zero;
+  int withhold;  // test of the error path: CTA 0's last warp never requests its second chunk
   const uint8_t* xg;  // prep output: x' fragments [N][G][4][64 B] fp16, zq [G][16] fp32, fac [8] fp32
   float inv_sqrt_k;
   int NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
@@ -447,11 +448,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   // slot's barrier (rows past M read as zero)
   uint32_t ui = u0;
   int issued = 0;
+  // a chunk whose copy was never requested (hq_set_test_fault): its wait runs
+  // out and is not drained
+  const int withheld = (p.withhold && blockIdx.x == 0 && warp == kWarps - 1) ? 1 : -1;
   auto issue = [&](int slot) {
     const uint32_t tile = ui / G, g0 = ui % G;
     const int m0 = tile * kRows;
     uint8_t* base = ring + slot * ring_stride;
-    if (lane == 0) {
+    if (lane == 0 && issued != withheld) {
       uint32_t bytes = CH * kRows * GB;
       if constexpr (G >= 8) {
         bytes += kRows * 16;
@@ -653,7 +657,9 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   if (!ok) {
     if (lane == 0) record_error(p.status, HQ_DEV_TIMEOUT);
     // Let copies still in flight land before the CTA's shared memory is released.
-    for (int k = consumed; k < issued; ++k) (void)mbar_wait(&bars[k % p.NS], (k / p.NS) & 1);
+    for (int k = consumed; k < issued; ++k) {
+      if (k != withheld) (void)mbar_wait(&bars[k % p.NS], (k / p.NS) & 1);
+    }
   }
 }
 
@@ -861,6 +867,7 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = a.zero;
+  p.withhold = take_test_fault() ? 1 : 0;
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;
   switch (a.bits) {

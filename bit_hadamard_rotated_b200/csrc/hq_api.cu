@@ -15,6 +15,17 @@ static std::atomic<int> g_tc_min_batch{0};
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+// GEMV launches that still have to withhold one copy (hq_set_test_fault).
+static std::atomic<int> g_test_faults{0};
+
+bool take_test_fault() {
+  int n = g_test_faults.load(std::memory_order_relaxed);
+  while (n > 0) {
+    if (g_test_faults.compare_exchange_weak(n, n - 1, std::memory_order_relaxed)) return true;
+  }
+  return false;
+}
+
 static bool aligned(const void* p, uintptr_t a) {
   return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0;
 }
@@ -116,6 +127,11 @@ const char* hq_status_string(hq_status s) {
 }
 
 uint64_t hq_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int hq_set_test_fault(int n) {
+  if (n < 0) return g_test_faults.load();
+  return g_test_faults.exchange(n);
+}
 
 int hq_set_tc_min_batch(int n) {
   if (n < 0) return g_tc_min_batch.load();

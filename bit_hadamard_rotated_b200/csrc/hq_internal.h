@@ -20,6 +20,8 @@ enum : uint32_t {
 
 // Counts every kernel launch libhq enqueues (hq_launch_count).
 void note_launch();
+// True (and one fewer pending) if hq_set_test_fault asked for a withheld copy.
+bool take_test_fault();
 
 cudaError_t launch_rotate(hq_dtype id, hq_dtype od, const void* x, void* out, int n_rows, int K,
                           const int8_t* signs, cudaStream_t st);

@@ -281,6 +281,16 @@ int hq_linear_uses_tensor_cores(const hq_weight* w, int batch);
  * Returns the previous value; negative values change nothing. */
 int hq_set_tc_min_batch(int n);
 
+/* For tests of the device error path (no counterpart on the pages): the next
+ * n launches of the small-batch GEMV kernel each leave one shared-memory copy
+ * of CTA 0's last warp unrequested (its second chunk: a launch where that warp
+ * has fewer than two chunks withholds nothing), so that warp's bounded wait runs out
+ * (after about one second) and records HQ_ERR_TIMEOUT in the status word
+ * (hq_check_status, hq_linear_noalloc_check_status); that call's outputs are
+ * then incomplete.  Nothing faults and the context stays usable.  Returns the
+ * previous count; n < 0 only reads it. */
+int hq_set_test_fault(int n);
+
 #ifdef __cplusplus
 }
 #endif
