@@ -66,8 +66,8 @@ def lib():
             L.hqo_fwht.argtypes = [vp, i]
             L.hqo_rotate.argtypes = [vp, vp, i, vp]
             L.hqo_rotate_f16.argtypes = [vp, vp, i, vp]
-            L.hqo_dequant_dot.argtypes = [i, i, i, i, vp, vp, vp, i, i, i, vp, vp]
-            L.hqo_linear.argtypes = [i, i, i, i, vp, vp, vp, vp, i, i, i, vp, vp]
+            L.hqo_dequant_dot.argtypes = [i, i, i, i, vp, vp, vp, vp, i, i, i, vp, vp]
+            L.hqo_linear.argtypes = [i, i, i, i, vp, vp, vp, vp, vp, i, i, i, vp, vp]
             L.hqo_moe.argtypes = [vp, i, i, i, vp, i, vp, vp, i, vp, vp, i, i, vp, vp, vp]
             L.hqo_f64_to_f16.argtypes = [ctypes.c_double]
             L.hqo_f64_to_f16.restype = ctypes.c_uint16
@@ -164,9 +164,12 @@ def rotate(x, signs=None) -> np.ndarray:
     return out.reshape(x.shape)
 
 
-def dequant_dot(bits, M, K, zero, q, scales, xr, m_begin=0, m_end=None, with_bound=True):
-    """y[n][m] = sum_k scale.(q - zero).xr[n][k] for already-rotated xr [N][K]."""
+def dequant_dot(bits, M, K, zero, q, scales, xr, m_begin=0, m_end=None, with_bound=True,
+                zeros=None):
+    """y[n][m] = sum_k scale.(q - z).xr[n][k] for already-rotated xr [N][K]; z =
+    zeros[m][k/128] (uint8 [M][K/128]) if given, else the scalar zero."""
     q = _c(q, np.uint32)
+    zr = _c(zeros, np.uint8)
     sc = np.ascontiguousarray(scales).view(np.uint16) if np.asarray(scales).dtype == np.float16 \
         else _c(scales, np.uint16)
     xr = _c(xr, np.float64).reshape(-1, K)
@@ -174,12 +177,14 @@ def dequant_dot(bits, M, K, zero, q, scales, xr, m_begin=0, m_end=None, with_bou
     m_end = M if m_end is None else m_end
     y = np.zeros((N, M), np.float64)
     b = np.zeros((N, M), np.float64) if with_bound else None
-    lib().hqo_dequant_dot(bits, M, K, zero, _p(q), _p(sc), _p(xr), N, m_begin, m_end, _p(y), _p(b))
+    lib().hqo_dequant_dot(bits, M, K, zero, _p(zr), _p(q), _p(sc), _p(xr), N, m_begin, m_end, _p(y),
+                          _p(b))
     return (y, b) if with_bound else y
 
 
-def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads=1):
+def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads=1, zeros=None):
     """Full rotated linear in fp64.  x: fp16 [N][K].  Returns (y, bound) float64 [N][M].
+    zeros: per-group zero points uint8 [M][K/128] (else the scalar zero).
 
     threads > 1 splits the output rows across Python threads (the C call
     releases the GIL), each running the unchanged scalar code on its rows.
@@ -187,6 +192,7 @@ def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads
     q = _c(q, np.uint32)
     sc = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
     s = _c(signs, np.int8)
+    zr = _c(zeros, np.uint8)
     x16 = np.ascontiguousarray(x, dtype=np.float16).reshape(-1, K).view(np.uint16)
     N = x16.shape[0]
     m_end = M if m_end is None else m_end
@@ -194,7 +200,7 @@ def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads
     b = np.zeros((N, M), np.float64)
 
     def run(lo, hi):
-        lib().hqo_linear(bits, M, K, zero, _p(q), _p(sc), _p(s), _p(x16), N, lo, hi, _p(y), _p(b))
+        lib().hqo_linear(bits, M, K, zero, _p(zr), _p(q), _p(sc), _p(s), _p(x16), N, lo, hi, _p(y), _p(b))
 
     if threads <= 1:
         run(m_begin, m_end)

@@ -92,9 +92,9 @@ void hqo_rotate_f16(const uint16_t* x, const int8_t* signs, int K,
   free(xd);
 }
 
-void hqo_dequant_dot(int bits, int M, int K, int zero, const uint32_t* q,
-                     const uint16_t* scales, const double* xr, int N,
-                     int m_begin, int m_end, double* y, double* bound) {
+void hqo_dequant_dot(int bits, int M, int K, int zero, const uint8_t* zeros,
+                     const uint32_t* q, const uint16_t* scales, const double* xr,
+                     int N, int m_begin, int m_end, double* y, double* bound) {
   const int G = K / 128;
   const size_t words_per_row = (size_t)K * (size_t)bits / 32;
   uint8_t* codes = (uint8_t*)malloc((size_t)K);
@@ -103,7 +103,8 @@ void hqo_dequant_dot(int bits, int M, int K, int zero, const uint32_t* q,
     hqo_unpack(q + (size_t)m * words_per_row, bits, (size_t)K, codes);
     for (int k = 0; k < K; ++k) {
       double s = hqo_f16_to_f64(scales[(size_t)m * G + k / 128]);
-      w[k] = s * (double)((int)codes[k] - zero);
+      int z = zeros ? (int)zeros[(size_t)m * G + k / 128] : zero;
+      w[k] = s * (double)((int)codes[k] - z);
     }
     for (int n = 0; n < N; ++n) {
       const double* xn = xr + (size_t)n * K;
@@ -121,14 +122,15 @@ void hqo_dequant_dot(int bits, int M, int K, int zero, const uint32_t* q,
   free(codes);
 }
 
-void hqo_linear(int bits, int M, int K, int zero, const uint32_t* q,
-                const uint16_t* scales, const int8_t* signs, const uint16_t* x,
-                int N, int m_begin, int m_end, double* y, double* bound) {
+void hqo_linear(int bits, int M, int K, int zero, const uint8_t* zeros,
+                const uint32_t* q, const uint16_t* scales, const int8_t* signs,
+                const uint16_t* x, int N, int m_begin, int m_end, double* y,
+                double* bound) {
   double* xr = (double*)malloc(sizeof(double) * (size_t)N * (size_t)K);
   for (int n = 0; n < N; ++n) {
     hqo_rotate_f16(x + (size_t)n * K, signs, K, xr + (size_t)n * K);
   }
-  hqo_dequant_dot(bits, M, K, zero, q, scales, xr, N, m_begin, m_end, y,
+  hqo_dequant_dot(bits, M, K, zero, zeros, q, scales, xr, N, m_begin, m_end, y,
                   bound);
   free(xr);
 }
@@ -156,10 +158,10 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
     }
     for (int j = 0; j < k; ++j) {
       const hqo_expert* e = &experts[topk_ids[(size_t)t * k + j]];
-      hqo_dequant_dot(e->bits, inter, hidden, e->zero, e->q_gate, e->s_gate,
-                      xr, 1, 0, inter, g, NULL);
-      hqo_dequant_dot(e->bits, inter, hidden, e->zero, e->q_up, e->s_up, xr,
-                      1, 0, inter, u, NULL);
+      hqo_dequant_dot(e->bits, inter, hidden, e->zero, NULL, e->q_gate,
+                      e->s_gate, xr, 1, 0, inter, g, NULL);
+      hqo_dequant_dot(e->bits, inter, hidden, e->zero, NULL, e->q_up, e->s_up,
+                      xr, 1, 0, inter, u, NULL);
       for (int i = 0; i < inter; ++i) {
         h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
       }
@@ -168,8 +170,8 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
                sizeof(double) * (size_t)inter);
       }
       hqo_rotate(h, s_mid, inter, hr);
-      hqo_dequant_dot(e->bits, hidden, inter, e->zero, e->q_down, e->s_down,
-                      hr, 1, 0, hidden, d, db);
+      hqo_dequant_dot(e->bits, hidden, inter, e->zero, NULL, e->q_down,
+                      e->s_down, hr, 1, 0, hidden, d, db);
       double wj = (double)topk_w[(size_t)t * k + j];
       for (int i = 0; i < hidden; ++i) {
         yt[i] += wj * d[i];

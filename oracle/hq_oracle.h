@@ -64,21 +64,24 @@ void hqo_rotate(const double* x, const int8_t* signs, int K, double* out);
 void hqo_rotate_f16(const uint16_t* x, const int8_t* signs, int K, double* out);
 
 /* Dequantise-and-dot for output rows [m_begin, m_end):
- *   y[n][m]     = sum_k scale[m][k/128] * (q[m][k] - zero) * xr[n][k]
- *   bound[n][m] = sum_k |scale[m][k/128] * (q[m][k] - zero) * xr[n][k]|
+ *   y[n][m]     = sum_k scale[m][k/128] * (q[m][k] - z[m][k/128]) * xr[n][k]
+ *   bound[n][m] = sum_k |scale[m][k/128] * (q[m][k] - z[m][k/128]) * xr[n][k]|
+ * z[m][g] = zeros[m][g] (uint8 [M][K/128], per-group zero points, the GPTQ
+ * form) when zeros is not NULL, else the per-tensor integer `zero`.
  * q: row-major packed codes, K*bits/32 words per row.
  * scales: fp16 bit patterns [M][K/128].  xr: already-rotated inputs [N][K].
  * y, bound: [N][M] (only columns m_begin..m_end-1 are written; bound may be
  * NULL). */
-void hqo_dequant_dot(int bits, int M, int K, int zero, const uint32_t* q,
-                     const uint16_t* scales, const double* xr, int N,
-                     int m_begin, int m_end, double* y, double* bound);
+void hqo_dequant_dot(int bits, int M, int K, int zero, const uint8_t* zeros,
+                     const uint32_t* q, const uint16_t* scales, const double* xr,
+                     int N, int m_begin, int m_end, double* y, double* bound);
 
 /* The whole rotated linear for rows [m_begin, m_end): rotate each of the N
- * fp16 input rows with signs, then hqo_dequant_dot. */
-void hqo_linear(int bits, int M, int K, int zero, const uint32_t* q,
-                const uint16_t* scales, const int8_t* signs, const uint16_t* x,
-                int N, int m_begin, int m_end, double* y, double* bound);
+ * fp16 input rows with signs, then hqo_dequant_dot (zeros as there). */
+void hqo_linear(int bits, int M, int K, int zero, const uint8_t* zeros,
+                const uint32_t* q, const uint16_t* scales, const int8_t* signs,
+                const uint16_t* x, int N, int m_begin, int m_end, double* y,
+                double* bound);
 
 /* One routed expert: three packed linears with a shared bit width. */
 typedef struct {

@@ -249,6 +249,29 @@ def test_linear_equals_explicit_dense_weff(bits, M, K, N):
     assert np.all(np.abs(y) <= b * (1 + 1e-12))
 
 
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_linear_per_group_zeros_equals_dense(bits):
+    """Per-group zero points (the GPTQ form, one uint8 per row and group):
+    the oracle's linear equals x' . (scale (q - z[m][k/128]))^T built densely
+    with numpy, and a constant zeros array equals the scalar zero."""
+    M, K, N = 20, 512, 3
+    d = _mk(bits, M, K, N, 40 + bits)
+    rng = np.random.default_rng(bits)
+    zeros = rng.integers(0, 1 << bits, size=(M, K // 128)).astype(np.uint8)
+    y, b = oracle.linear(bits, M, K, 0, d["q"], d["scales"], d["signs"], d["x"], zeros=zeros)
+    codes = np.stack([np_unpack(d["q"][m], bits, K) for m in range(M)])
+    sc = np.repeat(np.asarray(d["scales"], dtype=np.float16).astype(np.float64), 128, axis=1)
+    Wq = sc * (codes - np.repeat(zeros.astype(np.int64), 128, axis=1))
+    H = scipy.linalg.hadamard(K).astype(np.float64)
+    xr = (H @ (sign_vec(d["signs"], K)[:, None] * d["x"].astype(np.float64).T)).T / np.sqrt(K)
+    assert np.allclose(y, xr @ Wq.T, rtol=1e-12, atol=1e-12)
+    assert np.allclose(b, np.abs(Wq[None] * xr[:, None, :]).sum(axis=2), rtol=1e-12, atol=1e-12)
+    zc = np.full((M, K // 128), d["zero"], np.uint8)
+    y2, b2 = oracle.linear(bits, M, K, 0, d["q"], d["scales"], d["signs"], d["x"], zeros=zc)
+    y3, b3 = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
+    assert np.array_equal(y2, y3) and np.array_equal(b2, b3)
+
+
 def test_linear_row_ranges_compose():
     d = _mk(4, 50, 256, 2, 21)
     y_all, b_all = oracle.linear(4, 50, 256, 8, d["q"], d["scales"], d["signs"], d["x"])
