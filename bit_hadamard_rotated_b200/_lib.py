@@ -25,7 +25,7 @@ _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
 class HqWeight(ctypes.Structure):
     _fields_ = [("bits", _i), ("M", _i), ("K", _i), ("zero", _i),
-                ("qweight", _vp), ("scales", _vp), ("signs", _vp)]
+                ("qweight", _vp), ("scales", _vp), ("signs", _vp), ("zeros", _vp)]
 
 
 class HqExpert(ctypes.Structure):

@@ -62,15 +62,19 @@ constexpr int kRows = 16;
 constexpr int kXsBlock = 64;
 __host__ __device__ constexpr size_t gemv_xs_col(int G) { return static_cast<size_t>(G) * 4 * kXsBlock + 64; }
 // Shared memory after a batch block's zero-point terms: the per-column output
-// factors 2^(24 - e) (8 floats) and the FWHT's per-warp maxima (16 floats).  The zero-point terms themselves, zq [G][4][4]
-// fp32: for group g and lane quad t, {z(2t), z(2t+1), z(2t), z(2t+1)} with
-// z(n) = -zero sum_k x'_k 2^(e-24) of column n (0 for absent columns), the
-// initial value of the lane's MMA accumulator fragment (rows g and g + 8).
+// factors 2^(24 - e) (8 floats) and the FWHT's per-warp maxima (16 floats).
+// The zero-point terms themselves, zq [G][4][4] fp32: for group g and lane
+// quad t, {z(2t), z(2t+1), z(2t), z(2t+1)} with z(n) = -zero sum_k x'_k
+// 2^(e-24) of column n (0 for absent columns), the initial value of the
+// lane's MMA accumulator fragment (rows g and g + 8).  With per-group zero
+// points the factor zero is left out (1) and applied per row and group.
 constexpr int kZcTail = 32 + 64;
 
 struct GemvParams {
   CUtensorMap qmap3;  // codes as [G][M][16 bits bytes]; box CH groups x 16 rows (one slot)
   CUtensorMap smap;  // scales as fp16 [M][K/128]; box 8 x 16 rows (K >= 1024 only)
+  CUtensorMap zmap;  // per-group zero points as uint8 [M][K/128]; box 16 x 16 rows (K >= 2048)
+  const uint8_t* zeros;  // per-group zero points, or nullptr for the scalar zero
   const uint32_t* q;
   const uint16_t* scales;
   const __half* x;
@@ -309,6 +313,28 @@ template <> struct DecodeViews<3> {
   __device__ __forceinline__ uint32_t pair(int p) const { return P[p]; }
 };
 
+// The CH per-group zero points of a lane's row for one chunk (uint8 each):
+// one 8-, 4-, 2- or 1-byte shared-memory load.
+template <int CH>
+struct ZeroVec {
+  uint32_t h[(CH + 3) / 4];
+  __device__ __forceinline__ void load(const uint8_t* p) {
+    if constexpr (CH == 8) {
+      const uint2 v = *reinterpret_cast<const uint2*>(p);
+      h[0] = v.x; h[1] = v.y;
+    } else if constexpr (CH == 4) {
+      h[0] = *reinterpret_cast<const uint32_t*>(p);
+    } else if constexpr (CH == 2) {
+      h[0] = *reinterpret_cast<const uint16_t*>(p);
+    } else {
+      h[0] = *p;
+    }
+  }
+  __device__ __forceinline__ float get(int j) const {
+    return static_cast<float>((h[j >> 2] >> (8 * (j & 3))) & 0xFFu);
+  }
+};
+
 // The lane's two 32-code bundles (rows g and g + 8) of group j of a slot.
 template <int BITS>
 __device__ __forceinline__ void load_pair_rows(const uint8_t* ra, int j, int g, int t, uint32_t (&wa)[BITS],
@@ -338,14 +364,19 @@ __device__ __forceinline__ void load_pair_rows(const uint8_t* ra, int j, int g, 
 // covered by the other chain's, and each MMA's four A registers are masked
 // out of the code words right before it (measured ~5 % faster than decoding
 // a group's 32 registers first).
-template <int BITS, int CH>
+template <int BITS, int CH, bool PGZ>
 __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* sca, const uint8_t* scb,
-                                           const float4* zq4, const uint8_t* const (&xb)[4], int g, int t,
-                                           float (&acc)[4]) {
+                                           const uint8_t* zra, const uint8_t* zrb, const float4* zq4,
+                                           const uint8_t* const (&xb)[4], int g, int t, float (&acc)[4]) {
   constexpr int JP = CH >= 2 ? 2 : 1;  // groups in flight
   ScaleVec<CH> sva, svb;
   sva.load(sca);
   svb.load(scb);
+  ZeroVec<CH> zva, zvb;
+  if constexpr (PGZ) {
+    zva.load(zra);
+    zvb.load(zrb);
+  }
   // row g of group j at base + j 16 GB + g GB (row g + 8 at + 8 GB); lane t
   // owns bytes [4 t BITS, 4 (t + 1) BITS) of the row (8-bit: 16-byte chunks
   // 2t, 2t + 1 in the 128-byte swizzle, XOR row % 8)
@@ -359,10 +390,19 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* s
     for (int q = 0; q < JP; ++q) {
       load_pair_rows<BITS>(ra, j0 + q, g, t, wa[q], wb[q]);
       const float4 z = zq4[(j0 + q) * 4];
-      c[q][0] = z.x;
-      c[q][1] = z.y;
-      c[q][2] = z.z;
-      c[q][3] = z.w;
+      if constexpr (PGZ) {
+        // the group's zero-point term of each row: its zero times -sum x'
+        const float za = zva.get(j0 + q), zb = zvb.get(j0 + q);
+        c[q][0] = za * z.x;
+        c[q][1] = za * z.y;
+        c[q][2] = zb * z.z;
+        c[q][3] = zb * z.w;
+      } else {
+        c[q][0] = z.x;
+        c[q][1] = z.y;
+        c[q][2] = z.z;
+        c[q][3] = z.w;
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) bq[q][i] = *reinterpret_cast<const uint4*>(xb[i] + (j0 + q) * kXsGroup);
     }
@@ -429,12 +469,19 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   // slot: [CH groups][16 rows][16 bits bytes] codes (one TMA box; 8-bit rows
   // in the 128-byte swizzle), then the scales: K >= 1024: the tile's [16 rows]
   // [8 halves] of the aligned block of 8 groups holding the chunk; K < 1024:
-  // the tile's [16 rows][G halves]
+  // the tile's [16 rows][G halves]; then, with per-group zero points, the
+  // zeros: K >= 2048: the tile's [16 rows][16 bytes] of the aligned block of
+  // 16 groups holding the chunk; K < 2048: the tile's [16 rows][G bytes]
   constexpr int sc_off = CH * kRows * GB;
+  constexpr int z_off = sc_off + (G >= 8 ? kRows * 16 : ((kRows * G * 2 + 15) & ~15));
+  const bool pgz = p.zeros != nullptr;
 
   if (tid == 0) {
     prefetch_tensormap(&p.qmap3);
     if constexpr (G >= 8) prefetch_tensormap(&p.smap);
+    if constexpr (G >= 16) {
+      if (pgz) prefetch_tensormap(&p.zmap);
+    }
   }
   if (lane == 0) {
     for (int i = 0; i < p.NS; ++i) mbar_init(&bars[i], 1);
@@ -456,23 +503,46 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     const int m0 = tile * kRows;
     uint8_t* base = ring + slot * ring_stride;
     if (lane == 0 && issued != withheld) {
+      // bytes the slot's barrier expects; plain-copied remainders are written
+      // before the arrival, which releases them to the consumers
       uint32_t bytes = CH * kRows * GB;
+      int s_bulk = 0, z_bulk = 0;
+      const uint8_t* s_src = reinterpret_cast<const uint8_t*>(p.scales) + static_cast<size_t>(m0) * G * 2;
+      const uint8_t* z_src = pgz ? p.zeros + static_cast<size_t>(m0) * G : nullptr;
       if constexpr (G >= 8) {
         bytes += kRows * 16;
-        mbar_arrive_expect_tx(&bars[slot], bytes);
-        tma_load_2d(base + sc_off, &p.smap, static_cast<int>(g0 & ~7u), m0, &bars[slot]);
       } else {
         // the tile's scales are one contiguous span; bulk-copy its 16-byte
         // multiple, plain-copy the rest (only a last, partial tile has one)
         const int span = min(kRows, p.M - m0) * G * 2;
-        const int bulk = span & ~15;
-        bytes += bulk;
-        const uint8_t* src = reinterpret_cast<const uint8_t*>(p.scales) + static_cast<size_t>(m0) * G * 2;
-        for (int i = bulk; i < span; i += 2) {
-          *reinterpret_cast<uint16_t*>(base + sc_off + i) = *reinterpret_cast<const uint16_t*>(src + i);
+        s_bulk = span & ~15;
+        bytes += s_bulk;
+        for (int i = s_bulk; i < span; i += 2) {
+          *reinterpret_cast<uint16_t*>(base + sc_off + i) = *reinterpret_cast<const uint16_t*>(s_src + i);
         }
-        mbar_arrive_expect_tx(&bars[slot], bytes);
-        if (bulk > 0) bulk_g2s(base + sc_off, src, bulk, &bars[slot]);
+      }
+      if (pgz) {
+        if constexpr (G >= 16) {
+          bytes += kRows * 16;
+        } else {
+          const int span = min(kRows, p.M - m0) * G;
+          z_bulk = span & ~15;
+          bytes += z_bulk;
+          for (int i = z_bulk; i < span; ++i) base[z_off + i] = z_src[i];
+        }
+      }
+      mbar_arrive_expect_tx(&bars[slot], bytes);
+      if constexpr (G >= 8) {
+        tma_load_2d(base + sc_off, &p.smap, static_cast<int>(g0 & ~7u), m0, &bars[slot]);
+      } else {
+        if (s_bulk > 0) bulk_g2s(base + sc_off, s_src, s_bulk, &bars[slot]);
+      }
+      if (pgz) {
+        if constexpr (G >= 16) {
+          tma_load_2d(base + z_off, &p.zmap, static_cast<int>(g0 & ~15u), m0, &bars[slot]);
+        } else {
+          if (z_bulk > 0) bulk_g2s(base + z_off, z_src, z_bulk, &bars[slot]);
+        }
       }
       tma_load_3d(base, &p.qmap3, 0, m0, static_cast<int>(g0), &bars[slot]);
     }
@@ -507,7 +577,8 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       const int e = row_scale_exp(red_max(red, FS::THREADS / 32) * p.inv_sqrt_k);
       if (tid == 0) fac[n] = pow2f(24 - e);
       const float sc = p.inv_sqrt_k * pow2f(e);
-      put_groups<BITS, (G + kWarps - 1) / kWarps>(fl, buf, warp, kWarps, n, G, sc, p.zero, xs, zq, lane);
+      put_groups<BITS, (G + kWarps - 1) / kWarps>(fl, buf, warp, kWarps, n, G, sc, pgz ? 1 : p.zero, xs, zq,
+                                                  lane);
       // buf becomes a TMA destination after the loop: order this thread's
       // accesses to it before that copy (generic -> async proxy)
       fence_proxy_async_smem();
@@ -588,7 +659,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     }
     const uint8_t* const xb[4] = {xs_lane + g0 * kXsGroup + rot[0], xs_lane + g0 * kXsGroup + rot[1],
                                   xs_lane + g0 * kXsGroup + rot[2], xs_lane + g0 * kXsGroup + rot[3]};
-    gemv_chunk<BITS, CH>(base, sca, scb, zq_lane + g0 * 4, xb, g, t, acc);
+    if (pgz) {
+      const uint8_t* zr = base + z_off;
+      const uint8_t* zra = G >= 16 ? zr + g * 16 + (g0 & 15u) : zr + g * G + g0;
+      const uint8_t* zrb = G >= 16 ? zr + (g + 8) * 16 + (g0 & 15u) : zr + (g + 8) * G + g0;
+      gemv_chunk<BITS, CH, true>(base, sca, scb, zra, zrb, zq_lane + g0 * 4, xb, g, t, acc);
+    } else {
+      gemv_chunk<BITS, CH, false>(base, sca, scb, nullptr, nullptr, zq_lane + g0 * 4, xb, g, t, acc);
+    }
     __syncwarp();
     if (ui < u1) issue(slot);
     uc += CH;
@@ -674,7 +752,7 @@ struct GemvPlan {
 constexpr size_t kMaxSmem = 227 * 1024;
 constexpr int kMaxNS = 4;
 
-static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t budget) {
+static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, bool pgz, size_t budget) {
   GemvPlan pl;
   const int G = K / kGroup;
   const size_t xs = gemv_xs_bytes(G, nb);
@@ -683,8 +761,9 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
   // atom) or 128-byte boundaries (TMA destinations)
   const size_t ring_off = (zc_off + gemv_zq_bytes(G) + kZcTail + 1023) & ~static_cast<size_t>(1023);
   const int sc_bytes = G >= 8 ? kRows * 16 : ((kRows * G * 2 + 15) & ~15);
+  const int z_bytes = pgz ? (G >= 16 ? kRows * 16 : kRows * G) : 0;
   const int align = bits == 8 ? 1024 : 128;
-  const int slot = (ch * kRows * 16 * bits + sc_bytes + align - 1) & ~(align - 1);
+  const int slot = (ch * kRows * 16 * bits + sc_bytes + z_bytes + align - 1) & ~(align - 1);
   // a fused rotation's FWHT buffer (K floats + one pad word per 32) is the
   // last slot of every warp, before that slot is first filled
   if (gemv_fused_rotation(K, nb) &&
@@ -710,20 +789,20 @@ static GemvPlan gemv_plan_shape(int bits, int K, int nb, int ch, int ns, size_t 
 // Chunk lengths the kernels are built for: the full one (gemv_ch_max) and
 // half of it; the deepest ring (2 to 4 slots a warp) of the longer chunk that
 // fits, else of the shorter one.
-static GemvPlan gemv_plan(int bits, int K, int nb) {
+static GemvPlan gemv_plan(int bits, int K, int nb, bool pgz) {
   const int G = K / kGroup;
   const int chf = gemv_ch_max(bits, G);
   for (int ch : {chf, chf > 1 ? chf / 2 : 0}) {
     if (ch == 0) break;
     for (int ns = kMaxNS; ns >= 2; --ns) {
-      const GemvPlan pl = gemv_plan_shape(bits, K, nb, ch, ns, kMaxSmem);
+      const GemvPlan pl = gemv_plan_shape(bits, K, nb, ch, ns, pgz, kMaxSmem);
       if (pl.smem != 0) return pl;
     }
   }
   return GemvPlan{};
 }
 
-size_t gemv_smem_bytes(int bits, int K, int nb) { return gemv_plan(bits, K, nb).smem; }
+size_t gemv_smem_bytes(int bits, int K, int nb, bool pgz) { return gemv_plan(bits, K, nb, pgz).smem; }
 
 int sm_count() {
   static int sms = 0;
@@ -791,7 +870,7 @@ static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
 #define HQ_PREP(LK)                                                                          \
   launch_pdl(gemv_prep_kernel<BITS, LK>, g, dim3(prep_warps(LK) * 32),                         \
              (FwhtShape<LK, prep_logw(LK)>::SMEM_FLOATS + 32) * sizeof(float), st, true, x, a.signs, \
-             xg, a.N, a.zero, inv)
+             xg, a.N, a.zeros != nullptr ? 1 : a.zero, inv)
   switch (K) {
     case 128: return HQ_PREP(7);
     case 256: return HQ_PREP(8);
@@ -808,7 +887,7 @@ static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
 }
 
 cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
-  const GemvPlan pl = gemv_plan(a.bits, a.K, a.N);
+  const GemvPlan pl = gemv_plan(a.bits, a.K, a.N, a.zeros != nullptr);
   if (pl.smem == 0) return cudaErrorInvalidValue;
   const bool fused = gemv_fused_rotation(a.K, a.N);
   cudaError_t e = cudaSuccess;
@@ -839,6 +918,12 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
                       a.bits == 8 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
     if (e != cudaSuccess) return e;
   }
+  if (a.zeros != nullptr && G >= 16) {  // zeros [M][G] uint8, one box = 16 groups x 16 rows
+    e = tensor_map_2d(&p.zmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.zeros, static_cast<uint64_t>(G),
+                      static_cast<uint64_t>(a.M), static_cast<uint64_t>(G), 16, kRows,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (e != cudaSuccess) return e;
+  }
   if (G >= 8) {  // scales [M][G] fp16, one box = 8 groups x 16 rows
     e = tensor_map_2d(&p.smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, a.scales, static_cast<uint64_t>(G),
                       static_cast<uint64_t>(a.M), static_cast<uint64_t>(G) * 2, 8, kRows,
@@ -867,6 +952,7 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = a.zero;
+  p.zeros = a.zeros;
   p.withhold = take_test_fault() ? 1 : 0;
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;

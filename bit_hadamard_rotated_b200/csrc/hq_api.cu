@@ -52,13 +52,14 @@ static hq_status check_weight(const hq_weight* w) {
   if (w->qweight == nullptr || w->scales == nullptr) return HQ_ERR_INVALID_ARG;
   if (!aligned(w->qweight, 16) || !aligned(w->scales, 16)) return HQ_ERR_INVALID_ARG;
   if (w->signs != nullptr && !aligned(w->signs, 16)) return HQ_ERR_INVALID_ARG;
+  if (w->zeros != nullptr && !aligned(w->zeros, 16)) return HQ_ERR_INVALID_ARG;
   return HQ_OK;
 }
 
 // Largest GEMV batch block whose ring plan fits in one CTA.
-static int gemv_col_block(int bits, int K) {
+static int gemv_col_block(int bits, int K, bool pgz) {
   for (int nb = kMaxColBlock; nb >= 1; nb >>= 1) {
-    if (gemv_smem_bytes(bits, K, nb) != 0) return nb;
+    if (gemv_smem_bytes(bits, K, nb, pgz) != 0) return nb;
   }
   return 0;
 }
@@ -75,7 +76,7 @@ static bool use_tc(const hq_weight* w, int batch) {
     // wins; 2-bit rows and smaller K stay on the GEMV up to batch 8
     min_batch = (w->bits >= 3 && w->K >= 8192) ? 5 : 9;
   }
-  return batch >= min_batch &&
+  return batch >= min_batch && w->zeros == nullptr &&
          tc_col_block(w->bits, w->K) > 0;
 }
 
@@ -95,7 +96,7 @@ struct LinearWs {
 
 static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
-  const int nb = gemv_col_block(w->bits, w->K);
+  const int nb = gemv_col_block(w->bits, w->K, w->zeros != nullptr);
   const size_t xp_bytes = use_tc(w, batch)
                               ? align256(tc_xp_bytes(w->bits, w->K, batch))
                               : align256(gemv_scratch_bytes(w->K, nb > 0 ? std::min(nb, std::max(batch, 1)) : 1));
@@ -168,7 +169,7 @@ int hq_linear_uses_tensor_cores(const hq_weight* w, int batch) {
 int hq_linear_launches(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch <= 0) return 0;
   if (use_tc(w, batch)) return tc_launches(w->bits, w->K, batch);
-  const int nb = gemv_col_block(w->bits, w->K);
+  const int nb = gemv_col_block(w->bits, w->K, w->zeros != nullptr);
   if (nb == 0) return 0;
   int n = 0;
   for (int n0 = 0; n0 < batch; n0 += nb) n += gemv_launches(w->K, std::min(nb, batch - n0));
@@ -206,7 +207,7 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     a.counters = l.counters;
     return from_cuda(launch_linear_tc(a, st));
   }
-  const int nb = gemv_col_block(w->bits, w->K);
+  const int nb = gemv_col_block(w->bits, w->K, w->zeros != nullptr);
   if (nb == 0) return HQ_ERR_UNSUPPORTED;
   for (int n0 = 0; n0 < batch; n0 += nb) {
     GemvArgs a;
@@ -223,6 +224,7 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     a.ldy = w->M;
     a.status = l.status;
     a.xg = l.xp;
+    a.zeros = w->zeros;
     const cudaError_t e = launch_gemv(a, st);
     if (e != cudaSuccess) return from_cuda(e);
   }

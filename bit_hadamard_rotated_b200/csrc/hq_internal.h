@@ -36,11 +36,12 @@ struct GemvArgs {
   int ldy;
   uint32_t* status;
   void* xg;       // gemv_scratch_bytes(K, N) bytes, 16-byte aligned: prep output
+  const uint8_t* zeros = nullptr;  // per-group zero points [M][K/128], or nullptr: zero
 };
 
-// Shared memory the GEMV needs for a batch block of nb <= 8 rows (0 if no
-// ring configuration fits in one CTA).
-size_t gemv_smem_bytes(int bits, int K, int nb);
+// Shared memory the GEMV needs for a batch block of nb <= 8 rows, with or
+// without per-group zero points (0 if no ring configuration fits in one CTA).
+size_t gemv_smem_bytes(int bits, int K, int nb, bool pgz);
 // Scratch for the rotated activations of one GEMV launch of nb <= 8 columns.
 size_t gemv_scratch_bytes(int K, int nb);
 // Streaming multiprocessors of the current device (148 if the query fails).

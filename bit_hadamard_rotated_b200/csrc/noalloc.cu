@@ -70,7 +70,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
   if (!pow2(w->K) || w->K < 128 || w->K > 32768) return HQ_ERR_UNSUPPORTED;
   if (w->zero < 0 || w->zero >= (1 << w->bits)) return HQ_ERR_INVALID_ARG;
   if (!w->qweight || !w->scales || !aligned(w->qweight, 16) || !aligned(w->scales, 16) ||
-      (w->signs && !aligned(w->signs, 16))) {
+      (w->signs && !aligned(w->signs, 16)) || (w->zeros && !aligned(w->zeros, 16))) {
     return HQ_ERR_INVALID_ARG;
   }
   if (batch < 0 || batch > 65535) return HQ_ERR_INVALID_ARG;
@@ -78,7 +78,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
   int nb = 0;
   for (int b = 8; b >= 1 && nb == 0; b >>= 1) {
-    if (gemv_smem_bytes(w->bits, w->K, b) != 0) nb = b;
+    if (gemv_smem_bytes(w->bits, w->K, b, w->zeros != nullptr) != 0) nb = b;
   }
   if (nb == 0) return HQ_ERR_UNSUPPORTED;
   // beyond what the fixed scratch holds (cannot happen for a supported K)
@@ -109,6 +109,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     a.ldy = w->M;
     a.status = reinterpret_cast<uint32_t*>(scratch);
     a.xg = scratch + kStatus;
+    a.zeros = w->zeros;
     if (launch_gemv(a, st) != cudaSuccess) {
       (void)cudaGetLastError();
       return HQ_ERR_CUDA;

@@ -75,12 +75,17 @@ def hq_quantize(W: torch.Tensor, bits: int, signs: torch.Tensor | None = None,
 
 
 def make_weight(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
-                bits: int, zero: int | None = None) -> HqWeight:
+                bits: int, zero: int | None = None, zeros: torch.Tensor | None = None) -> HqWeight:
+    """Weight descriptor; zeros: optional per-group zero points uint8 [M][K/128]."""
     M = qweight.shape[0]
     K = qweight.shape[1] * 32 // bits
     z = (1 << (bits - 1)) if zero is None else int(zero)
+    if zeros is not None and (zeros.dtype != torch.uint8 or tuple(zeros.shape) != (M, K // 128)
+                              or not zeros.is_contiguous()):
+        raise ValueError(f"zeros must be contiguous uint8 [{M}][{K // 128}]")
     return HqWeight(bits, M, K, z, qweight.data_ptr(), scales.data_ptr(),
-                    None if signs is None else signs.data_ptr())
+                    None if signs is None else signs.data_ptr(),
+                    None if zeros is None else zeros.data_ptr())
 
 
 def hq_linear_workspace_size(w: HqWeight, batch: int) -> int:
@@ -106,10 +111,11 @@ def _check_linear_io(w: HqWeight, x: torch.Tensor, out: torch.Tensor | None, dev
 def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
               x: torch.Tensor, bits: int, zero: int | None = None,
               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-              stream=None) -> torch.Tensor:
-    """y[n][m] = sum_k scale (q - zero) x'[n][k]; x fp16 [N][K] -> y fp32 [N][M]."""
-    _need_cuda(qweight, scales, signs, x)
-    w = make_weight(qweight, scales, signs, bits, zero)
+              stream=None, zeros: torch.Tensor | None = None) -> torch.Tensor:
+    """y[n][m] = sum_k scale (q - zero) x'[n][k]; x fp16 [N][K] -> y fp32 [N][M]
+    (zero per tensor, or per row and group with zeros uint8 [M][K/128])."""
+    _need_cuda(qweight, scales, signs, x, zeros)
+    w = make_weight(qweight, scales, signs, bits, zero, zeros)
     _check_linear_io(w, x, out, qweight.device)
     N = x.shape[0]
     with torch.cuda.device(qweight.device):
@@ -126,11 +132,12 @@ def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor |
 
 def hq_linear_noalloc(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
                       x: torch.Tensor, bits: int, zero: int | None = None,
-                      out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                      out: torch.Tensor | None = None, stream=None,
+                      zeros: torch.Tensor | None = None) -> torch.Tensor:
     """hq_linear without a workspace (the library's fixed device scratch is
     used instead; calls must not overlap on the GPU)."""
-    _need_cuda(qweight, scales, signs, x)
-    w = make_weight(qweight, scales, signs, bits, zero)
+    _need_cuda(qweight, scales, signs, x, zeros)
+    w = make_weight(qweight, scales, signs, bits, zero, zeros)
     _check_linear_io(w, x, out, qweight.device)
     N = x.shape[0]
     with torch.cuda.device(qweight.device):
@@ -149,10 +156,10 @@ def hq_linear_noalloc_check_status(stream=None) -> None:
 class RotatedLinear:
     """A packed, rotated linear layer bound to its device tensors and workspace."""
 
-    def __init__(self, qweight, scales, signs, bits, zero=None, max_batch=64):
-        _need_cuda(qweight, scales, signs)
-        self.qweight, self.scales, self.signs, self.bits = qweight, scales, signs, bits
-        self.w = make_weight(qweight, scales, signs, bits, zero)
+    def __init__(self, qweight, scales, signs, bits, zero=None, max_batch=64, zeros=None):
+        _need_cuda(qweight, scales, signs, zeros)
+        self.qweight, self.scales, self.signs, self.bits, self.zeros = qweight, scales, signs, bits, zeros
+        self.w = make_weight(qweight, scales, signs, bits, zero, zeros)
         self.workspace = torch.zeros(max(hq_linear_workspace_size(self.w, max_batch), 256),
                                      dtype=torch.uint8, device=qweight.device)
         # per-call marshalling reduced to the two tensor pointers and the stream

@@ -22,7 +22,8 @@
  *                [32w, 32w+32)).  For bits = 3, three words carry 32 codes and
  *                codes 10 and 21 of each triplet straddle a word boundary.
  *   dequant      w[m][k] = scale[m][k/128] * (q[m][k] - zero), group size 128
- *                along K, scale an IEEE fp16 bit pattern, zero an integer.
+ *                along K, scale an IEEE fp16 bit pattern, zero an integer
+ *                (one per tensor, or one per row and group: hq_weight.zeros).
  *   linear       y[n][m] = sum_k w[m][k] * x'[n][k], fp32 output.
  *
  * Conventions:
@@ -91,6 +92,12 @@ typedef struct {
   const uint32_t* qweight; /* [M][K*bits/32] packed codes, 16-byte aligned */
   const uint16_t* scales;  /* [M][K/128] fp16 bit patterns, 16-byte aligned */
   const int8_t* signs;     /* [K] rotation signs, or NULL for s = 1 */
+  const uint8_t* zeros;    /* [M][K/128] per-group zero points (each < 2^bits), or
+                              NULL: `zero` for every group.  16-byte aligned.  The
+                              per-group form is GPTQ's usual one; with it, every
+                              batch runs the small-batch kernel in blocks of up to
+                              8 columns (the tensor-core path takes the scalar
+                              zero only). */
 } hq_weight;
 
 /*

@@ -49,6 +49,7 @@ class Expert(ctypes.Structure):
         ("bits", ctypes.c_int), ("zero", ctypes.c_int),
         ("q_gate", ctypes.c_void_p), ("q_up", ctypes.c_void_p), ("q_down", ctypes.c_void_p),
         ("s_gate", ctypes.c_void_p), ("s_up", ctypes.c_void_p), ("s_down", ctypes.c_void_p),
+        ("signs_in", ctypes.c_void_p), ("signs_mid", ctypes.c_void_p),
     ]
 
 
@@ -218,7 +219,8 @@ def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads
 def moe(experts, hidden, inter, x, topk_ids, topk_w, s_in, s_mid, t_begin=0, t_end=None,
         want_h=False, threads=1):
     """MoE expert layer in fp64.  experts: list of dicts with keys bits, zero,
-    q_gate, q_up, q_down (uint32 arrays) and s_gate, s_up, s_down (fp16 arrays).
+    q_gate, q_up, q_down (uint32 arrays) and s_gate, s_up, s_down (fp16 arrays),
+    and optionally the expert's own rotation signs signs_in, signs_mid (int8).
     Returns (y [T][hidden], bound [T][hidden], h [T*k][inter] or None)."""
     keep = []
     arr = (Expert * len(experts))()
@@ -226,8 +228,10 @@ def moe(experts, hidden, inter, x, topk_ids, topk_w, s_in, s_mid, t_begin=0, t_e
         qs = [_c(e[n], np.uint32) for n in ("q_gate", "q_up", "q_down")]
         ss = [np.ascontiguousarray(e[n], dtype=np.float16).view(np.uint16)
               for n in ("s_gate", "s_up", "s_down")]
-        keep += qs + ss
-        arr[i] = Expert(int(e["bits"]), int(e["zero"]), *[a.ctypes.data for a in qs + ss])
+        own = [_c(e.get(n), np.int8) for n in ("signs_in", "signs_mid")]
+        keep += qs + ss + [o for o in own if o is not None]
+        arr[i] = Expert(int(e["bits"]), int(e["zero"]), *[a.ctypes.data for a in qs + ss],
+                        *[None if o is None else o.ctypes.data for o in own])
     x16 = np.ascontiguousarray(x, dtype=np.float16).reshape(-1, hidden).view(np.uint16)
     T = x16.shape[0]
     ids = _c(topk_ids, np.int32).reshape(T, -1)

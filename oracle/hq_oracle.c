@@ -148,6 +148,7 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
   double* hr = (double*)malloc(sizeof(double) * (size_t)inter);
   double* d = (double*)malloc(sizeof(double) * (size_t)hidden);
   double* db = (double*)malloc(sizeof(double) * (size_t)hidden);
+  double* xe = (double*)malloc(sizeof(double) * (size_t)hidden);
   for (int t = t_begin; t < t_end; ++t) {
     hqo_rotate_f16(x + (size_t)t * hidden, s_in, hidden, xr);
     double* yt = y + (size_t)t * hidden;
@@ -158,10 +159,16 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
     }
     for (int j = 0; j < k; ++j) {
       const hqo_expert* e = &experts[topk_ids[(size_t)t * k + j]];
+      /* the expert's own input signs rotate the token again */
+      const double* xin = xr;
+      if (e->signs_in) {
+        hqo_rotate_f16(x + (size_t)t * hidden, e->signs_in, hidden, xe);
+        xin = xe;
+      }
       hqo_dequant_dot(e->bits, inter, hidden, e->zero, NULL, e->q_gate,
-                      e->s_gate, xr, 1, 0, inter, g, NULL);
+                      e->s_gate, xin, 1, 0, inter, g, NULL);
       hqo_dequant_dot(e->bits, inter, hidden, e->zero, NULL, e->q_up, e->s_up,
-                      xr, 1, 0, inter, u, NULL);
+                      xin, 1, 0, inter, u, NULL);
       for (int i = 0; i < inter; ++i) {
         h[i] = g[i] / (1.0 + exp(-g[i])) * u[i];
       }
@@ -169,7 +176,7 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
         memcpy(h_out + ((size_t)t * k + j) * inter, h,
                sizeof(double) * (size_t)inter);
       }
-      hqo_rotate(h, s_mid, inter, hr);
+      hqo_rotate(h, e->signs_mid ? e->signs_mid : s_mid, inter, hr);
       hqo_dequant_dot(e->bits, hidden, inter, e->zero, NULL, e->q_down,
                       e->s_down, hr, 1, 0, hidden, d, db);
       double wj = (double)topk_w[(size_t)t * k + j];
@@ -179,6 +186,7 @@ void hqo_moe(const hqo_expert* experts, int n_experts, int hidden, int inter,
       }
     }
   }
+  free(xe);
   free(db);
   free(d);
   free(hr);

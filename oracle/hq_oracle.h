@@ -93,9 +93,12 @@ typedef struct {
   const uint16_t* s_gate; /* [inter][hidden/128] */
   const uint16_t* s_up;   /* [inter][hidden/128] */
   const uint16_t* s_down; /* [hidden][inter/128] */
+  const int8_t* signs_in;  /* [hidden] this expert's own rotation signs, or NULL */
+  const int8_t* signs_mid; /* [inter] likewise for its down projection, or NULL */
 } hqo_expert;
 
-/* MoE expert layer for tokens [t_begin, t_end):
+/* MoE expert layer for tokens [t_begin, t_end) (s_in, s_mid: the expert's
+ * own signs_in / signs_mid where it has them, else the shared vectors):
  *   x'_t   = rot(x_t, s_in)                        (hidden)
  *   g, u   = W_gate^e x'_t, W_up^e x'_t            (inter)
  *   h      = g / (1 + exp(-g)) * u                 (SwiGLU)

@@ -339,3 +339,36 @@ def test_linear_k32768(bits, N):
     y = run_linear(d).cpu().numpy()
     want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"], threads=8)
     assert_within(y, want, bound, what=f"K32768 b{bits} N{N}")
+
+
+# ---------------------------------------------------------------- per-group zero points
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+@pytest.mark.parametrize("M,K,N", [(16, 128, 1), (37, 256, 3), (100, 1024, 2), (257, 2048, 1),
+                                   (333, 4096, 5), (96, 8192, 8), (40, 16384, 2), (300, 4096, 19)])
+def test_linear_per_group_zeros(bits, M, K, N):
+    """Per-group zero points (uint8 [M][K/128], the GPTQ form): the small-batch
+    kernel loads them beside the scales (a TMA box of 16 groups from K = 2048,
+    the tile's span below) and starts each group's accumulator at its own
+    row's zero-point term; batches past 8 run in blocks of 8 columns."""
+    from bit_hadamard_rotated_b200 import hq_linear
+    d = synth.linear(M, K, bits, N, seed=70 + M + K + bits)
+    rng = np.random.default_rng(M + bits)
+    zeros = rng.integers(0, 1 << bits, size=(M, K // 128)).astype(np.uint8)
+    y = hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]), dev(d["x"]), bits,
+                  zeros=dev(zeros)).cpu().numpy()
+    want, bound = oracle.linear(bits, M, K, 0, d["q"], d["scales"], d["signs"], d["x"], zeros=zeros)
+    assert_within(y, want, bound, what=f"zeros b{bits} M{M} K{K} N{N}")
+
+
+def test_linear_per_group_zeros_full_size_sampled():
+    from bit_hadamard_rotated_b200 import hq_linear
+    M, K, bits, N = 28672, 8192, 2, 1
+    d = synth.linear(M, K, bits, N, seed=5, scale_dist="loguniform", outlier_frac=0.01)
+    zeros = np.random.default_rng(3).integers(0, 4, size=(M, K // 128)).astype(np.uint8)
+    y = hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]), dev(d["x"]), bits,
+                  zeros=dev(zeros)).cpu().numpy()
+    rng = np.random.default_rng(7)
+    for m in sample_rows(M, rng):
+        want, bound = oracle.linear(bits, M, K, 0, d["q"], d["scales"], d["signs"], d["x"], m_begin=m,
+                                    m_end=m + 1, zeros=zeros)
+        assert_within(y[:, m], want[:, m], bound[:, m], what=f"row {m}")

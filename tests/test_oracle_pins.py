@@ -285,6 +285,8 @@ def _small_moe(seed, E=6, hidden=256, inter=128, T=5, k=2, probs=(0.4, 0.3, 0.3)
 
 
 def _dense_expert_chain(e, x_row, s_in, s_mid, hidden, inter):
+    s_in = e.get("signs_in", s_in) if e.get("signs_in") is not None else s_in
+    s_mid = e.get("signs_mid", s_mid) if e.get("signs_mid") is not None else s_mid
     _, Wg = dense_weff(e["q_gate"], e["s_gate"], e["bits"], e["zero"], inter, hidden, s_in)
     _, Wu = dense_weff(e["q_up"], e["s_up"], e["bits"], e["zero"], inter, hidden, s_in)
     _, Wd = dense_weff(e["q_down"], e["s_down"], e["bits"], e["zero"], hidden, inter, s_mid)
@@ -361,6 +363,31 @@ def test_moe_bound_base_for_several_slots():
             assert np.allclose(b[t], want, rtol=1e-12, atol=1e-14)
             assert np.allclose(y[t], want_y, rtol=1e-11, atol=1e-12)
             assert np.all(np.abs(y[t]) <= b[t] * (1 + 1e-12))
+
+
+def test_moe_per_expert_signs_equals_dense_chain():
+    """Experts with their own rotation signs (some with signs_in, some with
+    signs_mid, some with both, the rest on the shared vectors): every token's
+    output equals the weighted sum of dense chains built with each expert's
+    signs."""
+    m = _small_moe(36, k=3, E=6)
+    rng = np.random.default_rng(36)
+    for i, e in enumerate(m["experts"]):
+        if i % 3 != 2:
+            e["signs_in"] = synth.signs(rng, m["hidden"])
+        if i % 2 == 1:
+            e["signs_mid"] = synth.signs(rng, m["inter"])
+    y, b, _ = oracle.moe(m["experts"], m["hidden"], m["inter"], m["x"], m["topk_ids"], m["topk_w"],
+                         m["s_in"], m["s_mid"])
+    for t in range(m["T"]):
+        want = np.zeros(m["hidden"])
+        for j in range(m["k"]):
+            e = m["experts"][int(m["topk_ids"][t, j])]
+            d, _ = _dense_expert_chain(e, m["x"][t].astype(np.float64), m["s_in"], m["s_mid"],
+                                       m["hidden"], m["inter"])
+            want += float(m["topk_w"][t, j]) * d
+        assert np.allclose(y[t], want, rtol=1e-11, atol=1e-12)
+        assert np.all(np.abs(y[t]) <= b[t] * (1 + 1e-12))
 
 
 # ---------------------------------------------------------------- routing inputs
