@@ -30,7 +30,7 @@ class HqWeight(ctypes.Structure):
 
 class HqExpert(ctypes.Structure):
     _fields_ = [("bits", _i), ("zero", _i), ("q_gate", _vp), ("q_up", _vp), ("q_down", _vp),
-                ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp)]
+                ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp), ("signs_in", _vp), ("signs_mid", _vp)]
 
 
 class HqError(RuntimeError):

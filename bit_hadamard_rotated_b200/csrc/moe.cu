@@ -12,6 +12,9 @@
 //                         (scaled by a power of two 2^e per token that puts
 //                         its largest |x'| just below 2^14, undone exactly in
 //                         the phase epilogue, as is the same scale of h');
+//                         and, for each of the token's pairs whose expert has
+//                         its own input signs, x_t rotated with those signs,
+//                         in that expert's layout;
 //   2. moe_phase_kernel<A>  gate and up of every touched expert in one launch,
 //                         SwiGLU in the epilogue -> h [pairs][inter];
 //   3. moe_rot_h_kernel   h' = H diag(s_mid) h / sqrt(inter) per pair, in the
@@ -58,6 +61,9 @@ struct Ws {
   float* hsum;     // [P][G_i]
   float* hfac;     // [P] output factor 2^(24 - e) of each pair's scaled h'
   float* d;        // [P][hidden]
+  uint16_t* xpl;   // [P][G_h][4][kXq] x rotated with the pair's expert's own signs (pair index t k + j)
+  float* xpsum;    // [P][G_h]
+  float* xpfac;    // [P]
 };
 
 struct Dims {
@@ -92,7 +98,7 @@ static size_t a256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct MoePlan {
   moe::Dims d;
-  size_t off[16];
+  size_t off[18];
   size_t bytes;
 };
 
@@ -108,7 +114,7 @@ static MoePlan moe_plan(int E, int hidden, int inter, int T, int k) {
   d.nb_max = std::min(E, d.P) + (d.P + 7) / 8;  // bound on sum_e ceil(cnt_e / 8)
   d.grid = std::min(sm_count(), moe::kMaxGrid);
   const size_t Gh = hidden / kGroup, Gi = inter / kGroup;
-  const size_t sizes[15] = {
+  const size_t sizes[18] = {
       256,                                             // status
       sizeof(int) * E,                                 // counts
       sizeof(int) * (E + 1),                           // offsets
@@ -124,9 +130,12 @@ static MoePlan moe_plan(int E, int hidden, int inter, int T, int k) {
       4 * static_cast<size_t>(d.P) * Gi,                   // hsum
       4 * static_cast<size_t>(d.P) * hidden,               // d
       4 * static_cast<size_t>(d.P),                        // hfac
+      2 * static_cast<size_t>(d.P) * Gh * 4 * moe::kXq,    // xpl
+      4 * static_cast<size_t>(d.P) * Gh,                   // xpsum
+      4 * static_cast<size_t>(d.P),                        // xpfac
   };
   size_t o = 0;
-  for (int i = 0; i < 15; ++i) {
+  for (int i = 0; i < 18; ++i) {
     pl.off[i] = o;
     o += a256(sizes[i]);
   }
@@ -152,6 +161,9 @@ static moe::Ws moe_ws(void* base, const MoePlan& pl) {
   w.hsum = reinterpret_cast<float*>(b + pl.off[12]);
   w.d = reinterpret_cast<float*>(b + pl.off[13]);
   w.hfac = reinterpret_cast<float*>(b + pl.off[14]);
+  w.xpl = reinterpret_cast<uint16_t*>(b + pl.off[15]);
+  w.xpsum = reinterpret_cast<float*>(b + pl.off[16]);
+  w.xpfac = reinterpret_cast<float*>(b + pl.off[17]);
   return w;
 }
 
@@ -159,8 +171,11 @@ namespace moe {
 
 __device__ __forceinline__ bool valid_desc(const hq_expert& e) {
   const bool bits_ok = e.bits == 2 || e.bits == 3 || e.bits == 4 || e.bits == 8;
-  return bits_ok && e.zero >= 0 && e.zero < (1 << e.bits) && e.q_gate && e.q_up && e.q_down &&
-         e.s_gate && e.s_up && e.s_down;
+  // the kernels read sign vectors in 16-byte pieces: a misaligned one is a bad descriptor
+  const bool signs_ok = (reinterpret_cast<uintptr_t>(e.signs_in) & 15u) == 0 &&
+                        (reinterpret_cast<uintptr_t>(e.signs_mid) & 15u) == 0;
+  return bits_ok && signs_ok && e.zero >= 0 && e.zero < (1 << e.bits) && e.q_gate && e.q_up &&
+         e.q_down && e.s_gate && e.s_up && e.s_down;
 }
 
 // The routing CTA (block 0 of the first launch).  Stable counting sort of the
@@ -413,6 +428,25 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
     write_layout_bits(bits_of[L], buf, sc, G, w.xl + row * G * 4 * kXq, w.xsum + row * G,
                       tid >> 5, S::THREADS / 32, tid & 31);
   }
+  // pairs of this token whose expert brings its own input signs: x_t rotated
+  // with them, in that expert's layout (rows of bad ids or descriptors are
+  // never read: their pairs are skipped)
+  for (int j = 0; j < d.k; ++j) {
+    const int i = t * d.k + j;
+    const int e = ids[i];
+    if (e < 0 || e >= d.E) continue;  // uniform over the block
+    const hq_expert de = ex[e];
+    if (de.signs_in == nullptr || !valid_desc(de)) continue;
+    __syncthreads();  // buf and red are free again
+    const auto own = sign_bits<S::E>(de.signs_in + tid * S::E);
+    load_chunk<__half, S::E>(x + static_cast<size_t>(t) * S::K + tid * S::E, v);
+    flip_signs<S::E>(own, v);
+    fwht_block<LOGK, 5>(v, buf, red);
+    const int ej = row_scale_exp(red_max(red, S::W) * inv);
+    if (tid == 0) w.xpfac[i] = pow2f(24 - ej);
+    write_layout_bits(de.bits, buf, inv * pow2f(ej), G, w.xpl + static_cast<size_t>(i) * G * 4 * kXq,
+                      w.xpsum + static_cast<size_t>(i) * G, tid >> 5, S::THREADS / 32, tid & 31);
+  }
 }
 
 // One CTA per sorted pair position: rotate h and write it in the layout of
@@ -429,11 +463,13 @@ __global__ void __launch_bounds__(FwhtShape<LOGK>::THREADS)
   pdl_wait();
   if (p >= w.offsets[d.E]) return;  // block-uniform: no barrier is skipped by part of it
   const int e = ids[w.sorted[p]];
-  const int bits = ex[e].bits;
+  const hq_expert de = ex[e];
+  const int bits = de.bits;
   float v[S::E];
   float* red = buf + S::SMEM_FLOATS;
   load_chunk<float, S::E>(w.h + static_cast<size_t>(p) * S::K + tid * S::E, v);
-  flip_signs<S::E>(neg, v);
+  // the expert's own signs for its down projection, where it has them
+  flip_signs<S::E>(de.signs_mid != nullptr ? sign_bits<S::E>(de.signs_mid + tid * S::E) : neg, v);
   fwht_block<LOGK, 5>(v, buf, red);
   const int ex_ = row_scale_exp(red_max(red, S::W) * inv);
   if (tid == 0) w.hfac[p] = pow2f(24 - ex_);
@@ -547,6 +583,7 @@ struct SegInfo {
   int col0;          // column offset of the block in the staged fragments
   int L;             // activation layout (bit width) of phase A
   float fac[8];      // output factor 2^(24 - e) of each column (token or pair)
+  int own;           // phase A: the expert rotates its tokens with its own signs
 };
 
 struct PassMeta {
@@ -602,11 +639,21 @@ struct RingState {
 };
 
 // B-operand row of column col of a segment (the token's rotated activations
-// in phase A, the pair's rotated h in phase B).
+// in phase A -- per pair when the expert has its own signs --, the pair's
+// rotated h in phase B), in the buffers seg_bsrc and seg_sums name.
 template <int PHASE>
 __device__ __forceinline__ size_t seg_brow(const Ws& w, const Dims& d, const SegInfo& sg, int col) {
   const int p = sg.off + col;
-  return PHASE == 0 ? static_cast<size_t>(sg.L) * d.T + w.sorted[p] / d.k : static_cast<size_t>(p);
+  if (PHASE != 0) return static_cast<size_t>(p);
+  return sg.own ? static_cast<size_t>(w.sorted[p]) : static_cast<size_t>(sg.L) * d.T + w.sorted[p] / d.k;
+}
+template <int PHASE>
+__device__ __forceinline__ const uint16_t* seg_bsrc(const Ws& w, const SegInfo& sg) {
+  return PHASE == 0 ? (sg.own ? w.xpl : w.xl) : w.hl;
+}
+template <int PHASE>
+__device__ __forceinline__ const float* seg_sums(const Ws& w, const SegInfo& sg) {
+  return PHASE == 0 ? (sg.own ? w.xpsum : w.xsum) : w.hsum;
 }
 
 // Epilogue of one item: rows g, g+8 of the lane's fragments, columns 2t,
@@ -648,7 +695,7 @@ template <int PHASE, int LOGK, int BITS>
 __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, int ub, const Ws& w,
                                             const Dims& d, RingState& rs,
                                             const float* zc, const uint4* xs, int cols,
-                                            const uint16_t* bsrc, int u0, float4 (&part)[2][2],
+                                            int u0, float4 (&part)[2][2],
                                             int (&ptile)[2], int lane) {
   constexpr int NMAT = 2;  // gate and up, or the two halves of a down tile
   constexpr int GB = 16 * BITS;  // code bytes of one row in one group
@@ -745,7 +792,8 @@ __device__ __forceinline__ void phase_piece(const SegInfo& sg, int k, int ua, in
 #pragma unroll
     for (int i = 0; i < 4; ++i) bo[i] = i ^ sw;
   } else {
-    bl = has_b ? reinterpret_cast<const uint4*>(bsrc + (seg_brow<PHASE>(w, d, sg, g) * G * 4 + t) * kXq) : zero_blk;
+    bl = has_b ? reinterpret_cast<const uint4*>(seg_bsrc<PHASE>(w, sg) + (seg_brow<PHASE>(w, d, sg, g) * G * 4 + t) * kXq)
+               : zero_blk;
     bstep = has_b ? 4 * kXq / 8 : 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) bo[i] = i;
@@ -869,8 +917,6 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
   pdl_launch_dependents();
   pdl_wait();  // routing lists and activations come from the previous kernels
   const int* bounds = w.bounds + PHASE * (kMaxGrid + 1);
-  const uint16_t* bsrc = PHASE == 0 ? w.xl : w.hl;
-  const float* sums = PHASE == 0 ? w.xsum : w.hsum;
   const int ib = bounds[blockIdx.x], ie = bounds[blockIdx.x + 1];
   RingState rs{ring, bars, 0, 0, true};  // this warp's ring, over the whole kernel
 
@@ -918,6 +964,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
         sg.ncol = ncol;
         sg.col0 = pc - ncol;
         sg.L = layout_index(sg.ed.bits);
+        sg.own = sg.ed.signs_in != nullptr ? 1 : 0;
       }
       if (lane == nseg - 1) {
         pm.nseg = nseg;
@@ -939,19 +986,20 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
           const int gg = r >> 4, q = (r >> 2) & 3, pc = r & 3;
           const int col = sg.col0 + cl;
           cp_async16(xs + ((gg * cols + col) * 4 + q) * 4 + (pc ^ bswz(col, q)),
-                     bsrc + ((seg_brow<PHASE>(w, d, sg, cl) * G + gg) * 4 + q) * kXq + pc * 8, 16);
+                     seg_bsrc<PHASE>(w, sg) + ((seg_brow<PHASE>(w, d, sg, cl) * G + gg) * 4 + q) * kXq + pc * 8, 16);
         }
       }
       // output factors of the segment's columns (written before the barrier
       // below, read by the epilogue after it)
       if (tid < sg.ncol) {
-        pm.seg[k].fac[tid] = PHASE == 0 ? w.xfac[w.sorted[sg.off + tid] / d.k] : w.hfac[sg.off + tid];
+        pm.seg[k].fac[tid] = PHASE == 0 ? (sg.own ? w.xpfac[w.sorted[sg.off + tid]] : w.xfac[w.sorted[sg.off + tid] / d.k])
+                                        : w.hfac[sg.off + tid];
       }
       // -zero * sum_k x' * 2^-24 per group and column (0 for absent columns)
       const float zneg = -static_cast<float>(sg.ed.zero) * 5.9604644775390625e-8f;
       for (int i = tid; i < G * 8; i += kWarps * 32) {
         const int gg = i >> 3, cl = i & 7;
-        zc[k * G * 8 + i] = cl < sg.ncol ? zneg * sums[seg_brow<PHASE>(w, d, sg, cl) * G + gg] : 0.f;
+        zc[k * G * 8 + i] = cl < sg.ncol ? zneg * seg_sums<PHASE>(w, sg)[seg_brow<PHASE>(w, d, sg, cl) * G + gg] : 0.f;
       }
     }
     if constexpr (BSMEM) asm volatile("cp.async.wait_all;" ::: "memory");
@@ -977,10 +1025,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1)
       const int sa = max(u0, sg.unit0), sb = min(u1, sg.unit0 + (sg.item1 - sg.item0) * G);
       if (sa >= sb) continue;
       switch (sg.ed.bits) {
-        case 2: phase_piece<PHASE, LOGK, 2>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
-        case 3: phase_piece<PHASE, LOGK, 3>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
-        case 4: phase_piece<PHASE, LOGK, 4>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
-        default: phase_piece<PHASE, LOGK, 8>(sg, k, sa, sb, w, d, rs, zc, xs, cols, bsrc, u0, part, ptile, lane); break;
+        case 2: phase_piece<PHASE, LOGK, 2>(sg, k, sa, sb, w, d, rs, zc, xs, cols, u0, part, ptile, lane); break;
+        case 3: phase_piece<PHASE, LOGK, 3>(sg, k, sa, sb, w, d, rs, zc, xs, cols, u0, part, ptile, lane); break;
+        case 4: phase_piece<PHASE, LOGK, 4>(sg, k, sa, sb, w, d, rs, zc, xs, cols, u0, part, ptile, lane); break;
+        default: phase_piece<PHASE, LOGK, 8>(sg, k, sa, sb, w, d, rs, zc, xs, cols, u0, part, ptile, lane); break;
       }
     }
     // ---- tiles split between warps: each warp leaves its partial sums in

@@ -230,11 +230,14 @@ def hq_moe_workspace_size(n_experts, hidden, inter, T, k) -> int:
 
 def expert_table(experts: list[dict], device) -> torch.Tensor:
     """Device array of hq_expert descriptors (bytes) for a list of expert dicts
-    holding CUDA tensors q_gate, q_up, q_down, s_gate, s_up, s_down."""
+    holding CUDA tensors q_gate, q_up, q_down, s_gate, s_up, s_down, and
+    optionally the expert's own rotation signs signs_in, signs_mid."""
     arr = (HqExpert * len(experts))()
     for i, e in enumerate(experts):
+        own = [e.get(n) for n in ("signs_in", "signs_mid")]
         arr[i] = HqExpert(int(e["bits"]), int(e["zero"]), *[e[n].data_ptr() for n in
-                          ("q_gate", "q_up", "q_down", "s_gate", "s_up", "s_down")])
+                          ("q_gate", "q_up", "q_down", "s_gate", "s_up", "s_down")],
+                          *[None if o is None else o.data_ptr() for o in own])
     raw = bytes(memoryview(arr).cast("B"))
     return torch.frombuffer(bytearray(raw), dtype=torch.uint8).to(device)
 

@@ -144,6 +144,9 @@ typedef struct {
   const uint16_t* s_gate; /* [inter][hidden/128] fp16 */
   const uint16_t* s_up;   /* [inter][hidden/128] fp16 */
   const uint16_t* s_down; /* [hidden][inter/128] fp16 */
+  const int8_t* signs_in;  /* [hidden] this expert's own rotation signs for gate/up,
+                              or NULL: the call's signs_in (16-byte aligned) */
+  const int8_t* signs_mid; /* [inter] its own signs for down, or NULL: the call's */
 } hq_expert;
 
 size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k);
@@ -151,7 +154,8 @@ size_t hq_moe_workspace_size(int n_experts, int hidden, int inter, int T, int k)
 /*
  * hq_moe_experts -- the routed-expert part of an MoE layer, all experts and
  * bit widths in one pass per phase, no host synchronisation:
- *   x'_t  = H_hidden diag(s_in) x_t / sqrt(hidden)
+ *   x'_t  = H_hidden diag(s_in) x_t / sqrt(hidden)   (s_in, s_mid: the expert's
+ *                                                    own signs where it has them)
  *   g, u  = W_gate^e x'_t,  W_up^e x'_t           for e = topk_ids[t][j]
  *   h     = g / (1 + exp(-g)) * u                  (SwiGLU)
  *   h'    = H_inter diag(s_mid) h / sqrt(inter)

@@ -42,6 +42,9 @@ def device_experts(experts):
             d[n] = dev(e[n].view(np.int32))
         for n in ("s_gate", "s_up", "s_down"):
             d[n] = dev(e[n])
+        for n in ("signs_in", "signs_mid"):
+            if e.get(n) is not None:
+                d[n] = dev(e[n])
         out.append(d)
     return out
 
@@ -228,15 +231,17 @@ def _check_stages(m, ws):
             # gate/up + SwiGLU: h = silu(g) u with g, u each within 2e-3 of their own
             # L1 bases Bg, Bu; to first order |dh| <= max|silu'| |u| dg + |silu(g)| du
             # (max silu' = 1.0998), plus the product of the two errors
-            g, bg = oracle.dequant_dot(e["bits"], I, H, e["zero"], e["q_gate"], e["s_gate"], xr[t:t + 1])
-            u, bu = oracle.dequant_dot(e["bits"], I, H, e["zero"], e["q_up"], e["s_up"], xr[t:t + 1])
+            xt = xr[t:t + 1] if e.get("signs_in") is None else oracle.rotate(m["x"][t:t + 1], e["signs_in"])
+            g, bg = oracle.dequant_dot(e["bits"], I, H, e["zero"], e["q_gate"], e["s_gate"], xt)
+            u, bu = oracle.dequant_dot(e["bits"], I, H, e["zero"], e["q_up"], e["s_up"], xt)
             g, bg, u, bu = g[0], bg[0], u[0], bu[0]
             silu = g / (1.0 + np.exp(-g))
             lim = rel * (1.1 * np.abs(u) * bg + np.abs(silu) * bu) + 1.1 * rel * rel * bg * bu + 1e-5
             err = np.abs(h_gpu[r].astype(np.float64) - h_want[t * k + j])
             assert np.all(err <= lim), ("h", t, j, float(np.max(err / lim)))
             # down, fed the GPU's own h: d = W_down H diag(s_mid) h_gpu / sqrt(inter)
-            hr = oracle.rotate(h_gpu[r].astype(np.float64), m["s_mid"])
+            hr = oracle.rotate(h_gpu[r].astype(np.float64),
+                               m["s_mid"] if e.get("signs_mid") is None else e["signs_mid"])
             dw, db = oracle.dequant_dot(e["bits"], H, I, e["zero"], e["q_down"], e["s_down"], hr[None, :])
             err = np.abs(d_gpu[r].astype(np.float64) - dw[0])
             lim = rel * db[0] + 1e-5
@@ -262,3 +267,25 @@ def test_moe_stagewise(which):
     _check_stages(m, ws)
     want, bound, _ = oracle_moe(m)
     check(y, want, bound, which)
+
+
+# ---------------------------------------------------------------- per-expert rotation signs
+@pytest.mark.parametrize("hidden,inter,T,k", [(2048, 512, 32, 8), (256, 128, 9, 3), (8192, 256, 5, 2)])
+def test_moe_per_expert_signs(hidden, inter, T, k):
+    """Experts with their own rotation signs beside experts on the shared
+    vectors: x rotated again per pair with the expert's signs_in, h with its
+    signs_mid; stage-wise and end-to-end parity as above."""
+    from bit_hadamard_rotated_b200 import hq_moe_workspace_size
+    E = 16 if hidden == 2048 else 6
+    m = synth.moe(seed=13 + hidden, E=E, hidden=hidden, inter=inter, T=T, k=k)
+    rng = np.random.default_rng(hidden)
+    for i, e in enumerate(m["experts"]):
+        if i % 3 != 2:
+            e["signs_in"] = synth.signs(rng, hidden)
+        if i % 2 == 1:
+            e["signs_mid"] = synth.signs(rng, inter)
+    ws = torch.zeros(hq_moe_workspace_size(E, hidden, inter, T, k), dtype=torch.uint8, device="cuda")
+    y, _ = run_moe(m, ws=ws)
+    _check_stages(m, ws)
+    want, bound, _ = oracle_moe(m)
+    check(y, want, bound, "per-expert signs")
