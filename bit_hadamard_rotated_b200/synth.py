@@ -119,3 +119,15 @@ def touched_weight_bytes(inp: dict) -> int:
         for n in ("q_gate", "q_up", "q_down", "s_gate", "s_up", "s_down"):
             total += ex[n].nbytes
     return total
+
+
+def readout(V: int = 157184, K: int = 2048, N: int = 1, seed: int = 0) -> dict:
+    """An 8-bit lm_head stored as high and low nibble planes (each a uniform
+    4-bit packed matrix [V][K/8] words, so the 8-bit codes 16 hi + lo are
+    uniform too), fp16 scales U[0.005, 0.02], zero point 128, signs, x ~ N(0, 1)
+    fp16 [N][K].  Default sizes: a 157,184-token vocabulary over hidden 2048."""
+    rng = _rng(seed, V, K, N, 8)
+    hi = packed_words(rng, V, K, 4)
+    lo = packed_words(rng, V, K, 4)
+    return dict(V=V, K=K, N=N, zero=128, hi=hi, lo=lo, scales=scales_uniform(rng, V, K),
+                signs=signs(rng, K), x=activations(rng, N, K))

@@ -73,8 +73,10 @@ def lib():
             L.hqo_f64_to_f16.argtypes = [ctypes.c_double]
             L.hqo_f64_to_f16.restype = ctypes.c_uint16
             L.hqo_quantize.argtypes = [vp, i, i, i, vp, i, i, vp, vp, vp]
+            L.hqo_readout.argtypes = [vp, vp, vp, vp, i, i, i, vp, i, i, ctypes.c_double, vp, vp, vp,
+                                      vp, vp]
             for f in ("hqo_unpack", "hqo_pack", "hqo_fwht", "hqo_rotate", "hqo_rotate_f16",
-                      "hqo_dequant_dot", "hqo_linear", "hqo_moe", "hqo_quantize"):
+                      "hqo_dequant_dot", "hqo_linear", "hqo_moe", "hqo_quantize", "hqo_readout"):
                 getattr(L, f).restype = None
             _lib = L
     return _lib
@@ -259,3 +261,22 @@ def moe(experts, hidden, inter, x, topk_ids, topk_w, s_in, s_mid, t_begin=0, t_e
             t.join()
     del keep
     return y, b, h
+
+
+def readout(hi, lo, scales, signs, V, K, zero, x, topk, beta=6.0, want_all=False):
+    """Nibble-split screened readout (hq_oracle.h).  hi, lo: uint32 4-bit planes
+    [V][K/8]; x fp16 [N][K].  Returns (ids int32 [N][topk], logits float64
+    [N][topk], cand uint8 [N][V], y_all [N][V] or None, e [N][V] or None)."""
+    hi, lo = _c(hi, np.uint32), _c(lo, np.uint32)
+    sc = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
+    s = _c(signs, np.int8)
+    x16 = np.ascontiguousarray(x, dtype=np.float16).reshape(-1, K).view(np.uint16)
+    N = x16.shape[0]
+    ids = np.zeros((N, topk), np.int32)
+    out = np.zeros((N, topk), np.float64)
+    cand = np.zeros((N, V), np.uint8)
+    ya = np.zeros((N, V), np.float64) if want_all else None
+    ea = np.zeros((N, V), np.float64) if want_all else None
+    lib().hqo_readout(_p(hi), _p(lo), _p(sc), _p(s), V, K, zero, _p(x16), N, topk, float(beta), _p(ids),
+                      _p(out), _p(cand), _p(ya), _p(ea))
+    return ids, out, cand, ya, ea

@@ -259,3 +259,73 @@ void hqo_quantize(const double* W, int M, int K, int bits, const int8_t* signs,
   free(q);
   free(r);
 }
+
+void hqo_readout(const uint32_t* hi, const uint32_t* lo, const uint16_t* scales,
+                 const int8_t* signs, int V, int K, int zero, const uint16_t* x, int N,
+                 int topk, double beta, int32_t* ids, double* out, uint8_t* cand,
+                 double* y_all, double* e_out) {
+  const int G = K / 128;
+  const size_t wpr = (size_t)K * 4 / 32; /* words per row of a 4-bit plane */
+  double* xr = (double*)malloc(sizeof(double) * (size_t)K);
+  uint8_t* ch = (uint8_t*)malloc((size_t)K);
+  uint8_t* cl = (uint8_t*)malloc((size_t)K);
+  double* y = (double*)malloc(sizeof(double) * (size_t)V);
+  double* L = (double*)malloc(sizeof(double) * (size_t)V);
+  double* U = (double*)malloc(sizeof(double) * (size_t)V);
+  for (int n = 0; n < N; ++n) {
+    hqo_rotate_f16(x + (size_t)n * K, signs, K, xr);
+    for (int m = 0; m < V; ++m) {
+      hqo_unpack(hi + (size_t)m * wpr, 4, (size_t)K, ch);
+      hqo_unpack(lo + (size_t)m * wpr, 4, (size_t)K, cl);
+      double ye = 0.0, ys = 0.0, var = 0.0;
+      for (int k = 0; k < K; ++k) {
+        double s = hqo_f16_to_f64(scales[(size_t)m * G + k / 128]);
+        ye += s * (double)(16 * (int)ch[k] + (int)cl[k] - zero) * xr[k];
+        ys += s * (16.0 * (double)ch[k] + 7.5 - (double)zero) * xr[k];
+        var += s * s * xr[k] * xr[k];
+      }
+      double sd = sqrt(21.25 * var);
+      y[m] = ye;
+      L[m] = ys - beta * sd;
+      U[m] = ys + beta * sd;
+      if (y_all) y_all[(size_t)n * V + m] = ye;
+      if (e_out) e_out[(size_t)n * V + m] = ys;
+    }
+    /* tau: the topk-th largest L (selection by repeated maximum: O(topk V)) */
+    double tau = INFINITY;
+    {
+      uint8_t* taken = (uint8_t*)calloc((size_t)V, 1);
+      for (int r = 0; r < topk; ++r) {
+        int best = -1;
+        for (int m = 0; m < V; ++m) {
+          if (!taken[m] && (best < 0 || L[m] > L[best])) best = m;
+        }
+        taken[best] = 1;
+        tau = L[best];
+      }
+      free(taken);
+    }
+    /* the topk candidates of largest exact y, ties to the lower index */
+    uint8_t* used = (uint8_t*)calloc((size_t)V, 1);
+    for (int r = 0; r < topk; ++r) {
+      int best = -1;
+      for (int m = 0; m < V; ++m) {
+        if (used[m] || U[m] < tau) continue;
+        if (best < 0 || y[m] > y[best]) best = m;
+      }
+      used[best] = 1;
+      ids[(size_t)n * topk + r] = best;
+      out[(size_t)n * topk + r] = y[best];
+    }
+    free(used);
+    if (cand) {
+      for (int m = 0; m < V; ++m) cand[(size_t)n * V + m] = U[m] >= tau ? 1 : 0;
+    }
+  }
+  free(U);
+  free(L);
+  free(y);
+  free(cl);
+  free(ch);
+  free(xr);
+}

@@ -135,6 +135,30 @@ void hqo_quantize(const double* W, int M, int K, int bits, const int8_t* signs,
                   int m_begin, int m_end, uint32_t* qweight, uint16_t* scales,
                   double* rotated);
 
+/* Nibble-split screened readout over an 8-bit lm_head (the "high/low nibble
+ * split planes ... for screened readout" of the LLaDA2.2-mini Orin-Nano model
+ * card, file list and Properties table; the pages give no rule, this is the
+ * library's).  W has 8-bit codes q = 16 hi + lo (zero point `zero`, group-128
+ * fp16 scales), stored as two 4-bit planes hi[V][K/8], lo[V][K/8] (hqo_pack
+ * layout).  For each batch row n, with x' = H diag(s) x_n / sqrt(K):
+ *   exact     y[m]  = sum_k scale (16 hi + lo - zero) x'_k
+ *   screen    e[m]  = sum_k scale (16 hi + 7.5 - zero) x'_k   (low nibble at
+ *                     its mean; reads only the high plane)
+ *   spread    sd[m] = sqrt(21.25 sum_k scale^2 x'_k^2)   (standard deviation
+ *                     of the low-nibble term if the low nibbles were
+ *                     independent and uniform on 0..15: variance 255/12)
+ *   bounds    L[m] = e[m] - beta sd[m],  U[m] = e[m] + beta sd[m]
+ *   tau       = the topk-th largest L
+ *   cand[m]   = U[m] >= tau
+ *   result    the topk rows of largest exact y among the candidates (ties to
+ *             the lower row index), ids and y, descending.
+ * cand (optional, [N][V] bytes), y_all (optional, [N][V] exact logits of
+ * every row), e_out (optional, [N][V]).  ids [N][topk] int32, out [N][topk]. */
+void hqo_readout(const uint32_t* hi, const uint32_t* lo, const uint16_t* scales,
+                 const int8_t* signs, int V, int K, int zero, const uint16_t* x, int N,
+                 int topk, double beta, int32_t* ids, double* out, uint8_t* cand,
+                 double* y_all, double* e_out);
+
 #ifdef __cplusplus
 }
 #endif

@@ -390,6 +390,51 @@ def test_moe_per_expert_signs_equals_dense_chain():
         assert np.all(np.abs(y[t]) <= b[t] * (1 + 1e-12))
 
 
+# ---------------------------------------------------------------- nibble-split screened readout
+def _merged_codes(r):
+    hi = np.stack([np_unpack(r["hi"][m], 4, r["K"]) for m in range(r["V"])])
+    lo = np.stack([np_unpack(r["lo"][m], 4, r["K"]) for m in range(r["V"])])
+    return hi, lo
+
+
+@pytest.mark.parametrize("topk", [1, 5])
+def test_readout_exact_topk_and_screen_decomposition(topk):
+    """The oracle's readout: exact logits equal a dense numpy product of the
+    merged 8-bit codes (16 hi + lo); the screen e plus the low-nibble
+    remainder sum scale (lo - 7.5) x' (numpy) is the exact logit; the returned
+    ids are the topk of the exact logits (numpy's stable descending order), all
+    of them candidates."""
+    r = synth.readout(V=300, K=256, N=2, seed=topk)
+    ids, out, cand, ya, ea = oracle.readout(r["hi"], r["lo"], r["scales"], r["signs"], r["V"], r["K"],
+                                            r["zero"], r["x"], topk, want_all=True)
+    hi, lo = _merged_codes(r)
+    sc = np.repeat(r["scales"].astype(np.float64), 128, axis=1)
+    W = sc * (16 * hi + lo - r["zero"])
+    H = scipy.linalg.hadamard(r["K"]).astype(np.float64)
+    xr = (H @ (sign_vec(r["signs"], r["K"])[:, None] * r["x"].astype(np.float64).T)).T / np.sqrt(r["K"])
+    assert np.allclose(ya, xr @ W.T, rtol=1e-12, atol=1e-12)
+    rem = xr @ (sc * (lo - 7.5)).T
+    assert np.allclose(ea + rem, ya, rtol=1e-11, atol=1e-11)
+    for n in range(2):
+        order = np.argsort(-ya[n], kind="stable")[:topk]
+        assert ids[n].tolist() == order.tolist()
+        assert np.allclose(out[n], ya[n, order], rtol=0, atol=0)
+        assert np.all(cand[n, order] == 1)
+
+
+def test_readout_screen_band():
+    """beta = 0: the candidates are exactly the rows whose screen reaches the
+    topk-th largest screen (numpy); a huge beta keeps every row."""
+    r = synth.readout(V=400, K=256, N=1, seed=9)
+    _, _, cand, _, ea = oracle.readout(r["hi"], r["lo"], r["scales"], r["signs"], r["V"], r["K"], r["zero"],
+                                       r["x"], 7, beta=0.0, want_all=True)
+    tau = np.sort(ea[0])[::-1][6]
+    assert np.array_equal(cand[0].astype(bool), ea[0] >= tau)
+    _, _, cand2, _, _ = oracle.readout(r["hi"], r["lo"], r["scales"], r["signs"], r["V"], r["K"], r["zero"],
+                                       r["x"], 7, beta=1e9)
+    assert np.all(cand2 == 1)
+
+
 # ---------------------------------------------------------------- routing inputs
 def test_routing_weights_and_ties():
     rng = np.random.default_rng(5)
