@@ -33,6 +33,11 @@ class HqExpert(ctypes.Structure):
                 ("s_gate", _vp), ("s_up", _vp), ("s_down", _vp), ("signs_in", _vp), ("signs_mid", _vp)]
 
 
+class HqReadout(ctypes.Structure):
+    _fields_ = [("V", _i), ("K", _i), ("zero", _i), ("hi", _vp), ("lo", _vp), ("scales", _vp),
+                ("signs", _vp)]
+
+
 class HqError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -77,6 +82,13 @@ def lib() -> ctypes.CDLL:
         L.hq_linear_noalloc.restype = _i
         L.hq_linear_noalloc_check_status.argtypes = [_vp]
         L.hq_linear_noalloc_check_status.restype = _i
+        L.hq_readout_workspace_size.argtypes = [ctypes.POINTER(HqReadout), _i]
+        L.hq_readout_workspace_size.restype = _sz
+        L.hq_readout_topk.argtypes = [ctypes.POINTER(HqReadout), _vp, _i, _i, ctypes.c_float, _vp, _vp,
+                                      _vp, _sz, _vp]
+        L.hq_readout_topk.restype = _i
+        L.hq_split_nibbles.argtypes = [_vp, _i, _i, _vp, _vp, _vp]
+        L.hq_split_nibbles.restype = _i
         L.hq_quantize.argtypes = [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]
         L.hq_quantize.restype = _i
         L.hq_moe_workspace_offset.argtypes = [_i, _i, _i, _i, _i, _i]

@@ -84,7 +84,7 @@ struct GemvParams {
   int M, N, ldy;
   uint32_t U;       // units = n_tiles * G
   uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
-  int zero;
+  float zero;  // the zero point (fractional only for the screened readout's high plane)
   int withhold;  // test of the error path: CTA 0's last warp never requests its second chunk
   const uint8_t* xg;  // prep output: x' fragments [N][G][4][64 B] fp16, zq [G][16] fp32, fac [8] fp32
   float inv_sqrt_k;
@@ -143,7 +143,7 @@ __host__ __device__ constexpr int zq_index(int gg, int t, int j) { return (gg * 
 // zero-point reductions overlap.
 template <int BITS, int GPW>
 __device__ __forceinline__ void put_groups(const FragLane<BITS>& fl, const float* buf, int warp, int nw,
-                                           int n, int G, float sc, int zero, uint16_t* xs, float* zq,
+                                           int n, int G, float sc, float zero, uint16_t* xs, float* zq,
                                            int lane) {
   const int s = lane >> 2, t = lane & 3;
   uint16_t hv[GPW][4];
@@ -178,7 +178,7 @@ __device__ __forceinline__ void put_groups(const FragLane<BITS>& fl, const float
                                 ((((s >> 1) + t) & 3) << 4) + (s & 1) * 8) = pk;
       if (lane < 2) {
         zq[zq_index(gg, n >> 1, (n & 1) + 2 * lane)] =
-            -static_cast<float>(zero) * part[i] * 5.9604644775390625e-8f;
+            -zero * part[i] * 5.9604644775390625e-8f;
       }
     }
   }
@@ -200,7 +200,7 @@ template <int BITS, int LOGK>
 __global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const __half* __restrict__ x,
                                                                  const int8_t* __restrict__ signs,
                                                                  uint8_t* __restrict__ xg, int N,
-                                                                 int zero, float inv_sqrt_k) {
+                                                                 float zero, float inv_sqrt_k) {
   using FS = FwhtShape<LOGK, prep_logw(LOGK)>;
   constexpr int kPrepWarps = prep_warps(LOGK);
   constexpr int K = 1 << LOGK;
@@ -577,7 +577,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       const int e = row_scale_exp(red_max(red, FS::THREADS / 32) * p.inv_sqrt_k);
       if (tid == 0) fac[n] = pow2f(24 - e);
       const float sc = p.inv_sqrt_k * pow2f(e);
-      put_groups<BITS, (G + kWarps - 1) / kWarps>(fl, buf, warp, kWarps, n, G, sc, pgz ? 1 : p.zero, xs, zq,
+      put_groups<BITS, (G + kWarps - 1) / kWarps>(fl, buf, warp, kWarps, n, G, sc, pgz ? 1.f : p.zero, xs, zq,
                                                   lane);
       // buf becomes a TMA destination after the loop: order this thread's
       // accesses to it before that copy (generic -> async proxy)
@@ -861,6 +861,9 @@ int gemv_launches(int K, int nb) { return gemv_fused_rotation(K, nb) ? 1 : 2; }
 
 size_t gemv_scratch_bytes(int K, int nb) { return gemv_xg_bytes(K / kGroup, nb); }
 
+// The zero point the kernels apply: the integer one, or a fractional override.
+static float gemv_zero(const GemvArgs& a) { return a.zero_frac ? a.zero_f : static_cast<float>(a.zero); }
+
 template <int BITS>
 static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
   const dim3 g(a.N);
@@ -870,7 +873,7 @@ static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
 #define HQ_PREP(LK)                                                                          \
   launch_pdl(gemv_prep_kernel<BITS, LK>, g, dim3(prep_warps(LK) * 32),                         \
              (FwhtShape<LK, prep_logw(LK)>::SMEM_FLOATS + 32) * sizeof(float), st, true, x, a.signs, \
-             xg, a.N, a.zeros != nullptr ? 1 : a.zero, inv)
+             xg, a.N, a.zeros != nullptr ? 1.f : gemv_zero(a), inv)
   switch (K) {
     case 128: return HQ_PREP(7);
     case 256: return HQ_PREP(8);
@@ -951,7 +954,7 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.buf_off = pl.buf_off;
   p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   p.xg = static_cast<const uint8_t*>(a.xg);
-  p.zero = a.zero;
+  p.zero = gemv_zero(a);
   p.zeros = a.zeros;
   p.withhold = take_test_fault() ? 1 : 0;
   p.ring_off = pl.ring_off;

@@ -37,6 +37,8 @@ struct GemvArgs {
   uint32_t* status;
   void* xg;       // gemv_scratch_bytes(K, N) bytes, 16-byte aligned: prep output
   const uint8_t* zeros = nullptr;  // per-group zero points [M][K/128], or nullptr: zero
+  bool zero_frac = false;           // use zero_f (a fractional zero point) instead of zero
+  float zero_f = 0.f;
 };
 
 // Shared memory the GEMV needs for a batch block of nb <= 8 rows, with or

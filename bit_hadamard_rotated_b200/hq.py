@@ -9,7 +9,7 @@ import ctypes
 
 import torch
 
-from ._lib import (HQ_BF16, HQ_F16, HQ_F32, HqError, HqExpert, HqWeight, check, lib)
+from ._lib import (HQ_BF16, HQ_F16, HQ_F32, HqError, HqExpert, HqReadout, HqWeight, check, lib)
 
 _DT = {torch.float16: HQ_F16, torch.bfloat16: HQ_BF16, torch.float32: HQ_F32}
 
@@ -224,6 +224,44 @@ class RotatedLinear:
         check(lib().hq_check_status(_ptr(self.workspace), _stream(stream)), "device status")
 
 
+class ScreenedReadout:
+    """An 8-bit lm_head kept as nibble planes (hi, lo: int32 [V][K/8] 4-bit
+    layout; scales fp16 [V][K/128]; signs int8 [K] or None), with its own
+    workspace for batches up to max_batch (<= 8)."""
+
+    def __init__(self, hi, lo, scales, signs, zero=128, max_batch=8):
+        _need_cuda(hi, lo, scales, signs)
+        V, K = hi.shape[0], hi.shape[1] * 8
+        self.tensors = (hi, lo, scales, signs)
+        self.r = HqReadout(V, K, int(zero), hi.data_ptr(), lo.data_ptr(), scales.data_ptr(),
+                           None if signs is None else signs.data_ptr())
+        need = int(lib().hq_readout_workspace_size(ctypes.byref(self.r), max_batch))
+        if need == 0:
+            raise ValueError("unsupported readout shape or batch")
+        self.workspace = torch.zeros(need, dtype=torch.uint8, device=hi.device)
+
+    def topk(self, x, k, beta=6.0, stream=None):
+        """(ids int32 [N][k], logits fp32 [N][k]) of the largest exact logits."""
+        _need_cuda(x)
+        N = x.shape[0]
+        ids = torch.empty((N, k), dtype=torch.int32, device=x.device)
+        out = torch.empty((N, k), dtype=torch.float32, device=x.device)
+        check(lib().hq_readout_topk(ctypes.byref(self.r), _ptr(x.contiguous()), N, k, float(beta), _ptr(ids),
+                                    _ptr(out), _ptr(self.workspace), self.workspace.numel(),
+                                    _stream(stream)), "hq_readout_topk")
+        return ids, out
+
+
+def hq_split_nibbles(q8: torch.Tensor, K: int, stream=None):
+    """(hi, lo) int32 [rows][K/8] nibble planes of 8-bit packed codes q8 [rows][K/4]."""
+    _need_cuda(q8)
+    rows = q8.shape[0]
+    hi = torch.empty((rows, K // 8), dtype=torch.int32, device=q8.device)
+    lo = torch.empty_like(hi)
+    check(lib().hq_split_nibbles(_ptr(q8), rows, K, _ptr(hi), _ptr(lo), _stream(stream)), "hq_split_nibbles")
+    return hi, lo
+
+
 def hq_moe_workspace_size(n_experts, hidden, inter, T, k) -> int:
     return int(lib().hq_moe_workspace_size(n_experts, hidden, inter, T, k))
 
@@ -283,6 +321,6 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
-__all__ = ["hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
+__all__ = ["ScreenedReadout", "hq_split_nibbles", "hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
            "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

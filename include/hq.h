@@ -227,6 +227,53 @@ hq_status hq_quantize(const void* W, hq_dtype w_dtype, int M, int K, int bits,
                       const int8_t* signs, uint32_t* qweight, uint16_t* scales,
                       hq_stream_t stream);
 
+/* An 8-bit lm_head kept as high and low nibble planes: codes q = 16 hi + lo,
+ * w[m][k] = scale[m][k/128] (q - zero), in the rotated basis. */
+typedef struct {
+  int V;                  /* rows (vocabulary), >= 1 */
+  int K;                  /* input features: power of two, 128 <= K <= 32768 */
+  int zero;               /* integer zero point of the 8-bit codes, 0..255 (128 usual) */
+  const uint32_t* hi;     /* [V][K/8] high nibbles, 4-bit layout (as a 4-bit hq_weight) */
+  const uint32_t* lo;     /* [V][K/8] low nibbles, likewise */
+  const uint16_t* scales; /* [V][K/128] fp16 */
+  const int8_t* signs;    /* [K] rotation signs, or NULL */
+} hq_readout_weight;
+
+/* Bytes of workspace hq_readout_topk needs (0 on a bad argument). */
+size_t hq_readout_workspace_size(const hq_readout_weight* r, int batch);
+
+/*
+ * hq_readout_topk -- the topk rows of largest logit y[n][m] = sum_k w[m][k]
+ * x'[n][k] (x' = H_K diag(s) x[n] / sqrt(K)), reading the high-nibble plane
+ * of every row but the low-nibble plane of screened candidates only.
+ * Screening rule (the pages give none; this library's): the screen
+ * e[m] = sum_k scale (16 hi + 7.5 - zero) x'_k puts each low nibble at its
+ * mean; the low nibbles' term has standard deviation sd[m] = sqrt(21.25
+ * sum_k scale^2 x'_k^2) were they independent and uniform on 0..15; rows with
+ * e + beta sd at or above the topk-th largest e - beta sd (taken, on the GPU,
+ * at the lower edge of its bin in a histogram of the top 11 bits, which only
+ * widens the set) get their exact logit from both planes; the topk largest
+ * exact logits are returned, descending, ties to the lower row.  The result
+ * is exact whenever no candidate's low-nibble term strays beyond beta
+ * standard deviations (beta = 6 in tests).
+ * x: [batch][K] fp16, 1 <= batch <= 8.  ids: [batch][topk] int32, logits:
+ * [batch][topk] fp32.  1 <= topk <= 256, topk <= V.  beta >= 0.
+ * workspace: >= hq_readout_workspace_size bytes, zero-filled before first
+ * use; calls leave it ready for the next call.
+ * Cites: "8-bit lm_head.bin + nibble-split lm_head_split.bin (screened
+ * readout)" (LLaDA2.2-mini Orin-Nano model card, Properties table and file
+ * list).
+ */
+hq_status hq_readout_topk(const hq_readout_weight* r, const uint16_t* x, int batch, int topk,
+                          float beta, int32_t* ids, float* logits, void* workspace,
+                          size_t ws_bytes, hq_stream_t stream);
+
+/* Splits 8-bit packed codes q8 [rows][K/4] into high and low nibble planes
+ * hi, lo [rows][K/8] (4-bit layout): the "same codes split into high/low
+ * nibble planes" of the model card's file list.  K a multiple of 8. */
+hq_status hq_split_nibbles(const uint32_t* q8, int rows, int K, uint32_t* hi, uint32_t* lo,
+                           hq_stream_t stream);
+
 /* Intermediates an hq_moe_experts call leaves in its workspace, for checking
  * the layer stage by stage:
  *   HQ_MOE_POS  int32 [T*k]: row of pair (t, j) (index t*k + j) in the two
