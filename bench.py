@@ -422,12 +422,39 @@ def measure_configs(device, stream, pk, l2):
         "frac_hbm": round(tb / (us * 1e-6) / 1e9 / pk["hbm"], 4), "launches": 5}
     del tables
 
+    res["readout_157184x2048_top8"] = measure_readout(device, stream, pk, gen)
+
     sweep = {}
     for b in (2, 3, 4, 8):
         for N in (1, 2, 4, 8, 16, 32, 64, 128):
             sweep[f"b{b}_n{N}"] = linear_point(8192, 8192, b, N)
     res["sweep_8192x8192"] = sweep
     return res
+
+
+def measure_readout(device, stream, pk, gen):
+    """The screened top-8 readout over the 157,184 x 2048 8-bit lm_head kept
+    as nibble planes, batch 1, against the plain 8-bit linear over the same
+    codes; two copies of the planes alternated (16-bit codes, 2 x 322 MB > L2)."""
+    from bit_hadamard_rotated_b200 import RotatedLinear, ScreenedReadout, hq_split_nibbles
+    V, K = 157184, 2048
+    signs = torch.from_numpy(synth.signs(np.random.default_rng(1), K)).to(device)
+    ros, lins = [], []
+    for _ in range(2):
+        q8 = torch.randint(-2**31, 2**31 - 1, (V, K // 4), dtype=torch.int32, device=device, generator=gen)
+        sc = (torch.rand((V, K // 128), device=device, generator=gen) * 0.015 + 0.005).half()
+        hi, lo = hq_split_nibbles(q8, K)
+        ros.append(ScreenedReadout(hi, lo, sc, signs, 128, max_batch=1))
+        lins.append(RotatedLinear(q8, sc, signs, 8, 128, max_batch=1))
+    x = torch.randn((1, K), device=device, generator=gen).half()
+    y = torch.empty((1, V), dtype=torch.float32, device=device)
+    us_ro = _graph_us(stream, device, [lambda r=r: r.topk(x, 8, stream=stream) for r in ros] * 4)
+    us_lin = _graph_us(stream, device, [lambda l=l: l(x, out=y) for l in lins] * 4)
+    hi_bytes = V * K // 2 + V * (K // 128) * 2
+    return {"us_screened_top8": round(us_ro, 2), "us_plain_8bit_linear": round(us_lin, 2),
+            "high_plane_gbs": round(hi_bytes / (us_ro * 1e-6) / 1e9, 1),
+            "frac_hbm_high_plane": round(hi_bytes / (us_ro * 1e-6) / 1e9 / pk["hbm"], 4),
+            "launches": 5, "batch": 1}
 
 
 class _Rt:
