@@ -131,3 +131,20 @@ def readout(V: int = 157184, K: int = 2048, N: int = 1, seed: int = 0) -> dict:
     lo = packed_words(rng, V, K, 4)
     return dict(V=V, K=K, N=N, zero=128, hi=hi, lo=lo, scales=scales_uniform(rng, V, K),
                 signs=signs(rng, K), x=activations(rng, N, K))
+
+
+def kv(T: int = 32768, n_kv: int = 4, d: int = 128, n_q: int = 32, n_heads: int = 16,
+       seed: int = 0) -> dict:
+    """One attention layer's keys and values for T tokens (fp16 [T][n_kv][d],
+    N(0, 1); keys with a seeded 2 % of channels x8, the same for every token, as
+    key caches usually have) and a block of n_q query tokens (fp16
+    [n_q][n_heads][d], N(0, 1)).  Defaults: a 32K-token context, 4 kv heads of
+    128 channels, 16 query heads, one 32-token denoising block."""
+    rng = _rng(seed, T, n_kv, d, n_q, n_heads)
+    k = rng.standard_normal((T, n_kv, d))
+    ch = rng.choice(d, size=max(1, d // 50), replace=False)
+    k[:, :, ch] *= 8.0
+    v = rng.standard_normal((T, n_kv, d))
+    q = rng.standard_normal((n_q, n_heads, d))
+    return dict(T=T, n_kv=n_kv, d=d, n_q=n_q, n_heads=n_heads, k=k.astype(np.float16),
+                v=v.astype(np.float16), q=q.astype(np.float16))

@@ -329,3 +329,77 @@ void hqo_readout(const uint32_t* hi, const uint32_t* lo, const uint16_t* scales,
   free(ch);
   free(xr);
 }
+
+void hqo_kv_quant_group(const uint16_t* x, int n, int stride, uint8_t* codes,
+                        uint16_t* scale, uint16_t* mn) {
+  float lo = (float)hqo_f16_to_f64(x[0]), hi = lo;
+  for (int i = 1; i < n; ++i) {
+    float v = (float)hqo_f16_to_f64(x[(size_t)i * stride]);
+    if (v < lo) lo = v;
+    if (v > hi) hi = v;
+  }
+  volatile float span = hi - lo; /* single-precision steps, in this order */
+  volatile float sf = span / 15.0f;
+  uint16_t s16 = hqo_f64_to_f16((double)sf);
+  uint16_t m16 = hqo_f64_to_f16((double)lo);
+  float s = (float)hqo_f16_to_f64(s16), m = (float)hqo_f16_to_f64(m16);
+  for (int i = 0; i < n; ++i) {
+    int c = 0;
+    if (s > 0.0f) {
+      volatile float diff = (float)hqo_f16_to_f64(x[(size_t)i * stride]) - m;
+      volatile float r = diff / s;
+      c = (int)rintf(r);
+      if (c < 0) c = 0;
+      if (c > 15) c = 15;
+    }
+    codes[i] = (uint8_t)c;
+  }
+  *scale = s16;
+  *mn = m16;
+}
+
+void hqo_kv_attend(const uint8_t* kc, const uint16_t* ks, const uint16_t* km,
+                   const uint8_t* vc, const uint16_t* vs, const uint16_t* vm,
+                   int n_kv, int d, int T, const uint16_t* q, int n_q, int n_heads,
+                   double* out, double* base) {
+  const int G = n_heads / n_kv;
+  const int nb = T / 32;
+  double* sc = (double*)malloc(sizeof(double) * (size_t)T);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+  for (int i = 0; i < n_q; ++i) {
+    for (int j = 0; j < n_heads; ++j) {
+      const int h = j / G;
+      for (int c = 0; c < d; ++c) qd[c] = hqo_f16_to_f64(q[((size_t)i * n_heads + j) * d + c]);
+      double mx = -INFINITY;
+      for (int t = 0; t < T; ++t) {
+        const int b = t / 32;
+        double acc = 0.0;
+        for (int c = 0; c < d; ++c) {
+          size_t kb = ((size_t)h * nb + b) * d + c;
+          double kv = hqo_f16_to_f64(ks[kb]) * (double)kc[kb * 32 + (t % 32)] + hqo_f16_to_f64(km[kb]);
+          acc += qd[c] * kv;
+        }
+        sc[t] = acc / sqrt((double)d);
+        if (sc[t] > mx) mx = sc[t];
+      }
+      double l = 0.0;
+      for (int t = 0; t < T; ++t) {
+        sc[t] = exp(sc[t] - mx);
+        l += sc[t];
+      }
+      for (int c = 0; c < d; ++c) {
+        double o = 0.0, bs = 0.0;
+        for (int t = 0; t < T; ++t) {
+          size_t vt = (size_t)h * T + t;
+          double v = hqo_f16_to_f64(vs[vt]) * (double)vc[vt * d + c] + hqo_f16_to_f64(vm[vt]);
+          o += sc[t] / l * v;
+          bs += sc[t] / l * fabs(v);
+        }
+        out[((size_t)i * n_heads + j) * d + c] = o;
+        if (base) base[((size_t)i * n_heads + j) * d + c] = bs;
+      }
+    }
+  }
+  free(qd);
+  free(sc);
+}

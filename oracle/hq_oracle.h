@@ -159,6 +159,32 @@ void hqo_readout(const uint32_t* hi, const uint32_t* lo, const uint16_t* scales,
                  int topk, double beta, int32_t* ids, double* out, uint8_t* cand,
                  double* y_all, double* e_out);
 
+/* int4 KV cache ("Runtime int4 (keys per channel per 32-token block, values
+ * per token)": LLaDA2.2-mini Orin-Nano model card, Properties table; the
+ * quantiser is this library's reading, asymmetric min/scale with 4-bit codes).
+ * One group of n values x (fp16 bit patterns, stride `stride` elements):
+ *   lo = min x, hi = max x                     (in float)
+ *   scale = fp16(float(hi - lo) / 15), mn = fp16(lo)      (round to nearest even)
+ *   code_i = clamp(rintf((x_i - mn) / scale), 0, 15), 0 where scale = 0
+ * computed in IEEE single precision (the decision's precision).  Keys: a group
+ * is one channel of one head over a 32-token block; values: all head_dim
+ * channels of one head for one token.  codes receives n bytes. */
+void hqo_kv_quant_group(const uint16_t* x, int n, int stride, uint8_t* codes,
+                        uint16_t* scale, uint16_t* mn);
+
+/* Attention over a dequantised cache, fp64: for each query row r (query
+ * token i, head j; kv head j / (n_heads / n_kv)):
+ *   s_t = (q_r . k_t) / sqrt(d),  p = softmax over t < T,  out_r = sum_t p_t v_t
+ * with k_t[c] = k_scale[c of t's block] code + k_min, v_t[c] = v_scale[t] code
+ * + v_min[t].  kc: [n_kv][T/32][d][32] key codes (one byte each), ks, km:
+ * [n_kv][T/32][d] fp16; vc: [n_kv][T][d] value codes, vs, vm: [n_kv][T].
+ * q: [n_q][n_heads][d] fp16; out, base: [n_q][n_heads][d] (base = sum_t p_t
+ * |v_t[c]|, the tolerance base; may be NULL). */
+void hqo_kv_attend(const uint8_t* kc, const uint16_t* ks, const uint16_t* km,
+                   const uint8_t* vc, const uint16_t* vs, const uint16_t* vm,
+                   int n_kv, int d, int T, const uint16_t* q, int n_q, int n_heads,
+                   double* out, double* base);
+
 #ifdef __cplusplus
 }
 #endif

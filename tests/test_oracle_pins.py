@@ -435,6 +435,55 @@ def test_readout_screen_band():
     assert np.all(cand2 == 1)
 
 
+# ---------------------------------------------------------------- int4 KV cache
+def test_kv_quant_group_nearest_code_and_range():
+    """Each 4-bit code of a group is a nearest point of the grid mn + scale c
+    (brute force over the 16 codes, in float64 of the float32 decision), the
+    scale is float16((float32 max - float32 min) / 15) and mn float16(min)
+    (numpy's float32 and float16 roundings)."""
+    r = synth.kv(T=64, n_kv=2, d=32, n_q=1, n_heads=2, seed=3)
+    cache = oracle.kv_quantize(r["k"], r["v"])
+    for h in range(2):
+        for b in range(2):
+            for c in range(32):
+                x = r["k"][32 * b:32 * b + 32, h, c].astype(np.float32)
+                s = np.float16((x.max() - x.min()) / np.float32(15))
+                assert cache["ks"][h, b, c] == s and cache["km"][h, b, c] == np.float16(x.min())
+                grid = np.float64(cache["km"][h, b, c]) + np.float64(s) * np.arange(16)
+                codes = cache["kc"][h, b, c]
+                err = np.abs(x[:, None].astype(np.float64) - grid[None, :])
+                assert np.all(err[np.arange(32), codes] <= err.min(axis=1) + 1e-6 * np.abs(grid).max())
+        for t in range(64):
+            x = r["v"][t, h].astype(np.float32)
+            s = np.float16((x.max() - x.min()) / np.float32(15))
+            assert cache["vs"][h, t] == s and cache["vm"][h, t] == np.float16(x.min())
+            assert cache["vc"][h, t].max() <= 15
+
+
+def test_kv_attend_equals_dense_softmax_attention():
+    """The oracle's attention over the int4 cache equals a dense numpy softmax
+    attention over the dequantised keys and values (grouped heads)."""
+    r = synth.kv(T=96, n_kv=2, d=32, n_q=3, n_heads=4, seed=5)
+    cache = oracle.kv_quantize(r["k"], r["v"])
+    out, base = oracle.kv_attend(cache, 96, r["q"])
+    K = (cache["ks"].astype(np.float64)[..., None] * cache["kc"] + cache["km"].astype(np.float64)[..., None])
+    K = K.transpose(0, 1, 3, 2).reshape(2, 96, 32)                       # [h][t][c]
+    V = cache["vs"].astype(np.float64)[..., None] * cache["vc"] + cache["vm"].astype(np.float64)[..., None]
+    q = r["q"].astype(np.float64)
+    for i in range(3):
+        for j in range(4):
+            h = j // 2
+            s = K[h] @ q[i, j] / np.sqrt(32)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            assert np.allclose(out[i, j], p @ V[h], rtol=1e-12, atol=1e-12)
+            assert np.allclose(base[i, j], p @ np.abs(V[h]), rtol=1e-12, atol=1e-12)
+    # equal keys: uniform weights, the output is the values' mean
+    c2 = dict(cache, kc=np.zeros_like(cache["kc"]), km=np.zeros_like(cache["km"]))
+    out2, _ = oracle.kv_attend(c2, 96, r["q"])
+    assert np.allclose(out2[0, 0], V[0].mean(axis=0), rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- routing inputs
 def test_routing_weights_and_ties():
     rng = np.random.default_rng(5)
