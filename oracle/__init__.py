@@ -74,12 +74,13 @@ def lib():
             L.hqo_f64_to_f16.restype = ctypes.c_uint16
             L.hqo_quantize.argtypes = [vp, i, i, i, vp, i, i, vp, vp, vp]
             L.hqo_kv_quant_group.argtypes = [vp, i, i, vp, vp, vp]
+            L.hqo_kv_quantize.argtypes = [vp, vp, i, i, i, vp, vp, vp, vp, vp, vp]
             L.hqo_kv_attend.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, vp, i, i, vp, vp]
             L.hqo_readout.argtypes = [vp, vp, vp, vp, i, i, i, vp, i, i, ctypes.c_double, vp, vp, vp,
                                       vp, vp]
             for f in ("hqo_unpack", "hqo_pack", "hqo_fwht", "hqo_rotate", "hqo_rotate_f16",
                       "hqo_dequant_dot", "hqo_linear", "hqo_moe", "hqo_quantize", "hqo_readout",
-                      "hqo_kv_quant_group", "hqo_kv_attend"):
+                      "hqo_kv_quant_group", "hqo_kv_quantize", "hqo_kv_attend"):
                 getattr(L, f).restype = None
             _lib = L
     return _lib
@@ -302,33 +303,19 @@ def kv_quantize(k, v):
     vc = np.zeros((n_kv, T, d), np.uint8)
     vs = np.zeros((n_kv, T), np.uint16)
     vm = np.zeros((n_kv, T), np.uint16)
-    L = lib()
-    one_s, one_m = np.zeros(1, np.uint16), np.zeros(1, np.uint16)
-    for h in range(n_kv):
-        for b in range(nb):
-            for c in range(d):
-                col = np.ascontiguousarray(kb[32 * b:32 * b + 32, h, c])
-                codes = np.zeros(32, np.uint8)
-                L.hqo_kv_quant_group(_p(col), 32, 1, _p(codes), _p(one_s), _p(one_m))
-                kc[h, b, c] = codes
-                ks[h, b, c], km[h, b, c] = one_s[0], one_m[0]
-        for t in range(T):
-            row = np.ascontiguousarray(vb[t, h])
-            codes = np.zeros(d, np.uint8)
-            L.hqo_kv_quant_group(_p(row), d, 1, _p(codes), _p(one_s), _p(one_m))
-            vc[h, t] = codes
-            vs[h, t], vm[h, t] = one_s[0], one_m[0]
+    lib().hqo_kv_quantize(_p(kb), _p(vb), T, n_kv, d, _p(kc), _p(ks), _p(km), _p(vc), _p(vs), _p(vm))
     return dict(kc=kc, ks=ks.view(np.float16), km=km.view(np.float16), vc=vc, vs=vs.view(np.float16),
                 vm=vm.view(np.float16))
 
 
 def kv_attend(cache, T, q):
     """Attention of q fp16 [n_q][n_heads][d] over the first T tokens of a
-    kv_quantize cache, fp64.  Returns (out, base) [n_q][n_heads][d]."""
+    kv_quantize cache (T >= 1, any), fp64.  Returns (out, base) [n_q][n_heads][d]."""
     n_kv, _, d, _ = cache["kc"].shape
-    kc = np.ascontiguousarray(cache["kc"][:, :T // 32])
-    ks = np.ascontiguousarray(cache["ks"][:, :T // 32]).view(np.uint16)
-    km = np.ascontiguousarray(cache["km"][:, :T // 32]).view(np.uint16)
+    nb = (T + 31) // 32
+    kc = np.ascontiguousarray(cache["kc"][:, :nb])
+    ks = np.ascontiguousarray(cache["ks"][:, :nb]).view(np.uint16)
+    km = np.ascontiguousarray(cache["km"][:, :nb]).view(np.uint16)
     vc = np.ascontiguousarray(cache["vc"][:, :T])
     vs = np.ascontiguousarray(cache["vs"][:, :T]).view(np.uint16)
     vm = np.ascontiguousarray(cache["vm"][:, :T]).view(np.uint16)

@@ -358,12 +358,30 @@ void hqo_kv_quant_group(const uint16_t* x, int n, int stride, uint8_t* codes,
   *mn = m16;
 }
 
+void hqo_kv_quantize(const uint16_t* k, const uint16_t* v, int T, int n_kv, int d, uint8_t* kc,
+                     uint16_t* ks, uint16_t* km, uint8_t* vc, uint16_t* vs, uint16_t* vm) {
+  const int nb = T / 32;
+  for (int h = 0; h < n_kv; ++h) {
+    for (int b = 0; b < nb; ++b) {
+      for (int c = 0; c < d; ++c) { /* channel c over the block's 32 tokens */
+        const size_t g = ((size_t)h * nb + b) * d + c;
+        hqo_kv_quant_group(k + ((size_t)32 * b * n_kv + h) * d + c, 32, n_kv * d, kc + g * 32, ks + g,
+                           km + g);
+      }
+    }
+    for (int t = 0; t < T; ++t) { /* all channels of token t */
+      const size_t g = (size_t)h * T + t;
+      hqo_kv_quant_group(v + ((size_t)t * n_kv + h) * d, d, 1, vc + g * d, vs + g, vm + g);
+    }
+  }
+}
+
 void hqo_kv_attend(const uint8_t* kc, const uint16_t* ks, const uint16_t* km,
                    const uint8_t* vc, const uint16_t* vs, const uint16_t* vm,
                    int n_kv, int d, int T, const uint16_t* q, int n_q, int n_heads,
                    double* out, double* base) {
   const int G = n_heads / n_kv;
-  const int nb = T / 32;
+  const int nb = (T + 31) / 32; /* key blocks that tokens 0 .. T-1 fall in */
   double* sc = (double*)malloc(sizeof(double) * (size_t)T);
   double* qd = (double*)malloc(sizeof(double) * (size_t)d);
   for (int i = 0; i < n_q; ++i) {

@@ -172,12 +172,20 @@ void hqo_readout(const uint32_t* hi, const uint32_t* lo, const uint16_t* scales,
 void hqo_kv_quant_group(const uint16_t* x, int n, int stride, uint8_t* codes,
                         uint16_t* scale, uint16_t* mn);
 
+/* The whole cache of T tokens (T a multiple of 32): k, v fp16
+ * [T][n_kv][d]; kc [n_kv][T/32][d][32], ks, km [n_kv][T/32][d], vc
+ * [n_kv][T][d], vs, vm [n_kv][T], each group through hqo_kv_quant_group. */
+void hqo_kv_quantize(const uint16_t* k, const uint16_t* v, int T, int n_kv, int d, uint8_t* kc,
+                     uint16_t* ks, uint16_t* km, uint8_t* vc, uint16_t* vs, uint16_t* vm);
+
 /* Attention over a dequantised cache, fp64: for each query row r (query
  * token i, head j; kv head j / (n_heads / n_kv)):
  *   s_t = (q_r . k_t) / sqrt(d),  p = softmax over t < T,  out_r = sum_t p_t v_t
  * with k_t[c] = k_scale[c of t's block] code + k_min, v_t[c] = v_scale[t] code
- * + v_min[t].  kc: [n_kv][T/32][d][32] key codes (one byte each), ks, km:
- * [n_kv][T/32][d] fp16; vc: [n_kv][T][d] value codes, vs, vm: [n_kv][T].
+ * + v_min[t].  T >= 1 need not be a multiple of 32: the key arrays hold
+ * the nb = ceil(T/32) blocks that tokens 0 .. T-1 fall in, and only those
+ * tokens are attended.  kc: [n_kv][nb][d][32] key codes (one byte each), ks,
+ * km: [n_kv][nb][d] fp16; vc: [n_kv][T][d] value codes, vs, vm: [n_kv][T].
  * q: [n_q][n_heads][d] fp16; out, base: [n_q][n_heads][d] (base = sum_t p_t
  * |v_t[c]|, the tolerance base; may be NULL). */
 void hqo_kv_attend(const uint8_t* kc, const uint16_t* ks, const uint16_t* km,

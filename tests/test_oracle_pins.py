@@ -478,6 +478,16 @@ def test_kv_attend_equals_dense_softmax_attention():
             p /= p.sum()
             assert np.allclose(out[i, j], p @ V[h], rtol=1e-12, atol=1e-12)
             assert np.allclose(base[i, j], p @ np.abs(V[h]), rtol=1e-12, atol=1e-12)
+    # a prefix of T = 75 tokens (not a whole number of blocks): only tokens
+    # 0..74 enter the softmax
+    out3, _ = oracle.kv_attend(cache, 75, r["q"])
+    for i in range(3):
+        for j in range(4):
+            h = j // 2
+            s = K[h, :75] @ q[i, j] / np.sqrt(32)
+            p = np.exp(s - s.max())
+            p /= p.sum()
+            assert np.allclose(out3[i, j], p @ V[h, :75], rtol=1e-12, atol=1e-12)
     # equal keys: uniform weights, the output is the values' mean
     c2 = dict(cache, kc=np.zeros_like(cache["kc"]), km=np.zeros_like(cache["km"]))
     out2, _ = oracle.kv_attend(c2, 96, r["q"])
