@@ -38,6 +38,11 @@ class HqReadout(ctypes.Structure):
                 ("signs", _vp)]
 
 
+class HqKvCache(ctypes.Structure):
+    _fields_ = [("head_dim", _i), ("n_kv_heads", _i), ("capacity", _i), ("k_codes", _vp), ("k_scale", _vp),
+                ("k_min", _vp), ("v_codes", _vp), ("v_scale", _vp), ("v_min", _vp)]
+
+
 class HqError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -88,6 +93,14 @@ def lib() -> ctypes.CDLL:
                                       _vp, _sz, _vp]
         L.hq_readout_topk.restype = _i
         L.hq_split_nibbles.argtypes = [_vp, _i, _i, _vp, _vp, _vp]
+        L.hq_kv_append.argtypes = [ctypes.POINTER(HqKvCache), _vp, _vp, _i, _i, _vp]
+        L.hq_kv_append.restype = _i
+        L.hq_kv_attend_workspace_size.argtypes = [ctypes.POINTER(HqKvCache), _i, _i, _i]
+        L.hq_kv_attend_workspace_size.restype = _sz
+        L.hq_kv_attend.argtypes = [ctypes.POINTER(HqKvCache), _i, _vp, _i, _i, _vp, _vp, _sz, _vp]
+        L.hq_kv_attend.restype = _i
+        L.hq_kv_attend_launches.argtypes = []
+        L.hq_kv_attend_launches.restype = _i
         L.hq_split_nibbles.restype = _i
         L.hq_quantize.argtypes = [_vp, _i, _i, _i, _i, _vp, _vp, _vp, _vp]
         L.hq_quantize.restype = _i

@@ -9,7 +9,8 @@ import ctypes
 
 import torch
 
-from ._lib import (HQ_BF16, HQ_F16, HQ_F32, HqError, HqExpert, HqReadout, HqWeight, check, lib)
+from ._lib import (HQ_BF16, HQ_F16, HQ_F32, HqError, HqExpert, HqKvCache, HqReadout, HqWeight, check,
+                   lib)
 
 _DT = {torch.float16: HQ_F16, torch.bfloat16: HQ_BF16, torch.float32: HQ_F32}
 
@@ -252,6 +253,63 @@ class ScreenedReadout:
         return ids, out
 
 
+class KVCache:
+    """The int4 KV cache of one attention layer (layout: include/hq.h,
+    hq_kv_cache), allocated on `device` for `capacity` tokens (a multiple of
+    32) of n_kv_heads heads of head_dim channels."""
+
+    def __init__(self, n_kv_heads: int, head_dim: int, capacity: int, device):
+        if capacity % 32 != 0 or capacity < 32:
+            raise ValueError("capacity must be a positive multiple of 32")
+        nb, d = capacity // 32, head_dim
+        dev = torch.device(device)
+        if dev.type != "cuda":
+            raise RuntimeError("KVCache lives in CUDA device memory")
+        self.n_kv_heads, self.head_dim, self.capacity = n_kv_heads, head_dim, capacity
+        self.k_codes = torch.zeros((n_kv_heads, nb, 32, d // 2), dtype=torch.uint8, device=dev)
+        self.k_scale = torch.zeros((n_kv_heads, nb, d), dtype=torch.float16, device=dev)
+        self.k_min = torch.zeros_like(self.k_scale)
+        self.v_codes = torch.zeros((n_kv_heads, nb, d, 16), dtype=torch.uint8, device=dev)
+        self.v_scale = torch.zeros((n_kv_heads, capacity), dtype=torch.float16, device=dev)
+        self.v_min = torch.zeros_like(self.v_scale)
+        self.c = HqKvCache(head_dim, n_kv_heads, capacity, self.k_codes.data_ptr(), self.k_scale.data_ptr(),
+                           self.k_min.data_ptr(), self.v_codes.data_ptr(), self.v_scale.data_ptr(),
+                           self.v_min.data_ptr())
+        self._ws = None
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, pos: int, stream=None) -> None:
+        """Quantise k, v (fp16 [n][n_kv_heads][head_dim], n a multiple of 32)
+        into positions pos .. pos + n - 1."""
+        _need_cuda(k, v)
+        if k.dtype != torch.float16 or v.dtype != torch.float16 or k.shape != v.shape:
+            raise ValueError("k and v must be fp16 tensors of one shape")
+        k, v = k.contiguous(), v.contiguous()
+        check(lib().hq_kv_append(ctypes.byref(self.c), _ptr(k), _ptr(v), int(pos), int(k.shape[0]),
+                                 _stream(stream)), "hq_kv_append")
+
+    def workspace_size(self, n_tokens: int, n_q: int, n_heads: int) -> int:
+        return int(lib().hq_kv_attend_workspace_size(ctypes.byref(self.c), n_tokens, n_q, n_heads))
+
+    def attend(self, q: torch.Tensor, n_tokens: int, out=None, workspace=None, stream=None) -> torch.Tensor:
+        """Attention of q (fp16 [n_q][n_heads][head_dim]) over the first
+        n_tokens cached tokens; returns fp32 [n_q][n_heads][head_dim]."""
+        _need_cuda(q)
+        if q.dtype != torch.float16 or q.dim() != 3 or q.shape[2] != self.head_dim:
+            raise ValueError("q must be fp16 [n_q][n_heads][head_dim]")
+        q = q.contiguous()
+        n_q, n_heads = q.shape[0], q.shape[1]
+        if out is None:
+            out = torch.empty((n_q, n_heads, self.head_dim), dtype=torch.float32, device=q.device)
+        if workspace is None:
+            need = self.workspace_size(n_tokens, max(n_q, 1), n_heads)
+            if self._ws is None or self._ws.numel() < need:
+                self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+            workspace = self._ws
+        check(lib().hq_kv_attend(ctypes.byref(self.c), int(n_tokens), _ptr(q), n_q, n_heads, _ptr(out),
+                                 _ptr(workspace), workspace.numel(), _stream(stream)), "hq_kv_attend")
+        return out
+
+
 def hq_split_nibbles(q8: torch.Tensor, K: int, stream=None):
     """(hi, lo) int32 [rows][K/8] nibble planes of 8-bit packed codes q8 [rows][K/4]."""
     _need_cuda(q8)
@@ -321,6 +379,6 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
-__all__ = ["ScreenedReadout", "hq_split_nibbles", "hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
+__all__ = ["KVCache", "ScreenedReadout", "hq_split_nibbles", "hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
            "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

@@ -274,6 +274,71 @@ hq_status hq_readout_topk(const hq_readout_weight* r, const uint16_t* x, int bat
 hq_status hq_split_nibbles(const uint32_t* q8, int rows, int K, uint32_t* hi, uint32_t* lo,
                            hq_stream_t stream);
 
+/*
+ * The int4 KV cache of one attention layer: keys quantised per channel per
+ * 32-token block, values per token ("KV Cache Format: Runtime int4 (keys per
+ * channel per 32-token block, values per token)": LLaDA2.2-mini Orin-Nano
+ * model card, Properties table).  Each group of values x gets, in IEEE single
+ * precision, scale = fp16((max x - min x) / 15), mn = fp16(min x) and codes
+ * clamp(rint((x - mn) / scale), 0, 15) (0 where scale = 0); x ~ scale * code
+ * + mn.  The caller allocates the six arrays (device memory; the library
+ * keeps no pointer past a call); with nb = capacity / 32 and d = head_dim:
+ *   k_codes [n_kv][nb][32 tokens][d/2] bytes  channel c of a token in byte
+ *                                             c/2, low nibble for even c
+ *   k_scale, k_min [n_kv][nb][d]   fp16       one group per (block, channel)
+ *   v_codes [n_kv][nb][d][16] bytes           token t of a block in byte t/2
+ *                                             of its channel's line, low
+ *                                             nibble for even t
+ *   v_scale, v_min [n_kv][capacity] fp16      one group per token
+ * head_dim 64 or 128 (HQ_ERR_UNSUPPORTED otherwise); capacity a multiple of
+ * 32, <= 2^24; all six arrays 16-byte aligned.
+ */
+typedef struct {
+  int head_dim;
+  int n_kv_heads;
+  int capacity;
+  uint8_t* k_codes;
+  uint16_t* k_scale;
+  uint16_t* k_min;
+  uint8_t* v_codes;
+  uint16_t* v_scale;
+  uint16_t* v_min;
+} hq_kv_cache;
+
+/* Quantises n_new new tokens into cache positions pos .. pos + n_new - 1.
+ * k, v: fp16 [n_new][n_kv_heads][head_dim] (device).  pos and n_new are
+ * multiples of 32 (whole key blocks), pos + n_new <= capacity; n_new = 0
+ * launches nothing.  Bit-exact with the quantiser above. */
+hq_status hq_kv_append(const hq_kv_cache* cache, const uint16_t* k, const uint16_t* v, int pos,
+                       int n_new, hq_stream_t stream);
+
+/* Bytes of workspace hq_kv_attend needs (0 on a bad argument). */
+size_t hq_kv_attend_workspace_size(const hq_kv_cache* cache, int n_tokens, int n_q, int n_heads);
+
+/* Kernels one hq_kv_attend call enqueues. */
+int hq_kv_attend_launches(void);
+
+/*
+ * hq_kv_attend -- softmax attention of n_q query tokens over the first
+ * n_tokens tokens of the cache, grouped-query: head j reads kv head
+ * j / (n_heads / n_kv_heads).  For query token i, head j, kv head h:
+ *   s_t = q[i][j] . k_h(t) / sqrt(head_dim),  p = softmax_t(s),
+ *   out[i][j] = sum_t p_t v_h(t),
+ * k_h(t), v_h(t) the dequantised cached key and value; no causal mask (every
+ * query sees all n_tokens, as a block of tokens being denoised together
+ * does).  q: fp16 [n_q][n_heads][head_dim], 16-byte aligned; out: fp32
+ * [n_q][n_heads][head_dim], 16-byte aligned.  1 <= n_tokens <= capacity,
+ * and every 32-token block that n_tokens reaches must have been appended.
+ * n_q * n_heads / n_kv_heads <= 4096 (HQ_ERR_UNSUPPORTED above); n_q = 0
+ * launches nothing.  workspace: >= hq_kv_attend_workspace_size bytes,
+ * 256-byte aligned (HQ_ERR_WORKSPACE otherwise); any contents.
+ * Numerics: keys enter the tensor cores as two fp16 planes (hi + lo, about
+ * 2^-22 relative) and p * v_scale likewise; sums in fp32.
+ */
+hq_status hq_kv_attend(const hq_kv_cache* cache, int n_tokens, const uint16_t* q, int n_q,
+                       int n_heads, float* out, void* workspace, size_t ws_bytes,
+                       hq_stream_t stream);
+
 /* Intermediates an hq_moe_experts call leaves in its workspace, for checking
  * the layer stage by stage:
  *   HQ_MOE_POS  int32 [T*k]: row of pair (t, j) (index t*k + j) in the two

@@ -189,3 +189,41 @@ def test_moe_workspace_offsets(L):
     none = ctypes.c_size_t(-1).value
     assert L.hq_moe_workspace_offset(E, H + 1, I, T, k, HQ_MOE_H) == none
     assert L.hq_moe_workspace_offset(E, H, I, T, k, 7) == none
+
+
+def test_kv_cache_rejects_bad_args(L):
+    """hq_kv_append / hq_kv_attend validate the cache and the call on the host."""
+    from bit_hadamard_rotated_b200._lib import HqKvCache
+
+    def cache(d=128, n_kv=4, cap=1024, kc=FAKE, vs=FAKE):
+        return HqKvCache(d, n_kv, cap, kc, FAKE, FAKE, FAKE, vs, FAKE)
+
+    c = cache()
+    ws = L.hq_kv_attend_workspace_size(ctypes.byref(c), 1000, 32, 16)
+    # 1000 tokens = 32 blocks, one per chunk (37 chunks per kv head would fill
+    # the SMs); per chunk 128 rows x (128 + 4) floats, for 4 kv heads
+    assert ws == 4 * 4 * 32 * 128 * 132
+    assert L.hq_kv_attend_workspace_size(ctypes.byref(c), 1025, 32, 16) == 0     # past capacity
+    assert L.hq_kv_attend_workspace_size(ctypes.byref(c), 1000, 32, 6) == 0      # heads not a multiple
+    assert L.hq_kv_attend_workspace_size(ctypes.byref(cache(d=96)), 1000, 32, 16) == 0
+    assert L.hq_kv_attend_launches() == 2
+    # append: whole blocks inside the capacity, supported head_dim, aligned arrays
+    assert L.hq_kv_append(ctypes.byref(cache(d=96)), FAKE, FAKE, 0, 32, None) == HQ_ERR_UNSUPPORTED
+    assert L.hq_kv_append(ctypes.byref(c), FAKE, FAKE, 16, 32, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_kv_append(ctypes.byref(c), FAKE, FAKE, 0, 48, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_kv_append(ctypes.byref(c), FAKE, FAKE, 1024, 32, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_kv_append(ctypes.byref(cache(cap=1000)), FAKE, FAKE, 0, 32, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_kv_append(ctypes.byref(cache(kc=FAKE + 8)), FAKE, FAKE, 0, 32, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_kv_append(ctypes.byref(c), None, FAKE, 0, 32, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_kv_append(ctypes.byref(c), FAKE, FAKE, 0, 0, None) == HQ_OK          # nothing to do
+    assert L.hq_kv_append(None, FAKE, FAKE, 0, 32, None) == HQ_ERR_INVALID_ARG
+    # attend
+    att = L.hq_kv_attend
+    assert att(ctypes.byref(c), 1000, FAKE, 0, 16, FAKE, FAKE, 1 << 30, None) == HQ_OK  # n_q = 0
+    assert att(ctypes.byref(c), 0, FAKE, 32, 16, FAKE, FAKE, 1 << 30, None) == HQ_ERR_INVALID_ARG
+    assert att(ctypes.byref(c), 1025, FAKE, 32, 16, FAKE, FAKE, 1 << 30, None) == HQ_ERR_INVALID_ARG
+    assert att(ctypes.byref(c), 1000, FAKE, 32, 15, FAKE, FAKE, 1 << 30, None) == HQ_ERR_INVALID_ARG
+    assert att(ctypes.byref(c), 1000, FAKE + 2, 32, 16, FAKE, FAKE, 1 << 30, None) == HQ_ERR_INVALID_ARG
+    assert att(ctypes.byref(c), 1000, FAKE, 32, 16, FAKE, FAKE, ws - 1, None) == HQ_ERR_WORKSPACE
+    assert att(ctypes.byref(c), 1000, FAKE, 32, 16, FAKE, FAKE + 16, ws, None) == HQ_ERR_WORKSPACE
+    assert att(ctypes.byref(c), 1000, FAKE, 1025, 16, FAKE, FAKE, 1 << 30, None) == HQ_ERR_UNSUPPORTED
