@@ -423,6 +423,7 @@ def measure_configs(device, stream, pk, l2):
     del tables
 
     res["readout_157184x2048_top8"] = measure_readout(device, stream, pk, gen)
+    res["kv_attend_32768x4x128_q32"] = measure_kv(device, stream, pk, l2)
 
     sweep = {}
     for b in (2, 3, 4, 8):
@@ -455,6 +456,36 @@ def measure_readout(device, stream, pk, gen):
             "high_plane_gbs": round(hi_bytes / (us_ro * 1e-6) / 1e9, 1),
             "frac_hbm_high_plane": round(hi_bytes / (us_ro * 1e-6) / 1e9 / pk["hbm"], 4),
             "launches": 5, "batch": 1}
+
+
+def measure_kv(device, stream, pk, l2):
+    """Attention of a 32-token block (16 heads, 4 kv heads of 128 channels)
+    over a 32K-token int4 cache, and its quantisation of the block (append);
+    enough caches cycled that every call reads HBM.  FLOPs: 4 R T d per kv
+    head (scores and P.V, R = 128 query rows); bytes: the cache's codes,
+    scales and minima."""
+    from bit_hadamard_rotated_b200 import KVCache
+    T, n_kv, d, n_q, n_heads = 32768, 4, 128, 32, 16
+    cache_bytes = n_kv * T * d + n_kv * (T // 32) * d * 4 + n_kv * T * 4
+    copies = max(2, math.ceil(3 * l2 / cache_bytes))
+    caches = []
+    for _ in range(copies):
+        c = KVCache(n_kv, d, T, device)
+        c.append(torch.randn((T, n_kv, d), device=device).half(), torch.randn((T, n_kv, d), device=device).half(), 0)
+        caches.append(c)
+    q = torch.randn((n_q, n_heads, d), device=device).half()
+    out = torch.empty((n_q, n_heads, d), dtype=torch.float32, device=device)
+    ws = torch.empty(caches[0].workspace_size(T, n_q, n_heads), dtype=torch.uint8, device=device)
+    us = _graph_us(stream, device, [lambda c=c: c.attend(q, T, out=out, workspace=ws, stream=stream)
+                                    for c in caches])
+    kb, vb = torch.randn((32, n_kv, d), device=device).half(), torch.randn((32, n_kv, d), device=device).half()
+    us_app = _graph_us(stream, device, [lambda c=c: c.append(kb, vb, T - 32, stream=stream) for c in caches])
+    flops = 4.0 * (n_q * n_heads // n_kv) * T * d * n_kv
+    del caches
+    return {"us": round(us, 2), "tflops": round(flops / (us * 1e-6) / 1e12, 2),
+            "frac_bf16_peak": round(flops / (us * 1e-6) / 1e12 / pk["bf16"], 4),
+            "cache_gbs": round(cache_bytes / (us * 1e-6) / 1e9, 1), "us_append_32_tokens": round(us_app, 2),
+            "launches": 2}
 
 
 class _Rt:
