@@ -64,6 +64,8 @@ def lib():
             L.hqo_f16_to_f64.restype = ctypes.c_double
             L.hqo_unpack.argtypes = [vp, i, sz, vp]
             L.hqo_pack.argtypes = [vp, i, sz, vp]
+            L.hqo_unpack_planes2.argtypes = [vp, sz, vp]
+            L.hqo_pack_planes2.argtypes = [vp, sz, vp]
             L.hqo_fwht.argtypes = [vp, i]
             L.hqo_rotate.argtypes = [vp, vp, i, vp]
             L.hqo_rotate_f16.argtypes = [vp, vp, i, vp]
@@ -78,7 +80,7 @@ def lib():
             L.hqo_kv_attend.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, vp, i, i, vp, vp]
             L.hqo_readout.argtypes = [vp, vp, vp, vp, i, i, i, vp, i, i, ctypes.c_double, vp, vp, vp,
                                       vp, vp]
-            for f in ("hqo_unpack", "hqo_pack", "hqo_fwht", "hqo_rotate", "hqo_rotate_f16",
+            for f in ("hqo_unpack", "hqo_pack", "hqo_unpack_planes2", "hqo_pack_planes2", "hqo_fwht", "hqo_rotate", "hqo_rotate_f16",
                       "hqo_dequant_dot", "hqo_linear", "hqo_moe", "hqo_quantize", "hqo_readout",
                       "hqo_kv_quant_group", "hqo_kv_quantize", "hqo_kv_attend"):
                 getattr(L, f).restype = None
@@ -147,6 +149,29 @@ def pack(codes, bits: int) -> np.ndarray:
     return out
 
 
+def unpack_planes2(words, n_codes: int) -> np.ndarray:
+    """2-bit codes from the bit-plane layout (hq_oracle.h, hqo_unpack_planes2)."""
+    words = _c(words, np.uint32)
+    assert n_codes % 32 == 0 and words.size * 16 >= n_codes
+    out = np.empty(n_codes, np.uint8)
+    lib().hqo_unpack_planes2(_p(words), n_codes, _p(out))
+    return out
+
+
+def pack_planes2(codes) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    assert codes.size % 32 == 0
+    out = np.empty(codes.size // 16, np.uint32)
+    lib().hqo_pack_planes2(_p(codes), codes.size, _p(out))
+    return out
+
+
+def planes_to_packed2(q, M, K) -> np.ndarray:
+    """[M][K/16] bit-plane words -> the same codes in the packed 2-bit stream."""
+    q = _c(q, np.uint32).reshape(M, K // 16)
+    return np.stack([pack(unpack_planes2(q[m], K), 2) for m in range(M)])
+
+
 def fwht(v) -> np.ndarray:
     v = np.array(v, dtype=np.float64, copy=True)
     lib().hqo_fwht(_p(v), v.size)
@@ -172,10 +197,11 @@ def rotate(x, signs=None) -> np.ndarray:
 
 
 def dequant_dot(bits, M, K, zero, q, scales, xr, m_begin=0, m_end=None, with_bound=True,
-                zeros=None):
+                zeros=None, planes=False):
     """y[n][m] = sum_k scale.(q - z).xr[n][k] for already-rotated xr [N][K]; z =
-    zeros[m][k/128] (uint8 [M][K/128]) if given, else the scalar zero."""
-    q = _c(q, np.uint32)
+    zeros[m][k/128] (uint8 [M][K/128]) if given, else the scalar zero.
+    planes: q holds 2-bit codes in the bit-plane layout."""
+    q = planes_to_packed2(q, M, K) if planes else _c(q, np.uint32)
     zr = _c(zeros, np.uint8)
     sc = np.ascontiguousarray(scales).view(np.uint16) if np.asarray(scales).dtype == np.float16 \
         else _c(scales, np.uint16)
@@ -189,14 +215,17 @@ def dequant_dot(bits, M, K, zero, q, scales, xr, m_begin=0, m_end=None, with_bou
     return (y, b) if with_bound else y
 
 
-def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads=1, zeros=None):
+def linear(bits, M, K, zero, q, scales, signs, x, m_begin=0, m_end=None, threads=1, zeros=None,
+           planes=False):
     """Full rotated linear in fp64.  x: fp16 [N][K].  Returns (y, bound) float64 [N][M].
     zeros: per-group zero points uint8 [M][K/128] (else the scalar zero).
+    planes: q holds 2-bit codes in the bit-plane layout (converted to the
+    packed stream first: the codes, and so the result, are the same).
 
     threads > 1 splits the output rows across Python threads (the C call
     releases the GIL), each running the unchanged scalar code on its rows.
     """
-    q = _c(q, np.uint32)
+    q = planes_to_packed2(q, M, K) if planes else _c(q, np.uint32)
     sc = np.ascontiguousarray(scales, dtype=np.float16).view(np.uint16)
     s = _c(signs, np.int8)
     zr = _c(zeros, np.uint8)

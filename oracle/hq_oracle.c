@@ -58,6 +58,22 @@ void hqo_pack(const uint8_t* codes, int bits, size_t n_codes,
   }
 }
 
+void hqo_unpack_planes2(const uint32_t* words, size_t n_codes, uint8_t* codes) {
+  for (size_t j = 0; j < n_codes; ++j) {
+    const uint32_t lo = (words[2 * (j / 32)] >> (j % 32)) & 1u;     /* plane 0 */
+    const uint32_t hi = (words[2 * (j / 32) + 1] >> (j % 32)) & 1u; /* plane 1 */
+    codes[j] = (uint8_t)(lo | (hi << 1));
+  }
+}
+
+void hqo_pack_planes2(const uint8_t* codes, size_t n_codes, uint32_t* words) {
+  memset(words, 0, (n_codes / 32) * 2 * sizeof(uint32_t));
+  for (size_t j = 0; j < n_codes; ++j) {
+    words[2 * (j / 32)] |= (uint32_t)(codes[j] & 1u) << (j % 32);
+    words[2 * (j / 32) + 1] |= (uint32_t)((codes[j] >> 1) & 1u) << (j % 32);
+  }
+}
+
 /* Sylvester-order butterflies: at stride h, (a, b) -> (a + b, a - b). */
 void hqo_fwht(double* v, int n) {
   for (int h = 1; h < n; h *= 2) {

@@ -49,6 +49,15 @@ double hqo_f16_to_f64(uint16_t h);
  * stream in words.  codes[j] = stream bits [bits*j, bits*j+bits). */
 void hqo_unpack(const uint32_t* words, int bits, size_t n_codes, uint8_t* codes);
 
+/* 2-bit codes kept as two bit-planes ("2-bit bit-planes ... kept that way for
+ * the whole run": Qwen3-8B BPDQ 2-bit card, introduction; the page gives no
+ * layout, this is the library's): per span of 32 codes j = 32 s + i, word 2s
+ * holds bit 0 of each code (bit i), word 2s + 1 bit 1; code = b0 + 2 b1.
+ * n_codes a multiple of 32. */
+void hqo_unpack_planes2(const uint32_t* words, size_t n_codes, uint8_t* codes);
+/* Inverse of hqo_unpack_planes2 (n_codes / 16 words, fully overwritten). */
+void hqo_pack_planes2(const uint8_t* codes, size_t n_codes, uint32_t* words);
+
 /* Inverse of hqo_unpack.  Words must have room for ceil(bits*n_codes/32)
  * entries; they are fully overwritten (unused high bits are zero). */
 void hqo_pack(const uint8_t* codes, int bits, size_t n_codes, uint32_t* words);

@@ -35,6 +35,13 @@ def np_unpack(words, bits, n):
     return (stream << np.arange(bits)).sum(axis=1)
 
 
+def np_pack(codes, bits):
+    """Little-endian bit stream of the codes via numpy.packbits."""
+    c = np.asarray(codes, dtype=np.int64)
+    stream = ((c[:, None] >> np.arange(bits)) & 1).astype(np.uint8).reshape(-1)
+    return np.packbits(stream, bitorder="little").view("<u4").astype(np.uint32)
+
+
 def sign_vec(signs, K):
     return np.ones(K) if signs is None else np.where(np.asarray(signs) < 0, -1.0, 1.0)
 
@@ -183,6 +190,39 @@ def test_three_bit_straddling_codes_single_bits():
         want = np.zeros(32, np.int64)
         want[p // 3] = 1 << (p % 3)
         assert np.array_equal(codes, want), p
+
+
+def test_bit_planes_match_numpy_and_round_trip():
+    """2-bit codes in the bit-plane layout: code 32 s + i = bit i of word 2s
+    plus twice bit i of word 2s + 1 (numpy's unpackbits, little bit order),
+    single-bit fixtures, and the round trip."""
+    rng = np.random.default_rng(17)
+    words = rng.integers(0, 2**32, size=2 * 40, dtype=np.uint64).astype(np.uint32)
+    bits = np.unpackbits(words.view(np.uint8), bitorder="little").reshape(-1, 32)   # [word][bit]
+    want = (bits[0::2] + 2 * bits[1::2]).reshape(-1)
+    got = oracle.unpack_planes2(words, 40 * 32)
+    assert np.array_equal(got, want)
+    assert np.array_equal(oracle.pack_planes2(got), words)
+    one = np.zeros(4, np.uint32)
+    one[3] = np.uint32(1 << 5)                     # plane 1 of span 1, bit 5: code 37 = 2
+    c = oracle.unpack_planes2(one, 64)
+    assert c[37] == 2 and c.sum() == 2
+    one[2] = np.uint32(1 << 5)                     # plane 0 too: code 37 = 3
+    assert oracle.unpack_planes2(one, 64)[37] == 3
+
+
+def test_linear_bit_planes_equals_packed_linear():
+    """The linear over bit-plane words equals the linear over the same codes in
+    the packed 2-bit stream (codes rebuilt through numpy's unpackbits)."""
+    d = synth.linear(24, 256, 2, 2, seed=9)
+    rng = np.random.default_rng(4)
+    planes = rng.integers(0, 2**32, size=(24, 256 // 16), dtype=np.uint64).astype(np.uint32)
+    bits = np.unpackbits(planes.view(np.uint8), axis=1, bitorder="little").reshape(24, -1, 2, 32)
+    codes = (bits[:, :, 0] + 2 * bits[:, :, 1]).reshape(24, 256).astype(np.uint8)
+    packed = np.stack([np_pack(codes[m], 2) for m in range(24)])
+    y_p, b_p = oracle.linear(2, 24, 256, 2, planes, d["scales"], d["signs"], d["x"], planes=True)
+    y_q, b_q = oracle.linear(2, 24, 256, 2, packed, d["scales"], d["signs"], d["x"])
+    assert np.array_equal(y_p, y_q) and np.array_equal(b_p, b_q)
 
 
 # ---------------------------------------------------------------- dequant + dot
