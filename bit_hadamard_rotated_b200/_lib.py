@@ -19,13 +19,14 @@ HQ_OK, HQ_ERR_INVALID_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_WORKSPACE, HQ_ERR_CUDA, HQ
     HQ_ERR_TIMEOUT = range(7)
 HQ_F16, HQ_BF16, HQ_F32 = 0, 1, 2
 HQ_MOE_POS, HQ_MOE_H, HQ_MOE_D = 0, 1, 2
+HQ_LAYOUT_PACKED, HQ_LAYOUT_BITPLANES = 0, 1
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
 
 class HqWeight(ctypes.Structure):
     _fields_ = [("bits", _i), ("M", _i), ("K", _i), ("zero", _i),
-                ("qweight", _vp), ("scales", _vp), ("signs", _vp), ("zeros", _vp)]
+                ("qweight", _vp), ("scales", _vp), ("signs", _vp), ("zeros", _vp), ("layout", _i)]
 
 
 class HqExpert(ctypes.Structure):
@@ -93,6 +94,8 @@ def lib() -> ctypes.CDLL:
                                       _vp, _sz, _vp]
         L.hq_readout_topk.restype = _i
         L.hq_split_nibbles.argtypes = [_vp, _i, _i, _vp, _vp, _vp]
+        L.hq_to_bitplanes.argtypes = [_vp, _sz, _vp, _vp]
+        L.hq_to_bitplanes.restype = _i
         L.hq_kv_append.argtypes = [ctypes.POINTER(HqKvCache), _vp, _vp, _i, _i, _vp]
         L.hq_kv_append.restype = _i
         L.hq_kv_attend_workspace_size.argtypes = [ctypes.POINTER(HqKvCache), _i, _i, _i]

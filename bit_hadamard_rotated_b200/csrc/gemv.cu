@@ -86,6 +86,7 @@ struct GemvParams {
   uint32_t tq, tr;  // tiles per CTA: n_tiles = tq * grid + tr
   float zero;  // the zero point (fractional only for the screened readout's high plane)
   int withhold;  // test of the error path: CTA 0's last warp never requests its second chunk
+  int planes;    // 2-bit codes in the bit-plane layout
   const uint8_t* xg;  // prep output: x' fragments [N][G][4][64 B] fp16, zq [G][16] fp32, fac [8] fp32
   float inv_sqrt_k;
   int NS, slot_bytes, zc_off, buf_off, ring_off, bar_off;
@@ -117,19 +118,33 @@ __host__ __device__ constexpr int gemv_ch_max(int bits, int G) {
 // ---------------------------------------------------------------- rotation -> B fragments
 // Lane (s, t) of a warp writes the B-fragment quad of step s for k-quad t:
 // the code fields (columns kc, exponent offsets ka) of its four values.
+// With bit-plane 2-bit codes (planes) the bundle's two words are rebuilt as
+// the packed words of its even and of its odd codes (plane_bundle), so bundle
+// code c is code 2c (c < 16) or 2 (c - 16) + 1 of the 32.
 template <int BITS>
 struct FragLane {
   int kc[4], ka[4];
-  __device__ __forceinline__ explicit FragLane(int lane) {
+  __device__ __forceinline__ FragLane(int lane, bool planes) {
     const int s = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       const PairDesc pd = Pairs<BITS>::get(2 * s + (r >> 1));
-      kc[r] = 32 * t + ((r & 1) ? pd.c_hi : pd.c_lo);
+      const int c = (r & 1) ? pd.c_hi : pd.c_lo;
+      kc[r] = 32 * t + (planes ? (c < 16 ? 2 * c : 2 * (c - 16) + 1) : c);
       ka[r] = (r & 1) ? pd.a_hi : pd.a_lo;
     }
   }
 };
+
+// A 32-code bundle in the bit-plane layout (w[0]: bit 0 of codes 0..31, w[1]:
+// bit 1) as two packed 2-bit words: the even codes 0, 2, .., 30, then the odd
+// ones.  Bit 2m of the first word is b0 of code 2m, bit 2m + 1 its b1 (from
+// bit 2m of w[1]); likewise for the odd codes one bit further up.
+__device__ __forceinline__ void plane_bundle(uint32_t (&w)[2]) {
+  const uint32_t p0 = w[0], p1 = w[1];
+  w[0] = (p0 & 0x55555555u) | ((p1 << 1) & 0xAAAAAAAAu);
+  w[1] = ((p0 >> 1) & 0x55555555u) | (p1 & 0xAAAAAAAAu);
+}
 
 // Index in zq of value j (0..3) of lane quad t for group gg.
 __host__ __device__ constexpr int zq_index(int gg, int t, int j) { return (gg * 4 + t) * 4 + j; }
@@ -200,7 +215,7 @@ template <int BITS, int LOGK>
 __global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const __half* __restrict__ x,
                                                                  const int8_t* __restrict__ signs,
                                                                  uint8_t* __restrict__ xg, int N,
-                                                                 float zero, float inv_sqrt_k) {
+                                                                 float zero, float inv_sqrt_k, int planes) {
   using FS = FwhtShape<LOGK, prep_logw(LOGK)>;
   constexpr int kPrepWarps = prep_warps(LOGK);
   constexpr int K = 1 << LOGK;
@@ -213,7 +228,7 @@ __global__ void __launch_bounds__(prep_warps(LOGK) * 32) gemv_prep_kernel(const 
   float* zq = reinterpret_cast<float*>(xg + gemv_xs_bytes(G, N));
   float* fac = zq + G * 16;
   float* red = buf + FS::SMEM_FLOATS;  // per-warp maxima of the transform
-  const FragLane<BITS> fl(lane);
+  const FragLane<BITS> fl(lane, planes != 0);
   const SignMask<FS::E> neg =
       tid < FS::THREADS ? sign_bits<FS::E>(signs ? signs + tid * FS::E : nullptr) : 0u;
   pdl_wait();  // x is the previous kernel's output; xg may still be read by it
@@ -364,7 +379,7 @@ __device__ __forceinline__ void load_pair_rows(const uint8_t* ra, int j, int g, 
 // covered by the other chain's, and each MMA's four A registers are masked
 // out of the code words right before it (measured ~5 % faster than decoding
 // a group's 32 registers first).
-template <int BITS, int CH, bool PGZ>
+template <int BITS, int CH, bool PGZ, bool PL = false>
 __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* sca, const uint8_t* scb,
                                            const uint8_t* zra, const uint8_t* zrb, const float4* zq4,
                                            const uint8_t* const (&xb)[4], int g, int t, float (&acc)[4]) {
@@ -389,6 +404,10 @@ __device__ __forceinline__ void gemv_chunk(const uint8_t* base, const uint8_t* s
 #pragma unroll
     for (int q = 0; q < JP; ++q) {
       load_pair_rows<BITS>(ra, j0 + q, g, t, wa[q], wb[q]);
+      if constexpr (PL) {
+        plane_bundle(wa[q]);
+        plane_bundle(wb[q]);
+      }
       const float4 z = zq4[(j0 + q) * 4];
       if constexpr (PGZ) {
         // the group's zero-point term of each row: its zero times -sum x'
@@ -475,6 +494,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
   constexpr int sc_off = CH * kRows * GB;
   constexpr int z_off = sc_off + (G >= 8 ? kRows * 16 : ((kRows * G * 2 + 15) & ~15));
   const bool pgz = p.zeros != nullptr;
+  const bool planes = p.planes != 0;
 
   if (tid == 0) {
     prefetch_tensormap(&p.qmap3);
@@ -563,7 +583,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
     const SignMask<FS::E> neg =
         tid < FS::THREADS ? sign_bits<FS::E>(p.signs ? p.signs + tid * FS::E : nullptr) : 0u;
     float* buf = reinterpret_cast<float*>(smem + p.ring_off + (p.NS - 1) * ring_stride);
-    const FragLane<BITS> fl(lane);
+    const FragLane<BITS> fl(lane, p.planes != 0);
     zq_clear_absent(zq, G, p.N, tid, kWarps * 32);
     float* red = fac + 8;
     pdl_wait();
@@ -663,7 +683,13 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv_kernel(const __grid_const
       const uint8_t* zr = base + z_off;
       const uint8_t* zra = G >= 16 ? zr + g * 16 + (g0 & 15u) : zr + g * G + g0;
       const uint8_t* zrb = G >= 16 ? zr + (g + 8) * 16 + (g0 & 15u) : zr + (g + 8) * G + g0;
-      gemv_chunk<BITS, CH, true>(base, sca, scb, zra, zrb, zq_lane + g0 * 4, xb, g, t, acc);
+      if (BITS == 2 && planes) {
+        gemv_chunk<BITS, CH, true, BITS == 2>(base, sca, scb, zra, zrb, zq_lane + g0 * 4, xb, g, t, acc);
+      } else {
+        gemv_chunk<BITS, CH, true>(base, sca, scb, zra, zrb, zq_lane + g0 * 4, xb, g, t, acc);
+      }
+    } else if (BITS == 2 && planes) {
+      gemv_chunk<BITS, CH, false, BITS == 2>(base, sca, scb, nullptr, nullptr, zq_lane + g0 * 4, xb, g, t, acc);
     } else {
       gemv_chunk<BITS, CH, false>(base, sca, scb, nullptr, nullptr, zq_lane + g0 * 4, xb, g, t, acc);
     }
@@ -873,7 +899,7 @@ static cudaError_t gemv_prep_b(int K, const GemvArgs& a, cudaStream_t st) {
 #define HQ_PREP(LK)                                                                          \
   launch_pdl(gemv_prep_kernel<BITS, LK>, g, dim3(prep_warps(LK) * 32),                         \
              (FwhtShape<LK, prep_logw(LK)>::SMEM_FLOATS + 32) * sizeof(float), st, true, x, a.signs, \
-             xg, a.N, a.zeros != nullptr ? 1.f : gemv_zero(a), inv)
+             xg, a.N, a.zeros != nullptr ? 1.f : gemv_zero(a), inv, a.planes ? 1 : 0)
   switch (K) {
     case 128: return HQ_PREP(7);
     case 256: return HQ_PREP(8);
@@ -956,6 +982,7 @@ cudaError_t launch_gemv(const GemvArgs& a, cudaStream_t st) {
   p.xg = static_cast<const uint8_t*>(a.xg);
   p.zero = gemv_zero(a);
   p.zeros = a.zeros;
+  p.planes = a.planes ? 1 : 0;
   p.withhold = take_test_fault() ? 1 : 0;
   p.ring_off = pl.ring_off;
   p.bar_off = pl.bar_off;

@@ -53,6 +53,8 @@ static hq_status check_weight(const hq_weight* w) {
   if (!aligned(w->qweight, 16) || !aligned(w->scales, 16)) return HQ_ERR_INVALID_ARG;
   if (w->signs != nullptr && !aligned(w->signs, 16)) return HQ_ERR_INVALID_ARG;
   if (w->zeros != nullptr && !aligned(w->zeros, 16)) return HQ_ERR_INVALID_ARG;
+  if (w->layout != HQ_LAYOUT_PACKED && w->layout != HQ_LAYOUT_BITPLANES) return HQ_ERR_INVALID_ARG;
+  if (w->layout == HQ_LAYOUT_BITPLANES && w->bits != 2) return HQ_ERR_UNSUPPORTED;
   return HQ_OK;
 }
 
@@ -76,7 +78,7 @@ static bool use_tc(const hq_weight* w, int batch) {
     // wins; 2-bit rows and smaller K stay on the GEMV up to batch 8
     min_batch = (w->bits >= 3 && w->K >= 8192) ? 5 : 9;
   }
-  return batch >= min_batch && w->zeros == nullptr &&
+  return batch >= min_batch && w->zeros == nullptr && w->layout == HQ_LAYOUT_PACKED &&
          tc_col_block(w->bits, w->K) > 0;
 }
 
@@ -225,6 +227,7 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     a.status = l.status;
     a.xg = l.xp;
     a.zeros = w->zeros;
+    a.planes = w->layout == HQ_LAYOUT_BITPLANES;
     const cudaError_t e = launch_gemv(a, st);
     if (e != cudaSuccess) return from_cuda(e);
   }

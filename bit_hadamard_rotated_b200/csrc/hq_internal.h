@@ -38,6 +38,7 @@ struct GemvArgs {
   void* xg;       // gemv_scratch_bytes(K, N) bytes, 16-byte aligned: prep output
   const uint8_t* zeros = nullptr;  // per-group zero points [M][K/128], or nullptr: zero
   bool zero_frac = false;           // use zero_f (a fractional zero point) instead of zero
+  bool planes = false;              // 2-bit codes in the bit-plane layout
   float zero_f = 0.f;
 };
 

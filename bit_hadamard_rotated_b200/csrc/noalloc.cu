@@ -73,6 +73,8 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
       (w->signs && !aligned(w->signs, 16)) || (w->zeros && !aligned(w->zeros, 16))) {
     return HQ_ERR_INVALID_ARG;
   }
+  if (w->layout != HQ_LAYOUT_PACKED && w->layout != HQ_LAYOUT_BITPLANES) return HQ_ERR_INVALID_ARG;
+  if (w->layout == HQ_LAYOUT_BITPLANES && w->bits != 2) return HQ_ERR_UNSUPPORTED;
   if (batch < 0 || batch > 65535) return HQ_ERR_INVALID_ARG;
   if (batch == 0) return HQ_OK;
   if (!x || !y || !aligned(x, 16) || !aligned(y, 16)) return HQ_ERR_INVALID_ARG;
@@ -110,6 +112,7 @@ extern "C" hq_status hq_linear_noalloc(const hq_weight* w, const uint16_t* x, in
     a.status = reinterpret_cast<uint32_t*>(scratch);
     a.xg = scratch + kStatus;
     a.zeros = w->zeros;
+    a.planes = w->layout == HQ_LAYOUT_BITPLANES;
     if (launch_gemv(a, st) != cudaSuccess) {
       (void)cudaGetLastError();
       return HQ_ERR_CUDA;

@@ -76,8 +76,10 @@ def hq_quantize(W: torch.Tensor, bits: int, signs: torch.Tensor | None = None,
 
 
 def make_weight(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
-                bits: int, zero: int | None = None, zeros: torch.Tensor | None = None) -> HqWeight:
-    """Weight descriptor; zeros: optional per-group zero points uint8 [M][K/128]."""
+                bits: int, zero: int | None = None, zeros: torch.Tensor | None = None,
+                planes: bool = False) -> HqWeight:
+    """Weight descriptor; zeros: optional per-group zero points uint8 [M][K/128];
+    planes: 2-bit codes in the bit-plane layout (hq_to_bitplanes)."""
     M = qweight.shape[0]
     K = qweight.shape[1] * 32 // bits
     z = (1 << (bits - 1)) if zero is None else int(zero)
@@ -86,7 +88,7 @@ def make_weight(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor
         raise ValueError(f"zeros must be contiguous uint8 [{M}][{K // 128}]")
     return HqWeight(bits, M, K, z, qweight.data_ptr(), scales.data_ptr(),
                     None if signs is None else signs.data_ptr(),
-                    None if zeros is None else zeros.data_ptr())
+                    None if zeros is None else zeros.data_ptr(), 1 if planes else 0)
 
 
 def hq_linear_workspace_size(w: HqWeight, batch: int) -> int:
@@ -112,11 +114,12 @@ def _check_linear_io(w: HqWeight, x: torch.Tensor, out: torch.Tensor | None, dev
 def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
               x: torch.Tensor, bits: int, zero: int | None = None,
               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-              stream=None, zeros: torch.Tensor | None = None) -> torch.Tensor:
+              stream=None, zeros: torch.Tensor | None = None, planes: bool = False) -> torch.Tensor:
     """y[n][m] = sum_k scale (q - zero) x'[n][k]; x fp16 [N][K] -> y fp32 [N][M]
-    (zero per tensor, or per row and group with zeros uint8 [M][K/128])."""
+    (zero per tensor, or per row and group with zeros uint8 [M][K/128];
+    planes: 2-bit codes in the bit-plane layout)."""
     _need_cuda(qweight, scales, signs, x, zeros)
-    w = make_weight(qweight, scales, signs, bits, zero, zeros)
+    w = make_weight(qweight, scales, signs, bits, zero, zeros, planes)
     _check_linear_io(w, x, out, qweight.device)
     N = x.shape[0]
     with torch.cuda.device(qweight.device):
@@ -134,11 +137,11 @@ def hq_linear(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor |
 def hq_linear_noalloc(qweight: torch.Tensor, scales: torch.Tensor, signs: torch.Tensor | None,
                       x: torch.Tensor, bits: int, zero: int | None = None,
                       out: torch.Tensor | None = None, stream=None,
-                      zeros: torch.Tensor | None = None) -> torch.Tensor:
+                      zeros: torch.Tensor | None = None, planes: bool = False) -> torch.Tensor:
     """hq_linear without a workspace (the library's fixed device scratch is
     used instead; calls must not overlap on the GPU)."""
     _need_cuda(qweight, scales, signs, x, zeros)
-    w = make_weight(qweight, scales, signs, bits, zero, zeros)
+    w = make_weight(qweight, scales, signs, bits, zero, zeros, planes)
     _check_linear_io(w, x, out, qweight.device)
     N = x.shape[0]
     with torch.cuda.device(qweight.device):
@@ -157,10 +160,10 @@ def hq_linear_noalloc_check_status(stream=None) -> None:
 class RotatedLinear:
     """A packed, rotated linear layer bound to its device tensors and workspace."""
 
-    def __init__(self, qweight, scales, signs, bits, zero=None, max_batch=64, zeros=None):
+    def __init__(self, qweight, scales, signs, bits, zero=None, max_batch=64, zeros=None, planes=False):
         _need_cuda(qweight, scales, signs, zeros)
         self.qweight, self.scales, self.signs, self.bits, self.zeros = qweight, scales, signs, bits, zeros
-        self.w = make_weight(qweight, scales, signs, bits, zero, zeros)
+        self.w = make_weight(qweight, scales, signs, bits, zero, zeros, planes)
         self.workspace = torch.zeros(max(hq_linear_workspace_size(self.w, max_batch), 256),
                                      dtype=torch.uint8, device=qweight.device)
         # per-call marshalling reduced to the two tensor pointers and the stream
@@ -310,6 +313,17 @@ class KVCache:
         return out
 
 
+def hq_to_bitplanes(q2: torch.Tensor, stream=None) -> torch.Tensor:
+    """Packed 2-bit codes (int32 [..][K/16]) -> the same codes in the bit-plane
+    layout (same shape)."""
+    _need_cuda(q2)
+    if q2.dtype != torch.int32 or not q2.is_contiguous():
+        raise ValueError("q2 must be a contiguous int32 tensor")
+    out = torch.empty_like(q2)
+    check(lib().hq_to_bitplanes(_ptr(q2), q2.numel() * 16, _ptr(out), _stream(stream)), "hq_to_bitplanes")
+    return out
+
+
 def hq_split_nibbles(q8: torch.Tensor, K: int, stream=None):
     """(hi, lo) int32 [rows][K/8] nibble planes of 8-bit packed codes q8 [rows][K/4]."""
     _need_cuda(q8)
@@ -379,6 +393,6 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
-__all__ = ["KVCache", "ScreenedReadout", "hq_split_nibbles", "hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
+__all__ = ["hq_to_bitplanes", "KVCache", "ScreenedReadout", "hq_split_nibbles", "hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
            "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]

@@ -83,6 +83,15 @@ typedef enum {
 
 typedef enum { HQ_F16 = 0, HQ_BF16 = 1, HQ_F32 = 2 } hq_dtype;
 
+/* Storage of the codes of a weight row.  HQ_LAYOUT_PACKED: the little-endian
+ * bit stream above.  HQ_LAYOUT_BITPLANES (2-bit codes only): the codes as two
+ * bit-planes ("2-bit bit-planes ... kept that way for the whole run": Qwen3-8B
+ * BPDQ 2-bit card, introduction; the page gives no layout, this is the
+ * library's): per span of 32 codes k = 32 s + i, word 2s holds bit 0 of each
+ * code (at bit i), word 2s + 1 bit 1, so q = b0 + 2 b1.  Same size as the
+ * packed stream (K/16 words a row).  hq_to_bitplanes converts. */
+typedef enum { HQ_LAYOUT_PACKED = 0, HQ_LAYOUT_BITPLANES = 1 } hq_layout;
+
 /* One packed, rotated weight matrix W [M][K]. */
 typedef struct {
   int bits;                /* 2, 3, 4 or 8 */
@@ -98,6 +107,11 @@ typedef struct {
                               batch runs the small-batch kernel in blocks of up to
                               8 columns (the tensor-core path takes the scalar
                               zero only). */
+  int layout;              /* hq_layout of qweight (HQ_LAYOUT_PACKED = 0 when the
+                              struct is zero-initialised).  HQ_LAYOUT_BITPLANES
+                              needs bits = 2 (HQ_ERR_UNSUPPORTED otherwise) and,
+                              like per-group zeros, runs every batch on the
+                              small-batch kernel in blocks of up to 8 columns. */
 } hq_weight;
 
 /*
@@ -338,6 +352,13 @@ int hq_kv_attend_launches(void);
 hq_status hq_kv_attend(const hq_kv_cache* cache, int n_tokens, const uint16_t* q, int n_q,
                        int n_heads, float* out, void* workspace, size_t ws_bytes,
                        hq_stream_t stream);
+
+/* Converts 2-bit codes from the packed stream (n_codes / 16 words) to the
+ * bit-plane layout of HQ_LAYOUT_BITPLANES (as many words).  n_codes a
+ * multiple of 32; both arrays 8-byte aligned; 0 launches nothing.
+ * Bit-exact. */
+hq_status hq_to_bitplanes(const uint32_t* packed, size_t n_codes, uint32_t* planes,
+                          hq_stream_t stream);
 
 /* Intermediates an hq_moe_experts call leaves in its workspace, for checking
  * the layer stage by stage:

@@ -33,9 +33,10 @@ def test_status_strings(L):
 
 
 def W(**kw):
-    d = dict(bits=4, M=64, K=4096, zero=8, qweight=FAKE, scales=FAKE, signs=None)
+    d = dict(bits=4, M=64, K=4096, zero=8, qweight=FAKE, scales=FAKE, signs=None, zeros=None, layout=0)
     d.update(kw)
-    return HqWeight(d["bits"], d["M"], d["K"], d["zero"], d["qweight"], d["scales"], d["signs"])
+    return HqWeight(d["bits"], d["M"], d["K"], d["zero"], d["qweight"], d["scales"], d["signs"], d["zeros"],
+                    d["layout"])
 
 
 def lin(L, w, batch=1, x=FAKE, y=FAKE, ws=FAKE, ws_bytes=1 << 30):
@@ -50,6 +51,8 @@ def lin(L, w, batch=1, x=FAKE, y=FAKE, ws=FAKE, ws_bytes=1 << 30):
     (dict(zero=16), HQ_ERR_INVALID_ARG), (dict(zero=-1), HQ_ERR_INVALID_ARG),
     (dict(qweight=FAKE + 8), HQ_ERR_INVALID_ARG), (dict(scales=FAKE + 2), HQ_ERR_INVALID_ARG),
     (dict(signs=FAKE + 1), HQ_ERR_INVALID_ARG), (dict(qweight=None), HQ_ERR_INVALID_ARG),
+    (dict(layout=1), HQ_ERR_UNSUPPORTED), (dict(layout=2), HQ_ERR_INVALID_ARG),
+    (dict(bits=2, zero=2, layout=-1), HQ_ERR_INVALID_ARG), (dict(zeros=FAKE + 4), HQ_ERR_INVALID_ARG),
 ])
 def test_linear_rejects_bad_weight(L, kw, want):
     before = L.hq_launch_count()
@@ -227,3 +230,14 @@ def test_kv_cache_rejects_bad_args(L):
     assert att(ctypes.byref(c), 1000, FAKE, 32, 16, FAKE, FAKE, ws - 1, None) == HQ_ERR_WORKSPACE
     assert att(ctypes.byref(c), 1000, FAKE, 32, 16, FAKE, FAKE + 16, ws, None) == HQ_ERR_WORKSPACE
     assert att(ctypes.byref(c), 1000, FAKE, 1025, 16, FAKE, FAKE, 1 << 30, None) == HQ_ERR_UNSUPPORTED
+
+
+def test_to_bitplanes_rejects_bad_args(L):
+    before = L.hq_launch_count()
+    assert L.hq_to_bitplanes(FAKE, 48, FAKE, None) == HQ_ERR_INVALID_ARG       # not whole 32-code spans
+    assert L.hq_to_bitplanes(FAKE + 4, 64, FAKE, None) == HQ_ERR_INVALID_ARG   # misaligned
+    assert L.hq_to_bitplanes(None, 64, FAKE, None) == HQ_ERR_INVALID_ARG
+    assert L.hq_to_bitplanes(FAKE, 0, FAKE, None) == HQ_OK                      # nothing to do
+    assert L.hq_launch_count() == before
+    # the bit-plane layout is accepted for 2-bit weights (fails later, on the fake workspace size)
+    assert lin(L, W(bits=2, zero=2, layout=1), ws_bytes=0) == HQ_ERR_WORKSPACE

@@ -372,3 +372,42 @@ def test_linear_per_group_zeros_full_size_sampled():
         want, bound = oracle.linear(bits, M, K, 0, d["q"], d["scales"], d["signs"], d["x"], m_begin=m,
                                     m_end=m + 1, zeros=zeros)
         assert_within(y[:, m], want[:, m], bound[:, m], what=f"row {m}")
+
+
+# ---------------------------------------------------------------- 2-bit bit-plane storage
+@pytest.mark.parametrize("M,K,N,pgz", [(16, 128, 1, False), (37, 256, 3, False), (100, 1024, 2, True),
+                                       (333, 4096, 5, False), (96, 8192, 8, False), (200, 8192, 1, True),
+                                       (40, 16384, 2, False), (300, 32768, 1, False), (300, 4096, 19, True)])
+def test_linear_bit_planes(M, K, N, pgz):
+    """2-bit codes kept as bit-planes (HQ_LAYOUT_BITPLANES): the small-batch
+    kernel rebuilds each 32-code bundle's packed words in registers and reads
+    the activations in the matching order; batches past 8 run in blocks of 8.
+    Random words are valid plane words, so the synthetic q serves as is."""
+    from bit_hadamard_rotated_b200 import hq_linear
+    d = synth.linear(M, K, 2, N, seed=80 + M + K + N, scale_dist="loguniform", outlier_frac=0.01)
+    zeros = np.random.default_rng(M).integers(0, 4, size=(M, K // 128)).astype(np.uint8) if pgz else None
+    y = hq_linear(dev(d["q"].view(np.int32)), dev(d["scales"]), dev(d["signs"]), dev(d["x"]), 2,
+                  zeros=None if zeros is None else dev(zeros), planes=True).cpu().numpy()
+    want, bound = oracle.linear(2, M, K, 2, d["q"], d["scales"], d["signs"], d["x"], zeros=zeros, planes=True,
+                                threads=4)
+    assert_within(y, want, bound, what=f"planes M{M} K{K} N{N} pgz{pgz}")
+
+
+def test_to_bitplanes_bit_exact_and_linear_full_size_sampled():
+    """hq_to_bitplanes against the oracle's plane packer, then the 28672 x 8192
+    layer in bit-plane form at batch 1 on sampled rows."""
+    from bit_hadamard_rotated_b200 import hq_linear, hq_linear_noalloc, hq_to_bitplanes
+    M, K, N = 28672, 8192, 1
+    d = synth.linear(M, K, 2, N, seed=12, scale_dist="loguniform", outlier_frac=0.01)
+    planes = hq_to_bitplanes(dev(d["q"].view(np.int32))).cpu().numpy().view(np.uint32)
+    rng = np.random.default_rng(5)
+    for m in rng.choice(M, 64, replace=False):
+        assert np.array_equal(planes[m], oracle.pack_planes2(oracle.unpack(d["q"][m], 2, K))), m
+    gp = dev(planes.view(np.int32))
+    y = hq_linear(gp, dev(d["scales"]), dev(d["signs"]), dev(d["x"]), 2, planes=True).cpu().numpy()
+    y2 = hq_linear_noalloc(gp, dev(d["scales"]), dev(d["signs"]), dev(d["x"]), 2, planes=True).cpu().numpy()
+    # the planes hold d["q"]'s codes: the packed-stream oracle applies
+    for m in sample_rows(M, rng):
+        want, bound = oracle.linear(2, M, K, 2, d["q"], d["scales"], d["signs"], d["x"], m_begin=m, m_end=m + 1)
+        assert_within(y[:, m], want[:, m], bound[:, m], what=f"row {m}")
+        assert_within(y2[:, m], want[:, m], bound[:, m], what=f"noalloc row {m}")
