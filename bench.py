@@ -475,7 +475,7 @@ def measure_kv(device, stream, pk, l2):
         caches.append(c)
     q = torch.randn((n_q, n_heads, d), device=device).half()
     out = torch.empty((n_q, n_heads, d), dtype=torch.float32, device=device)
-    ws = torch.empty(caches[0].workspace_size(T, n_q, n_heads), dtype=torch.uint8, device=device)
+    ws = torch.zeros(caches[0].workspace_size(T, n_q, n_heads), dtype=torch.uint8, device=device)
     us = _graph_us(stream, device, [lambda c=c: c.attend(q, T, out=out, workspace=ws, stream=stream)
                                     for c in caches])
     kb, vb = torch.randn((32, n_kv, d), device=device).half(), torch.randn((32, n_kv, d), device=device).half()

@@ -306,11 +306,17 @@ class KVCache:
         if workspace is None:
             need = self.workspace_size(n_tokens, max(n_q, 1), n_heads)
             if self._ws is None or self._ws.numel() < need:
-                self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+                self._ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=q.device)
             workspace = self._ws
         check(lib().hq_kv_attend(ctypes.byref(self.c), int(n_tokens), _ptr(q), n_q, n_heads, _ptr(out),
                                  _ptr(workspace), workspace.numel(), _stream(stream)), "hq_kv_attend")
         return out
+
+    def check_status(self, workspace=None, stream=None) -> None:
+        """Raise HqError if an attend call on this workspace recorded a device error."""
+        ws = self._ws if workspace is None else workspace
+        if ws is not None:
+            check(lib().hq_check_status(_ptr(ws), _stream(stream)), "hq_kv_attend status")
 
 
 def hq_to_bitplanes(q2: torch.Tensor, stream=None) -> torch.Tensor:

@@ -345,9 +345,16 @@ int hq_kv_attend_launches(void);
  * and every 32-token block that n_tokens reaches must have been appended.
  * n_q * n_heads / n_kv_heads <= 4096 (HQ_ERR_UNSUPPORTED above); n_q = 0
  * launches nothing.  workspace: >= hq_kv_attend_workspace_size bytes,
- * 256-byte aligned (HQ_ERR_WORKSPACE otherwise); any contents.
- * Numerics: keys enter the tensor cores as two fp16 planes (hi + lo, about
- * 2^-22 relative) and p * v_scale likewise; sums in fp32.
+ * 256-byte aligned (HQ_ERR_WORKSPACE otherwise), zero-filled before its
+ * first use: its first word is a status word that a bounded device-side wait
+ * which ran out sets (read and cleared by hq_check_status).
+ * Numerics: a score is sum_c q_c s_c code + sum_c q_c min_c with every
+ * product exact in the tensor cores (the key scale split into two fp16
+ * halves whose products with a 4-bit code are exact), sums in fp32; p *
+ * v_scale enters as fp16 hi + lo (about 2^-22 relative); exp through the
+ * hardware 2^x (about 2^-22 relative).  Key groups whose scale times 15
+ * exceeds 65504 (a group spanning more than the fp16 range, keys beyond
+ * about +-32752 of both signs) are outside this exactness and overflow.
  */
 hq_status hq_kv_attend(const hq_kv_cache* cache, int n_tokens, const uint16_t* q, int n_q,
                        int n_heads, float* out, void* workspace, size_t ws_bytes,

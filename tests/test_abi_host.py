@@ -203,9 +203,10 @@ def test_kv_cache_rejects_bad_args(L):
 
     c = cache()
     ws = L.hq_kv_attend_workspace_size(ctypes.byref(c), 1000, 32, 16)
-    # 1000 tokens = 32 blocks, one per chunk (37 chunks per kv head would fill
-    # the SMs); per chunk 128 rows x (128 + 4) floats, for 4 kv heads
-    assert ws == 4 * 4 * 32 * 128 * 132
+    # 1000 tokens = 8 steps of 128, one per chunk (37 chunks per kv head would
+    # fill the SMs); a 256-byte status word, then per chunk 128 rows x
+    # (128 + 4) floats, for 4 kv heads
+    assert ws == 256 + 4 * 4 * 8 * 128 * 132
     assert L.hq_kv_attend_workspace_size(ctypes.byref(c), 1025, 32, 16) == 0     # past capacity
     assert L.hq_kv_attend_workspace_size(ctypes.byref(c), 1000, 32, 6) == 0      # heads not a multiple
     assert L.hq_kv_attend_workspace_size(ctypes.byref(cache(d=96)), 1000, 32, 16) == 0

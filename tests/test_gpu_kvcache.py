@@ -4,15 +4,17 @@ fp64 oracle.
 Codes, scales and minima are decided in IEEE single precision on both sides,
 so they must match bit for bit.  The attention output is floating point; its
 bound follows from the kernel's arithmetic, row by row:
-  - a dequantised key k = fl32(scale code + min) enters the tensor cores as
-    fp16 hi + lo, within 2^-22 |k| of k; products are exact and the 2d of
-    them per score are summed in fp32, so |ds_t| <= g_d S with
-    g_d = (2d + 4) 2^-24 and S = max_t sum_c |q_c k_tc| / sqrt(d);
+  - a score is sum_c q_c s_c n_tc + sum_c q_c m_c with every product exact in
+    the tensor cores (s = s_hi + s_lo, both halves times the code exact in
+    fp16; q and m fp16) and 3d products summed in fp32, so
+    |ds_t| <= g_d S with g_d = (3d + 4) 2^-24 and
+    S = max_t sum_c |q_c| (|k_tc| + 2 |m_c|) / sqrt(d) (|s n| <= |k| + |m|);
   - a score error moves the softmax weights by p_t (ds_t - sum p ds), so the
     output moves by at most 2 g_d S sum_t p_t |v_t| = 2 g_d S base;
-  - p v_scale enters as fp16 hi + lo (2^-22) and the weighted values are
-    summed in fp32 over at most T + 64 terms (inside a chunk, then across
-    chunks): g_T = (T + 64) 2^-24 relative to base.
+  - exp is the hardware 2^x (about 2^-22 relative), p v_scale enters as fp16
+    hi + lo (2^-22) and the weighted values are summed in fp32 over at most
+    T + 64 terms (inside a chunk, then across chunks): g_T = (T + 64) 2^-24
+    relative to base.
   tol = (2 g_d S + g_T + 2^-20) base + 1e-6.
 """
 import numpy as np
@@ -65,13 +67,15 @@ def tolerance(cache, T, q, base):
     """The bound of the module docstring for every output element."""
     n_kv, _, d, _ = cache["kc"].shape
     nb = (T + 31) // 32
+    km = np.abs(cache["km"][:, :nb].astype(np.float64))[..., None]
     K = (cache["ks"][:, :nb].astype(np.float64)[..., None] * cache["kc"][:, :nb]
          + cache["km"][:, :nb].astype(np.float64)[..., None])
-    K = np.abs(K.transpose(0, 1, 3, 2).reshape(n_kv, nb * 32, d)[:, :T])      # [h][t][c]
+    K = np.abs(K) + 2 * km                                                    # |k| + 2 |m|
+    K = K.transpose(0, 1, 3, 2).reshape(n_kv, nb * 32, d)[:, :T]              # [h][t][c]
     n_q, n_heads, _ = q.shape
     G = n_heads // n_kv
     qa = np.abs(q.astype(np.float64))
-    g_d = (2 * d + 4) * 2.0**-24
+    g_d = (3 * d + 4) * 2.0**-24
     g_T = (T + 64) * 2.0**-24
     tol = np.empty_like(base)
     for j in range(n_heads):
@@ -137,6 +141,7 @@ def test_attend_parity(T_app, T, n_kv, d, n_q, n_heads):
     n0 = hq_launch_count()
     check_attention(c, o, T, r["q"])
     assert hq_launch_count() - n0 == 2
+    c.check_status()
 
 
 def test_attend_large_scores():
