@@ -37,6 +37,7 @@ namespace ro {
 constexpr int kHistBits = 11;  // top bits of the order-preserving key in the coarse histogram
 constexpr int kHist = 1 << kHistBits;
 constexpr int kFinalCap = 2048;  // entries the final CTA sorts in shared memory
+constexpr int kRankMax = 512;    // lists up to this long are ranked directly (count^2 compares)
 constexpr int kMaxTopk = 256;
 constexpr int kMaxBatch = 8;
 constexpr int kBoundsThreads = 256;
@@ -159,6 +160,46 @@ __global__ void __launch_bounds__(kBoundsThreads)
 // edge of the histogram bin holding the topk-th largest L); then each warp
 // takes 32 rows, and for every row with U >= threshold computes its exact
 // logit from both planes and appends (logit, row) to the batch row's list.
+// The bin (of kHist, counted from the top) holding the need-th largest key,
+// and the number of entries in the bins above it: one warp, two rounds of
+// loads (each lane sums 64 bins; then the crossing lane's 64 bins, two per
+// lane), with inclusive scans across the lanes.
+__device__ __forceinline__ void top_bin(const uint32_t* h, uint32_t need, int lane, int* bin_out,
+                                        uint32_t* above_out) {
+  const int hi_bin = kHist - 64 * lane - 1;  // lane l: bins [hi_bin - 63, hi_bin]
+  uint32_t c = 0;
+  const uint4* g4 = reinterpret_cast<const uint4*>(h + hi_bin - 63);
+#pragma unroll
+  for (int b = 0; b < 16; ++b) {
+    const uint4 v = g4[b];
+    c += v.x + v.y + v.z + v.w;
+  }
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int first = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;  // crossing lane
+  const uint32_t base = __shfl_sync(0xffffffffu, incl - c, first);       // entries above its bins
+  const int top = kHist - 64 * first - 1;
+  // lane j: bins top - 2 j and top - 2 j - 1
+  const uint32_t b0 = h[top - 2 * lane], b1 = h[top - 2 * lane - 1];
+  uint32_t pair = b0 + b1, inc2 = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc2, o);
+    if (lane >= o) inc2 += y;
+  }
+  const uint32_t before_pair = base + inc2 - pair;  // entries above bin top - 2 j
+  const int j = __ffs(__ballot_sync(0xffffffffu, base + inc2 >= need)) - 1;
+  const uint32_t bp = __shfl_sync(0xffffffffu, before_pair, j);
+  const uint32_t first_of_pair = __shfl_sync(0xffffffffu, b0, j);
+  const bool in_first = bp + first_of_pair >= need;
+  *bin_out = in_first ? top - 2 * j : top - 2 * j - 1;
+  *above_out = in_first ? bp : bp + first_of_pair;
+}
+
 __global__ void __launch_bounds__(kRefineWarps * 32)
     ro_refine_kernel(const uint32_t* __restrict__ hi, const uint32_t* __restrict__ lo,
                      const uint16_t* __restrict__ scales, Ws w, Dims d) {
@@ -168,35 +209,10 @@ __global__ void __launch_bounds__(kRefineWarps * 32)
   const int n = blockIdx.y;
   pdl_wait();
   if (warp == 0) {
-    // lane l sums bins [kHist - 64 (l + 1), kHist - 64 l) (from the top)
-    const uint32_t* gh = w.hist + static_cast<size_t>(n) * kHist;
-    const int hi_bin = kHist - 64 * lane - 1;
-    uint32_t c = 0;
-    const uint4* g4 = reinterpret_cast<const uint4*>(gh + hi_bin - 63);
-#pragma unroll
-    for (int b = 0; b < 16; ++b) {
-      const uint4 v = g4[b];
-      c += v.x + v.y + v.z + v.w;
-    }
-    uint32_t incl = c;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t need = static_cast<uint32_t>(d.topk);
-    const unsigned crossing = __ballot_sync(0xffffffffu, incl >= need);
-    const int first = __ffs(crossing) - 1;  // the lane whose bins hold the topk-th largest
-    if (lane == first) {
-      uint32_t acc = incl - c;
-      int bin = hi_bin;
-      for (int b = 0; b < 64; ++b) {
-        acc += gh[hi_bin - b];
-        bin = hi_bin - b;
-        if (acc >= need) break;
-      }
-      s_tau = funkey(static_cast<uint32_t>(bin) << (32 - kHistBits));
-    }
+    int bin;
+    uint32_t above;
+    top_bin(w.hist + static_cast<size_t>(n) * kHist, static_cast<uint32_t>(d.topk), lane, &bin, &above);
+    if (lane == 0) s_tau = funkey(static_cast<uint32_t>(bin) << (32 - kHistBits));
   }
   __syncthreads();
   const float tau = s_tau;
@@ -215,6 +231,9 @@ __global__ void __launch_bounds__(kRefineWarps * 32)
     const uint32_t* lr = lo + static_cast<size_t>(m) * words;
     const __half* sr = reinterpret_cast<const __half*>(scales) + static_cast<size_t>(m) * G;
     float acc = 0.f;
+    // the loads of 8 iterations are independent: unrolled, they are issued
+    // together (one round trip to L2 per 8 instead of one per iteration)
+#pragma unroll 8
     for (int wd = lane; wd < words; wd += 32) {
       const uint32_t h = hr[wd], l = lr[wd];
       const float4 xa = *reinterpret_cast<const float4*>(xr + 8 * wd);
@@ -248,7 +267,7 @@ __device__ __forceinline__ bool before(float2 a, float2 b) {
 // first topk written out; the row's counters are cleared for the next call.
 __global__ void __launch_bounds__(kFinalThreads)
     ro_final_kernel(Ws w, Dims d, int32_t* __restrict__ ids, float* __restrict__ out) {
-  __shared__ uint32_t hist[kHist];
+  __shared__ __align__(16) uint32_t hist[kHist];
   __shared__ float2 keep[kFinalCap];
   __shared__ uint32_t s_prefix, s_need, s_kept;
   pdl_launch_dependents();
@@ -257,6 +276,26 @@ __global__ void __launch_bounds__(kFinalThreads)
   pdl_wait();
   const uint32_t count = w.cnt[n];
   const float2* lst = w.list + static_cast<size_t>(n) * d.V;
+  if (count <= static_cast<uint32_t>(kRankMax)) {
+    // a short list: every candidate's rank is the number of entries before
+    // it in (logit descending, row ascending), a total order, so the ranks
+    // 0 .. topk - 1 are the output positions
+    for (uint32_t i = tid; i < count; i += kFinalThreads) keep[i] = lst[i];
+    __syncthreads();
+    for (uint32_t i = tid; i < count; i += kFinalThreads) {
+      const float2 v = keep[i];
+      uint32_t rank = 0;
+      for (uint32_t j = 0; j < count; ++j) rank += before(keep[j], v) ? 1u : 0u;
+      if (rank < static_cast<uint32_t>(d.topk)) {
+        ids[static_cast<size_t>(n) * d.topk + rank] = __float_as_int(v.y);
+        out[static_cast<size_t>(n) * d.topk + rank] = v.x;
+      }
+    }
+    uint32_t* gh = w.hist + static_cast<size_t>(n) * kHist;
+    for (int i = tid; i < kHist; i += kFinalThreads) gh[i] = 0u;
+    if (tid == 0) w.cnt[n] = 0u;
+    return;
+  }
   uint32_t prefix = 0u, pmask = 0u;
   if (tid == 0) {
     s_need = static_cast<uint32_t>(d.topk);
@@ -274,10 +313,16 @@ __global__ void __launch_bounds__(kFinalThreads)
     }
     __syncthreads();
     if (warp == 0) {
+      // the bin from the top where the count reaches s_need: each lane sums
+      // per = nb / 32 bins, a scan across lanes finds the crossing lane, then
+      // its bins (per / 32 a lane) are scanned the same way
       const int nb = static_cast<int>(bmask) + 1, per = nb / 32;
       const int top = nb - per * lane - 1;
       uint32_t c = 0;
-      for (int b = 0; b < per; ++b) c += hist[top - b];
+      for (int b = 0; b < per; b += 4) {
+        const uint4 v = *reinterpret_cast<const uint4*>(&hist[top - per + 1 + b]);
+        c += v.x + v.y + v.z + v.w;
+      }
       uint32_t incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -286,13 +331,28 @@ __global__ void __launch_bounds__(kFinalThreads)
       }
       const uint32_t need = s_need;
       const int first = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;
-      if (lane == first) {
-        uint32_t acc = incl - c;
-        int bin = top;
-        for (int b = 0; b < per; ++b) {
-          bin = top - b;
-          if (acc + hist[bin] >= need) break;
-          acc += hist[bin];
+      const uint32_t base = __shfl_sync(0xffffffffu, incl - c, first);
+      const int ftop = nb - per * first - 1;
+      const int q = per / 32;  // bins per lane in the second scan (1 or 2)
+      uint32_t bv[2] = {0u, 0u}, own = 0u;
+      for (int k = 0; k < q; ++k) {
+        bv[k] = hist[ftop - q * lane - k];
+        own += bv[k];
+      }
+      uint32_t inc2 = own;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc2, o);
+        if (lane >= o) inc2 += y;
+      }
+      const int j = __ffs(__ballot_sync(0xffffffffu, base + inc2 >= need)) - 1;
+      if (lane == j) {
+        uint32_t acc = base + inc2 - own;  // entries above this lane's bins
+        int bin = ftop - q * lane;
+        for (int k = 0; k < q; ++k) {
+          bin = ftop - q * lane - k;
+          if (acc + bv[k] >= need) break;
+          acc += bv[k];
         }
         s_need = need - acc;
         s_prefix = prefix | (static_cast<uint32_t>(bin) << sh);
