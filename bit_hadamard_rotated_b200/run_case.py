@@ -1,9 +1,12 @@
-"""Run one hq_linear (or one MoE layer) case a few times on seeded synthetic inputs.
+"""Run one hq_linear (or one MoE layer, KV attention or screened readout) case a
+few times on seeded synthetic inputs.
 
 A reproducible target for profilers and quick timing:
 
     python -m bit_hadamard_rotated_b200.run_case --M 12288 --K 4096 --bits 2 --batch 1
     python -m bit_hadamard_rotated_b200.run_case --moe
+    python -m bit_hadamard_rotated_b200.run_case --kv --tokens 8192
+    python -m bit_hadamard_rotated_b200.run_case --readout
 
 Inputs come from bit_hadamard_rotated_b200.synth (seeded); every call goes
 through the C ABI.  Prints the mean device time per call (CUDA events around
@@ -17,7 +20,50 @@ import numpy as np
 import torch
 
 from . import synth
-from .hq import RotatedLinear, expert_table, hq_check_status, hq_moe_experts, hq_moe_workspace_size
+from .hq import (KVCache, RotatedLinear, ScreenedReadout, expert_table, hq_check_status, hq_moe_experts,
+                 hq_moe_workspace_size)
+
+
+def _timed(fn, a):
+    for _ in range(a.warmup):
+        fn()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(a.reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / max(a.reps, 1)
+
+
+def run_kv(a):
+    """Attention of a 32-token block (16 heads) over an int4 cache of --tokens
+    tokens (4 kv heads of 128 channels), filled by hq_kv_append."""
+    r = synth.kv(T=a.tokens, seed=a.seed)
+    dev = torch.device("cuda", 0)
+    c = KVCache(r["n_kv"], r["d"], r["T"], dev)
+    c.append(torch.from_numpy(r["k"]).to(dev), torch.from_numpy(r["v"]).to(dev), 0)
+    q = torch.from_numpy(r["q"]).to(dev)
+    out = torch.empty((r["n_q"], r["n_heads"], r["d"]), dtype=torch.float32, device=dev)
+    us = _timed(lambda: c.attend(q, r["T"], out=out), a)
+    c.check_status()
+    R = r["n_q"] * r["n_heads"] // r["n_kv"]
+    flops = 4.0 * R * r["T"] * r["d"] * r["n_kv"]
+    print(f"kv attend T={r['T']} kv heads {r['n_kv']} d={r['d']} query tokens {r['n_q']} x {r['n_heads']} heads: "
+          f"{us:.2f} us/call ({flops / (us * 1e-6) / 1e12:.1f} TFLOP/s)")
+
+
+def run_readout(a):
+    """Screened top-8 readout over the 157,184 x 2048 8-bit lm_head (nibble planes), batch 1."""
+    r = synth.readout(N=1, seed=a.seed)
+    dev = torch.device("cuda", 0)
+    hi = torch.from_numpy(r["hi"].view(np.int32)).to(dev)
+    lo = torch.from_numpy(r["lo"].view(np.int32)).to(dev)
+    ro = ScreenedReadout(hi, lo, torch.from_numpy(r["scales"]).to(dev), torch.from_numpy(r["signs"]).to(dev),
+                         r["zero"], max_batch=1)
+    x = torch.from_numpy(r["x"]).to(dev)
+    us = _timed(lambda: ro.topk(x, 8), a)
+    print(f"screened readout V={r['V']} K={r['K']} top-8 batch 1: {us:.2f} us/call")
 
 
 def run_linear(a):
@@ -91,10 +137,20 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--moe", action="store_true", help="run the MoE expert layer instead")
+    ap.add_argument("--kv", action="store_true", help="run the int4 KV attention instead")
+    ap.add_argument("--tokens", type=int, default=8192, help="cached tokens for --kv")
+    ap.add_argument("--readout", action="store_true", help="run the screened readout instead")
     a = ap.parse_args()
     if not torch.cuda.is_available():
         raise SystemExit("run_case needs a CUDA device")
-    run_moe(a) if a.moe else run_linear(a)
+    if a.moe:
+        run_moe(a)
+    elif a.kv:
+        run_kv(a)
+    elif a.readout:
+        run_readout(a)
+    else:
+        run_linear(a)
 
 
 if __name__ == "__main__":
