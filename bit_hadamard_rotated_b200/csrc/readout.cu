@@ -61,6 +61,8 @@ struct Ws {
   float* U;        // [N][V]
   uint32_t* hist;  // [N][kHist] histogram of L's top bits (zero between calls)
   uint32_t* cnt;   // [N] candidates listed (zero between calls)
+  uint32_t* done;  // [N] bounds CTAs finished (zero between calls)
+  float* tau;      // [N] candidate threshold (lower edge of the topk-th largest L's bin)
   float2* list;    // [N][V] (exact logit, row as int bits)
 };
 
@@ -85,7 +87,7 @@ static Plan plan(int V, int K, int N) {
       4 * static_cast<size_t>(N) * V,
       4 * static_cast<size_t>(N) * V,
       4 * static_cast<size_t>(N) * kHist,
-      4 * static_cast<size_t>(N),
+      4 * 3 * static_cast<size_t>(kMaxBatch),  // cnt [N], done [N], tau [N] (kMaxBatch each)
       8 * static_cast<size_t>(N) * V,
   };
   size_t o = 0;
@@ -107,12 +109,54 @@ static Ws carve(void* base, const Plan& pl) {
   w.U = reinterpret_cast<float*>(b + pl.off[4]);
   w.hist = reinterpret_cast<uint32_t*>(b + pl.off[5]);
   w.cnt = reinterpret_cast<uint32_t*>(b + pl.off[6]);
+  w.done = w.cnt + kMaxBatch;
+  w.tau = reinterpret_cast<float*>(w.cnt + 2 * kMaxBatch);
   w.list = reinterpret_cast<float2*>(b + pl.off[7]);
   return w;
 }
 
 // Grid (ceil(V / 256), N): per row m of batch row n, sd, L and U; U stored, the
 // top 11 bits of L's key counted (shared-memory histogram, then merged).
+// The bin (of kHist, counted from the top) holding the need-th largest key,
+// and the number of entries in the bins above it: one warp, two rounds of
+// loads (each lane sums 64 bins; then the crossing lane's 64 bins, two per
+// lane), with inclusive scans across the lanes.
+__device__ __forceinline__ void top_bin(const uint32_t* h, uint32_t need, int lane, int* bin_out,
+                                        uint32_t* above_out) {
+  const int hi_bin = kHist - 64 * lane - 1;  // lane l: bins [hi_bin - 63, hi_bin]
+  uint32_t c = 0;
+  const uint4* g4 = reinterpret_cast<const uint4*>(h + hi_bin - 63);
+#pragma unroll
+  for (int b = 0; b < 16; ++b) {
+    const uint4 v = __ldcg(g4 + b);
+    c += v.x + v.y + v.z + v.w;
+  }
+  uint32_t incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int first = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;  // crossing lane
+  const uint32_t base = __shfl_sync(0xffffffffu, incl - c, first);       // entries above its bins
+  const int top = kHist - 64 * first - 1;
+  // lane j: bins top - 2 j and top - 2 j - 1
+  const uint32_t b0 = __ldcg(h + top - 2 * lane), b1 = __ldcg(h + top - 2 * lane - 1);
+  uint32_t pair = b0 + b1, inc2 = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc2, o);
+    if (lane >= o) inc2 += y;
+  }
+  const uint32_t before_pair = base + inc2 - pair;  // entries above bin top - 2 j
+  const int j = __ffs(__ballot_sync(0xffffffffu, base + inc2 >= need)) - 1;
+  const uint32_t bp = __shfl_sync(0xffffffffu, before_pair, j);
+  const uint32_t first_of_pair = __shfl_sync(0xffffffffu, b0, j);
+  const bool in_first = bp + first_of_pair >= need;
+  *bin_out = in_first ? top - 2 * j : top - 2 * j - 1;
+  *above_out = in_first ? bp : bp + first_of_pair;
+}
+
 __global__ void __launch_bounds__(kBoundsThreads)
     ro_bounds_kernel(const uint16_t* __restrict__ scales, Ws w, Dims d) {
   __shared__ float x2[256];     // sum of x'^2 over each group (G <= 256)
@@ -154,68 +198,37 @@ __global__ void __launch_bounds__(kBoundsThreads)
   for (int i = tid; i < kHist; i += kBoundsThreads) {
     if (hist[i] != 0u) atomicAdd(&gh[i], hist[i]);
   }
+  // the last CTA of the row to finish finds the threshold once (every other
+  // CTA's histogram adds are visible after its fence and counter increment)
+  __shared__ bool s_last;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(w.done + n, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (s_last && warp == 0) {
+    __threadfence();
+    int bin;
+    uint32_t above;
+    top_bin(gh, static_cast<uint32_t>(d.topk), lane, &bin, &above);
+    if (lane == 0) {
+      w.tau[n] = funkey(static_cast<uint32_t>(bin) << (32 - kHistBits));
+      w.done[n] = 0u;
+    }
+  }
 }
 
 // Grid (ceil(V / (32 warps)), N): warp 0 first finds the threshold (the lower
 // edge of the histogram bin holding the topk-th largest L); then each warp
 // takes 32 rows, and for every row with U >= threshold computes its exact
 // logit from both planes and appends (logit, row) to the batch row's list.
-// The bin (of kHist, counted from the top) holding the need-th largest key,
-// and the number of entries in the bins above it: one warp, two rounds of
-// loads (each lane sums 64 bins; then the crossing lane's 64 bins, two per
-// lane), with inclusive scans across the lanes.
-__device__ __forceinline__ void top_bin(const uint32_t* h, uint32_t need, int lane, int* bin_out,
-                                        uint32_t* above_out) {
-  const int hi_bin = kHist - 64 * lane - 1;  // lane l: bins [hi_bin - 63, hi_bin]
-  uint32_t c = 0;
-  const uint4* g4 = reinterpret_cast<const uint4*>(h + hi_bin - 63);
-#pragma unroll
-  for (int b = 0; b < 16; ++b) {
-    const uint4 v = g4[b];
-    c += v.x + v.y + v.z + v.w;
-  }
-  uint32_t incl = c;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  const int first = __ffs(__ballot_sync(0xffffffffu, incl >= need)) - 1;  // crossing lane
-  const uint32_t base = __shfl_sync(0xffffffffu, incl - c, first);       // entries above its bins
-  const int top = kHist - 64 * first - 1;
-  // lane j: bins top - 2 j and top - 2 j - 1
-  const uint32_t b0 = h[top - 2 * lane], b1 = h[top - 2 * lane - 1];
-  uint32_t pair = b0 + b1, inc2 = pair;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, inc2, o);
-    if (lane >= o) inc2 += y;
-  }
-  const uint32_t before_pair = base + inc2 - pair;  // entries above bin top - 2 j
-  const int j = __ffs(__ballot_sync(0xffffffffu, base + inc2 >= need)) - 1;
-  const uint32_t bp = __shfl_sync(0xffffffffu, before_pair, j);
-  const uint32_t first_of_pair = __shfl_sync(0xffffffffu, b0, j);
-  const bool in_first = bp + first_of_pair >= need;
-  *bin_out = in_first ? top - 2 * j : top - 2 * j - 1;
-  *above_out = in_first ? bp : bp + first_of_pair;
-}
-
 __global__ void __launch_bounds__(kRefineWarps * 32)
     ro_refine_kernel(const uint32_t* __restrict__ hi, const uint32_t* __restrict__ lo,
                      const uint16_t* __restrict__ scales, Ws w, Dims d) {
-  __shared__ float s_tau;
   pdl_launch_dependents();
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n = blockIdx.y;
   pdl_wait();
-  if (warp == 0) {
-    int bin;
-    uint32_t above;
-    top_bin(w.hist + static_cast<size_t>(n) * kHist, static_cast<uint32_t>(d.topk), lane, &bin, &above);
-    if (lane == 0) s_tau = funkey(static_cast<uint32_t>(bin) << (32 - kHistBits));
-  }
-  __syncthreads();
-  const float tau = s_tau;
+  const float tau = w.tau[n];
   const int words = d.K / 8;  // uint32 words of a 4-bit plane row
   const int G = d.K / kGroup;
   const float* xr = w.xr + static_cast<size_t>(n) * d.K;
