@@ -271,7 +271,7 @@ def run_ours(a):
                         "frac_bf16_peak": round(tf / pk["bf16"], 4),
                         "weight_gbs": round(wb / (us * 1e-6) / 1e9, 1),
                         "frac_hbm": round(wb / (us * 1e-6) / 1e9 / pk["hbm"], 4),
-                        "path": "tensor cores" if lins[0].uses_tensor_cores(n) else "GEMV",
+                        "path": lins[0].path(n),
                         "launches_per_call": lins[0].launches(n),
                         "timing": f"{reps} back-to-back calls in one graph, {copies} weight "
                                   f"copies cycled"}
@@ -380,7 +380,7 @@ def measure_configs(device, stream, pk, l2):
         tf = 2.0 * M * K * N / (us * 1e-6) / 1e12
         r = {"us": round(us, 3), "weight_gbs": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm"], 4),
              "tflops": round(tf, 2), "frac_bf16_peak": round(tf / pk["bf16"], 4),
-             "path": "tensor cores" if lins[0].uses_tensor_cores(N) else "GEMV",
+             "path": lins[0].path(N),
              "launches": lins[0].launches(N)}
         del lins
         return r

@@ -20,6 +20,7 @@ HQ_OK, HQ_ERR_INVALID_ARG, HQ_ERR_UNSUPPORTED, HQ_ERR_WORKSPACE, HQ_ERR_CUDA, HQ
 HQ_F16, HQ_BF16, HQ_F32 = 0, 1, 2
 HQ_MOE_POS, HQ_MOE_H, HQ_MOE_D = 0, 1, 2
 HQ_LAYOUT_PACKED, HQ_LAYOUT_BITPLANES = 0, 1
+HQ_PATH_GEMV, HQ_PATH_TENSOR, HQ_PATH_GEMV32 = 0, 1, 2
 
 _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -115,6 +116,10 @@ def lib() -> ctypes.CDLL:
         L.hq_set_test_fault.restype = _i
         L.hq_set_tc_min_batch.argtypes = [_i]
         L.hq_set_tc_min_batch.restype = _i
+        L.hq_set_gemv32_min_batch.argtypes = [_i]
+        L.hq_set_gemv32_min_batch.restype = _i
+        L.hq_linear_path.argtypes = [ctypes.POINTER(HqWeight), _i]
+        L.hq_linear_path.restype = _i
         _lib = L
     return _lib
 

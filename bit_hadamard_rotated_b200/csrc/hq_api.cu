@@ -12,6 +12,8 @@ namespace hq {
 static std::atomic<uint64_t> g_launches{0};
 // Batch from which hq_linear uses the tensor-core GEMM; 0 = automatic.
 static std::atomic<int> g_tc_min_batch{0};
+// Batch from which hq_linear uses the 32-row GEMV (up to batch 16); 0 = automatic.
+static std::atomic<int> g_g32_min_batch{0};
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
@@ -33,6 +35,11 @@ static bool is_pow2(long v) { return v > 0 && (v & (v - 1)) == 0; }
 static size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 constexpr size_t kStatusBytes = 256;
+// Words of the counter region (after the tensor-core GEMM's per-CTA-boundary
+// counters) that the 32-row GEMV's rotation gate uses.
+constexpr int kG32SyncWord = 192;
+static_assert(kG32SyncWord >= kMaxTcGrid && (kG32SyncWord + 2) * 4 <= static_cast<int>(kTcCounterBytes),
+              "gate words inside the counter region, past the tensor-core counters");
 constexpr int kMaxColBlock = 8;
 
 static hq_status from_cuda(cudaError_t e) {
@@ -66,21 +73,32 @@ static int gemv_col_block(int bits, int K, bool pgz) {
   return 0;
 }
 
-// Batches of at least the tensor-core threshold run on the tcgen05 GEMM
-// (when a tile plan fits this width and K); smaller ones on the GEMV.
-static bool use_tc(const hq_weight* w, int batch) {
-  int min_batch = g_tc_min_batch.load(std::memory_order_relaxed);
-  if (min_batch == 0) {
-    // automatic, from batch sweeps on B200: the GEMV stages its activation
-    // fragments (2.5 K bytes per column) in shared memory; past ~90 KB of
-    // them (5 columns at K = 8192) its copy rings become too shallow for
-    // 3/4/8-bit rows, and the tensor-core GEMM (flat in time up to batch 32)
-    // wins; 2-bit rows and smaller K stay on the GEMV up to batch 8
-    min_batch = (w->bits >= 3 && w->K >= 8192) ? 5 : 9;
-  }
-  return batch >= min_batch && w->zeros == nullptr && w->layout == HQ_LAYOUT_PACKED &&
-         tc_col_block(w->bits, w->K) > 0;
+// The batch-8 GEMV stages its activation fragments (2 K bytes per column) in
+// shared memory for the whole of K; past ~90 KB of them (5 columns at
+// K = 8192) its copy rings become too shallow for 3/4/8-bit rows.  From there
+// (batch 5 at K >= 8192, 3/4/8 bits; batch 9 otherwise) up to batch 16 the
+// 32-row GEMV, which stages K in slices, takes over where it applies, and the
+// tensor-core GEMM beyond (or where it does not apply).
+static int auto_min_batch(const hq_weight* w) { return (w->bits >= 3 && w->K >= 8192) ? 5 : 9; }
+
+static bool tc_fits(const hq_weight* w) {
+  return w->zeros == nullptr && w->layout == HQ_LAYOUT_PACKED && tc_col_block(w->bits, w->K) > 0;
 }
+
+static hq_path path_of(const hq_weight* w, int batch) {
+  const int tc_min = g_tc_min_batch.load(std::memory_order_relaxed);
+  if (tc_min > 0 && batch >= tc_min && tc_fits(w)) return HQ_PATH_TENSOR;
+  int g32_min = g_g32_min_batch.load(std::memory_order_relaxed);
+  if (g32_min == 0) g32_min = auto_min_batch(w);
+  if (batch >= g32_min && batch <= 16 && w->zeros == nullptr &&
+      gemv32_supported(w->bits, w->M, w->K, batch)) {
+    return HQ_PATH_GEMV32;
+  }
+  if (tc_min == 0 && batch >= auto_min_batch(w) && tc_fits(w)) return HQ_PATH_TENSOR;
+  return HQ_PATH_GEMV;
+}
+
+static bool use_tc(const hq_weight* w, int batch) { return path_of(w, batch) == HQ_PATH_TENSOR; }
 
 // hq_linear workspace: [status 256 B] [tensor-core tile counters 1 KiB, zero
 // between calls] [on the tensor-core path the rotated activation images
@@ -99,9 +117,11 @@ struct LinearWs {
 static LinearWs linear_ws(void* base, const hq_weight* w, int batch) {
   LinearWs l{};
   const int nb = gemv_col_block(w->bits, w->K, w->zeros != nullptr);
-  const size_t xp_bytes = use_tc(w, batch)
-                              ? align256(tc_xp_bytes(w->bits, w->K, batch))
-                              : align256(gemv_scratch_bytes(w->K, nb > 0 ? std::min(nb, std::max(batch, 1)) : 1));
+  const hq_path path = batch > 0 ? path_of(w, batch) : HQ_PATH_GEMV;
+  const size_t xp_bytes =
+      path == HQ_PATH_TENSOR   ? align256(tc_xp_bytes(w->bits, w->K, batch))
+      : path == HQ_PATH_GEMV32 ? align256(gemv32_scratch_bytes(w->K, batch))
+                               : align256(gemv_scratch_bytes(w->K, nb > 0 ? std::min(nb, std::max(batch, 1)) : 1));
   uint8_t* b = static_cast<uint8_t*>(base);
   l.status = reinterpret_cast<uint32_t*>(b);
   l.counters = reinterpret_cast<uint32_t*>(b + kStatusBytes);
@@ -141,6 +161,16 @@ int hq_set_tc_min_batch(int n) {
   return g_tc_min_batch.exchange(n);
 }
 
+int hq_set_gemv32_min_batch(int n) {
+  if (n < 0) return g_g32_min_batch.load();
+  return g_g32_min_batch.exchange(n);
+}
+
+int hq_linear_path(const hq_weight* w, int batch) {
+  if (check_weight(w) != HQ_OK || batch <= 0) return -1;
+  return static_cast<int>(path_of(w, batch));
+}
+
 hq_status hq_rotate(const void* x, hq_dtype x_dtype, void* x_rot, hq_dtype out_dtype, int n_rows,
                     int K, const int8_t* signs, hq_stream_t stream) {
   if (n_rows < 0) return HQ_ERR_INVALID_ARG;
@@ -170,7 +200,9 @@ int hq_linear_uses_tensor_cores(const hq_weight* w, int batch) {
 
 int hq_linear_launches(const hq_weight* w, int batch) {
   if (check_weight(w) != HQ_OK || batch <= 0) return 0;
-  if (use_tc(w, batch)) return tc_launches(w->bits, w->K, batch);
+  const hq_path path = path_of(w, batch);
+  if (path == HQ_PATH_TENSOR) return tc_launches(w->bits, w->K, batch);
+  if (path == HQ_PATH_GEMV32) return gemv32_launches(w->bits, w->M, w->K, batch);
   const int nb = gemv_col_block(w->bits, w->K, w->zeros != nullptr);
   if (nb == 0) return 0;
   int n = 0;
@@ -191,7 +223,27 @@ hq_status hq_linear(const hq_weight* w, const uint16_t* x, int batch, float* y, 
     return HQ_ERR_WORKSPACE;
   }
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (use_tc(w, batch)) {
+  const hq_path path = path_of(w, batch);
+  if (path == HQ_PATH_GEMV32) {
+    GemvArgs a;
+    a.bits = w->bits;
+    a.M = w->M;
+    a.K = w->K;
+    a.N = batch;
+    a.zero = w->zero;
+    a.q = w->qweight;
+    a.scales = w->scales;
+    a.x = x;
+    a.signs = w->signs;
+    a.y = y;
+    a.ldy = w->M;
+    a.status = l.status;
+    a.xg = l.xp;
+    a.planes = w->layout == HQ_LAYOUT_BITPLANES;
+    a.sync = l.counters + kG32SyncWord;
+    return from_cuda(launch_gemv32(a, st));
+  }
+  if (path == HQ_PATH_TENSOR) {
     TcArgs a;
     a.bits = w->bits;
     a.M = w->M;

@@ -40,6 +40,7 @@ struct GemvArgs {
   bool zero_frac = false;           // use zero_f (a fractional zero point) instead of zero
   bool planes = false;              // 2-bit codes in the bit-plane layout
   float zero_f = 0.f;
+  uint32_t* sync = nullptr;  // two words, zero between calls: the 32-row GEMV's rotation gate
 };
 
 // Shared memory the GEMV needs for a batch block of nb <= 8 rows, with or
@@ -66,6 +67,14 @@ cudaError_t tensor_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, const voi
 cudaError_t tensor_map_3d(CUtensorMap* map, CUtensorMapDataType dtype, const void* base,
                           const uint64_t (&dims)[3], const uint64_t (&strides_bytes)[2],
                           const uint32_t (&box)[3], CUtensorMapSwizzle swizzle);
+
+// The 32-row GEMV for batches up to 16 (gemv32.cu): whether a launch shape
+// fits (K >= 1024, the scalar zero point, at most 16 tiles per CTA), the
+// scratch for its prep output, and one prep + GEMV launch pair.
+bool gemv32_supported(int bits, int M, int K, int N);
+int gemv32_launches(int bits, int M, int K, int N);
+size_t gemv32_scratch_bytes(int K, int N);
+cudaError_t launch_gemv32(const GemvArgs& a, cudaStream_t st);
 
 // Tensor-core path (tcgen05) for larger batches.
 struct TcArgs {

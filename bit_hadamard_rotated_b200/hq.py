@@ -185,8 +185,14 @@ class RotatedLinear:
         return int(lib().hq_linear_launches(ctypes.byref(self.w), batch))
 
     def uses_tensor_cores(self, batch: int) -> bool:
-        """Whether a call of this batch runs on the tensor-core GEMM (else the GEMV)."""
+        """Whether a call of this batch runs on the tensor-core GEMM (else a GEMV)."""
         return int(lib().hq_linear_uses_tensor_cores(ctypes.byref(self.w), batch)) == 1
+
+    def path(self, batch: int) -> str:
+        """The kernel family a call of this batch runs on: "GEMV", "tensor cores"
+        or "GEMV32" (32-row tiles, up to 16 columns)."""
+        p = int(lib().hq_linear_path(ctypes.byref(self.w), batch))
+        return {0: "GEMV", 1: "tensor cores", 2: "GEMV32"}[p]
 
     def __call__(self, x, out=None, stream=None):
         N = x.shape[0]
@@ -399,6 +405,10 @@ def hq_set_tc_min_batch(n: int) -> int:
     return int(lib().hq_set_tc_min_batch(n))
 
 
+def hq_set_gemv32_min_batch(n: int) -> int:
+    return int(lib().hq_set_gemv32_min_batch(n))
+
+
 __all__ = ["hq_to_bitplanes", "KVCache", "ScreenedReadout", "hq_split_nibbles", "hq_quantize", "hq_rotate", "hq_linear", "hq_linear_noalloc", "hq_linear_noalloc_check_status", "hq_linear_workspace_size", "RotatedLinear",
            "hq_moe_experts", "hq_moe_workspace_size", "expert_table", "hq_check_status",
-           "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "HqError", "make_weight"]
+           "hq_unpack_codes", "hq_launch_count", "hq_set_tc_min_batch", "hq_set_gemv32_min_batch", "HqError", "make_weight"]

@@ -427,10 +427,34 @@ int hq_moe_launches(void);
 int hq_linear_uses_tensor_cores(const hq_weight* w, int batch);
 
 /* Batch size from which hq_linear uses the tensor-core GEMM (when K >= 1024).
- * 0 (the default) selects it automatically: from batch 5 for 3/4/8-bit codes
- * with K >= 8192, else from batch 9.  A value >= 1 applies to every weight.
+ * 0 (the default) selects it automatically: from batch 17 where the 32-row
+ * GEMV takes batches up to 16 (hq_linear_path), else from batch 5 for
+ * 3/4/8-bit codes with K >= 8192 and from batch 9 otherwise.  A value >= 1
+ * applies to every weight and takes precedence over the 32-row GEMV.
  * Returns the previous value; negative values change nothing. */
 int hq_set_tc_min_batch(int n);
+
+/* The kernel family hq_linear runs a weight and batch on. */
+typedef enum {
+  HQ_PATH_GEMV = 0,    /* register-decode GEMV, batch blocks of up to 8 */
+  HQ_PATH_TENSOR = 1,  /* tcgen05 GEMM (codes dequantised into tensor memory) */
+  HQ_PATH_GEMV32 = 2   /* register-decode GEMV over 32-row tiles, up to 16 columns */
+} hq_path;
+
+/* The hq_path of hq_linear for this weight and batch; -1 for an invalid
+ * weight or batch < 1 (nothing is launched).  The 32-row GEMV applies to the
+ * packed and bit-plane layouts with the scalar zero point, K >= 1024 and at
+ * most 16 x 148 32-row tiles' worth of rows per streaming multiprocessor
+ * count (M <= 75,776 on a B200). */
+int hq_linear_path(const hq_weight* w, int batch);
+
+/* Batch size from which hq_linear uses the 32-row GEMV (batches up to 16,
+ * where it applies).  0 (the default) selects it automatically: from batch 5
+ * for 3/4/8-bit codes with K >= 8192, else from batch 9.  n >= 1 applies to
+ * every weight (n = 1: every batch up to 16); an explicit
+ * hq_set_tc_min_batch still takes precedence.  Returns the previous value;
+ * negative values change nothing. */
+int hq_set_gemv32_min_batch(int n);
 
 /* For tests of the device error path (no counterpart on the pages): the next
  * n launches of the small-batch GEMV kernel each leave one shared-memory copy

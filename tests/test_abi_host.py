@@ -169,15 +169,46 @@ def test_linear_path_choice():
     from bit_hadamard_rotated_b200._lib import lib
     L = lib()
 
-    def path(bits, K, batch):
-        w = HqWeight(bits, 256, K, 1 << (bits - 1), FAKE, FAKE, None)
-        return L.hq_linear_uses_tensor_cores(ctypes.byref(w), batch)
+    from bit_hadamard_rotated_b200._lib import HQ_PATH_GEMV, HQ_PATH_GEMV32, HQ_PATH_TENSOR
 
-    assert path(3, 8192, 4) == 0 and path(3, 8192, 5) == 1
-    assert path(8, 16384, 5) == 1 and path(4, 4096, 8) == 0 and path(4, 4096, 9) == 1
-    assert path(2, 8192, 8) == 0 and path(2, 8192, 9) == 1
-    assert path(4, 512, 64) == 0      # K < 1024: GEMV at every batch
-    assert path(4, 4096, 0) == -1 and path(5, 4096, 4) == -1
+    def weight(bits, K, M=256):
+        return HqWeight(bits, M, K, 1 << (bits - 1), FAKE, FAKE, None)
+
+    def tc(bits, K, batch, M=256):
+        return L.hq_linear_uses_tensor_cores(ctypes.byref(weight(bits, K, M)), batch)
+
+    def path(bits, K, batch, M=256):
+        return L.hq_linear_path(ctypes.byref(weight(bits, K, M)), batch)
+
+    G, T, G32 = HQ_PATH_GEMV, HQ_PATH_TENSOR, HQ_PATH_GEMV32
+    assert path(3, 8192, 4) == G and path(3, 8192, 5) == G32 and path(3, 8192, 16) == G32
+    assert path(3, 8192, 17) == T and tc(3, 8192, 17) == 1 and tc(3, 8192, 5) == 0
+    assert path(8, 16384, 5) == G32 and path(4, 4096, 8) == G and path(4, 4096, 9) == G32
+    assert path(2, 8192, 8) == G and path(2, 8192, 9) == G32 and path(2, 8192, 64) == T
+    assert path(4, 512, 64) == G and path(4, 512, 12) == G   # K < 1024: GEMV at every batch
+    # at most 16 tiles of 32 rows per CTA: beyond 16 x 32 x SMs rows the tensor cores
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148
+    assert path(2, 4096, 12, M=16 * 32 * sms) == G32 and path(2, 4096, 12, M=16 * 32 * sms + 1) == T
+    assert path(4, 4096, 0) == -1 and path(5, 4096, 4) == -1 and tc(4, 4096, 0) == -1
+    # launches: the rotation inside the 32-row GEMV when every batch row has a
+    # CTA (8 tiles of 32 rows < 12 rows: a prep kernel first)
+    assert L.hq_linear_launches(ctypes.byref(weight(2, 8192)), 12) == 2
+    assert L.hq_linear_launches(ctypes.byref(weight(2, 8192, M=1024)), 12) == 1
+    assert L.hq_linear_launches(ctypes.byref(weight(2, 16384, M=1024)), 12) == 2
+    # overrides: an explicit tensor-core threshold wins; the 32-row GEMV from batch 1
+    assert L.hq_set_gemv32_min_batch(-1) == 0
+    old = L.hq_set_gemv32_min_batch(1)
+    try:
+        assert path(2, 8192, 1) == G32 and path(2, 4096, 16) == G32 and path(2, 4096, 17) == T
+        prev = L.hq_set_tc_min_batch(9)
+        try:
+            assert path(2, 8192, 8) == G32 and path(2, 8192, 9) == T
+        finally:
+            L.hq_set_tc_min_batch(prev)
+    finally:
+        L.hq_set_gemv32_min_batch(old)
+    assert L.hq_set_gemv32_min_batch(-1) == 0
 
 
 def test_moe_workspace_offsets(L):

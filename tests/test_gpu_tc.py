@@ -28,7 +28,12 @@ def gpu():
     build.build()
     import bit_hadamard_rotated_b200._lib as L
     L.lib()
-    return torch.device("cuda:0")
+    # batches 9..16 (5..16 for 3/4/8-bit rows at K >= 8192) go to the 32-row
+    # GEMV by default; this module checks the tensor-core GEMM at those sizes too
+    from bit_hadamard_rotated_b200 import hq_set_gemv32_min_batch
+    old = hq_set_gemv32_min_batch(1 << 20)
+    yield torch.device("cuda:0")
+    hq_set_gemv32_min_batch(old)
 
 
 def dev(a):
@@ -101,17 +106,26 @@ def test_tc_linear_parity(bits, M, K, N):
     assert_within(y, want, bound, what=f"tc b{bits} M{M} K{K} N{N}")
 
 
-@pytest.mark.parametrize("bits,N", [(3, 5), (4, 6), (8, 8), (2, 8), (4, 4)])
+@pytest.mark.parametrize("bits,N", [(3, 5), (4, 6), (8, 8), (2, 8), (4, 4), (2, 12), (8, 16), (3, 17)])
 def test_small_batches_at_large_k_either_path(bits, N):
-    """At K = 8192 batches from 5 of 3/4/8-bit codes take the tensor-core GEMM
-    (automatic switch), 2-bit rows and batch 4 the GEMV; both match the oracle."""
+    """The automatic switch at K = 8192: batches from 5 of 3/4/8-bit codes and
+    from 9 of 2-bit codes take the 32-row GEMV up to batch 16, the tensor-core
+    GEMM beyond, smaller batches the GEMV; all match the oracle."""
     import ctypes
-    from bit_hadamard_rotated_b200._lib import lib
+    from bit_hadamard_rotated_b200 import hq_set_gemv32_min_batch
+    from bit_hadamard_rotated_b200._lib import HQ_PATH_GEMV, HQ_PATH_GEMV32, HQ_PATH_TENSOR, lib
     M, K = 300, 8192
     d = synth.linear(M, K, bits, N, seed=31 + bits + N)
     _, _, _, w = weight(d)
-    assert lib().hq_linear_uses_tensor_cores(ctypes.byref(w), N) == (1 if bits >= 3 and N >= 5 else 0)
-    y, launches, expect = run(d)
+    want_path = (HQ_PATH_TENSOR if N > 16 else
+                 HQ_PATH_GEMV32 if N >= (5 if bits >= 3 else 9) else HQ_PATH_GEMV)
+    old = hq_set_gemv32_min_batch(0)
+    try:
+        assert lib().hq_linear_path(ctypes.byref(w), N) == want_path
+        assert lib().hq_linear_uses_tensor_cores(ctypes.byref(w), N) == (1 if want_path == HQ_PATH_TENSOR else 0)
+        y, launches, expect = run(d)
+    finally:
+        hq_set_gemv32_min_batch(old)
     assert launches == expect
     want, bound = oracle.linear(bits, M, K, d["zero"], d["q"], d["scales"], d["signs"], d["x"])
     assert_within(y, want, bound, what=f"b{bits} N{N} K{K}")
