@@ -67,6 +67,7 @@ struct G32Params {
   const int8_t* signs;
   float zero, inv_sqrt_k;
   uint32_t* sync;
+  int withhold;  // test of the error path: CTA 0 does not publish its rotated row
 };
 
 // Row n of the batch, rotated by this CTA (512 threads) and written to xg in
@@ -159,31 +160,45 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
   // ---- the warp's code ring (lane 0 issues): unit i of its sequence is
   // slice i / len, unit a + i % len of that slice
   const int total = S * len;
+  const int tl_a = len > 0 ? a / GS : 0, gl_a = len > 0 ? a - tl_a * GS : 0;  // the range's first unit
   int issued = 0;
+  int i_s = 0, i_u = a, i_tl = tl_a, i_gl = gl_a;  // the next unit to request (slice, unit, tile, group)
   auto issue = [&](int slot) {
     if (lane == 0) {
-      const int s = issued / len, u = a + issued % len;
-      const int tl = u / GS, gl = u - tl * GS;
       mbar_arrive_expect_tx(&bars[slot], kTRows * GB);
-      tma_load_3d(ring + slot * ring_stride, &p.qmap, 0, (tile0 + tl) * kTRows, s * GS + gl, &bars[slot]);
+      tma_load_3d(ring + slot * ring_stride, &p.qmap, 0, (tile0 + i_tl) * kTRows, i_s * GS + i_gl, &bars[slot]);
     }
     ++issued;
+    if (++i_u == b) {
+      i_u = a;
+      i_tl = tl_a;
+      i_gl = gl_a;
+      ++i_s;
+    } else if (++i_gl == GS) {
+      i_gl = 0;
+      ++i_tl;
+    }
   };
   for (int s = 0; s < NS && issued < total; ++s) issue(s);
 
-  // ---- slice s into buffer s & 1 (one thread): the columns' fragments of
-  // its groups (one bulk copy per column) and the tiles' scales (one box per
-  // tile; rows past M read as zero)
+  // ---- slice s into buffer s & 1 (one whole warp): the columns' fragments
+  // of its groups (one bulk copy per column, lanes 0..N-1) and the tiles'
+  // scales (one box per tile, lanes 16..16+ntile-1; rows past M read as zero)
   auto issue_slice = [&](int s) {
     uint8_t* xb = xbuf + (s & 1) * p.xbuf_bytes;
     const uint32_t frag = static_cast<uint32_t>(GS) * 4 * kXsBlock;
-    const uint32_t bytes = static_cast<uint32_t>(N) * frag + static_cast<uint32_t>(ntile) * kTRows * GS * 2;
-    xlast[s & 1] = s;
-    mbar_arrive_expect_tx(&xbar[s & 1], bytes);
-    for (int n = 0; n < N; ++n) {
-      bulk_g2s(xb + n * p.xcol, p.xg + n * gemv_xs_col(G) + static_cast<size_t>(s) * frag, frag, &xbar[s & 1]);
+    if (lane == 0) {
+      xlast[s & 1] = s;
+      mbar_arrive_expect_tx(&xbar[s & 1], static_cast<uint32_t>(N) * frag +
+                                              static_cast<uint32_t>(ntile) * kTRows * GS * 2);
     }
-    for (int tl = 0; tl < ntile; ++tl) {
+    __syncwarp();
+    if (lane < N) {
+      bulk_g2s(xb + lane * p.xcol, p.xg + lane * gemv_xs_col(G) + static_cast<size_t>(s) * frag, frag,
+               &xbar[s & 1]);
+    }
+    if (lane >= 16 && lane - 16 < ntile) {
+      const int tl = lane - 16;
       tma_load_2d(xb + p.scale_off + tl * kTRows * GS * 2, &p.smap, s * GS, (tile0 + tl) * kTRows, &xbar[s & 1]);
     }
   };
@@ -202,7 +217,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
       }
       asm volatile("fence.proxy.async.global;" ::: "memory");
       __syncthreads();
-      if (tid == 0) {
+      if (tid == 0 && !(p.withhold && c == 0)) {
         __threadfence();
         atomicAdd(p.sync, 1u);
       }
@@ -232,7 +247,7 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
     const int zbytes = G * NB * 64 + 32 * NB;
     const uint8_t* src = p.xg + gemv_xs_bytes(G, N);
     for (int i = tid * 16; i < zbytes; i += kWarps * 32 * 16) cp_async16(smem + i, src + i, 16);
-    if (tid == 0) {
+    if (warp == 0) {
       issue_slice(0);
       if (S > 1) issue_slice(1);
     }
@@ -272,10 +287,10 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
   for (int s = 0; s < S && ok; ++s) {
     const uint32_t xb_s = s_base + p.x_off + (s & 1) * p.xbuf_bytes;
     if (len > 0) ok = __all_sync(0xffffffffu, mbar_wait(&xbar[s & 1], (s >> 1) & 1));
-    for (int u = a; ok && u < b; ++u) {
+    int tl = tl_a, gl = gl_a;  // the unit's tile and group in the slice
+    for (int u = a; ok && u < b; ++u, (++gl == GS ? (gl = 0, ++tl) : 0)) {
       ok = __all_sync(0xffffffffu, mbar_wait(&bars[slot], sph));
       if (!ok) break;
-      const int tl = u / GS, gl = u - tl * GS;
       const uint32_t codes = ring_s + slot * ring_stride + row_s;
       // the lane's 32-code bundle of row g + 8 r (r < 4: tiles 0 and 1)
       auto load_row = [&](int r, uint32_t (&wr)[BITS]) {
@@ -310,16 +325,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
         for (int i = 0; i < 4; ++i) bq[nb][i] = lds128(xb_s + xl[nb] + gl * (4 * kXsBlock) + rot[i]);
         z[nb] = lds128f(zq_s + (ga * NB + nb) * 64);
       }
-      float cc[2][NB][4];
+      // the chains start at the zero-point terms (C of the first MMA)
+      float zc[NB][4], cc[2][NB][4];
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-#pragma unroll
-        for (int nb = 0; nb < NB; ++nb) {
-          cc[r][nb][0] = z[nb].x;
-          cc[r][nb][1] = z[nb].y;
-          cc[r][nb][2] = z[nb].z;
-          cc[r][nb][3] = z[nb].w;
-        }
+      for (int nb = 0; nb < NB; ++nb) {
+        zc[nb][0] = z[nb].x;
+        zc[nb][1] = z[nb].y;
+        zc[nb][2] = z[nb].z;
+        zc[nb][3] = z[nb].w;
       }
       if constexpr (BITS == 3 || BITS == 8) {
         // 16 (3-bit) or 8 (8-bit) registers per decoded bundle: one tile at a time
@@ -338,7 +351,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
             for (int nb = 0; nb < NB; ++nb) {
               const uint32_t b0 = (st & 1) ? bq[nb][st >> 1].z : bq[nb][st >> 1].x;
               const uint32_t b1 = (st & 1) ? bq[nb][st >> 1].w : bq[nb][st >> 1].y;
-              mma_16816_acc(cc[r][nb], av, b0, b1);
+              if (st == 0) {
+                mma_16816(cc[r][nb], av, b0, b1, zc[nb]);
+              } else {
+                mma_16816_acc(cc[r][nb], av, b0, b1);
+              }
             }
           }
         }
@@ -361,7 +378,11 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
             for (int nb = 0; nb < NB; ++nb) {
               const uint32_t b0 = (st & 1) ? bq[nb][st >> 1].z : bq[nb][st >> 1].x;
               const uint32_t b1 = (st & 1) ? bq[nb][st >> 1].w : bq[nb][st >> 1].y;
-              mma_16816_acc(cc[r][nb], av, b0, b1);
+              if (st == 0) {
+                mma_16816(cc[r][nb], av, b0, b1, zc[nb]);
+              } else {
+                mma_16816_acc(cc[r][nb], av, b0, b1);
+              }
             }
           }
         }
@@ -408,14 +429,14 @@ __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_con
     // warps refills the buffer with slice s + 2
     fence_proxy_async_smem();
     __syncwarp();
+    uint32_t last = 0;
     if (lane == 0) {
       __threadfence_block();
       const uint32_t old = atomicAdd(&xcnt[s & 1], 1u);
-      if (old + 1u == static_cast<uint32_t>(((s >> 1) + 1) * n_busy) && s + 2 < S) {
-        __threadfence_block();
-        issue_slice(s + 2);
-      }
+      last = old + 1u == static_cast<uint32_t>(((s >> 1) + 1) * n_busy) && s + 2 < S;
+      if (last) __threadfence_block();
     }
+    if (__shfl_sync(0xffffffffu, last, 0)) issue_slice(s + 2);
   }
 
   // ---- end: every warp has consumed its units (or given up)
@@ -653,6 +674,7 @@ cudaError_t launch_gemv32(const GemvArgs& a, cudaStream_t st) {
   p.zero = static_cast<float>(a.zero);
   p.inv_sqrt_k = static_cast<float>(1.0 / sqrt(static_cast<double>(a.K)));
   p.sync = a.sync;
+  p.withhold = p.fused && take_test_fault() ? 1 : 0;
   switch (a.bits) {
     case 2: return g32_launch_b<2>(a, pl, p, st);
     case 3: return g32_launch_b<3>(a, pl, p, st);

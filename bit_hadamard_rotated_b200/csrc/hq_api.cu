@@ -74,12 +74,20 @@ static int gemv_col_block(int bits, int K, bool pgz) {
 }
 
 // The batch-8 GEMV stages its activation fragments (2 K bytes per column) in
-// shared memory for the whole of K; past ~90 KB of them (5 columns at
-// K = 8192) its copy rings become too shallow for 3/4/8-bit rows.  From there
-// (batch 5 at K >= 8192, 3/4/8 bits; batch 9 otherwise) up to batch 16 the
-// 32-row GEMV, which stages K in slices, takes over where it applies, and the
-// tensor-core GEMM beyond (or where it does not apply).
-static int auto_min_batch(const hq_weight* w) { return (w->bits >= 3 && w->K >= 8192) ? 5 : 9; }
+// shared memory for the whole of K and reads them from there once per 16-row
+// tile; the 32-row GEMV stages K in slices and reads them once per 32 rows,
+// with its rotation in the same launch.  Batch sweeps on B200 (12288 x 4096,
+// 8192^2, 28672 x 8192, 4096^2) put the switch at batch 4 for 8-bit rows,
+// 5 for 3/4-bit rows and 6 for 2-bit rows (9 above 16384 rows, where the
+// batch-8 GEMV's long tile ranges keep it ahead); up to batch 16, then the
+// tensor-core GEMM.
+static int g32_auto_min_batch(const hq_weight* w) {
+  return w->bits == 8 ? 4 : w->bits >= 3 ? 5 : (w->M > 16384 ? 9 : 6);
+}
+// Where the 32-row GEMV does not apply: the tensor-core GEMM from batch 5 for
+// 3/4/8-bit codes with K >= 8192 (its shared-memory rings stay deep where the
+// batch-8 GEMV's become shallow), else from batch 9.
+static int tc_auto_min_batch(const hq_weight* w) { return (w->bits >= 3 && w->K >= 8192) ? 5 : 9; }
 
 static bool tc_fits(const hq_weight* w) {
   return w->zeros == nullptr && w->layout == HQ_LAYOUT_PACKED && tc_col_block(w->bits, w->K) > 0;
@@ -89,12 +97,12 @@ static hq_path path_of(const hq_weight* w, int batch) {
   const int tc_min = g_tc_min_batch.load(std::memory_order_relaxed);
   if (tc_min > 0 && batch >= tc_min && tc_fits(w)) return HQ_PATH_TENSOR;
   int g32_min = g_g32_min_batch.load(std::memory_order_relaxed);
-  if (g32_min == 0) g32_min = auto_min_batch(w);
+  if (g32_min == 0) g32_min = g32_auto_min_batch(w);
   if (batch >= g32_min && batch <= 16 && w->zeros == nullptr &&
       gemv32_supported(w->bits, w->M, w->K, batch)) {
     return HQ_PATH_GEMV32;
   }
-  if (tc_min == 0 && batch >= auto_min_batch(w) && tc_fits(w)) return HQ_PATH_TENSOR;
+  if (tc_min == 0 && batch >= tc_auto_min_batch(w) && tc_fits(w)) return HQ_PATH_TENSOR;
   return HQ_PATH_GEMV;
 }
 

@@ -449,8 +449,9 @@ typedef enum {
 int hq_linear_path(const hq_weight* w, int batch);
 
 /* Batch size from which hq_linear uses the 32-row GEMV (batches up to 16,
- * where it applies).  0 (the default) selects it automatically: from batch 5
- * for 3/4/8-bit codes with K >= 8192, else from batch 9.  n >= 1 applies to
+ * where it applies).  0 (the default) selects it automatically: from batch 4
+ * for 8-bit codes, 5 for 3/4-bit codes, 6 for 2-bit codes (9 above 16384
+ * rows), from batch sweeps on B200.  n >= 1 applies to
  * every weight (n = 1: every batch up to 16); an explicit
  * hq_set_tc_min_batch still takes precedence.  Returns the previous value;
  * negative values change nothing. */
@@ -462,8 +463,11 @@ int hq_set_gemv32_min_batch(int n);
  * has fewer than two chunks withholds nothing), so that warp's bounded wait runs out
  * (after about one second) and records HQ_ERR_TIMEOUT in the status word
  * (hq_check_status, hq_linear_noalloc_check_status); that call's outputs are
- * then incomplete.  Nothing faults and the context stays usable.  Returns the
- * previous count; n < 0 only reads it. */
+ * then incomplete.  A 32-row GEMV launch that rotates its batch itself takes
+ * one of the n instead: its CTA 0 does not publish its rotated row, so every
+ * CTA's bounded wait at the rotation gate runs out the same way (the
+ * workspace must then be zeroed again).  Nothing faults and the context stays
+ * usable.  Returns the previous count; n < 0 only reads it. */
 int hq_set_test_fault(int n);
 
 #ifdef __cplusplus

@@ -181,11 +181,17 @@ def test_linear_path_choice():
         return L.hq_linear_path(ctypes.byref(weight(bits, K, M)), batch)
 
     G, T, G32 = HQ_PATH_GEMV, HQ_PATH_TENSOR, HQ_PATH_GEMV32
+    # the 32-row GEMV from batch 4 (8-bit), 5 (3/4-bit), 6 (2-bit; 9 above
+    # 16384 rows) up to 16, the tensor cores beyond
     assert path(3, 8192, 4) == G and path(3, 8192, 5) == G32 and path(3, 8192, 16) == G32
     assert path(3, 8192, 17) == T and tc(3, 8192, 17) == 1 and tc(3, 8192, 5) == 0
-    assert path(8, 16384, 5) == G32 and path(4, 4096, 8) == G and path(4, 4096, 9) == G32
-    assert path(2, 8192, 8) == G and path(2, 8192, 9) == G32 and path(2, 8192, 64) == T
+    assert path(8, 4096, 3) == G and path(8, 4096, 4) == G32 and path(8, 16384, 5) == G32
+    assert path(4, 4096, 4) == G and path(4, 4096, 5) == G32 and path(4, 4096, 9) == G32
+    assert path(2, 8192, 5) == G and path(2, 8192, 6) == G32 and path(2, 8192, 64) == T
+    assert path(2, 8192, 8, M=28672) == G and path(2, 8192, 9, M=28672) == G32
     assert path(4, 512, 64) == G and path(4, 512, 12) == G   # K < 1024: GEMV at every batch
+    # where the 32-row GEMV does not apply (per-group zeros, K < 1024) the
+    # tensor cores keep their own thresholds
     # at most 16 tiles of 32 rows per CTA: beyond 16 x 32 x SMs rows the tensor cores
     import torch
     sms = torch.cuda.get_device_properties(0).multi_processor_count if torch.cuda.is_available() else 148

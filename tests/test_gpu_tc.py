@@ -106,11 +106,11 @@ def test_tc_linear_parity(bits, M, K, N):
     assert_within(y, want, bound, what=f"tc b{bits} M{M} K{K} N{N}")
 
 
-@pytest.mark.parametrize("bits,N", [(3, 5), (4, 6), (8, 8), (2, 8), (4, 4), (2, 12), (8, 16), (3, 17)])
+@pytest.mark.parametrize("bits,N", [(3, 5), (4, 6), (8, 8), (2, 8), (4, 4), (2, 5), (2, 12), (8, 16), (3, 17)])
 def test_small_batches_at_large_k_either_path(bits, N):
-    """The automatic switch at K = 8192: batches from 5 of 3/4/8-bit codes and
-    from 9 of 2-bit codes take the 32-row GEMV up to batch 16, the tensor-core
-    GEMM beyond, smaller batches the GEMV; all match the oracle."""
+    """The automatic switch at K = 8192 (300 rows): batches from 4 of 8-bit,
+    5 of 3/4-bit and 6 of 2-bit codes take the 32-row GEMV up to batch 16, the
+    tensor-core GEMM beyond, smaller batches the GEMV; all match the oracle."""
     import ctypes
     from bit_hadamard_rotated_b200 import hq_set_gemv32_min_batch
     from bit_hadamard_rotated_b200._lib import HQ_PATH_GEMV, HQ_PATH_GEMV32, HQ_PATH_TENSOR, lib
@@ -118,7 +118,7 @@ def test_small_batches_at_large_k_either_path(bits, N):
     d = synth.linear(M, K, bits, N, seed=31 + bits + N)
     _, _, _, w = weight(d)
     want_path = (HQ_PATH_TENSOR if N > 16 else
-                 HQ_PATH_GEMV32 if N >= (5 if bits >= 3 else 9) else HQ_PATH_GEMV)
+                 HQ_PATH_GEMV32 if N >= {2: 6, 3: 5, 4: 5, 8: 4}[bits] else HQ_PATH_GEMV)
     old = hq_set_gemv32_min_batch(0)
     try:
         assert lib().hq_linear_path(ctypes.byref(w), N) == want_path
