@@ -47,7 +47,7 @@ WORKLOAD = "rotated dense MLP linear M=28672 K=8192, 2-bit group-128, batch 1"
 GRAPH_CALLS = 2048       # calls per captured graph at most
 # Files the GEMV kernel is built from: the ncu traffic figure in the profile
 # summary is reported only while their hash matches the one it was taken at.
-GEMV_SOURCES = ["gemv.cu", "fwht.cuh", "hq_common.cuh", "hq_internal.h", "hq_io.cuh",
+GEMV_SOURCES = ["gemv.cu", "gemv_frag.cuh", "fwht.cuh", "hq_common.cuh", "hq_internal.h", "hq_io.cuh",
                 "hq_launch.cuh", "hq_layout.cuh"]
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "gemv_kernel_28672x8192_b2_n1.md")
 

@@ -98,17 +98,6 @@ __device__ __forceinline__ void g32_rotate_row(const G32Params& p, int n, float*
   put_groups<BITS, (G + kWarps - 1) / kWarps, NB>(fl, buf, warp, kWarps, n, G, sc, p.zero, xs, zq, lane);
 }
 
-// Wait (bounded) until *ctr >= target; false after ~kWaitLimitNs.
-__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target) {
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
-    if (v >= target) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
-    __nanosleep(64);
-  }
-}
 
 // Slice buffer b (0, 1) of slice s: buffer s & 1, its (s >> 1)-th fill.
 template <int BITS, int NB, bool PL>

@@ -93,6 +93,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Wait (bounded) until the global counter *ctr reaches target (acquire:
+// what was written before the increments is visible after); false after
+// ~kWaitLimitNs.  For CTAs of one launch that are all resident at once.
+__device__ __forceinline__ bool wait_count(const uint32_t* ctr, uint32_t target) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ctr) : "memory");
+    if (v >= target) return true;
+    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+}
+
 // One bulk (non-tensor TMA) copy global -> shared, completing on `bar`.
 // dst and src 16-byte aligned, bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes,
