@@ -279,3 +279,18 @@ def test_to_bitplanes_rejects_bad_args(L):
     assert L.hq_launch_count() == before
     # the bit-plane layout is accepted for 2-bit weights (fails later, on the fake workspace size)
     assert lin(L, W(bits=2, zero=2, layout=1), ws_bytes=0) == HQ_ERR_WORKSPACE
+
+
+def test_linear_workspace_grows_with_batch():
+    """A workspace sized for a batch serves every smaller batch (RotatedLinear
+    sizes one for its max_batch): hq_linear_workspace_size never shrinks as the
+    batch grows, across the GEMV, 32-row GEMV and tensor-core paths."""
+    from bit_hadamard_rotated_b200._lib import lib
+    L = lib()
+    for bits in (2, 3, 4, 8):
+        for K in (128, 1024, 8192, 32768):
+            for M in (16, 4096, 28672, 100000):
+                w = HqWeight(bits, M, K, 1 << (bits - 1), FAKE, FAKE, None)
+                sizes = [L.hq_linear_workspace_size(ctypes.byref(w), b) for b in range(1, 130)]
+                assert all(s > 0 for s in sizes)
+                assert all(b >= a for a, b in zip(sizes, sizes[1:])), (bits, K, M)
