@@ -139,8 +139,10 @@ size_t hq_linear_workspace_size(const hq_weight* w, int batch);
  * x: [batch][K] fp16 activations.  batch >= 0 (0 launches nothing).
  * y: [batch][M] fp32 output.
  * workspace: >= hq_linear_workspace_size(w, batch) bytes.
- * Small batches run a fused unpack-dequant kernel that streams the packed
- * codes; larger batches run a tensor-core GEMM.  Both accumulate in fp32.
+ * Small batches run a fused unpack-dequant GEMV that streams the packed
+ * codes; batches up to 16 a 32-row variant of it (activations staged in K
+ * slices); larger batches a tensor-core GEMM (hq_linear_path tells which).
+ * All accumulate in fp32.
  * Cites: group-128 codes, 2/3/4-bit experts and 8-bit non-expert layers
  * (LLaDA2.2-mini Orin-Nano model card, Properties table).
  */
@@ -200,8 +202,8 @@ hq_status hq_moe_experts(const hq_expert* experts, int n_experts, int hidden, in
  * pointers but no allocator).  The pages have no counterpart: this is a
  * packaging variant of hq_linear, same arguments minus the workspace, results
  * within the same tolerance: every batch runs the GEMV kernels in blocks of up
- * to 8 columns (the tensor-core path that hq_linear uses from batch 9 needs a
- * workspace for its activation images).
+ * to 8 columns (the 32-row GEMV and tensor-core paths that hq_linear uses for
+ * larger batches need a workspace for their activation images).
  * Its scratch is a 512 KiB array in the library's device memory, held on every
  * GPU that loads the library until the process exits: the status word and the
  * rotated activations of one batch block (at most 332 KiB).  Limits:
