@@ -31,6 +31,13 @@
 //     bytes) through a private ring of TMA slots, issued ahead across slice
 //     boundaries; weights do not depend on earlier kernels, so the first
 //     slots are requested before griddepcontrol.wait.
+//   * For K <= 8192 and at least as many CTAs as batch rows, the batch is
+//     rotated inside the launch: CTA n < N rotates row n (the GEMV's 512-thread
+//     FWHT and fragment writer, gemv_frag.cuh) into the workspace and counts
+//     it on a counter there; every CTA waits (bounded) until all N rows are
+//     in, and the last CTA past that gate puts the counter words back to zero.
+//     All CTAs are resident at once (one per SM, grid <= SMs).  Otherwise
+//     gemv_prep_kernel runs first.
 //
 // Every wait is bounded (hq_common.cuh); a CTA that gives up records
 // HQ_DEV_TIMEOUT, lets its copies in flight land and stores nothing.
@@ -98,8 +105,7 @@ __device__ __forceinline__ void g32_rotate_row(const G32Params& p, int n, float*
   put_groups<BITS, (G + kWarps - 1) / kWarps, NB>(fl, buf, warp, kWarps, n, G, sc, p.zero, xs, zq, lane);
 }
 
-
-// Slice buffer b (0, 1) of slice s: buffer s & 1, its (s >> 1)-th fill.
+// Slice s lives in buffer s & 1 (its (s >> 1)-th fill).
 template <int BITS, int NB, bool PL>
 __global__ void __launch_bounds__(kWarps * 32, 1) gemv32_kernel(const __grid_constant__ G32Params p) {
   constexpr int GB = 16 * BITS;  // bytes of one group of one row
