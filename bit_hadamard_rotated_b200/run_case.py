@@ -7,6 +7,7 @@ A reproducible target for profilers and quick timing:
     python -m bit_hadamard_rotated_b200.run_case --moe
     python -m bit_hadamard_rotated_b200.run_case --kv --tokens 8192
     python -m bit_hadamard_rotated_b200.run_case --readout
+    python -m bit_hadamard_rotated_b200.run_case --M 8192 --K 8192 --batch 16 --tc-min-batch 1
 
 Inputs come from bit_hadamard_rotated_b200.synth (seeded); every call goes
 through the C ABI.  Prints the mean device time per call (CUDA events around
@@ -86,7 +87,7 @@ def run_linear(a):
     us = e0.elapsed_time(e1) * 1e3 / max(a.reps, 1)
     wb = d["q"].nbytes + d["scales"].nbytes
     print(f"linear M={a.M} K={a.K} b{a.bits} batch {a.batch}: {us:.2f} us/call "
-          f"({wb / (us * 1e-6) / 1e9:.0f} GB/s weights, {lin.launches(a.batch)} launches/call)")
+          f"({wb / (us * 1e-6) / 1e9:.0f} GB/s weights, {lin.launches(a.batch)} launches/call, {lin.path(a.batch)})")
 
 
 def run_moe(a):
@@ -140,9 +141,15 @@ def main():
     ap.add_argument("--kv", action="store_true", help="run the int4 KV attention instead")
     ap.add_argument("--tokens", type=int, default=8192, help="cached tokens for --kv")
     ap.add_argument("--readout", action="store_true", help="run the screened readout instead")
+    ap.add_argument("--gemv32-min-batch", type=int, default=0,
+                    help="hq_set_gemv32_min_batch before the run (0: automatic)")
+    ap.add_argument("--tc-min-batch", type=int, default=0, help="hq_set_tc_min_batch before the run (0: automatic)")
     a = ap.parse_args()
     if not torch.cuda.is_available():
         raise SystemExit("run_case needs a CUDA device")
+    from .hq import hq_set_gemv32_min_batch, hq_set_tc_min_batch
+    hq_set_gemv32_min_batch(a.gemv32_min_batch)
+    hq_set_tc_min_batch(a.tc_min_batch)
     if a.moe:
         run_moe(a)
     elif a.kv:
